@@ -1,0 +1,359 @@
+"""Benchmark of the Lighthouse Attention hot path (forward + backward) on B200.
+
+python bench.py [--gpus N] [--steps K] [--warmup W] [--impl lh|reference] [--workload NAME]
+
+One step = the whole hot path over one batch of synthetic input: pool+score,
+top-K descent, gather, causal attention, scatter (forward) and block sums,
+attention backward, spread (backward), each a liblh kernel called through the
+C ABI. Default workload: ctx512k (B1 H16 N524288 D128 bf16, p8 L4 K1024,
+sub-sequence S = 25600). Prints one JSON line on rank 0.
+
+Multi-GPU (torchrun, one process per GPU): every rank runs its own batch of
+the same workload (the (b, h) problems are independent; no collective on the
+data path), so per-GPU work is fixed ("scaling": "weak"); the time is the max
+over ranks. `--impl reference` times the CPU oracle on the host cores instead.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from long_context_symmetric_b200 import lh, synth  # noqa: E402
+
+METRIC = "Lighthouse attn fwd+bwd tokens/s at 512K on 1 B200; % HBM / tensor roofline"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def workload_desc(w):
+    return (f"{w.name}: B{w.B} H{w.H} N{w.N} D{w.D} {w.dtype} p{w.p} L{w.L} K{w.K}, "
+            f"recipe {w.recipe}, accumulation {w.mode}")
+
+
+def stage_work(w, pl):
+    """Algorithmic bytes (memory stages) or FLOPs (attention) per launch of each stage."""
+    e = 2 if w.dtype == "bf16" else 4
+    B, H, N, D, S, E = w.B, w.H, w.N, w.D, pl.S, pl.E
+    tok = B * N * H * D * e
+    sub = B * H * S * D
+    return {
+        "pool": ("bytes", 3 * tok + 3 * B * H * E * D * e + 2 * B * H * E * 8),
+        "select": ("bytes", 2 * B * H * E * 8 + B * H * (S + E + (w.L - 1) * w.K) * 4),
+        "gather": ("bytes", 6 * sub * e + B * H * S * 4),
+        "attn_fwd": ("flops", 2.0 * B * H * S * S * D),
+        "scatter": ("bytes", tok + sub * 4 + B * H * E * 4),
+        "scatter_bwd": ("bytes", tok + sub * 4 + sub * e + B * H * S * 4),
+        "attn_bwd": ("flops", 5.0 * B * H * S * S * D),
+        "spread": ("bytes", 3 * tok + 3 * sub * 4 + B * H * E * 4),
+    }
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.idx = device_index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, val in zip(names, parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def cpu_sample(w, heads=1, seed=None):
+    """Time the CPU oracle (forward + backward) on `heads` heads of the workload."""
+    import numpy as np  # noqa: F401
+
+    import oracle as orc
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        cores = os.cpu_count() or 1
+    q, k, v = synth.make_inputs(w, device="cpu", seed=seed, B=1, H=heads)
+    do = synth.make_dout(w, device="cpu", seed=seed, B=1, H=heads)
+    Q, K, V, dO = (x.to(torch.float64).numpy() for x in (q, k, v, do))
+    t0 = time.perf_counter()
+    for h in range(heads):
+        fw = orc.forward_head(Q[0, :, h], K[0, :, h], V[0, :, h], w.p, w.L, w.K, w.dtype, w.mode)
+        orc.backward_head(fw, dO[0, :, h], w.p, w.mode)
+    dt = time.perf_counter() - t0
+    # heads are independent problems of equal size: the whole job is B*H head-problems
+    tok_s = (w.B * w.N) / (dt / heads * w.B * w.H)
+    return tok_s, dt, cores
+
+
+def run_reference(args, w):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    for _ in range(args.warmup):
+        cpu_sample(w, heads=1, seed=w.seed + 1)
+    times = []
+    cores = 1
+    for i in range(args.steps):
+        _, dt, cores = cpu_sample(w, heads=1, seed=w.seed + 2 + i)
+        times.append(dt)
+    per_head = sum(times) / len(times)
+    value = (w.B * w.N) / (per_head * w.B * w.H)
+    sample = (f"one (b,h) head per step (N={w.N} tokens, whole pyramid, selection, S={lh_plan_S(w)} "
+              f"sub-sequence, attention fwd+bwd, scatter/spread) of {w.B * w.H} heads; "
+              f"tokens/s scaled to the whole job")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": per_head * 1e3 * w.B * w.H, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": workload_desc(w), "l2": "n/a (host)"},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def lh_plan_S(w):
+    return lh.plan(lh.make_config(w.B, w.H, w.N, w.D, w.p, w.L, w.K, w.dtype, w.mode)).S
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="lh", choices=["lh", "reference"])
+    ap.add_argument("--workload", default="ctx512k", choices=list(synth.WORKLOADS))
+    ap.add_argument("--e2e-steps", type=int, default=2)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    w = synth.WORKLOADS[args.workload]
+
+    if args.impl == "reference":
+        run_reference(args, w)
+        return
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+        pg = dist
+
+    cfg = lh.make_config(w.B, w.H, w.N, w.D, w.p, w.L, w.K, w.dtype, w.mode)
+    ws = lh.Workspace(cfg, dev, backward=True)
+    pl = ws.plan
+    q, k, v = synth.make_inputs(w, device=dev, seed=w.seed + 101 * rank)
+    do = synth.make_dout(w, device=dev, seed=w.seed + 101 * rank)
+    o, dq, dk, dv = (torch.empty_like(q) for _ in range(4))
+    stream = torch.cuda.current_stream(dev)
+    stages = ["pool", "select", "gather", "attn_fwd", "scatter", "scatter_bwd", "attn_bwd", "spread"]
+
+    def step(ev=None):
+        def mark(i):
+            if ev is not None:
+                ev[i].record(stream)
+        mark(0)
+        lh.pool(cfg, q, k, v, ws.pyr_q, ws.pyr_k, ws.pyr_v, ws.sq, stream)
+        mark(1)
+        lh.score_topk(cfg, ws.sq, ws.sel, ws.map, ws.slot, ws.ws, stream=stream)
+        mark(2)
+        lh.gather(cfg, q, k, v, ws.pyr_q, ws.pyr_k, ws.pyr_v, ws.map, ws.qs, ws.ks, ws.vs, stream)
+        mark(3)
+        lh.attn_fwd(cfg, ws.qs, ws.ks, ws.vs, ws.os, ws.lse, stream)
+        mark(4)
+        lh.scatter(cfg, ws.os, ws.slot, o, stream)
+        mark(5)
+        lh.scatter_bwd(cfg, do, ws.os, ws.slot, ws.dos, ws.delta, stream)
+        mark(6)
+        lh.attn_bwd(cfg, ws.qs, ws.ks, ws.vs, ws.dos, ws.lse, ws.delta, ws.dqs, ws.dks, ws.dvs, stream)
+        mark(7)
+        lh.spread(cfg, ws.dqs, ws.dks, ws.dvs, ws.slot, dq, dk, dv, stream)
+        mark(8)
+
+    for _ in range(max(args.warmup, 0)):
+        step()
+    torch.cuda.synchronize(dev)
+    st, detail = lh.get_device_error(stream)
+    if st != 0:
+        raise RuntimeError(f"device error {st} ({detail}) during warm-up")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(stages) + 1)]
+           for _ in range(args.steps)]
+    sampler = ClockSampler(local)
+    if pg:
+        pg.barrier()
+    torch.cuda.synchronize(dev)
+    sampler.start()
+    time.sleep(0.3)
+    launches0 = lh.launch_count()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for i in range(args.steps):
+        step(evs[i])
+    t_end.record(stream)
+    torch.cuda.synchronize(dev)
+    launches = lh.launch_count() - launches0
+    clocks = sampler.stop()
+    if pg:
+        pg.barrier()
+    ms_total = t_start.elapsed_time(t_end)
+    if pg:
+        t = torch.tensor([ms_total], device=dev)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        ms_total = float(t.item())
+    ms_step = ms_total / args.steps
+    stage_ms = {s: sum(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(args.steps)) / args.steps
+                for j, s in enumerate(stages)}
+    st, detail = lh.get_device_error(stream)
+    if st != 0:
+        raise RuntimeError(f"device error {st} ({detail}) in the timed region")
+
+    # end-to-end through the public API: pinned host inputs -> device, fwd + bwd, results -> host
+    e2e = None
+    if args.e2e_steps > 0:
+        hq, hk, hv, hdo = (x.cpu().pin_memory() for x in (q, k, v, do))
+        ho, hdq, hdk, hdv = (torch.empty(q.shape, dtype=q.dtype).pin_memory() for _ in range(4))
+        dq_, dk_, dv_ = (torch.empty_like(q) for _ in range(3))
+        q_, k_, v_, do_, o_ = (torch.empty_like(q) for _ in range(5))
+        h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv, hdo))
+        d2h = sum(x.numel() * x.element_size() for x in (ho, hdq, hdk, hdv))
+
+        def e2e_step():
+            for dst, src in ((q_, hq), (k_, hk), (v_, hv), (do_, hdo)):
+                dst.copy_(src, non_blocking=True)
+            lh.forward(cfg, q_, k_, v_, o_, ws, stream)
+            lh.backward(cfg, do_, dq_, dk_, dv_, ws, stream)
+            for dst, src in ((ho, o_), (hdq, dq_), (hdk, dk_), (hdv, dv_)):
+                dst.copy_(src, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize(dev)
+        if pg:
+            pg.barrier()
+        a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        b_.record(stream)
+        torch.cuda.synchronize(dev)
+        e2e_ms = a.elapsed_time(b_) / args.e2e_steps
+        if pg:
+            t = torch.tensor([e2e_ms], device=dev)
+            pg.all_reduce(t, op=pg.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+        e2e = {"value": world * w.B * w.N / (e2e_ms / 1e3), "unit": "tokens/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
+
+    peaks, peak_kind = load_peaks()
+    work = stage_work(w, pl)
+    frac = {}
+    for s in stages:
+        kind, amount = work[s]
+        sec = stage_ms[s] / 1e3
+        if kind == "bytes":
+            ach = amount / sec / 1e9
+            frac[s] = {"ms": round(stage_ms[s], 4), "achieved": round(ach, 1), "unit": "GB/s",
+                       "frac": round(ach / peaks["hbm_gbs"], 4), "bound": "hbm"}
+        else:
+            ach = amount / sec / 1e12
+            frac[s] = {"ms": round(stage_ms[s], 4), "achieved": round(ach, 2), "unit": "TFLOP/s",
+                       "frac": round(ach / peaks["bf16_tflops_sustained"], 4), "bound": "tensor"}
+    dom = max(stages, key=lambda s: stage_ms[s])
+    kind, amount = work[dom]
+    roofline = {
+        "kernel": dom, "bound": frac[dom]["bound"], "achieved": frac[dom]["achieved"],
+        "peak": peaks["hbm_gbs"] if kind == "bytes" else peaks["bf16_tflops_sustained"],
+        "unit": frac[dom]["unit"], "frac": frac[dom]["frac"], "traffic": None,
+        "peak_source": f"{peak_kind} ({'hbm_gbs' if kind == 'bytes' else 'bf16_tflops_sustained'})",
+    }
+
+    cpu_baseline = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        tok_s, dt, cores = cpu_sample(w, heads=1)
+        cpu_baseline = {"value": tok_s, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                        "sample": f"oracle fwd+bwd of head (0,0) of {workload_desc(w)}; {dt:.1f} s; "
+                                  f"tokens/s scaled to all {w.B * w.H} heads"}
+
+    value = world * w.B * w.N / (ms_step / 1e3)
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+        "config": {"workload": workload_desc(w), "S": pl.S,
+                   "l2": "inputs larger than L2 (Q, K, V, dO: 8.6 GB per step), no flush",
+                   "parallelism": f"dp{world} (independent batches per GPU)"},
+        "roofline": roofline, "stages": frac, "cpu_baseline": cpu_baseline, "e2e": e2e,
+        "gpu_launches": launches, "clocks": clocks,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if pg:
+        pg.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

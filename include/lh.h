@@ -1,0 +1,208 @@
+/*
+ * lh.h — C ABI of liblh, the sm_100a (B200) implementation of the Lighthouse
+ * Attention hot path.
+ *
+ * Method: "Long Context Pre-Training with Lighthouse Attention" (Peng, Ghosh,
+ * Quesnelle; arXiv 2605.06554), §3.1: a training-only wrapper around causal
+ * scaled dot-product attention. Forward: (i) mean-pool Q, K and V into an
+ * L-level pyramid with factor p; (ii) score pyramid entries by l2 norm and
+ * select with a top-K descent; gather the selection, ordered by position,
+ * into one causal sub-sequence; (iii) dense causal attention (Eq. (1)) on that
+ * sub-sequence; (iv) scatter each output back onto the tokens its entry
+ * covers. Backward (Fig. 1, gradient path): through the scatter, the
+ * attention and the gather/pool; the selection takes no gradient.
+ *
+ * Conventions for every entry point:
+ *  - All tensor pointers are DEVICE pointers to caller-owned, contiguous,
+ *    16-byte aligned buffers. liblh never allocates device memory, never
+ *    frees it, and never keeps a pointer after the call returns.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *    stream). All work is enqueued asynchronously on it; no entry point
+ *    synchronises the host except lh_get_device_error.
+ *  - Arguments are validated before anything is launched; on any error
+ *    nothing is launched and the status says why. LH_ERR_CUDA means a launch
+ *    failed (cudaGetLastError was not cudaSuccess after it).
+ *  - Element types: `dtype` buffers hold bf16 or fp32 per lh_config.dtype;
+ *    buffers typed float / double / int32_t below are always that type.
+ *
+ * Layouts (row-major, last index fastest):
+ *   tokens  Q, K, V, O, dO, dQ, dK, dV     [B][N][H][D]   dtype
+ *   pyramid pyr_q, pyr_k, pyr_v            [B][H][E][D]   dtype, levels 1..L-1
+ *           (E = sum_{l>=1} n_l; level l starts at entry plan.lvl_off[l])
+ *   squared norms sq                       [2][B][H][E]   double ([0]: query, [1]: key)
+ *   selection sel                          [B][H][L-1][K] int32 (row l-1: level l)
+ *   gather map                             [B][H][S]      int32, (level << 28) | index
+ *   slot table                             [B][H][E]      int32, 2*slot + expanded, or -1
+ *   sub-sequence qs, ks, vs, dos           [B][H][S][D]   dtype
+ *   attention out os, grads dqs, dks, dvs  [B][H][S][D]   float
+ *   lse, delta                             [B][H][S]      float
+ */
+#ifndef LH_H
+#define LH_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define LH_MAX_LEVELS 8
+#define LH_MAX_K 4096
+
+typedef enum {
+  LH_OK = 0,
+  LH_ERR_NULL = 1,       /* a required pointer is NULL */
+  LH_ERR_SHAPE = 2,      /* sizes outside the supported set (see lh_plan) */
+  LH_ERR_ALIGN = 3,      /* a buffer is not 16-byte aligned */
+  LH_ERR_DTYPE = 4,      /* unknown dtype */
+  LH_ERR_MODE = 5,       /* unknown accumulation mode */
+  LH_ERR_WORKSPACE = 6,  /* workspace smaller than plan.ws_bytes */
+  LH_ERR_CUDA = 7,       /* a CUDA launch or runtime call failed */
+  LH_ERR_TIMEOUT = 8,    /* a bounded device-side wait gave up (reported by lh_get_device_error) */
+  LH_ERR_DEVICE = 9      /* a device-side check failed (reported by lh_get_device_error) */
+} lh_status;
+
+typedef enum { LH_BF16 = 0, LH_FP32 = 1 } lh_dtype;
+
+/* Accumulation of the steps that add several contributions into one token
+ * (forward scatter, backward spread). The pages' scatter-back has an
+ * fp-atomic default and a deterministic int-atomic variant ("Lighthouse
+ * Attention Technique", throughput paragraph). Here each token's sum is
+ * formed by the thread that owns the token (no atomics), so both modes are
+ * run-to-run deterministic; they differ in arithmetic:
+ *   LH_ACC_FP32    fp32 sum, coarse level first (counterpart of fp-atomic)
+ *   LH_ACC_FIXED64 int64 fixed point, one count = 2^-32: each contribution
+ *                  w*x is rounded to a count (x * 2^32 / p^l in double,
+ *                  round half to even) and counts add exactly, so the result
+ *                  is independent of summation order (counterpart of
+ *                  int-atomic). Sums must stay below 2^31 in magnitude. */
+typedef enum { LH_ACC_FP32 = 0, LH_ACC_FIXED64 = 1 } lh_accum;
+
+typedef struct {
+  int B, H, N, D;   /* batch, heads, tokens, head dim (D in {64, 128}) */
+  int p, L, K;      /* pool factor (>= 2), levels (1..LH_MAX_LEVELS), top-K budget (1..LH_MAX_K) */
+  lh_dtype dtype;   /* element type of tokens, pyramid, sub-sequence, outputs */
+  lh_accum accum;   /* accumulation mode of lh_scatter / lh_spread */
+} lh_config;
+
+typedef struct {
+  int S;                              /* sub-sequence length (same for every (b,h)) */
+  int E;                              /* entries of levels 1..L-1 per (b,h) */
+  int n[LH_MAX_LEVELS];               /* n_l = N / p^l */
+  int k[LH_MAX_LEVELS];               /* entries expanded at level l (l >= 1) */
+  int c[LH_MAX_LEVELS];               /* entries of level l in the sub-sequence */
+  int lvl_off[LH_MAX_LEVELS];         /* start of level l (l >= 1) within E; lvl_off[0] = 0 unused */
+  size_t ws_bytes;                    /* workspace bytes lh_score_topk / lh_forward need */
+} lh_plan_t;
+
+/* Library version (major*10000 + minor*100 + patch). */
+int lh_version(void);
+
+/* Human-readable name of a status code (static string). */
+const char* lh_status_string(lh_status s);
+
+/* Sizes of one problem. Pure host function, no CUDA call.
+ * Source: [LH] §1 size law S = O(LpK + N/p^(L-1)) under the descent reading:
+ * c_{L-1} = n_{L-1}; k_l = min(K, c_l); c_{l-1} = p * k_l.
+ * Errors: LH_ERR_NULL, LH_ERR_SHAPE (B,H,N < 1; D not 64/128; p < 2;
+ * L outside 1..LH_MAX_LEVELS; K outside 1..LH_MAX_K; N % p^(L-1) != 0;
+ * N or S >= 2^28), LH_ERR_DTYPE, LH_ERR_MODE. */
+lh_status lh_plan(const lh_config* cfg, lh_plan_t* out);
+
+/* (i) Pyramid pool + squared norms. [LH] §3.1 stage (i), Fig. 2 steps 1-2.
+ * For levels l = 1..L-1: entry i of pyr_x holds mean of tokens
+ * [i p^l, (i+1) p^l), formed in fp64 level by level (each level's sum is the
+ * left-to-right sum of its p children's sums) and rounded to nearest-even
+ * into dtype. sq[0] / sq[1] hold the squared l2 norm of the fp64 query / key
+ * means in a pinned order (8-component chunks summed left to right, chunk
+ * partials combined by a stride-halving tree). Nothing is written when L = 1.
+ * Inputs q, k, v; outputs pyr_q, pyr_k, pyr_v, sq. */
+lh_status lh_pool(const lh_config* cfg, const void* q, const void* k, const void* v,
+                  void* pyr_q, void* pyr_k, void* pyr_v, double* sq, void* stream);
+
+/* (ii) Score, top-K descent, ordering. [LH] §3.1 stage (ii), Fig. 2 step 3,
+ * Fig. 1 (topological sort into one causal sequence).
+ * score(l,i) = max(sq[0], sq[1]). The coarsest level is kept whole; at each
+ * level l = L-1..1 the first k_l candidates in the order (score desc, index
+ * asc) are expanded (chunked bitonic sort in shared memory) and their p
+ * children become the next level's candidates and sub-sequence entries.
+ * Entries are ordered by (last covered token, level) ascending.
+ * Outputs: sel (ascending indices, unused tail = -1), map, slot table.
+ * ws: device workspace of at least plan.ws_bytes (contents not kept).
+ * When L = 1, map is the identity and sel/slot/ws are not touched (may be NULL). */
+lh_status lh_score_topk(const lh_config* cfg, const double* sq, int32_t* sel, int32_t* map,
+                        int32_t* slot, void* ws, size_t ws_bytes, void* stream);
+
+/* Dense gather: sub-sequence row j of xs = entry map[j] of x (level 0: the
+ * token row of q/k/v; level >= 1: the pyramid row). Bit-exact copy.
+ * [LH] Fig. 1 (dense gather); "Lighthouse Attention Technique" (sort, then gather). */
+lh_status lh_gather(const lh_config* cfg, const void* q, const void* k, const void* v,
+                    const void* pyr_q, const void* pyr_k, const void* pyr_v, const int32_t* map,
+                    void* qs, void* ks, void* vs, void* stream);
+
+/* (iii) Causal attention on the sub-sequence, [LH] Eq. (1), scale 1/sqrt(D):
+ * os = softmax(qs ks^T / sqrt(D) + causal mask) vs, lse = natural log of each
+ * row's softmax denominator. bf16: tcgen05 tensor cores, fp32 accumulate;
+ * fp32: fp32 SIMT. */
+lh_status lh_attn_fwd(const lh_config* cfg, const void* qs, const void* ks, const void* vs,
+                      float* os, float* lse, void* stream);
+
+/* (iv) Scatter back, [LH] §3.1 stage (iv): token t of o receives, for every
+ * sub-sequence entry covering t, that entry's row of os (weight 1), summed
+ * coarse level first under cfg->accum, rounded to dtype. */
+lh_status lh_scatter(const lh_config* cfg, const float* os, const int32_t* slot, void* o,
+                     void* stream);
+
+/* Backward of the scatter (adjoint, [LH] Fig. 1 gradient path): dos row j =
+ * sum of dout over the tokens entry j covers (fp32, level by level),
+ * rounded to dtype; delta[j] = sum_d (fp32 block sum)[d] * os[j][d]. */
+lh_status lh_scatter_bwd(const lh_config* cfg, const void* dout, const float* os,
+                         const int32_t* slot, void* dos, float* delta, void* stream);
+
+/* Backward of (iii): gradients of Eq. (1) with P recomputed from lse:
+ * dvs = P^T dos, dP = dos vs^T, dS = P o (dP - delta), dqs = dS ks / sqrt(D),
+ * dks = dS^T qs / sqrt(D). Deterministic (no atomics). */
+lh_status lh_attn_bwd(const lh_config* cfg, const void* qs, const void* ks, const void* vs,
+                      const void* dos, const float* lse, const float* delta,
+                      float* dqs, float* dks, float* dvs, void* stream);
+
+/* Backward of gather + mean-pool ([LH] Fig. 1 gradient path): token t of dx
+ * receives dxs[j] / p^l(j) for every entry j covering t, summed coarse first
+ * under cfg->accum, rounded to dtype; for x in {q, k, v}. */
+lh_status lh_spread(const lh_config* cfg, const float* dqs, const float* dks, const float* dvs,
+                    const int32_t* slot, void* dq, void* dk, void* dv, void* stream);
+
+/* Device buffers of one forward+backward, caller-owned (sizes from lh_plan). */
+typedef struct {
+  void *pyr_q, *pyr_k, *pyr_v;   /* [B][H][E][D] dtype */
+  double* sq;                    /* [2][B][H][E] */
+  int32_t *sel, *map, *slot;     /* [B][H][L-1][K], [B][H][S], [B][H][E] */
+  void *qs, *ks, *vs;            /* [B][H][S][D] dtype */
+  float *os, *lse;               /* [B][H][S][D], [B][H][S] */
+  void* ws; size_t ws_bytes;     /* plan.ws_bytes */
+  void* dos; float* delta;       /* [B][H][S][D] dtype, [B][H][S] */
+  float *dqs, *dks, *dvs;        /* [B][H][S][D] */
+} lh_buffers;
+
+/* Whole forward: lh_pool, lh_score_topk, lh_gather, lh_attn_fwd, lh_scatter. */
+lh_status lh_forward(const lh_config* cfg, const void* q, const void* k, const void* v, void* o,
+                     const lh_buffers* bufs, void* stream);
+
+/* Whole backward (after lh_forward with the same bufs): lh_scatter_bwd,
+ * lh_attn_bwd, lh_spread. */
+lh_status lh_backward(const lh_config* cfg, const void* dout, void* dq, void* dk, void* dv,
+                      const lh_buffers* bufs, void* stream);
+
+/* Reads and clears the device error word set by bounded waits and device
+ * checks (LH_OK, LH_ERR_TIMEOUT or LH_ERR_DEVICE); *detail receives the
+ * kernel-specific code (0 if none). Synchronises `stream`. */
+lh_status lh_get_device_error(void* stream, int* detail);
+
+/* Number of liblh kernels launched by this process so far. */
+unsigned long long lh_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* LH_H */

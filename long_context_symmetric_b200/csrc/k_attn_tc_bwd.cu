@@ -1,0 +1,445 @@
+// Causal flash attention on the sub-sequence with tcgen05 tensor cores,
+// backward pass (bf16 operands, fp32 accumulate, deterministic: no atomics).
+//
+// "Long Context Pre-Training with Lighthouse Attention", Fig. 1: the gradient
+// flows through the attention on the gathered sub-sequence. With P recomputed
+// from the forward lse (natural log):
+//   P = exp(S / sqrt(d) - lse),  dV = P^T dO,  dP = dO V^T,
+//   dS = P o (dP - delta),  dQ = dS K / sqrt(d),  dK = dS^T Q / sqrt(d).
+//
+// Two kernels, each one CTA per 128-row tile and heavy tiles first:
+//  k_bwd_dkdv_tc  per key tile j, over query tiles i >= j:
+//      S^T = K_j Q_i^T and dP^T = V_j dO_i^T into TMEM; the compute warps (one
+//      thread per key row = TMEM lane) form P^T and dS^T and store them as bf16
+//      back into the same TMEM columns; then dV += P^T dO_i and dK += dS^T Q_i
+//      take their A operand straight from TMEM.
+//  k_bwd_dq_tc    per query tile i, over key tiles j <= i:
+//      S = Q_i K_j^T and dP = dO_i V_j^T into TMEM; dS (bf16) back into TMEM;
+//      dQ += dS K_j.
+// Q_i/dO_i (dkdv) or K_j/V_j (dq) stream through a 2-stage TMA ring; the
+// operands that stay fixed for the CTA are loaded once. Same warp roles and
+// bounded waits as the forward kernel.
+#include "tc_ptx.cuh"
+
+namespace lh {
+
+bool make_tmap_bf16(CUtensorMap* m, const void* base, int D, int S, int BH);
+
+namespace {
+
+using namespace tc;
+
+constexpr int kT = 128;              // rows per tile (both directions)
+constexpr int kSub = 128 * 64 * 2;   // 128 x 64 bf16 swizzle tile
+constexpr int kStages = 2;
+
+// A operand from TMEM (M rows in lanes, 16-bit K elements packed two per column).
+__device__ __forceinline__ void umma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc,
+                                             uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
+      ::"r"(d_tmem), "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, "
+      "%13, %14, %15, %16};"
+      ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+
+__device__ __forceinline__ void named_bar_sync(int id, int n) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+
+template <int D>
+struct BwdLayout {
+  static constexpr int SUB = D / 64;
+  static constexpr int FIX0 = 0;                               // fixed operand 0 (K_j or Q_i)
+  static constexpr int FIX1 = FIX0 + SUB * kSub;               // fixed operand 1 (V_j or dO_i)
+  static constexpr int RING = FIX1 + SUB * kSub;               // stages of (A, B) streamed tiles
+  static constexpr int STAGE = 2 * SUB * kSub;
+  static constexpr int VEC = RING + kStages * STAGE;           // lse / delta per query (dkdv)
+  static constexpr int BAR = VEC + 2 * 2 * kT * 4;
+  static constexpr int BYTES = (BAR + 256 + 1024) > 120 * 1024 ? (BAR + 256 + 1024) : 120 * 1024;
+};
+
+struct BwdBars {
+  uint64_t fix_full, ring_full[kStages], ring_empty[kStages], s_ready, ds_ready, acc_done, done, drain;
+  uint32_t tmem_base;
+  Abort abort;
+};
+
+// Shared prologue: barriers, TMEM allocation (512 columns).
+__device__ __forceinline__ void bwd_setup(BwdBars* bars, int warp) {
+  if (threadIdx.x == 0) {
+    mbar_init(&bars->fix_full, 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&bars->ring_full[s], 1);
+      mbar_init(&bars->ring_empty[s], 1);
+    }
+    mbar_init(&bars->s_ready, 1);
+    mbar_init(&bars->ds_ready, 128);
+    mbar_init(&bars->acc_done, 1);
+    mbar_init(&bars->done, 1);
+    mbar_init(&bars->drain, 1);
+    bars->abort.flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    __syncwarp();
+    tmem_alloc(&bars->tmem_base, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+}
+
+__device__ __forceinline__ void bwd_teardown(uint32_t tbase, int warp) {
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) {
+    __syncwarp();
+    tmem_dealloc(tbase, 512);
+  }
+}
+
+// Producer: the two fixed tiles once, then `n` pairs of streamed tiles at
+// rows (first + t) * 128 of maps ma, mb.
+template <int D>
+__device__ void bwd_produce(uint8_t* sm, BwdBars* bars, const CUtensorMap* f0, const CUtensorMap* f1,
+                            int frow, const CUtensorMap* ma, const CUtensorMap* mb, int first, int n,
+                            int bh, volatile Abort* ab, int* err) {
+  using Lay = BwdLayout<D>;
+  constexpr int SUB = Lay::SUB;
+  mbar_expect_tx(&bars->fix_full, 2 * SUB * kSub);
+  for (int c = 0; c < SUB; ++c) {
+    tma_load_3d(sm + Lay::FIX0 + c * kSub, f0, &bars->fix_full, 64 * c, frow * kT, bh);
+    tma_load_3d(sm + Lay::FIX1 + c * kSub, f1, &bars->fix_full, 64 * c, frow * kT, bh);
+  }
+  int issued = 0;
+  for (int t = 0; t < n; ++t) {
+    const int st = t % kStages;
+    if (t >= kStages && !mbar_wait(&bars->ring_empty[st], ((t / kStages) - 1) & 1, ab, err, 11)) break;
+    uint8_t* base = sm + Lay::RING + st * Lay::STAGE;
+    mbar_expect_tx(&bars->ring_full[st], Lay::STAGE);
+    for (int c = 0; c < SUB; ++c) {
+      tma_load_3d(base + c * kSub, ma, &bars->ring_full[st], 64 * c, (first + t) * kT, bh);
+      tma_load_3d(base + (SUB + c) * kSub, mb, &bars->ring_full[st], 64 * c, (first + t) * kT, bh);
+    }
+    issued = t + 1;
+  }
+  if (ab->flag) {
+    Abort none{0};
+    mbar_wait(&bars->fix_full, 0, &none, nullptr, 0);
+    for (int t = issued - kStages < 0 ? 0 : issued - kStages; t < issued; ++t)
+      mbar_wait(&bars->ring_full[t % kStages], (t / kStages) & 1, &none, nullptr, 0);
+  }
+}
+
+// MMA issuer shared by both kernels. Per streamed tile t:
+//   X  = F0 * A_t^T  (TMEM cols 0..127),  Y = F1 * B_t^T (TMEM cols 128..255)
+// then, once the compute warps have turned X/Y into bf16 operands in place,
+//   acc0 += Xbf * B_t   (dkdv: dV += P^T dO)      [only when two_acc]
+//   acc1 += Ybf * G_t   (dkdv: dK += dS^T Q;  dq: dQ += dS K)
+// G_t = A_t for dkdv (Q), and the streamed A tile (K_j) for dq.
+template <int D, bool TWO_ACC>
+__device__ void bwd_mma(uint8_t* sm, BwdBars* bars, uint32_t tbase, int n, volatile Abort* ab, int* err) {
+  using Lay = BwdLayout<D>;
+  constexpr int SUB = Lay::SUB;
+  constexpr uint32_t IDX = idesc_bf16(kT, kT, false);
+  constexpr uint32_t IDACC = idesc_bf16(kT, D, true);
+  const uint32_t sbase = smem_u32(sm);
+  const uint32_t tX = tbase, tY = tbase + 128;
+  const uint32_t tAcc0 = tbase + 256, tAcc1 = tbase + 256 + (TWO_ACC ? D : 0);
+  auto accumulate = [&](int tt) -> bool {
+    if (!mbar_wait(&bars->ds_ready, tt & 1, ab, err, 14)) return false;
+    tc_fence_after();
+    const int st = tt % kStages;
+    const uint32_t ring = sbase + Lay::RING + st * Lay::STAGE;
+    const uint32_t tileA = ring, tileB = ring + SUB * kSub;
+#pragma unroll
+    for (int kk = 0; kk < kT / 16; ++kk) {
+      if (TWO_ACC) {
+        const uint64_t b = sdesc_sw128(tileB + kk * 2048, kSub, 1024);
+        umma_bf16_ts(tAcc0, tX + 8 * kk, b, IDACC, (tt > 0 || kk > 0) ? 1u : 0u);
+      }
+      const uint64_t g = sdesc_sw128(tileA + kk * 2048, kSub, 1024);
+      umma_bf16_ts(tAcc1, tY + 8 * kk, g, IDACC, (tt > 0 || kk > 0) ? 1u : 0u);
+    }
+    umma_commit(&bars->ring_empty[st]);
+    return true;
+  };
+  bool ok = mbar_wait(&bars->fix_full, 0, ab, err, 12);
+  for (int t = 0; ok && t < n; ++t) {
+    const int st = t % kStages;
+    if (!mbar_wait(&bars->ring_full[st], (t / kStages) & 1, ab, err, 13)) { ok = false; break; }
+    // accumulate tile t-1 first and let it finish: its A operands are the bf16
+    // values in X/Y, which the MMAs of tile t overwrite (MMAs into different
+    // accumulators are not ordered among themselves)
+    if (t >= 1) {
+      if (!accumulate(t - 1)) { ok = false; break; }
+      umma_commit(&bars->acc_done);
+      if (!mbar_wait(&bars->acc_done, (t - 1) & 1, ab, err, 19)) { ok = false; break; }
+    }
+    tc_fence_after();
+    const uint32_t ring = sbase + Lay::RING + st * Lay::STAGE;
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+      const uint32_t koff = (kk >> 2) * kSub + (kk & 3) * 32;
+      umma_bf16(tX, sdesc_sw128(sbase + Lay::FIX0 + koff, 16, 1024), sdesc_sw128(ring + koff, 16, 1024),
+                IDX, kk > 0 ? 1u : 0u);
+    }
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+      const uint32_t koff = (kk >> 2) * kSub + (kk & 3) * 32;
+      umma_bf16(tY, sdesc_sw128(sbase + Lay::FIX1 + koff, 16, 1024),
+                sdesc_sw128(ring + SUB * kSub + koff, 16, 1024), IDX, kk > 0 ? 1u : 0u);
+    }
+    umma_commit(&bars->s_ready);
+  }
+  if (ok && accumulate(n - 1)) umma_commit(&bars->done);
+  umma_commit(&bars->drain);
+  Abort none{0};
+  mbar_wait(&bars->drain, 0, &none, nullptr, 0);
+}
+
+// ---------------------------------------------------------------- dK, dV
+template <int D>
+__global__ void __launch_bounds__(192, 1)
+k_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
+              const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tdo,
+              const float* __restrict__ lse, const float* __restrict__ delta, float* __restrict__ dks,
+              float* __restrict__ dvs, int S, float c2, float scale, int* err) {
+  using Lay = BwdLayout<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  BwdBars* bars = reinterpret_cast<BwdBars*>(sm + Lay::BAR);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int ntiles = gridDim.x;
+  const int j = blockIdx.x;            // key tile; small j has the most query tiles
+  const int bh = blockIdx.y;
+  const int n = ntiles - j;            // query tiles i = j .. ntiles-1
+  bwd_setup(bars, warp);
+  const uint32_t tbase = bars->tmem_base;
+  volatile Abort* ab = &bars->abort;
+
+  if (warp == 0) {
+    if (lane == 0) bwd_produce<D>(sm, bars, &tk, &tv, j, &tq, &tdo, j, n, bh, ab, err);
+  } else if (warp == 1) {
+    if (lane == 0) bwd_mma<D, true>(sm, bars, tbase, n, ab, err);
+  } else {
+    const int quarter = warp & 3;
+    const int m = quarter * 32 + lane;                  // key row within the tile / TMEM lane
+    const int ctid = threadIdx.x - 64;                  // 0..127
+    const uint32_t la = (uint32_t)(quarter * 32) << 16;
+    const int key = j * kT + m;
+    float* vec = reinterpret_cast<float*>(sm + Lay::VEC);   // [2][2][128]: lse2, delta
+    bool ok = true;
+    // every compute thread runs all n iterations (and their named barrier), also
+    // after a wind-down, so no warp can be left waiting at the barrier
+    for (int t = 0; t < n; ++t) {
+      const int i = j + t;
+      float* lse2 = vec + (t & 1) * 256;
+      float* dl = lse2 + 128;
+      {
+        const int q = i * kT + ctid;
+        lse2[ctid] = q < S ? lse[(size_t)bh * S + q] * 1.4426950408889634f : 0.f;
+        dl[ctid] = q < S ? delta[(size_t)bh * S + q] : 0.f;
+      }
+      named_bar_sync(1, 128);
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bars->s_ready, t & 1, ab, err, 15));
+      if (!ok) continue;
+      tc_fence_after();
+      const bool diag = (i == j);
+      const int qlim = S - 1 - i * kT;                  // last valid query column
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        uint32_t s[32], dp[32];
+        tmem_ld32(tbase + la + 32 * c, s);
+        tmem_ld32(tbase + la + 128 + 32 * c, dp);
+        tmem_wait_ld();
+        uint32_t pk[16], dk[16];
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          float pe[2], de[2];
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const int col = 32 * c + e + u;
+            const bool valid = col <= qlim && (!diag || col >= m);
+            const float p = valid ? ex2(__uint_as_float(s[e + u]) * c2 - lse2[col]) : 0.f;
+            pe[u] = p;
+            de[u] = p * (__uint_as_float(dp[e + u]) - dl[col]);
+          }
+          pk[e >> 1] = pack_bf16(pe[0], pe[1]);
+          dk[e >> 1] = pack_bf16(de[0], de[1]);
+        }
+        // bf16 results go to columns already read (16 per 32 consumed)
+        tmem_st16(tbase + la + 16 * c, pk);
+        tmem_st16(tbase + la + 128 + 16 * c, dk);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&bars->ds_ready);
+    }
+    if (ok && __all_sync(0xffffffffu, mbar_wait(&bars->done, 0, ab, err, 16))) {
+      tc_fence_after();
+      if (key < S) {
+        float* ddv = dvs + ((size_t)bh * S + key) * D;
+        float* ddk = dks + ((size_t)bh * S + key) * D;
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t a[32], b[32];
+          tmem_ld32(tbase + la + 256 + 32 * c, a);
+          tmem_ld32(tbase + la + 256 + D + 32 * c, b);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; e += 4) {
+            *reinterpret_cast<float4*>(ddv + 32 * c + e) =
+                make_float4(__uint_as_float(a[e]), __uint_as_float(a[e + 1]), __uint_as_float(a[e + 2]),
+                            __uint_as_float(a[e + 3]));
+            *reinterpret_cast<float4*>(ddk + 32 * c + e) =
+                make_float4(__uint_as_float(b[e]) * scale, __uint_as_float(b[e + 1]) * scale,
+                            __uint_as_float(b[e + 2]) * scale, __uint_as_float(b[e + 3]) * scale);
+          }
+        }
+      } else {
+        // rows past S still take part in the warp-collective TMEM loads
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t a[32], b[32];
+          tmem_ld32(tbase + la + 256 + 32 * c, a);
+          tmem_ld32(tbase + la + 256 + D + 32 * c, b);
+          tmem_wait_ld();
+        }
+      }
+    }
+  }
+  bwd_teardown(tbase, warp);
+}
+
+// ---------------------------------------------------------------- dQ
+template <int D>
+__global__ void __launch_bounds__(192, 1)
+k_bwd_dq_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
+            const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tdo,
+            const float* __restrict__ lse, const float* __restrict__ delta, float* __restrict__ dqs,
+            int S, float c2, float scale, int* err) {
+  using Lay = BwdLayout<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  BwdBars* bars = reinterpret_cast<BwdBars*>(sm + Lay::BAR);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int ntiles = gridDim.x;
+  const int i = ntiles - 1 - (int)blockIdx.x;     // query tile; late tiles have the most key tiles
+  const int bh = blockIdx.y;
+  const int n = i + 1;                            // key tiles j = 0 .. i
+  bwd_setup(bars, warp);
+  const uint32_t tbase = bars->tmem_base;
+  volatile Abort* ab = &bars->abort;
+
+  if (warp == 0) {
+    if (lane == 0) bwd_produce<D>(sm, bars, &tq, &tdo, i, &tk, &tv, 0, n, bh, ab, err);
+  } else if (warp == 1) {
+    if (lane == 0) bwd_mma<D, false>(sm, bars, tbase, n, ab, err);
+  } else {
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;            // query row within the tile / TMEM lane
+    const uint32_t la = (uint32_t)(quarter * 32) << 16;
+    const int q = i * kT + r;
+    const float lse2 = q < S ? lse[(size_t)bh * S + q] * 1.4426950408889634f : 0.f;
+    const float dl = q < S ? delta[(size_t)bh * S + q] : 0.f;
+    bool ok = true;
+    for (int jj = 0; jj < n; ++jj) {
+      if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_ready, jj & 1, ab, err, 17))) { ok = false; break; }
+      tc_fence_after();
+      const bool diag = (jj == i);
+      const int klim = min(diag ? r : kT - 1, S - 1 - jj * kT);   // last valid key column
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        uint32_t s[32], dp[32];
+        tmem_ld32(tbase + la + 32 * c, s);
+        tmem_ld32(tbase + la + 128 + 32 * c, dp);
+        tmem_wait_ld();
+        uint32_t dk[16];
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          float de[2];
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const int col = 32 * c + e + u;
+            const float p = col <= klim ? ex2(__uint_as_float(s[e + u]) * c2 - lse2) : 0.f;
+            de[u] = p * (__uint_as_float(dp[e + u]) - dl);
+          }
+          dk[e >> 1] = pack_bf16(de[0], de[1]);
+        }
+        tmem_st16(tbase + la + 128 + 16 * c, dk);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&bars->ds_ready);
+    }
+    if (ok && __all_sync(0xffffffffu, mbar_wait(&bars->done, 0, ab, err, 18))) {
+      tc_fence_after();
+      float* dst = dqs + ((size_t)bh * S + q) * D;
+#pragma unroll 1
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t a[32];
+        tmem_ld32(tbase + la + 256 + 32 * c, a);
+        tmem_wait_ld();
+        if (q < S) {
+#pragma unroll
+          for (int e = 0; e < 32; e += 4)
+            *reinterpret_cast<float4*>(dst + 32 * c + e) =
+                make_float4(__uint_as_float(a[e]) * scale, __uint_as_float(a[e + 1]) * scale,
+                            __uint_as_float(a[e + 2]) * scale, __uint_as_float(a[e + 3]) * scale);
+        }
+      }
+    }
+  }
+  bwd_teardown(tbase, warp);
+}
+
+template <int D>
+cudaError_t bwd_tc_t(const Geom& g, const void* qs, const void* ks, const void* vs, const void* dos,
+                     const float* lse, const float* delta, float* dqs, float* dks, float* dvs, int* err,
+                     cudaStream_t s) {
+  CUtensorMap tq, tk, tv, tdo;
+  const int BH = g.B * g.H;
+  if (!make_tmap_bf16(&tq, qs, D, g.S, BH) || !make_tmap_bf16(&tk, ks, D, g.S, BH) ||
+      !make_tmap_bf16(&tv, vs, D, g.S, BH) || !make_tmap_bf16(&tdo, dos, D, g.S, BH))
+    return cudaErrorInvalidValue;
+  const int smem = BwdLayout<D>::BYTES;
+  cudaError_t e = cudaFuncSetAttribute(k_bwd_dkdv_tc<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(k_bwd_dq_tc<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  const float scale = (float)(1.0 / sqrt((double)D));
+  const float c2 = (float)(1.4426950408889634 / sqrt((double)D));
+  dim3 grid((g.S + kT - 1) / kT, BH);
+  k_bwd_dkdv_tc<D><<<grid, 192, smem, s>>>(tq, tk, tv, tdo, lse, delta, dks, dvs, g.S, c2, scale, err);
+  count_launch();
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  k_bwd_dq_tc<D><<<grid, 192, smem, s>>>(tq, tk, tv, tdo, lse, delta, dqs, g.S, c2, scale, err);
+  count_launch();
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_attn_bwd_tc(const Geom& g, const void* qs, const void* ks, const void* vs,
+                               const void* dos, const float* lse, const float* delta, float* dqs,
+                               float* dks, float* dvs, int* err, cudaStream_t s) {
+  return g.D == 64 ? bwd_tc_t<64>(g, qs, ks, vs, dos, lse, delta, dqs, dks, dvs, err, s)
+                   : bwd_tc_t<128>(g, qs, ks, vs, dos, lse, delta, dqs, dks, dvs, err, s);
+}
+
+}  // namespace lh

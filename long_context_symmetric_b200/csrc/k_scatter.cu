@@ -1,0 +1,380 @@
+// Scatter back (forward), its adjoint (block sums, backward) and the spread of
+// the sub-sequence gradients onto the tokens (backward of gather + mean-pool).
+//
+// "Long Context Pre-Training with Lighthouse Attention", §3.1 stage (iv):
+// every output of the sub-sequence is written back onto the p^l token positions
+// its entry stands for; Fig. 1: gradients flow back through the scatter, the
+// attention and the gather to the pyramid pool.
+//
+// B200 design: owner-computes instead of atomics. The entries covering token t
+// are the chain of its ancestors (t / p^l at level l) from the coarsest level
+// down to the first entry that was not expanded; the slot table written by
+// lh_score_topk gives each ancestor's slot and expanded bit (levels >= 1), and a
+// token included at level 0 sits p - (t mod p) slots before its level-1
+// parent. One thread owns 8 components of one (token, head) row, sums its
+// contributions coarse level first in registers and writes the row once:
+// every output byte is written exactly once, no read-modify-write, and the
+// result does not depend on scheduling. The accumulation arithmetic follows
+// lh_accum (fp32, or int64 fixed point with one count = 2^-32).
+#include "lh_common.cuh"
+
+namespace lh {
+namespace {
+
+constexpr double kTwo32 = 4294967296.0;
+constexpr double kTwoM32 = 1.0 / 4294967296.0;
+
+// Accumulator for one thread's 8 components.
+template <int FIXED> struct Acc;
+template <> struct Acc<0> {
+  float v[8];
+  __device__ __forceinline__ void zero() {
+#pragma unroll
+    for (int d = 0; d < 8; ++d) v[d] = 0.f;
+  }
+  __device__ __forceinline__ void add(const float (&x)[8], float w, double, double) {
+#pragma unroll
+    for (int d = 0; d < 8; ++d) v[d] = __fadd_rn(v[d], __fmul_rn(x[d], w));
+  }
+  __device__ __forceinline__ void value(float (&o)[8]) const {
+#pragma unroll
+    for (int d = 0; d < 8; ++d) o[d] = v[d];
+  }
+  __device__ __forceinline__ void value64(double (&o)[8]) const {
+#pragma unroll
+    for (int d = 0; d < 8; ++d) o[d] = v[d];
+  }
+};
+template <> struct Acc<1> {
+  long long v[8];
+  __device__ __forceinline__ void zero() {
+#pragma unroll
+    for (int d = 0; d < 8; ++d) v[d] = 0;
+  }
+  // count = round_half_even(x * 2^32 / den), den = p^l (1 for weight 1); the
+  // quotient is formed as one IEEE division, or as the (identical) exact
+  // scaling by 1/den when den is a power of two (inv != 0)
+  __device__ __forceinline__ void add(const float (&x)[8], float, double den, double inv) {
+#pragma unroll
+    for (int d = 0; d < 8; ++d) {
+      const double t = __dmul_rn((double)x[d], kTwo32);
+      const double qt = den == 1.0 ? t : (inv != 0.0 ? __dmul_rn(t, inv) : __ddiv_rn(t, den));
+      v[d] += __double2ll_rn(qt);
+    }
+  }
+  __device__ __forceinline__ void value64(double (&o)[8]) const {
+#pragma unroll
+    for (int d = 0; d < 8; ++d) o[d] = __dmul_rn(__ll2double_rn(v[d]), kTwoM32);
+  }
+};
+
+template <typename T, int FIXED>
+__device__ __forceinline__ void store_acc(T* dst, const Acc<FIXED>& a);
+
+template <>
+__device__ __forceinline__ void store_acc<__nv_bfloat16, 0>(__nv_bfloat16* dst, const Acc<0>& a) {
+  float o[8];
+  a.value(o);
+  Vec8<__nv_bfloat16>::store_f32(dst, o);
+}
+template <>
+__device__ __forceinline__ void store_acc<float, 0>(float* dst, const Acc<0>& a) {
+  float o[8];
+  a.value(o);
+  Vec8<float>::store_f32(dst, o);
+}
+template <>
+__device__ __forceinline__ void store_acc<__nv_bfloat16, 1>(__nv_bfloat16* dst, const Acc<1>& a) {
+  double o[8];
+  a.value64(o);
+  Vec8<__nv_bfloat16>::store_f64(dst, o);
+}
+template <>
+__device__ __forceinline__ void store_acc<float, 1>(float* dst, const Acc<1>& a) {
+  double o[8];
+  a.value64(o);
+  Vec8<float>::store_f64(dst, o);
+}
+
+// Sum, over the entries covering token t of head bh, of w_l * src[slot] (8 components).
+template <int FIXED, bool WEIGHTED>
+__device__ __forceinline__ void chain_sum(const Geom& g, const float* __restrict__ src,
+                                          const int32_t* __restrict__ slot_h, long long bh, int t,
+                                          int c8, Acc<FIXED>& acc) {
+  acc.zero();
+  float x[8];
+  if (g.L == 1) {
+    load8_f32(src + ((size_t)bh * g.S + t) * g.D + c8 * 8, x);
+    acc.add(x, 1.f, 1.0, 1.0);
+    return;
+  }
+  int l = g.L - 1;
+  int e = __ldg(slot_h + g.off[l] + (int)(t / g.pl[l]));
+  while (true) {
+    const int s = e >> 1;
+    load8_f32(src + ((size_t)bh * g.S + s) * g.D + c8 * 8, x);
+    const double den = WEIGHTED ? (double)g.pl[l] : 1.0;
+    const double inv = g.pow2 ? 1.0 / den : 0.0;     // exact when p is a power of two
+    acc.add(x, WEIGHTED ? (float)(1.0 / den) : 1.f, den, inv);
+    if (!(e & 1)) break;          // not expanded: no finer entry covers t
+    if (l == 1) {                 // expanded level-1 parent: t itself is in the sub-sequence
+      const int s0 = s - g.p + (t % g.p);
+      load8_f32(src + ((size_t)bh * g.S + s0) * g.D + c8 * 8, x);
+      acc.add(x, 1.f, 1.0, 1.0);
+      break;
+    }
+    --l;
+    e = __ldg(slot_h + g.off[l] + (int)(t / g.pl[l]));
+  }
+}
+
+// o[b][t][h][:] = sum of os rows covering t. One thread per 8 output components.
+template <typename T, int FIXED>
+__global__ void __launch_bounds__(256) k_scatter(const float* __restrict__ os,
+                                                 const int32_t* __restrict__ slot,
+                                                 T* __restrict__ o, Geom g) {
+  const int C8 = g.D >> 3;
+  const long long total = (long long)g.B * g.N * g.H * C8;
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
+       i += (long long)gridDim.x * blockDim.x) {
+    const int c8 = (int)(i % C8);
+    const long long r = i / C8;                 // (b, t, h) row
+    const int h = (int)(r % g.H);
+    const long long bt = r / g.H;
+    const int t = (int)(bt % g.N);
+    const long long b = bt / g.N;
+    const long long bh = b * g.H + h;
+    Acc<FIXED> acc;
+    chain_sum<FIXED, false>(g, os, slot + bh * g.E, bh, t, c8, acc);
+    store_acc<T, FIXED>(o + r * g.D + c8 * 8, acc);
+  }
+}
+
+// dx[b][t][h][:] = sum of dxs rows covering t, weighted 1/p^l; three tensors (grid.y).
+template <typename T, int FIXED>
+__global__ void __launch_bounds__(256) k_spread(const float* __restrict__ dqs,
+                                                const float* __restrict__ dks,
+                                                const float* __restrict__ dvs,
+                                                const int32_t* __restrict__ slot,
+                                                T* __restrict__ dq, T* __restrict__ dk,
+                                                T* __restrict__ dv, Geom g) {
+  const int C8 = g.D >> 3;
+  const long long total = (long long)g.B * g.N * g.H * C8;
+  const float* src = blockIdx.y == 0 ? dqs : (blockIdx.y == 1 ? dks : dvs);
+  T* dst = blockIdx.y == 0 ? dq : (blockIdx.y == 1 ? dk : dv);
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
+       i += (long long)gridDim.x * blockDim.x) {
+    const int c8 = (int)(i % C8);
+    const long long r = i / C8;
+    const int h = (int)(r % g.H);
+    const long long bt = r / g.H;
+    const int t = (int)(bt % g.N);
+    const long long b = bt / g.N;
+    const long long bh = b * g.H + h;
+    Acc<FIXED> acc;
+    chain_sum<FIXED, true>(g, src, slot + bh * g.E, bh, t, c8, acc);
+    store_acc<T, FIXED>(dst + r * g.D + c8 * 8, acc);
+  }
+}
+
+// Backward of the scatter: dos[j] = sum of dout over the tokens entry j covers,
+// delta[j] = <dos_fp32[j], os[j]>. A thread owns 8 components of one head and
+// walks the tokens of one coarsest block in order; level sums are fp32 and
+// formed level by level (each the left-to-right sum of its p children), so
+// every token row of dout is read exactly once.
+template <typename T, int LV>
+__global__ void __launch_bounds__(256) k_blocksum(const T* __restrict__ dout,
+                                                  const float* __restrict__ os,
+                                                  const int32_t* __restrict__ slot,
+                                                  T* __restrict__ dos, float* __restrict__ delta,
+                                                  Geom g, int hg, int yb) {
+  const int C8 = g.D >> 3;
+  const int b = blockIdx.z;
+  const int head = blockIdx.y * hg + threadIdx.x / C8;
+  const int chunk = threadIdx.x % C8;
+  const int cb = blockIdx.x * yb + threadIdx.y;
+  const int ncoarse = g.n[g.L - 1];
+  const bool live = head < g.H && cb < ncoarse;
+  const int p = g.p;
+  const long long P = g.pl[LV];
+  const size_t tok_stride = (size_t)g.H * g.D;
+  const long long bh = (long long)b * g.H + head;
+  const T* src = dout + ((size_t)b * g.N + (size_t)cb * P) * tok_stride + (size_t)head * g.D + chunk * 8;
+  const int32_t* slot_h = slot + bh * g.E;
+
+  // one included entry: write its row and its delta
+  auto emit = [&](int s, const float (&v)[8]) {
+    float part = 0.f;
+    float ov[8];
+    if (live && s >= 0) {
+      load8_f32(os + ((size_t)bh * g.S + s) * g.D + chunk * 8, ov);
+#pragma unroll
+      for (int d = 0; d < 8; ++d) part = fmaf(v[d], ov[d], part);
+    }
+    for (int off = C8 >> 1; off >= 1; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
+    if (live && s >= 0) {
+      Vec8<T>::store_f32(dos + ((size_t)bh * g.S + s) * g.D + chunk * 8, v);
+      if (chunk == 0) delta[(size_t)bh * g.S + s] = part;
+    }
+  };
+
+  float acc[LV + 1][8];   // acc[l]: running sum of the open entry of level l (acc[0] unused)
+  const long long ngroups = P / p;
+  for (long long g1 = 0; g1 < ngroups; ++g1) {
+    const long long i1 = (long long)cb * (P / p) + g1;      // level-1 index
+    const int e1 = live ? __ldg(slot_h + g.off[1] + (int)i1) : -1;
+    const int s1 = e1 >= 0 ? (e1 >> 1) : -1;
+    const bool tok_in = e1 >= 0 && (e1 & 1);                 // children (tokens) included
+    float s[8];
+    for (int c = 0; c < p; ++c) {
+      float x[8];
+      if (live) Vec8<T>::load_f32(src + (size_t)(g1 * p + c) * tok_stride, x);
+      else {
+#pragma unroll
+        for (int d = 0; d < 8; ++d) x[d] = 0.f;
+      }
+      if (c == 0) {
+#pragma unroll
+        for (int d = 0; d < 8; ++d) s[d] = x[d];
+      } else {
+#pragma unroll
+        for (int d = 0; d < 8; ++d) s[d] = __fadd_rn(s[d], x[d]);
+      }
+      emit(tok_in ? s1 - p + c : -1, x);
+    }
+#pragma unroll
+    for (int d = 0; d < 8; ++d) acc[1][d] = s[d];
+    emit(s1, s);
+    long long gi = i1;
+#pragma unroll
+    for (int l = 2; l <= LV; ++l) {
+      const int pos = (int)(gi % p);
+      if (pos == 0) {
+#pragma unroll
+        for (int d = 0; d < 8; ++d) acc[l][d] = acc[l - 1][d];
+      } else {
+#pragma unroll
+        for (int d = 0; d < 8; ++d) acc[l][d] = __fadd_rn(acc[l][d], acc[l - 1][d]);
+      }
+      if (pos != p - 1) break;
+      gi /= p;
+      const int e = live ? __ldg(slot_h + g.off[l] + (int)gi) : -1;
+      emit(e >= 0 ? (e >> 1) : -1, acc[l]);
+    }
+  }
+}
+
+// L == 1: dos = dout transposed to [B][H][N][D]; delta = <dout, os>.
+template <typename T>
+__global__ void __launch_bounds__(256) k_blocksum_l1(const T* __restrict__ dout,
+                                                     const float* __restrict__ os,
+                                                     T* __restrict__ dos, float* __restrict__ delta,
+                                                     Geom g) {
+  const int C8 = g.D >> 3;
+  const long long total = (long long)g.B * g.H * g.N * C8;
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
+       i += (long long)gridDim.x * blockDim.x) {
+    const int c8 = (int)(i % C8);
+    const long long r = i / C8;          // (b, h, t) row of dos
+    const int t = (int)(r % g.N);
+    const long long bh = r / g.N;
+    const int h = (int)(bh % g.H);
+    const long long b = bh / g.H;
+    float x[8], ov[8];
+    Vec8<T>::load_f32(dout + ((b * g.N + t) * g.H + h) * g.D + c8 * 8, x);
+    load8_f32(os + r * g.D + c8 * 8, ov);
+    float part = 0.f;
+#pragma unroll
+    for (int d = 0; d < 8; ++d) part = fmaf(x[d], ov[d], part);
+    for (int off = C8 >> 1; off >= 1; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
+    Vec8<T>::store_f32(dos + r * g.D + c8 * 8, x);
+    if (c8 == 0) delta[r] = part;
+  }
+}
+
+int grid_for(long long total) {
+  long long blocks = (total + 255) / 256;
+  if (blocks > 148 * 16) blocks = 148 * 16;
+  return (int)blocks;
+}
+
+template <typename T>
+cudaError_t scatter_t(const Geom& g, const float* os, const int32_t* slot, void* o, cudaStream_t s) {
+  const long long total = (long long)g.B * g.N * g.H * (g.D / 8);
+  if (g.accum == LH_ACC_FIXED64)
+    k_scatter<T, 1><<<grid_for(total), 256, 0, s>>>(os, slot, (T*)o, g);
+  else
+    k_scatter<T, 0><<<grid_for(total), 256, 0, s>>>(os, slot, (T*)o, g);
+  count_launch();
+  return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t spread_t(const Geom& g, const float* dqs, const float* dks, const float* dvs,
+                     const int32_t* slot, void* dq, void* dk, void* dv, cudaStream_t s) {
+  const long long total = (long long)g.B * g.N * g.H * (g.D / 8);
+  dim3 grid(grid_for(total), 3);
+  if (g.accum == LH_ACC_FIXED64)
+    k_spread<T, 1><<<grid, 256, 0, s>>>(dqs, dks, dvs, slot, (T*)dq, (T*)dk, (T*)dv, g);
+  else
+    k_spread<T, 0><<<grid, 256, 0, s>>>(dqs, dks, dvs, slot, (T*)dq, (T*)dk, (T*)dv, g);
+  count_launch();
+  return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t blocksum_t(const Geom& g, const void* dout, const float* os, const int32_t* slot,
+                       void* dos, float* delta, cudaStream_t s) {
+  if (g.L == 1) {
+    const long long total = (long long)g.B * g.H * g.N * (g.D / 8);
+    k_blocksum_l1<T><<<grid_for(total), 256, 0, s>>>((const T*)dout, os, (T*)dos, delta, g);
+    count_launch();
+    return cudaGetLastError();
+  }
+  const int C8 = g.D / 8;
+  int hg = g.H;
+  while (hg * C8 > 256) {
+    --hg;
+    while (g.H % hg) --hg;
+  }
+  const int ncoarse = g.n[g.L - 1];
+  int yb = 1;
+  while (yb * 2 * hg * C8 <= 256 && yb * 2 <= ncoarse) yb *= 2;
+  dim3 block(hg * C8, yb);
+  dim3 grid((ncoarse + yb - 1) / yb, g.H / hg, g.B);
+  const T* d = (const T*)dout;
+  T* o = (T*)dos;
+  switch (g.L - 1) {
+#define LH_BS_CASE(n) \
+    case n: k_blocksum<T, n><<<grid, block, 0, s>>>(d, os, slot, o, delta, g, hg, yb); break;
+    LH_BS_CASE(1) LH_BS_CASE(2) LH_BS_CASE(3) LH_BS_CASE(4)
+    LH_BS_CASE(5) LH_BS_CASE(6) LH_BS_CASE(7)
+#undef LH_BS_CASE
+    default: return cudaErrorInvalidValue;
+  }
+  count_launch();
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_scatter(const Geom& g, lh_dtype dt, const float* os, const int32_t* slot,
+                           void* o, cudaStream_t s) {
+  return dt == LH_BF16 ? scatter_t<__nv_bfloat16>(g, os, slot, o, s)
+                       : scatter_t<float>(g, os, slot, o, s);
+}
+
+cudaError_t launch_spread(const Geom& g, lh_dtype dt, const float* dqs, const float* dks,
+                          const float* dvs, const int32_t* slot, void* dq, void* dk, void* dv,
+                          cudaStream_t s) {
+  return dt == LH_BF16 ? spread_t<__nv_bfloat16>(g, dqs, dks, dvs, slot, dq, dk, dv, s)
+                       : spread_t<float>(g, dqs, dks, dvs, slot, dq, dk, dv, s);
+}
+
+cudaError_t launch_scatter_bwd(const Geom& g, lh_dtype dt, const void* dout, const float* os,
+                               const int32_t* slot, void* dos, float* delta, cudaStream_t s) {
+  return dt == LH_BF16 ? blocksum_t<__nv_bfloat16>(g, dout, os, slot, dos, delta, s)
+                       : blocksum_t<float>(g, dout, os, slot, dos, delta, s);
+}
+
+}  // namespace lh

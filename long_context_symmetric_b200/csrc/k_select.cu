@@ -1,0 +1,286 @@
+// Hierarchical top-K descent + post-order of the selection, one CTA per (b, h).
+//
+// "Long Context Pre-Training with Lighthouse Attention", §3.1 stage (ii) and
+// Fig. 2 step 3 (chunked bitonic top-K, parents kept, tree pruned), Fig. 1 (the
+// gathered hierarchy is sorted topologically into one causal sequence);
+// "Lighthouse Attention Technique" (positions sorted before the gather, no
+// holes in the causal sequence).
+//
+// Per level l = L-1 .. 1 (all entries of level L-1 are the first candidates):
+//   score = max(|mean_Q|^2, |mean_K|^2) (fp64, from lh_pool)
+//   the first k_l candidates in the order (score desc, index asc) are expanded,
+//   found with a bitonic sorting network over shared-memory chunks of at most
+//   8192 (score, position) keys; when the candidates exceed one chunk, the
+//   current best k_l are kept at the head of the chunk and the rest is refilled
+//   with new candidates, chunk after chunk (k_l <= 4096).
+//   the p children of each expanded entry, in index order, are the next
+//   level's candidates and sub-sequence entries.
+// Post-order: every included entry's subtree (itself plus its included
+// descendants) occupies a contiguous run of slots ending at the entry, coarse
+// entries in index order. Subtree sizes are formed bottom-up, run starts
+// top-down; slot = start + size - 1. This equals sorting the entries by
+// (last covered token, level).
+//
+// Per-level working arrays (candidate index, expanded flag, rank among the
+// expanded, subtree size, run start) live in the caller's workspace
+// (5 * S int32 per (b,h)); the sort keys live in shared memory.
+#include "lh_common.cuh"
+
+namespace lh {
+namespace {
+
+constexpr int kThreads = 1024;
+constexpr int kChunk = 8192;   // sort keys per shared-memory chunk (12 bytes each)
+
+struct SelArgs {
+  Geom g;
+  int lvl_base[LH_MAX_LEVELS];   // start of level l's arrays inside one array of the per-head ws
+};
+
+__device__ __forceinline__ bool precedes(unsigned long long sa, unsigned pa, unsigned long long sb,
+                                         unsigned pb) {
+  return sa > sb || (sa == sb && pa < pb);
+}
+
+// Block-wide exclusive scan of in[0..n) into out[0..n); returns the total.
+// `in` and `out` may alias. All threads must call it.
+__device__ int block_exclusive_scan(const int* in, int* out, int n, int* warp_tot) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int carry = 0;
+  for (int base = 0; base < n; base += kThreads) {
+    const int i = base + threadIdx.x;
+    const int x = i < n ? in[i] : 0;
+    int incl = x;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    if (lane == 31) warp_tot[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+      int t = warp_tot[lane];
+      int ti = t;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        int y = __shfl_up_sync(0xffffffffu, ti, o);
+        if (lane >= o) ti += y;
+      }
+      warp_tot[lane] = ti - t;      // exclusive prefix of warp totals
+      if (lane == 31) warp_tot[32] = ti;
+    }
+    __syncthreads();
+    if (i < n) out[i] = carry + warp_tot[warp] + incl - x;
+    carry += warp_tot[32];
+    __syncthreads();
+  }
+  return carry;
+}
+
+// Bitonic sort of keys[0..n) (n a power of two) so that index 0 comes first
+// under `precedes`.
+__device__ void bitonic_sort(unsigned long long* sk, unsigned* sp, int n) {
+  for (int size = 2; size <= n; size <<= 1) {
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      for (int i = threadIdx.x; i < (n >> 1); i += kThreads) {
+        const int lo = 2 * i - (i & (stride - 1));
+        const int hi = lo + stride;
+        const bool up = (lo & size) == 0;
+        const unsigned long long a = sk[lo], b = sk[hi];
+        const unsigned pa = sp[lo], pb = sp[hi];
+        const bool sw = up ? precedes(b, pb, a, pa) : precedes(a, pa, b, pb);
+        if (sw) {
+          sk[lo] = b; sk[hi] = a;
+          sp[lo] = pb; sp[hi] = pa;
+        }
+      }
+      __syncthreads();
+    }
+  }
+}
+
+__device__ __forceinline__ unsigned long long score_bits(const double* sqq, const double* sqk,
+                                                         int e) {
+  const double s = fmax(sqq[e], sqk[e]);
+  return (unsigned long long)__double_as_longlong(s);   // s >= 0: bit order = value order
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+k_select(const double* __restrict__ sq, int32_t* __restrict__ sel, int32_t* __restrict__ map,
+         int32_t* __restrict__ slot, int32_t* __restrict__ ws, SelArgs a) {
+  extern __shared__ unsigned char smem_raw[];
+  unsigned long long* sk = reinterpret_cast<unsigned long long*>(smem_raw);
+  unsigned* sp = reinterpret_cast<unsigned*>(sk + kChunk);
+  __shared__ int warp_tot[33];
+
+  const Geom& g = a.g;
+  const int bh = blockIdx.x;
+  const int L = g.L, p = g.p, S = g.S;
+  const double* sqq = sq + (size_t)bh * g.E;
+  const double* sqk = sq + ((size_t)g.B * g.H + bh) * g.E;
+  int32_t* cand = ws + (size_t)bh * 5 * S;
+  int32_t* flag = cand + S;
+  int32_t* rank = flag + S;
+  int32_t* size = rank + S;
+  int32_t* start = size + S;
+  int32_t* slot_h = slot + (size_t)bh * g.E;
+  int32_t* sel_h = sel + (size_t)bh * (L - 1) * g.K;
+  int32_t* map_h = map + (size_t)bh * S;
+
+  // levels 1..L-2 hold entries that may stay out of the sub-sequence
+  for (int l = 1; l <= L - 2; ++l)
+    for (int i = threadIdx.x; i < g.n[l]; i += kThreads) slot_h[g.off[l] + i] = -1;
+  {
+    int32_t* c0 = cand + a.lvl_base[L - 1];
+    for (int i = threadIdx.x; i < g.n[L - 1]; i += kThreads) c0[i] = i;
+  }
+  __syncthreads();
+
+  // ---------------- descent
+  for (int l = L - 1; l >= 1; --l) {
+    const int c = g.c[l], k = g.k[l];
+    int32_t* cl = cand + a.lvl_base[l];
+    int32_t* fl = flag + a.lvl_base[l];
+    const double* sq_l = sqq + g.off[l];
+    const double* sk_l = sqk + g.off[l];
+    if (k >= c) {
+      for (int q = threadIdx.x; q < c; q += kThreads) fl[q] = 1;
+    } else {
+      for (int q = threadIdx.x; q < c; q += kThreads) fl[q] = 0;
+      // chunked top-k: best k stay at the head of the chunk between rounds
+      int n2 = 1;
+      while (n2 < (c < kChunk ? c : kChunk)) n2 <<= 1;
+      int next = 0, held = 0;
+      while (next < c) {
+        const int room = n2 - held;
+        const int take = min(room, c - next);
+        for (int i = threadIdx.x; i < room; i += kThreads) {
+          if (i < take) {
+            const int qpos = next + i;
+            sk[held + i] = score_bits(sq_l, sk_l, cl[qpos]);
+            sp[held + i] = (unsigned)qpos;
+          } else {
+            sk[held + i] = 0ull;            // sentinel: after every real candidate
+            sp[held + i] = 0xFFFFFFFFu;
+          }
+        }
+        __syncthreads();
+        bitonic_sort(sk, sp, n2);
+        next += take;
+        held = k;
+      }
+      for (int r = threadIdx.x; r < k; r += kThreads) fl[sp[r]] = 1;
+    }
+    __syncthreads();
+    // rank among expanded (exclusive scan), selection output, next candidates
+    int32_t* rl = rank + a.lvl_base[l];
+    block_exclusive_scan(fl, rl, c, warp_tot);
+    int32_t* cn = cand + a.lvl_base[l - 1];
+    int32_t* sel_l = sel_h + (size_t)(l - 1) * g.K;
+    for (int q = threadIdx.x; q < c; q += kThreads) {
+      if (fl[q]) {
+        const int r = rl[q];
+        const int e = cl[q];
+        sel_l[r] = e;
+        for (int j = 0; j < p; ++j) cn[r * p + j] = e * p + j;
+      }
+    }
+    for (int r = k + threadIdx.x; r < g.K; r += kThreads) sel_l[r] = -1;
+    __syncthreads();
+  }
+
+  // ---------------- subtree sizes, bottom-up
+  {
+    int32_t* f0 = flag + a.lvl_base[0];
+    int32_t* s0 = size + a.lvl_base[0];
+    for (int q = threadIdx.x; q < g.c[0]; q += kThreads) { f0[q] = 0; s0[q] = 1; }
+  }
+  __syncthreads();
+  for (int l = 1; l <= L - 1; ++l) {
+    const int32_t* fl = flag + a.lvl_base[l];
+    const int32_t* rl = rank + a.lvl_base[l];
+    int32_t* sl = size + a.lvl_base[l];
+    const int32_t* sc = size + a.lvl_base[l - 1];
+    for (int q = threadIdx.x; q < g.c[l]; q += kThreads) {
+      int sz = 1;
+      if (fl[q]) {
+        const int base = rl[q] * p;
+        for (int j = 0; j < p; ++j) sz += sc[base + j];
+      }
+      sl[q] = sz;
+    }
+    __syncthreads();
+  }
+
+  // ---------------- run starts, top-down
+  block_exclusive_scan(size + a.lvl_base[L - 1], start + a.lvl_base[L - 1], g.c[L - 1], warp_tot);
+  __syncthreads();
+  for (int l = L - 1; l >= 1; --l) {
+    const int32_t* fl = flag + a.lvl_base[l];
+    const int32_t* rl = rank + a.lvl_base[l];
+    const int32_t* stl = start + a.lvl_base[l];
+    const int32_t* sc = size + a.lvl_base[l - 1];
+    int32_t* stc = start + a.lvl_base[l - 1];
+    for (int q = threadIdx.x; q < g.c[l]; q += kThreads) {
+      if (fl[q]) {
+        int s = stl[q];
+        const int base = rl[q] * p;
+        for (int j = 0; j < p; ++j) {
+          stc[base + j] = s;
+          s += sc[base + j];
+        }
+      }
+    }
+    __syncthreads();
+  }
+
+  // ---------------- outputs: gather map and slot table
+  for (int l = 0; l <= L - 1; ++l) {
+    const int32_t* cl = cand + a.lvl_base[l];
+    const int32_t* fl = flag + a.lvl_base[l];
+    const int32_t* sl = size + a.lvl_base[l];
+    const int32_t* stl = start + a.lvl_base[l];
+    for (int q = threadIdx.x; q < g.c[l]; q += kThreads) {
+      const int sidx = stl[q] + sl[q] - 1;
+      const int e = cl[q];
+      map_h[sidx] = (l << 28) | e;
+      if (l >= 1) slot_h[g.off[l] + e] = 2 * sidx + (fl[q] ? 1 : 0);
+    }
+  }
+}
+
+// L == 1: the sub-sequence is the token sequence itself.
+__global__ void k_identity_map(int32_t* __restrict__ map, long long total, int N) {
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
+       i += (long long)gridDim.x * blockDim.x)
+    map[i] = (int32_t)(i % N);
+}
+
+}  // namespace
+
+cudaError_t launch_select(const Geom& g, const double* sq, int32_t* sel, int32_t* map,
+                          int32_t* slot, int32_t* ws, cudaStream_t s) {
+  if (g.L == 1) {
+    const long long total = (long long)g.B * g.H * g.N;
+    const int blocks = (int)((total + 255) / 256 < 148 * 8 ? (total + 255) / 256 : 148 * 8);
+    k_identity_map<<<blocks, 256, 0, s>>>(map, total, g.N);
+    count_launch();
+    return cudaGetLastError();
+  }
+  SelArgs a;
+  a.g = g;
+  int base = 0;
+  for (int l = 0; l < LH_MAX_LEVELS; ++l) {
+    a.lvl_base[l] = base;
+    if (l < g.L) base += g.c[l];
+  }
+  const size_t smem = (size_t)kChunk * (sizeof(unsigned long long) + sizeof(unsigned));
+  cudaError_t e = cudaFuncSetAttribute(k_select, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem);
+  if (e != cudaSuccess) return e;
+  k_select<<<g.B * g.H, kThreads, smem, s>>>(sq, sel, map, slot, ws, a);
+  count_launch();
+  return cudaGetLastError();
+}
+
+}  // namespace lh

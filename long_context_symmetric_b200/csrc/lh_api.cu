@@ -1,0 +1,323 @@
+// Host side of the liblh C ABI: sizes, argument validation, launches.
+// Every entry point validates everything before it launches anything, never
+// allocates, never synchronises (except lh_get_device_error) and reports
+// launch failures as LH_ERR_CUDA.
+#include <atomic>
+#include <cmath>
+#include <cstdlib>
+#include <cstring>
+
+#include "lh_common.cuh"
+
+namespace lh {
+
+// Device error word: [0] = lh_status, [1] = kernel-specific detail. Kernels with
+// bounded waits write it (first writer wins) instead of trapping.
+__device__ int g_dev_error[2];
+
+static std::atomic<unsigned long long> g_launches{0};
+void count_launch(int n) { g_launches.fetch_add((unsigned long long)n); }
+
+cudaError_t launch_attn_fwd_simt(const Geom& g, lh_dtype dt, const void* qs, const void* ks,
+                                 const void* vs, float* os, float* lse, cudaStream_t s);
+cudaError_t launch_attn_bwd_simt(const Geom& g, lh_dtype dt, const void* qs, const void* ks,
+                                 const void* vs, const void* dos, const float* lse,
+                                 const float* delta, float* dqs, float* dks, float* dvs,
+                                 cudaStream_t s);
+
+cudaError_t launch_attn_fwd_tc(const Geom& g, const void* qs, const void* ks, const void* vs,
+                               float* os, float* lse, int* err, cudaStream_t s);
+
+// bf16 runs on the tcgen05 tensor-core kernel; fp32 on the fp32 SIMT kernel.
+// LH_ATTN_SIMT=1 in the environment routes bf16 through the SIMT kernel too
+// (same results up to fp32 rounding; a debugging aid).
+static bool force_simt() {
+  const char* e = std::getenv("LH_ATTN_SIMT");
+  return e && e[0] == '1';
+}
+
+cudaError_t launch_attn_fwd(const Geom& g, lh_dtype dt, const void* qs, const void* ks,
+                            const void* vs, float* os, float* lse, int* err, cudaStream_t s) {
+  if (dt == LH_BF16 && !force_simt()) return launch_attn_fwd_tc(g, qs, ks, vs, os, lse, err, s);
+  return launch_attn_fwd_simt(g, dt, qs, ks, vs, os, lse, s);
+}
+
+cudaError_t launch_attn_bwd_tc(const Geom& g, const void* qs, const void* ks, const void* vs,
+                               const void* dos, const float* lse, const float* delta, float* dqs,
+                               float* dks, float* dvs, int* err, cudaStream_t s);
+
+cudaError_t launch_attn_bwd(const Geom& g, lh_dtype dt, const void* qs, const void* ks,
+                            const void* vs, const void* dos, const float* lse, const float* delta,
+                            float* dqs, float* dks, float* dvs, int* err, cudaStream_t s) {
+  if (dt == LH_BF16 && !force_simt())
+    return launch_attn_bwd_tc(g, qs, ks, vs, dos, lse, delta, dqs, dks, dvs, err, s);
+  return launch_attn_bwd_simt(g, dt, qs, ks, vs, dos, lse, delta, dqs, dks, dvs, s);
+}
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+int* g_err_ptr[kMaxDevices] = {nullptr};
+
+// Device address of g_dev_error on the current device (looked up once per device).
+int* device_error_ptr() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  if (!g_err_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_dev_error) != cudaSuccess) return nullptr;
+    g_err_ptr[dev] = (int*)p;
+  }
+  return g_err_ptr[dev];
+}
+
+bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+lh_status make_geom(const lh_config* cfg, Geom* g, lh_plan_t* out) {
+  if (!cfg) return LH_ERR_NULL;
+  if (cfg->dtype != LH_BF16 && cfg->dtype != LH_FP32) return LH_ERR_DTYPE;
+  if (cfg->accum != LH_ACC_FP32 && cfg->accum != LH_ACC_FIXED64) return LH_ERR_MODE;
+  const int B = cfg->B, H = cfg->H, N = cfg->N, D = cfg->D, p = cfg->p, L = cfg->L, K = cfg->K;
+  if (B < 1 || H < 1 || N < 1) return LH_ERR_SHAPE;
+  if (D != 64 && D != 128) return LH_ERR_SHAPE;
+  if (p < 2 || L < 1 || L > LH_MAX_LEVELS || K < 1 || K > LH_MAX_K) return LH_ERR_SHAPE;
+  if (N >= (1 << 28)) return LH_ERR_SHAPE;
+  long long pl[LH_MAX_LEVELS];
+  pl[0] = 1;
+  for (int l = 1; l < LH_MAX_LEVELS; ++l) {
+    pl[l] = pl[l - 1] * p;
+    if (pl[l] > (1LL << 40)) pl[l] = 1LL << 40;   // only levels < L are used
+  }
+  if (pl[L - 1] > N || N % pl[L - 1] != 0) return LH_ERR_SHAPE;
+  Geom G;
+  std::memset(&G, 0, sizeof(G));
+  G.B = B; G.H = H; G.N = N; G.D = D; G.p = p; G.L = L; G.K = K;
+  for (int l = 0; l < LH_MAX_LEVELS; ++l) G.pl[l] = pl[l];
+  for (int l = 0; l < L; ++l) G.n[l] = (int)(N / pl[l]);
+  G.c[L - 1] = G.n[L - 1];
+  long long cand = G.n[L - 1];
+  for (int l = L - 1; l >= 1; --l) {
+    G.k[l] = (int)(cand < K ? cand : K);
+    G.c[l - 1] = p * G.k[l];
+    cand = G.c[l - 1];
+  }
+  long long S = 0;
+  for (int l = 0; l < L; ++l) S += G.c[l];
+  if (S >= (1LL << 28)) return LH_ERR_SHAPE;
+  G.S = (int)S;
+  int E = 0;
+  for (int l = 1; l < L; ++l) {
+    G.off[l] = E;
+    E += G.n[l];
+  }
+  G.E = E;
+  G.pow2 = (p & (p - 1)) == 0;
+  G.accum = cfg->accum;
+  *g = G;
+  if (out) {
+    std::memset(out, 0, sizeof(*out));
+    out->S = G.S;
+    out->E = G.E;
+    for (int l = 0; l < LH_MAX_LEVELS; ++l) {
+      out->n[l] = G.n[l];
+      out->k[l] = G.k[l];
+      out->c[l] = G.c[l];
+      out->lvl_off[l] = G.off[l];
+    }
+    out->ws_bytes = L > 1 ? (size_t)B * H * 5 * (size_t)G.S * sizeof(int32_t) : 0;
+  }
+  return LH_OK;
+}
+
+#define LH_REQ(p) do { if (!(p)) return LH_ERR_NULL; if (!aligned16(p)) return LH_ERR_ALIGN; } while (0)
+#define LH_CUDA(call) do { if ((call) != cudaSuccess) return LH_ERR_CUDA; } while (0)
+
+}  // namespace
+}  // namespace lh
+
+using namespace lh;
+
+extern "C" {
+
+int lh_version(void) { return 100; }
+
+const char* lh_status_string(lh_status s) {
+  switch (s) {
+    case LH_OK: return "ok";
+    case LH_ERR_NULL: return "null pointer";
+    case LH_ERR_SHAPE: return "unsupported sizes";
+    case LH_ERR_ALIGN: return "buffer not 16-byte aligned";
+    case LH_ERR_DTYPE: return "unknown dtype";
+    case LH_ERR_MODE: return "unknown accumulation mode";
+    case LH_ERR_WORKSPACE: return "workspace too small";
+    case LH_ERR_CUDA: return "CUDA launch or runtime error";
+    case LH_ERR_TIMEOUT: return "device-side wait timed out";
+    case LH_ERR_DEVICE: return "device-side check failed";
+  }
+  return "unknown status";
+}
+
+lh_status lh_plan(const lh_config* cfg, lh_plan_t* out) {
+  if (!out) return LH_ERR_NULL;
+  Geom g;
+  return make_geom(cfg, &g, out);
+}
+
+lh_status lh_pool(const lh_config* cfg, const void* q, const void* k, const void* v, void* pyr_q,
+                  void* pyr_k, void* pyr_v, double* sq, void* stream) {
+  Geom g;
+  lh_status st = make_geom(cfg, &g, nullptr);
+  if (st != LH_OK) return st;
+  LH_REQ(q); LH_REQ(k); LH_REQ(v);
+  if (g.L == 1) return LH_OK;
+  LH_REQ(pyr_q); LH_REQ(pyr_k); LH_REQ(pyr_v); LH_REQ(sq);
+  LH_CUDA(launch_pool(g, cfg->dtype, q, k, v, pyr_q, pyr_k, pyr_v, sq, (cudaStream_t)stream));
+  return LH_OK;
+}
+
+lh_status lh_score_topk(const lh_config* cfg, const double* sq, int32_t* sel, int32_t* map,
+                        int32_t* slot, void* ws, size_t ws_bytes, void* stream) {
+  Geom g;
+  lh_plan_t pl;
+  lh_status st = make_geom(cfg, &g, &pl);
+  if (st != LH_OK) return st;
+  LH_REQ(map);
+  if (g.L > 1) {
+    LH_REQ(sq); LH_REQ(sel); LH_REQ(slot); LH_REQ(ws);
+    if (ws_bytes < pl.ws_bytes) return LH_ERR_WORKSPACE;
+  }
+  LH_CUDA(launch_select(g, sq, sel, map, slot, (int32_t*)ws, (cudaStream_t)stream));
+  return LH_OK;
+}
+
+lh_status lh_gather(const lh_config* cfg, const void* q, const void* k, const void* v,
+                    const void* pyr_q, const void* pyr_k, const void* pyr_v, const int32_t* map,
+                    void* qs, void* ks, void* vs, void* stream) {
+  Geom g;
+  lh_status st = make_geom(cfg, &g, nullptr);
+  if (st != LH_OK) return st;
+  LH_REQ(q); LH_REQ(k); LH_REQ(v); LH_REQ(map); LH_REQ(qs); LH_REQ(ks); LH_REQ(vs);
+  if (g.L > 1) { LH_REQ(pyr_q); LH_REQ(pyr_k); LH_REQ(pyr_v); }
+  LH_CUDA(launch_gather(g, cfg->dtype, q, k, v, pyr_q, pyr_k, pyr_v, map, qs, ks, vs,
+                        (cudaStream_t)stream));
+  return LH_OK;
+}
+
+lh_status lh_attn_fwd(const lh_config* cfg, const void* qs, const void* ks, const void* vs,
+                      float* os, float* lse, void* stream) {
+  Geom g;
+  lh_status st = make_geom(cfg, &g, nullptr);
+  if (st != LH_OK) return st;
+  LH_REQ(qs); LH_REQ(ks); LH_REQ(vs); LH_REQ(os); LH_REQ(lse);
+  LH_CUDA(launch_attn_fwd(g, cfg->dtype, qs, ks, vs, os, lse, device_error_ptr(),
+                          (cudaStream_t)stream));
+  return LH_OK;
+}
+
+lh_status lh_scatter(const lh_config* cfg, const float* os, const int32_t* slot, void* o,
+                     void* stream) {
+  Geom g;
+  lh_status st = make_geom(cfg, &g, nullptr);
+  if (st != LH_OK) return st;
+  LH_REQ(os); LH_REQ(o);
+  if (g.L > 1) LH_REQ(slot);
+  LH_CUDA(launch_scatter(g, cfg->dtype, os, slot, o, (cudaStream_t)stream));
+  return LH_OK;
+}
+
+lh_status lh_scatter_bwd(const lh_config* cfg, const void* dout, const float* os,
+                         const int32_t* slot, void* dos, float* delta, void* stream) {
+  Geom g;
+  lh_status st = make_geom(cfg, &g, nullptr);
+  if (st != LH_OK) return st;
+  LH_REQ(dout); LH_REQ(os); LH_REQ(dos); LH_REQ(delta);
+  if (g.L > 1) LH_REQ(slot);
+  LH_CUDA(launch_scatter_bwd(g, cfg->dtype, dout, os, slot, dos, delta, (cudaStream_t)stream));
+  return LH_OK;
+}
+
+lh_status lh_attn_bwd(const lh_config* cfg, const void* qs, const void* ks, const void* vs,
+                      const void* dos, const float* lse, const float* delta, float* dqs,
+                      float* dks, float* dvs, void* stream) {
+  Geom g;
+  lh_status st = make_geom(cfg, &g, nullptr);
+  if (st != LH_OK) return st;
+  LH_REQ(qs); LH_REQ(ks); LH_REQ(vs); LH_REQ(dos); LH_REQ(lse); LH_REQ(delta);
+  LH_REQ(dqs); LH_REQ(dks); LH_REQ(dvs);
+  LH_CUDA(launch_attn_bwd(g, cfg->dtype, qs, ks, vs, dos, lse, delta, dqs, dks, dvs,
+                          device_error_ptr(), (cudaStream_t)stream));
+  return LH_OK;
+}
+
+lh_status lh_spread(const lh_config* cfg, const float* dqs, const float* dks, const float* dvs,
+                    const int32_t* slot, void* dq, void* dk, void* dv, void* stream) {
+  Geom g;
+  lh_status st = make_geom(cfg, &g, nullptr);
+  if (st != LH_OK) return st;
+  LH_REQ(dqs); LH_REQ(dks); LH_REQ(dvs); LH_REQ(dq); LH_REQ(dk); LH_REQ(dv);
+  if (g.L > 1) LH_REQ(slot);
+  LH_CUDA(launch_spread(g, cfg->dtype, dqs, dks, dvs, slot, dq, dk, dv, (cudaStream_t)stream));
+  return LH_OK;
+}
+
+lh_status lh_forward(const lh_config* cfg, const void* q, const void* k, const void* v, void* o,
+                     const lh_buffers* b, void* stream) {
+  if (!b) return LH_ERR_NULL;
+  Geom g;
+  lh_plan_t pl;
+  lh_status st = make_geom(cfg, &g, &pl);
+  if (st != LH_OK) return st;
+  // validate everything up front so that nothing is launched on error
+  LH_REQ(q); LH_REQ(k); LH_REQ(v); LH_REQ(o); LH_REQ(b->map); LH_REQ(b->qs); LH_REQ(b->ks);
+  LH_REQ(b->vs); LH_REQ(b->os); LH_REQ(b->lse);
+  if (g.L > 1) {
+    LH_REQ(b->pyr_q); LH_REQ(b->pyr_k); LH_REQ(b->pyr_v); LH_REQ(b->sq); LH_REQ(b->sel);
+    LH_REQ(b->slot); LH_REQ(b->ws);
+    if (b->ws_bytes < pl.ws_bytes) return LH_ERR_WORKSPACE;
+  }
+  if ((st = lh_pool(cfg, q, k, v, b->pyr_q, b->pyr_k, b->pyr_v, b->sq, stream)) != LH_OK) return st;
+  if ((st = lh_score_topk(cfg, b->sq, b->sel, b->map, b->slot, b->ws, b->ws_bytes, stream)) != LH_OK)
+    return st;
+  if ((st = lh_gather(cfg, q, k, v, b->pyr_q, b->pyr_k, b->pyr_v, b->map, b->qs, b->ks, b->vs,
+                      stream)) != LH_OK)
+    return st;
+  if ((st = lh_attn_fwd(cfg, b->qs, b->ks, b->vs, b->os, b->lse, stream)) != LH_OK) return st;
+  return lh_scatter(cfg, b->os, b->slot, o, stream);
+}
+
+lh_status lh_backward(const lh_config* cfg, const void* dout, void* dq, void* dk, void* dv,
+                      const lh_buffers* b, void* stream) {
+  if (!b) return LH_ERR_NULL;
+  Geom g;
+  lh_status st = make_geom(cfg, &g, nullptr);
+  if (st != LH_OK) return st;
+  LH_REQ(dout); LH_REQ(dq); LH_REQ(dk); LH_REQ(dv); LH_REQ(b->os); LH_REQ(b->dos);
+  LH_REQ(b->delta); LH_REQ(b->qs); LH_REQ(b->ks); LH_REQ(b->vs); LH_REQ(b->lse);
+  LH_REQ(b->dqs); LH_REQ(b->dks); LH_REQ(b->dvs);
+  if (g.L > 1) LH_REQ(b->slot);
+  if ((st = lh_scatter_bwd(cfg, dout, b->os, b->slot, b->dos, b->delta, stream)) != LH_OK) return st;
+  if ((st = lh_attn_bwd(cfg, b->qs, b->ks, b->vs, b->dos, b->lse, b->delta, b->dqs, b->dks, b->dvs,
+                        stream)) != LH_OK)
+    return st;
+  return lh_spread(cfg, b->dqs, b->dks, b->dvs, b->slot, dq, dk, dv, stream);
+}
+
+lh_status lh_get_device_error(void* stream, int* detail) {
+  int h[2] = {0, 0};
+  const int zero[2] = {0, 0};
+  cudaStream_t s = (cudaStream_t)stream;
+  if (cudaMemcpyFromSymbolAsync(h, g_dev_error, sizeof(h), 0, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return LH_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return LH_ERR_CUDA;
+  if (h[0] != 0) {
+    if (cudaMemcpyToSymbolAsync(g_dev_error, zero, sizeof(zero), 0, cudaMemcpyHostToDevice, s) != cudaSuccess)
+      return LH_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return LH_ERR_CUDA;
+  }
+  if (detail) *detail = h[1];
+  return (lh_status)h[0];
+}
+
+unsigned long long lh_launch_count(void) { return g_launches.load(); }
+
+}  // extern "C"

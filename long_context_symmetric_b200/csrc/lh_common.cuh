@@ -1,0 +1,161 @@
+// Device-side helpers shared by the liblh kernels (sm_100a).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "lh.h"
+
+namespace lh {
+
+// Problem geometry, computed once on the host by lh_plan and passed by value.
+struct Geom {
+  int B, H, N, D, p, L, K, S, E;
+  int n[LH_MAX_LEVELS];
+  int k[LH_MAX_LEVELS];
+  int c[LH_MAX_LEVELS];
+  int off[LH_MAX_LEVELS];      // start of level l (>= 1) in the per-head E axis
+  long long pl[LH_MAX_LEVELS]; // p^l
+  int pow2;                    // p is a power of two (division by p^l is exact scaling)
+  int accum;                   // lh_accum
+};
+
+// Element I/O: 8 consecutive components of a dtype row.
+template <typename T> struct Vec8;
+
+template <> struct Vec8<__nv_bfloat16> {
+  struct Raw { uint4 a; };
+  static __device__ __forceinline__ void load_raw(const __nv_bfloat16* p, Raw& r) {
+    r.a = __ldg(reinterpret_cast<const uint4*>(p));
+  }
+  static __device__ __forceinline__ void raw_f64(const Raw& r, double (&x)[8]) {
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&r.a);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      float2 f = __bfloat1622float2(h[i]);
+      x[2 * i] = (double)f.x;
+      x[2 * i + 1] = (double)f.y;
+    }
+  }
+  static __device__ __forceinline__ void raw_f32(const Raw& r, float (&x)[8]) {
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&r.a);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      float2 f = __bfloat1622float2(h[i]);
+      x[2 * i] = f.x;
+      x[2 * i + 1] = f.y;
+    }
+  }
+  static __device__ __forceinline__ void load_f64(const __nv_bfloat16* p, double (&x)[8]) {
+    uint4 r = __ldg(reinterpret_cast<const uint4*>(p));
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&r);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      float2 f = __bfloat1622float2(h[i]);
+      x[2 * i] = (double)f.x;
+      x[2 * i + 1] = (double)f.y;
+    }
+  }
+  static __device__ __forceinline__ void load_f32(const __nv_bfloat16* p, float (&x)[8]) {
+    uint4 r = __ldg(reinterpret_cast<const uint4*>(p));
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&r);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      float2 f = __bfloat1622float2(h[i]);
+      x[2 * i] = f.x;
+      x[2 * i + 1] = f.y;
+    }
+  }
+  static __device__ __forceinline__ void store_f64(__nv_bfloat16* p, const double (&x)[8]) {
+    uint4 r;
+    __nv_bfloat16* h = reinterpret_cast<__nv_bfloat16*>(&r);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) h[i] = __double2bfloat16(x[i]);   // one rounding, nearest-even
+    *reinterpret_cast<uint4*>(p) = r;
+  }
+  static __device__ __forceinline__ void store_f32(__nv_bfloat16* p, const float (&x)[8]) {
+    uint4 r;
+    __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&r);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(x[2 * i], x[2 * i + 1]);
+    *reinterpret_cast<uint4*>(p) = r;
+  }
+};
+
+template <> struct Vec8<float> {
+  struct Raw { float4 a, b; };
+  static __device__ __forceinline__ void load_raw(const float* p, Raw& r) {
+    r.a = __ldg(reinterpret_cast<const float4*>(p));
+    r.b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+  }
+  static __device__ __forceinline__ void raw_f64(const Raw& r, double (&x)[8]) {
+    x[0] = r.a.x; x[1] = r.a.y; x[2] = r.a.z; x[3] = r.a.w;
+    x[4] = r.b.x; x[5] = r.b.y; x[6] = r.b.z; x[7] = r.b.w;
+  }
+  static __device__ __forceinline__ void raw_f32(const Raw& r, float (&x)[8]) {
+    x[0] = r.a.x; x[1] = r.a.y; x[2] = r.a.z; x[3] = r.a.w;
+    x[4] = r.b.x; x[5] = r.b.y; x[6] = r.b.z; x[7] = r.b.w;
+  }
+  static __device__ __forceinline__ void load_f64(const float* p, double (&x)[8]) {
+    float4 a = __ldg(reinterpret_cast<const float4*>(p));
+    float4 b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+    x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
+    x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+  }
+  static __device__ __forceinline__ void load_f32(const float* p, float (&x)[8]) {
+    float4 a = __ldg(reinterpret_cast<const float4*>(p));
+    float4 b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+    x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
+    x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+  }
+  static __device__ __forceinline__ void store_f64(float* p, const double (&x)[8]) {
+    float4 a = make_float4(__double2float_rn(x[0]), __double2float_rn(x[1]),
+                           __double2float_rn(x[2]), __double2float_rn(x[3]));
+    float4 b = make_float4(__double2float_rn(x[4]), __double2float_rn(x[5]),
+                           __double2float_rn(x[6]), __double2float_rn(x[7]));
+    reinterpret_cast<float4*>(p)[0] = a;
+    reinterpret_cast<float4*>(p)[1] = b;
+  }
+  static __device__ __forceinline__ void store_f32(float* p, const float (&x)[8]) {
+    reinterpret_cast<float4*>(p)[0] = make_float4(x[0], x[1], x[2], x[3]);
+    reinterpret_cast<float4*>(p)[1] = make_float4(x[4], x[5], x[6], x[7]);
+  }
+};
+
+__device__ __forceinline__ void load8_f32(const float* p, float (&x)[8]) {
+  float4 a = __ldg(reinterpret_cast<const float4*>(p));
+  float4 b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+  x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
+  x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+}
+
+// Map entry packing: (level << 28) | index.
+__device__ __forceinline__ int map_level(int e) { return (int)((unsigned)e >> 28); }
+__device__ __forceinline__ int map_index(int e) { return e & 0x0FFFFFFF; }
+
+}  // namespace lh
+
+// Host-side launchers (defined next to each kernel, called by lh_api.cu).
+namespace lh {
+cudaError_t launch_pool(const Geom& g, lh_dtype dt, const void* q, const void* k, const void* v,
+                        void* pq, void* pk, void* pv, double* sq, cudaStream_t s);
+cudaError_t launch_select(const Geom& g, const double* sq, int32_t* sel, int32_t* map,
+                          int32_t* slot, int32_t* ws, cudaStream_t s);
+cudaError_t launch_gather(const Geom& g, lh_dtype dt, const void* q, const void* k, const void* v,
+                          const void* pq, const void* pk, const void* pv, const int32_t* map,
+                          void* qs, void* ks, void* vs, cudaStream_t s);
+cudaError_t launch_scatter(const Geom& g, lh_dtype dt, const float* os, const int32_t* slot,
+                           void* o, cudaStream_t s);
+cudaError_t launch_scatter_bwd(const Geom& g, lh_dtype dt, const void* dout, const float* os,
+                               const int32_t* slot, void* dos, float* delta, cudaStream_t s);
+cudaError_t launch_spread(const Geom& g, lh_dtype dt, const float* dqs, const float* dks,
+                          const float* dvs, const int32_t* slot, void* dq, void* dk, void* dv,
+                          cudaStream_t s);
+cudaError_t launch_attn_fwd(const Geom& g, lh_dtype dt, const void* qs, const void* ks,
+                            const void* vs, float* os, float* lse, int* err, cudaStream_t s);
+cudaError_t launch_attn_bwd(const Geom& g, lh_dtype dt, const void* qs, const void* ks,
+                            const void* vs, const void* dos, const float* lse, const float* delta,
+                            float* dqs, float* dks, float* dvs, int* err, cudaStream_t s);
+void count_launch(int n = 1);
+}  // namespace lh

@@ -8,3 +8,10 @@ if ROOT not in sys.path:
 
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a)")
+
+
+def pytest_sessionstart(session):
+    # the tests load liblh.so from the source tree: build it (incrementally) first
+    from long_context_symmetric_b200 import build
+
+    build.build()

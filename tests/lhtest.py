@@ -1,0 +1,145 @@
+"""Helpers shared by the GPU parity tests: run the CUDA path stage by stage
+through the C ABI and compare each stage with the CPU oracle."""
+
+from __future__ import annotations
+
+import math
+
+import numpy as np
+import torch
+
+import oracle as orc
+from long_context_symmetric_b200 import lh, synth
+
+# Tolerances on outputs and gradients against the fp64 oracle: 1e-5 (fp32) and
+# 2e-2 (bf16) max-abs, applied to the error beyond the final rounding of the
+# result into its storage dtype (that rounding alone is up to half an ulp:
+# 0.031 for a bf16 value in [8, 16)).
+ATOL = {"fp32": 1e-5, "bf16": 2e-2}
+
+
+def half_ulp(ref: np.ndarray, dtype: str) -> np.ndarray:
+    bits = {"fp32": 24, "bf16": 8}[dtype]
+    a = np.abs(ref)
+    e = np.floor(np.log2(np.where(a > 0, a, 1.0)))
+    return np.where(a > 0, 2.0 ** (e - bits), 0.0)
+
+
+def excess_error(gpu: np.ndarray, ref: np.ndarray, dtype: str) -> float:
+    """max over elements of |gpu - ref| - half_ulp_dtype(ref)."""
+    return float(np.max(np.abs(gpu - ref) - half_ulp(ref, dtype))) if gpu.size else 0.0
+
+
+def to64(t: torch.Tensor) -> np.ndarray:
+    return t.detach().to("cpu", torch.float64).numpy()
+
+
+class Case:
+    def __init__(self, name, B, H, N, D, dtype, p, L, K, recipe="iid", accum="fp", seed=7):
+        self.name, self.B, self.H, self.N, self.D = name, B, H, N, D
+        self.dtype, self.p, self.L, self.K = dtype, p, L, K
+        self.recipe, self.accum, self.seed = recipe, accum, seed
+
+    def workload(self):
+        return synth.Workload(self.name, self.B, self.H, self.N, self.D, self.dtype, self.p, self.L,
+                              self.K, self.recipe, self.accum, True, self.seed)
+
+    def cfg(self):
+        return lh.make_config(self.B, self.H, self.N, self.D, self.p, self.L, self.K, self.dtype,
+                              self.accum)
+
+    def __repr__(self):
+        return self.name
+
+
+def case_of(w: synth.Workload) -> Case:
+    return Case(w.name, w.B, w.H, w.N, w.D, w.dtype, w.p, w.L, w.K, w.recipe, w.mode, w.seed)
+
+
+def run_gpu(case: Case, q, k, v, do=None, stream=None):
+    """Whole path, stage by stage, through the C ABI. Returns the workspace and outputs."""
+    cfg = case.cfg()
+    ws = lh.Workspace(cfg, q.device, backward=do is not None)
+    o = torch.empty_like(q)
+    lh.pool(cfg, q, k, v, ws.pyr_q, ws.pyr_k, ws.pyr_v, ws.sq, stream)
+    lh.score_topk(cfg, ws.sq, ws.sel, ws.map, ws.slot, ws.ws, stream=stream)
+    lh.gather(cfg, q, k, v, ws.pyr_q, ws.pyr_k, ws.pyr_v, ws.map, ws.qs, ws.ks, ws.vs, stream)
+    lh.attn_fwd(cfg, ws.qs, ws.ks, ws.vs, ws.os, ws.lse, stream)
+    lh.scatter(cfg, ws.os, ws.slot, o, stream)
+    out = dict(ws=ws, o=o)
+    if do is not None:
+        dq, dk, dv = (torch.empty_like(q) for _ in range(3))
+        lh.scatter_bwd(cfg, do, ws.os, ws.slot, ws.dos, ws.delta, stream)
+        lh.attn_bwd(cfg, ws.qs, ws.ks, ws.vs, ws.dos, ws.lse, ws.delta, ws.dqs, ws.dks, ws.dvs, stream)
+        lh.spread(cfg, ws.dqs, ws.dks, ws.dvs, ws.slot, dq, dk, dv, stream)
+        out.update(dq=dq, dk=dk, dv=dv)
+    torch.cuda.synchronize()
+    st, detail = lh.get_device_error()
+    assert st == 0, f"device error {st} detail {detail}"
+    return out
+
+
+def expected_slot_table(fw, case: Case, pl) -> np.ndarray:
+    """Slot table implied by the oracle's selection and order."""
+    E = pl.E
+    tab = np.full(max(E, 1), -1, dtype=np.int64)
+    slot_of = {(int(l), int(i)): j for j, (l, i) in enumerate(zip(fw["lvl"], fw["idx"]))}
+    for l in range(1, case.L):
+        sel = set(int(x) for x in fw["sel"][l]) if fw["sel"][l] is not None else set()
+        for i in fw["included"][l]:
+            j = slot_of[(l, int(i))]
+            tab[pl.lvl_off[l] + int(i)] = 2 * j + (1 if int(i) in sel else 0)
+    return tab[:E]
+
+
+def compare_head(case: Case, res, q, k, v, do, b: int, h: int, check_bwd=True):
+    """Run the oracle on head (b, h) and compare every stage of the GPU run."""
+    dt = case.dtype
+    pl = lh.plan(case.cfg())
+    ws = res["ws"]
+    qh, kh, vh = (to64(x[b, :, h, :]) for x in (q, k, v))
+    fw = orc.forward_head(qh, kh, vh, case.p, case.L, case.K, dt, case.accum)
+    assert fw["plan"].S == pl.S
+    # (i) pyramid and squared norms: bit-exact
+    for l in range(1, case.L):
+        o0, n = pl.lvl_off[l], pl.n[l]
+        for name, gpu_t, ref in (("q", ws.pyr_q, fw["stored_q"]), ("k", ws.pyr_k, fw["stored_k"]),
+                                 ("v", ws.pyr_v, fw["stored_v"])):
+            got = to64(gpu_t[b, h, o0:o0 + n])
+            assert np.array_equal(got, ref[l]), f"pyramid {name} level {l}"
+        assert np.array_equal(ws.sq[0, b, h, o0:o0 + n].cpu().numpy(), fw["sq_q"][l]), f"sq_q level {l}"
+        assert np.array_equal(ws.sq[1, b, h, o0:o0 + n].cpu().numpy(), fw["sq_k"][l]), f"sq_k level {l}"
+    # (ii) selection, order, slot table: bit-exact
+    for l in range(1, case.L):
+        kl = pl.k[l]
+        got = ws.sel[b, h, l - 1].cpu().numpy()
+        assert np.array_equal(got[:kl], fw["sel"][l]), f"sel level {l}"
+        assert np.all(got[kl:] == -1)
+    m = ws.map[b, h].cpu().numpy().astype(np.int64)
+    assert np.array_equal(m >> 28, fw["lvl"]) and np.array_equal(m & 0x0FFFFFFF, fw["idx"]), "map"
+    if case.L > 1:
+        assert np.array_equal(ws.slot[b, h].cpu().numpy().astype(np.int64),
+                              expected_slot_table(fw, case, pl)), "slot table"
+    # gather: bit-exact
+    for name, gpu_t, ref in (("qs", ws.qs, fw["qs"]), ("ks", ws.ks, fw["ks"]), ("vs", ws.vs, fw["vs"])):
+        assert np.array_equal(to64(gpu_t[b, h]), ref), name
+    # (iii) attention
+    atol = ATOL[dt]
+    err_os = float(np.max(np.abs(to64(ws.os[b, h]) - fw["os"])))
+    err_lse = float(np.max(np.abs(to64(ws.lse[b, h]) - fw["lse"])))
+    assert err_os <= atol, f"os err {err_os}"
+    assert err_lse <= atol, f"lse err {err_lse}"
+    # (iv) scatter
+    err_o = excess_error(to64(res["o"][b, :, h, :]), fw["o"], dt)
+    assert err_o <= atol, f"o err {err_o}"
+    errs = dict(os=err_os, lse=err_lse, o=err_o)
+    if do is None or not check_bwd:
+        return errs
+    bw = orc.backward_head(fw, to64(do[b, :, h, :]), case.p, case.accum)
+    err_dos = excess_error(to64(ws.dos[b, h]), bw["dos"], dt)
+    assert err_dos <= atol * max(1.0, float(np.max(np.abs(bw["dos"])))) , f"dos err {err_dos}"
+    for name in ("dq", "dk", "dv"):
+        e = excess_error(to64(res[name][b, :, h, :]), bw[name], dt)
+        errs[name] = e
+        assert e <= atol, f"{name} err {e}"
+    return errs
