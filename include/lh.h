@@ -33,7 +33,8 @@
  *   selection sel                          [B][H][L-1][K] int32 (row l-1: level l)
  *   gather map                             [B][H][S]      int32, (level << 28) | index
  *   slot table                             [B][H][E]      int32, 2*slot + expanded, or -1
- *   sub-sequence qs, ks, vs, dos           [B][H][S][D]   dtype
+ *   sub-sequence qs, ks, vs                [B][H][S][D]   dtype
+ *   backward operands qh, kh, vh, dos      [B][H][S][D]   fp16 for bf16 I/O, fp32 for fp32 I/O
  *   attention out os, grads dqs, dks, dvs  [B][H][S][D]   float
  *   lse, delta                             [B][H][S]      float
  */
@@ -136,10 +137,13 @@ lh_status lh_score_topk(const lh_config* cfg, const double* sq, int32_t* sel, in
 
 /* Dense gather: sub-sequence row j of xs = entry map[j] of x (level 0: the
  * token row of q/k/v; level >= 1: the pyramid row). Bit-exact copy.
- * [LH] Fig. 1 (dense gather); "Lighthouse Attention Technique" (sort, then gather). */
+ * [LH] Fig. 1 (dense gather); "Lighthouse Attention Technique" (sort, then gather).
+ * For bf16 I/O, qh/kh/vh (all three, or all NULL) receive fp16 copies of the
+ * same rows in the same pass: the operands lh_attn_bwd needs. The conversion is
+ * exact for bf16 values of magnitude in [2^-14, 65504]. Ignored for fp32 I/O. */
 lh_status lh_gather(const lh_config* cfg, const void* q, const void* k, const void* v,
                     const void* pyr_q, const void* pyr_k, const void* pyr_v, const int32_t* map,
-                    void* qs, void* ks, void* vs, void* stream);
+                    void* qs, void* ks, void* vs, void* qh, void* kh, void* vh, void* stream);
 
 /* (iii) Causal attention on the sub-sequence, [LH] Eq. (1), scale 1/sqrt(D):
  * os = softmax(qs ks^T / sqrt(D) + causal mask) vs, lse = natural log of each
@@ -155,14 +159,21 @@ lh_status lh_scatter(const lh_config* cfg, const float* os, const int32_t* slot,
                      void* stream);
 
 /* Backward of the scatter (adjoint, [LH] Fig. 1 gradient path): dos row j =
- * sum of dout over the tokens entry j covers (fp32, level by level),
- * rounded to dtype; delta[j] = sum_d (fp32 block sum)[d] * os[j][d]. */
+ * sum of dout over the tokens entry j covers (fp32, level by level), stored
+ * as the backward operand type (fp16 for bf16 I/O: the block sums of pooled
+ * entries need more significand than bf16 has; fp32 for fp32 I/O);
+ * delta[j] = sum_d (fp32 block sum)[d] * os[j][d]. A block sum beyond the fp16
+ * range is reported by lh_get_device_error (LH_ERR_DEVICE, detail 100). */
 lh_status lh_scatter_bwd(const lh_config* cfg, const void* dout, const float* os,
                          const int32_t* slot, void* dos, float* delta, void* stream);
 
 /* Backward of (iii): gradients of Eq. (1) with P recomputed from lse:
  * dvs = P^T dos, dP = dos vs^T, dS = P o (dP - delta), dqs = dS ks / sqrt(D),
- * dks = dS^T qs / sqrt(D). Deterministic (no atomics). */
+ * dks = dS^T qs / sqrt(D). Deterministic (no atomics). qs/ks/vs/dos are the
+ * backward operands: for bf16 I/O the fp16 copies from lh_gather and the fp16
+ * dos from lh_scatter_bwd (tcgen05 kernels, fp16 operands, fp32 accumulate);
+ * for fp32 I/O the fp32 sub-sequence (SIMT kernels). A dS beyond the fp16
+ * range is reported by lh_get_device_error (LH_ERR_DEVICE, detail 101). */
 lh_status lh_attn_bwd(const lh_config* cfg, const void* qs, const void* ks, const void* vs,
                       const void* dos, const float* lse, const float* delta,
                       float* dqs, float* dks, float* dvs, void* stream);
@@ -179,9 +190,10 @@ typedef struct {
   double* sq;                    /* [2][B][H][E] */
   int32_t *sel, *map, *slot;     /* [B][H][L-1][K], [B][H][S], [B][H][E] */
   void *qs, *ks, *vs;            /* [B][H][S][D] dtype */
+  void *qh, *kh, *vh;            /* [B][H][S][D] fp16 copies (bf16 I/O with a backward; else NULL) */
   float *os, *lse;               /* [B][H][S][D], [B][H][S] */
   void* ws; size_t ws_bytes;     /* plan.ws_bytes */
-  void* dos; float* delta;       /* [B][H][S][D] dtype, [B][H][S] */
+  void* dos; float* delta;       /* [B][H][S][D] fp16 (bf16 I/O) or fp32, [B][H][S] */
   float *dqs, *dks, *dvs;        /* [B][H][S][D] */
 } lh_buffers;
 

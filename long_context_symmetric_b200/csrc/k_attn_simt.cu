@@ -31,6 +31,10 @@ template <>
 __device__ __forceinline__ float ld1<__nv_bfloat16>(const __nv_bfloat16* p) {
   return __bfloat162float(*p);
 }
+template <>
+__device__ __forceinline__ float ld1<__half>(const __half* p) {
+  return __half2float(*p);
+}
 
 // rows [r0, r0+nrows) of a [S][D] matrix into smem (stride ld), zero past S
 template <typename T, int D>
@@ -349,9 +353,10 @@ cudaError_t launch_attn_bwd_simt(const Geom& g, lh_dtype dt, const void* qs, con
                                  const void* vs, const void* dos, const float* lse,
                                  const float* delta, float* dqs, float* dks, float* dvs,
                                  cudaStream_t s) {
+  // bf16 I/O: the backward's operands are the fp16 copies (see lh_attn_bwd)
   if (dt == LH_BF16)
-    return g.D == 64 ? bwd_t<__nv_bfloat16, 64>(g, qs, ks, vs, dos, lse, delta, dqs, dks, dvs, s)
-                     : bwd_t<__nv_bfloat16, 128>(g, qs, ks, vs, dos, lse, delta, dqs, dks, dvs, s);
+    return g.D == 64 ? bwd_t<__half, 64>(g, qs, ks, vs, dos, lse, delta, dqs, dks, dvs, s)
+                     : bwd_t<__half, 128>(g, qs, ks, vs, dos, lse, delta, dqs, dks, dvs, s);
   return g.D == 64 ? bwd_t<float, 64>(g, qs, ks, vs, dos, lse, delta, dqs, dks, dvs, s)
                    : bwd_t<float, 128>(g, qs, ks, vs, dos, lse, delta, dqs, dks, dvs, s);
 }

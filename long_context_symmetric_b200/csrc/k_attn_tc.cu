@@ -297,15 +297,16 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 
 }  // namespace
 
-// [BH][S][D] bf16 viewed as a 3-D tensor (D, S, BH); boxes of 64 columns x 128 rows.
-bool make_tmap_bf16(CUtensorMap* m, const void* base, int D, int S, int BH) {
+// [BH][S][D] 16-bit elements (bf16, or fp16 when `fp16`) viewed as a 3-D tensor
+// (D, S, BH); boxes of 64 columns x 128 rows, 128-byte swizzle.
+bool make_tmap_16(CUtensorMap* m, const void* base, int D, int S, int BH, bool fp16) {
   auto fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)S, (cuuint64_t)BH};
   cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)S * D * 2};
   cuuint32_t box[3] = {64, 128, 1};
   cuuint32_t es[3] = {1, 1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+  return fn(m, fp16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -315,8 +316,8 @@ static cudaError_t fwd_tc_t(const Geom& g, const void* qs, const void* ks, const
                             float* lse, int* err, cudaStream_t s) {
   CUtensorMap tq, tk, tv;
   const int BH = g.B * g.H;
-  if (!make_tmap_bf16(&tq, qs, D, g.S, BH) || !make_tmap_bf16(&tk, ks, D, g.S, BH) ||
-      !make_tmap_bf16(&tv, vs, D, g.S, BH))
+  if (!make_tmap_16(&tq, qs, D, g.S, BH, false) || !make_tmap_16(&tk, ks, D, g.S, BH, false) ||
+      !make_tmap_16(&tv, vs, D, g.S, BH, false))
     return cudaErrorInvalidValue;
   const int smem = FwdLayout<D>::BYTES;
   cudaError_t e = cudaFuncSetAttribute(k_attn_fwd_tc<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);

@@ -1,5 +1,5 @@
 // Causal flash attention on the sub-sequence with tcgen05 tensor cores,
-// backward pass (bf16 operands, fp32 accumulate, deterministic: no atomics).
+// backward pass (fp16 operands, fp32 accumulate, deterministic: no atomics).
 //
 // "Long Context Pre-Training with Lighthouse Attention", Fig. 1: the gradient
 // flows through the attention on the gathered sub-sequence. With P recomputed
@@ -7,15 +7,22 @@
 //   P = exp(S / sqrt(d) - lse),  dV = P^T dO,  dP = dO V^T,
 //   dS = P o (dP - delta),  dQ = dS K / sqrt(d),  dK = dS^T Q / sqrt(d).
 //
-// Two kernels, each one CTA per 128-row tile and heavy tiles first:
+// Operands are fp16 (11-bit significand): dO of a pooled entry is a block sum
+// of up to p^(L-1) token gradients, and dS inherits that range, so bf16 operands
+// would leave gradient errors several times the stated bound (measured against
+// the fp64 oracle at 512K context); q/k/v arrive as exact fp16 copies of the
+// bf16 sub-sequence. Two kernels, each one CTA per 128-row tile, heavy tiles
+// first:
 //  k_bwd_dkdv_tc  per key tile j, over query tiles i >= j:
 //      S^T = K_j Q_i^T and dP^T = V_j dO_i^T into TMEM; the compute warps (one
-//      thread per key row = TMEM lane) form P^T and dS^T and store them as bf16
+//      thread per key row = TMEM lane) form P^T and dS^T and store them as fp16
 //      back into the same TMEM columns; then dV += P^T dO_i and dK += dS^T Q_i
 //      take their A operand straight from TMEM.
 //  k_bwd_dq_tc    per query tile i, over key tiles j <= i:
-//      S = Q_i K_j^T and dP = dO_i V_j^T into TMEM; dS (bf16) back into TMEM;
-//      dQ += dS K_j.
+//      S = Q_i K_j^T and dP = dO_i V_j^T into TMEM; dS split into an fp16 head
+//      and an fp16 remainder (dS = hi + lo to about 2^-22 relative) back into
+//      TMEM; dQ += hi K_j + lo K_j.
+// A dS beyond the fp16 range is reported as LH_ERR_DEVICE, detail 101.
 // Q_i/dO_i (dkdv) or K_j/V_j (dq) stream through a 2-stage TMA ring; the
 // operands that stay fixed for the CTA are loaded once. Same warp roles and
 // bounded waits as the forward kernel.
@@ -23,7 +30,7 @@
 
 namespace lh {
 
-bool make_tmap_bf16(CUtensorMap* m, const void* base, int D, int S, int BH);
+bool make_tmap_16(CUtensorMap* m, const void* base, int D, int S, int BH, bool fp16);
 
 namespace {
 
@@ -34,7 +41,7 @@ constexpr int kSub = 128 * 64 * 2;   // 128 x 64 bf16 swizzle tile
 constexpr int kStages = 2;
 
 // A operand from TMEM (M rows in lanes, 16-bit K elements packed two per column).
-__device__ __forceinline__ void umma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc,
+__device__ __forceinline__ void umma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc,
                                              uint32_t idesc, uint32_t accumulate) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
@@ -146,16 +153,15 @@ __device__ void bwd_produce(uint8_t* sm, BwdBars* bars, const CUtensorMap* f0, c
 
 // MMA issuer shared by both kernels. Per streamed tile t:
 //   X  = F0 * A_t^T  (TMEM cols 0..127),  Y = F1 * B_t^T (TMEM cols 128..255)
-// then, once the compute warps have turned X/Y into bf16 operands in place,
-//   acc0 += Xbf * B_t   (dkdv: dV += P^T dO)      [only when two_acc]
-//   acc1 += Ybf * G_t   (dkdv: dK += dS^T Q;  dq: dQ += dS K)
-// G_t = A_t for dkdv (Q), and the streamed A tile (K_j) for dq.
+// then, once the compute warps have turned X/Y into fp16 operands in place,
+//   dkdv (TWO_ACC): acc0 += Xh * B_t (dV += P^T dO),  acc1 += Yh * A_t (dK += dS^T Q)
+//   dq:             acc1 += Xh * A_t + Yh * A_t       (dQ += (dS_hi + dS_lo) K)
 template <int D, bool TWO_ACC>
 __device__ void bwd_mma(uint8_t* sm, BwdBars* bars, uint32_t tbase, int n, volatile Abort* ab, int* err) {
   using Lay = BwdLayout<D>;
   constexpr int SUB = Lay::SUB;
-  constexpr uint32_t IDX = idesc_bf16(kT, kT, false);
-  constexpr uint32_t IDACC = idesc_bf16(kT, D, true);
+  constexpr uint32_t IDX = idesc_f16(kT, kT, false);
+  constexpr uint32_t IDACC = idesc_f16(kT, D, true);
   const uint32_t sbase = smem_u32(sm);
   const uint32_t tX = tbase, tY = tbase + 128;
   const uint32_t tAcc0 = tbase + 256, tAcc1 = tbase + 256 + (TWO_ACC ? D : 0);
@@ -167,12 +173,14 @@ __device__ void bwd_mma(uint8_t* sm, BwdBars* bars, uint32_t tbase, int n, volat
     const uint32_t tileA = ring, tileB = ring + SUB * kSub;
 #pragma unroll
     for (int kk = 0; kk < kT / 16; ++kk) {
+      const uint64_t g = sdesc_sw128(tileA + kk * 2048, kSub, 1024);
       if (TWO_ACC) {
         const uint64_t b = sdesc_sw128(tileB + kk * 2048, kSub, 1024);
-        umma_bf16_ts(tAcc0, tX + 8 * kk, b, IDACC, (tt > 0 || kk > 0) ? 1u : 0u);
+        umma_f16_ts(tAcc0, tX + 8 * kk, b, IDACC, (tt > 0 || kk > 0) ? 1u : 0u);
+      } else {
+        umma_f16_ts(tAcc1, tX + 8 * kk, g, IDACC, (tt > 0 || kk > 0) ? 1u : 0u);
       }
-      const uint64_t g = sdesc_sw128(tileA + kk * 2048, kSub, 1024);
-      umma_bf16_ts(tAcc1, tY + 8 * kk, g, IDACC, (tt > 0 || kk > 0) ? 1u : 0u);
+      umma_f16_ts(tAcc1, tY + 8 * kk, g, IDACC, (TWO_ACC && tt == 0 && kk == 0) ? 0u : 1u);
     }
     umma_commit(&bars->ring_empty[st]);
     return true;
@@ -194,13 +202,13 @@ __device__ void bwd_mma(uint8_t* sm, BwdBars* bars, uint32_t tbase, int n, volat
 #pragma unroll
     for (int kk = 0; kk < D / 16; ++kk) {
       const uint32_t koff = (kk >> 2) * kSub + (kk & 3) * 32;
-      umma_bf16(tX, sdesc_sw128(sbase + Lay::FIX0 + koff, 16, 1024), sdesc_sw128(ring + koff, 16, 1024),
+      umma_f16(tX, sdesc_sw128(sbase + Lay::FIX0 + koff, 16, 1024), sdesc_sw128(ring + koff, 16, 1024),
                 IDX, kk > 0 ? 1u : 0u);
     }
 #pragma unroll
     for (int kk = 0; kk < D / 16; ++kk) {
       const uint32_t koff = (kk >> 2) * kSub + (kk & 3) * 32;
-      umma_bf16(tY, sdesc_sw128(sbase + Lay::FIX1 + koff, 16, 1024),
+      umma_f16(tY, sdesc_sw128(sbase + Lay::FIX1 + koff, 16, 1024),
                 sdesc_sw128(ring + SUB * kSub + koff, 16, 1024), IDX, kk > 0 ? 1u : 0u);
     }
     umma_commit(&bars->s_ready);
@@ -242,6 +250,7 @@ k_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CU
     const uint32_t la = (uint32_t)(quarter * 32) << 16;
     const int key = j * kT + m;
     float* vec = reinterpret_cast<float*>(sm + Lay::VEC);   // [2][2][128]: lse2, delta
+    float dsmax = 0.f;
     bool ok = true;
     // every compute thread runs all n iterations (and their named barrier), also
     // after a wind-down, so no warp can be left waiting at the barrier
@@ -277,11 +286,12 @@ k_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CU
             const float p = valid ? ex2(__uint_as_float(s[e + u]) * c2 - lse2[col]) : 0.f;
             pe[u] = p;
             de[u] = p * (__uint_as_float(dp[e + u]) - dl[col]);
+            dsmax = fmaxf(dsmax, fabsf(de[u]));
           }
-          pk[e >> 1] = pack_bf16(pe[0], pe[1]);
-          dk[e >> 1] = pack_bf16(de[0], de[1]);
+          pk[e >> 1] = pack_f16(pe[0], pe[1]);
+          dk[e >> 1] = pack_f16(de[0], de[1]);
         }
-        // bf16 results go to columns already read (16 per 32 consumed)
+        // fp16 results go to columns already read (16 per 32 consumed)
         tmem_st16(tbase + la + 16 * c, pk);
         tmem_st16(tbase + la + 128 + 16 * c, dk);
       }
@@ -289,6 +299,7 @@ k_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CU
       tc_fence_before();
       mbar_arrive(&bars->ds_ready);
     }
+    if (!(dsmax <= kHalfMax)) report_error(err, LH_ERR_DEVICE, 101);
     if (ok && __all_sync(0xffffffffu, mbar_wait(&bars->done, 0, ab, err, 16))) {
       tc_fence_after();
       if (key < S) {
@@ -356,6 +367,7 @@ k_bwd_dq_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
     const int q = i * kT + r;
     const float lse2 = q < S ? lse[(size_t)bh * S + q] * 1.4426950408889634f : 0.f;
     const float dl = q < S ? delta[(size_t)bh * S + q] : 0.f;
+    float dsmax = 0.f;
     bool ok = true;
     for (int jj = 0; jj < n; ++jj) {
       if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_ready, jj & 1, ab, err, 17))) { ok = false; break; }
@@ -368,24 +380,31 @@ k_bwd_dq_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
         tmem_ld32(tbase + la + 32 * c, s);
         tmem_ld32(tbase + la + 128 + 32 * c, dp);
         tmem_wait_ld();
-        uint32_t dk[16];
+        uint32_t hi[16], lo[16];
 #pragma unroll
         for (int e = 0; e < 32; e += 2) {
-          float de[2];
+          float h[2], rl[2];
 #pragma unroll
           for (int u = 0; u < 2; ++u) {
             const int col = 32 * c + e + u;
             const float p = col <= klim ? ex2(__uint_as_float(s[e + u]) * c2 - lse2) : 0.f;
-            de[u] = p * (__uint_as_float(dp[e + u]) - dl);
+            const float ds = p * (__uint_as_float(dp[e + u]) - dl);
+            dsmax = fmaxf(dsmax, fabsf(ds));
+            h[u] = __half2float(__float2half_rn(ds));
+            rl[u] = ds - h[u];
           }
-          dk[e >> 1] = pack_bf16(de[0], de[1]);
+          hi[e >> 1] = pack_f16(h[0], h[1]);
+          lo[e >> 1] = pack_f16(rl[0], rl[1]);
         }
-        tmem_st16(tbase + la + 128 + 16 * c, dk);
+        // head into the (consumed) S columns, remainder into the (consumed) dP columns
+        tmem_st16(tbase + la + 16 * c, hi);
+        tmem_st16(tbase + la + 128 + 16 * c, lo);
       }
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&bars->ds_ready);
     }
+    if (!(dsmax <= kHalfMax)) report_error(err, LH_ERR_DEVICE, 101);
     if (ok && __all_sync(0xffffffffu, mbar_wait(&bars->done, 0, ab, err, 18))) {
       tc_fence_after();
       float* dst = dqs + ((size_t)bh * S + q) * D;
@@ -413,8 +432,8 @@ cudaError_t bwd_tc_t(const Geom& g, const void* qs, const void* ks, const void* 
                      cudaStream_t s) {
   CUtensorMap tq, tk, tv, tdo;
   const int BH = g.B * g.H;
-  if (!make_tmap_bf16(&tq, qs, D, g.S, BH) || !make_tmap_bf16(&tk, ks, D, g.S, BH) ||
-      !make_tmap_bf16(&tv, vs, D, g.S, BH) || !make_tmap_bf16(&tdo, dos, D, g.S, BH))
+  if (!make_tmap_16(&tq, qs, D, g.S, BH, true) || !make_tmap_16(&tk, ks, D, g.S, BH, true) ||
+      !make_tmap_16(&tv, vs, D, g.S, BH, true) || !make_tmap_16(&tdo, dos, D, g.S, BH, true))
     return cudaErrorInvalidValue;
   const int smem = BwdLayout<D>::BYTES;
   cudaError_t e = cudaFuncSetAttribute(k_bwd_dkdv_tc<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);

@@ -178,16 +178,19 @@ __global__ void __launch_bounds__(256) k_spread(const float* __restrict__ dqs,
 }
 
 // Backward of the scatter: dos[j] = sum of dout over the tokens entry j covers,
-// delta[j] = <dos_fp32[j], os[j]>. A thread owns 8 components of one head and
+// delta[j] = <dos_fp32[j], os[j]>. dos is stored as the backward's operand
+// type TO (fp16 for bf16 I/O: block sums of up to p^(L-1) tokens need more
+// significand than bf16 has; a sum beyond the fp16 range is reported as
+// LH_ERR_DEVICE, detail 100). A thread owns 8 components of one head and
 // walks the tokens of one coarsest block in order; level sums are fp32 and
 // formed level by level (each the left-to-right sum of its p children), so
 // every token row of dout is read exactly once.
-template <typename T, int LV>
+template <typename T, typename TO, int LV>
 __global__ void __launch_bounds__(256) k_blocksum(const T* __restrict__ dout,
                                                   const float* __restrict__ os,
                                                   const int32_t* __restrict__ slot,
-                                                  T* __restrict__ dos, float* __restrict__ delta,
-                                                  Geom g, int hg, int yb) {
+                                                  TO* __restrict__ dos, float* __restrict__ delta,
+                                                  Geom g, int hg, int yb, int* err) {
   const int C8 = g.D >> 3;
   const int b = blockIdx.z;
   const int head = blockIdx.y * hg + threadIdx.x / C8;
@@ -213,8 +216,12 @@ __global__ void __launch_bounds__(256) k_blocksum(const T* __restrict__ dout,
     }
     for (int off = C8 >> 1; off >= 1; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
     if (live && s >= 0) {
-      Vec8<T>::store_f32(dos + ((size_t)bh * g.S + s) * g.D + chunk * 8, v);
+      Vec8<TO>::store_f32(dos + ((size_t)bh * g.S + s) * g.D + chunk * 8, v);
       if (chunk == 0) delta[(size_t)bh * g.S + s] = part;
+      float mx = 0.f;
+#pragma unroll
+      for (int d = 0; d < 8; ++d) mx = fmaxf(mx, fabsf(v[d]));
+      if (sizeof(TO) == 2 && !(mx <= kHalfMax)) report_error(err, LH_ERR_DEVICE, 100);
     }
   };
 
@@ -265,10 +272,10 @@ __global__ void __launch_bounds__(256) k_blocksum(const T* __restrict__ dout,
 }
 
 // L == 1: dos = dout transposed to [B][H][N][D]; delta = <dout, os>.
-template <typename T>
+template <typename T, typename TO>
 __global__ void __launch_bounds__(256) k_blocksum_l1(const T* __restrict__ dout,
                                                      const float* __restrict__ os,
-                                                     T* __restrict__ dos, float* __restrict__ delta,
+                                                     TO* __restrict__ dos, float* __restrict__ delta,
                                                      Geom g) {
   const int C8 = g.D >> 3;
   const long long total = (long long)g.B * g.H * g.N * C8;
@@ -287,7 +294,7 @@ __global__ void __launch_bounds__(256) k_blocksum_l1(const T* __restrict__ dout,
 #pragma unroll
     for (int d = 0; d < 8; ++d) part = fmaf(x[d], ov[d], part);
     for (int off = C8 >> 1; off >= 1; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
-    Vec8<T>::store_f32(dos + r * g.D + c8 * 8, x);
+    Vec8<TO>::store_f32(dos + r * g.D + c8 * 8, x);
     if (c8 == 0) delta[r] = part;
   }
 }
@@ -324,10 +331,11 @@ cudaError_t spread_t(const Geom& g, const float* dqs, const float* dks, const fl
 
 template <typename T>
 cudaError_t blocksum_t(const Geom& g, const void* dout, const float* os, const int32_t* slot,
-                       void* dos, float* delta, cudaStream_t s) {
+                       void* dos, float* delta, int* err, cudaStream_t s) {
+  using TO = typename BwdOperand<T>::type;
   if (g.L == 1) {
     const long long total = (long long)g.B * g.H * g.N * (g.D / 8);
-    k_blocksum_l1<T><<<grid_for(total), 256, 0, s>>>((const T*)dout, os, (T*)dos, delta, g);
+    k_blocksum_l1<T, TO><<<grid_for(total), 256, 0, s>>>((const T*)dout, os, (TO*)dos, delta, g);
     count_launch();
     return cudaGetLastError();
   }
@@ -343,10 +351,10 @@ cudaError_t blocksum_t(const Geom& g, const void* dout, const float* os, const i
   dim3 block(hg * C8, yb);
   dim3 grid((ncoarse + yb - 1) / yb, g.H / hg, g.B);
   const T* d = (const T*)dout;
-  T* o = (T*)dos;
+  TO* o = (TO*)dos;
   switch (g.L - 1) {
 #define LH_BS_CASE(n) \
-    case n: k_blocksum<T, n><<<grid, block, 0, s>>>(d, os, slot, o, delta, g, hg, yb); break;
+    case n: k_blocksum<T, TO, n><<<grid, block, 0, s>>>(d, os, slot, o, delta, g, hg, yb, err); break;
     LH_BS_CASE(1) LH_BS_CASE(2) LH_BS_CASE(3) LH_BS_CASE(4)
     LH_BS_CASE(5) LH_BS_CASE(6) LH_BS_CASE(7)
 #undef LH_BS_CASE
@@ -372,9 +380,9 @@ cudaError_t launch_spread(const Geom& g, lh_dtype dt, const float* dqs, const fl
 }
 
 cudaError_t launch_scatter_bwd(const Geom& g, lh_dtype dt, const void* dout, const float* os,
-                               const int32_t* slot, void* dos, float* delta, cudaStream_t s) {
-  return dt == LH_BF16 ? blocksum_t<__nv_bfloat16>(g, dout, os, slot, dos, delta, s)
-                       : blocksum_t<float>(g, dout, os, slot, dos, delta, s);
+                               const int32_t* slot, void* dos, float* delta, int* err, cudaStream_t s) {
+  return dt == LH_BF16 ? blocksum_t<__nv_bfloat16>(g, dout, os, slot, dos, delta, err, s)
+                       : blocksum_t<float>(g, dout, os, slot, dos, delta, err, s);
 }
 
 }  // namespace lh

@@ -2,6 +2,7 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -123,6 +124,40 @@ template <> struct Vec8<float> {
   }
 };
 
+// fp16 rows: the backward's tensor-core operands (11-bit significand; every
+// bf16 value with magnitude in [2^-14, 65504] converts exactly).
+template <> struct Vec8<__half> {
+  static __device__ __forceinline__ void load_f32(const __half* p, float (&x)[8]) {
+    uint4 r = __ldg(reinterpret_cast<const uint4*>(p));
+    const __half2* h = reinterpret_cast<const __half2*>(&r);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      float2 f = __half22float2(h[i]);
+      x[2 * i] = f.x;
+      x[2 * i + 1] = f.y;
+    }
+  }
+  static __device__ __forceinline__ void store_f32(__half* p, const float (&x)[8]) {
+    uint4 r;
+    __half2* h = reinterpret_cast<__half2*>(&r);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) h[i] = __floats2half2_rn(x[2 * i], x[2 * i + 1]);
+    *reinterpret_cast<uint4*>(p) = r;
+  }
+};
+
+// Element type of the backward's sub-sequence operands (dos, and the q/k/v
+// copies the backward reads): fp16 for bf16 I/O, fp32 for fp32 I/O.
+template <typename T> struct BwdOperand { using type = float; };
+template <> struct BwdOperand<__nv_bfloat16> { using type = __half; };
+
+// Largest finite fp16 value; block sums beyond it are reported, not stored as inf.
+constexpr float kHalfMax = 65504.f;
+
+__device__ __forceinline__ void report_error(int* err, int code, int detail) {
+  if (err && atomicCAS(err, 0, code) == 0) atomicExch(err + 1, detail);
+}
+
 __device__ __forceinline__ void load8_f32(const float* p, float (&x)[8]) {
   float4 a = __ldg(reinterpret_cast<const float4*>(p));
   float4 b = __ldg(reinterpret_cast<const float4*>(p) + 1);
@@ -144,11 +179,11 @@ cudaError_t launch_select(const Geom& g, const double* sq, int32_t* sel, int32_t
                           int32_t* slot, int32_t* ws, cudaStream_t s);
 cudaError_t launch_gather(const Geom& g, lh_dtype dt, const void* q, const void* k, const void* v,
                           const void* pq, const void* pk, const void* pv, const int32_t* map,
-                          void* qs, void* ks, void* vs, cudaStream_t s);
+                          void* qs, void* ks, void* vs, void* qh, void* kh, void* vh, cudaStream_t s);
 cudaError_t launch_scatter(const Geom& g, lh_dtype dt, const float* os, const int32_t* slot,
                            void* o, cudaStream_t s);
 cudaError_t launch_scatter_bwd(const Geom& g, lh_dtype dt, const void* dout, const float* os,
-                               const int32_t* slot, void* dos, float* delta, cudaStream_t s);
+                               const int32_t* slot, void* dos, float* delta, int* err, cudaStream_t s);
 cudaError_t launch_spread(const Geom& g, lh_dtype dt, const float* dqs, const float* dks,
                           const float* dvs, const int32_t* slot, void* dq, void* dk, void* dv,
                           cudaStream_t s);
