@@ -30,6 +30,7 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
+from long_context_symmetric_b200 import dist as lhdist  # noqa: E402
 from long_context_symmetric_b200 import lh, synth  # noqa: E402
 
 METRIC = "Lighthouse attn fwd+bwd tokens/s at 512K on 1 B200; % HBM / tensor roofline"
@@ -189,24 +190,18 @@ def main():
         run_reference(args, w)
         return
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    info = lhdist.rank_info()
+    world, rank, local = info.world, info.rank, info.local
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    pg = None
-    if world > 1:
-        import datetime
-
-        import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
-        pg = dist
+    lhdist.init("nccl", dev, timeout_s=120)
 
     cfg = lh.make_config(w.B, w.H, w.N, w.D, w.p, w.L, w.K, w.dtype, w.mode)
     ws = lh.Workspace(cfg, dev, backward=True)
     pl = ws.plan
-    q, k, v = synth.make_inputs(w, device=dev, seed=w.seed + 101 * rank)
-    do = synth.make_dout(w, device=dev, seed=w.seed + 101 * rank)
+    seed = lhdist.replica_seed(w.seed, rank)       # each rank: its own batch of the workload
+    q, k, v = synth.make_inputs(w, device=dev, seed=seed)
+    do = synth.make_dout(w, device=dev, seed=seed)
     o, dq, dk, dv = (torch.empty_like(q) for _ in range(4))
     stream = torch.cuda.current_stream(dev)
     bwd_ops = (ws.qh, ws.kh, ws.vh) if w.dtype == "bf16" else (ws.qs, ws.ks, ws.vs)
@@ -245,8 +240,7 @@ def main():
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(stages) + 1)]
            for _ in range(args.steps)]
     sampler = ClockSampler(local)
-    if pg:
-        pg.barrier()
+    lhdist.barrier()
     torch.cuda.synchronize(dev)
     sampler.start()
     time.sleep(0.3)
@@ -260,13 +254,8 @@ def main():
     torch.cuda.synchronize(dev)
     launches = lh.launch_count() - launches0
     clocks = sampler.stop()
-    if pg:
-        pg.barrier()
-    ms_total = t_start.elapsed_time(t_end)
-    if pg:
-        t = torch.tensor([ms_total], device=dev)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        ms_total = float(t.item())
+    lhdist.barrier()
+    ms_total = lhdist.max_over_ranks(t_start.elapsed_time(t_end), dev)
     ms_step = ms_total / args.steps
     stage_ms = {s: sum(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(args.steps)) / args.steps
                 for j, s in enumerate(stages)}
@@ -294,20 +283,15 @@ def main():
 
         e2e_step()
         torch.cuda.synchronize(dev)
-        if pg:
-            pg.barrier()
+        lhdist.barrier()
         a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
         for _ in range(args.e2e_steps):
             e2e_step()
         b_.record(stream)
         torch.cuda.synchronize(dev)
-        e2e_ms = a.elapsed_time(b_) / args.e2e_steps
-        if pg:
-            t = torch.tensor([e2e_ms], device=dev)
-            pg.all_reduce(t, op=pg.ReduceOp.MAX)
-            e2e_ms = float(t.item())
-        e2e = {"value": world * w.B * w.N / (e2e_ms / 1e3), "unit": "tokens/s",
+        e2e_ms = lhdist.max_over_ranks(a.elapsed_time(b_) / args.e2e_steps, dev)
+        e2e = {"value": lhdist.job_throughput(w.B * w.N, world, e2e_ms / 1e3), "unit": "tokens/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
 
     peaks, peak_kind = load_peaks()
@@ -340,7 +324,7 @@ def main():
                         "sample": f"oracle fwd+bwd of head (0,0) of {workload_desc(w)}; {dt:.1f} s; "
                                   f"tokens/s scaled to all {w.B * w.H} heads"}
 
-    value = world * w.B * w.N / (ms_step / 1e3)
+    value = lhdist.job_throughput(w.B * w.N, world, ms_step / 1e3)
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
@@ -353,8 +337,7 @@ def main():
     }
     if rank == 0:
         print(json.dumps(line), flush=True)
-    if pg:
-        pg.destroy_process_group()
+    lhdist.shutdown()
 
 
 if __name__ == "__main__":

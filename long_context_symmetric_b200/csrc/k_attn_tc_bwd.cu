@@ -302,15 +302,17 @@ k_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CU
     if (!(dsmax <= kHalfMax)) report_error(err, LH_ERR_DEVICE, 101);
     if (ok && __all_sync(0xffffffffu, mbar_wait(&bars->done, 0, ab, err, 16))) {
       tc_fence_after();
-      if (key < S) {
-        float* ddv = dvs + ((size_t)bh * S + key) * D;
-        float* ddk = dks + ((size_t)bh * S + key) * D;
+      float* ddv = dvs + ((size_t)bh * S + key) * D;
+      float* ddk = dks + ((size_t)bh * S + key) * D;
 #pragma unroll 1
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t a[32], b[32];
-          tmem_ld32(tbase + la + 256 + 32 * c, a);
-          tmem_ld32(tbase + la + 256 + D + 32 * c, b);
-          tmem_wait_ld();
+      for (int c = 0; c < D / 32; ++c) {
+        // the TMEM loads are warp-collective (.sync.aligned): every lane runs
+        // them, rows past S included; only the stores are per-row
+        uint32_t a[32], b[32];
+        tmem_ld32(tbase + la + 256 + 32 * c, a);
+        tmem_ld32(tbase + la + 256 + D + 32 * c, b);
+        tmem_wait_ld();
+        if (key < S) {
 #pragma unroll
           for (int e = 0; e < 32; e += 4) {
             *reinterpret_cast<float4*>(ddv + 32 * c + e) =
@@ -320,15 +322,6 @@ k_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CU
                 make_float4(__uint_as_float(b[e]) * scale, __uint_as_float(b[e + 1]) * scale,
                             __uint_as_float(b[e + 2]) * scale, __uint_as_float(b[e + 3]) * scale);
           }
-        }
-      } else {
-        // rows past S still take part in the warp-collective TMEM loads
-#pragma unroll 1
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t a[32], b[32];
-          tmem_ld32(tbase + la + 256 + 32 * c, a);
-          tmem_ld32(tbase + la + 256 + D + 32 * c, b);
-          tmem_wait_ld();
         }
       }
     }
