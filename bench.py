@@ -60,7 +60,7 @@ def stage_work(w, pl):
     return {
         "pool": ("bytes", 3 * tok + 3 * B * H * E * D * e + 2 * B * H * E * 8),
         "select": ("bytes", 2 * B * H * E * 8 + B * H * (S + E + (w.L - 1) * w.K) * 4),
-        "gather": ("bytes", 6 * sub * e + (3 * sub * 2 if w.dtype == "bf16" else 0) + B * H * S * 4),
+        "gather": ("bytes", 6 * sub * e + B * H * S * 4),
         "attn_fwd": ("flops", 2.0 * B * H * S * S * D),
         "scatter": ("bytes", tok + sub * 4 + B * H * E * 4),
         "scatter_bwd": ("bytes", tok + sub * 4 + sub * (2 if w.dtype == "bf16" else 4) + B * H * S * 4),
@@ -204,7 +204,6 @@ def main():
     do = synth.make_dout(w, device=dev, seed=seed)
     o, dq, dk, dv = (torch.empty_like(q) for _ in range(4))
     stream = torch.cuda.current_stream(dev)
-    bwd_ops = (ws.qh, ws.kh, ws.vh) if w.dtype == "bf16" else (ws.qs, ws.ks, ws.vs)
     stages = ["pool", "select", "gather", "attn_fwd", "scatter", "scatter_bwd", "attn_bwd", "spread"]
 
     def step(ev=None):
@@ -216,8 +215,7 @@ def main():
         mark(1)
         lh.score_topk(cfg, ws.sq, ws.sel, ws.map, ws.slot, ws.ws, stream=stream)
         mark(2)
-        lh.gather(cfg, q, k, v, ws.pyr_q, ws.pyr_k, ws.pyr_v, ws.map, ws.qs, ws.ks, ws.vs,
-                  ws.qh, ws.kh, ws.vh, stream)
+        lh.gather(cfg, q, k, v, ws.pyr_q, ws.pyr_k, ws.pyr_v, ws.map, ws.qs, ws.ks, ws.vs, stream)
         mark(3)
         lh.attn_fwd(cfg, ws.qs, ws.ks, ws.vs, ws.os, ws.lse, stream)
         mark(4)
@@ -225,7 +223,7 @@ def main():
         mark(5)
         lh.scatter_bwd(cfg, do, ws.os, ws.slot, ws.dos, ws.delta, stream)
         mark(6)
-        lh.attn_bwd(cfg, *bwd_ops, ws.dos, ws.lse, ws.delta, ws.dqs, ws.dks, ws.dvs, stream)
+        lh.attn_bwd(cfg, ws.qs, ws.ks, ws.vs, ws.dos, ws.lse, ws.delta, ws.dqs, ws.dks, ws.dvs, stream)
         mark(7)
         lh.spread(cfg, ws.dqs, ws.dks, ws.dvs, ws.slot, dq, dk, dv, stream)
         mark(8)

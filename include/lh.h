@@ -33,8 +33,8 @@
  *   selection sel                          [B][H][L-1][K] int32 (row l-1: level l)
  *   gather map                             [B][H][S]      int32, (level << 28) | index
  *   slot table                             [B][H][E]      int32, 2*slot + expanded, or -1
- *   sub-sequence qs, ks, vs                [B][H][S][D]   dtype
- *   backward operands qh, kh, vh, dos      [B][H][S][D]   fp16 for bf16 I/O, fp32 for fp32 I/O
+ *   sub-sequence qs, ks, vs, and dos       [B][H][S][D]   attention operand type: fp16 for
+ *                                                         bf16 I/O, fp32 for fp32 I/O
  *   attention out os, grads dqs, dks, dvs  [B][H][S][D]   float
  *   lse, delta                             [B][H][S]      float
  */
@@ -136,19 +136,21 @@ lh_status lh_score_topk(const lh_config* cfg, const double* sq, int32_t* sel, in
                         int32_t* slot, void* ws, size_t ws_bytes, void* stream);
 
 /* Dense gather: sub-sequence row j of xs = entry map[j] of x (level 0: the
- * token row of q/k/v; level >= 1: the pyramid row). Bit-exact copy.
- * [LH] Fig. 1 (dense gather); "Lighthouse Attention Technique" (sort, then gather).
- * For bf16 I/O, qh/kh/vh (all three, or all NULL) receive fp16 copies of the
- * same rows in the same pass: the operands lh_attn_bwd needs. The conversion is
- * exact for bf16 values of magnitude in [2^-14, 65504]. Ignored for fp32 I/O. */
+ * token row of q/k/v; level >= 1: the pyramid row), in the attention operand
+ * type: an exact copy for fp32 I/O; for bf16 I/O the value in fp16, rounded to
+ * nearest-even, which is exact for every bf16 magnitude in [2^-14, 65504] (a
+ * magnitude above 65504 is reported by lh_get_device_error: LH_ERR_DEVICE,
+ * detail 102). fp16 gives the attention's P and dS operands 11 significant
+ * bits instead of bf16's 8. [LH] Fig. 1 (dense gather); "Lighthouse Attention
+ * Technique" (sort, then gather). */
 lh_status lh_gather(const lh_config* cfg, const void* q, const void* k, const void* v,
                     const void* pyr_q, const void* pyr_k, const void* pyr_v, const int32_t* map,
-                    void* qs, void* ks, void* vs, void* qh, void* kh, void* vh, void* stream);
+                    void* qs, void* ks, void* vs, void* stream);
 
 /* (iii) Causal attention on the sub-sequence, [LH] Eq. (1), scale 1/sqrt(D):
  * os = softmax(qs ks^T / sqrt(D) + causal mask) vs, lse = natural log of each
- * row's softmax denominator. bf16: tcgen05 tensor cores, fp32 accumulate;
- * fp32: fp32 SIMT. */
+ * row's softmax denominator. bf16 I/O: tcgen05 tensor cores on the fp16
+ * sub-sequence, P as fp16, fp32 accumulate; fp32 I/O: fp32 SIMT. */
 lh_status lh_attn_fwd(const lh_config* cfg, const void* qs, const void* ks, const void* vs,
                       float* os, float* lse, void* stream);
 
@@ -169,11 +171,11 @@ lh_status lh_scatter_bwd(const lh_config* cfg, const void* dout, const float* os
 
 /* Backward of (iii): gradients of Eq. (1) with P recomputed from lse:
  * dvs = P^T dos, dP = dos vs^T, dS = P o (dP - delta), dqs = dS ks / sqrt(D),
- * dks = dS^T qs / sqrt(D). Deterministic (no atomics). qs/ks/vs/dos are the
- * backward operands: for bf16 I/O the fp16 copies from lh_gather and the fp16
- * dos from lh_scatter_bwd (tcgen05 kernels, fp16 operands, fp32 accumulate);
- * for fp32 I/O the fp32 sub-sequence (SIMT kernels). A dS beyond the fp16
- * range is reported by lh_get_device_error (LH_ERR_DEVICE, detail 101). */
+ * dks = dS^T qs / sqrt(D). Deterministic (no atomics). bf16 I/O: tcgen05
+ * kernels on the fp16 sub-sequence and fp16 dos, fp32 accumulate (dS feeding
+ * dqs is split into an fp16 head and remainder); fp32 I/O: SIMT kernels. A dS
+ * beyond the fp16 range is reported by lh_get_device_error (LH_ERR_DEVICE,
+ * detail 101). */
 lh_status lh_attn_bwd(const lh_config* cfg, const void* qs, const void* ks, const void* vs,
                       const void* dos, const float* lse, const float* delta,
                       float* dqs, float* dks, float* dvs, void* stream);
@@ -189,8 +191,7 @@ typedef struct {
   void *pyr_q, *pyr_k, *pyr_v;   /* [B][H][E][D] dtype */
   double* sq;                    /* [2][B][H][E] */
   int32_t *sel, *map, *slot;     /* [B][H][L-1][K], [B][H][S], [B][H][E] */
-  void *qs, *ks, *vs;            /* [B][H][S][D] dtype */
-  void *qh, *kh, *vh;            /* [B][H][S][D] fp16 copies (bf16 I/O with a backward; else NULL) */
+  void *qs, *ks, *vs;            /* [B][H][S][D] fp16 (bf16 I/O) or fp32 */
   float *os, *lse;               /* [B][H][S][D], [B][H][S] */
   void* ws; size_t ws_bytes;     /* plan.ws_bytes */
   void* dos; float* delta;       /* [B][H][S][D] fp16 (bf16 I/O) or fp32, [B][H][S] */

@@ -3,8 +3,8 @@
 // "Long Context Pre-Training with Lighthouse Attention", Eq. (1) and §3.1
 // stage (iii): softmax(Q K^T / sqrt(d) + M) V with the lower-triangular mask,
 // on the gathered sub-sequence. This is the fp32 path (tensor cores cannot
-// hold fp32 operands at fp32 precision) and the reference-precision path for
-// bf16 inputs (each bf16 operand is widened to fp32 exactly).
+// hold fp32 operands at fp32 precision); with LH_ATTN_SIMT=1 it also serves
+// bf16 I/O (whose sub-sequence holds fp16 values, widened to fp32 exactly).
 //
 // Forward: one CTA per (b, h, 64-row query tile); K/V tiles of 64 rows staged
 // in shared memory as fp32 (row stride D+1 so the lane-per-key dot products are
@@ -342,9 +342,10 @@ cudaError_t bwd_t(const Geom& g, const void* qs, const void* ks, const void* vs,
 
 cudaError_t launch_attn_fwd_simt(const Geom& g, lh_dtype dt, const void* qs, const void* ks,
                                  const void* vs, float* os, float* lse, cudaStream_t s) {
+  // bf16 I/O: the sub-sequence holds fp16 values (see lh_gather)
   if (dt == LH_BF16)
-    return g.D == 64 ? fwd_t<__nv_bfloat16, 64>(g, qs, ks, vs, os, lse, s)
-                     : fwd_t<__nv_bfloat16, 128>(g, qs, ks, vs, os, lse, s);
+    return g.D == 64 ? fwd_t<__half, 64>(g, qs, ks, vs, os, lse, s)
+                     : fwd_t<__half, 128>(g, qs, ks, vs, os, lse, s);
   return g.D == 64 ? fwd_t<float, 64>(g, qs, ks, vs, os, lse, s)
                    : fwd_t<float, 128>(g, qs, ks, vs, os, lse, s);
 }
@@ -353,7 +354,7 @@ cudaError_t launch_attn_bwd_simt(const Geom& g, lh_dtype dt, const void* qs, con
                                  const void* vs, const void* dos, const float* lse,
                                  const float* delta, float* dqs, float* dks, float* dvs,
                                  cudaStream_t s) {
-  // bf16 I/O: the backward's operands are the fp16 copies (see lh_attn_bwd)
+  // bf16 I/O: the sub-sequence and dos hold fp16 values
   if (dt == LH_BF16)
     return g.D == 64 ? bwd_t<__half, 64>(g, qs, ks, vs, dos, lse, delta, dqs, dks, dvs, s)
                      : bwd_t<__half, 128>(g, qs, ks, vs, dos, lse, delta, dqs, dks, dvs, s);

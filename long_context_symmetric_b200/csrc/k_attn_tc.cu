@@ -1,9 +1,13 @@
-// Causal flash attention on the sub-sequence with tcgen05 tensor cores (bf16
-// in, fp32 accumulate), forward pass.
+// Causal flash attention on the sub-sequence with tcgen05 tensor cores (fp16
+// operands, fp32 accumulate), forward pass.
 //
 // "Long Context Pre-Training with Lighthouse Attention", Eq. (1) and §3.1
 // stage (iii): the gathered sub-sequence is a dense causal sequence, so this is
-// plain causal attention softmax(Q K^T / sqrt(d) + M) V over S entries.
+// plain causal attention softmax(Q K^T / sqrt(d) + M) V over S entries. For
+// bf16 I/O the sub-sequence arrives as exact fp16 values (lh_gather), and P
+// enters the P V product as fp16: 11 significant bits instead of bf16's 8
+// keep the output within the stated tolerance (with bf16 P, errors of 1.5e-2
+// in the attention output were measured on scaled inputs).
 //
 // One CTA per (b, h, 128-row query tile); heavy (late) tiles are scheduled
 // first. Warp roles (192 threads):
@@ -17,7 +21,7 @@
 //             TMEM, causal mask on the diagonal tile, online softmax in the
 //             exp2 domain with a lazily updated running max (the output is
 //             rescaled in TMEM only when the max grows by more than 2^8), P
-//             written to shared memory as bf16 in the MMA's K-major swizzled
+//             written to shared memory as fp16 in the MMA's K-major swizzled
 //             layout; finally O / l and lse are written.
 // Every mbarrier wait is bounded (tc::mbar_wait): on timeout the kernel records
 // LH_ERR_TIMEOUT, drains its outstanding copies and MMAs, frees TMEM, returns.
@@ -64,8 +68,8 @@ k_attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CU
               int S, float c2, int* err) {
   using Lay = FwdLayout<D>;
   constexpr int SUB = Lay::SUB;
-  constexpr uint32_t IDS = idesc_bf16(kBM, kBN, false);   // S = Q K^T, both K-major
-  constexpr uint32_t IDO = idesc_bf16(kBM, D, true);      // O = P V, V MN-major
+  constexpr uint32_t IDS = idesc_f16(kBM, kBN, false);    // S = Q K^T, both K-major
+  constexpr uint32_t IDO = idesc_f16(kBM, D, true);       // O = P V, V MN-major
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   FwdBars* bars = reinterpret_cast<FwdBars*>(sm + Lay::BAR);
@@ -141,7 +145,7 @@ k_attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CU
         for (int kk = 0; kk < kBN / 16; ++kk) {
           const uint64_t a = sdesc_sw128(sbase + Lay::P + (kk >> 2) * kSub + (kk & 3) * 32, 16, 1024);
           const uint64_t b = sdesc_sw128(sbase + Lay::V + st * SUB * kSub + kk * 2048, kSub, 1024);
-          umma_bf16(dO, a, b, IDO, (jj > 0 || kk > 0) ? 1u : 0u);
+          umma_f16(dO, a, b, IDO, (jj > 0 || kk > 0) ? 1u : 0u);
         }
         umma_commit(&bars->o_done);
         umma_commit(&bars->kv_empty[st]);
@@ -159,7 +163,7 @@ k_attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CU
           const uint32_t koff = (kk >> 2) * kSub + (kk & 3) * 32;
           const uint64_t a = sdesc_sw128(sbase + Lay::Q + koff, 16, 1024);
           const uint64_t b = sdesc_sw128(sbase + Lay::K + st * SUB * kSub + koff, 16, 1024);
-          umma_bf16(dS, a, b, IDS, kk > 0 ? 1u : 0u);
+          umma_f16(dS, a, b, IDS, kk > 0 ? 1u : 0u);
         }
         umma_commit(&bars->s_full[sb]);
         if (j >= 1 && !issue_pv(j - 1)) { ok = false; break; }
@@ -224,7 +228,7 @@ k_attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CU
         const float p0 = ex2(__uint_as_float(s[2 * c]) - m_new);
         const float p1 = ex2(__uint_as_float(s[2 * c + 1]) - m_new);
         sum += p0 + p1;
-        pk[c] = pack_bf16(p0, p1);
+        pk[c] = pack_f16(p0, p1);
       }
       l_run = l_run * alpha + sum;
       m_run = m_new;
@@ -316,8 +320,8 @@ static cudaError_t fwd_tc_t(const Geom& g, const void* qs, const void* ks, const
                             float* lse, int* err, cudaStream_t s) {
   CUtensorMap tq, tk, tv;
   const int BH = g.B * g.H;
-  if (!make_tmap_16(&tq, qs, D, g.S, BH, false) || !make_tmap_16(&tk, ks, D, g.S, BH, false) ||
-      !make_tmap_16(&tv, vs, D, g.S, BH, false))
+  if (!make_tmap_16(&tq, qs, D, g.S, BH, true) || !make_tmap_16(&tk, ks, D, g.S, BH, true) ||
+      !make_tmap_16(&tv, vs, D, g.S, BH, true))
     return cudaErrorInvalidValue;
   const int smem = FwdLayout<D>::BYTES;
   cudaError_t e = cudaFuncSetAttribute(k_attn_fwd_tc<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);

@@ -3,33 +3,33 @@
 // "Long Context Pre-Training with Lighthouse Attention", Fig. 1 (the dense
 // gather feeds one contiguous causal sequence to the attention); "Lighthouse
 // Attention Technique" (the selection is sorted by position, then gathered).
-// Row j of qs/ks/vs ([B][H][S][D]) is a bit-exact copy of entry map[j]: a token
-// row of q/k/v ([B][N][H][D]) for level 0, a pyramid row ([B][H][E][D]) above.
-// One thread moves 16 bytes; consecutive threads cover a row, so stores are
-// fully coalesced and each source row is read as whole 32-byte sectors.
-// For bf16 I/O the same pass can also write fp16 copies (qh, kh, vh), the
-// operands of the tensor-core backward; the conversion is exact for every bf16
-// value of magnitude in [2^-14, 65504].
+// Row j of qs/ks/vs ([B][H][S][D]) is entry map[j]: a token row of q/k/v
+// ([B][N][H][D]) for level 0, a pyramid row ([B][H][E][D]) above, stored in the
+// attention operand type: an exact copy for fp32 I/O; for bf16 I/O the fp16
+// value (nearest-even; exact for every bf16 magnitude in [2^-14, 65504], and a
+// magnitude above 65504 is reported as LH_ERR_DEVICE, detail 102). fp16 keeps
+// 11 significant bits for the attention's P and dS operands where bf16 keeps 8.
+// Reading 16 bytes per thread (8 bf16 -> 8 fp16, or 4 fp32); consecutive
+// threads cover a row, so stores are fully coalesced.
 #include "lh_common.cuh"
 
 namespace lh {
 namespace {
 
+template <bool TO_F16>
 __global__ void __launch_bounds__(256) k_gather(const uint4* __restrict__ q, const uint4* __restrict__ k,
                                                 const uint4* __restrict__ v, const uint4* __restrict__ pq,
                                                 const uint4* __restrict__ pk, const uint4* __restrict__ pv,
                                                 const int32_t* __restrict__ map, uint4* __restrict__ qs,
-                                                uint4* __restrict__ ks, uint4* __restrict__ vs,
-                                                uint4* __restrict__ qh, uint4* __restrict__ kh,
-                                                uint4* __restrict__ vh, Geom g,
-                                                int vpr /* 16-byte vectors per row */) {
+                                                uint4* __restrict__ ks, uint4* __restrict__ vs, Geom g,
+                                                int vpr /* 16-byte vectors per row */, int* err) {
   const long long rows = (long long)g.B * g.H * g.S;
   const long long total = rows * vpr;
   const int tensor = blockIdx.y;
   const uint4* x = tensor == 0 ? q : (tensor == 1 ? k : v);
   const uint4* px = tensor == 0 ? pq : (tensor == 1 ? pk : pv);
   uint4* xs = tensor == 0 ? qs : (tensor == 1 ? ks : vs);
-  uint4* xh = tensor == 0 ? qh : (tensor == 1 ? kh : vh);
+  bool big = false;
   for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
        i += (long long)gridDim.x * blockDim.x) {
     const long long row = i / vpr;
@@ -45,34 +45,43 @@ __global__ void __launch_bounds__(256) k_gather(const uint4* __restrict__ q, con
       src = px + (bh * g.E + g.off[l] + idx) * vpr;
     }
     const uint4 val = __ldg(src + c);
-    xs[i] = val;
-    if (xh) {
+    if (TO_F16) {
       const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&val);
       uint4 hv;
       __half2* h2 = reinterpret_cast<__half2*>(&hv);
 #pragma unroll
-      for (int u = 0; u < 4; ++u) h2[u] = __float22half2_rn(__bfloat1622float2(b2[u]));
-      xh[i] = hv;
+      for (int u = 0; u < 4; ++u) {
+        const float2 f = __bfloat1622float2(b2[u]);
+        big |= !(fabsf(f.x) <= kHalfMax) || !(fabsf(f.y) <= kHalfMax);
+        h2[u] = __float22half2_rn(f);
+      }
+      xs[i] = hv;
+    } else {
+      xs[i] = val;
     }
   }
+  if (TO_F16 && big) report_error(err, LH_ERR_DEVICE, 102);
 }
 
 }  // namespace
 
 cudaError_t launch_gather(const Geom& g, lh_dtype dt, const void* q, const void* k, const void* v,
                           const void* pq, const void* pk, const void* pv, const int32_t* map,
-                          void* qs, void* ks, void* vs, void* qh, void* kh, void* vh, cudaStream_t s) {
+                          void* qs, void* ks, void* vs, int* err, cudaStream_t s) {
   const int esz = dt == LH_BF16 ? 2 : 4;
   const int vpr = g.D * esz / 16;
   const long long total = (long long)g.B * g.H * g.S * vpr;
   long long blocks = (total + 255) / 256;
   if (blocks > 148 * 16) blocks = 148 * 16;
   dim3 grid((unsigned)blocks, 3);
-  k_gather<<<grid, 256, 0, s>>>((const uint4*)q, (const uint4*)k, (const uint4*)v, (const uint4*)pq,
-                                (const uint4*)pk, (const uint4*)pv, map, (uint4*)qs, (uint4*)ks,
-                                (uint4*)vs, dt == LH_BF16 ? (uint4*)qh : nullptr,
-                                dt == LH_BF16 ? (uint4*)kh : nullptr, dt == LH_BF16 ? (uint4*)vh : nullptr,
-                                g, vpr);
+  if (dt == LH_BF16)
+    k_gather<true><<<grid, 256, 0, s>>>((const uint4*)q, (const uint4*)k, (const uint4*)v,
+                                        (const uint4*)pq, (const uint4*)pk, (const uint4*)pv, map,
+                                        (uint4*)qs, (uint4*)ks, (uint4*)vs, g, vpr, err);
+  else
+    k_gather<false><<<grid, 256, 0, s>>>((const uint4*)q, (const uint4*)k, (const uint4*)v,
+                                         (const uint4*)pq, (const uint4*)pk, (const uint4*)pv, map,
+                                         (uint4*)qs, (uint4*)ks, (uint4*)vs, g, vpr, err);
   count_launch();
   return cudaGetLastError();
 }

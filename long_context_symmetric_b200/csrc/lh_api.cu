@@ -28,9 +28,9 @@ cudaError_t launch_attn_bwd_simt(const Geom& g, lh_dtype dt, const void* qs, con
 cudaError_t launch_attn_fwd_tc(const Geom& g, const void* qs, const void* ks, const void* vs,
                                float* os, float* lse, int* err, cudaStream_t s);
 
-// bf16 runs on the tcgen05 tensor-core kernel; fp32 on the fp32 SIMT kernel.
-// LH_ATTN_SIMT=1 in the environment routes bf16 through the SIMT kernel too
-// (same results up to fp32 rounding; a debugging aid).
+// bf16 I/O runs on the tcgen05 tensor-core kernels (fp16 operands); fp32 on
+// the fp32 SIMT kernels. LH_ATTN_SIMT=1 in the environment routes bf16 I/O
+// through the SIMT kernels too (a debugging aid).
 static bool force_simt() {
   const char* e = std::getenv("LH_ATTN_SIMT");
   return e && e[0] == '1';
@@ -192,17 +192,14 @@ lh_status lh_score_topk(const lh_config* cfg, const double* sq, int32_t* sel, in
 
 lh_status lh_gather(const lh_config* cfg, const void* q, const void* k, const void* v,
                     const void* pyr_q, const void* pyr_k, const void* pyr_v, const int32_t* map,
-                    void* qs, void* ks, void* vs, void* qh, void* kh, void* vh, void* stream) {
+                    void* qs, void* ks, void* vs, void* stream) {
   Geom g;
   lh_status st = make_geom(cfg, &g, nullptr);
   if (st != LH_OK) return st;
   LH_REQ(q); LH_REQ(k); LH_REQ(v); LH_REQ(map); LH_REQ(qs); LH_REQ(ks); LH_REQ(vs);
   if (g.L > 1) { LH_REQ(pyr_q); LH_REQ(pyr_k); LH_REQ(pyr_v); }
-  const bool copies = cfg->dtype == LH_BF16 && (qh || kh || vh);
-  if (copies) { LH_REQ(qh); LH_REQ(kh); LH_REQ(vh); }
   LH_CUDA(launch_gather(g, cfg->dtype, q, k, v, pyr_q, pyr_k, pyr_v, map, qs, ks, vs,
-                        copies ? qh : nullptr, copies ? kh : nullptr, copies ? vh : nullptr,
-                        (cudaStream_t)stream));
+                        device_error_ptr(), (cudaStream_t)stream));
   return LH_OK;
 }
 
@@ -283,7 +280,7 @@ lh_status lh_forward(const lh_config* cfg, const void* q, const void* k, const v
   if ((st = lh_score_topk(cfg, b->sq, b->sel, b->map, b->slot, b->ws, b->ws_bytes, stream)) != LH_OK)
     return st;
   if ((st = lh_gather(cfg, q, k, v, b->pyr_q, b->pyr_k, b->pyr_v, b->map, b->qs, b->ks, b->vs,
-                      b->qh, b->kh, b->vh, stream)) != LH_OK)
+                      stream)) != LH_OK)
     return st;
   if ((st = lh_attn_fwd(cfg, b->qs, b->ks, b->vs, b->os, b->lse, stream)) != LH_OK) return st;
   return lh_scatter(cfg, b->os, b->slot, o, stream);
@@ -295,17 +292,12 @@ lh_status lh_backward(const lh_config* cfg, const void* dout, void* dq, void* dk
   Geom g;
   lh_status st = make_geom(cfg, &g, nullptr);
   if (st != LH_OK) return st;
-  // the backward's q/k/v operands: fp16 copies for bf16 I/O, the sub-sequence itself for fp32
-  const bool h16 = cfg->dtype == LH_BF16;
-  const void* oq = h16 ? b->qh : b->qs;
-  const void* ok_ = h16 ? b->kh : b->ks;
-  const void* ov = h16 ? b->vh : b->vs;
   LH_REQ(dout); LH_REQ(dq); LH_REQ(dk); LH_REQ(dv); LH_REQ(b->os); LH_REQ(b->dos);
-  LH_REQ(b->delta); LH_REQ(oq); LH_REQ(ok_); LH_REQ(ov); LH_REQ(b->lse);
+  LH_REQ(b->delta); LH_REQ(b->qs); LH_REQ(b->ks); LH_REQ(b->vs); LH_REQ(b->lse);
   LH_REQ(b->dqs); LH_REQ(b->dks); LH_REQ(b->dvs);
   if (g.L > 1) LH_REQ(b->slot);
   if ((st = lh_scatter_bwd(cfg, dout, b->os, b->slot, b->dos, b->delta, stream)) != LH_OK) return st;
-  if ((st = lh_attn_bwd(cfg, oq, ok_, ov, b->dos, b->lse, b->delta, b->dqs, b->dks, b->dvs,
+  if ((st = lh_attn_bwd(cfg, b->qs, b->ks, b->vs, b->dos, b->lse, b->delta, b->dqs, b->dks, b->dvs,
                         stream)) != LH_OK)
     return st;
   return lh_spread(cfg, b->dqs, b->dks, b->dvs, b->slot, dq, dk, dv, stream);

@@ -146,8 +146,8 @@ template <> struct Vec8<__half> {
   }
 };
 
-// Element type of the backward's sub-sequence operands (dos, and the q/k/v
-// copies the backward reads): fp16 for bf16 I/O, fp32 for fp32 I/O.
+// Attention operand type of the sub-sequence (qs, ks, vs, dos): fp16 for bf16
+// I/O, fp32 for fp32 I/O.
 template <typename T> struct BwdOperand { using type = float; };
 template <> struct BwdOperand<__nv_bfloat16> { using type = __half; };
 
@@ -179,7 +179,7 @@ cudaError_t launch_select(const Geom& g, const double* sq, int32_t* sel, int32_t
                           int32_t* slot, int32_t* ws, cudaStream_t s);
 cudaError_t launch_gather(const Geom& g, lh_dtype dt, const void* q, const void* k, const void* v,
                           const void* pq, const void* pk, const void* pv, const int32_t* map,
-                          void* qs, void* ks, void* vs, void* qh, void* kh, void* vh, cudaStream_t s);
+                          void* qs, void* ks, void* vs, int* err, cudaStream_t s);
 cudaError_t launch_scatter(const Geom& g, lh_dtype dt, const float* os, const int32_t* slot,
                            void* o, cudaStream_t s);
 cudaError_t launch_scatter_bwd(const Geom& g, lh_dtype dt, const void* dout, const float* os,

@@ -47,8 +47,7 @@ class Plan(ctypes.Structure):
 class Buffers(ctypes.Structure):
     _fields_ = [("pyr_q", c_void_p), ("pyr_k", c_void_p), ("pyr_v", c_void_p), ("sq", c_void_p),
                 ("sel", c_void_p), ("map", c_void_p), ("slot", c_void_p), ("qs", c_void_p),
-                ("ks", c_void_p), ("vs", c_void_p), ("qh", c_void_p), ("kh", c_void_p),
-                ("vh", c_void_p), ("os", c_void_p), ("lse", c_void_p),
+                ("ks", c_void_p), ("vs", c_void_p), ("os", c_void_p), ("lse", c_void_p),
                 ("ws", c_void_p), ("ws_bytes", c_size_t), ("dos", c_void_p), ("delta", c_void_p),
                 ("dqs", c_void_p), ("dks", c_void_p), ("dvs", c_void_p)]
 
@@ -62,7 +61,7 @@ _SIGS = {
     "lh_pool": ([ctypes.POINTER(Config)] + [c_void_p] * 8, c_int),
     "lh_score_topk": ([ctypes.POINTER(Config), c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                        c_size_t, c_void_p], c_int),
-    "lh_gather": ([ctypes.POINTER(Config)] + [c_void_p] * 14, c_int),
+    "lh_gather": ([ctypes.POINTER(Config)] + [c_void_p] * 11, c_int),
     "lh_attn_fwd": ([ctypes.POINTER(Config)] + [c_void_p] * 6, c_int),
     "lh_scatter": ([ctypes.POINTER(Config)] + [c_void_p] * 4, c_int),
     "lh_scatter_bwd": ([ctypes.POINTER(Config)] + [c_void_p] * 6, c_int),
@@ -146,11 +145,9 @@ def score_topk(cfg, sq, sel, map_, slot, ws, ws_bytes=None, stream=None):
                                nbytes, _stream(stream)), "lh_score_topk")
 
 
-def gather(cfg, q, k, v, pyr_q, pyr_k, pyr_v, map_, qs, ks, vs, qh=None, kh=None, vh=None,
-           stream=None):
+def gather(cfg, q, k, v, pyr_q, pyr_k, pyr_v, map_, qs, ks, vs, stream=None):
     _check(lib().lh_gather(ctypes.byref(cfg), _p(q), _p(k), _p(v), _p(pyr_q), _p(pyr_k), _p(pyr_v),
-                           _p(map_), _p(qs), _p(ks), _p(vs), _p(qh), _p(kh), _p(vh),
-                           _stream(stream)), "lh_gather")
+                           _p(map_), _p(qs), _p(ks), _p(vs), _stream(stream)), "lh_gather")
 
 
 def attn_fwd(cfg, qs, ks, vs, os_, lse, stream=None):
@@ -209,13 +206,9 @@ class Workspace:
         self.sel = z(B, H, max(L - 1, 1), K, dtype=i32)
         self.map = z(B, H, S, dtype=i32)
         self.slot = z(B, H, e1, dtype=i32)
-        self.qs, self.ks, self.vs = (z(B, H, S, D) for _ in range(3))
-        # backward operands: fp16 copies of the sub-sequence for bf16 I/O
+        # attention operand type of the sub-sequence: fp16 for bf16 I/O
         bop = torch.float16 if cfg.dtype == LH_BF16 else dt
-        if backward and cfg.dtype == LH_BF16:
-            self.qh, self.kh, self.vh = (z(B, H, S, D, dtype=bop) for _ in range(3))
-        else:
-            self.qh = self.kh = self.vh = None
+        self.qs, self.ks, self.vs = (z(B, H, S, D, dtype=bop) for _ in range(3))
         self.os = z(B, H, S, D, dtype=f32)
         self.lse = z(B, H, S, dtype=f32)
         self.ws = z(max(pl.ws_bytes, 16), dtype=torch.uint8)
@@ -227,8 +220,7 @@ class Workspace:
             self.dos = self.delta = self.dqs = self.dks = self.dvs = None
         self.c = Buffers(
             _p(self.pyr_q), _p(self.pyr_k), _p(self.pyr_v), _p(self.sq), _p(self.sel), _p(self.map),
-            _p(self.slot), _p(self.qs), _p(self.ks), _p(self.vs), _p(self.qh), _p(self.kh),
-            _p(self.vh), _p(self.os), _p(self.lse),
+            _p(self.slot), _p(self.qs), _p(self.ks), _p(self.vs), _p(self.os), _p(self.lse),
             _p(self.ws), self.ws.numel(), _p(self.dos), _p(self.delta), _p(self.dqs), _p(self.dks),
             _p(self.dvs))
 

@@ -72,10 +72,7 @@ def test_entry_points_validate_before_launch():
     assert lib.lh_pool(r, None, a, a, a, a, a, a, None) == LH_ERR_NULL
     assert lib.lh_pool(r, m, a, a, a, a, a, a, None) == LH_ERR_ALIGN
     assert lib.lh_score_topk(r, a, a, a, a, a, 16, None) == LH_ERR_WORKSPACE
-    assert lib.lh_gather(r, a, a, a, a, a, a, None, a, a, a, None, None, None, None) == LH_ERR_NULL
-    cfg16 = lh.make_config(1, 2, 4096, 64, 4, 3, 16, "bf16")
-    # fp16 copies are all-or-none
-    assert lib.lh_gather(ctypes.byref(cfg16), a, a, a, a, a, a, a, a, a, a, a, None, None, None) == LH_ERR_NULL
+    assert lib.lh_gather(r, a, a, a, a, a, a, None, a, a, a, None) == LH_ERR_NULL
     assert lib.lh_attn_fwd(r, a, a, a, m, a, None) == LH_ERR_ALIGN
     assert lib.lh_scatter(r, a, None, a, None) == LH_ERR_NULL
     assert lib.lh_scatter_bwd(r, a, a, a, a, None, None) == LH_ERR_NULL
