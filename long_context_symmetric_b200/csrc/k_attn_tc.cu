@@ -20,9 +20,13 @@
 //   warps 2-5 softmax, one thread per query row (= TMEM lane): scores from
 //             TMEM, causal mask on the diagonal tile, online softmax in the
 //             exp2 domain with a lazily updated running max (the output is
-//             rescaled in TMEM only when the max grows by more than 2^8), P
-//             written to shared memory as fp16 in the MMA's K-major swizzled
-//             layout; finally O / l and lse are written.
+//             rescaled in TMEM only when the max grows by more than 2^8); P is
+//             split into an fp16 head (to shared memory, in the MMA's K-major
+//             swizzled layout) and an fp16 remainder (to spare TMEM columns),
+//             and O += P_hi V + P_lo V, so O carries P to about 2^-22 instead
+//             of fp16's 2^-12 (the backward's delta = <dO, O> needs that: at
+//             512K context with outlier tokens the fp16-only O put delta off
+//             by 0.07); finally O / l and lse are written.
 // Every mbarrier wait is bounded (tc::mbar_wait): on timeout the kernel records
 // LH_ERR_TIMEOUT, drains its outstanding copies and MMAs, frees TMEM, returns.
 #include <cudaTypedefs.h>
@@ -41,6 +45,7 @@ constexpr int kBN = 128;       // key rows per tile
 constexpr int kSub = 128 * 64 * 2;   // one 128-row x 64-column bf16 swizzle tile (16 KB)
 constexpr int kStages = 2;
 constexpr float kLn2f = 0.6931471805599453f;
+constexpr uint32_t kPlo = 384;       // TMEM columns of the fp16 remainder of P (64 columns)
 
 template <int D>
 struct FwdLayout {
@@ -147,6 +152,11 @@ k_attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CU
           const uint64_t b = sdesc_sw128(sbase + Lay::V + st * SUB * kSub + kk * 2048, kSub, 1024);
           umma_f16(dO, a, b, IDO, (jj > 0 || kk > 0) ? 1u : 0u);
         }
+#pragma unroll
+        for (int kk = 0; kk < kBN / 16; ++kk) {
+          const uint64_t b = sdesc_sw128(sbase + Lay::V + st * SUB * kSub + kk * 2048, kSub, 1024);
+          umma_f16_ts(dO, tbase + kPlo + 8 * kk, b, IDO, 1u);
+        }
         umma_commit(&bars->o_done);
         umma_commit(&bars->kv_empty[st]);
         return true;
@@ -222,13 +232,11 @@ k_attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CU
         alpha = ex2(m_run - m_new);
       }
       float sum = 0.f;
-      uint32_t pk[64];
 #pragma unroll
-      for (int c = 0; c < 64; ++c) {
-        const float p0 = ex2(__uint_as_float(s[2 * c]) - m_new);
-        const float p1 = ex2(__uint_as_float(s[2 * c + 1]) - m_new);
-        sum += p0 + p1;
-        pk[c] = pack_f16(p0, p1);
+      for (int c = 0; c < 128; ++c) {
+        const float pc = ex2(__uint_as_float(s[c]) - m_new);
+        sum += pc;
+        s[c] = __float_as_uint(pc);
       }
       l_run = l_run * alpha + sum;
       m_run = m_new;
@@ -249,11 +257,27 @@ k_attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CU
           tmem_wait_st();
         }
       }
+      // head fp16(P) to shared memory, remainder P - fp16(P) to TMEM (two per column)
 #pragma unroll
-      for (int c16 = 0; c16 < 16; ++c16) {
-        uint4 v = make_uint4(pk[4 * c16], pk[4 * c16 + 1], pk[4 * c16 + 2], pk[4 * c16 + 3]);
-        *reinterpret_cast<uint4*>(P0 + (c16 >> 3) * kSub + sw128_off(r, c16 & 7)) = v;
+      for (int c = 0; c < 4; ++c) {
+        uint32_t hi[16], lo[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const float p0 = __uint_as_float(s[32 * c + 2 * e]);
+          const float p1 = __uint_as_float(s[32 * c + 2 * e + 1]);
+          hi[e] = pack_f16(p0, p1);
+          const float2 h = __half22float2(*reinterpret_cast<const __half2*>(&hi[e]));
+          lo[e] = pack_f16(p0 - h.x, p1 - h.y);
+        }
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+          const int c16 = 4 * c + q4;       // 16-byte chunk (8 columns) of the 128-column row
+          *reinterpret_cast<uint4*>(P0 + (c16 >> 3) * kSub + sw128_off(r, c16 & 7)) =
+              make_uint4(hi[4 * q4], hi[4 * q4 + 1], hi[4 * q4 + 2], hi[4 * q4 + 3]);
+        }
+        tmem_st16(tbase + lane_addr + kPlo + 16 * c, lo);
       }
+      tmem_wait_st();
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(&bars->p_full);

@@ -178,7 +178,7 @@ __global__ void __launch_bounds__(256) k_spread(const float* __restrict__ dqs,
 }
 
 // Backward of the scatter: dos[j] = sum of dout over the tokens entry j covers,
-// delta[j] = <dos_fp32[j], os[j]>. dos is stored as the backward's operand
+// delta[j] = <dos[j], os[j]> with dos as stored. dos is stored as the backward's operand
 // type TO (fp16 for bf16 I/O: block sums of up to p^(L-1) tokens need more
 // significand than bf16 has; a sum beyond the fp16 range is reported as
 // LH_ERR_DEVICE, detail 100). A thread owns 8 components of one head and
@@ -211,8 +211,10 @@ __global__ void __launch_bounds__(256) k_blocksum(const T* __restrict__ dout,
     float ov[8];
     if (live && s >= 0) {
       load8_f32(os + ((size_t)bh * g.S + s) * g.D + chunk * 8, ov);
+      // delta from the stored (rounded) dos: the values the backward's dP uses
 #pragma unroll
-      for (int d = 0; d < 8; ++d) part = fmaf(v[d], ov[d], part);
+      for (int d = 0; d < 8; ++d)
+        part = fmaf(sizeof(TO) == 2 ? __half2float(__float2half_rn(v[d])) : v[d], ov[d], part);
     }
     for (int off = C8 >> 1; off >= 1; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
     if (live && s >= 0) {
