@@ -183,8 +183,14 @@ def main():
     ap.add_argument("--workload", default="ctx512k", choices=list(synth.WORKLOADS))
     ap.add_argument("--e2e-steps", type=int, default=2)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--heads", type=int, default=None,
+                    help="smaller case of the same recipe (fewer heads), e.g. for an ncu capture")
+    ap.add_argument("--tokens", type=int, default=None, help="smaller case of the same recipe (fewer tokens)")
     args = ap.parse_args()
     w = synth.WORKLOADS[args.workload]
+    if args.heads or args.tokens:
+        import dataclasses
+        w = dataclasses.replace(w, H=args.heads or w.H, N=args.tokens or w.N)
 
     if args.impl == "reference":
         run_reference(args, w)
