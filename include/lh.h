@@ -215,6 +215,25 @@ lh_status lh_get_device_error(void* stream, int* detail);
 /* Number of liblh kernels launched by this process so far. */
 unsigned long long lh_launch_count(void);
 
+/* lh_score_topk without a caller workspace (the paper has no counterpart: this
+ * is for callers, not the method). Some callers cannot provide or allocate a
+ * device workspace: a fixed arena that owns all device memory and may not
+ * grow, or a hot path that may not call cudaMalloc because it can synchronise
+ * the device. This variant keeps the descent's scratch in a fixed 8 MiB device
+ * array inside liblh, which every GPU that loads the library holds until the
+ * process exits; nothing is allocated per call.
+ * Same inputs, outputs, results and errors as lh_score_topk, plus
+ * LH_ERR_WORKSPACE when the problem needs more scratch than the array holds
+ * (plan.ws_bytes > 8 MiB, i.e. 5*S*B*H > 2,097,152; checked before any launch).
+ * The first call on each device looks up the array's device address
+ * (cudaGetSymbolAddress), so make that first call before any stream capture.
+ * All calls share the one array, and it keeps the previous call's contents
+ * (every scratch word is written before it is read, so nothing needs
+ * clearing). Calls that overlap on the GPU, from different streams or host
+ * threads, race on it: serialise them. */
+lh_status lh_score_topk_noalloc(const lh_config* cfg, const double* sq, int32_t* sel, int32_t* map,
+                                int32_t* slot, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

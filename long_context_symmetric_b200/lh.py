@@ -71,6 +71,7 @@ _SIGS = {
     "lh_backward": ([ctypes.POINTER(Config)] + [c_void_p] * 4 + [ctypes.POINTER(Buffers), c_void_p], c_int),
     "lh_get_device_error": ([c_void_p, ctypes.POINTER(c_int)], c_int),
     "lh_launch_count": ([], ctypes.c_ulonglong),
+    "lh_score_topk_noalloc": ([ctypes.POINTER(Config)] + [c_void_p] * 5, c_int),
 }
 
 
@@ -143,6 +144,12 @@ def score_topk(cfg, sq, sel, map_, slot, ws, ws_bytes=None, stream=None):
     nbytes = ws_bytes if ws_bytes is not None else (ws.numel() * ws.element_size() if ws is not None else 0)
     _check(lib().lh_score_topk(ctypes.byref(cfg), _p(sq), _p(sel), _p(map_), _p(slot), _p(ws),
                                nbytes, _stream(stream)), "lh_score_topk")
+
+
+def score_topk_noalloc(cfg, sq, sel, map_, slot, stream=None):
+    """lh_score_topk with the descent's scratch in liblh's fixed device array (no workspace)."""
+    _check(lib().lh_score_topk_noalloc(ctypes.byref(cfg), _p(sq), _p(sel), _p(map_), _p(slot),
+                                       _stream(stream)), "lh_score_topk_noalloc")
 
 
 def gather(cfg, q, k, v, pyr_q, pyr_k, pyr_v, map_, qs, ks, vs, stream=None):
