@@ -177,6 +177,174 @@ __global__ void __launch_bounds__(256) k_spread(const float* __restrict__ dqs,
   }
 }
 
+// Packed output row chunk: the value written for 8 components of one token.
+template <typename T> struct Packed;
+template <> struct Packed<__nv_bfloat16> {
+  uint4 v;
+  __device__ __forceinline__ void from(const Acc<0>& a) {
+    __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&v);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(a.v[2 * i], a.v[2 * i + 1]);
+  }
+  __device__ __forceinline__ void from(const Acc<1>& a) {
+    double o[8];
+    a.value64(o);
+    __nv_bfloat16* h = reinterpret_cast<__nv_bfloat16*>(&v);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) h[i] = __double2bfloat16(o[i]);
+  }
+  __device__ __forceinline__ void store(__nv_bfloat16* p) const { *reinterpret_cast<uint4*>(p) = v; }
+};
+template <> struct Packed<float> {
+  float4 a, b;
+  __device__ __forceinline__ void from(const Acc<0>& x) {
+    a = make_float4(x.v[0], x.v[1], x.v[2], x.v[3]);
+    b = make_float4(x.v[4], x.v[5], x.v[6], x.v[7]);
+  }
+  __device__ __forceinline__ void from(const Acc<1>& x) {
+    double o[8];
+    x.value64(o);
+    a = make_float4(__double2float_rn(o[0]), __double2float_rn(o[1]), __double2float_rn(o[2]),
+                    __double2float_rn(o[3]));
+    b = make_float4(__double2float_rn(o[4]), __double2float_rn(o[5]), __double2float_rn(o[6]),
+                    __double2float_rn(o[7]));
+  }
+  __device__ __forceinline__ void store(float* p) const {
+    reinterpret_cast<float4*>(p)[0] = a;
+    reinterpret_cast<float4*>(p)[1] = b;
+  }
+};
+
+// Contribution of one level-l row (weight 1/p^l when WEIGHTED and l >= 1, else 1).
+template <int FIXED, bool WEIGHTED>
+__device__ __forceinline__ void add_level(Acc<FIXED>& acc, const float (&x)[8], const Geom& g, int l) {
+  const double den = (WEIGHTED && l >= 1) ? (double)g.pl[l] : 1.0;
+  const double inv = g.pow2 ? 1.0 / den : 0.0;
+  acc.add(x, (float)(1.0 / den), den, inv);
+}
+
+// Scatter / spread walking one coarsest block in token order (L >= 2).
+// Every token under a level-l entry shares that entry's contribution, so the
+// thread keeps acc[l] = sum of the contributions of levels >= l and refreshes
+// it only where a level-l entry starts (integer countdowns, no division). When
+// no level-0 row covers the token (its level-1 parent was not expanded), the
+// output equals the previous token's and the converted value is stored again.
+// Result and summation order (coarse level first) are those of chain_sum.
+// One thread: 8 components of one head; CTA: a head group (x) by coarsest
+// blocks (y). grid.z = batch x tensors.
+template <typename T, int FIXED, bool WEIGHTED, int LV>
+__global__ void __launch_bounds__(256) k_scatter_tree(const float* __restrict__ s0,
+                                                      const float* __restrict__ s1,
+                                                      const float* __restrict__ s2,
+                                                      const int32_t* __restrict__ slot,
+                                                      T* __restrict__ d0, T* __restrict__ d1,
+                                                      T* __restrict__ d2, Geom g, int hg, int yb,
+                                                      int ntens) {
+  const int C8 = g.D >> 3;
+  const int tensor = blockIdx.z % ntens;
+  const int b = blockIdx.z / ntens;
+  const int head = blockIdx.y * hg + threadIdx.x / C8;
+  const int chunk = threadIdx.x % C8;
+  const int cb = blockIdx.x * yb + threadIdx.y;
+  if (cb >= g.n[LV]) return;           // no collectives below: a thread may leave
+  const float* src = tensor == 0 ? s0 : (tensor == 1 ? s1 : s2);
+  T* dst = tensor == 0 ? d0 : (tensor == 1 ? d1 : d2);
+  const long long bh = (long long)b * g.H + head;
+  const int32_t* slot_h = slot + bh * g.E;
+  const float* srow = src + (size_t)bh * g.S * g.D + chunk * 8;
+  const long long P = g.pl[LV];
+  const size_t tstride = (size_t)g.H * g.D;
+  T* out = dst + ((size_t)b * g.N + (size_t)cb * P) * tstride + (size_t)head * g.D + chunk * 8;
+
+  Acc<FIXED> acc[LV + 1];              // acc[l]: contributions of levels >= l (l >= 1)
+  bool expd[LV + 1];                   // entry of level l expanded (its children included)
+  int rem[LV + 1];                     // tokens left in the current level-l entry
+  int idx[LV + 1];                     // index of the current level-l entry
+  float x[8];
+  int sl1 = 0, r0 = 0;                 // slot of the current level-1 entry, token offset in it
+  {
+    const int e = __ldg(slot_h + g.off[LV] + cb);
+    load8_f32(srow + (size_t)(e >> 1) * g.D, x);
+    acc[LV].zero();
+    add_level<FIXED, WEIGHTED>(acc[LV], x, g, LV);
+    expd[LV] = e & 1;
+    if (LV == 1) sl1 = e >> 1;
+  }
+#pragma unroll
+  for (int l = 1; l < LV; ++l) {
+    rem[l] = 0;
+    idx[l] = (int)((long long)cb * (P / g.pl[l])) - 1;
+  }
+  Packed<T> pk;
+  bool pk_ok = false;
+  for (long long t = 0; t < P; ++t) {
+#pragma unroll
+    for (int l = LV - 1; l >= 1; --l) {
+      if (rem[l] == 0) {               // a level-l entry starts here (finer ones too)
+        rem[l] = (int)g.pl[l];
+        ++idx[l];
+        if (expd[l + 1]) {
+          const int e = __ldg(slot_h + g.off[l] + idx[l]);
+          load8_f32(srow + (size_t)(e >> 1) * g.D, x);
+          acc[l] = acc[l + 1];
+          add_level<FIXED, WEIGHTED>(acc[l], x, g, l);
+          expd[l] = e & 1;
+          if (l == 1) sl1 = e >> 1;
+        } else {
+          acc[l] = acc[l + 1];
+          expd[l] = false;
+        }
+        if (l == 1) r0 = 0;
+        pk_ok = false;
+      }
+      --rem[l];
+    }
+    T* o = out + (size_t)t * tstride;
+    if (expd[1]) {                     // the token itself is in the sub-sequence
+      load8_f32(srow + (size_t)(sl1 - g.p + r0) * g.D, x);
+      Acc<FIXED> a = acc[1];
+      add_level<FIXED, WEIGHTED>(a, x, g, 0);
+      Packed<T> q;
+      q.from(a);
+      q.store(o);
+    } else {
+      if (!pk_ok) {
+        pk.from(acc[1]);
+        pk_ok = true;
+      }
+      pk.store(o);
+    }
+    if (LV == 1 && ++r0 == g.p) r0 = 0;
+    else if (LV > 1) ++r0;
+  }
+}
+
+template <typename T, int FIXED, bool WEIGHTED>
+cudaError_t tree_t(const Geom& g, const float* s0, const float* s1, const float* s2,
+                   const int32_t* slot, T* d0, T* d1, T* d2, int ntens, cudaStream_t s) {
+  const int C8 = g.D / 8;
+  int hg = g.H;
+  while (hg * C8 > 256) {
+    --hg;
+    while (g.H % hg) --hg;
+  }
+  const int ncoarse = g.n[g.L - 1];
+  int yb = 1;
+  while (yb * 2 * hg * C8 <= 256 && yb * 2 <= ncoarse) yb *= 2;
+  dim3 block(hg * C8, yb);
+  dim3 grid((ncoarse + yb - 1) / yb, g.H / hg, g.B * ntens);
+  switch (g.L - 1) {
+#define LH_TREE_CASE(n) \
+    case n: k_scatter_tree<T, FIXED, WEIGHTED, n><<<grid, block, 0, s>>>(s0, s1, s2, slot, d0, d1, d2, g, hg, yb, ntens); break;
+    LH_TREE_CASE(1) LH_TREE_CASE(2) LH_TREE_CASE(3) LH_TREE_CASE(4)
+    LH_TREE_CASE(5) LH_TREE_CASE(6) LH_TREE_CASE(7)
+#undef LH_TREE_CASE
+    default: return cudaErrorInvalidValue;
+  }
+  count_launch();
+  return cudaGetLastError();
+}
+
 // Backward of the scatter: dos[j] = sum of dout over the tokens entry j covers,
 // delta[j] = <dos[j], os[j]> with dos as stored. dos is stored as the backward's operand
 // type TO (fp16 for bf16 I/O: block sums of up to p^(L-1) tokens need more
@@ -309,6 +477,10 @@ int grid_for(long long total) {
 
 template <typename T>
 cudaError_t scatter_t(const Geom& g, const float* os, const int32_t* slot, void* o, cudaStream_t s) {
+  if (g.L > 1)
+    return g.accum == LH_ACC_FIXED64
+               ? tree_t<T, 1, false>(g, os, os, os, slot, (T*)o, (T*)o, (T*)o, 1, s)
+               : tree_t<T, 0, false>(g, os, os, os, slot, (T*)o, (T*)o, (T*)o, 1, s);
   const long long total = (long long)g.B * g.N * g.H * (g.D / 8);
   if (g.accum == LH_ACC_FIXED64)
     k_scatter<T, 1><<<grid_for(total), 256, 0, s>>>(os, slot, (T*)o, g);
@@ -321,6 +493,10 @@ cudaError_t scatter_t(const Geom& g, const float* os, const int32_t* slot, void*
 template <typename T>
 cudaError_t spread_t(const Geom& g, const float* dqs, const float* dks, const float* dvs,
                      const int32_t* slot, void* dq, void* dk, void* dv, cudaStream_t s) {
+  if (g.L > 1)
+    return g.accum == LH_ACC_FIXED64
+               ? tree_t<T, 1, true>(g, dqs, dks, dvs, slot, (T*)dq, (T*)dk, (T*)dv, 3, s)
+               : tree_t<T, 0, true>(g, dqs, dks, dvs, slot, (T*)dq, (T*)dk, (T*)dv, 3, s);
   const long long total = (long long)g.B * g.N * g.H * (g.D / 8);
   dim3 grid(grid_for(total), 3);
   if (g.accum == LH_ACC_FIXED64)
