@@ -399,29 +399,42 @@ __global__ void __launch_bounds__(256) k_blocksum(const T* __restrict__ dout,
   const long long ngroups = P / p;
   for (long long g1 = 0; g1 < ngroups; ++g1) {
     const long long i1 = (long long)cb * (P / p) + g1;      // level-1 index
+    // the group's token rows and its level-1 slot entry, all loads issued together
     const int e1 = live ? __ldg(slot_h + g.off[1] + (int)i1) : -1;
-    const int s1 = e1 >= 0 ? (e1 >> 1) : -1;
-    const bool tok_in = e1 >= 0 && (e1 & 1);                 // children (tokens) included
     float s[8];
-    for (int c = 0; c < p; ++c) {
-      float x[8];
-      if (live) Vec8<T>::load_f32(src + (size_t)(g1 * p + c) * tok_stride, x);
-      else {
+    for (int c0 = 0; c0 < p; c0 += 8) {
+      const int nb = min(8, p - c0);
+      typename Vec8<T>::Raw raw[8];
 #pragma unroll
-        for (int d = 0; d < 8; ++d) x[d] = 0.f;
+      for (int u = 0; u < 8; ++u)
+        if (u < nb && live) Vec8<T>::load_raw(src + (size_t)(g1 * p + c0 + u) * tok_stride, raw[u]);
+      const int s1 = e1 >= 0 ? (e1 >> 1) : -1;
+      const bool tok_in = e1 >= 0 && (e1 & 1);               // children (tokens) included
+      // tokens are emitted only where some lane of the warp has them included
+      const bool any_tok = __any_sync(0xffffffffu, tok_in);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        if (u < nb) {
+          float x[8];
+          if (live) Vec8<T>::raw_f32(raw[u], x);
+          else {
+#pragma unroll
+            for (int d = 0; d < 8; ++d) x[d] = 0.f;
+          }
+          if (c0 + u == 0) {
+#pragma unroll
+            for (int d = 0; d < 8; ++d) s[d] = x[d];
+          } else {
+#pragma unroll
+            for (int d = 0; d < 8; ++d) s[d] = __fadd_rn(s[d], x[d]);
+          }
+          if (any_tok) emit(tok_in ? s1 - p + c0 + u : -1, x);
+        }
       }
-      if (c == 0) {
-#pragma unroll
-        for (int d = 0; d < 8; ++d) s[d] = x[d];
-      } else {
-#pragma unroll
-        for (int d = 0; d < 8; ++d) s[d] = __fadd_rn(s[d], x[d]);
-      }
-      emit(tok_in ? s1 - p + c : -1, x);
     }
 #pragma unroll
     for (int d = 0; d < 8; ++d) acc[1][d] = s[d];
-    emit(s1, s);
+    if (__any_sync(0xffffffffu, e1 >= 0)) emit(e1 >= 0 ? (e1 >> 1) : -1, s);
     long long gi = i1;
 #pragma unroll
     for (int l = 2; l <= LV; ++l) {
@@ -436,7 +449,7 @@ __global__ void __launch_bounds__(256) k_blocksum(const T* __restrict__ dout,
       if (pos != p - 1) break;
       gi /= p;
       const int e = live ? __ldg(slot_h + g.off[l] + (int)gi) : -1;
-      emit(e >= 0 ? (e >> 1) : -1, acc[l]);
+      if (__any_sync(0xffffffffu, e >= 0)) emit(e >= 0 ? (e >> 1) : -1, acc[l]);
     }
   }
 }
