@@ -14,10 +14,10 @@
 // bf16 sub-sequence. Two kernels, each one CTA per 128-row tile, heavy tiles
 // first:
 //  k_bwd_dkdv_tc  per key tile j, over query tiles i >= j:
-//      S^T = K_j Q_i^T and dP^T = V_j dO_i^T into TMEM; the compute warps (one
-//      thread per key row = TMEM lane) form P^T and dS^T and store them as fp16
-//      back into the same TMEM columns; then dV += P^T dO_i and dK += dS^T Q_i
-//      take their A operand straight from TMEM.
+//      S^T = K_j Q_i^T and dP^T = V_j dO_i^T into TMEM; the compute warps (two
+//      per TMEM lane quarter, each on half of the columns) form P^T and dS^T
+//      and store them as fp16 back into the same TMEM columns; then
+//      dV += P^T dO_i and dK += dS^T Q_i take their A operand from TMEM.
 //  k_bwd_dq_tc    per query tile i, over key tiles j <= i:
 //      S = Q_i K_j^T and dP = dO_i V_j^T into TMEM; dS split into an fp16 head
 //      and an fp16 remainder (dS = hi + lo to about 2^-22 relative) back into
@@ -39,6 +39,11 @@ using namespace tc;
 constexpr int kT = 128;              // rows per tile (both directions)
 constexpr int kSub = 128 * 64 * 2;   // 128 x 64 bf16 swizzle tile
 constexpr int kStages = 2;
+// Warp roles: 0 producer, 1 MMA issuer, 2..9 compute. Two compute warps share
+// each TMEM lane quarter (warps w and w+4), each taking half of a tile's 128
+// columns, so every SM sub-partition has two compute warps to interleave.
+constexpr int kComputeThreads = 256;
+constexpr int kThreads = 64 + kComputeThreads;
 
 __device__ __forceinline__ void named_bar_sync(int id, int n) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
@@ -71,7 +76,7 @@ __device__ __forceinline__ void bwd_setup(BwdBars* bars, int warp) {
       mbar_init(&bars->ring_empty[s], 1);
     }
     mbar_init(&bars->s_ready, 1);
-    mbar_init(&bars->ds_ready, 128);
+    mbar_init(&bars->ds_ready, kComputeThreads);
     mbar_init(&bars->acc_done, 1);
     mbar_init(&bars->done, 1);
     mbar_init(&bars->drain, 1);
@@ -153,14 +158,17 @@ __device__ void bwd_mma(uint8_t* sm, BwdBars* bars, uint32_t tbase, int n, volat
     const uint32_t tileA = ring, tileB = ring + SUB * kSub;
 #pragma unroll
     for (int kk = 0; kk < kT / 16; ++kk) {
+      // packed operand columns: k-steps 0-3 at 8kk, 4-7 at 8kk + 32 (each half
+      // of the tile packs into its own 64 columns)
+      const uint32_t acol = 8 * kk + (kk >= 4 ? 32 : 0);
       const uint64_t g = sdesc_sw128(tileA + kk * 2048, kSub, 1024);
       if (TWO_ACC) {
         const uint64_t b = sdesc_sw128(tileB + kk * 2048, kSub, 1024);
-        umma_f16_ts(tAcc0, tX + 8 * kk, b, IDACC, (tt > 0 || kk > 0) ? 1u : 0u);
+        umma_f16_ts(tAcc0, tX + acol, b, IDACC, (tt > 0 || kk > 0) ? 1u : 0u);
       } else {
-        umma_f16_ts(tAcc1, tX + 8 * kk, g, IDACC, (tt > 0 || kk > 0) ? 1u : 0u);
+        umma_f16_ts(tAcc1, tX + acol, g, IDACC, (tt > 0 || kk > 0) ? 1u : 0u);
       }
-      umma_f16_ts(tAcc1, tY + 8 * kk, g, IDACC, (TWO_ACC && tt == 0 && kk == 0) ? 0u : 1u);
+      umma_f16_ts(tAcc1, tY + acol, g, IDACC, (TWO_ACC && tt == 0 && kk == 0) ? 0u : 1u);
     }
     umma_commit(&bars->ring_empty[st]);
     return true;
@@ -201,7 +209,7 @@ __device__ void bwd_mma(uint8_t* sm, BwdBars* bars, uint32_t tbase, int n, volat
 
 // ---------------------------------------------------------------- dK, dV
 template <int D>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(kThreads, 1)
 k_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
               const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tdo,
               const float* __restrict__ lse, const float* __restrict__ delta, float* __restrict__ dks,
@@ -225,8 +233,9 @@ k_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CU
     if (lane == 0) bwd_mma<D, true>(sm, bars, tbase, n, ab, err);
   } else {
     const int quarter = warp & 3;
+    const int half = (warp - 2) >> 2;                   // which 64 of the 128 columns
     const int m = quarter * 32 + lane;                  // key row within the tile / TMEM lane
-    const int ctid = threadIdx.x - 64;                  // 0..127
+    const int ctid = threadIdx.x - 64;                  // 0..255
     const uint32_t la = (uint32_t)(quarter * 32) << 16;
     const int key = j * kT + m;
     float* vec = reinterpret_cast<float*>(sm + Lay::VEC);   // [2][2][128]: lse2, delta
@@ -239,18 +248,18 @@ k_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CU
       float* lse2 = vec + (t & 1) * 256;
       float* dl = lse2 + 128;
       {
-        const int q = i * kT + ctid;
-        lse2[ctid] = q < S ? lse[(size_t)bh * S + q] * 1.4426950408889634f : 0.f;
-        dl[ctid] = q < S ? delta[(size_t)bh * S + q] : 0.f;
+        const int q = i * kT + (ctid & 127);
+        if (ctid < 128) lse2[ctid] = q < S ? lse[(size_t)bh * S + q] * 1.4426950408889634f : 0.f;
+        else dl[ctid - 128] = q < S ? delta[(size_t)bh * S + q] : 0.f;
       }
-      named_bar_sync(1, 128);
+      named_bar_sync(1, kComputeThreads);
       if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bars->s_ready, t & 1, ab, err, 15));
       if (!ok) continue;
       tc_fence_after();
       const bool diag = (i == j);
       const int qlim = S - 1 - i * kT;                  // last valid query column
 #pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
+      for (int c = 2 * half; c < 2 * half + 2; ++c) {
         uint32_t s[32], dp[32];
         tmem_ld32(tbase + la + 32 * c, s);
         tmem_ld32(tbase + la + 128 + 32 * c, dp);
@@ -271,9 +280,10 @@ k_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CU
           pk[e >> 1] = pack_f16(pe[0], pe[1]);
           dk[e >> 1] = pack_f16(de[0], de[1]);
         }
-        // fp16 results go to columns already read (16 per 32 consumed)
-        tmem_st16(tbase + la + 16 * c, pk);
-        tmem_st16(tbase + la + 128 + 16 * c, dk);
+        // fp16 results go to columns this warp has already read: chunk c's 16
+        // packed columns at 16c + 32*half (each half packs inside its own 64)
+        tmem_st16(tbase + la + 16 * c + 32 * half, pk);
+        tmem_st16(tbase + la + 128 + 16 * c + 32 * half, dk);
       }
       tmem_wait_st();
       tc_fence_before();
@@ -285,7 +295,7 @@ k_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CU
       float* ddv = dvs + ((size_t)bh * S + key) * D;
       float* ddk = dks + ((size_t)bh * S + key) * D;
 #pragma unroll 1
-      for (int c = 0; c < D / 32; ++c) {
+      for (int c = half * (D / 64); c < (half + 1) * (D / 64); ++c) {
         // the TMEM loads are warp-collective (.sync.aligned): every lane runs
         // them, rows past S included; only the stores are per-row
         uint32_t a[32], b[32];
@@ -311,7 +321,7 @@ k_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CU
 
 // ---------------------------------------------------------------- dQ
 template <int D>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(kThreads, 1)
 k_bwd_dq_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
             const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tdo,
             const float* __restrict__ lse, const float* __restrict__ delta, float* __restrict__ dqs,
@@ -335,6 +345,7 @@ k_bwd_dq_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
     if (lane == 0) bwd_mma<D, false>(sm, bars, tbase, n, ab, err);
   } else {
     const int quarter = warp & 3;
+    const int half = (warp - 2) >> 2;             // which 64 of the 128 columns
     const int r = quarter * 32 + lane;            // query row within the tile / TMEM lane
     const uint32_t la = (uint32_t)(quarter * 32) << 16;
     const int q = i * kT + r;
@@ -348,7 +359,7 @@ k_bwd_dq_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
       const bool diag = (jj == i);
       const int klim = min(diag ? r : kT - 1, S - 1 - jj * kT);   // last valid key column
 #pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
+      for (int c = 2 * half; c < 2 * half + 2; ++c) {
         uint32_t s[32], dp[32];
         tmem_ld32(tbase + la + 32 * c, s);
         tmem_ld32(tbase + la + 128 + 32 * c, dp);
@@ -369,9 +380,10 @@ k_bwd_dq_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
           hi[e >> 1] = pack_f16(h[0], h[1]);
           lo[e >> 1] = pack_f16(rl[0], rl[1]);
         }
-        // head into the (consumed) S columns, remainder into the (consumed) dP columns
-        tmem_st16(tbase + la + 16 * c, hi);
-        tmem_st16(tbase + la + 128 + 16 * c, lo);
+        // head into the (consumed) S columns, remainder into the (consumed) dP
+        // columns, packed inside this half's own 64 columns
+        tmem_st16(tbase + la + 16 * c + 32 * half, hi);
+        tmem_st16(tbase + la + 128 + 16 * c + 32 * half, lo);
       }
       tmem_wait_st();
       tc_fence_before();
@@ -382,7 +394,7 @@ k_bwd_dq_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
       tc_fence_after();
       float* dst = dqs + ((size_t)bh * S + q) * D;
 #pragma unroll 1
-      for (int c = 0; c < D / 32; ++c) {
+      for (int c = half * (D / 64); c < (half + 1) * (D / 64); ++c) {
         uint32_t a[32];
         tmem_ld32(tbase + la + 256 + 32 * c, a);
         tmem_wait_ld();
@@ -416,11 +428,11 @@ cudaError_t bwd_tc_t(const Geom& g, const void* qs, const void* ks, const void* 
   const float scale = (float)(1.0 / sqrt((double)D));
   const float c2 = (float)(1.4426950408889634 / sqrt((double)D));
   dim3 grid((g.S + kT - 1) / kT, BH);
-  k_bwd_dkdv_tc<D><<<grid, 192, smem, s>>>(tq, tk, tv, tdo, lse, delta, dks, dvs, g.S, c2, scale, err);
+  k_bwd_dkdv_tc<D><<<grid, kThreads, smem, s>>>(tq, tk, tv, tdo, lse, delta, dks, dvs, g.S, c2, scale, err);
   count_launch();
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  k_bwd_dq_tc<D><<<grid, 192, smem, s>>>(tq, tk, tv, tdo, lse, delta, dqs, g.S, c2, scale, err);
+  k_bwd_dq_tc<D><<<grid, kThreads, smem, s>>>(tq, tk, tv, tdo, lse, delta, dqs, g.S, c2, scale, err);
   count_launch();
   return cudaGetLastError();
 }
