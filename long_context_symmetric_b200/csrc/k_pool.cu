@@ -19,115 +19,164 @@
 // D/8 lanes of a head are consecutive lanes of one warp. A thread walks the
 // p^(L-1) tokens of one coarsest-level block in order, keeping one running fp64
 // sum per level (carry chain), and emits each entry when its last child is in.
+// Rows arrive through a shared-memory ring filled by bulk async copies.
 // HBM traffic: every token row is read once; pyramid rows and norms written once.
-#include "lh_common.cuh"
+#include "tc_ptx.cuh"
 
 namespace lh {
 namespace {
 
+using tc::mbar_init;
+using tc::fence_mbar_init;
+using tc::mbar_expect_tx;
+using tc::smem_u32;
+
 struct PoolArgs {
   Geom g;
-  int hg;        // heads per CTA
-  int yb;        // coarsest blocks per CTA (blockDim.y)
-  int ncoarse;   // coarsest blocks per batch row
+  int hg;          // heads per CTA (a divisor of H)
+  int ts;          // tokens per shared-memory stage
+  int ns;          // stages in the ring
+  int row_bytes;   // bytes of one token row of the head group
 };
 
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+      ::"r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// One CTA: one coarsest block of one tensor for one head group. Token rows of
+// the head group stream through a ring of shared-memory stages filled by 1-D
+// bulk async copies (one copy per stage when the group is the whole row), so
+// the loads in flight do not depend on registers; each thread then reads its
+// 16 bytes of every row from shared memory.
 template <typename T, int LV>
-__global__ void __launch_bounds__(256) k_pool(const T* __restrict__ q, const T* __restrict__ k,
-                                              const T* __restrict__ v, T* __restrict__ pq,
-                                              T* __restrict__ pk, T* __restrict__ pv,
-                                              double* __restrict__ sq, PoolArgs a) {
+__global__ void __launch_bounds__(256, 2) k_pool(const T* __restrict__ q, const T* __restrict__ k,
+                                                 const T* __restrict__ v, T* __restrict__ pq,
+                                                 T* __restrict__ pk, T* __restrict__ pv,
+                                                 double* __restrict__ sq, PoolArgs a, int* err) {
+  extern __shared__ __align__(128) uint8_t smem[];
   const Geom& g = a.g;
   const int C8 = g.D >> 3;
   const int tensor = blockIdx.z % 3;
   const int b = blockIdx.z / 3;
-  const int head = blockIdx.y * a.hg + threadIdx.x / C8;
+  const int hg0 = blockIdx.y * a.hg;
+  const int head = hg0 + threadIdx.x / C8;
   const int chunk = threadIdx.x % C8;
-  const int cb = blockIdx.x * a.yb + threadIdx.y;
-  const bool live = head < g.H && cb < a.ncoarse;   // whole head groups share liveness
+  const int cb = blockIdx.x;
   const T* x = tensor == 0 ? q : (tensor == 1 ? k : v);
   T* pyr = tensor == 0 ? pq : (tensor == 1 ? pk : pv);
   const int p = g.p;
   const long long P = g.pl[LV];
   const size_t tok_stride = (size_t)g.H * g.D;
-  const T* src = x + ((size_t)b * g.N + (size_t)cb * P) * tok_stride + (size_t)head * g.D + chunk * 8;
+  const T* src0 = x + ((size_t)b * g.N + (size_t)cb * P) * tok_stride + (size_t)hg0 * g.D;
   T* dst_head = pyr + ((size_t)b * g.H + head) * (size_t)g.E * g.D + chunk * 8;
   double* sq_head = (tensor < 2) ? sq + ((size_t)tensor * g.B * g.H + (size_t)b * g.H + head) * g.E
                                  : nullptr;
+  // lanes of this warp that exist (a head group narrower than a warp)
+  const int wbase = threadIdx.x & ~31;
+  const unsigned wmask = (wbase + 32 <= (int)blockDim.x) ? 0xffffffffu
+                                                         : ((1u << (blockDim.x - wbase)) - 1u);
 
-  double acc[LV][8];   // acc[l-1]: running sum of the open entry of level l
-  const long long ngroups = P / p;   // level-1 entries in this block
+  const int row_bytes = a.row_bytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + (size_t)a.ns * a.ts * row_bytes);
+  const int nstages = (int)((P + a.ts - 1) / a.ts);
+  const bool contiguous = (a.hg == g.H);
+  if (threadIdx.x == 0) {
+    for (int s2 = 0; s2 < a.ns; ++s2) mbar_init(&full[s2], 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  auto issue = [&](int kk) {
+    const int slot = kk % a.ns;
+    const long long t0 = (long long)kk * a.ts;
+    const int nt = (int)min((long long)a.ts, P - t0);
+    uint8_t* dst = smem + (size_t)slot * a.ts * row_bytes;
+    mbar_expect_tx(&full[slot], (uint32_t)(nt * row_bytes));
+    if (contiguous) {
+      bulk_load(dst, src0 + t0 * tok_stride, (uint32_t)(nt * row_bytes), &full[slot]);
+    } else {
+      for (int u = 0; u < nt; ++u)
+        bulk_load(dst + (size_t)u * row_bytes, src0 + (t0 + u) * tok_stride, (uint32_t)row_bytes,
+                  &full[slot]);
+    }
+  };
+  if (threadIdx.x == 0)
+    for (int kk = 0; kk < a.ns && kk < nstages; ++kk) issue(kk);
 
-  for (long long g1 = 0; g1 < ngroups; ++g1) {
-    // level 1: p tokens, left to right from the first child
-    double s[8];
-    for (int c0 = 0; c0 < p; c0 += 8) {
-      const int nb = min(8, p - c0);
-      typename Vec8<T>::Raw raw[8];
+  double acc[LV][8];                    // acc[l-1]: running sum of the open entry of level l
+  double (&s)[8] = acc[0];
+  long long gi1 = (long long)cb * (P / p);   // index of the open level-1 entry
+  int c = 0;                            // position of the next token in its level-1 entry
+  tc::Abort none{0};
+  for (int kk = 0; kk < nstages; ++kk) {
+    const int slot = kk % a.ns;
+    const bool ok = tc::mbar_wait(&full[slot], (kk / a.ns) & 1, &none, err, 200);
+    if (__syncthreads_or(!ok)) break;   // copies never landed: reported, all threads leave
+    const long long t0 = (long long)kk * a.ts;
+    const int nt = (int)min((long long)a.ts, P - t0);
+    const uint8_t* buf = smem + (size_t)slot * a.ts * row_bytes + (size_t)threadIdx.x * 8 * sizeof(T);
+    for (int u = 0; u < nt; ++u) {
+      typename Vec8<T>::Raw raw = *reinterpret_cast<const typename Vec8<T>::Raw*>(buf + (size_t)u * row_bytes);
+      double xr[8];
+      Vec8<T>::raw_f64(raw, xr);
+      if (c == 0) {
 #pragma unroll
-      for (int u = 0; u < 8; ++u)
-        if (u < nb && live) Vec8<T>::load_raw(src + (size_t)(g1 * p + c0 + u) * tok_stride, raw[u]);
+        for (int d = 0; d < 8; ++d) s[d] = xr[d];
+      } else {
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        if (u < nb) {
-          double xr[8];
-          Vec8<T>::raw_f64(raw[u], xr);
-          if (c0 + u == 0) {
+        for (int d = 0; d < 8; ++d) s[d] = __dadd_rn(s[d], xr[d]);
+      }
+      if (++c < p) continue;
+      c = 0;
+      // level-1 entry gi1 complete: emit it, then carry upward while levels complete
+      long long gi = gi1++;
 #pragma unroll
-            for (int d = 0; d < 8; ++d) s[d] = xr[d];
+      for (int l = 1; l <= LV; ++l) {
+        if (l > 1) {
+          const int pos = (int)(gi % p);   // gi here is the level-(l-1) index
+          if (pos == 0) {
+#pragma unroll
+            for (int d = 0; d < 8; ++d) acc[l - 1][d] = acc[l - 2][d];
           } else {
 #pragma unroll
-            for (int d = 0; d < 8; ++d) s[d] = __dadd_rn(s[d], xr[d]);
+            for (int d = 0; d < 8; ++d) acc[l - 1][d] = __dadd_rn(acc[l - 1][d], acc[l - 2][d]);
           }
+          if (pos != p - 1) break;
+          gi /= p;
         }
-      }
-    }
+        // entry (l, gi) complete
+        double m[8];
+        if (g.pow2) {
+          const double inv = 1.0 / (double)g.pl[l];   // exact: p^l is a power of two
 #pragma unroll
-    for (int d = 0; d < 8; ++d) acc[0][d] = s[d];
-    // emit level 1, then carry the completed sum upward while levels complete
-    long long gi = (long long)cb * (P / p) + g1;   // index of this level-1 entry
-#pragma unroll
-    for (int l = 1; l <= LV; ++l) {
-      if (l > 1) {
-        const int pos = (int)(gi % p);   // gi here is the level-(l-1) index
-        if (pos == 0) {
-#pragma unroll
-          for (int d = 0; d < 8; ++d) acc[l - 1][d] = acc[l - 2][d];
+          for (int d = 0; d < 8; ++d) m[d] = __dmul_rn(acc[l - 1][d], inv);
         } else {
+          const double den = (double)g.pl[l];
 #pragma unroll
-          for (int d = 0; d < 8; ++d) acc[l - 1][d] = __dadd_rn(acc[l - 1][d], acc[l - 2][d]);
+          for (int d = 0; d < 8; ++d) m[d] = __ddiv_rn(acc[l - 1][d], den);
         }
-        if (pos != p - 1) break;
-        gi /= p;
-      }
-      // entry (l, gi) complete
-      double m[8];
-      if (g.pow2) {
-        const double inv = 1.0 / (double)g.pl[l];   // exact: p^l is a power of two
+        const size_t e = (size_t)g.off[l] + gi;
+        Vec8<T>::store_f64(dst_head + e * g.D, m);
+        if (tensor < 2) {
+          double part = __dmul_rn(m[0], m[0]);
 #pragma unroll
-        for (int d = 0; d < 8; ++d) m[d] = __dmul_rn(acc[l - 1][d], inv);
-      } else {
-        const double den = (double)g.pl[l];
-#pragma unroll
-        for (int d = 0; d < 8; ++d) m[d] = __ddiv_rn(acc[l - 1][d], den);
-      }
-      const size_t e = (size_t)g.off[l] + gi;
-      if (live) Vec8<T>::store_f64(dst_head + e * g.D, m);
-      if (tensor < 2) {
-        double part = __dmul_rn(m[0], m[0]);
-#pragma unroll
-        for (int d = 1; d < 8; ++d) part = __dadd_rn(part, __dmul_rn(m[d], m[d]));
-        for (int off = C8 >> 1; off >= 1; off >>= 1)
-          part = __dadd_rn(part, __shfl_xor_sync(0xffffffffu, part, off));
-        if (live && chunk == 0) sq_head[e] = part;
+          for (int d = 1; d < 8; ++d) part = __dadd_rn(part, __dmul_rn(m[d], m[d]));
+          for (int off = C8 >> 1; off >= 1; off >>= 1)
+            part = __dadd_rn(part, __shfl_xor_sync(wmask, part, off));
+          if (chunk == 0) sq_head[e] = part;
+        }
       }
     }
+    __syncthreads();                    // every thread is done with this stage
+    if (threadIdx.x == 0 && kk + a.ns < nstages) issue(kk + a.ns);
   }
 }
 
 template <typename T>
 cudaError_t launch_t(const Geom& g, const void* q, const void* k, const void* v, void* pq,
-                     void* pk, void* pv, double* sq, cudaStream_t s) {
+                     void* pk, void* pv, double* sq, int* err, cudaStream_t s) {
   const int LV = g.L - 1;
   if (LV < 1) return cudaSuccess;
   PoolArgs a;
@@ -139,16 +188,26 @@ cudaError_t launch_t(const Geom& g, const void* q, const void* k, const void* v,
     while (g.H % hg) --hg;
   }
   a.hg = hg;
-  a.ncoarse = g.n[g.L - 1];
-  a.yb = 1;
-  while (a.yb * 2 * hg * C8 <= 256 && a.yb * 2 <= a.ncoarse) a.yb *= 2;
-  dim3 block(hg * C8, a.yb);
-  dim3 grid((a.ncoarse + a.yb - 1) / a.yb, g.H / hg, 3 * g.B);
+  a.row_bytes = hg * g.D * (int)sizeof(T);
+  const long long P = g.pl[LV];
+  int ts = 1;
+  while (ts * 2 * a.row_bytes <= 32768 && ts * 2 <= P) ts *= 2;
+  a.ts = ts;
+  a.ns = 3;
+  const size_t smem = (size_t)a.ns * a.ts * a.row_bytes + a.ns * sizeof(uint64_t);
+  cudaError_t e = cudaFuncSetAttribute(k_pool<T, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  (void)e;
+  dim3 block(hg * C8);
+  dim3 grid(g.n[g.L - 1], g.H / hg, 3 * g.B);
   const T* tq = (const T*)q; const T* tk = (const T*)k; const T* tv = (const T*)v;
   T* tpq = (T*)pq; T* tpk = (T*)pk; T* tpv = (T*)pv;
   switch (LV) {
-#define LH_POOL_CASE(n) \
-    case n: k_pool<T, n><<<grid, block, 0, s>>>(tq, tk, tv, tpq, tpk, tpv, sq, a); break;
+#define LH_POOL_CASE(n)                                                                              \
+    case n:                                                                                          \
+      e = cudaFuncSetAttribute(k_pool<T, n>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem); \
+      if (e != cudaSuccess) return e;                                                                \
+      k_pool<T, n><<<grid, block, smem, s>>>(tq, tk, tv, tpq, tpk, tpv, sq, a, err);                 \
+      break;
     LH_POOL_CASE(1) LH_POOL_CASE(2) LH_POOL_CASE(3) LH_POOL_CASE(4)
     LH_POOL_CASE(5) LH_POOL_CASE(6) LH_POOL_CASE(7)
 #undef LH_POOL_CASE
@@ -161,9 +220,9 @@ cudaError_t launch_t(const Geom& g, const void* q, const void* k, const void* v,
 }  // namespace
 
 cudaError_t launch_pool(const Geom& g, lh_dtype dt, const void* q, const void* k, const void* v,
-                        void* pq, void* pk, void* pv, double* sq, cudaStream_t s) {
-  if (dt == LH_BF16) return launch_t<__nv_bfloat16>(g, q, k, v, pq, pk, pv, sq, s);
-  return launch_t<float>(g, q, k, v, pq, pk, pv, sq, s);
+                        void* pq, void* pk, void* pv, double* sq, int* err, cudaStream_t s) {
+  if (dt == LH_BF16) return launch_t<__nv_bfloat16>(g, q, k, v, pq, pk, pv, sq, err, s);
+  return launch_t<float>(g, q, k, v, pq, pk, pv, sq, err, s);
 }
 
 }  // namespace lh

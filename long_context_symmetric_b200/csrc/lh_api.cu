@@ -171,7 +171,8 @@ lh_status lh_pool(const lh_config* cfg, const void* q, const void* k, const void
   LH_REQ(q); LH_REQ(k); LH_REQ(v);
   if (g.L == 1) return LH_OK;
   LH_REQ(pyr_q); LH_REQ(pyr_k); LH_REQ(pyr_v); LH_REQ(sq);
-  LH_CUDA(launch_pool(g, cfg->dtype, q, k, v, pyr_q, pyr_k, pyr_v, sq, (cudaStream_t)stream));
+  LH_CUDA(launch_pool(g, cfg->dtype, q, k, v, pyr_q, pyr_k, pyr_v, sq, device_error_ptr(),
+                      (cudaStream_t)stream));
   return LH_OK;
 }
 

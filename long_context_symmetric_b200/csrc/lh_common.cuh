@@ -174,7 +174,7 @@ __device__ __forceinline__ int map_index(int e) { return e & 0x0FFFFFFF; }
 // Host-side launchers (defined next to each kernel, called by lh_api.cu).
 namespace lh {
 cudaError_t launch_pool(const Geom& g, lh_dtype dt, const void* q, const void* k, const void* v,
-                        void* pq, void* pk, void* pv, double* sq, cudaStream_t s);
+                        void* pq, void* pk, void* pv, double* sq, int* err, cudaStream_t s);
 cudaError_t launch_select(const Geom& g, const double* sq, int32_t* sel, int32_t* map,
                           int32_t* slot, int32_t* ws, cudaStream_t s);
 cudaError_t launch_gather(const Geom& g, lh_dtype dt, const void* q, const void* k, const void* v,
