@@ -62,7 +62,7 @@ struct BwdLayout {
 };
 
 struct BwdBars {
-  uint64_t fix_full, ring_full[kStages], ring_empty[kStages], s_ready, ds_ready, acc_done, done, drain;
+  uint64_t fix_full, ring_full[kStages], ring_empty[kStages], s_ready[2], ds_ready[2], done, drain;
   uint32_t tmem_base;
   Abort abort;
 };
@@ -75,9 +75,10 @@ __device__ __forceinline__ void bwd_setup(BwdBars* bars, int warp) {
       mbar_init(&bars->ring_full[s], 1);
       mbar_init(&bars->ring_empty[s], 1);
     }
-    mbar_init(&bars->s_ready, 1);
-    mbar_init(&bars->ds_ready, kComputeThreads);
-    mbar_init(&bars->acc_done, 1);
+    for (int h = 0; h < 2; ++h) {
+      mbar_init(&bars->s_ready[h], 1);
+      mbar_init(&bars->ds_ready[h], kComputeThreads / 2);
+    }
     mbar_init(&bars->done, 1);
     mbar_init(&bars->drain, 1);
     bars->abort.flag = 0;
@@ -136,72 +137,76 @@ __device__ void bwd_produce(uint8_t* sm, BwdBars* bars, const CUtensorMap* f0, c
   }
 }
 
-// MMA issuer shared by both kernels. Per streamed tile t:
-//   X  = F0 * A_t^T  (TMEM cols 0..127),  Y = F1 * B_t^T (TMEM cols 128..255)
-// then, once the compute warps have turned X/Y into fp16 operands in place,
-//   dkdv (TWO_ACC): acc0 += Xh * B_t (dV += P^T dO),  acc1 += Yh * A_t (dK += dS^T Q)
-//   dq:             acc1 += Xh * A_t + Yh * A_t       (dQ += (dS_hi + dS_lo) K)
+// MMA issuer shared by both kernels, pipelined by half tiles. For streamed
+// tile t and half h (its rows 64h..64h+63):
+//   X_h = F0 * A_t[h]^T (TMEM cols 64h..64h+63), Y_h = F1 * B_t[h]^T (cols 128+64h..)
+// and, once compute warpgroup h has turned X_h/Y_h into fp16 operands in place,
+//   dkdv (TWO_ACC): acc0 += Xh * B_t[h] (dV += P^T dO),  acc1 += Yh * A_t[h] (dK += dS^T Q)
+//   dq:             acc1 += Xh * A_t[h] + Yh * A_t[h]   (dQ += (dS_hi + dS_lo) K)
+// Issue order: acc(t-1, 0), X/Y_0(t), acc(t-1, 1), X/Y_1(t), ... so the tensor
+// core works on one half while the other half's warps compute. acc(t-1, h)
+// reads the fp16 values that X/Y_h(t) then overwrite; MMAs issued by one thread
+// execute in issue order, which makes that safe without a wait.
 template <int D, bool TWO_ACC>
 __device__ void bwd_mma(uint8_t* sm, BwdBars* bars, uint32_t tbase, int n, volatile Abort* ab, int* err) {
   using Lay = BwdLayout<D>;
   constexpr int SUB = Lay::SUB;
-  constexpr uint32_t IDX = idesc_f16(kT, kT, false);
+  constexpr uint32_t IDX = idesc_f16(kT, 64, false);
   constexpr uint32_t IDACC = idesc_f16(kT, D, true);
   const uint32_t sbase = smem_u32(sm);
   const uint32_t tX = tbase, tY = tbase + 128;
   const uint32_t tAcc0 = tbase + 256, tAcc1 = tbase + 256 + (TWO_ACC ? D : 0);
-  auto accumulate = [&](int tt) -> bool {
-    if (!mbar_wait(&bars->ds_ready, tt & 1, ab, err, 14)) return false;
+  auto issue_xy = [&](int t, int h) {
+    const uint32_t ring = sbase + Lay::RING + (t % kStages) * Lay::STAGE;
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+      const uint32_t koff = (kk >> 2) * kSub + (kk & 3) * 32;
+      umma_f16(tX + 64 * h, sdesc_sw128(sbase + Lay::FIX0 + koff, 16, 1024),
+               sdesc_sw128(ring + koff + 8192 * h, 16, 1024), IDX, kk > 0 ? 1u : 0u);
+    }
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+      const uint32_t koff = (kk >> 2) * kSub + (kk & 3) * 32;
+      umma_f16(tY + 64 * h, sdesc_sw128(sbase + Lay::FIX1 + koff, 16, 1024),
+               sdesc_sw128(ring + SUB * kSub + koff + 8192 * h, 16, 1024), IDX, kk > 0 ? 1u : 0u);
+    }
+    umma_commit(&bars->s_ready[h]);
+  };
+  auto accumulate = [&](int tt, int h) -> bool {
+    if (!mbar_wait(&bars->ds_ready[h], tt & 1, ab, err, 14)) return false;
     tc_fence_after();
     const int st = tt % kStages;
     const uint32_t ring = sbase + Lay::RING + st * Lay::STAGE;
     const uint32_t tileA = ring, tileB = ring + SUB * kSub;
 #pragma unroll
-    for (int kk = 0; kk < kT / 16; ++kk) {
-      // packed operand columns: k-steps 0-3 at 8kk, 4-7 at 8kk + 32 (each half
-      // of the tile packs into its own 64 columns)
-      const uint32_t acol = 8 * kk + (kk >= 4 ? 32 : 0);
-      const uint64_t g = sdesc_sw128(tileA + kk * 2048, kSub, 1024);
+    for (int kk = 0; kk < 4; ++kk) {
+      const uint32_t acol = 64 * h + 8 * kk;        // half h's packed operand columns
+      const uint32_t roff = (4 * h + kk) * 2048;     // its 16 rows of the streamed tiles
+      const uint32_t first = (tt == 0 && h == 0 && kk == 0) ? 0u : 1u;
+      const uint64_t g = sdesc_sw128(tileA + roff, kSub, 1024);
       if (TWO_ACC) {
-        const uint64_t b = sdesc_sw128(tileB + kk * 2048, kSub, 1024);
-        umma_f16_ts(tAcc0, tX + acol, b, IDACC, (tt > 0 || kk > 0) ? 1u : 0u);
+        const uint64_t b = sdesc_sw128(tileB + roff, kSub, 1024);
+        umma_f16_ts(tAcc0, tX + acol, b, IDACC, first);
+        umma_f16_ts(tAcc1, tY + acol, g, IDACC, first);
       } else {
-        umma_f16_ts(tAcc1, tX + acol, g, IDACC, (tt > 0 || kk > 0) ? 1u : 0u);
+        umma_f16_ts(tAcc1, tX + acol, g, IDACC, first);
+        umma_f16_ts(tAcc1, tY + acol, g, IDACC, 1u);
       }
-      umma_f16_ts(tAcc1, tY + acol, g, IDACC, (TWO_ACC && tt == 0 && kk == 0) ? 0u : 1u);
     }
-    umma_commit(&bars->ring_empty[st]);
+    if (h == 1) umma_commit(&bars->ring_empty[st]);
     return true;
   };
   bool ok = mbar_wait(&bars->fix_full, 0, ab, err, 12);
   for (int t = 0; ok && t < n; ++t) {
     const int st = t % kStages;
     if (!mbar_wait(&bars->ring_full[st], (t / kStages) & 1, ab, err, 13)) { ok = false; break; }
-    // accumulate tile t-1 first and let it finish: its A operands are the bf16
-    // values in X/Y, which the MMAs of tile t overwrite (MMAs into different
-    // accumulators are not ordered among themselves)
-    if (t >= 1) {
-      if (!accumulate(t - 1)) { ok = false; break; }
-      umma_commit(&bars->acc_done);
-      if (!mbar_wait(&bars->acc_done, (t - 1) & 1, ab, err, 19)) { ok = false; break; }
+    for (int h = 0; h < 2; ++h) {
+      if (t >= 1 && !accumulate(t - 1, h)) { ok = false; break; }
+      tc_fence_after();
+      issue_xy(t, h);
     }
-    tc_fence_after();
-    const uint32_t ring = sbase + Lay::RING + st * Lay::STAGE;
-#pragma unroll
-    for (int kk = 0; kk < D / 16; ++kk) {
-      const uint32_t koff = (kk >> 2) * kSub + (kk & 3) * 32;
-      umma_f16(tX, sdesc_sw128(sbase + Lay::FIX0 + koff, 16, 1024), sdesc_sw128(ring + koff, 16, 1024),
-                IDX, kk > 0 ? 1u : 0u);
-    }
-#pragma unroll
-    for (int kk = 0; kk < D / 16; ++kk) {
-      const uint32_t koff = (kk >> 2) * kSub + (kk & 3) * 32;
-      umma_f16(tY, sdesc_sw128(sbase + Lay::FIX1 + koff, 16, 1024),
-                sdesc_sw128(ring + SUB * kSub + koff, 16, 1024), IDX, kk > 0 ? 1u : 0u);
-    }
-    umma_commit(&bars->s_ready);
   }
-  if (ok && accumulate(n - 1)) umma_commit(&bars->done);
+  if (ok && accumulate(n - 1, 0) && accumulate(n - 1, 1)) umma_commit(&bars->done);
   umma_commit(&bars->drain);
   Abort none{0};
   mbar_wait(&bars->drain, 0, &none, nullptr, 0);
@@ -245,15 +250,17 @@ k_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CU
     // after a wind-down, so no warp can be left waiting at the barrier
     for (int t = 0; t < n; ++t) {
       const int i = j + t;
-      float* lse2 = vec + (t & 1) * 256;
+      // this half's 64 query columns: lse (log2 units) and delta, double-buffered
+      float* lse2 = vec + (t & 1) * 256 + 64 * half;
       float* dl = lse2 + 128;
       {
-        const int q = i * kT + (ctid & 127);
-        if (ctid < 128) lse2[ctid] = q < S ? lse[(size_t)bh * S + q] * 1.4426950408889634f : 0.f;
-        else dl[ctid - 128] = q < S ? delta[(size_t)bh * S + q] : 0.f;
+        const int hid = ctid & 127;                 // thread within the half
+        const int q = i * kT + 64 * half + (hid & 63);
+        if (hid < 64) lse2[hid] = q < S ? lse[(size_t)bh * S + q] * 1.4426950408889634f : 0.f;
+        else dl[hid - 64] = q < S ? delta[(size_t)bh * S + q] : 0.f;
       }
-      named_bar_sync(1, kComputeThreads);
-      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bars->s_ready, t & 1, ab, err, 15));
+      named_bar_sync(1 + half, kComputeThreads / 2);
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bars->s_ready[half], t & 1, ab, err, 15));
       if (!ok) continue;
       tc_fence_after();
       const bool diag = (i == j);
@@ -272,9 +279,9 @@ k_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CU
           for (int u = 0; u < 2; ++u) {
             const int col = 32 * c + e + u;
             const bool valid = col <= qlim && (!diag || col >= m);
-            const float p = valid ? ex2(__uint_as_float(s[e + u]) * c2 - lse2[col]) : 0.f;
+            const float p = valid ? ex2(__uint_as_float(s[e + u]) * c2 - lse2[col - 64 * half]) : 0.f;
             pe[u] = p;
-            de[u] = p * (__uint_as_float(dp[e + u]) - dl[col]);
+            de[u] = p * (__uint_as_float(dp[e + u]) - dl[col - 64 * half]);
             dsmax = fmaxf(dsmax, fabsf(de[u]));
           }
           pk[e >> 1] = pack_f16(pe[0], pe[1]);
@@ -287,7 +294,7 @@ k_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CU
       }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&bars->ds_ready);
+      mbar_arrive(&bars->ds_ready[half]);
     }
     if (!(dsmax <= kHalfMax)) report_error(err, LH_ERR_DEVICE, 101);
     if (ok && __all_sync(0xffffffffu, mbar_wait(&bars->done, 0, ab, err, 16))) {
@@ -354,7 +361,7 @@ k_bwd_dq_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
     float dsmax = 0.f;
     bool ok = true;
     for (int jj = 0; jj < n; ++jj) {
-      if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_ready, jj & 1, ab, err, 17))) { ok = false; break; }
+      if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_ready[half], jj & 1, ab, err, 17))) { ok = false; break; }
       tc_fence_after();
       const bool diag = (jj == i);
       const int klim = min(diag ? r : kT - 1, S - 1 - jj * kT);   // last valid key column
@@ -387,7 +394,7 @@ k_bwd_dq_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
       }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&bars->ds_ready);
+      mbar_arrive(&bars->ds_ready[half]);
     }
     if (!(dsmax <= kHalfMax)) report_error(err, LH_ERR_DEVICE, 101);
     if (ok && __all_sync(0xffffffffu, mbar_wait(&bars->done, 0, ab, err, 18))) {
