@@ -206,24 +206,24 @@ k_attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CU
       tmem_wait_ld();
       tc_fence_before();
       mbar_arrive(&bars->s_free[sb]);
-      // scale into the log2 domain, causal mask on the diagonal tile
-      float mx = -INFINITY;
+      // causal mask on the diagonal tile; the running max is taken on the raw
+      // scores (c2 > 0, and rounding is monotone, so max(s) c2 = max(s c2))
       if (j == it) {
         const int lim = min(r, S - 1 - j * kBN);   // last valid column of this row
 #pragma unroll
-        for (int c = 0; c < 128; ++c) {
-          const float x = c <= lim ? __uint_as_float(s[c]) * c2 : -INFINITY;
-          s[c] = __float_as_uint(x);
-          mx = fmaxf(mx, x);
-        }
-      } else {
-#pragma unroll
-        for (int c = 0; c < 128; ++c) {
-          const float x = __uint_as_float(s[c]) * c2;
-          s[c] = __float_as_uint(x);
-          mx = fmaxf(mx, x);
-        }
+        for (int c = 0; c < 128; ++c)
+          if (c > lim) s[c] = __float_as_uint(-INFINITY);
       }
+      float mq[4];
+#pragma unroll
+      for (int g = 0; g < 4; ++g) {
+        mq[g] = __uint_as_float(s[32 * g]);
+#pragma unroll
+        for (int c = 1; c < 31; c += 2)
+          mq[g] = fmax3(mq[g], __uint_as_float(s[32 * g + c]), __uint_as_float(s[32 * g + c + 1]));
+        mq[g] = fmaxf(mq[g], __uint_as_float(s[32 * g + 31]));
+      }
+      const float mx = fmax3(fmaxf(mq[0], mq[1]), mq[2], mq[3]) * c2;
       float m_new = m_run, alpha = 1.f;
       if (j == 0) {
         m_new = mx;
@@ -231,13 +231,19 @@ k_attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CU
         m_new = mx;
         alpha = ex2(m_run - m_new);
       }
-      float sum = 0.f;
+      // P = 2^(s c2 - m), two columns per packed FMA; four partial sums
+      const float2 cc = make_float2(c2, c2), nm = make_float2(-m_new, -m_new);
+      float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
-      for (int c = 0; c < 128; ++c) {
-        const float pc = ex2(__uint_as_float(s[c]) - m_new);
-        sum += pc;
-        s[c] = __float_as_uint(pc);
+      for (int c = 0; c < 128; c += 2) {
+        const float2 x = __ffma2_rn(make_float2(__uint_as_float(s[c]), __uint_as_float(s[c + 1])), cc, nm);
+        const float2 pc = make_float2(ex2(x.x), ex2(x.y));
+        acc[(c >> 1) & 3] = __fadd2_rn(acc[(c >> 1) & 3], pc);
+        s[c] = __float_as_uint(pc.x);
+        s[c + 1] = __float_as_uint(pc.y);
       }
+      const float2 a01 = __fadd2_rn(acc[0], acc[1]), a23 = __fadd2_rn(acc[2], acc[3]);
+      const float sum = (a01.x + a23.x) + (a01.y + a23.y);
       l_run = l_run * alpha + sum;
       m_run = m_new;
       if (j >= 1) {
@@ -263,11 +269,12 @@ k_attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CU
         uint32_t hi[16], lo[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
-          const float p0 = __uint_as_float(s[32 * c + 2 * e]);
-          const float p1 = __uint_as_float(s[32 * c + 2 * e + 1]);
-          hi[e] = pack_f16(p0, p1);
-          const float2 h = __half22float2(*reinterpret_cast<const __half2*>(&hi[e]));
-          lo[e] = pack_f16(p0 - h.x, p1 - h.y);
+          const float2 pp = make_float2(__uint_as_float(s[32 * c + 2 * e]), __uint_as_float(s[32 * c + 2 * e + 1]));
+          const __half2 h = __float22half2_rn(pp);
+          const float2 rem = __ffma2_rn(__half22float2(h), make_float2(-1.f, -1.f), pp);   // p - hi, exact
+          const __half2 l = __float22half2_rn(rem);
+          hi[e] = *reinterpret_cast<const uint32_t*>(&h);
+          lo[e] = *reinterpret_cast<const uint32_t*>(&l);
         }
 #pragma unroll
         for (int q4 = 0; q4 < 4; ++q4) {

@@ -22,7 +22,8 @@
 //      S = Q_i K_j^T and dP = dO_i V_j^T into TMEM; dS split into an fp16 head
 //      and an fp16 remainder (dS = hi + lo to about 2^-22 relative) back into
 //      TMEM; dQ += hi K_j + lo K_j.
-// A dS beyond the fp16 range is reported as LH_ERR_DEVICE, detail 101.
+// A dS whose fp16 rounding overflows (or is NaN) is reported as LH_ERR_DEVICE,
+// detail 101.
 // Q_i/dO_i (dkdv) or K_j/V_j (dq) stream through a 2-stage TMA ring; the
 // operands that stay fixed for the CTA are loaded once. Same warp roles and
 // bounded waits as the forward kernel.
@@ -212,6 +213,69 @@ __device__ void bwd_mma(uint8_t* sm, BwdBars* bars, uint32_t tbase, int n, volat
   mbar_wait(&bars->drain, 0, &none, nullptr, 0);
 }
 
+__device__ __forceinline__ float2 f2(uint32_t a, uint32_t b) {
+  return make_float2(__uint_as_float(a), __uint_as_float(b));
+}
+__device__ __forceinline__ uint32_t h2_bits(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
+
+// One 32-column chunk of this thread's key row of S^T and dP^T (dK/dV kernel):
+// P^T = 2^(S^T c2 - lse2) and dS^T = P^T o (dP^T - delta) as fp16 pairs, two
+// columns per packed fp32 instruction. nl2/ndl hold -lse2 and -delta of the
+// chunk's 32 query columns (the same for every lane: broadcast reads). MASK:
+// columns outside [vlo, vhi] (causal diagonal, rows past S) get P = 0.
+template <bool MASK>
+__device__ __forceinline__ void dkdv_chunk(const uint32_t (&s)[32], const uint32_t (&dp)[32],
+                                           const float* nl2, const float* ndl, float c2, int col0, int vlo,
+                                           int vhi, uint32_t (&pk)[16], uint32_t (&dk)[16], __half2& hm) {
+  const float2 cc = make_float2(c2, c2);
+#pragma unroll
+  for (int e = 0; e < 32; e += 4) {
+    const float4 a = *reinterpret_cast<const float4*>(nl2 + e);
+    const float4 b = *reinterpret_cast<const float4*>(ndl + e);
+#pragma unroll
+    for (int u = 0; u < 4; u += 2) {
+      const float2 x = __ffma2_rn(f2(s[e + u], s[e + u + 1]), cc, u ? make_float2(a.z, a.w) : make_float2(a.x, a.y));
+      float p0 = ex2(x.x), p1 = ex2(x.y);
+      if (MASK) {
+        const int col = col0 + e + u;
+        if (col < vlo || col > vhi) p0 = 0.f;
+        if (col + 1 < vlo || col + 1 > vhi) p1 = 0.f;
+      }
+      const float2 d = __fadd2_rn(f2(dp[e + u], dp[e + u + 1]), u ? make_float2(b.z, b.w) : make_float2(b.x, b.y));
+      const __half2 ds = __float22half2_rn(__fmul2_rn(make_float2(p0, p1), d));
+      hm = __hmax2_nan(hm, __habs2(ds));
+      pk[(e + u) >> 1] = pack_f16(p0, p1);
+      dk[(e + u) >> 1] = h2_bits(ds);
+    }
+  }
+}
+
+// One 32-column chunk of this thread's query row of S and dP (dQ kernel): dS as
+// an fp16 head and an fp16 remainder (hi + lo = dS to about 2^-22 relative).
+// nl2 = -lse2, ndl = -delta of the row. MASK: key columns past vhi get P = 0.
+template <bool MASK>
+__device__ __forceinline__ void dq_chunk(const uint32_t (&s)[32], const uint32_t (&dp)[32], float nl2, float ndl,
+                                         float c2, int col0, int vhi, uint32_t (&hi)[16], uint32_t (&lo)[16],
+                                         __half2& hm) {
+  const float2 cc = make_float2(c2, c2), nl = make_float2(nl2, nl2), nd = make_float2(ndl, ndl);
+  const float2 m1 = make_float2(-1.f, -1.f);
+#pragma unroll
+  for (int e = 0; e < 32; e += 2) {
+    const float2 x = __ffma2_rn(f2(s[e], s[e + 1]), cc, nl);
+    float p0 = ex2(x.x), p1 = ex2(x.y);
+    if (MASK) {
+      if (col0 + e > vhi) p0 = 0.f;
+      if (col0 + e + 1 > vhi) p1 = 0.f;
+    }
+    const float2 ds = __fmul2_rn(make_float2(p0, p1), __fadd2_rn(f2(dp[e], dp[e + 1]), nd));
+    const __half2 h = __float22half2_rn(ds);
+    hm = __hmax2_nan(hm, __habs2(h));
+    const float2 r = __ffma2_rn(__half22float2(h), m1, ds);     // ds - hi, exact
+    hi[e >> 1] = h2_bits(h);
+    lo[e >> 1] = h2_bits(__float22half2_rn(r));
+  }
+}
+
 // ---------------------------------------------------------------- dK, dV
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -243,59 +307,62 @@ k_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CU
     const int ctid = threadIdx.x - 64;                  // 0..255
     const uint32_t la = (uint32_t)(quarter * 32) << 16;
     const int key = j * kT + m;
-    float* vec = reinterpret_cast<float*>(sm + Lay::VEC);   // [2][2][128]: lse2, delta
-    float dsmax = 0.f;
+    float* vec = reinterpret_cast<float*>(sm + Lay::VEC);   // [2][2][128]: -lse2, -delta
+    // this thread's share of a query tile's -lse2 / -delta (thread hid of the
+    // half: column 64*half + (hid & 63)), fetched one tile ahead
+    const int hid = ctid & 127;
+    const float* vsrc = (hid < 64 ? lse : delta) + (size_t)bh * S;
+    const float vmul = hid < 64 ? -1.4426950408889634f : -1.f;
+    auto fetch = [&](int i) -> float {
+      const int q = i * kT + 64 * half + (hid & 63);
+      return q < S ? vsrc[q] : 0.f;
+    };
+    float nxt = fetch(j);
+    __half2 hm = __float2half2_rn(0.f);
     bool ok = true;
     // every compute thread runs all n iterations (and their named barrier), also
     // after a wind-down, so no warp can be left waiting at the barrier
     for (int t = 0; t < n; ++t) {
       const int i = j + t;
-      // this half's 64 query columns: lse (log2 units) and delta, double-buffered
-      float* lse2 = vec + (t & 1) * 256 + 64 * half;
-      float* dl = lse2 + 128;
-      {
-        const int hid = ctid & 127;                 // thread within the half
-        const int q = i * kT + 64 * half + (hid & 63);
-        if (hid < 64) lse2[hid] = q < S ? lse[(size_t)bh * S + q] * 1.4426950408889634f : 0.f;
-        else dl[hid - 64] = q < S ? delta[(size_t)bh * S + q] : 0.f;
-      }
+      // this half's 64 query columns, double-buffered by tile parity
+      float* nl2 = vec + (t & 1) * 256 + 64 * half;
+      float* ndl = nl2 + 128;
+      (hid < 64 ? nl2 : ndl)[hid & 63] = nxt * vmul;
       named_bar_sync(1 + half, kComputeThreads / 2);
+      if (t + 1 < n) nxt = fetch(i + 1);
       if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bars->s_ready[half], t & 1, ab, err, 15));
       if (!ok) continue;
       tc_fence_after();
-      const bool diag = (i == j);
-      const int qlim = S - 1 - i * kT;                  // last valid query column
-#pragma unroll 1
-      for (int c = 2 * half; c < 2 * half + 2; ++c) {
-        uint32_t s[32], dp[32];
-        tmem_ld32(tbase + la + 32 * c, s);
-        tmem_ld32(tbase + la + 128 + 32 * c, dp);
-        tmem_wait_ld();
-        uint32_t pk[16], dk[16];
-#pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          float pe[2], de[2];
-#pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const int col = 32 * c + e + u;
-            const bool valid = col <= qlim && (!diag || col >= m);
-            const float p = valid ? ex2(__uint_as_float(s[e + u]) * c2 - lse2[col - 64 * half]) : 0.f;
-            pe[u] = p;
-            de[u] = p * (__uint_as_float(dp[e + u]) - dl[col - 64 * half]);
-            dsmax = fmaxf(dsmax, fabsf(de[u]));
-          }
-          pk[e >> 1] = pack_f16(pe[0], pe[1]);
-          dk[e >> 1] = pack_f16(de[0], de[1]);
-        }
-        // fp16 results go to columns this warp has already read: chunk c's 16
-        // packed columns at 16c + 32*half (each half packs inside its own 64)
-        tmem_st16(tbase + la + 16 * c + 32 * half, pk);
-        tmem_st16(tbase + la + 128 + 16 * c + 32 * half, dk);
-      }
+      const int vlo = i == j ? m : 0;                   // causal: query col >= key row
+      const int vhi = min(kT - 1, S - 1 - i * kT);      // last valid query column
+      const bool mask = vlo > 0 || vhi < kT - 1 || i == j;
+      // chunk c0 = 2*half, then c0 + 1; the second chunk's loads overlap the
+      // first chunk's arithmetic
+      const int c0 = 2 * half;
+      uint32_t s0[32], d0[32], s1[32], d1[32], pk[16], dk[16];
+      tmem_ld32(tbase + la + 32 * c0, s0);
+      tmem_ld32(tbase + la + 128 + 32 * c0, d0);
+      tmem_wait_ld_regs(s0);
+      reg_fence32(d0);
+      tmem_ld32(tbase + la + 32 * c0 + 32, s1);
+      tmem_ld32(tbase + la + 160 + 32 * c0, d1);
+      if (mask) dkdv_chunk<true>(s0, d0, nl2, ndl, c2, 32 * c0, vlo, vhi, pk, dk, hm);
+      else dkdv_chunk<false>(s0, d0, nl2, ndl, c2, 32 * c0, vlo, vhi, pk, dk, hm);
+      // fp16 results go to columns this warp has already read: chunk c's 16
+      // packed columns at 16c + 32*half (each half packs inside its own 64)
+      tmem_st16(tbase + la + 16 * c0 + 32 * half, pk);
+      tmem_st16(tbase + la + 128 + 16 * c0 + 32 * half, dk);
+      tmem_wait_ld_regs(s1);
+      reg_fence32(d1);
+      if (mask) dkdv_chunk<true>(s1, d1, nl2 + 32, ndl + 32, c2, 32 * c0 + 32, vlo, vhi, pk, dk, hm);
+      else dkdv_chunk<false>(s1, d1, nl2 + 32, ndl + 32, c2, 32 * c0 + 32, vlo, vhi, pk, dk, hm);
+      tmem_st16(tbase + la + 16 * c0 + 16 + 32 * half, pk);
+      tmem_st16(tbase + la + 128 + 16 * c0 + 16 + 32 * half, dk);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&bars->ds_ready[half]);
     }
+    const float dsmax = __half2float(__hmax_nan(__low2half(hm), __high2half(hm)));
     if (!(dsmax <= kHalfMax)) report_error(err, LH_ERR_DEVICE, 101);
     if (ok && __all_sync(0xffffffffu, mbar_wait(&bars->done, 0, ab, err, 16))) {
       tc_fence_after();
@@ -356,46 +423,41 @@ k_bwd_dq_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
     const int r = quarter * 32 + lane;            // query row within the tile / TMEM lane
     const uint32_t la = (uint32_t)(quarter * 32) << 16;
     const int q = i * kT + r;
-    const float lse2 = q < S ? lse[(size_t)bh * S + q] * 1.4426950408889634f : 0.f;
-    const float dl = q < S ? delta[(size_t)bh * S + q] : 0.f;
-    float dsmax = 0.f;
+    const float nl2 = q < S ? lse[(size_t)bh * S + q] * -1.4426950408889634f : 0.f;
+    const float ndl = q < S ? -delta[(size_t)bh * S + q] : 0.f;
+    __half2 hm = __float2half2_rn(0.f);
     bool ok = true;
     for (int jj = 0; jj < n; ++jj) {
       if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_ready[half], jj & 1, ab, err, 17))) { ok = false; break; }
       tc_fence_after();
-      const bool diag = (jj == i);
-      const int klim = min(diag ? r : kT - 1, S - 1 - jj * kT);   // last valid key column
-#pragma unroll 1
-      for (int c = 2 * half; c < 2 * half + 2; ++c) {
-        uint32_t s[32], dp[32];
-        tmem_ld32(tbase + la + 32 * c, s);
-        tmem_ld32(tbase + la + 128 + 32 * c, dp);
-        tmem_wait_ld();
-        uint32_t hi[16], lo[16];
-#pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          float h[2], rl[2];
-#pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const int col = 32 * c + e + u;
-            const float p = col <= klim ? ex2(__uint_as_float(s[e + u]) * c2 - lse2) : 0.f;
-            const float ds = p * (__uint_as_float(dp[e + u]) - dl);
-            dsmax = fmaxf(dsmax, fabsf(ds));
-            h[u] = __half2float(__float2half_rn(ds));
-            rl[u] = ds - h[u];
-          }
-          hi[e >> 1] = pack_f16(h[0], h[1]);
-          lo[e >> 1] = pack_f16(rl[0], rl[1]);
-        }
-        // head into the (consumed) S columns, remainder into the (consumed) dP
-        // columns, packed inside this half's own 64 columns
-        tmem_st16(tbase + la + 16 * c + 32 * half, hi);
-        tmem_st16(tbase + la + 128 + 16 * c + 32 * half, lo);
-      }
+      const int klim = min(jj == i ? r : kT - 1, S - 1 - jj * kT);   // last valid key column
+      const bool mask = klim < kT - 1;
+      // chunk c0 = 2*half, then c0 + 1 (its loads overlap chunk c0's arithmetic);
+      // head into the (consumed) S columns, remainder into the (consumed) dP
+      // columns, packed inside this half's own 64 columns
+      const int c0 = 2 * half;
+      uint32_t s0[32], d0[32], s1[32], d1[32], hi[16], lo[16];
+      tmem_ld32(tbase + la + 32 * c0, s0);
+      tmem_ld32(tbase + la + 128 + 32 * c0, d0);
+      tmem_wait_ld_regs(s0);
+      reg_fence32(d0);
+      tmem_ld32(tbase + la + 32 * c0 + 32, s1);
+      tmem_ld32(tbase + la + 160 + 32 * c0, d1);
+      if (mask) dq_chunk<true>(s0, d0, nl2, ndl, c2, 32 * c0, klim, hi, lo, hm);
+      else dq_chunk<false>(s0, d0, nl2, ndl, c2, 32 * c0, klim, hi, lo, hm);
+      tmem_st16(tbase + la + 16 * c0 + 32 * half, hi);
+      tmem_st16(tbase + la + 128 + 16 * c0 + 32 * half, lo);
+      tmem_wait_ld_regs(s1);
+      reg_fence32(d1);
+      if (mask) dq_chunk<true>(s1, d1, nl2, ndl, c2, 32 * c0 + 32, klim, hi, lo, hm);
+      else dq_chunk<false>(s1, d1, nl2, ndl, c2, 32 * c0 + 32, klim, hi, lo, hm);
+      tmem_st16(tbase + la + 16 * c0 + 16 + 32 * half, hi);
+      tmem_st16(tbase + la + 128 + 16 * c0 + 16 + 32 * half, lo);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&bars->ds_ready[half]);
     }
+    const float dsmax = __half2float(__hmax_nan(__low2half(hm), __high2half(hm)));
     if (!(dsmax <= kHalfMax)) report_error(err, LH_ERR_DEVICE, 101);
     if (ok && __all_sync(0xffffffffu, mbar_wait(&bars->done, 0, ab, err, 18))) {
       tc_fence_after();
