@@ -94,9 +94,9 @@ k_attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CU
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bars->s_full[s], 1);
-      mbar_init(&bars->s_free[s], 128);
+      mbar_init(&bars->s_free[s], 4);      // one arrival per softmax warp
     }
-    mbar_init(&bars->p_full, 128);
+    mbar_init(&bars->p_full, 4);
     mbar_init(&bars->o_done, 1);
     mbar_init(&bars->drain, 1);
     bars->abort.flag = 0;
@@ -205,7 +205,7 @@ k_attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CU
       }
       tmem_wait_ld();
       tc_fence_before();
-      mbar_arrive(&bars->s_free[sb]);
+      mbar_arrive_warp(&bars->s_free[sb]);
       // causal mask on the diagonal tile; the running max is taken on the raw
       // scores (c2 > 0, and rounding is monotone, so max(s) c2 = max(s c2))
       if (j == it) {
@@ -287,7 +287,7 @@ k_attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CU
       tmem_wait_st();
       fence_proxy_async_smem();
       tc_fence_before();
-      mbar_arrive(&bars->p_full);
+      mbar_arrive_warp(&bars->p_full);
     }
     if (ok && __all_sync(0xffffffffu, mbar_wait(&bars->o_done, (nkv - 1) & 1, ab, err, 8))) {
       tc_fence_after();
@@ -333,13 +333,13 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 }  // namespace
 
 // [BH][S][D] 16-bit elements (bf16, or fp16 when `fp16`) viewed as a 3-D tensor
-// (D, S, BH); boxes of 64 columns x 128 rows, 128-byte swizzle.
-bool make_tmap_16(CUtensorMap* m, const void* base, int D, int S, int BH, bool fp16) {
+// (D, S, BH); boxes of 64 columns x `box_rows` rows, 128-byte swizzle.
+bool make_tmap_16(CUtensorMap* m, const void* base, int D, int S, int BH, bool fp16, int box_rows) {
   auto fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)S, (cuuint64_t)BH};
   cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)S * D * 2};
-  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
   cuuint32_t es[3] = {1, 1, 1};
   return fn(m, fp16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -351,8 +351,8 @@ static cudaError_t fwd_tc_t(const Geom& g, const void* qs, const void* ks, const
                             float* lse, int* err, cudaStream_t s) {
   CUtensorMap tq, tk, tv;
   const int BH = g.B * g.H;
-  if (!make_tmap_16(&tq, qs, D, g.S, BH, true) || !make_tmap_16(&tk, ks, D, g.S, BH, true) ||
-      !make_tmap_16(&tv, vs, D, g.S, BH, true))
+  if (!make_tmap_16(&tq, qs, D, g.S, BH, true, kBM) || !make_tmap_16(&tk, ks, D, g.S, BH, true, kBN) ||
+      !make_tmap_16(&tv, vs, D, g.S, BH, true, kBN))
     return cudaErrorInvalidValue;
   const int smem = FwdLayout<D>::BYTES;
   cudaError_t e = cudaFuncSetAttribute(k_attn_fwd_tc<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);

@@ -14,72 +14,94 @@
 // bf16 sub-sequence. Two kernels, each one CTA per 128-row tile, heavy tiles
 // first:
 //  k_bwd_dkdv_tc  per key tile j, over query tiles i >= j:
-//      S^T = K_j Q_i^T and dP^T = V_j dO_i^T into TMEM; the compute warps (two
-//      per TMEM lane quarter, each on half of the columns) form P^T and dS^T
-//      and store them as fp16 back into the same TMEM columns; then
-//      dV += P^T dO_i and dK += dS^T Q_i take their A operand from TMEM.
-//  k_bwd_dq_tc    per query tile i, over key tiles j <= i:
-//      S = Q_i K_j^T and dP = dO_i V_j^T into TMEM; dS split into an fp16 head
-//      and an fp16 remainder (dS = hi + lo to about 2^-22 relative) back into
-//      TMEM; dQ += hi K_j + lo K_j.
+//      X = S^T = K_j Q_i^T and Y = dP^T = V_j dO_i^T (TMEM); the compute warps
+//      form P^T and dS^T and store them as fp16 into Y's columns; then
+//      dK += dS^T Q_i and dV += P^T dO_i take their A operand from TMEM.
+//  k_bwd_dq_tc    per query tile i, over key tiles j <= i (Q_i and dO_i are
+//      held in TMEM as the A operand of X and Y):
+//      X = S = Q_i K_j^T and Y = dP = dO_i V_j^T; dS is split into an fp16 head
+//      and an fp16 remainder (dS = hi + lo to about 2^-22 relative) stored into
+//      Y's columns; dQ += hi K_j + lo K_j.
 // A dS whose fp16 rounding overflows (or is NaN) is reported as LH_ERR_DEVICE,
 // detail 101.
-// Q_i/dO_i (dkdv) or K_j/V_j (dq) stream through a 2-stage TMA ring; the
-// operands that stay fixed for the CTA are loaded once. Same warp roles and
-// bounded waits as the forward kernel.
+//
+// Pipeline (tensor core order per streamed tile t):  X(t+1), acc(t), Y(t+1).
+// The compute warps copy X(t) into registers and release it at once, so X(t+1)
+// runs while they exponentiate; they read Y(t) and write the fp16 operands of
+// acc(t) into Y's columns, so Y(t+1) follows acc(t) (tcgen05.mma ops issued by
+// one thread execute in order, which orders those reuses). All score MMAs are
+// full 128 x 128 tiles: N = 64 halves run at about two thirds of the rate and
+// lose more when the compute warps use TMEM at the same time (measured).
+// Streamed tiles come through a TMA ring whose two operands have their own
+// full/empty barriers, so each is refilled as soon as its last reader is done.
+// Bounded waits as in the forward kernel.
 #include "tc_ptx.cuh"
 
 namespace lh {
 
-bool make_tmap_16(CUtensorMap* m, const void* base, int D, int S, int BH, bool fp16);
+bool make_tmap_16(CUtensorMap* m, const void* base, int D, int S, int BH, bool fp16, int box_rows);
 
 namespace {
 
 using namespace tc;
 
 constexpr int kT = 128;              // rows per tile (both directions)
-constexpr int kSub = 128 * 64 * 2;   // 128 x 64 bf16 swizzle tile
-constexpr int kStages = 2;
+constexpr int kSub = 128 * 64 * 2;   // 128 x 64 16-bit swizzle tile
+constexpr int kMaxStages = 3;
+// TMEM columns: X at 0, Y at 128, accumulators from 256 (dkdv: dV, then dK;
+// dq: dQ), and in the dQ kernel the fixed Q_i / dO_i (D/2 packed columns each)
+constexpr uint32_t kColY = 128, kColAcc = 256, kFixCol = 384;
 // Warp roles: 0 producer, 1 MMA issuer, 2..9 compute. Two compute warps share
-// each TMEM lane quarter (warps w and w+4), each taking half of a tile's 128
+// each TMEM lane quarter (warps w and w+4), each taking 64 of a tile's 128
 // columns, so every SM sub-partition has two compute warps to interleave.
-constexpr int kComputeThreads = 256;
+constexpr int kComputeWarps = 8;
+constexpr int kComputeThreads = 32 * kComputeWarps;
 constexpr int kThreads = 64 + kComputeThreads;
 
 __device__ __forceinline__ void named_bar_sync(int id, int n) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
 }
 
-template <int D>
+// FIXT: the fixed operands live in TMEM (dQ kernel), which leaves room for a
+// third ring stage; otherwise (dK/dV kernel, whose TMEM holds two accumulators)
+// they are shared-memory tiles.
+template <int D, bool FIXT>
 struct BwdLayout {
   static constexpr int SUB = D / 64;
-  static constexpr int FIX0 = 0;                               // fixed operand 0 (K_j or Q_i)
-  static constexpr int FIX1 = FIX0 + SUB * kSub;               // fixed operand 1 (V_j or dO_i)
-  static constexpr int RING = FIX1 + SUB * kSub;               // stages of (A, B) streamed tiles
+  static constexpr int NST = FIXT ? 3 : 2;                     // ring stages
+  static constexpr int FIX0 = 0;                               // fixed operand 0 (K_j)
+  static constexpr int FIX1 = FIX0 + (FIXT ? 0 : SUB * kSub);  // fixed operand 1 (V_j)
+  static constexpr int RING = FIX1 + (FIXT ? 0 : SUB * kSub);  // stages of streamed tiles (A_t, B_t)
   static constexpr int STAGE = 2 * SUB * kSub;
-  static constexpr int VEC = RING + kStages * STAGE;           // lse / delta per query (dkdv)
-  static constexpr int BAR = VEC + 2 * 2 * kT * 4;
+  static constexpr int VEC = RING + NST * STAGE;               // lse / delta per query (dkdv)
+  static constexpr int BAR = VEC + (FIXT ? 0 : 2 * 2 * kT * 4);
   static constexpr int BYTES = (BAR + 256 + 1024) > 120 * 1024 ? (BAR + 256 + 1024) : 120 * 1024;
 };
 
+// ring_full/ring_empty[stage][o]: o = 0 the streamed operand A_t (Q_i in dkdv,
+// K_j in dq), o = 1 the operand B_t (dO_i in dkdv, V_j in dq).
 struct BwdBars {
-  uint64_t fix_full, ring_full[kStages], ring_empty[kStages], s_ready[2], ds_ready[2], done, drain;
+  uint64_t fix_full, ring_full[kMaxStages][2], ring_empty[kMaxStages][2];
+  uint64_t x_full, y_full, x_free, ds_ready, done, drain;
   uint32_t tmem_base;
   Abort abort;
 };
 
-// Shared prologue: barriers, TMEM allocation (512 columns).
+// Shared prologue: barriers, TMEM allocation (512 columns). fix_full counts one
+// arrival (the copy of the fixed tiles) or, with FIXT, one per compute warp.
+template <bool FIXT>
 __device__ __forceinline__ void bwd_setup(BwdBars* bars, int warp) {
   if (threadIdx.x == 0) {
-    mbar_init(&bars->fix_full, 1);
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(&bars->ring_full[s], 1);
-      mbar_init(&bars->ring_empty[s], 1);
-    }
-    for (int h = 0; h < 2; ++h) {
-      mbar_init(&bars->s_ready[h], 1);
-      mbar_init(&bars->ds_ready[h], kComputeThreads / 2);
-    }
+    mbar_init(&bars->fix_full, FIXT ? kComputeWarps : 1);
+    for (int s = 0; s < kMaxStages; ++s)
+      for (int o = 0; o < 2; ++o) {
+        mbar_init(&bars->ring_full[s][o], 1);
+        mbar_init(&bars->ring_empty[s][o], 1);
+      }
+    mbar_init(&bars->x_full, 1);
+    mbar_init(&bars->y_full, 1);
+    mbar_init(&bars->x_free, kComputeWarps);     // one arrival per compute warp
+    mbar_init(&bars->ds_ready, kComputeWarps);
     mbar_init(&bars->done, 1);
     mbar_init(&bars->drain, 1);
     bars->abort.flag = 0;
@@ -105,109 +127,141 @@ __device__ __forceinline__ void bwd_teardown(uint32_t tbase, int warp) {
   }
 }
 
-// Producer: the two fixed tiles once, then `n` pairs of streamed tiles at
-// rows (first + t) * 128 of maps ma, mb.
-template <int D>
+// Producer: the two fixed tiles once (unless FIXT), then `n` streamed tiles of
+// rows (first + t) * 128 of maps ma (operand A_t) and mb (B_t).
+template <int D, bool FIXT>
 __device__ void bwd_produce(uint8_t* sm, BwdBars* bars, const CUtensorMap* f0, const CUtensorMap* f1,
                             int frow, const CUtensorMap* ma, const CUtensorMap* mb, int first, int n,
                             int bh, volatile Abort* ab, int* err) {
-  using Lay = BwdLayout<D>;
-  constexpr int SUB = Lay::SUB;
-  mbar_expect_tx(&bars->fix_full, 2 * SUB * kSub);
-  for (int c = 0; c < SUB; ++c) {
-    tma_load_3d(sm + Lay::FIX0 + c * kSub, f0, &bars->fix_full, 64 * c, frow * kT, bh);
-    tma_load_3d(sm + Lay::FIX1 + c * kSub, f1, &bars->fix_full, 64 * c, frow * kT, bh);
-  }
-  int issued = 0;
-  for (int t = 0; t < n; ++t) {
-    const int st = t % kStages;
-    if (t >= kStages && !mbar_wait(&bars->ring_empty[st], ((t / kStages) - 1) & 1, ab, err, 11)) break;
-    uint8_t* base = sm + Lay::RING + st * Lay::STAGE;
-    mbar_expect_tx(&bars->ring_full[st], Lay::STAGE);
+  using Lay = BwdLayout<D, FIXT>;
+  constexpr int SUB = Lay::SUB, NST = Lay::NST;
+  if (!FIXT) {
+    mbar_expect_tx(&bars->fix_full, 2 * SUB * kSub);
     for (int c = 0; c < SUB; ++c) {
-      tma_load_3d(base + c * kSub, ma, &bars->ring_full[st], 64 * c, (first + t) * kT, bh);
-      tma_load_3d(base + (SUB + c) * kSub, mb, &bars->ring_full[st], 64 * c, (first + t) * kT, bh);
+      tma_load_3d(sm + Lay::FIX0 + c * kSub, f0, &bars->fix_full, 64 * c, frow * kT, bh);
+      tma_load_3d(sm + Lay::FIX1 + c * kSub, f1, &bars->fix_full, 64 * c, frow * kT, bh);
     }
-    issued = t + 1;
+  }
+  int issued = 0;                        // (tile, operand) loads issued, in order
+  for (int t = 0; t < n; ++t) {
+    const int st = t % NST;
+    uint8_t* base = sm + Lay::RING + st * Lay::STAGE;
+    bool go = true;
+    for (int o = 0; o < 2; ++o) {
+      if (t >= NST && !mbar_wait(&bars->ring_empty[st][o], ((t / NST) - 1) & 1, ab, err, 11)) {
+        go = false;
+        break;
+      }
+      uint64_t* full = &bars->ring_full[st][o];
+      mbar_expect_tx(full, SUB * kSub);
+      for (int c = 0; c < SUB; ++c)
+        tma_load_3d(base + (o * SUB + c) * kSub, o ? mb : ma, full, 64 * c, (first + t) * kT, bh);
+      issued = 2 * t + o + 1;
+    }
+    if (!go) break;
   }
   if (ab->flag) {
+    // wind-down: let the copies still in flight land before the CTA exits
     Abort none{0};
-    mbar_wait(&bars->fix_full, 0, &none, nullptr, 0);
-    for (int t = issued - kStages < 0 ? 0 : issued - kStages; t < issued; ++t)
-      mbar_wait(&bars->ring_full[t % kStages], (t / kStages) & 1, &none, nullptr, 0);
+    if (!FIXT) mbar_wait(&bars->fix_full, 0, &none, nullptr, 0);
+    for (int u = issued - 2 * NST < 0 ? 0 : issued - 2 * NST; u < issued; ++u)
+      mbar_wait(&bars->ring_full[(u >> 1) % NST][u & 1], ((u >> 1) / NST) & 1, &none, nullptr, 0);
   }
 }
 
-// MMA issuer shared by both kernels, pipelined by half tiles. For streamed
-// tile t and half h (its rows 64h..64h+63):
-//   X_h = F0 * A_t[h]^T (TMEM cols 64h..64h+63), Y_h = F1 * B_t[h]^T (cols 128+64h..)
-// and, once compute warpgroup h has turned X_h/Y_h into fp16 operands in place,
-//   dkdv (TWO_ACC): acc0 += Xh * B_t[h] (dV += P^T dO),  acc1 += Yh * A_t[h] (dK += dS^T Q)
-//   dq:             acc1 += Xh * A_t[h] + Yh * A_t[h]   (dQ += (dS_hi + dS_lo) K)
-// Issue order: acc(t-1, 0), X/Y_0(t), acc(t-1, 1), X/Y_1(t), ... so the tensor
-// core works on one half while the other half's warps compute. acc(t-1, h)
-// reads the fp16 values that X/Y_h(t) then overwrite; MMAs issued by one thread
-// execute in issue order, which makes that safe without a wait.
-template <int D, bool TWO_ACC>
+// MMA issuer shared by both kernels. For streamed tile t in stage st:
+//   X(t) = F0 * A_t^T -> cols 0..127,  Y(t) = F1 * B_t^T -> cols 128..255
+//   (F0/F1: shared-memory tiles, or with FIXT the TMEM columns kFixCol..),
+//   acc(t), A operand from Y's columns (fp16 pairs; chunk c = 32 columns of
+//   the tile, its first 16 packed columns hold P^T / dS_hi, the next 16 dS^T /
+//   dS_lo):
+//     dkdv (TWO_ACC): dK += dS^T A_t, then dV += P^T B_t
+//     dq:             dQ += dS_hi A_t + dS_lo A_t
+// Issue order: X(0), Y(0), then per t: X(t+1), acc(t), Y(t+1).
+template <int D, bool TWO_ACC, bool FIXT>
 __device__ void bwd_mma(uint8_t* sm, BwdBars* bars, uint32_t tbase, int n, volatile Abort* ab, int* err) {
-  using Lay = BwdLayout<D>;
-  constexpr int SUB = Lay::SUB;
-  constexpr uint32_t IDX = idesc_f16(kT, 64, false);
-  constexpr uint32_t IDACC = idesc_f16(kT, D, true);
+  using Lay = BwdLayout<D, FIXT>;
+  constexpr int SUB = Lay::SUB, NST = Lay::NST;
+  constexpr uint32_t IDX = idesc_f16(kT, kT, false);      // scores: both operands K-major
+  constexpr uint32_t IDACC = idesc_f16(kT, D, true);      // accumulate: B MN-major
   const uint32_t sbase = smem_u32(sm);
-  const uint32_t tX = tbase, tY = tbase + 128;
-  const uint32_t tAcc0 = tbase + 256, tAcc1 = tbase + 256 + (TWO_ACC ? D : 0);
-  auto issue_xy = [&](int t, int h) {
-    const uint32_t ring = sbase + Lay::RING + (t % kStages) * Lay::STAGE;
+  const uint32_t tX = tbase, tY = tbase + kColY;
+  const uint32_t tAcc0 = tbase + kColAcc, tAcc1 = tbase + kColAcc + (TWO_ACC ? D : 0);
+  auto ring = [&](int t) -> uint32_t { return sbase + Lay::RING + (t % NST) * Lay::STAGE; };
+  auto issue_x = [&](int t) {
+    const uint32_t tile = ring(t);
 #pragma unroll
     for (int kk = 0; kk < D / 16; ++kk) {
       const uint32_t koff = (kk >> 2) * kSub + (kk & 3) * 32;
-      umma_f16(tX + 64 * h, sdesc_sw128(sbase + Lay::FIX0 + koff, 16, 1024),
-               sdesc_sw128(ring + koff + 8192 * h, 16, 1024), IDX, kk > 0 ? 1u : 0u);
+      const uint64_t b = sdesc_sw128(tile + koff, 16, 1024);
+      if (FIXT) umma_f16_ts(tX, tbase + kFixCol + 8 * kk, b, IDX, kk > 0 ? 1u : 0u);
+      else umma_f16(tX, sdesc_sw128(sbase + Lay::FIX0 + koff, 16, 1024), b, IDX, kk > 0 ? 1u : 0u);
     }
-#pragma unroll
-    for (int kk = 0; kk < D / 16; ++kk) {
-      const uint32_t koff = (kk >> 2) * kSub + (kk & 3) * 32;
-      umma_f16(tY + 64 * h, sdesc_sw128(sbase + Lay::FIX1 + koff, 16, 1024),
-               sdesc_sw128(ring + SUB * kSub + koff + 8192 * h, 16, 1024), IDX, kk > 0 ? 1u : 0u);
-    }
-    umma_commit(&bars->s_ready[h]);
+    umma_commit(&bars->x_full);
   };
-  auto accumulate = [&](int tt, int h) -> bool {
-    if (!mbar_wait(&bars->ds_ready[h], tt & 1, ab, err, 14)) return false;
-    tc_fence_after();
-    const int st = tt % kStages;
-    const uint32_t ring = sbase + Lay::RING + st * Lay::STAGE;
-    const uint32_t tileA = ring, tileB = ring + SUB * kSub;
+  auto issue_y = [&](int t) {
+    const uint32_t tile = ring(t) + SUB * kSub;
 #pragma unroll
-    for (int kk = 0; kk < 4; ++kk) {
-      const uint32_t acol = 64 * h + 8 * kk;        // half h's packed operand columns
-      const uint32_t roff = (4 * h + kk) * 2048;     // its 16 rows of the streamed tiles
-      const uint32_t first = (tt == 0 && h == 0 && kk == 0) ? 0u : 1u;
-      const uint64_t g = sdesc_sw128(tileA + roff, kSub, 1024);
-      if (TWO_ACC) {
-        const uint64_t b = sdesc_sw128(tileB + roff, kSub, 1024);
-        umma_f16_ts(tAcc0, tX + acol, b, IDACC, first);
-        umma_f16_ts(tAcc1, tY + acol, g, IDACC, first);
-      } else {
-        umma_f16_ts(tAcc1, tX + acol, g, IDACC, first);
-        umma_f16_ts(tAcc1, tY + acol, g, IDACC, 1u);
+    for (int kk = 0; kk < D / 16; ++kk) {
+      const uint32_t koff = (kk >> 2) * kSub + (kk & 3) * 32;
+      const uint64_t b = sdesc_sw128(tile + koff, 16, 1024);
+      if (FIXT) umma_f16_ts(tY, tbase + kFixCol + D / 2 + 8 * kk, b, IDX, kk > 0 ? 1u : 0u);
+      else umma_f16(tY, sdesc_sw128(sbase + Lay::FIX1 + koff, 16, 1024), b, IDX, kk > 0 ? 1u : 0u);
+    }
+    umma_commit(&bars->y_full);
+    if (!TWO_ACC) umma_commit(&bars->ring_empty[t % NST][1]);   // dq: V_j has no other reader
+  };
+  auto issue_acc = [&](int t) {
+    const int st = t % NST;
+    const uint32_t tileA = ring(t), tileB = tileA + SUB * kSub;
+    // slice kk = 16 rows of the streamed tiles; its packed operand columns
+    auto acol = [](int kk) -> uint32_t { return 32 * (kk >> 1) + 8 * (kk & 1); };
+    if (TWO_ACC) {
+#pragma unroll
+      for (int kk = 0; kk < kT / 16; ++kk)
+        umma_f16_ts(tAcc1, tY + acol(kk) + 16, sdesc_sw128(tileA + kk * 2048, kSub, 1024), IDACC,
+                    (t > 0 || kk > 0) ? 1u : 0u);
+      umma_commit(&bars->ring_empty[st][0]);
+#pragma unroll
+      for (int kk = 0; kk < kT / 16; ++kk)
+        umma_f16_ts(tAcc0, tY + acol(kk), sdesc_sw128(tileB + kk * 2048, kSub, 1024), IDACC,
+                    (t > 0 || kk > 0) ? 1u : 0u);
+      umma_commit(&bars->ring_empty[st][1]);
+    } else {
+#pragma unroll
+      for (int kk = 0; kk < kT / 16; ++kk) {
+        const uint64_t b = sdesc_sw128(tileA + kk * 2048, kSub, 1024);
+        umma_f16_ts(tAcc0, tY + acol(kk), b, IDACC, (t > 0 || kk > 0) ? 1u : 0u);
+        umma_f16_ts(tAcc0, tY + acol(kk) + 16, b, IDACC, 1u);
       }
+      umma_commit(&bars->ring_empty[st][0]);
     }
-    if (h == 1) umma_commit(&bars->ring_empty[st]);
-    return true;
   };
-  bool ok = mbar_wait(&bars->fix_full, 0, ab, err, 12);
+  auto ring_wait = [&](int t, int o) -> bool {
+    return mbar_wait(&bars->ring_full[t % NST][o], (t / NST) & 1, ab, err, 13);
+  };
+  bool ok = mbar_wait(&bars->fix_full, 0, ab, err, 12) && ring_wait(0, 0);
+  if (ok) {
+    tc_fence_after();
+    issue_x(0);
+    ok = ring_wait(0, 1);
+  }
+  if (ok) issue_y(0);
   for (int t = 0; ok && t < n; ++t) {
-    const int st = t % kStages;
-    if (!mbar_wait(&bars->ring_full[st], (t / kStages) & 1, ab, err, 13)) { ok = false; break; }
-    for (int h = 0; h < 2; ++h) {
-      if (t >= 1 && !accumulate(t - 1, h)) { ok = false; break; }
+    if (t + 1 < n) {
+      if (!ring_wait(t + 1, 0) || !mbar_wait(&bars->x_free, t & 1, ab, err, 14)) { ok = false; break; }
       tc_fence_after();
-      issue_xy(t, h);
+      issue_x(t + 1);
+    }
+    if (!mbar_wait(&bars->ds_ready, t & 1, ab, err, 15)) { ok = false; break; }
+    tc_fence_after();
+    issue_acc(t);
+    if (t + 1 < n) {
+      if (!ring_wait(t + 1, 1)) { ok = false; break; }
+      issue_y(t + 1);
     }
   }
-  if (ok && accumulate(n - 1, 0) && accumulate(n - 1, 1)) umma_commit(&bars->done);
+  if (ok) umma_commit(&bars->done);
   umma_commit(&bars->drain);
   Abort none{0};
   mbar_wait(&bars->drain, 0, &none, nullptr, 0);
@@ -218,20 +272,17 @@ __device__ __forceinline__ float2 f2(uint32_t a, uint32_t b) {
 }
 __device__ __forceinline__ uint32_t h2_bits(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
 
-// One 32-column chunk of this thread's key row of S^T and dP^T (dK/dV kernel):
-// P^T = 2^(S^T c2 - lse2) and dS^T = P^T o (dP^T - delta) as fp16 pairs, two
-// columns per packed fp32 instruction. nl2/ndl hold -lse2 and -delta of the
-// chunk's 32 query columns (the same for every lane: broadcast reads). MASK:
-// columns outside [vlo, vhi] (causal diagonal, rows past S) get P = 0.
+// 32 columns of this thread's key row (dK/dV kernel): P^T = 2^(S^T c2 - lse2)
+// in place, two columns per packed fp32 instruction. nl2 holds -lse2 of the
+// 32 query columns (the same for every lane: broadcast reads). MASK: columns
+// outside [vlo, vhi] (causal diagonal, rows past S) get P = 0.
 template <bool MASK>
-__device__ __forceinline__ void dkdv_chunk(const uint32_t (&s)[32], const uint32_t (&dp)[32],
-                                           const float* nl2, const float* ndl, float c2, int col0, int vlo,
-                                           int vhi, uint32_t (&pk)[16], uint32_t (&dk)[16], __half2& hm) {
+__device__ __forceinline__ void p_chunk_t(uint32_t (&s)[32], const float* nl2, float c2, int col0, int vlo,
+                                          int vhi) {
   const float2 cc = make_float2(c2, c2);
 #pragma unroll
   for (int e = 0; e < 32; e += 4) {
     const float4 a = *reinterpret_cast<const float4*>(nl2 + e);
-    const float4 b = *reinterpret_cast<const float4*>(ndl + e);
 #pragma unroll
     for (int u = 0; u < 4; u += 2) {
       const float2 x = __ffma2_rn(f2(s[e + u], s[e + u + 1]), cc, u ? make_float2(a.z, a.w) : make_float2(a.x, a.y));
@@ -241,24 +292,36 @@ __device__ __forceinline__ void dkdv_chunk(const uint32_t (&s)[32], const uint32
         if (col < vlo || col > vhi) p0 = 0.f;
         if (col + 1 < vlo || col + 1 > vhi) p1 = 0.f;
       }
+      s[e + u] = __float_as_uint(p0);
+      s[e + u + 1] = __float_as_uint(p1);
+    }
+  }
+}
+
+// dS^T = P^T o (dP^T - delta) for 32 columns; P^T and dS^T as fp16 pairs.
+// ndl holds -delta of the 32 query columns.
+__device__ __forceinline__ void ds_chunk_t(const uint32_t (&p)[32], const uint32_t (&dp)[32], const float* ndl,
+                                           uint32_t (&pk)[16], uint32_t (&dk)[16], __half2& hm) {
+#pragma unroll
+  for (int e = 0; e < 32; e += 4) {
+    const float4 b = *reinterpret_cast<const float4*>(ndl + e);
+#pragma unroll
+    for (int u = 0; u < 4; u += 2) {
+      const float2 pp = f2(p[e + u], p[e + u + 1]);
       const float2 d = __fadd2_rn(f2(dp[e + u], dp[e + u + 1]), u ? make_float2(b.z, b.w) : make_float2(b.x, b.y));
-      const __half2 ds = __float22half2_rn(__fmul2_rn(make_float2(p0, p1), d));
+      const __half2 ds = __float22half2_rn(__fmul2_rn(pp, d));
       hm = __hmax2_nan(hm, __habs2(ds));
-      pk[(e + u) >> 1] = pack_f16(p0, p1);
+      pk[(e + u) >> 1] = h2_bits(__float22half2_rn(pp));
       dk[(e + u) >> 1] = h2_bits(ds);
     }
   }
 }
 
-// One 32-column chunk of this thread's query row of S and dP (dQ kernel): dS as
-// an fp16 head and an fp16 remainder (hi + lo = dS to about 2^-22 relative).
-// nl2 = -lse2, ndl = -delta of the row. MASK: key columns past vhi get P = 0.
+// 32 columns of this thread's query row (dQ kernel): P = 2^(S c2 - lse2) in
+// place. nl2 = -lse2 of the row. MASK: key columns past vhi get P = 0.
 template <bool MASK>
-__device__ __forceinline__ void dq_chunk(const uint32_t (&s)[32], const uint32_t (&dp)[32], float nl2, float ndl,
-                                         float c2, int col0, int vhi, uint32_t (&hi)[16], uint32_t (&lo)[16],
-                                         __half2& hm) {
-  const float2 cc = make_float2(c2, c2), nl = make_float2(nl2, nl2), nd = make_float2(ndl, ndl);
-  const float2 m1 = make_float2(-1.f, -1.f);
+__device__ __forceinline__ void p_chunk(uint32_t (&s)[32], float nl2, float c2, int col0, int vhi) {
+  const float2 cc = make_float2(c2, c2), nl = make_float2(nl2, nl2);
 #pragma unroll
   for (int e = 0; e < 32; e += 2) {
     const float2 x = __ffma2_rn(f2(s[e], s[e + 1]), cc, nl);
@@ -267,7 +330,18 @@ __device__ __forceinline__ void dq_chunk(const uint32_t (&s)[32], const uint32_t
       if (col0 + e > vhi) p0 = 0.f;
       if (col0 + e + 1 > vhi) p1 = 0.f;
     }
-    const float2 ds = __fmul2_rn(make_float2(p0, p1), __fadd2_rn(f2(dp[e], dp[e + 1]), nd));
+    s[e] = __float_as_uint(p0);
+    s[e + 1] = __float_as_uint(p1);
+  }
+}
+
+// dS = P o (dP - delta) for 32 columns, as an fp16 head and an fp16 remainder.
+__device__ __forceinline__ void ds_chunk(const uint32_t (&p)[32], const uint32_t (&dp)[32], float ndl,
+                                         uint32_t (&hi)[16], uint32_t (&lo)[16], __half2& hm) {
+  const float2 nd = make_float2(ndl, ndl), m1 = make_float2(-1.f, -1.f);
+#pragma unroll
+  for (int e = 0; e < 32; e += 2) {
+    const float2 ds = __fmul2_rn(f2(p[e], p[e + 1]), __fadd2_rn(f2(dp[e], dp[e + 1]), nd));
     const __half2 h = __float22half2_rn(ds);
     hm = __hmax2_nan(hm, __habs2(h));
     const float2 r = __ffma2_rn(__half22float2(h), m1, ds);     // ds - hi, exact
@@ -279,11 +353,11 @@ __device__ __forceinline__ void dq_chunk(const uint32_t (&s)[32], const uint32_t
 // ---------------------------------------------------------------- dK, dV
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
-k_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
-              const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tdo,
+k_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
+              const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tdo,
               const float* __restrict__ lse, const float* __restrict__ delta, float* __restrict__ dks,
               float* __restrict__ dvs, int S, float c2, float scale, int* err) {
-  using Lay = BwdLayout<D>;
+  using Lay = BwdLayout<D, false>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   BwdBars* bars = reinterpret_cast<BwdBars*>(sm + Lay::BAR);
@@ -292,20 +366,21 @@ k_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CU
   const int j = blockIdx.x;            // key tile; small j has the most query tiles
   const int bh = blockIdx.y;
   const int n = ntiles - j;            // query tiles i = j .. ntiles-1
-  bwd_setup(bars, warp);
+  bwd_setup<false>(bars, warp);
   const uint32_t tbase = bars->tmem_base;
   volatile Abort* ab = &bars->abort;
 
   if (warp == 0) {
-    if (lane == 0) bwd_produce<D>(sm, bars, &tk, &tv, j, &tq, &tdo, j, n, bh, ab, err);
+    if (lane == 0) bwd_produce<D, false>(sm, bars, &tk, &tv, j, &tq, &tdo, j, n, bh, ab, err);
   } else if (warp == 1) {
-    if (lane == 0) bwd_mma<D, true>(sm, bars, tbase, n, ab, err);
+    if (lane == 0) bwd_mma<D, true, false>(sm, bars, tbase, n, ab, err);
   } else {
     const int quarter = warp & 3;
     const int half = (warp - 2) >> 2;                   // which 64 of the 128 columns
     const int m = quarter * 32 + lane;                  // key row within the tile / TMEM lane
     const int ctid = threadIdx.x - 64;                  // 0..255
     const uint32_t la = (uint32_t)(quarter * 32) << 16;
+    const uint32_t cX = tbase + la + 64 * half, cY = cX + kColY;
     const int key = j * kT + m;
     float* vec = reinterpret_cast<float*>(sm + Lay::VEC);   // [2][2][128]: -lse2, -delta
     // this thread's share of a query tile's -lse2 / -delta (thread hid of the
@@ -330,41 +405,49 @@ k_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CU
       (hid < 64 ? nl2 : ndl)[hid & 63] = nxt * vmul;
       named_bar_sync(1 + half, kComputeThreads / 2);
       if (t + 1 < n) nxt = fetch(i + 1);
-      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bars->s_ready[half], t & 1, ab, err, 15));
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bars->x_full, t & 1, ab, err, 16));
       if (!ok) continue;
       tc_fence_after();
+      // S^T: this warp's 64 columns into registers, then X is released
+      uint32_t p0[32], p1[32];
+      tmem_ld32(cX, p0);
+      tmem_ld32(cX + 32, p1);
+      tmem_wait_ld_regs(p0);
+      reg_fence32(p1);
+      tc_fence_before();
+      mbar_arrive_warp(&bars->x_free);
       const int vlo = i == j ? m : 0;                   // causal: query col >= key row
       const int vhi = min(kT - 1, S - 1 - i * kT);      // last valid query column
-      const bool mask = vlo > 0 || vhi < kT - 1 || i == j;
-      // chunk c0 = 2*half, then c0 + 1; the second chunk's loads overlap the
-      // first chunk's arithmetic
-      const int c0 = 2 * half;
-      uint32_t s0[32], d0[32], s1[32], d1[32], pk[16], dk[16];
-      tmem_ld32(tbase + la + 32 * c0, s0);
-      tmem_ld32(tbase + la + 128 + 32 * c0, d0);
-      tmem_wait_ld_regs(s0);
-      reg_fence32(d0);
-      tmem_ld32(tbase + la + 32 * c0 + 32, s1);
-      tmem_ld32(tbase + la + 160 + 32 * c0, d1);
-      if (mask) dkdv_chunk<true>(s0, d0, nl2, ndl, c2, 32 * c0, vlo, vhi, pk, dk, hm);
-      else dkdv_chunk<false>(s0, d0, nl2, ndl, c2, 32 * c0, vlo, vhi, pk, dk, hm);
-      // fp16 results go to columns this warp has already read: chunk c's 16
-      // packed columns at 16c + 32*half (each half packs inside its own 64)
-      tmem_st16(tbase + la + 16 * c0 + 32 * half, pk);
-      tmem_st16(tbase + la + 128 + 16 * c0 + 32 * half, dk);
-      tmem_wait_ld_regs(s1);
+      if (vlo > 0 || vhi < kT - 1 || i == j) {
+        p_chunk_t<true>(p0, nl2, c2, 64 * half, vlo, vhi);
+        p_chunk_t<true>(p1, nl2 + 32, c2, 64 * half + 32, vlo, vhi);
+      } else {
+        p_chunk_t<false>(p0, nl2, c2, 0, 0, 0);
+        p_chunk_t<false>(p1, nl2 + 32, c2, 0, 0, 0);
+      }
+      ok = __all_sync(0xffffffffu, mbar_wait(&bars->y_full, t & 1, ab, err, 17));
+      if (!ok) continue;
+      tc_fence_after();
+      // dP^T: both 32-column chunks, then P^T / dS^T as fp16 into the chunk's
+      // own (already read) columns: P^T at +0..15, dS^T at +16..31
+      uint32_t d0[32], d1[32], pk[16], dk[16];
+      tmem_ld32(cY, d0);
+      tmem_ld32(cY + 32, d1);
+      tmem_wait_ld_regs(d0);
       reg_fence32(d1);
-      if (mask) dkdv_chunk<true>(s1, d1, nl2 + 32, ndl + 32, c2, 32 * c0 + 32, vlo, vhi, pk, dk, hm);
-      else dkdv_chunk<false>(s1, d1, nl2 + 32, ndl + 32, c2, 32 * c0 + 32, vlo, vhi, pk, dk, hm);
-      tmem_st16(tbase + la + 16 * c0 + 16 + 32 * half, pk);
-      tmem_st16(tbase + la + 128 + 16 * c0 + 16 + 32 * half, dk);
+      ds_chunk_t(p0, d0, ndl, pk, dk, hm);
+      tmem_st16(cY, pk);
+      tmem_st16(cY + 16, dk);
+      ds_chunk_t(p1, d1, ndl + 32, pk, dk, hm);
+      tmem_st16(cY + 32, pk);
+      tmem_st16(cY + 48, dk);
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&bars->ds_ready[half]);
+      mbar_arrive_warp(&bars->ds_ready);
     }
     const float dsmax = __half2float(__hmax_nan(__low2half(hm), __high2half(hm)));
     if (!(dsmax <= kHalfMax)) report_error(err, LH_ERR_DEVICE, 101);
-    if (ok && __all_sync(0xffffffffu, mbar_wait(&bars->done, 0, ab, err, 16))) {
+    if (ok && __all_sync(0xffffffffu, mbar_wait(&bars->done, 0, ab, err, 18))) {
       tc_fence_after();
       float* ddv = dvs + ((size_t)bh * S + key) * D;
       float* ddk = dks + ((size_t)bh * S + key) * D;
@@ -373,8 +456,8 @@ k_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CU
         // the TMEM loads are warp-collective (.sync.aligned): every lane runs
         // them, rows past S included; only the stores are per-row
         uint32_t a[32], b[32];
-        tmem_ld32(tbase + la + 256 + 32 * c, a);
-        tmem_ld32(tbase + la + 256 + D + 32 * c, b);
+        tmem_ld32(tbase + la + kColAcc + 32 * c, a);
+        tmem_ld32(tbase + la + kColAcc + D + 32 * c, b);
         tmem_wait_ld();
         if (key < S) {
 #pragma unroll
@@ -396,11 +479,11 @@ k_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CU
 // ---------------------------------------------------------------- dQ
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
-k_bwd_dq_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
-            const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tdo,
+k_bwd_dq_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
+            const __half* __restrict__ qh, const __half* __restrict__ doh,
             const float* __restrict__ lse, const float* __restrict__ delta, float* __restrict__ dqs,
             int S, float c2, float scale, int* err) {
-  using Lay = BwdLayout<D>;
+  using Lay = BwdLayout<D, true>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   BwdBars* bars = reinterpret_cast<BwdBars*>(sm + Lay::BAR);
@@ -409,63 +492,89 @@ k_bwd_dq_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
   const int i = ntiles - 1 - (int)blockIdx.x;     // query tile; late tiles have the most key tiles
   const int bh = blockIdx.y;
   const int n = i + 1;                            // key tiles j = 0 .. i
-  bwd_setup(bars, warp);
+  bwd_setup<true>(bars, warp);
   const uint32_t tbase = bars->tmem_base;
   volatile Abort* ab = &bars->abort;
 
   if (warp == 0) {
-    if (lane == 0) bwd_produce<D>(sm, bars, &tq, &tdo, i, &tk, &tv, 0, n, bh, ab, err);
+    if (lane == 0) bwd_produce<D, true>(sm, bars, nullptr, nullptr, i, &tk, &tv, 0, n, bh, ab, err);
   } else if (warp == 1) {
-    if (lane == 0) bwd_mma<D, false>(sm, bars, tbase, n, ab, err);
+    if (lane == 0) bwd_mma<D, false, true>(sm, bars, tbase, n, ab, err);
   } else {
     const int quarter = warp & 3;
     const int half = (warp - 2) >> 2;             // which 64 of the 128 columns
     const int r = quarter * 32 + lane;            // query row within the tile / TMEM lane
     const uint32_t la = (uint32_t)(quarter * 32) << 16;
+    const uint32_t cX = tbase + la + 64 * half, cY = cX + kColY;
     const int q = i * kT + r;
     const float nl2 = q < S ? lse[(size_t)bh * S + q] * -1.4426950408889634f : 0.f;
     const float ndl = q < S ? -delta[(size_t)bh * S + q] : 0.f;
+    {
+      // fixed operands into TMEM as the score MMAs' A operand: lane r holds row
+      // q, column kFixCol + c the fp16 pair (2c, 2c+1) of Q_i (half-0 warps) or,
+      // D/2 columns on, of dO_i (half-1 warps); rows past S are zero
+      const uint4* src = reinterpret_cast<const uint4*>((half ? doh : qh) + ((size_t)bh * S + (q < S ? q : 0)) * D);
+#pragma unroll 1
+      for (int c = 0; c < D / 64; ++c) {
+        uint32_t w[32];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const uint4 x = q < S ? src[8 * c + e] : make_uint4(0, 0, 0, 0);
+          w[4 * e] = x.x; w[4 * e + 1] = x.y; w[4 * e + 2] = x.z; w[4 * e + 3] = x.w;
+        }
+        tmem_st32(tbase + la + kFixCol + half * (D / 2) + 32 * c, w);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive_warp(&bars->fix_full);
+    }
     __half2 hm = __float2half2_rn(0.f);
     bool ok = true;
     for (int jj = 0; jj < n; ++jj) {
-      if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_ready[half], jj & 1, ab, err, 17))) { ok = false; break; }
+      if (!__all_sync(0xffffffffu, mbar_wait(&bars->x_full, jj & 1, ab, err, 19))) { ok = false; break; }
       tc_fence_after();
+      uint32_t p0[32], p1[32];
+      tmem_ld32(cX, p0);
+      tmem_ld32(cX + 32, p1);
+      tmem_wait_ld_regs(p0);
+      reg_fence32(p1);
+      tc_fence_before();
+      mbar_arrive_warp(&bars->x_free);
       const int klim = min(jj == i ? r : kT - 1, S - 1 - jj * kT);   // last valid key column
-      const bool mask = klim < kT - 1;
-      // chunk c0 = 2*half, then c0 + 1 (its loads overlap chunk c0's arithmetic);
-      // head into the (consumed) S columns, remainder into the (consumed) dP
-      // columns, packed inside this half's own 64 columns
-      const int c0 = 2 * half;
-      uint32_t s0[32], d0[32], s1[32], d1[32], hi[16], lo[16];
-      tmem_ld32(tbase + la + 32 * c0, s0);
-      tmem_ld32(tbase + la + 128 + 32 * c0, d0);
-      tmem_wait_ld_regs(s0);
-      reg_fence32(d0);
-      tmem_ld32(tbase + la + 32 * c0 + 32, s1);
-      tmem_ld32(tbase + la + 160 + 32 * c0, d1);
-      if (mask) dq_chunk<true>(s0, d0, nl2, ndl, c2, 32 * c0, klim, hi, lo, hm);
-      else dq_chunk<false>(s0, d0, nl2, ndl, c2, 32 * c0, klim, hi, lo, hm);
-      tmem_st16(tbase + la + 16 * c0 + 32 * half, hi);
-      tmem_st16(tbase + la + 128 + 16 * c0 + 32 * half, lo);
-      tmem_wait_ld_regs(s1);
+      if (klim < kT - 1) {
+        p_chunk<true>(p0, nl2, c2, 64 * half, klim);
+        p_chunk<true>(p1, nl2, c2, 64 * half + 32, klim);
+      } else {
+        p_chunk<false>(p0, nl2, c2, 0, 0);
+        p_chunk<false>(p1, nl2, c2, 0, 0);
+      }
+      if (!__all_sync(0xffffffffu, mbar_wait(&bars->y_full, jj & 1, ab, err, 20))) { ok = false; break; }
+      tc_fence_after();
+      // dP: both chunks, then head / remainder into the chunk's own columns
+      uint32_t d0[32], d1[32], hi[16], lo[16];
+      tmem_ld32(cY, d0);
+      tmem_ld32(cY + 32, d1);
+      tmem_wait_ld_regs(d0);
       reg_fence32(d1);
-      if (mask) dq_chunk<true>(s1, d1, nl2, ndl, c2, 32 * c0 + 32, klim, hi, lo, hm);
-      else dq_chunk<false>(s1, d1, nl2, ndl, c2, 32 * c0 + 32, klim, hi, lo, hm);
-      tmem_st16(tbase + la + 16 * c0 + 16 + 32 * half, hi);
-      tmem_st16(tbase + la + 128 + 16 * c0 + 16 + 32 * half, lo);
+      ds_chunk(p0, d0, ndl, hi, lo, hm);
+      tmem_st16(cY, hi);
+      tmem_st16(cY + 16, lo);
+      ds_chunk(p1, d1, ndl, hi, lo, hm);
+      tmem_st16(cY + 32, hi);
+      tmem_st16(cY + 48, lo);
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&bars->ds_ready[half]);
+      mbar_arrive_warp(&bars->ds_ready);
     }
     const float dsmax = __half2float(__hmax_nan(__low2half(hm), __high2half(hm)));
     if (!(dsmax <= kHalfMax)) report_error(err, LH_ERR_DEVICE, 101);
-    if (ok && __all_sync(0xffffffffu, mbar_wait(&bars->done, 0, ab, err, 18))) {
+    if (ok && __all_sync(0xffffffffu, mbar_wait(&bars->done, 0, ab, err, 21))) {
       tc_fence_after();
       float* dst = dqs + ((size_t)bh * S + q) * D;
 #pragma unroll 1
       for (int c = half * (D / 64); c < (half + 1) * (D / 64); ++c) {
         uint32_t a[32];
-        tmem_ld32(tbase + la + 256 + 32 * c, a);
+        tmem_ld32(tbase + la + kColAcc + 32 * c, a);
         tmem_wait_ld();
         if (q < S) {
 #pragma unroll
@@ -486,22 +595,23 @@ cudaError_t bwd_tc_t(const Geom& g, const void* qs, const void* ks, const void* 
                      cudaStream_t s) {
   CUtensorMap tq, tk, tv, tdo;
   const int BH = g.B * g.H;
-  if (!make_tmap_16(&tq, qs, D, g.S, BH, true) || !make_tmap_16(&tk, ks, D, g.S, BH, true) ||
-      !make_tmap_16(&tv, vs, D, g.S, BH, true) || !make_tmap_16(&tdo, dos, D, g.S, BH, true))
+  if (!make_tmap_16(&tq, qs, D, g.S, BH, true, kT) || !make_tmap_16(&tk, ks, D, g.S, BH, true, kT) ||
+      !make_tmap_16(&tv, vs, D, g.S, BH, true, kT) || !make_tmap_16(&tdo, dos, D, g.S, BH, true, kT))
     return cudaErrorInvalidValue;
-  const int smem = BwdLayout<D>::BYTES;
+  const int smem = BwdLayout<D, false>::BYTES, smem_q = BwdLayout<D, true>::BYTES;
   cudaError_t e = cudaFuncSetAttribute(k_bwd_dkdv_tc<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(k_bwd_dq_tc<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  e = cudaFuncSetAttribute(k_bwd_dq_tc<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_q);
   if (e != cudaSuccess) return e;
   const float scale = (float)(1.0 / sqrt((double)D));
   const float c2 = (float)(1.4426950408889634 / sqrt((double)D));
   dim3 grid((g.S + kT - 1) / kT, BH);
-  k_bwd_dkdv_tc<D><<<grid, kThreads, smem, s>>>(tq, tk, tv, tdo, lse, delta, dks, dvs, g.S, c2, scale, err);
+  k_bwd_dkdv_tc<D><<<grid, kThreads, smem, s>>>(tk, tv, tq, tdo, lse, delta, dks, dvs, g.S, c2, scale, err);
   count_launch();
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  k_bwd_dq_tc<D><<<grid, kThreads, smem, s>>>(tq, tk, tv, tdo, lse, delta, dqs, g.S, c2, scale, err);
+  k_bwd_dq_tc<D><<<grid, kThreads, smem_q, s>>>(tk, tv, (const __half*)qs, (const __half*)dos, lse, delta, dqs,
+                                                g.S, c2, scale, err);
   count_launch();
   return cudaGetLastError();
 }
