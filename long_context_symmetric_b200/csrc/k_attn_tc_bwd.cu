@@ -22,8 +22,9 @@
 //      X = S = Q_i K_j^T and Y = dP = dO_i V_j^T; dS is split into an fp16 head
 //      and an fp16 remainder (dS = hi + lo to about 2^-22 relative) stored into
 //      Y's columns; dQ += hi K_j + lo K_j.
-// A dS whose fp16 rounding overflows (or is NaN) is reported as LH_ERR_DEVICE,
-// detail 101.
+// A dS whose fp16 rounding overflows (or any NaN) makes dK and dQ non-finite
+// (an infinite operand times any value, summed in fp32, stays inf or NaN), so
+// the epilogues check their fp32 results and report LH_ERR_DEVICE, detail 101.
 //
 // Pipeline (tensor core order per streamed tile t):  X(t+1), acc(t), Y(t+1).
 // The compute warps copy X(t) into registers and release it at once, so X(t+1)
@@ -33,7 +34,9 @@
 // full 128 x 128 tiles: N = 64 halves run at about two thirds of the rate and
 // lose more when the compute warps use TMEM at the same time (measured).
 // Streamed tiles come through a TMA ring whose two operands have their own
-// full/empty barriers, so each is refilled as soon as its last reader is done.
+// stages and full/empty barriers, so each is refilled as soon as its last
+// reader is done; the operand that X reads gets three stages, as X(t+2) is
+// issued right after acc(t), before a two-stage ring could have refilled it.
 // Bounded waits as in the forward kernel.
 #include "tc_ptx.cuh"
 
@@ -62,20 +65,25 @@ __device__ __forceinline__ void named_bar_sync(int id, int n) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
 }
 
-// FIXT: the fixed operands live in TMEM (dQ kernel), which leaves room for a
-// third ring stage; otherwise (dK/dV kernel, whose TMEM holds two accumulators)
-// they are shared-memory tiles.
+// FIXT: the fixed operands live in TMEM (dQ kernel); otherwise (dK/dV kernel,
+// whose TMEM holds two accumulators) they are shared-memory tiles. Barriers and
+// the lse/delta vector come first, the swizzled tiles from the next 1024-byte
+// boundary (TILES bytes, offsets below relative to that boundary); BYTES covers
+// the worst-case alignment gap of the dynamic shared-memory base.
 template <int D, bool FIXT>
 struct BwdLayout {
   static constexpr int SUB = D / 64;
-  static constexpr int NST = FIXT ? 3 : 2;                     // ring stages
+  static constexpr int OPB = SUB * kSub;                       // one 128-row operand tile
+  static constexpr int NSTA = 3;                               // stages of A_t (read by X and acc)
+  static constexpr int NSTB = FIXT ? 3 : 2;                    // stages of B_t
   static constexpr int FIX0 = 0;                               // fixed operand 0 (K_j)
-  static constexpr int FIX1 = FIX0 + (FIXT ? 0 : SUB * kSub);  // fixed operand 1 (V_j)
-  static constexpr int RING = FIX1 + (FIXT ? 0 : SUB * kSub);  // stages of streamed tiles (A_t, B_t)
-  static constexpr int STAGE = 2 * SUB * kSub;
-  static constexpr int VEC = RING + NST * STAGE;               // lse / delta per query (dkdv)
-  static constexpr int BAR = VEC + (FIXT ? 0 : 2 * 2 * kT * 4);
-  static constexpr int BYTES = (BAR + 256 + 1024) > 120 * 1024 ? (BAR + 256 + 1024) : 120 * 1024;
+  static constexpr int FIX1 = FIX0 + (FIXT ? 0 : OPB);         // fixed operand 1 (V_j)
+  static constexpr int RA = FIX1 + (FIXT ? 0 : OPB);           // A_t stages
+  static constexpr int RB = RA + NSTA * OPB;                   // B_t stages
+  static constexpr int TILES = RB + NSTB * OPB;
+  static constexpr int HEAD = 256 + (FIXT ? 0 : 2 * kT * 4);   // barriers, then -lse2 / -delta (dkdv)
+  static constexpr int BYTES = HEAD + 1024 + TILES;
+  static_assert(BYTES <= 227 * 1024, "shared memory");
 };
 
 // ring_full/ring_empty[stage][o]: o = 0 the streamed operand A_t (Q_i in dkdv,
@@ -86,6 +94,7 @@ struct BwdBars {
   uint32_t tmem_base;
   Abort abort;
 };
+static_assert(sizeof(BwdBars) <= 256, "barrier block");
 
 // Shared prologue: barriers, TMEM allocation (512 columns). fix_full counts one
 // arrival (the copy of the fixed tiles) or, with FIXT, one per compute warp.
@@ -134,7 +143,7 @@ __device__ void bwd_produce(uint8_t* sm, BwdBars* bars, const CUtensorMap* f0, c
                             int frow, const CUtensorMap* ma, const CUtensorMap* mb, int first, int n,
                             int bh, volatile Abort* ab, int* err) {
   using Lay = BwdLayout<D, FIXT>;
-  constexpr int SUB = Lay::SUB, NST = Lay::NST;
+  constexpr int SUB = Lay::SUB, NSTA = Lay::NSTA, NSTB = Lay::NSTB;
   if (!FIXT) {
     mbar_expect_tx(&bars->fix_full, 2 * SUB * kSub);
     for (int c = 0; c < SUB; ++c) {
@@ -144,18 +153,18 @@ __device__ void bwd_produce(uint8_t* sm, BwdBars* bars, const CUtensorMap* f0, c
   }
   int issued = 0;                        // (tile, operand) loads issued, in order
   for (int t = 0; t < n; ++t) {
-    const int st = t % NST;
-    uint8_t* base = sm + Lay::RING + st * Lay::STAGE;
     bool go = true;
     for (int o = 0; o < 2; ++o) {
-      if (t >= NST && !mbar_wait(&bars->ring_empty[st][o], ((t / NST) - 1) & 1, ab, err, 11)) {
+      const int nst = o ? NSTB : NSTA, st = t % nst;
+      if (t >= nst && !mbar_wait(&bars->ring_empty[st][o], ((t / nst) - 1) & 1, ab, err, 11)) {
         go = false;
         break;
       }
       uint64_t* full = &bars->ring_full[st][o];
-      mbar_expect_tx(full, SUB * kSub);
+      uint8_t* dst = sm + (o ? Lay::RB : Lay::RA) + st * Lay::OPB;
+      mbar_expect_tx(full, Lay::OPB);
       for (int c = 0; c < SUB; ++c)
-        tma_load_3d(base + (o * SUB + c) * kSub, o ? mb : ma, full, 64 * c, (first + t) * kT, bh);
+        tma_load_3d(dst + c * kSub, o ? mb : ma, full, 64 * c, (first + t) * kT, bh);
       issued = 2 * t + o + 1;
     }
     if (!go) break;
@@ -164,8 +173,12 @@ __device__ void bwd_produce(uint8_t* sm, BwdBars* bars, const CUtensorMap* f0, c
     // wind-down: let the copies still in flight land before the CTA exits
     Abort none{0};
     if (!FIXT) mbar_wait(&bars->fix_full, 0, &none, nullptr, 0);
-    for (int u = issued - 2 * NST < 0 ? 0 : issued - 2 * NST; u < issued; ++u)
-      mbar_wait(&bars->ring_full[(u >> 1) % NST][u & 1], ((u >> 1) / NST) & 1, &none, nullptr, 0);
+    // the latest load into each stage of each operand
+    const int na = (issued + 1) / 2, nb = issued / 2;   // tiles of A_t / B_t issued
+    for (int tt = na - NSTA < 0 ? 0 : na - NSTA; tt < na; ++tt)
+      mbar_wait(&bars->ring_full[tt % NSTA][0], (tt / NSTA) & 1, &none, nullptr, 0);
+    for (int tt = nb - NSTB < 0 ? 0 : nb - NSTB; tt < nb; ++tt)
+      mbar_wait(&bars->ring_full[tt % NSTB][1], (tt / NSTB) & 1, &none, nullptr, 0);
   }
 }
 
@@ -181,15 +194,16 @@ __device__ void bwd_produce(uint8_t* sm, BwdBars* bars, const CUtensorMap* f0, c
 template <int D, bool TWO_ACC, bool FIXT>
 __device__ void bwd_mma(uint8_t* sm, BwdBars* bars, uint32_t tbase, int n, volatile Abort* ab, int* err) {
   using Lay = BwdLayout<D, FIXT>;
-  constexpr int SUB = Lay::SUB, NST = Lay::NST;
+  constexpr int NSTA = Lay::NSTA, NSTB = Lay::NSTB;
   constexpr uint32_t IDX = idesc_f16(kT, kT, false);      // scores: both operands K-major
   constexpr uint32_t IDACC = idesc_f16(kT, D, true);      // accumulate: B MN-major
   const uint32_t sbase = smem_u32(sm);
   const uint32_t tX = tbase, tY = tbase + kColY;
   const uint32_t tAcc0 = tbase + kColAcc, tAcc1 = tbase + kColAcc + (TWO_ACC ? D : 0);
-  auto ring = [&](int t) -> uint32_t { return sbase + Lay::RING + (t % NST) * Lay::STAGE; };
+  auto tile_a = [&](int t) -> uint32_t { return sbase + Lay::RA + (t % NSTA) * Lay::OPB; };
+  auto tile_b = [&](int t) -> uint32_t { return sbase + Lay::RB + (t % NSTB) * Lay::OPB; };
   auto issue_x = [&](int t) {
-    const uint32_t tile = ring(t);
+    const uint32_t tile = tile_a(t);
 #pragma unroll
     for (int kk = 0; kk < D / 16; ++kk) {
       const uint32_t koff = (kk >> 2) * kSub + (kk & 3) * 32;
@@ -200,7 +214,7 @@ __device__ void bwd_mma(uint8_t* sm, BwdBars* bars, uint32_t tbase, int n, volat
     umma_commit(&bars->x_full);
   };
   auto issue_y = [&](int t) {
-    const uint32_t tile = ring(t) + SUB * kSub;
+    const uint32_t tile = tile_b(t);
 #pragma unroll
     for (int kk = 0; kk < D / 16; ++kk) {
       const uint32_t koff = (kk >> 2) * kSub + (kk & 3) * 32;
@@ -209,11 +223,10 @@ __device__ void bwd_mma(uint8_t* sm, BwdBars* bars, uint32_t tbase, int n, volat
       else umma_f16(tY, sdesc_sw128(sbase + Lay::FIX1 + koff, 16, 1024), b, IDX, kk > 0 ? 1u : 0u);
     }
     umma_commit(&bars->y_full);
-    if (!TWO_ACC) umma_commit(&bars->ring_empty[t % NST][1]);   // dq: V_j has no other reader
+    if (!TWO_ACC) umma_commit(&bars->ring_empty[t % NSTB][1]);   // dq: V_j has no other reader
   };
   auto issue_acc = [&](int t) {
-    const int st = t % NST;
-    const uint32_t tileA = ring(t), tileB = tileA + SUB * kSub;
+    const uint32_t tileA = tile_a(t), tileB = tile_b(t);
     // slice kk = 16 rows of the streamed tiles; its packed operand columns
     auto acol = [](int kk) -> uint32_t { return 32 * (kk >> 1) + 8 * (kk & 1); };
     if (TWO_ACC) {
@@ -221,12 +234,12 @@ __device__ void bwd_mma(uint8_t* sm, BwdBars* bars, uint32_t tbase, int n, volat
       for (int kk = 0; kk < kT / 16; ++kk)
         umma_f16_ts(tAcc1, tY + acol(kk) + 16, sdesc_sw128(tileA + kk * 2048, kSub, 1024), IDACC,
                     (t > 0 || kk > 0) ? 1u : 0u);
-      umma_commit(&bars->ring_empty[st][0]);
+      umma_commit(&bars->ring_empty[t % NSTA][0]);
 #pragma unroll
       for (int kk = 0; kk < kT / 16; ++kk)
         umma_f16_ts(tAcc0, tY + acol(kk), sdesc_sw128(tileB + kk * 2048, kSub, 1024), IDACC,
                     (t > 0 || kk > 0) ? 1u : 0u);
-      umma_commit(&bars->ring_empty[st][1]);
+      umma_commit(&bars->ring_empty[t % NSTB][1]);
     } else {
 #pragma unroll
       for (int kk = 0; kk < kT / 16; ++kk) {
@@ -234,11 +247,12 @@ __device__ void bwd_mma(uint8_t* sm, BwdBars* bars, uint32_t tbase, int n, volat
         umma_f16_ts(tAcc0, tY + acol(kk), b, IDACC, (t > 0 || kk > 0) ? 1u : 0u);
         umma_f16_ts(tAcc0, tY + acol(kk) + 16, b, IDACC, 1u);
       }
-      umma_commit(&bars->ring_empty[st][0]);
+      umma_commit(&bars->ring_empty[t % NSTA][0]);
     }
   };
   auto ring_wait = [&](int t, int o) -> bool {
-    return mbar_wait(&bars->ring_full[t % NST][o], (t / NST) & 1, ab, err, 13);
+    const int nst = o ? NSTB : NSTA;
+    return mbar_wait(&bars->ring_full[t % nst][o], (t / nst) & 1, ab, err, 13);
   };
   bool ok = mbar_wait(&bars->fix_full, 0, ab, err, 12) && ring_wait(0, 0);
   if (ok) {
@@ -301,7 +315,7 @@ __device__ __forceinline__ void p_chunk_t(uint32_t (&s)[32], const float* nl2, f
 // dS^T = P^T o (dP^T - delta) for 32 columns; P^T and dS^T as fp16 pairs.
 // ndl holds -delta of the 32 query columns.
 __device__ __forceinline__ void ds_chunk_t(const uint32_t (&p)[32], const uint32_t (&dp)[32], const float* ndl,
-                                           uint32_t (&pk)[16], uint32_t (&dk)[16], __half2& hm) {
+                                           uint32_t (&pk)[16], uint32_t (&dk)[16]) {
 #pragma unroll
   for (int e = 0; e < 32; e += 4) {
     const float4 b = *reinterpret_cast<const float4*>(ndl + e);
@@ -310,7 +324,6 @@ __device__ __forceinline__ void ds_chunk_t(const uint32_t (&p)[32], const uint32
       const float2 pp = f2(p[e + u], p[e + u + 1]);
       const float2 d = __fadd2_rn(f2(dp[e + u], dp[e + u + 1]), u ? make_float2(b.z, b.w) : make_float2(b.x, b.y));
       const __half2 ds = __float22half2_rn(__fmul2_rn(pp, d));
-      hm = __hmax2_nan(hm, __habs2(ds));
       pk[(e + u) >> 1] = h2_bits(__float22half2_rn(pp));
       dk[(e + u) >> 1] = h2_bits(ds);
     }
@@ -337,13 +350,12 @@ __device__ __forceinline__ void p_chunk(uint32_t (&s)[32], float nl2, float c2, 
 
 // dS = P o (dP - delta) for 32 columns, as an fp16 head and an fp16 remainder.
 __device__ __forceinline__ void ds_chunk(const uint32_t (&p)[32], const uint32_t (&dp)[32], float ndl,
-                                         uint32_t (&hi)[16], uint32_t (&lo)[16], __half2& hm) {
+                                         uint32_t (&hi)[16], uint32_t (&lo)[16]) {
   const float2 nd = make_float2(ndl, ndl), m1 = make_float2(-1.f, -1.f);
 #pragma unroll
   for (int e = 0; e < 32; e += 2) {
     const float2 ds = __fmul2_rn(f2(p[e], p[e + 1]), __fadd2_rn(f2(dp[e], dp[e + 1]), nd));
     const __half2 h = __float22half2_rn(ds);
-    hm = __hmax2_nan(hm, __habs2(h));
     const float2 r = __ffma2_rn(__half22float2(h), m1, ds);     // ds - hi, exact
     hi[e >> 1] = h2_bits(h);
     lo[e >> 1] = h2_bits(__float22half2_rn(r));
@@ -358,9 +370,9 @@ k_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CU
               const float* __restrict__ lse, const float* __restrict__ delta, float* __restrict__ dks,
               float* __restrict__ dvs, int S, float c2, float scale, int* err) {
   using Lay = BwdLayout<D, false>;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  BwdBars* bars = reinterpret_cast<BwdBars*>(sm + Lay::BAR);
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  BwdBars* bars = reinterpret_cast<BwdBars*>(smem_raw);
+  uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + Lay::HEAD + 1023) & ~(uintptr_t)1023);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int ntiles = gridDim.x;
   const int j = blockIdx.x;            // key tile; small j has the most query tiles
@@ -382,7 +394,7 @@ k_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CU
     const uint32_t la = (uint32_t)(quarter * 32) << 16;
     const uint32_t cX = tbase + la + 64 * half, cY = cX + kColY;
     const int key = j * kT + m;
-    float* vec = reinterpret_cast<float*>(sm + Lay::VEC);   // [2][2][128]: -lse2, -delta
+    float* vec = reinterpret_cast<float*>(smem_raw + 256);  // [2][128]: -lse2, -delta
     // this thread's share of a query tile's -lse2 / -delta (thread hid of the
     // half: column 64*half + (hid & 63)), fetched one tile ahead
     const int hid = ctid & 127;
@@ -393,15 +405,15 @@ k_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CU
       return q < S ? vsrc[q] : 0.f;
     };
     float nxt = fetch(j);
-    __half2 hm = __float2half2_rn(0.f);
     bool ok = true;
-    // every compute thread runs all n iterations (and their named barrier), also
-    // after a wind-down, so no warp can be left waiting at the barrier
+    // this half's 64 query columns
+    float* nl2 = vec + 64 * half;
+    float* ndl = nl2 + 128;
+    // every compute thread runs all n iterations (and their named barriers),
+    // also after a wind-down, so no warp can be left waiting at a barrier
     for (int t = 0; t < n; ++t) {
       const int i = j + t;
-      // this half's 64 query columns, double-buffered by tile parity
-      float* nl2 = vec + (t & 1) * 256 + 64 * half;
-      float* ndl = nl2 + 128;
+      named_bar_sync(1 + half, kComputeThreads / 2);   // the half is done with tile t-1's vector
       (hid < 64 ? nl2 : ndl)[hid & 63] = nxt * vmul;
       named_bar_sync(1 + half, kComputeThreads / 2);
       if (t + 1 < n) nxt = fetch(i + 1);
@@ -435,18 +447,16 @@ k_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CU
       tmem_ld32(cY + 32, d1);
       tmem_wait_ld_regs(d0);
       reg_fence32(d1);
-      ds_chunk_t(p0, d0, ndl, pk, dk, hm);
+      ds_chunk_t(p0, d0, ndl, pk, dk);
       tmem_st16(cY, pk);
       tmem_st16(cY + 16, dk);
-      ds_chunk_t(p1, d1, ndl + 32, pk, dk, hm);
+      ds_chunk_t(p1, d1, ndl + 32, pk, dk);
       tmem_st16(cY + 32, pk);
       tmem_st16(cY + 48, dk);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive_warp(&bars->ds_ready);
     }
-    const float dsmax = __half2float(__hmax_nan(__low2half(hm), __high2half(hm)));
-    if (!(dsmax <= kHalfMax)) report_error(err, LH_ERR_DEVICE, 101);
     if (ok && __all_sync(0xffffffffu, mbar_wait(&bars->done, 0, ab, err, 18))) {
       tc_fence_after();
       float* ddv = dvs + ((size_t)bh * S + key) * D;
@@ -460,6 +470,10 @@ k_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CU
         tmem_ld32(tbase + la + kColAcc + D + 32 * c, b);
         tmem_wait_ld();
         if (key < S) {
+          bool fin = true;
+#pragma unroll
+          for (int e = 0; e < 32; ++e) fin &= fabsf(__uint_as_float(b[e])) < INFINITY;
+          if (!fin) report_error(err, LH_ERR_DEVICE, 101);
 #pragma unroll
           for (int e = 0; e < 32; e += 4) {
             *reinterpret_cast<float4*>(ddv + 32 * c + e) =
@@ -484,9 +498,9 @@ k_bwd_dq_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUte
             const float* __restrict__ lse, const float* __restrict__ delta, float* __restrict__ dqs,
             int S, float c2, float scale, int* err) {
   using Lay = BwdLayout<D, true>;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  BwdBars* bars = reinterpret_cast<BwdBars*>(sm + Lay::BAR);
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  BwdBars* bars = reinterpret_cast<BwdBars*>(smem_raw);
+  uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + Lay::HEAD + 1023) & ~(uintptr_t)1023);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int ntiles = gridDim.x;
   const int i = ntiles - 1 - (int)blockIdx.x;     // query tile; late tiles have the most key tiles
@@ -528,7 +542,6 @@ k_bwd_dq_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUte
       tc_fence_before();
       mbar_arrive_warp(&bars->fix_full);
     }
-    __half2 hm = __float2half2_rn(0.f);
     bool ok = true;
     for (int jj = 0; jj < n; ++jj) {
       if (!__all_sync(0xffffffffu, mbar_wait(&bars->x_full, jj & 1, ab, err, 19))) { ok = false; break; }
@@ -556,18 +569,16 @@ k_bwd_dq_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUte
       tmem_ld32(cY + 32, d1);
       tmem_wait_ld_regs(d0);
       reg_fence32(d1);
-      ds_chunk(p0, d0, ndl, hi, lo, hm);
+      ds_chunk(p0, d0, ndl, hi, lo);
       tmem_st16(cY, hi);
       tmem_st16(cY + 16, lo);
-      ds_chunk(p1, d1, ndl, hi, lo, hm);
+      ds_chunk(p1, d1, ndl, hi, lo);
       tmem_st16(cY + 32, hi);
       tmem_st16(cY + 48, lo);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive_warp(&bars->ds_ready);
     }
-    const float dsmax = __half2float(__hmax_nan(__low2half(hm), __high2half(hm)));
-    if (!(dsmax <= kHalfMax)) report_error(err, LH_ERR_DEVICE, 101);
     if (ok && __all_sync(0xffffffffu, mbar_wait(&bars->done, 0, ab, err, 21))) {
       tc_fence_after();
       float* dst = dqs + ((size_t)bh * S + q) * D;
@@ -577,6 +588,10 @@ k_bwd_dq_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUte
         tmem_ld32(tbase + la + kColAcc + 32 * c, a);
         tmem_wait_ld();
         if (q < S) {
+          bool fin = true;
+#pragma unroll
+          for (int e = 0; e < 32; ++e) fin &= fabsf(__uint_as_float(a[e])) < INFINITY;
+          if (!fin) report_error(err, LH_ERR_DEVICE, 101);
 #pragma unroll
           for (int e = 0; e < 32; e += 4)
             *reinterpret_cast<float4*>(dst + 32 * c + e) =
