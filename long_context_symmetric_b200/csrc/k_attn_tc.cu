@@ -9,24 +9,30 @@
 // keep the output within the stated tolerance (with bf16 P, errors of 1.5e-2
 // in the attention output were measured on scaled inputs).
 //
-// One CTA per (b, h, 128-row query tile); heavy (late) tiles are scheduled
-// first. Warp roles (192 threads):
-//   warp 0    TMA producer: the Q tile once, then K/V tiles of 128 rows into a
-//             2-stage ring (128-byte swizzle, no multicast).
-//   warp 1    allocates 512 TMEM columns; lane 0 issues every tcgen05.mma:
-//             S_j = Q K_j^T into one of two TMEM score buffers, then
-//             O += P_{j-1} V_{j-1} into the TMEM output accumulator, so the
-//             tensor core computes S_{j+1} while the softmax warps work on S_j.
-//   warps 2-5 softmax, one thread per query row (= TMEM lane): scores from
-//             TMEM, causal mask on the diagonal tile, online softmax in the
-//             exp2 domain with a lazily updated running max (the output is
-//             rescaled in TMEM only when the max grows by more than 2^8); P is
-//             split into an fp16 head (to shared memory, in the MMA's K-major
-//             swizzled layout) and an fp16 remainder (to spare TMEM columns),
-//             and O += P_hi V + P_lo V, so O carries P to about 2^-22 instead
-//             of fp16's 2^-12 (the backward's delta = <dO, O> needs that: at
-//             512K context with outlier tokens the fp16-only O put delta off
-//             by 0.07); finally O / l and lse are written.
+// One CTA per (b, h, pair of 128-row query tiles A = 2m, B = 2m+1); heavy
+// (late) pairs are scheduled first. Warp roles (320 threads):
+//   warp 0    TMA producer: Q_A and Q_B once, then K and V tiles of 128 rows,
+//             each through its own 2-stage ring (128-byte swizzle, no
+//             multicast): K_j is released once both score MMAs have read it.
+//   warp 1    allocates all 512 TMEM columns (S_A, O_A, S_B, O_B, 128 each);
+//             lane 0 issues every tcgen05.mma, per key tile j:
+//               PV_A(j), S_A(j+1), PV_B(j), S_B(j+1)
+//             so one tile's softmax runs while the tensor core works on the
+//             other tile (about 1.5 tiles of MMA time for 1 tile of softmax).
+//   warps 2-5 softmax of tile A, warps 6-9 of tile B; one thread per query row
+//             (= TMEM lane): scores from TMEM, causal mask on the diagonal
+//             tile, online softmax in the exp2 domain with a lazily updated
+//             running max (O is rescaled in TMEM only when the max grows by
+//             more than 2^8); P is split into an fp16 head and an fp16
+//             remainder written into the score columns (each 32-column chunk
+//             holds its own 16 head and 16 remainder columns), and
+//             O += P_hi V + P_lo V as TMEM-operand MMAs, so O carries P to
+//             about 2^-22 instead of fp16's 2^-12 (the backward's
+//             delta = <dO, O> needs that: at 512K context with outlier tokens
+//             the fp16-only O put delta off by 0.07); finally O / l and lse.
+// Reuse of TMEM columns is ordered by the MMA stream: S_t(j+1) is issued after
+// PV_t(j), and tcgen05.mma ops issued by one thread execute in order, so once
+// S_t(j+1) is complete, PV_t(j) has finished reading P_t(j) and O_t is current.
 // Every mbarrier wait is bounded (tc::mbar_wait): on timeout the kernel records
 // LH_ERR_TIMEOUT, drains its outstanding copies and MMAs, frees TMEM, returns.
 #include <cudaTypedefs.h>
@@ -42,32 +48,36 @@ using namespace tc;
 
 constexpr int kBM = 128;       // query rows per tile
 constexpr int kBN = 128;       // key rows per tile
-constexpr int kSub = 128 * 64 * 2;   // one 128-row x 64-column bf16 swizzle tile (16 KB)
-constexpr int kStages = 2;
+constexpr int kSub = 128 * 64 * 2;   // one 128-row x 64-column 16-bit swizzle tile (16 KB)
 constexpr float kLn2f = 0.6931471805599453f;
-constexpr uint32_t kPlo = 384;       // TMEM columns of the fp16 remainder of P (64 columns)
+constexpr int kFwdThreads = 320;
 
+// Barriers first, then the swizzled tiles from the next 1024-byte boundary.
 template <int D>
 struct FwdLayout {
   static constexpr int SUB = D / 64;
-  static constexpr int Q = 0;
-  static constexpr int K = Q + SUB * kSub;
-  static constexpr int V = K + kStages * SUB * kSub;
-  static constexpr int P = V + kStages * SUB * kSub;
-  static constexpr int BAR = P + 2 * kSub;
-  // barriers + alignment slack; at least 120 KB so that one CTA (and its 512
-  // TMEM columns) occupies an SM
-  static constexpr int BYTES = (BAR + 256 + 1024) > 120 * 1024 ? (BAR + 256 + 1024) : 120 * 1024;
+  static constexpr int OPB = SUB * kSub;   // one 128-row operand tile
+  static constexpr int Q = 0;              // Q_A, Q_B
+  static constexpr int K = Q + 2 * OPB;    // 2 stages
+  static constexpr int V = K + 2 * OPB;    // 2 stages
+  static constexpr int TILES = V + 2 * OPB;
+  static constexpr int HEAD = 256;
+  static constexpr int BYTES = HEAD + 1024 + TILES;
+  static_assert(BYTES <= 227 * 1024, "shared memory");
 };
 
+// Per query tile t (0 = A, 1 = B): s_full (score MMA done), p_full (one
+// arrival per softmax warp), o_done (P V MMA done).
 struct FwdBars {
-  uint64_t q_full, kv_full[kStages], kv_empty[kStages], s_full[2], s_free[2], p_full, o_done, drain;
+  uint64_t q_full, k_full[2], k_empty[2], v_full[2], v_empty[2];
+  uint64_t s_full[2], p_full[2], o_done[2], drain;
   uint32_t tmem_base;
   Abort abort;
 };
+static_assert(sizeof(FwdBars) <= 256, "barrier block");
 
 template <int D>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(kFwdThreads, 1)
 k_attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
               const __grid_constant__ CUtensorMap tv, float* __restrict__ os, float* __restrict__ lse,
               int S, float c2, int* err) {
@@ -75,29 +85,31 @@ k_attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CU
   constexpr int SUB = Lay::SUB;
   constexpr uint32_t IDS = idesc_f16(kBM, kBN, false);    // S = Q K^T, both K-major
   constexpr uint32_t IDO = idesc_f16(kBM, D, true);       // O = P V, V MN-major
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  FwdBars* bars = reinterpret_cast<FwdBars*>(sm + Lay::BAR);
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  FwdBars* bars = reinterpret_cast<FwdBars*>(smem_raw);
+  uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + Lay::HEAD + 1023) & ~(uintptr_t)1023);
   const uint32_t sbase = smem_u32(sm);
 
-  const int ntiles = gridDim.x;
-  const int it = ntiles - 1 - (int)blockIdx.x;
+  const int ntiles = (S + kBM - 1) / kBM;
+  const int mp = (int)gridDim.x - 1 - (int)blockIdx.x;
+  const int itA = 2 * mp, itB = 2 * mp + 1;
+  const bool hasB = itB < ntiles;
+  const int nkvA = itA + 1, nkvB = hasB ? itB + 1 : 0;
+  const int nkv = hasB ? nkvB : nkvA;
   const int bh = blockIdx.y;
-  const int nkv = it + 1;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->q_full, 1);
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(&bars->kv_full[s], 1);
-      mbar_init(&bars->kv_empty[s], 1);
-    }
     for (int s = 0; s < 2; ++s) {
+      mbar_init(&bars->k_full[s], 1);
+      mbar_init(&bars->k_empty[s], 1);
+      mbar_init(&bars->v_full[s], 1);
+      mbar_init(&bars->v_empty[s], 1);
       mbar_init(&bars->s_full[s], 1);
-      mbar_init(&bars->s_free[s], 4);      // one arrival per softmax warp
+      mbar_init(&bars->p_full[s], 4);     // one arrival per softmax warp of the tile
+      mbar_init(&bars->o_done[s], 1);
     }
-    mbar_init(&bars->p_full, 4);
-    mbar_init(&bars->o_done, 1);
     mbar_init(&bars->drain, 1);
     bars->abort.flag = 0;
     fence_mbar_init();
@@ -116,197 +128,218 @@ k_attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CU
   if (warp == 0) {
     if (lane == 0) {
       // ---------------- producer
-      int issued = 0;
-      mbar_expect_tx(&bars->q_full, SUB * kSub);
-      for (int c = 0; c < SUB; ++c)
-        tma_load_3d(sm + Lay::Q + c * kSub, &tq, &bars->q_full, 64 * c, it * kBM, bh);
+      int ik = 0, iv = 0;            // K / V tiles issued
+      mbar_expect_tx(&bars->q_full, (hasB ? 2 : 1) * Lay::OPB);
+      for (int c = 0; c < SUB; ++c) {
+        tma_load_3d(sm + Lay::Q + c * kSub, &tq, &bars->q_full, 64 * c, itA * kBM, bh);
+        if (hasB) tma_load_3d(sm + Lay::Q + Lay::OPB + c * kSub, &tq, &bars->q_full, 64 * c, itB * kBM, bh);
+      }
       for (int j = 0; j < nkv; ++j) {
-        const int st = j % kStages;
-        if (j >= kStages && !mbar_wait(&bars->kv_empty[st], ((j / kStages) - 1) & 1, ab, err, 1)) break;
-        mbar_expect_tx(&bars->kv_full[st], 2 * SUB * kSub);
+        const int st = j & 1;
+        if (j >= 2 && !mbar_wait(&bars->k_empty[st], ((j >> 1) - 1) & 1, ab, err, 1)) break;
+        mbar_expect_tx(&bars->k_full[st], Lay::OPB);
         for (int c = 0; c < SUB; ++c)
-          tma_load_3d(sm + Lay::K + (st * SUB + c) * kSub, &tk, &bars->kv_full[st], 64 * c, j * kBN, bh);
+          tma_load_3d(sm + Lay::K + st * Lay::OPB + c * kSub, &tk, &bars->k_full[st], 64 * c, j * kBN, bh);
+        ik = j + 1;
+        if (j >= 2 && !mbar_wait(&bars->v_empty[st], ((j >> 1) - 1) & 1, ab, err, 1)) break;
+        mbar_expect_tx(&bars->v_full[st], Lay::OPB);
         for (int c = 0; c < SUB; ++c)
-          tma_load_3d(sm + Lay::V + (st * SUB + c) * kSub, &tv, &bars->kv_full[st], 64 * c, j * kBN, bh);
-        issued = j + 1;
+          tma_load_3d(sm + Lay::V + st * Lay::OPB + c * kSub, &tv, &bars->v_full[st], 64 * c, j * kBN, bh);
+        iv = j + 1;
       }
       if (ab->flag) {
         // wind-down: let the copies still in flight land before the CTA exits
         Abort none{0};
         mbar_wait(&bars->q_full, 0, &none, nullptr, 0);
-        for (int j = issued - kStages < 0 ? 0 : issued - kStages; j < issued; ++j)
-          mbar_wait(&bars->kv_full[j % kStages], (j / kStages) & 1, &none, nullptr, 0);
+        for (int j = ik - 2 < 0 ? 0 : ik - 2; j < ik; ++j)
+          mbar_wait(&bars->k_full[j & 1], (j >> 1) & 1, &none, nullptr, 0);
+        for (int j = iv - 2 < 0 ? 0 : iv - 2; j < iv; ++j)
+          mbar_wait(&bars->v_full[j & 1], (j >> 1) & 1, &none, nullptr, 0);
       }
     }
   } else if (warp == 1) {
     if (lane == 0) {
       // ---------------- MMA issuer
-      auto issue_pv = [&](int jj) -> bool {
-        if (!mbar_wait(&bars->p_full, jj & 1, ab, err, 5)) return false;
-        tc_fence_after();
-        const int st = jj % kStages;
-        const uint32_t dO = tbase + 256;
-#pragma unroll
-        for (int kk = 0; kk < kBN / 16; ++kk) {
-          const uint64_t a = sdesc_sw128(sbase + Lay::P + (kk >> 2) * kSub + (kk & 3) * 32, 16, 1024);
-          const uint64_t b = sdesc_sw128(sbase + Lay::V + st * SUB * kSub + kk * 2048, kSub, 1024);
-          umma_f16(dO, a, b, IDO, (jj > 0 || kk > 0) ? 1u : 0u);
-        }
-#pragma unroll
-        for (int kk = 0; kk < kBN / 16; ++kk) {
-          const uint64_t b = sdesc_sw128(sbase + Lay::V + st * SUB * kSub + kk * 2048, kSub, 1024);
-          umma_f16_ts(dO, tbase + kPlo + 8 * kk, b, IDO, 1u);
-        }
-        umma_commit(&bars->o_done);
-        umma_commit(&bars->kv_empty[st]);
-        return true;
-      };
-      bool ok = mbar_wait(&bars->q_full, 0, ab, err, 2);
-      for (int j = 0; ok && j < nkv; ++j) {
-        const int st = j % kStages, sb = j & 1;
-        if (!mbar_wait(&bars->kv_full[st], (j / kStages) & 1, ab, err, 3)) { ok = false; break; }
-        if (j >= 2 && !mbar_wait(&bars->s_free[sb], ((j >> 1) - 1) & 1, ab, err, 4)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t dS = tbase + sb * 128;
+      auto issue_s = [&](int t, int j) {       // S_t = Q_t K_j^T
+        const uint32_t kt = sbase + Lay::K + (j & 1) * Lay::OPB;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t koff = (kk >> 2) * kSub + (kk & 3) * 32;
-          const uint64_t a = sdesc_sw128(sbase + Lay::Q + koff, 16, 1024);
-          const uint64_t b = sdesc_sw128(sbase + Lay::K + st * SUB * kSub + koff, 16, 1024);
-          umma_f16(dS, a, b, IDS, kk > 0 ? 1u : 0u);
+          umma_f16(tbase + 256 * t, sdesc_sw128(sbase + Lay::Q + t * Lay::OPB + koff, 16, 1024),
+                   sdesc_sw128(kt + koff, 16, 1024), IDS, kk > 0 ? 1u : 0u);
         }
-        umma_commit(&bars->s_full[sb]);
-        if (j >= 1 && !issue_pv(j - 1)) { ok = false; break; }
+        umma_commit(&bars->s_full[t]);
+      };
+      auto issue_pv = [&](int t, int j) {      // O_t += P_hi V_j + P_lo V_j
+        const uint32_t vt = sbase + Lay::V + (j & 1) * Lay::OPB;
+        const uint32_t tS = tbase + 256 * t, tO = tS + 128;
+#pragma unroll
+        for (int kk = 0; kk < kBN / 16; ++kk) {
+          const uint64_t b = sdesc_sw128(vt + kk * 2048, kSub, 1024);
+          const uint32_t acol = 32 * (kk >> 1) + 8 * (kk & 1);
+          umma_f16_ts(tO, tS + acol, b, IDO, (j > 0 || kk > 0) ? 1u : 0u);
+          umma_f16_ts(tO, tS + acol + 16, b, IDO, 1u);
+        }
+        umma_commit(&bars->o_done[t]);
+      };
+      bool ok = mbar_wait(&bars->q_full, 0, ab, err, 2) && mbar_wait(&bars->k_full[0], 0, ab, err, 3);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0, 0);
+        if (hasB) issue_s(1, 0);
+        umma_commit(&bars->k_empty[0]);
       }
-      if (ok) issue_pv(nkv - 1);
+      for (int j = 0; ok && j < nkv; ++j) {
+        if (!mbar_wait(&bars->v_full[j & 1], (j >> 1) & 1, ab, err, 4)) { ok = false; break; }
+        bool kwait = false;
+        auto k_next = [&]() -> bool {
+          if (kwait) return true;
+          kwait = true;
+          return mbar_wait(&bars->k_full[(j + 1) & 1], ((j + 1) >> 1) & 1, ab, err, 3);
+        };
+        if (j < nkvA) {
+          if (!mbar_wait(&bars->p_full[0], j & 1, ab, err, 5)) { ok = false; break; }
+          tc_fence_after();
+          issue_pv(0, j);
+          if (j + 1 < nkvA) {
+            if (!k_next()) { ok = false; break; }
+            tc_fence_after();
+            issue_s(0, j + 1);
+          }
+        }
+        if (hasB) {
+          if (!mbar_wait(&bars->p_full[1], j & 1, ab, err, 5)) { ok = false; break; }
+          tc_fence_after();
+          issue_pv(1, j);
+          if (j + 1 < nkvB) {
+            if (!k_next()) { ok = false; break; }
+            tc_fence_after();
+            issue_s(1, j + 1);
+          }
+        }
+        umma_commit(&bars->v_empty[j & 1]);
+        if (j + 1 < nkv) umma_commit(&bars->k_empty[(j + 1) & 1]);
+      }
       // wait until every MMA issued here has finished before TMEM is released
       umma_commit(&bars->drain);
       Abort none{0};
       mbar_wait(&bars->drain, 0, &none, nullptr, 0);
     }
   } else {
-    // ---------------- softmax: one thread per query row / TMEM lane
-    const int quarter = warp & 3;
-    const int r = quarter * 32 + lane;
-    const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
-    const int q_row = it * kBM + r;
-    float m_run = 0.f, l_run = 0.f;
-    bool ok = true;
-    uint8_t* P0 = sm + Lay::P;
-    for (int j = 0; j < nkv; ++j) {
-      const int sb = j & 1;
-      if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full[sb], (j >> 1) & 1, ab, err, 6))) { ok = false; break; }
-      tc_fence_after();
-      uint32_t s[128];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t (&chunk)[32] = *reinterpret_cast<uint32_t(*)[32]>(&s[32 * c]);
-        tmem_ld32(tbase + lane_addr + sb * 128 + 32 * c, chunk);
-      }
-      tmem_wait_ld();
-      tc_fence_before();
-      mbar_arrive_warp(&bars->s_free[sb]);
-      // causal mask on the diagonal tile; the running max is taken on the raw
-      // scores (c2 > 0, and rounding is monotone, so max(s) c2 = max(s c2))
-      if (j == it) {
-        const int lim = min(r, S - 1 - j * kBN);   // last valid column of this row
-#pragma unroll
-        for (int c = 0; c < 128; ++c)
-          if (c > lim) s[c] = __float_as_uint(-INFINITY);
-      }
-      float mq[4];
-#pragma unroll
-      for (int g = 0; g < 4; ++g) {
-        mq[g] = __uint_as_float(s[32 * g]);
-#pragma unroll
-        for (int c = 1; c < 31; c += 2)
-          mq[g] = fmax3(mq[g], __uint_as_float(s[32 * g + c]), __uint_as_float(s[32 * g + c + 1]));
-        mq[g] = fmaxf(mq[g], __uint_as_float(s[32 * g + 31]));
-      }
-      const float mx = fmax3(fmaxf(mq[0], mq[1]), mq[2], mq[3]) * c2;
-      float m_new = m_run, alpha = 1.f;
-      if (j == 0) {
-        m_new = mx;
-      } else if (mx > m_run + 8.f) {
-        m_new = mx;
-        alpha = ex2(m_run - m_new);
-      }
-      // P = 2^(s c2 - m), two columns per packed FMA; four partial sums
-      const float2 cc = make_float2(c2, c2), nm = make_float2(-m_new, -m_new);
-      float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-#pragma unroll
-      for (int c = 0; c < 128; c += 2) {
-        const float2 x = __ffma2_rn(make_float2(__uint_as_float(s[c]), __uint_as_float(s[c + 1])), cc, nm);
-        const float2 pc = make_float2(ex2(x.x), ex2(x.y));
-        acc[(c >> 1) & 3] = __fadd2_rn(acc[(c >> 1) & 3], pc);
-        s[c] = __float_as_uint(pc.x);
-        s[c + 1] = __float_as_uint(pc.y);
-      }
-      const float2 a01 = __fadd2_rn(acc[0], acc[1]), a23 = __fadd2_rn(acc[2], acc[3]);
-      const float sum = (a01.x + a23.x) + (a01.y + a23.y);
-      l_run = l_run * alpha + sum;
-      m_run = m_new;
-      if (j >= 1) {
-        // PV_{j-1} done: the P buffer is free and O is current
-        if (!__all_sync(0xffffffffu, mbar_wait(&bars->o_done, (j - 1) & 1, ab, err, 7))) { ok = false; break; }
+    // ---------------- softmax: one thread per query row / TMEM lane of tile t
+    const int t = (warp - 2) >> 2;
+    const int it = t ? itB : itA;
+    if (t == 0 || hasB) {
+      const int quarter = warp & 3;
+      const int r = quarter * 32 + lane;
+      const uint32_t la = (uint32_t)(quarter * 32) << 16;
+      const uint32_t cS = tbase + la + 256 * t, cO = cS + 128;
+      const int q_row = it * kBM + r;
+      const int nk = it + 1;
+      float m_run = 0.f, l_run = 0.f;
+      bool ok = true;
+      for (int j = 0; j < nk; ++j) {
+        if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full[t], j & 1, ab, err, 6))) { ok = false; break; }
         tc_fence_after();
+        uint32_t s[128];
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          tmem_ld32(cS + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&s[32 * c]));
+        tmem_wait_ld_regs(*reinterpret_cast<uint32_t(*)[32]>(&s[0]));
+        reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&s[32]));
+        reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&s[64]));
+        reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&s[96]));
+        // causal mask on the diagonal tile; the running max is taken on the raw
+        // scores (c2 > 0, and rounding is monotone, so max(s) c2 = max(s c2))
+        if (j == it) {
+          const int lim = min(r, S - 1 - j * kBN);   // last valid column of this row
+#pragma unroll
+          for (int c = 0; c < 128; ++c)
+            if (c > lim) s[c] = __float_as_uint(-INFINITY);
+        }
+        float mq[4];
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          mq[g] = __uint_as_float(s[32 * g]);
+#pragma unroll
+          for (int c = 1; c < 31; c += 2)
+            mq[g] = fmax3(mq[g], __uint_as_float(s[32 * g + c]), __uint_as_float(s[32 * g + c + 1]));
+          mq[g] = fmaxf(mq[g], __uint_as_float(s[32 * g + 31]));
+        }
+        const float mx = fmax3(fmaxf(mq[0], mq[1]), mq[2], mq[3]) * c2;
+        float m_new = m_run, alpha = 1.f;
+        if (j == 0) {
+          m_new = mx;
+        } else if (mx > m_run + 8.f) {
+          m_new = mx;
+          alpha = ex2(m_run - m_new);
+        }
         if (__any_sync(0xffffffffu, alpha != 1.f)) {
+          // O_t is current: PV_t(j-1) finished before S_t(j) (same MMA stream)
 #pragma unroll 1
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t o[32];
-            tmem_ld32(tbase + lane_addr + 256 + 32 * c, o);
-            tmem_wait_ld();
+          for (int c = 0; c < D / 16; ++c) {
+            uint32_t o[16];
+            tmem_ld16(cO + 16 * c, o);
+            tmem_wait_ld_regs16(o);
 #pragma unroll
-            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-            tmem_st32(tbase + lane_addr + 256 + 32 * c, o);
+            for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+            tmem_st16(cO + 16 * c, o);
           }
-          tmem_wait_st();
         }
+        // P = 2^(s c2 - m): head and remainder of each 32-column chunk into
+        // that chunk's own score columns (+0..15 head, +16..31 remainder)
+        const float2 cc = make_float2(c2, c2), nm = make_float2(-m_new, -m_new);
+        const float2 m1 = make_float2(-1.f, -1.f);
+        float2 acc[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+#pragma unroll
+          for (int g = 0; g < 4; ++g) {          // 8 columns: 4 head and 4 remainder pairs
+            uint32_t hi[4], lo[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const int e = 4 * g + u;
+              const float2 x = __ffma2_rn(
+                  make_float2(__uint_as_float(s[32 * c + 2 * e]), __uint_as_float(s[32 * c + 2 * e + 1])), cc, nm);
+              const float2 pp = make_float2(ex2(x.x), ex2(x.y));
+              acc[u & 1] = __fadd2_rn(acc[u & 1], pp);
+              const __half2 h = __float22half2_rn(pp);
+              const __half2 l = __float22half2_rn(__ffma2_rn(__half22float2(h), m1, pp));   // p - hi, exact
+              hi[u] = *reinterpret_cast<const uint32_t*>(&h);
+              lo[u] = *reinterpret_cast<const uint32_t*>(&l);
+            }
+            tmem_st4(cS + 32 * c + 4 * g, hi[0], hi[1], hi[2], hi[3]);
+            tmem_st4(cS + 32 * c + 16 + 4 * g, lo[0], lo[1], lo[2], lo[3]);
+          }
+        }
+        const float2 a01 = __fadd2_rn(acc[0], acc[1]);
+        l_run = l_run * alpha + (a01.x + a01.y);
+        m_run = m_new;
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive_warp(&bars->p_full[t]);
       }
-      // head fp16(P) to shared memory, remainder P - fp16(P) to TMEM (two per column)
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t hi[16], lo[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const float2 pp = make_float2(__uint_as_float(s[32 * c + 2 * e]), __uint_as_float(s[32 * c + 2 * e + 1]));
-          const __half2 h = __float22half2_rn(pp);
-          const float2 rem = __ffma2_rn(__half22float2(h), make_float2(-1.f, -1.f), pp);   // p - hi, exact
-          const __half2 l = __float22half2_rn(rem);
-          hi[e] = *reinterpret_cast<const uint32_t*>(&h);
-          lo[e] = *reinterpret_cast<const uint32_t*>(&l);
-        }
-#pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
-          const int c16 = 4 * c + q4;       // 16-byte chunk (8 columns) of the 128-column row
-          *reinterpret_cast<uint4*>(P0 + (c16 >> 3) * kSub + sw128_off(r, c16 & 7)) =
-              make_uint4(hi[4 * q4], hi[4 * q4 + 1], hi[4 * q4 + 2], hi[4 * q4 + 3]);
-        }
-        tmem_st16(tbase + lane_addr + kPlo + 16 * c, lo);
-      }
-      tmem_wait_st();
-      fence_proxy_async_smem();
-      tc_fence_before();
-      mbar_arrive_warp(&bars->p_full);
-    }
-    if (ok && __all_sync(0xffffffffu, mbar_wait(&bars->o_done, (nkv - 1) & 1, ab, err, 8))) {
-      tc_fence_after();
-      const float inv = 1.f / l_run;
-      float* dst = os + ((size_t)bh * S + q_row) * D;
+      // PV_t(nk-2) finished before S_t(nk-1), so o_done's phase nk-1 is the
+      // only one left: its parity identifies it
+      if (ok && __all_sync(0xffffffffu, mbar_wait(&bars->o_done[t], (nk - 1) & 1, ab, err, 8))) {
+        tc_fence_after();
+        const float inv = 1.f / l_run;
+        float* dst = os + ((size_t)bh * S + q_row) * D;
 #pragma unroll 1
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t o[32];
-        tmem_ld32(tbase + lane_addr + 256 + 32 * c, o);
-        tmem_wait_ld();
-        if (q_row < S) {
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld32(cO + 32 * c, o);
+          tmem_wait_ld_regs(o);
+          if (q_row < S) {
 #pragma unroll
-          for (int e = 0; e < 32; e += 4)
-            *reinterpret_cast<float4*>(dst + 32 * c + e) =
-                make_float4(__uint_as_float(o[e]) * inv, __uint_as_float(o[e + 1]) * inv,
-                            __uint_as_float(o[e + 2]) * inv, __uint_as_float(o[e + 3]) * inv);
+            for (int e = 0; e < 32; e += 4)
+              *reinterpret_cast<float4*>(dst + 32 * c + e) =
+                  make_float4(__uint_as_float(o[e]) * inv, __uint_as_float(o[e + 1]) * inv,
+                              __uint_as_float(o[e + 2]) * inv, __uint_as_float(o[e + 3]) * inv);
+          }
         }
+        if (q_row < S) lse[(size_t)bh * S + q_row] = (m_run + log2f(l_run)) * kLn2f;
       }
-      if (q_row < S) lse[(size_t)bh * S + q_row] = (m_run + log2f(l_run)) * kLn2f;
     }
   }
   tc_fence_before();
@@ -358,8 +391,9 @@ static cudaError_t fwd_tc_t(const Geom& g, const void* qs, const void* ks, const
   cudaError_t e = cudaFuncSetAttribute(k_attn_fwd_tc<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   const float c2 = (float)(1.4426950408889634 / sqrt((double)D));
-  dim3 grid((g.S + kBM - 1) / kBM, BH);
-  k_attn_fwd_tc<D><<<grid, 192, smem, s>>>(tq, tk, tv, os, lse, g.S, c2, err);
+  const int ntiles = (g.S + kBM - 1) / kBM;
+  dim3 grid((ntiles + 1) / 2, BH);
+  k_attn_fwd_tc<D><<<grid, kFwdThreads, smem, s>>>(tq, tk, tv, os, lse, g.S, c2, err);
   count_launch();
   return cudaGetLastError();
 }
