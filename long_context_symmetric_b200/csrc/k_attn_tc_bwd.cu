@@ -17,20 +17,23 @@
 //      X = S^T = K_j Q_i^T and Y = dP^T = V_j dO_i^T (TMEM); the compute warps
 //      form P^T and dS^T and store them as fp16 into Y's columns; then
 //      dK += dS^T Q_i and dV += P^T dO_i take their A operand from TMEM.
-//  k_bwd_dq_tc    per query tile i, over key tiles j <= i (Q_i and dO_i are
-//      held in TMEM as the A operand of X and Y):
-//      X = S = Q_i K_j^T and Y = dP = dO_i V_j^T; dS is split into an fp16 head
-//      and an fp16 remainder (dS = hi + lo to about 2^-22 relative) stored into
-//      Y's columns; dQ += hi K_j + lo K_j.
+//  k_bwd_dq_tc    per query tile i, over key tiles j <= i:
+//      X = S = Q_i K_j^T and Y = dP = dO_i V_j^T, Y in two alternating TMEM
+//      buffers; dS is split into an fp16 head and an fp16 remainder
+//      (dS = hi + lo to about 2^-22 relative) stored into Y's columns;
+//      dQ += hi K_j + lo K_j.
 // A dS whose fp16 rounding overflows (or any NaN) makes dK and dQ non-finite
 // (an infinite operand times any value, summed in fp32, stays inf or NaN), so
 // the epilogues check their fp32 results and report LH_ERR_DEVICE, detail 101.
 //
-// Pipeline (tensor core order per streamed tile t):  X(t+1), acc(t), Y(t+1).
-// The compute warps copy X(t) into registers and release it at once, so X(t+1)
-// runs while they exponentiate; they read Y(t) and write the fp16 operands of
-// acc(t) into Y's columns, so Y(t+1) follows acc(t) (tcgen05.mma ops issued by
-// one thread execute in order, which orders those reuses). All score MMAs are
+// Pipeline (tensor core order per streamed tile t): dK/dV X(t+1), acc(t),
+// Y(t+1); dQ X(t+1), Y(t+1), acc(t). The compute warps copy X(t) into
+// registers and release it at once, so X(t+1) runs while they exponentiate;
+// they read Y(t) and write the fp16 operands of acc(t) into Y's columns, so in
+// the dK/dV kernel (whose TMEM holds two accumulators) Y(t+1) follows acc(t),
+// while the dQ kernel has a second Y buffer and computes Y(t+1) during the
+// compute warps' work on tile t (tcgen05.mma ops issued by one thread execute
+// in order, which orders every reuse of a TMEM column). All score MMAs are
 // full 128 x 128 tiles: N = 64 halves run at about two thirds of the rate and
 // lose more when the compute warps use TMEM at the same time (measured).
 // Streamed tiles come through a TMA ring whose two operands have their own
@@ -51,9 +54,10 @@ using namespace tc;
 constexpr int kT = 128;              // rows per tile (both directions)
 constexpr int kSub = 128 * 64 * 2;   // 128 x 64 16-bit swizzle tile
 constexpr int kMaxStages = 3;
-// TMEM columns: X at 0, Y at 128, accumulators from 256 (dkdv: dV, then dK;
-// dq: dQ), and in the dQ kernel the fixed Q_i / dO_i (D/2 packed columns each)
-constexpr uint32_t kColY = 128, kColAcc = 256, kFixCol = 384;
+// TMEM columns: X at 0, Y at 128 (dq: Y buffers at 128 and 256), accumulators
+// from 256 (dkdv: dV, then dK) or 384 (dq: dQ)
+constexpr uint32_t kColY = 128;
+__host__ __device__ constexpr uint32_t col_acc(bool two_acc) { return two_acc ? 256u : 384u; }
 // Warp roles: 0 producer, 1 MMA issuer, 2..9 compute. Two compute warps share
 // each TMEM lane quarter (warps w and w+4), each taking 64 of a tile's 128
 // columns, so every SM sub-partition has two compute warps to interleave.
@@ -61,27 +65,22 @@ constexpr int kComputeWarps = 8;
 constexpr int kComputeThreads = 32 * kComputeWarps;
 constexpr int kThreads = 64 + kComputeThreads;
 
-__device__ __forceinline__ void named_bar_sync(int id, int n) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
-}
-
-// FIXT: the fixed operands live in TMEM (dQ kernel); otherwise (dK/dV kernel,
-// whose TMEM holds two accumulators) they are shared-memory tiles. Barriers and
-// the lse/delta vector come first, the swizzled tiles from the next 1024-byte
-// boundary (TILES bytes, offsets below relative to that boundary); BYTES covers
-// the worst-case alignment gap of the dynamic shared-memory base.
-template <int D, bool FIXT>
+// Barriers and the lse/delta vector (dkdv) come first, the swizzled tiles from
+// the next 1024-byte boundary (TILES bytes, offsets below relative to that
+// boundary); BYTES covers the worst-case alignment gap of the dynamic
+// shared-memory base.
+template <int D>
 struct BwdLayout {
   static constexpr int SUB = D / 64;
   static constexpr int OPB = SUB * kSub;                       // one 128-row operand tile
   static constexpr int NSTA = 3;                               // stages of A_t (read by X and acc)
-  static constexpr int NSTB = FIXT ? 3 : 2;                    // stages of B_t
-  static constexpr int FIX0 = 0;                               // fixed operand 0 (K_j)
-  static constexpr int FIX1 = FIX0 + (FIXT ? 0 : OPB);         // fixed operand 1 (V_j)
-  static constexpr int RA = FIX1 + (FIXT ? 0 : OPB);           // A_t stages
+  static constexpr int NSTB = 2;                               // stages of B_t
+  static constexpr int FIX0 = 0;                               // fixed operand 0 (K_j / Q_i)
+  static constexpr int FIX1 = FIX0 + OPB;                      // fixed operand 1 (V_j / dO_i)
+  static constexpr int RA = FIX1 + OPB;                        // A_t stages
   static constexpr int RB = RA + NSTA * OPB;                   // B_t stages
   static constexpr int TILES = RB + NSTB * OPB;
-  static constexpr int HEAD = 256 + (FIXT ? 0 : 2 * kT * 4);   // barriers, then -lse2 / -delta (dkdv)
+  static constexpr int HEAD = 256 + 2 * kT * 4;                // barriers, then -lse2 / -delta (dkdv)
   static constexpr int BYTES = HEAD + 1024 + TILES;
   static_assert(BYTES <= 227 * 1024, "shared memory");
 };
@@ -90,25 +89,24 @@ struct BwdLayout {
 // K_j in dq), o = 1 the operand B_t (dO_i in dkdv, V_j in dq).
 struct BwdBars {
   uint64_t fix_full, ring_full[kMaxStages][2], ring_empty[kMaxStages][2];
-  uint64_t x_full, y_full, x_free, ds_ready, done, drain;
+  uint64_t x_full, y_full[2], x_free, ds_ready, done, drain;   // y_full[b]: Y buffer b
   uint32_t tmem_base;
   Abort abort;
 };
 static_assert(sizeof(BwdBars) <= 256, "barrier block");
 
-// Shared prologue: barriers, TMEM allocation (512 columns). fix_full counts one
-// arrival (the copy of the fixed tiles) or, with FIXT, one per compute warp.
-template <bool FIXT>
+// Shared prologue: barriers, TMEM allocation (512 columns).
 __device__ __forceinline__ void bwd_setup(BwdBars* bars, int warp) {
   if (threadIdx.x == 0) {
-    mbar_init(&bars->fix_full, FIXT ? kComputeWarps : 1);
+    mbar_init(&bars->fix_full, 1);
     for (int s = 0; s < kMaxStages; ++s)
       for (int o = 0; o < 2; ++o) {
         mbar_init(&bars->ring_full[s][o], 1);
         mbar_init(&bars->ring_empty[s][o], 1);
       }
     mbar_init(&bars->x_full, 1);
-    mbar_init(&bars->y_full, 1);
+    mbar_init(&bars->y_full[0], 1);
+    mbar_init(&bars->y_full[1], 1);
     mbar_init(&bars->x_free, kComputeWarps);     // one arrival per compute warp
     mbar_init(&bars->ds_ready, kComputeWarps);
     mbar_init(&bars->done, 1);
@@ -136,20 +134,18 @@ __device__ __forceinline__ void bwd_teardown(uint32_t tbase, int warp) {
   }
 }
 
-// Producer: the two fixed tiles once (unless FIXT), then `n` streamed tiles of
-// rows (first + t) * 128 of maps ma (operand A_t) and mb (B_t).
-template <int D, bool FIXT>
+// Producer: the two fixed tiles once, then `n` streamed tiles of rows
+// (first + t) * 128 of maps ma (operand A_t) and mb (B_t).
+template <int D>
 __device__ void bwd_produce(uint8_t* sm, BwdBars* bars, const CUtensorMap* f0, const CUtensorMap* f1,
                             int frow, const CUtensorMap* ma, const CUtensorMap* mb, int first, int n,
                             int bh, volatile Abort* ab, int* err) {
-  using Lay = BwdLayout<D, FIXT>;
+  using Lay = BwdLayout<D>;
   constexpr int SUB = Lay::SUB, NSTA = Lay::NSTA, NSTB = Lay::NSTB;
-  if (!FIXT) {
-    mbar_expect_tx(&bars->fix_full, 2 * SUB * kSub);
-    for (int c = 0; c < SUB; ++c) {
-      tma_load_3d(sm + Lay::FIX0 + c * kSub, f0, &bars->fix_full, 64 * c, frow * kT, bh);
-      tma_load_3d(sm + Lay::FIX1 + c * kSub, f1, &bars->fix_full, 64 * c, frow * kT, bh);
-    }
+  mbar_expect_tx(&bars->fix_full, 2 * Lay::OPB);
+  for (int c = 0; c < SUB; ++c) {
+    tma_load_3d(sm + Lay::FIX0 + c * kSub, f0, &bars->fix_full, 64 * c, frow * kT, bh);
+    tma_load_3d(sm + Lay::FIX1 + c * kSub, f1, &bars->fix_full, 64 * c, frow * kT, bh);
   }
   int issued = 0;                        // (tile, operand) loads issued, in order
   for (int t = 0; t < n; ++t) {
@@ -172,7 +168,7 @@ __device__ void bwd_produce(uint8_t* sm, BwdBars* bars, const CUtensorMap* f0, c
   if (ab->flag) {
     // wind-down: let the copies still in flight land before the CTA exits
     Abort none{0};
-    if (!FIXT) mbar_wait(&bars->fix_full, 0, &none, nullptr, 0);
+    mbar_wait(&bars->fix_full, 0, &none, nullptr, 0);
     // the latest load into each stage of each operand
     const int na = (issued + 1) / 2, nb = issued / 2;   // tiles of A_t / B_t issued
     for (int tt = na - NSTA < 0 ? 0 : na - NSTA; tt < na; ++tt)
@@ -182,79 +178,88 @@ __device__ void bwd_produce(uint8_t* sm, BwdBars* bars, const CUtensorMap* f0, c
   }
 }
 
-// MMA issuer shared by both kernels. For streamed tile t in stage st:
-//   X(t) = F0 * A_t^T -> cols 0..127,  Y(t) = F1 * B_t^T -> cols 128..255
-//   (F0/F1: shared-memory tiles, or with FIXT the TMEM columns kFixCol..),
-//   acc(t), A operand from Y's columns (fp16 pairs; chunk c = 32 columns of
+// MMA issuer shared by both kernels. For streamed tile t:
+//   X(t) = F0 * A_t^T -> cols 0..127,  Y(t) = F1 * B_t^T -> Y buffer of t
+//   (dkdv: cols 128..255; dq: buffer t & 1 at 128 + 128 (t & 1)),
+//   acc(t), A operand from that Y buffer (fp16 pairs; chunk c = 32 columns of
 //   the tile, its first 16 packed columns hold P^T / dS_hi, the next 16 dS^T /
 //   dS_lo):
 //     dkdv (TWO_ACC): dK += dS^T A_t, then dV += P^T B_t
 //     dq:             dQ += dS_hi A_t + dS_lo A_t
-// Issue order: X(0), Y(0), then per t: X(t+1), acc(t), Y(t+1).
-template <int D, bool TWO_ACC, bool FIXT>
+// Issue order: X(0), Y(0), then per t: dkdv X(t+1), acc(t), Y(t+1);
+// dq X(t+1), Y(t+1), acc(t).
+// Run by the whole (converged) MMA warp: every lane takes the same waits and
+// branches, one elected lane issues the MMAs and commits. Shared-memory
+// descriptors are built once per operand and advanced by constant offsets
+// (the start address, in 16-byte units, sits in the low 14 bits).
+template <int D, bool TWO_ACC>
 __device__ void bwd_mma(uint8_t* sm, BwdBars* bars, uint32_t tbase, int n, volatile Abort* ab, int* err) {
-  using Lay = BwdLayout<D, FIXT>;
+  using Lay = BwdLayout<D>;
   constexpr int NSTA = Lay::NSTA, NSTB = Lay::NSTB;
   constexpr uint32_t IDX = idesc_f16(kT, kT, false);      // scores: both operands K-major
   constexpr uint32_t IDACC = idesc_f16(kT, D, true);      // accumulate: B MN-major
+  constexpr uint32_t OPB16 = Lay::OPB >> 4;
+  const bool leader = elect_one();
   const uint32_t sbase = smem_u32(sm);
-  const uint32_t tX = tbase, tY = tbase + kColY;
-  const uint32_t tAcc0 = tbase + kColAcc, tAcc1 = tbase + kColAcc + (TWO_ACC ? D : 0);
-  auto tile_a = [&](int t) -> uint32_t { return sbase + Lay::RA + (t % NSTA) * Lay::OPB; };
-  auto tile_b = [&](int t) -> uint32_t { return sbase + Lay::RB + (t % NSTB) * Lay::OPB; };
+  const uint64_t dF0 = sdesc_sw128(sbase + Lay::FIX0, 16, 1024), dF1 = sdesc_sw128(sbase + Lay::FIX1, 16, 1024);
+  const uint64_t dA = sdesc_sw128(sbase + Lay::RA, 16, 1024), dB = sdesc_sw128(sbase + Lay::RB, 16, 1024);
+  const uint64_t dAm = sdesc_sw128(sbase + Lay::RA, kSub, 1024), dBm = sdesc_sw128(sbase + Lay::RB, kSub, 1024);
+  // K slice kk of a K-major tile: 16 columns = 32 bytes within a 64-column slab
+  auto kofs = [](int kk) -> uint64_t { return (uint64_t)((kk >> 2) * (kSub >> 4) + (kk & 3) * 2); };
+  const uint32_t tX = tbase;
+  auto tY = [&](int t) -> uint32_t { return tbase + kColY + (TWO_ACC ? 0u : 128u * (t & 1)); };
+  const uint32_t tAcc0 = tbase + col_acc(TWO_ACC), tAcc1 = tAcc0 + (TWO_ACC ? D : 0);
   auto issue_x = [&](int t) {
-    const uint32_t tile = tile_a(t);
+    const uint64_t b0 = dA + (uint64_t)((t % NSTA) * OPB16);
+    if (leader) {
 #pragma unroll
-    for (int kk = 0; kk < D / 16; ++kk) {
-      const uint32_t koff = (kk >> 2) * kSub + (kk & 3) * 32;
-      const uint64_t b = sdesc_sw128(tile + koff, 16, 1024);
-      if (FIXT) umma_f16_ts(tX, tbase + kFixCol + 8 * kk, b, IDX, kk > 0 ? 1u : 0u);
-      else umma_f16(tX, sdesc_sw128(sbase + Lay::FIX0 + koff, 16, 1024), b, IDX, kk > 0 ? 1u : 0u);
+      for (int kk = 0; kk < D / 16; ++kk) umma_f16(tX, dF0 + kofs(kk), b0 + kofs(kk), IDX, kk > 0 ? 1u : 0u);
+      umma_commit(&bars->x_full);
     }
-    umma_commit(&bars->x_full);
   };
   auto issue_y = [&](int t) {
-    const uint32_t tile = tile_b(t);
+    const uint64_t b0 = dB + (uint64_t)((t % NSTB) * OPB16);
+    const uint32_t y = tY(t);
+    if (leader) {
 #pragma unroll
-    for (int kk = 0; kk < D / 16; ++kk) {
-      const uint32_t koff = (kk >> 2) * kSub + (kk & 3) * 32;
-      const uint64_t b = sdesc_sw128(tile + koff, 16, 1024);
-      if (FIXT) umma_f16_ts(tY, tbase + kFixCol + D / 2 + 8 * kk, b, IDX, kk > 0 ? 1u : 0u);
-      else umma_f16(tY, sdesc_sw128(sbase + Lay::FIX1 + koff, 16, 1024), b, IDX, kk > 0 ? 1u : 0u);
+      for (int kk = 0; kk < D / 16; ++kk) umma_f16(y, dF1 + kofs(kk), b0 + kofs(kk), IDX, kk > 0 ? 1u : 0u);
+      umma_commit(&bars->y_full[TWO_ACC ? 0 : (t & 1)]);
+      if (!TWO_ACC) umma_commit(&bars->ring_empty[t % NSTB][1]);   // dq: V_j has no other reader
     }
-    umma_commit(&bars->y_full);
-    if (!TWO_ACC) umma_commit(&bars->ring_empty[t % NSTB][1]);   // dq: V_j has no other reader
   };
   auto issue_acc = [&](int t) {
-    const uint32_t tileA = tile_a(t), tileB = tile_b(t);
-    // slice kk = 16 rows of the streamed tiles; its packed operand columns
+    // 16-row slice kk of the streamed tiles: MN-major descriptor + kk * 2048 bytes;
+    // its packed operand columns in the Y buffer at acol(kk)
+    const uint64_t bA = dAm + (uint64_t)((t % NSTA) * OPB16), bB = dBm + (uint64_t)((t % NSTB) * OPB16);
+    const uint32_t y = tY(t);
     auto acol = [](int kk) -> uint32_t { return 32 * (kk >> 1) + 8 * (kk & 1); };
+    if (!leader) return;
     if (TWO_ACC) {
 #pragma unroll
       for (int kk = 0; kk < kT / 16; ++kk)
-        umma_f16_ts(tAcc1, tY + acol(kk) + 16, sdesc_sw128(tileA + kk * 2048, kSub, 1024), IDACC,
-                    (t > 0 || kk > 0) ? 1u : 0u);
+        umma_f16_ts(tAcc1, y + acol(kk) + 16, bA + kk * 128, IDACC, (t > 0 || kk > 0) ? 1u : 0u);
       umma_commit(&bars->ring_empty[t % NSTA][0]);
 #pragma unroll
       for (int kk = 0; kk < kT / 16; ++kk)
-        umma_f16_ts(tAcc0, tY + acol(kk), sdesc_sw128(tileB + kk * 2048, kSub, 1024), IDACC,
-                    (t > 0 || kk > 0) ? 1u : 0u);
+        umma_f16_ts(tAcc0, y + acol(kk), bB + kk * 128, IDACC, (t > 0 || kk > 0) ? 1u : 0u);
       umma_commit(&bars->ring_empty[t % NSTB][1]);
     } else {
 #pragma unroll
       for (int kk = 0; kk < kT / 16; ++kk) {
-        const uint64_t b = sdesc_sw128(tileA + kk * 2048, kSub, 1024);
-        umma_f16_ts(tAcc0, tY + acol(kk), b, IDACC, (t > 0 || kk > 0) ? 1u : 0u);
-        umma_f16_ts(tAcc0, tY + acol(kk) + 16, b, IDACC, 1u);
+        umma_f16_ts(tAcc0, y + acol(kk), bA + kk * 128, IDACC, (t > 0 || kk > 0) ? 1u : 0u);
+        umma_f16_ts(tAcc0, y + acol(kk) + 16, bA + kk * 128, IDACC, 1u);
       }
       umma_commit(&bars->ring_empty[t % NSTA][0]);
     }
   };
+  auto wait = [&](uint64_t* bar, uint32_t parity, int site) -> bool {
+    return __all_sync(0xffffffffu, mbar_wait(bar, parity, ab, err, site));
+  };
   auto ring_wait = [&](int t, int o) -> bool {
     const int nst = o ? NSTB : NSTA;
-    return mbar_wait(&bars->ring_full[t % nst][o], (t / nst) & 1, ab, err, 13);
+    return wait(&bars->ring_full[t % nst][o], (t / nst) & 1, 13);
   };
-  bool ok = mbar_wait(&bars->fix_full, 0, ab, err, 12) && ring_wait(0, 0);
+  bool ok = wait(&bars->fix_full, 0, 12) && ring_wait(0, 0);
   if (ok) {
     tc_fence_after();
     issue_x(0);
@@ -263,20 +268,28 @@ __device__ void bwd_mma(uint8_t* sm, BwdBars* bars, uint32_t tbase, int n, volat
   if (ok) issue_y(0);
   for (int t = 0; ok && t < n; ++t) {
     if (t + 1 < n) {
-      if (!ring_wait(t + 1, 0) || !mbar_wait(&bars->x_free, t & 1, ab, err, 14)) { ok = false; break; }
+      if (!ring_wait(t + 1, 0) || !wait(&bars->x_free, t & 1, 14)) { ok = false; break; }
       tc_fence_after();
       issue_x(t + 1);
+      if (!TWO_ACC) {
+        // dq: Y(t+1) overwrites the buffer that acc(t-1), issued earlier, read
+        if (!ring_wait(t + 1, 1)) { ok = false; break; }
+        issue_y(t + 1);
+      }
     }
-    if (!mbar_wait(&bars->ds_ready, t & 1, ab, err, 15)) { ok = false; break; }
+    if (!wait(&bars->ds_ready, t & 1, 15)) { ok = false; break; }
     tc_fence_after();
     issue_acc(t);
-    if (t + 1 < n) {
+    if (TWO_ACC && t + 1 < n) {
       if (!ring_wait(t + 1, 1)) { ok = false; break; }
       issue_y(t + 1);
     }
   }
-  if (ok) umma_commit(&bars->done);
-  umma_commit(&bars->drain);
+  if (leader) {
+    if (ok) umma_commit(&bars->done);
+    umma_commit(&bars->drain);
+  }
+  __syncwarp();
   Abort none{0};
   mbar_wait(&bars->drain, 0, &none, nullptr, 0);
 }
@@ -369,7 +382,7 @@ k_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CU
               const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tdo,
               const float* __restrict__ lse, const float* __restrict__ delta, float* __restrict__ dks,
               float* __restrict__ dvs, int S, float c2, float scale, int* err) {
-  using Lay = BwdLayout<D, false>;
+  using Lay = BwdLayout<D>;
   extern __shared__ __align__(16) uint8_t smem_raw[];
   BwdBars* bars = reinterpret_cast<BwdBars*>(smem_raw);
   uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + Lay::HEAD + 1023) & ~(uintptr_t)1023);
@@ -378,14 +391,14 @@ k_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CU
   const int j = blockIdx.x;            // key tile; small j has the most query tiles
   const int bh = blockIdx.y;
   const int n = ntiles - j;            // query tiles i = j .. ntiles-1
-  bwd_setup<false>(bars, warp);
+  bwd_setup(bars, warp);
   const uint32_t tbase = bars->tmem_base;
   volatile Abort* ab = &bars->abort;
 
   if (warp == 0) {
-    if (lane == 0) bwd_produce<D, false>(sm, bars, &tk, &tv, j, &tq, &tdo, j, n, bh, ab, err);
+    if (lane == 0) bwd_produce<D>(sm, bars, &tk, &tv, j, &tq, &tdo, j, n, bh, ab, err);
   } else if (warp == 1) {
-    if (lane == 0) bwd_mma<D, true, false>(sm, bars, tbase, n, ab, err);
+    bwd_mma<D, true>(sm, bars, tbase, n, ab, err);
   } else {
     const int quarter = warp & 3;
     const int half = (warp - 2) >> 2;                   // which 64 of the 128 columns
@@ -437,7 +450,7 @@ k_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CU
         p_chunk_t<false>(p0, nl2, c2, 0, 0, 0);
         p_chunk_t<false>(p1, nl2 + 32, c2, 0, 0, 0);
       }
-      ok = __all_sync(0xffffffffu, mbar_wait(&bars->y_full, t & 1, ab, err, 17));
+      ok = __all_sync(0xffffffffu, mbar_wait(&bars->y_full[0], t & 1, ab, err, 17));
       if (!ok) continue;
       tc_fence_after();
       // dP^T: both 32-column chunks, then P^T / dS^T as fp16 into the chunk's
@@ -466,8 +479,8 @@ k_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CU
         // the TMEM loads are warp-collective (.sync.aligned): every lane runs
         // them, rows past S included; only the stores are per-row
         uint32_t a[32], b[32];
-        tmem_ld32(tbase + la + kColAcc + 32 * c, a);
-        tmem_ld32(tbase + la + kColAcc + D + 32 * c, b);
+        tmem_ld32(tbase + la + col_acc(true) + 32 * c, a);
+        tmem_ld32(tbase + la + col_acc(true) + D + 32 * c, b);
         tmem_wait_ld();
         if (key < S) {
           bool fin = true;
@@ -493,11 +506,11 @@ k_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CU
 // ---------------------------------------------------------------- dQ
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
-k_bwd_dq_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
-            const __half* __restrict__ qh, const __half* __restrict__ doh,
+k_bwd_dq_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tdo,
+            const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
             const float* __restrict__ lse, const float* __restrict__ delta, float* __restrict__ dqs,
             int S, float c2, float scale, int* err) {
-  using Lay = BwdLayout<D, true>;
+  using Lay = BwdLayout<D>;
   extern __shared__ __align__(16) uint8_t smem_raw[];
   BwdBars* bars = reinterpret_cast<BwdBars*>(smem_raw);
   uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + Lay::HEAD + 1023) & ~(uintptr_t)1023);
@@ -506,42 +519,23 @@ k_bwd_dq_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUte
   const int i = ntiles - 1 - (int)blockIdx.x;     // query tile; late tiles have the most key tiles
   const int bh = blockIdx.y;
   const int n = i + 1;                            // key tiles j = 0 .. i
-  bwd_setup<true>(bars, warp);
+  bwd_setup(bars, warp);
   const uint32_t tbase = bars->tmem_base;
   volatile Abort* ab = &bars->abort;
 
   if (warp == 0) {
-    if (lane == 0) bwd_produce<D, true>(sm, bars, nullptr, nullptr, i, &tk, &tv, 0, n, bh, ab, err);
+    if (lane == 0) bwd_produce<D>(sm, bars, &tq, &tdo, i, &tk, &tv, 0, n, bh, ab, err);
   } else if (warp == 1) {
-    if (lane == 0) bwd_mma<D, false, true>(sm, bars, tbase, n, ab, err);
+    bwd_mma<D, false>(sm, bars, tbase, n, ab, err);
   } else {
     const int quarter = warp & 3;
     const int half = (warp - 2) >> 2;             // which 64 of the 128 columns
     const int r = quarter * 32 + lane;            // query row within the tile / TMEM lane
     const uint32_t la = (uint32_t)(quarter * 32) << 16;
-    const uint32_t cX = tbase + la + 64 * half, cY = cX + kColY;
+    const uint32_t cX = tbase + la + 64 * half;
     const int q = i * kT + r;
     const float nl2 = q < S ? lse[(size_t)bh * S + q] * -1.4426950408889634f : 0.f;
     const float ndl = q < S ? -delta[(size_t)bh * S + q] : 0.f;
-    {
-      // fixed operands into TMEM as the score MMAs' A operand: lane r holds row
-      // q, column kFixCol + c the fp16 pair (2c, 2c+1) of Q_i (half-0 warps) or,
-      // D/2 columns on, of dO_i (half-1 warps); rows past S are zero
-      const uint4* src = reinterpret_cast<const uint4*>((half ? doh : qh) + ((size_t)bh * S + (q < S ? q : 0)) * D);
-#pragma unroll 1
-      for (int c = 0; c < D / 64; ++c) {
-        uint32_t w[32];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const uint4 x = q < S ? src[8 * c + e] : make_uint4(0, 0, 0, 0);
-          w[4 * e] = x.x; w[4 * e + 1] = x.y; w[4 * e + 2] = x.z; w[4 * e + 3] = x.w;
-        }
-        tmem_st32(tbase + la + kFixCol + half * (D / 2) + 32 * c, w);
-      }
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive_warp(&bars->fix_full);
-    }
     bool ok = true;
     for (int jj = 0; jj < n; ++jj) {
       if (!__all_sync(0xffffffffu, mbar_wait(&bars->x_full, jj & 1, ab, err, 19))) { ok = false; break; }
@@ -561,8 +555,9 @@ k_bwd_dq_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUte
         p_chunk<false>(p0, nl2, c2, 0, 0);
         p_chunk<false>(p1, nl2, c2, 0, 0);
       }
-      if (!__all_sync(0xffffffffu, mbar_wait(&bars->y_full, jj & 1, ab, err, 20))) { ok = false; break; }
+      if (!__all_sync(0xffffffffu, mbar_wait(&bars->y_full[jj & 1], (jj >> 1) & 1, ab, err, 20))) { ok = false; break; }
       tc_fence_after();
+      const uint32_t cY = cX + kColY + 128 * (jj & 1);
       // dP: both chunks, then head / remainder into the chunk's own columns
       uint32_t d0[32], d1[32], hi[16], lo[16];
       tmem_ld32(cY, d0);
@@ -585,7 +580,7 @@ k_bwd_dq_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUte
 #pragma unroll 1
       for (int c = half * (D / 64); c < (half + 1) * (D / 64); ++c) {
         uint32_t a[32];
-        tmem_ld32(tbase + la + kColAcc + 32 * c, a);
+        tmem_ld32(tbase + la + col_acc(false) + 32 * c, a);
         tmem_wait_ld();
         if (q < S) {
           bool fin = true;
@@ -613,7 +608,7 @@ cudaError_t bwd_tc_t(const Geom& g, const void* qs, const void* ks, const void* 
   if (!make_tmap_16(&tq, qs, D, g.S, BH, true, kT) || !make_tmap_16(&tk, ks, D, g.S, BH, true, kT) ||
       !make_tmap_16(&tv, vs, D, g.S, BH, true, kT) || !make_tmap_16(&tdo, dos, D, g.S, BH, true, kT))
     return cudaErrorInvalidValue;
-  const int smem = BwdLayout<D, false>::BYTES, smem_q = BwdLayout<D, true>::BYTES;
+  const int smem = BwdLayout<D>::BYTES, smem_q = smem;
   cudaError_t e = cudaFuncSetAttribute(k_bwd_dkdv_tc<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(k_bwd_dq_tc<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_q);
@@ -625,8 +620,7 @@ cudaError_t bwd_tc_t(const Geom& g, const void* qs, const void* ks, const void* 
   count_launch();
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  k_bwd_dq_tc<D><<<grid, kThreads, smem_q, s>>>(tk, tv, (const __half*)qs, (const __half*)dos, lse, delta, dqs,
-                                                g.S, c2, scale, err);
+  k_bwd_dq_tc<D><<<grid, kThreads, smem_q, s>>>(tq, tdo, tk, tv, lse, delta, dqs, g.S, c2, scale, err);
   count_launch();
   return cudaGetLastError();
 }

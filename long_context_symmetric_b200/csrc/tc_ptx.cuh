@@ -35,6 +35,18 @@ __device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
+// Named barrier `id` (1..15) over the first n threads that reach it (n a
+// multiple of 32); barrier 0 is __syncthreads.
+__device__ __forceinline__ void named_bar_sync(int id, int n) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+// One lane of a converged warp (the same lane for every call in that warp).
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred;
+  asm volatile("{\n\t.reg .b32 r;\n\t.reg .pred p;\n\telect.sync r|p, 0xffffffff;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+               : "=r"(pred));
+  return pred != 0;
+}
 // One arrival per warp: every lane has done its own fences before this call;
 // the warp synchronises and lane 0 arrives (barrier counts are in warps).
 __device__ __forceinline__ void mbar_arrive_warp(uint64_t* bar) {
