@@ -158,73 +158,85 @@ k_attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CU
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      // ---------------- MMA issuer
-      auto issue_s = [&](int t, int j) {       // S_t = Q_t K_j^T
-        const uint32_t kt = sbase + Lay::K + (j & 1) * Lay::OPB;
+    // ---------------- MMA issuer: the whole (converged) warp takes the same
+    // waits and branches, one elected lane issues; shared-memory descriptors
+    // are built once per operand and advanced by constant offsets (the start
+    // address, in 16-byte units, sits in the low 14 bits)
+    const bool leader = elect_one();
+    constexpr uint32_t OPB16 = Lay::OPB >> 4;
+    const uint64_t dQ = sdesc_sw128(sbase + Lay::Q, 16, 1024), dK = sdesc_sw128(sbase + Lay::K, 16, 1024);
+    const uint64_t dV = sdesc_sw128(sbase + Lay::V, kSub, 1024);
+    auto kofs = [](int kk) -> uint64_t { return (uint64_t)((kk >> 2) * (kSub >> 4) + (kk & 3) * 2); };
+    auto issue_s = [&](int t, int j) {       // S_t = Q_t K_j^T
+      const uint64_t a0 = dQ + (uint64_t)(t * OPB16), b0 = dK + (uint64_t)((j & 1) * OPB16);
+      if (leader) {
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t koff = (kk >> 2) * kSub + (kk & 3) * 32;
-          umma_f16(tbase + 256 * t, sdesc_sw128(sbase + Lay::Q + t * Lay::OPB + koff, 16, 1024),
-                   sdesc_sw128(kt + koff, 16, 1024), IDS, kk > 0 ? 1u : 0u);
-        }
+        for (int kk = 0; kk < D / 16; ++kk)
+          umma_f16(tbase + 256 * t, a0 + kofs(kk), b0 + kofs(kk), IDS, kk > 0 ? 1u : 0u);
         umma_commit(&bars->s_full[t]);
-      };
-      auto issue_pv = [&](int t, int j) {      // O_t += P_hi V_j + P_lo V_j
-        const uint32_t vt = sbase + Lay::V + (j & 1) * Lay::OPB;
-        const uint32_t tS = tbase + 256 * t, tO = tS + 128;
+      }
+    };
+    auto issue_pv = [&](int t, int j) {      // O_t += P_hi V_j + P_lo V_j
+      const uint64_t b0 = dV + (uint64_t)((j & 1) * OPB16);
+      const uint32_t tS = tbase + 256 * t, tO = tS + 128;
+      if (leader) {
 #pragma unroll
         for (int kk = 0; kk < kBN / 16; ++kk) {
-          const uint64_t b = sdesc_sw128(vt + kk * 2048, kSub, 1024);
           const uint32_t acol = 32 * (kk >> 1) + 8 * (kk & 1);
-          umma_f16_ts(tO, tS + acol, b, IDO, (j > 0 || kk > 0) ? 1u : 0u);
-          umma_f16_ts(tO, tS + acol + 16, b, IDO, 1u);
+          umma_f16_ts(tO, tS + acol, b0 + kk * 128, IDO, (j > 0 || kk > 0) ? 1u : 0u);
+          umma_f16_ts(tO, tS + acol + 16, b0 + kk * 128, IDO, 1u);
         }
         umma_commit(&bars->o_done[t]);
-      };
-      bool ok = mbar_wait(&bars->q_full, 0, ab, err, 2) && mbar_wait(&bars->k_full[0], 0, ab, err, 3);
-      if (ok) {
-        tc_fence_after();
-        issue_s(0, 0);
-        if (hasB) issue_s(1, 0);
-        umma_commit(&bars->k_empty[0]);
       }
-      for (int j = 0; ok && j < nkv; ++j) {
-        if (!mbar_wait(&bars->v_full[j & 1], (j >> 1) & 1, ab, err, 4)) { ok = false; break; }
-        bool kwait = false;
-        auto k_next = [&]() -> bool {
-          if (kwait) return true;
-          kwait = true;
-          return mbar_wait(&bars->k_full[(j + 1) & 1], ((j + 1) >> 1) & 1, ab, err, 3);
-        };
-        if (j < nkvA) {
-          if (!mbar_wait(&bars->p_full[0], j & 1, ab, err, 5)) { ok = false; break; }
+    };
+    auto wait = [&](uint64_t* bar, uint32_t parity, int site) -> bool {
+      return __all_sync(0xffffffffu, mbar_wait(bar, parity, ab, err, site));
+    };
+    bool ok = wait(&bars->q_full, 0, 2) && wait(&bars->k_full[0], 0, 3);
+    if (ok) {
+      tc_fence_after();
+      issue_s(0, 0);
+      if (hasB) issue_s(1, 0);
+      if (leader) umma_commit(&bars->k_empty[0]);
+    }
+    for (int j = 0; ok && j < nkv; ++j) {
+      if (!wait(&bars->v_full[j & 1], (j >> 1) & 1, 4)) { ok = false; break; }
+      bool kwait = false;
+      auto k_next = [&]() -> bool {
+        if (kwait) return true;
+        kwait = true;
+        return wait(&bars->k_full[(j + 1) & 1], ((j + 1) >> 1) & 1, 3);
+      };
+      if (j < nkvA) {
+        if (!wait(&bars->p_full[0], j & 1, 5)) { ok = false; break; }
+        tc_fence_after();
+        issue_pv(0, j);
+        if (j + 1 < nkvA) {
+          if (!k_next()) { ok = false; break; }
           tc_fence_after();
-          issue_pv(0, j);
-          if (j + 1 < nkvA) {
-            if (!k_next()) { ok = false; break; }
-            tc_fence_after();
-            issue_s(0, j + 1);
-          }
+          issue_s(0, j + 1);
         }
-        if (hasB) {
-          if (!mbar_wait(&bars->p_full[1], j & 1, ab, err, 5)) { ok = false; break; }
+      }
+      if (hasB) {
+        if (!wait(&bars->p_full[1], j & 1, 5)) { ok = false; break; }
+        tc_fence_after();
+        issue_pv(1, j);
+        if (j + 1 < nkvB) {
+          if (!k_next()) { ok = false; break; }
           tc_fence_after();
-          issue_pv(1, j);
-          if (j + 1 < nkvB) {
-            if (!k_next()) { ok = false; break; }
-            tc_fence_after();
-            issue_s(1, j + 1);
-          }
+          issue_s(1, j + 1);
         }
+      }
+      if (leader) {
         umma_commit(&bars->v_empty[j & 1]);
         if (j + 1 < nkv) umma_commit(&bars->k_empty[(j + 1) & 1]);
       }
-      // wait until every MMA issued here has finished before TMEM is released
-      umma_commit(&bars->drain);
-      Abort none{0};
-      mbar_wait(&bars->drain, 0, &none, nullptr, 0);
     }
+    // wait until every MMA issued here has finished before TMEM is released
+    if (leader) umma_commit(&bars->drain);
+    __syncwarp();
+    Abort none{0};
+    mbar_wait(&bars->drain, 0, &none, nullptr, 0);
   } else {
     // ---------------- softmax: one thread per query row / TMEM lane of tile t
     const int t = (warp - 2) >> 2;
