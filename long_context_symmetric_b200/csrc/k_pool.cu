@@ -51,7 +51,12 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
 // bulk async copies (one copy per stage when the group is the whole row), so
 // the loads in flight do not depend on registers; each thread then reads its
 // 16 bytes of every row from shared memory.
-template <typename T, int LV>
+// PP: the pooling factor p as a compile-time constant when it is one of the
+// common values and a stage holds whole level-1 entries (ts % p == 0); then a
+// level-1 entry's p token rows are read and widened together, so the widening
+// conversions (a quarter-rate pipe) overlap instead of waiting on the add chain.
+// PP == 0: any p, one token at a time.
+template <typename T, int LV, int PP>
 __global__ void __launch_bounds__(256, 2) k_pool(const T* __restrict__ q, const T* __restrict__ k,
                                                  const T* __restrict__ v, T* __restrict__ pq,
                                                  T* __restrict__ pk, T* __restrict__ pv,
@@ -67,7 +72,7 @@ __global__ void __launch_bounds__(256, 2) k_pool(const T* __restrict__ q, const 
   const int cb = blockIdx.x;
   const T* x = tensor == 0 ? q : (tensor == 1 ? k : v);
   T* pyr = tensor == 0 ? pq : (tensor == 1 ? pk : pv);
-  const int p = g.p;
+  const int p = PP ? PP : g.p;
   const long long P = g.pl[LV];
   const size_t tok_stride = (size_t)g.H * g.D;
   const T* src0 = x + ((size_t)b * g.N + (size_t)cb * P) * tok_stride + (size_t)hg0 * g.D;
@@ -117,20 +122,9 @@ __global__ void __launch_bounds__(256, 2) k_pool(const T* __restrict__ q, const 
     const long long t0 = (long long)kk * a.ts;
     const int nt = (int)min((long long)a.ts, P - t0);
     const uint8_t* buf = smem + (size_t)slot * a.ts * row_bytes + (size_t)threadIdx.x * 8 * sizeof(T);
-    for (int u = 0; u < nt; ++u) {
-      typename Vec8<T>::Raw raw = *reinterpret_cast<const typename Vec8<T>::Raw*>(buf + (size_t)u * row_bytes);
-      double xr[8];
-      Vec8<T>::raw_f64(raw, xr);
-      if (c == 0) {
-#pragma unroll
-        for (int d = 0; d < 8; ++d) s[d] = xr[d];
-      } else {
-#pragma unroll
-        for (int d = 0; d < 8; ++d) s[d] = __dadd_rn(s[d], xr[d]);
-      }
-      if (++c < p) continue;
-      c = 0;
-      // level-1 entry gi1 complete: emit it, then carry upward while levels complete
+    // level-1 entry gi1 complete (its sum in acc[0]): emit it, then carry
+    // upward while levels complete
+    auto complete = [&]() {
       long long gi = gi1++;
 #pragma unroll
       for (int l = 1; l <= LV; ++l) {
@@ -168,6 +162,40 @@ __global__ void __launch_bounds__(256, 2) k_pool(const T* __restrict__ q, const 
           if (chunk == 0) sq_head[e] = part;
         }
       }
+    };
+    if constexpr (PP > 0) {
+      // whole level-1 entries: all PP rows read first, then widened and summed
+      // left to right
+      for (int u0 = 0; u0 < nt; u0 += PP) {
+        typename Vec8<T>::Raw raw[PP > 0 ? PP : 1];
+#pragma unroll
+        for (int u = 0; u < PP; ++u)
+          raw[u] = *reinterpret_cast<const typename Vec8<T>::Raw*>(buf + (size_t)(u0 + u) * row_bytes);
+#pragma unroll
+        for (int u = 0; u < PP; ++u) {
+          double xr[8];
+          Vec8<T>::raw_f64(raw[u], xr);
+#pragma unroll
+          for (int d = 0; d < 8; ++d) s[d] = u == 0 ? xr[d] : __dadd_rn(s[d], xr[d]);
+        }
+        complete();
+      }
+    } else {
+      for (int u = 0; u < nt; ++u) {
+        typename Vec8<T>::Raw raw = *reinterpret_cast<const typename Vec8<T>::Raw*>(buf + (size_t)u * row_bytes);
+        double xr[8];
+        Vec8<T>::raw_f64(raw, xr);
+        if (c == 0) {
+#pragma unroll
+          for (int d = 0; d < 8; ++d) s[d] = xr[d];
+        } else {
+#pragma unroll
+          for (int d = 0; d < 8; ++d) s[d] = __dadd_rn(s[d], xr[d]);
+        }
+        if (++c < p) continue;
+        c = 0;
+        complete();
+      }
     }
     __syncthreads();                    // every thread is done with this stage
     if (threadIdx.x == 0 && kk + a.ns < nstages) issue(kk + a.ns);
@@ -195,22 +223,27 @@ cudaError_t launch_t(const Geom& g, const void* q, const void* k, const void* v,
   a.ts = ts;
   a.ns = 3;
   const size_t smem = (size_t)a.ns * a.ts * a.row_bytes + a.ns * sizeof(uint64_t);
-  cudaError_t e = cudaFuncSetAttribute(k_pool<T, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  (void)e;
+  cudaError_t e = cudaSuccess;
+  // compile-time p when it divides the stage
+  const int pp = (a.ts % g.p == 0 && (g.p == 2 || g.p == 4 || g.p == 8)) ? g.p : 0;
   dim3 block(hg * C8);
   dim3 grid(g.n[g.L - 1], g.H / hg, 3 * g.B);
   const T* tq = (const T*)q; const T* tk = (const T*)k; const T* tv = (const T*)v;
   T* tpq = (T*)pq; T* tpk = (T*)pk; T* tpv = (T*)pv;
   switch (LV) {
-#define LH_POOL_CASE(n)                                                                              \
-    case n:                                                                                          \
-      e = cudaFuncSetAttribute(k_pool<T, n>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem); \
-      if (e != cudaSuccess) return e;                                                                \
-      k_pool<T, n><<<grid, block, smem, s>>>(tq, tk, tv, tpq, tpk, tpv, sq, a, err);                 \
+#define LH_POOL_PP(n, P)                                                                                \
+  e = cudaFuncSetAttribute(k_pool<T, n, P>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);    \
+  if (e != cudaSuccess) return e;                                                                       \
+  k_pool<T, n, P><<<grid, block, smem, s>>>(tq, tk, tv, tpq, tpk, tpv, sq, a, err);
+#define LH_POOL_CASE(n)                                                                                 \
+    case n:                                                                                             \
+      if (pp == 8) { LH_POOL_PP(n, 8) } else if (pp == 4) { LH_POOL_PP(n, 4) }                          \
+      else if (pp == 2) { LH_POOL_PP(n, 2) } else { LH_POOL_PP(n, 0) }                                  \
       break;
     LH_POOL_CASE(1) LH_POOL_CASE(2) LH_POOL_CASE(3) LH_POOL_CASE(4)
     LH_POOL_CASE(5) LH_POOL_CASE(6) LH_POOL_CASE(7)
 #undef LH_POOL_CASE
+#undef LH_POOL_PP
     default: return cudaErrorInvalidValue;
   }
   count_launch();
