@@ -8,11 +8,16 @@
 //
 // Per level l = L-1 .. 1 (all entries of level L-1 are the first candidates):
 //   score = max(|mean_Q|^2, |mean_K|^2) (fp64, from lh_pool)
-//   the first k_l candidates in the order (score desc, index asc) are expanded,
-//   found with a bitonic sorting network over shared-memory chunks of at most
-//   8192 (score, position) keys; when the candidates exceed one chunk, the
-//   current best k_l are kept at the head of the chunk and the rest is refilled
-//   with new candidates, chunk after chunk (k_l <= 4096).
+//   the first k_l candidates in the order (score desc, index asc) are expanded.
+//   Only the set matters (the sub-sequence order comes from the tree below),
+//   so for up to 8192 candidates it is found by a most-significant-digit
+//   radix select on the unique key (score bits, then position reversed): ten
+//   8-bit digit passes, each a 256-bin shared-memory histogram of the keys
+//   that still match the chosen prefix, give the k_l-th key, and every key at
+//   or above it is expanded. Beyond 8192 candidates the pages' chunked bitonic
+//   sort is used: a sorting network over shared-memory chunks of 8192
+//   (score, position) keys, the current best k_l kept at the head of the chunk
+//   and the rest refilled with new candidates, chunk after chunk (k_l <= 4096).
 //   the p children of each expanded entry, in index order, are the next
 //   level's candidates and sub-sequence entries.
 // Post-order: every included entry's subtree (itself plus its included
@@ -105,6 +110,85 @@ __device__ __forceinline__ unsigned long long score_bits(const double* sqq, cons
   return (unsigned long long)__double_as_longlong(s);   // s >= 0: bit order = value order
 }
 
+// Flags fl[q] = 1 for the k (< c <= kChunk) candidates q first in the order
+// (score desc, q asc), 0 for the rest. Key of q: hi = score bits, lo = c-1-q,
+// compared as (hi, lo) descending; keys are unique. hist: 257 ints of shared
+// memory, bc: 2 ints. All threads must call it.
+__device__ void radix_select_flags(const double* sq_l, const double* sk_l, const int32_t* cl, int c, int k,
+                                   int32_t* fl, int* hist, int* bc) {
+  constexpr int KPT = kChunk / kThreads;
+  const int lane = threadIdx.x & 31;
+  unsigned long long hi[KPT];
+  unsigned lo[KPT];
+  bool valid[KPT];
+#pragma unroll
+  for (int j = 0; j < KPT; ++j) {
+    const int q = threadIdx.x + j * kThreads;
+    valid[j] = q < c;
+    hi[j] = valid[j] ? score_bits(sq_l, sk_l, cl[q]) : 0ull;
+    lo[j] = valid[j] ? (unsigned)(c - 1 - q) : 0u;
+  }
+  unsigned long long thi = 0ull;   // chosen digits of the threshold key so far
+  unsigned tlo = 0u;
+  int kk = k;                      // rank of the threshold among keys matching the prefix
+  // passes 0..7: hi bits 63..0; passes 8, 9: lo bits 15..0 (c <= kChunk < 2^16)
+#pragma unroll 1
+  for (int pass = 0; pass < 10; ++pass) {
+    for (int i = threadIdx.x; i < 257; i += kThreads) hist[i] = 0;
+    __syncthreads();
+#pragma unroll
+    for (int j = 0; j < KPT; ++j) {
+      int d = 256;                 // 256: not counted
+      if (valid[j]) {
+        if (pass < 8) {
+          const int sh = 56 - 8 * pass;
+          const bool m = pass == 0 || (hi[j] >> (sh + 8)) == (thi >> (sh + 8));
+          if (m) d = (int)((hi[j] >> sh) & 0xFF);
+        } else {
+          const int sh = 8 * (9 - pass);
+          const bool m = hi[j] == thi && (pass == 8 || (lo[j] >> (sh + 8)) == (tlo >> (sh + 8)));
+          if (m) d = (int)((lo[j] >> sh) & 0xFF);
+        }
+      }
+      // one atomic per distinct digit of the warp
+      const unsigned same = __match_any_sync(0xffffffffu, d);
+      if (d < 256 && lane == __ffs(same) - 1) atomicAdd(&hist[d], __popc(same));
+    }
+    __syncthreads();
+    if (threadIdx.x < 32) {
+      // bins from the top: lane l sums bins 255-8l .. 248-8l
+      int loc[8], sum = 0;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) { loc[u] = hist[255 - 8 * lane - u]; sum += loc[u]; }
+      int incl = sum;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      int above = incl - sum;      // keys in bins above this lane's first bin
+      if (above < kk && kk <= incl) {
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          if (above < kk && kk <= above + loc[u]) { bc[0] = 255 - 8 * lane - u; bc[1] = kk - above; }
+          above += loc[u];
+        }
+      }
+    }
+    __syncthreads();
+    const int b = bc[0];
+    kk = bc[1];
+    if (pass < 8) thi |= (unsigned long long)b << (56 - 8 * pass);
+    else tlo |= (unsigned)b << (8 * (9 - pass));
+    __syncthreads();               // bc is rewritten by the next pass
+  }
+#pragma unroll
+  for (int j = 0; j < KPT; ++j) {
+    const int q = threadIdx.x + j * kThreads;
+    if (valid[j]) fl[q] = (hi[j] > thi || (hi[j] == thi && lo[j] >= tlo)) ? 1 : 0;
+  }
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
 k_select(const double* __restrict__ sq, int32_t* __restrict__ sel, int32_t* __restrict__ map,
          int32_t* __restrict__ slot, int32_t* __restrict__ ws, SelArgs a) {
@@ -112,6 +196,7 @@ k_select(const double* __restrict__ sq, int32_t* __restrict__ sel, int32_t* __re
   unsigned long long* sk = reinterpret_cast<unsigned long long*>(smem_raw);
   unsigned* sp = reinterpret_cast<unsigned*>(sk + kChunk);
   __shared__ int warp_tot[33];
+  __shared__ int hist[257], bcast[2];
 
   const Geom& g = a.g;
   const int bh = blockIdx.x;
@@ -145,6 +230,8 @@ k_select(const double* __restrict__ sq, int32_t* __restrict__ sel, int32_t* __re
     const double* sk_l = sqk + g.off[l];
     if (k >= c) {
       for (int q = threadIdx.x; q < c; q += kThreads) fl[q] = 1;
+    } else if (c <= kChunk) {
+      radix_select_flags(sq_l, sk_l, cl, c, k, fl, hist, bcast);
     } else {
       for (int q = threadIdx.x; q < c; q += kThreads) fl[q] = 0;
       // chunked top-k: best k stay at the head of the chunk between rounds
