@@ -16,7 +16,7 @@
 // every output byte is written exactly once, no read-modify-write, and the
 // result does not depend on scheduling. The accumulation arithmetic follows
 // lh_accum (fp32, or int64 fixed point with one count = 2^-32).
-#include "lh_common.cuh"
+#include "tc_ptx.cuh"   // lh_common.cuh, mbarrier helpers
 
 namespace lh {
 namespace {
@@ -454,6 +454,152 @@ __global__ void __launch_bounds__(256) k_blocksum(const T* __restrict__ dout,
   }
 }
 
+// Same block sums with the token rows streamed through a shared-memory ring
+// filled by 1-D bulk async copies (one CTA per coarsest block and head group;
+// hg * D / 8 threads, a multiple of 32). PP = p, a compile-time 2, 4 or 8 that
+// divides the stage: a level-1 group's PP rows are read from shared memory
+// together. Emission order and arithmetic are those of k_blocksum.
+struct RingArgs {
+  int hg;          // heads per CTA (a divisor of H)
+  int ts;          // tokens per stage
+  int ns;          // stages
+  int row_bytes;   // bytes of one token row of the head group
+};
+
+__device__ __forceinline__ void bs_bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+               ::"r"(tc::smem_u32(dst)), "l"(src), "r"(bytes), "r"(tc::smem_u32(bar))
+               : "memory");
+}
+
+template <typename T, typename TO, int LV, int PP>
+__global__ void __launch_bounds__(256, 2) k_blocksum_ring(const T* __restrict__ dout,
+                                                          const float* __restrict__ os,
+                                                          const int32_t* __restrict__ slot,
+                                                          TO* __restrict__ dos, float* __restrict__ delta,
+                                                          Geom g, RingArgs a, int* err) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int C8 = g.D >> 3;
+  const int b = blockIdx.z;
+  const int hg0 = blockIdx.y * a.hg;
+  const int head = hg0 + threadIdx.x / C8;
+  const int chunk = threadIdx.x % C8;
+  const int cb = blockIdx.x;
+  constexpr int p = PP;
+  const long long P = g.pl[LV];
+  const size_t tok_stride = (size_t)g.H * g.D;
+  const long long bh = (long long)b * g.H + head;
+  const T* src0 = dout + ((size_t)b * g.N + (size_t)cb * P) * tok_stride + (size_t)hg0 * g.D;
+  const int32_t* slot_h = slot + bh * g.E;
+  const int row_bytes = a.row_bytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + (size_t)a.ns * a.ts * row_bytes);
+  const int nstages = (int)((P + a.ts - 1) / a.ts);
+  const bool contiguous = (a.hg == g.H);
+  if (threadIdx.x == 0) {
+    for (int s2 = 0; s2 < a.ns; ++s2) tc::mbar_init(&full[s2], 1);
+    tc::fence_mbar_init();
+  }
+  __syncthreads();
+  auto issue = [&](int kk) {
+    const int si = kk % a.ns;
+    const long long t0 = (long long)kk * a.ts;
+    const int nt = (int)min((long long)a.ts, P - t0);
+    uint8_t* dst = smem + (size_t)si * a.ts * row_bytes;
+    tc::mbar_expect_tx(&full[si], (uint32_t)(nt * row_bytes));
+    if (contiguous) {
+      bs_bulk_load(dst, src0 + t0 * tok_stride, (uint32_t)(nt * row_bytes), &full[si]);
+    } else {
+      for (int u = 0; u < nt; ++u)
+        bs_bulk_load(dst + (size_t)u * row_bytes, src0 + (t0 + u) * tok_stride, (uint32_t)row_bytes, &full[si]);
+    }
+  };
+  if (threadIdx.x == 0)
+    for (int kk = 0; kk < a.ns && kk < nstages; ++kk) issue(kk);
+
+  // one included entry: write its row and its delta
+  auto emit = [&](int s, const float (&v)[8]) {
+    float part = 0.f;
+    float ov[8];
+    if (s >= 0) {
+      load8_f32(os + ((size_t)bh * g.S + s) * g.D + chunk * 8, ov);
+      // delta from the stored (rounded) dos: the values the backward's dP uses
+#pragma unroll
+      for (int d = 0; d < 8; ++d)
+        part = fmaf(sizeof(TO) == 2 ? __half2float(__float2half_rn(v[d])) : v[d], ov[d], part);
+    }
+    for (int off = C8 >> 1; off >= 1; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
+    if (s >= 0) {
+      Vec8<TO>::store_f32(dos + ((size_t)bh * g.S + s) * g.D + chunk * 8, v);
+      if (chunk == 0) delta[(size_t)bh * g.S + s] = part;
+      float mx = 0.f;
+#pragma unroll
+      for (int d = 0; d < 8; ++d) mx = fmaxf(mx, fabsf(v[d]));
+      if (sizeof(TO) == 2 && !(mx <= kHalfMax)) report_error(err, LH_ERR_DEVICE, 100);
+    }
+  };
+
+  float acc[LV + 1][8];   // acc[l]: running sum of the open entry of level l (acc[0] unused)
+  const long long i1_end = (long long)(cb + 1) * (P / p);
+  long long i1 = (long long)cb * (P / p);          // level-1 index of the next group
+  int e1n = __ldg(slot_h + g.off[1] + (int)i1);    // its slot entry, fetched one group ahead
+  tc::Abort none{0};
+  for (int kk = 0; kk < nstages; ++kk) {
+    const int si = kk % a.ns;
+    const bool ok = tc::mbar_wait(&full[si], (kk / a.ns) & 1, &none, err, 201);
+    if (__syncthreads_or(!ok)) break;   // copies never landed: reported, all threads leave
+    const long long t0 = (long long)kk * a.ts;
+    const int nt = (int)min((long long)a.ts, P - t0);
+    const uint8_t* buf = smem + (size_t)si * a.ts * row_bytes + (size_t)threadIdx.x * 8 * sizeof(T);
+    for (int u0 = 0; u0 < nt; u0 += p, ++i1) {
+      const int e1 = e1n;
+      if (i1 + 1 < i1_end) e1n = __ldg(slot_h + g.off[1] + (int)(i1 + 1));
+      typename Vec8<T>::Raw raw[p];
+#pragma unroll
+      for (int u = 0; u < p; ++u)
+        raw[u] = *reinterpret_cast<const typename Vec8<T>::Raw*>(buf + (size_t)(u0 + u) * row_bytes);
+      const int s1 = e1 >= 0 ? (e1 >> 1) : -1;
+      const bool tok_in = e1 >= 0 && (e1 & 1);               // children (tokens) included
+      // tokens are emitted only where some lane of the warp has them included
+      const bool any_tok = __any_sync(0xffffffffu, tok_in);
+      float sum[8];
+#pragma unroll
+      for (int u = 0; u < p; ++u) {
+        float x[8];
+        Vec8<T>::raw_f32(raw[u], x);
+        if (u == 0) {
+#pragma unroll
+          for (int d = 0; d < 8; ++d) sum[d] = x[d];
+        } else {
+#pragma unroll
+          for (int d = 0; d < 8; ++d) sum[d] = __fadd_rn(sum[d], x[d]);
+        }
+        if (any_tok) emit(tok_in ? s1 - p + u : -1, x);
+      }
+#pragma unroll
+      for (int d = 0; d < 8; ++d) acc[1][d] = sum[d];
+      if (__any_sync(0xffffffffu, e1 >= 0)) emit(e1 >= 0 ? (e1 >> 1) : -1, sum);
+      long long gi = i1;
+#pragma unroll
+      for (int l = 2; l <= LV; ++l) {
+        const int pos = (int)(gi % p);
+        if (pos == 0) {
+#pragma unroll
+          for (int d = 0; d < 8; ++d) acc[l][d] = acc[l - 1][d];
+        } else {
+#pragma unroll
+          for (int d = 0; d < 8; ++d) acc[l][d] = __fadd_rn(acc[l][d], acc[l - 1][d]);
+        }
+        if (pos != p - 1) break;
+        gi /= p;
+        const int e = __ldg(slot_h + g.off[l] + (int)gi);
+        if (__any_sync(0xffffffffu, e >= 0)) emit(e >= 0 ? (e >> 1) : -1, acc[l]);
+      }
+    }
+    __syncthreads();                    // every thread is done with this stage
+    if (threadIdx.x == 0 && kk + a.ns < nstages) issue(kk + a.ns);
+  }
+}
+
 // L == 1: dos = dout transposed to [B][H][N][D]; delta = <dout, os>.
 template <typename T, typename TO>
 __global__ void __launch_bounds__(256) k_blocksum_l1(const T* __restrict__ dout,
@@ -537,6 +683,42 @@ cudaError_t blocksum_t(const Geom& g, const void* dout, const float* os, const i
     while (g.H % hg) --hg;
   }
   const int ncoarse = g.n[g.L - 1];
+  if ((hg * C8) % 32 == 0 && (g.p == 2 || g.p == 4 || g.p == 8)) {
+    // ring-streamed variant: whole level-1 groups per stage
+    RingArgs a;
+    a.hg = hg;
+    a.row_bytes = hg * g.D * (int)sizeof(T);
+    const long long P = g.pl[g.L - 1];
+    int ts = 1;
+    while (ts * 2 * a.row_bytes <= 32768 && ts * 2 <= P) ts *= 2;
+    a.ts = ts;
+    a.ns = 3;
+    if (ts % g.p == 0) {
+      const size_t smem = (size_t)a.ns * a.ts * a.row_bytes + a.ns * sizeof(uint64_t);
+      dim3 rgrid(ncoarse, g.H / hg, g.B);
+      const T* d = (const T*)dout;
+      TO* o = (TO*)dos;
+      cudaError_t e = cudaSuccess;
+#define LH_BSR(n, P)                                                                                     \
+  e = cudaFuncSetAttribute(k_blocksum_ring<T, TO, n, P>, cudaFuncAttributeMaxDynamicSharedMemorySize,    \
+                           (int)smem);                                                                   \
+  if (e != cudaSuccess) return e;                                                                        \
+  k_blocksum_ring<T, TO, n, P><<<rgrid, hg * C8, smem, s>>>(d, os, slot, o, delta, g, a, err);
+#define LH_BSR_CASE(n)                                                                                   \
+    case n:                                                                                              \
+      if (g.p == 8) { LH_BSR(n, 8) } else if (g.p == 4) { LH_BSR(n, 4) } else { LH_BSR(n, 2) }          \
+      break;
+      switch (g.L - 1) {
+        LH_BSR_CASE(1) LH_BSR_CASE(2) LH_BSR_CASE(3) LH_BSR_CASE(4)
+        LH_BSR_CASE(5) LH_BSR_CASE(6) LH_BSR_CASE(7)
+        default: return cudaErrorInvalidValue;
+      }
+#undef LH_BSR_CASE
+#undef LH_BSR
+      count_launch();
+      return cudaGetLastError();
+    }
+  }
   int yb = 1;
   while (yb * 2 * hg * C8 <= 256 && yb * 2 <= ncoarse) yb *= 2;
   dim3 block(hg * C8, yb);
