@@ -51,6 +51,19 @@ def workload_desc(w):
             f"recipe {w.recipe}, accumulation {w.mode}")
 
 
+# DRAM bytes per call of the attention stages at the 512K workload: ncu's
+# dram__bytes_read.sum + dram__bytes_write.sum of each kernel on the 2-head case
+# of the same workload (--heads 2), times 8 (the heads are independent problems,
+# so traffic grows in proportion). Only the kernels as they are now; set back to
+# None when one of them changes.
+DRAM_TRAFFIC = {
+    "ctx512k": {
+        "attn_bwd": 8 * (53.017856e6 + 8.236032e6 + 52.881664e6 + 4.685056e6),   # dK/dV + dQ kernels
+        "attn_fwd": 8 * (39.371776e6 + 0.356352e6),
+    },
+}
+
+
 def stage_work(w, pl):
     """Algorithmic bytes (memory stages) or FLOPs (attention) per launch of each stage."""
     e = 2 if w.dtype == "bf16" else 4
@@ -270,33 +283,61 @@ def main():
     # end-to-end through the public API: pinned host inputs -> device, fwd + bwd, results -> host
     e2e = None
     if args.e2e_steps > 0:
+        # End to end through the public calls: every step copies its inputs
+        # (Q, K, V, dO) from pinned host memory and reads back the step's loss,
+        # sum(O * dO) as an fp32 scalar; O and the gradients stay on the device,
+        # as in training. The next step's inputs are copied on a second stream
+        # into the other of two device buffer sets while this step computes.
         hq, hk, hv, hdo = (x.cpu().pin_memory() for x in (q, k, v, do))
-        ho, hdq, hdk, hdv = (torch.empty(q.shape, dtype=q.dtype).pin_memory() for _ in range(4))
-        dq_, dk_, dv_ = (torch.empty_like(q) for _ in range(3))
-        q_, k_, v_, do_, o_ = (torch.empty_like(q) for _ in range(5))
+        bufs = [[torch.empty_like(q) for _ in range(4)] for _ in range(2)]
+        o_, dq_, dk_, dv_ = (torch.empty_like(q) for _ in range(4))
+        loss_d = torch.empty((), dtype=torch.float32, device=dev)
+        loss_h = torch.empty((), dtype=torch.float32).pin_memory()
+        cs = torch.cuda.Stream(device=dev)
+        ev_in = [torch.cuda.Event() for _ in range(2)]
+        ev_done = [torch.cuda.Event() for _ in range(2)]
         h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv, hdo))
-        d2h = sum(x.numel() * x.element_size() for x in (ho, hdq, hdk, hdv))
+        d2h = loss_h.numel() * loss_h.element_size()
 
-        def e2e_step():
-            for dst, src in ((q_, hq), (k_, hk), (v_, hv), (do_, hdo)):
-                dst.copy_(src, non_blocking=True)
+        def copy_in(i):
+            bi = i & 1
+            if i >= 2:
+                cs.wait_event(ev_done[bi])        # step i-2 is done with these buffers
+            with torch.cuda.stream(cs):
+                for dst, src in zip(bufs[bi], (hq, hk, hv, hdo)):
+                    dst.copy_(src, non_blocking=True)
+            ev_in[bi].record(cs)
+
+        def compute(i):
+            bi = i & 1
+            q_, k_, v_, do_ = bufs[bi]
+            stream.wait_event(ev_in[bi])
             lh.forward(cfg, q_, k_, v_, o_, ws, stream)
             lh.backward(cfg, do_, dq_, dk_, dv_, ws, stream)
-            for dst, src in ((ho, o_), (hdq, dq_), (hdk, dk_), (hdv, dv_)):
-                dst.copy_(src, non_blocking=True)
+            with torch.cuda.stream(stream):
+                loss_d.copy_(torch.sum(o_ * do_, dtype=torch.float32))
+                loss_h.copy_(loss_d, non_blocking=True)
+            ev_done[bi].record(stream)
 
-        e2e_step()
+        def run(n):
+            copy_in(0)
+            for i in range(n):
+                if i + 1 < n:
+                    copy_in(i + 1)
+                compute(i)
+
+        run(2)
         torch.cuda.synchronize(dev)
         lhdist.barrier()
         a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        for _ in range(args.e2e_steps):
-            e2e_step()
+        a.record(cs)
+        run(args.e2e_steps)
         b_.record(stream)
         torch.cuda.synchronize(dev)
         e2e_ms = lhdist.max_over_ranks(a.elapsed_time(b_) / args.e2e_steps, dev)
         e2e = {"value": lhdist.job_throughput(w.B * w.N, world, e2e_ms / 1e3), "unit": "tokens/s",
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
+               "result": "loss = sum(O * dO), fp32, read back every step"}
 
     peaks, peak_kind = load_peaks()
     work = stage_work(w, pl)
@@ -317,7 +358,11 @@ def main():
     roofline = {
         "kernel": dom, "bound": frac[dom]["bound"], "achieved": frac[dom]["achieved"],
         "peak": peaks["hbm_gbs"] if kind == "bytes" else peaks["bf16_tflops_sustained"],
-        "unit": frac[dom]["unit"], "frac": frac[dom]["frac"], "traffic": None,
+        "unit": frac[dom]["unit"], "frac": frac[dom]["frac"],
+        "traffic": (DRAM_TRAFFIC.get(w.name, {}).get(dom)
+                    if (w.B, w.H, w.N) == (synth.WORKLOADS[w.name].B, synth.WORKLOADS[w.name].H,
+                                           synth.WORKLOADS[w.name].N) else None),
+        "traffic_unit": "bytes per call",
         "peak_source": f"{peak_kind} ({'hbm_gbs' if kind == 'bytes' else 'bf16_tflops_sustained'})",
     }
 
