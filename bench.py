@@ -70,6 +70,18 @@ def stage_work(w, pl):
     B, H, N, D, S, E = w.B, w.H, w.N, w.D, pl.S, pl.E
     tok = B * N * H * D * e
     sub = B * H * S * D
+    if w.L == 1:
+        # no pyramid: pool does nothing, select writes the identity map
+        return {
+            "pool": ("bytes", 0),
+            "select": ("bytes", B * H * N * 4),
+            "gather": ("bytes", 6 * sub * e + B * H * S * 4),
+            "attn_fwd": ("flops", 2.0 * B * H * S * S * D),
+            "scatter": ("bytes", tok + sub * 4),
+            "scatter_bwd": ("bytes", tok + sub * 4 + sub * (2 if w.dtype == "bf16" else 4) + B * H * S * 4),
+            "attn_bwd": ("flops", 5.0 * B * H * S * S * D),
+            "spread": ("bytes", 3 * tok + 3 * sub * 4),
+        }
     return {
         "pool": ("bytes", 3 * tok + 3 * B * H * E * D * e + 2 * B * H * E * 8),
         "select": ("bytes", 2 * B * H * E * 8 + B * H * (S + E + (w.L - 1) * w.K) * 4),
@@ -80,6 +92,37 @@ def stage_work(w, pl):
         "attn_bwd": ("flops", 5.0 * B * H * S * S * D),
         "spread": ("bytes", 3 * tok + 3 * sub * 4 + B * H * E * 4),
     }
+
+
+def sdpa_context(q, k, v, do, iters=2):
+    """torch's own causal scaled_dot_product_attention, forward + backward, on the
+    full token sequence of the same inputs (a library baseline, timed with CUDA
+    events): median ms per step and the backend that ran."""
+    import torch.nn.functional as F
+    from torch.nn.attention import SDPBackend, sdpa_kernel
+    qt, kt, vt, dot = (x.transpose(1, 2) for x in (q, k, v, do))     # [B, H, N, D] views
+    last = "no backend"
+    for backend in (SDPBackend.CUDNN_ATTENTION, SDPBackend.FLASH_ATTENTION, SDPBackend.EFFICIENT_ATTENTION):
+        try:
+            with sdpa_kernel(backends=[backend]):
+                def step():
+                    qq, kq, vq = (t.detach().requires_grad_(True) for t in (qt, kt, vt))
+                    o = F.scaled_dot_product_attention(qq, kq, vq, is_causal=True)
+                    o.backward(dot)
+                step()
+                torch.cuda.synchronize()
+                times = []
+                for _ in range(iters):
+                    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    a.record()
+                    step()
+                    b.record()
+                    torch.cuda.synchronize()
+                    times.append(a.elapsed_time(b))
+                return {"ms_per_step": statistics.median(times), "backend": backend.name, "iters": iters}
+        except RuntimeError as e:        # backend not available for this shape or GPU
+            last = str(e).splitlines()[0][:200]
+    return {"unavailable": last}
 
 
 class ClockSampler:
@@ -196,6 +239,9 @@ def main():
     ap.add_argument("--workload", default="ctx512k", choices=list(synth.WORKLOADS))
     ap.add_argument("--e2e-steps", type=int, default=2)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sdpa-context", action="store_true",
+                    help="also time torch's scaled_dot_product_attention (causal, fwd+bwd) on the full "
+                         "token sequence of the same inputs, as context for the speed-up over dense attention")
     ap.add_argument("--heads", type=int, default=None,
                     help="smaller case of the same recipe (fewer heads), e.g. for an ncu capture")
     ap.add_argument("--tokens", type=int, default=None, help="smaller case of the same recipe (fewer tokens)")
@@ -344,6 +390,8 @@ def main():
     frac = {}
     for s in stages:
         kind, amount = work[s]
+        if amount == 0:
+            continue                  # a stage with nothing to do for this shape
         sec = stage_ms[s] / 1e3
         if kind == "bytes":
             ach = amount / sec / 1e9
@@ -353,7 +401,7 @@ def main():
             ach = amount / sec / 1e12
             frac[s] = {"ms": round(stage_ms[s], 4), "achieved": round(ach, 2), "unit": "TFLOP/s",
                        "frac": round(ach / peaks["bf16_tflops_sustained"], 4), "bound": "tensor"}
-    dom = max(stages, key=lambda s: stage_ms[s])
+    dom = max(frac, key=lambda s: stage_ms[s])
     kind, amount = work[dom]
     roofline = {
         "kernel": dom, "bound": frac[dom]["bound"], "achieved": frac[dom]["achieved"],
@@ -365,6 +413,12 @@ def main():
         "traffic_unit": "bytes per call",
         "peak_source": f"{peak_kind} ({'hbm_gbs' if kind == 'bytes' else 'bf16_tflops_sustained'})",
     }
+
+    context = None
+    if args.sdpa_context and rank == 0:
+        context = sdpa_context(q, k, v, do)
+        if "ms_per_step" in context:
+            context["lighthouse_speedup"] = context["ms_per_step"] / ms_step
 
     cpu_baseline = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -384,6 +438,8 @@ def main():
         "roofline": roofline, "stages": frac, "cpu_baseline": cpu_baseline, "e2e": e2e,
         "gpu_launches": launches, "clocks": clocks,
     }
+    if context is not None:
+        line["context_sdpa"] = context
     if rank == 0:
         print(json.dumps(line), flush=True)
     lhdist.shutdown()

@@ -94,7 +94,7 @@ typedef struct {
   int k[LH_MAX_LEVELS];               /* entries expanded at level l (l >= 1) */
   int c[LH_MAX_LEVELS];               /* entries of level l in the sub-sequence */
   int lvl_off[LH_MAX_LEVELS];         /* start of level l (l >= 1) within E; lvl_off[0] = 0 unused */
-  size_t ws_bytes;                    /* workspace bytes lh_score_topk / lh_forward need */
+  size_t ws_bytes;                    /* workspace bytes lh_score_topk / lh_forward need (0 if L == 1) */
 } lh_plan_t;
 
 /* Library version (major*10000 + minor*100 + patch). */

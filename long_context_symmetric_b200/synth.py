@@ -57,6 +57,9 @@ WORKLOADS = {
         Workload("ctx98k", 1, 16, 98304, 64, "bf16", 4, 4, 512, "iid", "fp", True, 3),
         Workload("ctx512k", 1, 16, 524288, 128, "bf16", 8, 4, 1024, "outliers", "fp", True, 4),
         Workload("ties131k", 1, 8, 131072, 128, "bf16", 4, 5, 512, "codebook", "fixed", True, 5),
+        # the 512K inputs (same recipe and seed) with L = 1: the sub-sequence is the
+        # whole token sequence, i.e. dense causal attention over all N tokens
+        Workload("dense512k", 1, 16, 524288, 128, "bf16", 8, 1, 1024, "outliers", "fp", True, 4),
     ]
 }
 
