@@ -215,6 +215,16 @@ lh_status lh_get_device_error(void* stream, int* detail);
 /* Number of liblh kernels launched by this process so far. */
 unsigned long long lh_launch_count(void);
 
+/* Diagnostics (the pages have no counterpart: this checks the failure path).
+ * Launches one warp that waits on an mbarrier nothing ever arrives on, through
+ * the same bounded wait every kernel uses, with a bound of `limit_cycles` SM
+ * clock cycles (1 .. 2e9). The wait gives up, the device error word records
+ * LH_ERR_TIMEOUT with detail 900 (lh_get_device_error returns it), the kernel
+ * ends normally and the context stays usable. `gave_up`: device int, set to 1
+ * when the wait gave up. LH_ERR_NULL / LH_ERR_SHAPE for bad arguments, checked
+ * before the launch. */
+lh_status lh_selftest_timeout(long long limit_cycles, int* gave_up, void* stream);
+
 /* lh_score_topk without a caller workspace (the paper has no counterpart: this
  * is for callers, not the method). Some callers cannot provide or allocate a
  * device workspace: a fixed arena that owns all device memory and may not

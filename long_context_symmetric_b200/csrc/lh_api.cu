@@ -45,6 +45,7 @@ cudaError_t launch_attn_fwd(const Geom& g, lh_dtype dt, const void* qs, const vo
 cudaError_t launch_attn_bwd_tc(const Geom& g, const void* qs, const void* ks, const void* vs,
                                const void* dos, const float* lse, const float* delta, float* dqs,
                                float* dks, float* dvs, int* err, cudaStream_t s);
+cudaError_t launch_selftest_wait(long long limit_cycles, int* err, int* gave_up, cudaStream_t s);
 
 cudaError_t launch_attn_bwd(const Geom& g, lh_dtype dt, const void* qs, const void* ks,
                             const void* vs, const void* dos, const float* lse, const float* delta,
@@ -302,6 +303,15 @@ lh_status lh_backward(const lh_config* cfg, const void* dout, void* dq, void* dk
                         stream)) != LH_OK)
     return st;
   return lh_spread(cfg, b->dqs, b->dks, b->dvs, b->slot, dq, dk, dv, stream);
+}
+
+lh_status lh_selftest_timeout(long long limit_cycles, int* gave_up, void* stream) {
+  if (!gave_up) return LH_ERR_NULL;
+  if (limit_cycles < 1 || limit_cycles > 2000000000LL) return LH_ERR_SHAPE;
+  int* err = device_error_ptr();
+  if (!err) return LH_ERR_CUDA;
+  return lh::launch_selftest_wait(limit_cycles, err, gave_up, (cudaStream_t)stream) == cudaSuccess ? LH_OK
+                                                                                                  : LH_ERR_CUDA;
 }
 
 lh_status lh_get_device_error(void* stream, int* detail) {

@@ -71,18 +71,18 @@ struct Abort {
   int flag;
 };
 
-// Bounded wait on phase `parity`. Returns false if the wait gave up (time
-// limit, or another role of the CTA already gave up); the first role to give
-// up records LH_ERR_TIMEOUT with `site` as detail.
+// Bounded wait on phase `parity`. Returns false if the wait gave up (after
+// `limit` SM clock cycles, or because another role of the CTA already gave up);
+// the first role to give up records LH_ERR_TIMEOUT with `site` as detail.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile Abort* ab,
-                                          int* err, int site) {
+                                          int* err, int site, long long limit = kWaitCycles) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 63) == 0) {
       if (ab->flag) return false;
-      if (clock64() - t0 > kWaitCycles) {
+      if (clock64() - t0 > limit) {
         ab->flag = 1;
         if (err && atomicCAS(err, 0, (int)LH_ERR_TIMEOUT) == 0) atomicExch(err + 1, site);
         return false;

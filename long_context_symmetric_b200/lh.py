@@ -71,6 +71,7 @@ _SIGS = {
     "lh_backward": ([ctypes.POINTER(Config)] + [c_void_p] * 4 + [ctypes.POINTER(Buffers), c_void_p], c_int),
     "lh_get_device_error": ([c_void_p, ctypes.POINTER(c_int)], c_int),
     "lh_launch_count": ([], ctypes.c_ulonglong),
+    "lh_selftest_timeout": ([ctypes.c_longlong, c_void_p, c_void_p], c_int),
     "lh_score_topk_noalloc": ([ctypes.POINTER(Config)] + [c_void_p] * 5, c_int),
 }
 
@@ -189,6 +190,13 @@ def get_device_error(stream=None):
 
 def launch_count() -> int:
     return int(lib().lh_launch_count())
+
+
+def selftest_timeout(limit_cycles: int, gave_up: torch.Tensor, stream=None):
+    """One warp waits, with the kernels' bounded wait, on an mbarrier nothing
+    arrives on; after `limit_cycles` SM cycles it gives up and records
+    LH_ERR_TIMEOUT (detail 900). `gave_up`: a device int32 tensor, set to 1."""
+    _check(lib().lh_selftest_timeout(int(limit_cycles), _p(gave_up), _stream(stream)), "lh_selftest_timeout")
 
 
 # ---------------------------------------------------------------------------
