@@ -57,7 +57,7 @@ typedef enum {
   LH_ERR_SHAPE = 2,      /* sizes outside the supported set (see lh_plan) */
   LH_ERR_ALIGN = 3,      /* a buffer is not 16-byte aligned */
   LH_ERR_DTYPE = 4,      /* unknown dtype */
-  LH_ERR_MODE = 5,       /* unknown accumulation mode */
+  LH_ERR_MODE = 5,       /* unknown accumulation mode or reading (lh_score, lh_ties, lh_order, lh_weight) */
   LH_ERR_WORKSPACE = 6,  /* workspace smaller than plan.ws_bytes */
   LH_ERR_CUDA = 7,       /* a CUDA launch or runtime call failed */
   LH_ERR_TIMEOUT = 8,    /* a bounded device-side wait gave up (reported by lh_get_device_error) */
@@ -80,11 +80,41 @@ typedef enum { LH_BF16 = 0, LH_FP32 = 1 } lh_dtype;
  *                  int-atomic). Sums must stay below 2^31 in magnitude. */
 typedef enum { LH_ACC_FP32 = 0, LH_ACC_FIXED64 = 1 } lh_accum;
 
+/* Readings of points the pages leave open, selectable (value 0 = the reading
+ * the library implements by default). The pages describe the score only as the
+ * l2 norm of the pooled summaries, "bidirectional" over queries and keys
+ * ("Long Context Pre-Training with Lighthouse Attention", §3.1 (ii) and Fig. 2);
+ * the entry order only as sorted by position with causality kept (Fig. 1); the
+ * scatter-back as distributing each output to the positions it represents
+ * (§3.1 (iv)). Ranking uses squared norms where the order is the same. */
+typedef enum {
+  LH_SCORE_MAX = 0,    /* max(|mean_q|^2, |mean_k|^2) */
+  LH_SCORE_K = 1,      /* |mean_k|^2 */
+  LH_SCORE_SUM = 2,    /* |mean_q| + |mean_k| (fp64 square roots, then their sum) */
+  LH_SCORE_PROD = 3    /* |mean_q|^2 * |mean_k|^2 (same order as |mean_q| * |mean_k|) */
+} lh_score;
+typedef enum {
+  LH_TIES_LOW_FIRST = 0,   /* equal scores: lower index first */
+  LH_TIES_HIGH_FIRST = 1   /* equal scores: higher index first */
+} lh_ties;
+typedef enum {
+  LH_ORDER_POST = 0,   /* by last covered token, finer level first (descendants before ancestors) */
+  LH_ORDER_PRE = 1     /* by first covered token, coarser level first (ancestors before descendants) */
+} lh_order;
+typedef enum {
+  LH_WEIGHT_ONE = 0,   /* forward scatter adds every covering entry's row with weight 1 */
+  LH_WEIGHT_MEAN = 1   /* ... with weight 1/p^l (the block-sum backward takes the same weights) */
+} lh_weight;
+
 typedef struct {
   int B, H, N, D;   /* batch, heads, tokens, head dim (D in {64, 128}) */
   int p, L, K;      /* pool factor (>= 2), levels (1..LH_MAX_LEVELS), top-K budget (1..LH_MAX_K) */
   lh_dtype dtype;   /* element type of tokens, pyramid, sub-sequence, outputs */
   lh_accum accum;   /* accumulation mode of lh_scatter / lh_spread */
+  lh_score score;   /* ranking score of pooled entries (lh_score_topk) */
+  lh_ties ties;     /* tie-break of equal scores (lh_score_topk) */
+  lh_order order;   /* entry order of the sub-sequence (lh_score_topk) */
+  lh_weight weight; /* weights of the forward scatter and of its adjoint lh_scatter_bwd */
 } lh_config;
 
 typedef struct {

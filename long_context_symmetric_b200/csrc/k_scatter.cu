@@ -118,7 +118,7 @@ __device__ __forceinline__ void chain_sum(const Geom& g, const float* __restrict
     acc.add(x, WEIGHTED ? (float)(1.0 / den) : 1.f, den, inv);
     if (!(e & 1)) break;          // not expanded: no finer entry covers t
     if (l == 1) {                 // expanded level-1 parent: t itself is in the sub-sequence
-      const int s0 = s - g.p + (t % g.p);
+      const int s0 = (g.order ? s + 1 : s - g.p) + (t % g.p);   // tokens before (post) / after (pre) it
       load8_f32(src + ((size_t)bh * g.S + s0) * g.D + c8 * 8, x);
       acc.add(x, 1.f, 1.0, 1.0);
       break;
@@ -301,7 +301,9 @@ __global__ void __launch_bounds__(256) k_scatter_tree(const float* __restrict__ 
     }
     T* o = out + (size_t)t * tstride;
     if (expd[1]) {                     // the token itself is in the sub-sequence
-      load8_f32(srow + (size_t)(sl1 - g.p + r0) * g.D, x);
+      // the p tokens of an expanded level-1 entry sit right before it
+      // (post-order) or right after it (pre-order)
+      load8_f32(srow + (size_t)((g.order ? sl1 + 1 : sl1 - g.p) + r0) * g.D, x);
       Acc<FIXED> a = acc[1];
       add_level<FIXED, WEIGHTED>(a, x, g, 0);
       Packed<T> q;
@@ -374,7 +376,11 @@ __global__ void __launch_bounds__(256) k_blocksum(const T* __restrict__ dout,
   const int32_t* slot_h = slot + bh * g.E;
 
   // one included entry: write its row and its delta
-  auto emit = [&](int s, const float (&v)[8]) {
+  // scale: the entry's weight in the forward scatter (1, or 1/p^l under LH_WEIGHT_MEAN)
+  auto emit = [&](int s, const float (&v0)[8], float scale) {
+    float v[8];
+#pragma unroll
+    for (int d = 0; d < 8; ++d) v[d] = v0[d] * scale;
     float part = 0.f;
     float ov[8];
     if (live && s >= 0) {
@@ -396,6 +402,9 @@ __global__ void __launch_bounds__(256) k_blocksum(const T* __restrict__ dout,
   };
 
   float acc[LV + 1][8];   // acc[l]: running sum of the open entry of level l (acc[0] unused)
+  float wl[LV + 1];        // weight of a level-l entry in the forward scatter
+#pragma unroll
+  for (int l = 0; l <= LV; ++l) wl[l] = g.weight == LH_WEIGHT_MEAN ? (float)(1.0 / (double)g.pl[l]) : 1.f;
   const long long ngroups = P / p;
   for (long long g1 = 0; g1 < ngroups; ++g1) {
     const long long i1 = (long long)cb * (P / p) + g1;      // level-1 index
@@ -428,13 +437,13 @@ __global__ void __launch_bounds__(256) k_blocksum(const T* __restrict__ dout,
 #pragma unroll
             for (int d = 0; d < 8; ++d) s[d] = __fadd_rn(s[d], x[d]);
           }
-          if (any_tok) emit(tok_in ? s1 - p + c0 + u : -1, x);
+          if (any_tok) emit(tok_in ? (g.order ? s1 + 1 : s1 - p) + c0 + u : -1, x, 1.f);
         }
       }
     }
 #pragma unroll
     for (int d = 0; d < 8; ++d) acc[1][d] = s[d];
-    if (__any_sync(0xffffffffu, e1 >= 0)) emit(e1 >= 0 ? (e1 >> 1) : -1, s);
+    if (__any_sync(0xffffffffu, e1 >= 0)) emit(e1 >= 0 ? (e1 >> 1) : -1, s, wl[1]);
     long long gi = i1;
 #pragma unroll
     for (int l = 2; l <= LV; ++l) {
@@ -449,11 +458,13 @@ __global__ void __launch_bounds__(256) k_blocksum(const T* __restrict__ dout,
       if (pos != p - 1) break;
       gi /= p;
       const int e = live ? __ldg(slot_h + g.off[l] + (int)gi) : -1;
-      if (__any_sync(0xffffffffu, e >= 0)) emit(e >= 0 ? (e >> 1) : -1, acc[l]);
+      if (__any_sync(0xffffffffu, e >= 0)) emit(e >= 0 ? (e >> 1) : -1, acc[l], wl[l]);
     }
   }
 }
 
+// (Token slots: the p tokens of an expanded level-1 entry sit right before its
+// slot in post-order, right after it in pre-order.)
 // Same block sums with the token rows streamed through a shared-memory ring
 // filled by 1-D bulk async copies (one CTA per coarsest block and head group;
 // hg * D / 8 threads, a multiple of 32). PP = p, a compile-time 2, 4 or 8 that
@@ -517,7 +528,11 @@ __global__ void __launch_bounds__(256, 2) k_blocksum_ring(const T* __restrict__ 
     for (int kk = 0; kk < a.ns && kk < nstages; ++kk) issue(kk);
 
   // one included entry: write its row and its delta
-  auto emit = [&](int s, const float (&v)[8]) {
+  // scale: the entry's weight in the forward scatter (1, or 1/p^l under LH_WEIGHT_MEAN)
+  auto emit = [&](int s, const float (&v0)[8], float scale) {
+    float v[8];
+#pragma unroll
+    for (int d = 0; d < 8; ++d) v[d] = v0[d] * scale;
     float part = 0.f;
     float ov[8];
     if (s >= 0) {
@@ -539,6 +554,9 @@ __global__ void __launch_bounds__(256, 2) k_blocksum_ring(const T* __restrict__ 
   };
 
   float acc[LV + 1][8];   // acc[l]: running sum of the open entry of level l (acc[0] unused)
+  float wl[LV + 1];        // weight of a level-l entry in the forward scatter
+#pragma unroll
+  for (int l = 0; l <= LV; ++l) wl[l] = g.weight == LH_WEIGHT_MEAN ? (float)(1.0 / (double)g.pl[l]) : 1.f;
   const long long i1_end = (long long)(cb + 1) * (P / p);
   long long i1 = (long long)cb * (P / p);          // level-1 index of the next group
   int e1n = __ldg(slot_h + g.off[1] + (int)i1);    // its slot entry, fetched one group ahead
@@ -573,11 +591,11 @@ __global__ void __launch_bounds__(256, 2) k_blocksum_ring(const T* __restrict__ 
 #pragma unroll
           for (int d = 0; d < 8; ++d) sum[d] = __fadd_rn(sum[d], x[d]);
         }
-        if (any_tok) emit(tok_in ? s1 - p + u : -1, x);
+        if (any_tok) emit(tok_in ? (g.order ? s1 + 1 : s1 - p) + u : -1, x, 1.f);
       }
 #pragma unroll
       for (int d = 0; d < 8; ++d) acc[1][d] = sum[d];
-      if (__any_sync(0xffffffffu, e1 >= 0)) emit(e1 >= 0 ? (e1 >> 1) : -1, sum);
+      if (__any_sync(0xffffffffu, e1 >= 0)) emit(e1 >= 0 ? (e1 >> 1) : -1, sum, wl[1]);
       long long gi = i1;
 #pragma unroll
       for (int l = 2; l <= LV; ++l) {
@@ -592,7 +610,7 @@ __global__ void __launch_bounds__(256, 2) k_blocksum_ring(const T* __restrict__ 
         if (pos != p - 1) break;
         gi /= p;
         const int e = __ldg(slot_h + g.off[l] + (int)gi);
-        if (__any_sync(0xffffffffu, e >= 0)) emit(e >= 0 ? (e >> 1) : -1, acc[l]);
+        if (__any_sync(0xffffffffu, e >= 0)) emit(e >= 0 ? (e >> 1) : -1, acc[l], wl[l]);
       }
     }
     __syncthreads();                    // every thread is done with this stage
@@ -636,10 +654,16 @@ int grid_for(long long total) {
 
 template <typename T>
 cudaError_t scatter_t(const Geom& g, const float* os, const int32_t* slot, void* o, cudaStream_t s) {
-  if (g.L > 1)
+  if (g.L > 1) {
+    // weights 1 (the default reading) or 1/p^l (LH_WEIGHT_MEAN)
+    if (g.weight == LH_WEIGHT_MEAN)
+      return g.accum == LH_ACC_FIXED64
+                 ? tree_t<T, 1, true>(g, os, os, os, slot, (T*)o, (T*)o, (T*)o, 1, s)
+                 : tree_t<T, 0, true>(g, os, os, os, slot, (T*)o, (T*)o, (T*)o, 1, s);
     return g.accum == LH_ACC_FIXED64
                ? tree_t<T, 1, false>(g, os, os, os, slot, (T*)o, (T*)o, (T*)o, 1, s)
                : tree_t<T, 0, false>(g, os, os, os, slot, (T*)o, (T*)o, (T*)o, 1, s);
+  }
   const long long total = (long long)g.B * g.N * g.H * (g.D / 8);
   if (g.accum == LH_ACC_FIXED64)
     k_scatter<T, 1><<<grid_for(total), 256, 0, s>>>(os, slot, (T*)o, g);

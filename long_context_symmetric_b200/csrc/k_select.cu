@@ -7,8 +7,10 @@
 // holes in the causal sequence).
 //
 // Per level l = L-1 .. 1 (all entries of level L-1 are the first candidates):
-//   score = max(|mean_Q|^2, |mean_K|^2) (fp64, from lh_pool)
-//   the first k_l candidates in the order (score desc, index asc) are expanded.
+//   score = max(|mean_Q|^2, |mean_K|^2) (fp64, from lh_pool); the other
+//   selectable readings: |mean_K|^2, |mean_Q| + |mean_K|, |mean_Q|^2 |mean_K|^2
+//   the first k_l candidates in the order (score desc, index asc; or index
+//   desc under the other tie reading) are expanded.
 //   Only the set matters (the sub-sequence order comes from the tree below),
 //   so for up to 8192 candidates it is found by a most-significant-digit
 //   radix select on the unique key (score bits, then position reversed): ten
@@ -24,7 +26,9 @@
 // descendants) occupies a contiguous run of slots ending at the entry, coarse
 // entries in index order. Subtree sizes are formed bottom-up, run starts
 // top-down; slot = start + size - 1. This equals sorting the entries by
-// (last covered token, level).
+// (last covered token, level). Pre-order (the other order reading): the run
+// starts at the entry, slot = start, children runs from start + 1; this equals
+// sorting by (first covered token, coarser level first).
 //
 // Per-level working arrays (candidate index, expanded flag, rank among the
 // expanded, subtree size, run start) live in the caller's workspace
@@ -43,8 +47,8 @@ struct SelArgs {
 };
 
 __device__ __forceinline__ bool precedes(unsigned long long sa, unsigned pa, unsigned long long sb,
-                                         unsigned pb) {
-  return sa > sb || (sa == sb && pa < pb);
+                                         unsigned pb, bool high_first) {
+  return sa > sb || (sa == sb && (high_first ? pa > pb : pa < pb));
 }
 
 // Block-wide exclusive scan of in[0..n) into out[0..n); returns the total.
@@ -84,7 +88,7 @@ __device__ int block_exclusive_scan(const int* in, int* out, int n, int* warp_to
 
 // Bitonic sort of keys[0..n) (n a power of two) so that index 0 comes first
 // under `precedes`.
-__device__ void bitonic_sort(unsigned long long* sk, unsigned* sp, int n) {
+__device__ void bitonic_sort(unsigned long long* sk, unsigned* sp, int n, bool high_first) {
   for (int size = 2; size <= n; size <<= 1) {
     for (int stride = size >> 1; stride > 0; stride >>= 1) {
       for (int i = threadIdx.x; i < (n >> 1); i += kThreads) {
@@ -93,7 +97,7 @@ __device__ void bitonic_sort(unsigned long long* sk, unsigned* sp, int n) {
         const bool up = (lo & size) == 0;
         const unsigned long long a = sk[lo], b = sk[hi];
         const unsigned pa = sp[lo], pb = sp[hi];
-        const bool sw = up ? precedes(b, pb, a, pa) : precedes(a, pa, b, pb);
+        const bool sw = up ? precedes(b, pb, a, pa, high_first) : precedes(a, pa, b, pb, high_first);
         if (sw) {
           sk[lo] = b; sk[hi] = a;
           sp[lo] = pb; sp[hi] = pa;
@@ -104,18 +108,28 @@ __device__ void bitonic_sort(unsigned long long* sk, unsigned* sp, int n) {
   }
 }
 
+// Score of entry e as an order-preserving 64-bit key (every score is >= 0, so
+// its bit pattern orders like its value). mode: lh_score.
 __device__ __forceinline__ unsigned long long score_bits(const double* sqq, const double* sqk,
-                                                         int e) {
-  const double s = fmax(sqq[e], sqk[e]);
-  return (unsigned long long)__double_as_longlong(s);   // s >= 0: bit order = value order
+                                                         int e, int mode) {
+  const double a = sqq[e], b = sqk[e];
+  double s;
+  switch (mode) {
+    case 1: s = b; break;                                           // |mean_k|^2
+    case 2: s = __dadd_rn(__dsqrt_rn(a), __dsqrt_rn(b)); break;     // |mean_q| + |mean_k|
+    case 3: s = __dmul_rn(a, b); break;                             // |mean_q|^2 |mean_k|^2
+    default: s = fmax(a, b);                                        // max of the squared norms
+  }
+  return (unsigned long long)__double_as_longlong(s);
 }
 
 // Flags fl[q] = 1 for the k (< c <= kChunk) candidates q first in the order
-// (score desc, q asc), 0 for the rest. Key of q: hi = score bits, lo = c-1-q,
-// compared as (hi, lo) descending; keys are unique. hist: 257 ints of shared
-// memory, bc: 2 ints. All threads must call it.
+// (score desc, q asc; q desc if high_first), 0 for the rest. Key of q: hi =
+// score bits, lo = c-1-q (q if high_first), compared as (hi, lo) descending;
+// keys are unique. hist: 257 ints of shared memory, bc: 2 ints. All threads
+// must call it.
 __device__ void radix_select_flags(const double* sq_l, const double* sk_l, const int32_t* cl, int c, int k,
-                                   int32_t* fl, int* hist, int* bc) {
+                                   int score_mode, bool high_first, int32_t* fl, int* hist, int* bc) {
   constexpr int KPT = kChunk / kThreads;
   const int lane = threadIdx.x & 31;
   unsigned long long hi[KPT];
@@ -125,8 +139,8 @@ __device__ void radix_select_flags(const double* sq_l, const double* sk_l, const
   for (int j = 0; j < KPT; ++j) {
     const int q = threadIdx.x + j * kThreads;
     valid[j] = q < c;
-    hi[j] = valid[j] ? score_bits(sq_l, sk_l, cl[q]) : 0ull;
-    lo[j] = valid[j] ? (unsigned)(c - 1 - q) : 0u;
+    hi[j] = valid[j] ? score_bits(sq_l, sk_l, cl[q], score_mode) : 0ull;
+    lo[j] = valid[j] ? (unsigned)(high_first ? q : c - 1 - q) : 0u;
   }
   unsigned long long thi = 0ull;   // chosen digits of the threshold key so far
   unsigned tlo = 0u;
@@ -231,10 +245,13 @@ k_select(const double* __restrict__ sq, int32_t* __restrict__ sel, int32_t* __re
     if (k >= c) {
       for (int q = threadIdx.x; q < c; q += kThreads) fl[q] = 1;
     } else if (c <= kChunk) {
-      radix_select_flags(sq_l, sk_l, cl, c, k, fl, hist, bcast);
+      radix_select_flags(sq_l, sk_l, cl, c, k, g.score, g.ties != 0, fl, hist, bcast);
     } else {
       for (int q = threadIdx.x; q < c; q += kThreads) fl[q] = 0;
-      // chunked top-k: best k stay at the head of the chunk between rounds
+      // chunked top-k: best k stay at the head of the chunk between rounds. With
+      // ties broken towards higher positions, positions are stored + 1 so that
+      // the sentinel (position 0) sorts after every real candidate.
+      const unsigned pos_shift = g.ties ? 1u : 0u;
       int n2 = 1;
       while (n2 < (c < kChunk ? c : kChunk)) n2 <<= 1;
       int next = 0, held = 0;
@@ -244,19 +261,19 @@ k_select(const double* __restrict__ sq, int32_t* __restrict__ sel, int32_t* __re
         for (int i = threadIdx.x; i < room; i += kThreads) {
           if (i < take) {
             const int qpos = next + i;
-            sk[held + i] = score_bits(sq_l, sk_l, cl[qpos]);
-            sp[held + i] = (unsigned)qpos;
+            sk[held + i] = score_bits(sq_l, sk_l, cl[qpos], g.score);
+            sp[held + i] = (unsigned)qpos + pos_shift;
           } else {
             sk[held + i] = 0ull;            // sentinel: after every real candidate
-            sp[held + i] = 0xFFFFFFFFu;
+            sp[held + i] = g.ties ? 0u : 0xFFFFFFFFu;
           }
         }
         __syncthreads();
-        bitonic_sort(sk, sp, n2);
+        bitonic_sort(sk, sp, n2, g.ties != 0);
         next += take;
         held = k;
       }
-      for (int r = threadIdx.x; r < k; r += kThreads) fl[sp[r]] = 1;
+      for (int r = threadIdx.x; r < k; r += kThreads) fl[sp[r] - pos_shift] = 1;
     }
     __syncthreads();
     // rank among expanded (exclusive scan), selection output, next candidates
@@ -310,7 +327,7 @@ k_select(const double* __restrict__ sq, int32_t* __restrict__ sel, int32_t* __re
     int32_t* stc = start + a.lvl_base[l - 1];
     for (int q = threadIdx.x; q < g.c[l]; q += kThreads) {
       if (fl[q]) {
-        int s = stl[q];
+        int s = stl[q] + (g.order ? 1 : 0);   // pre-order: the entry first, then its children's runs
         const int base = rl[q] * p;
         for (int j = 0; j < p; ++j) {
           stc[base + j] = s;
@@ -328,7 +345,7 @@ k_select(const double* __restrict__ sq, int32_t* __restrict__ sel, int32_t* __re
     const int32_t* sl = size + a.lvl_base[l];
     const int32_t* stl = start + a.lvl_base[l];
     for (int q = threadIdx.x; q < g.c[l]; q += kThreads) {
-      const int sidx = stl[q] + sl[q] - 1;
+      const int sidx = g.order ? stl[q] : stl[q] + sl[q] - 1;
       const int e = cl[q];
       map_h[sidx] = (l << 28) | e;
       if (l >= 1) slot_h[g.off[l] + e] = 2 * sidx + (fl[q] ? 1 : 0);

@@ -78,6 +78,9 @@ lh_status make_geom(const lh_config* cfg, Geom* g, lh_plan_t* out) {
   if (!cfg) return LH_ERR_NULL;
   if (cfg->dtype != LH_BF16 && cfg->dtype != LH_FP32) return LH_ERR_DTYPE;
   if (cfg->accum != LH_ACC_FP32 && cfg->accum != LH_ACC_FIXED64) return LH_ERR_MODE;
+  if ((unsigned)cfg->score > LH_SCORE_PROD || (unsigned)cfg->ties > LH_TIES_HIGH_FIRST ||
+      (unsigned)cfg->order > LH_ORDER_PRE || (unsigned)cfg->weight > LH_WEIGHT_MEAN)
+    return LH_ERR_MODE;
   const int B = cfg->B, H = cfg->H, N = cfg->N, D = cfg->D, p = cfg->p, L = cfg->L, K = cfg->K;
   if (B < 1 || H < 1 || N < 1) return LH_ERR_SHAPE;
   if (D != 64 && D != 128) return LH_ERR_SHAPE;
@@ -114,6 +117,10 @@ lh_status make_geom(const lh_config* cfg, Geom* g, lh_plan_t* out) {
   G.E = E;
   G.pow2 = (p & (p - 1)) == 0;
   G.accum = cfg->accum;
+  G.score = cfg->score;
+  G.ties = cfg->ties;
+  G.order = cfg->order;
+  G.weight = cfg->weight;
   *g = G;
   if (out) {
     std::memset(out, 0, sizeof(*out));
@@ -149,7 +156,7 @@ const char* lh_status_string(lh_status s) {
     case LH_ERR_SHAPE: return "unsupported sizes";
     case LH_ERR_ALIGN: return "buffer not 16-byte aligned";
     case LH_ERR_DTYPE: return "unknown dtype";
-    case LH_ERR_MODE: return "unknown accumulation mode";
+    case LH_ERR_MODE: return "unknown accumulation mode or reading";
     case LH_ERR_WORKSPACE: return "workspace too small";
     case LH_ERR_CUDA: return "CUDA launch or runtime error";
     case LH_ERR_TIMEOUT: return "device-side wait timed out";

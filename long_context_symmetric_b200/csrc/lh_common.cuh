@@ -20,6 +20,7 @@ struct Geom {
   long long pl[LH_MAX_LEVELS]; // p^l
   int pow2;                    // p is a power of two (division by p^l is exact scaling)
   int accum;                   // lh_accum
+  int score, ties, order, weight;   // lh_score, lh_ties, lh_order, lh_weight
 };
 
 // Element I/O: 8 consecutive components of a dtype row.

@@ -203,8 +203,23 @@ def sq_norm_pinned(m: np.ndarray) -> np.ndarray:
     return parts[0]
 
 
-def scores_head(means_q, means_k, L: int):
-    """Score of every entry of levels 1..L-1: max of the query and key squared norms (R2).
+def _score(a: np.ndarray, b: np.ndarray, score: str) -> np.ndarray:
+    """One level's ranking score from the query / key squared norms a, b (fp64)."""
+    if score == "max":          # max(|q|^2, |k|^2): the default reading
+        return np.maximum(a, b)
+    if score == "k":            # |k|^2 only
+        return b.copy()
+    if score == "sum":          # |q| + |k|: IEEE square roots, then their sum
+        return np.sqrt(a) + np.sqrt(b)
+    if score == "prod":         # |q|^2 |k|^2, ranks like |q| |k|
+        return a * b
+    raise ValueError(score)
+
+
+def scores_head(means_q, means_k, L: int, score: str = "max"):
+    """Score of every entry of levels 1..L-1 (R2a). Default reading: max of the
+    query and key squared norms; the alternatives kept behind this switch:
+    the key norm alone, the sum of the two norms, their product.
 
     Level 0 is never ranked (only levels >= 1 are candidates for expansion),
     so no level-0 score is formed. Returns (scores, sq_q, sq_k): lists indexed
@@ -212,7 +227,7 @@ def scores_head(means_q, means_k, L: int):
     """
     sq_q = [None] + [sq_norm_pinned(means_q[l]) for l in range(1, L)]
     sq_k = [None] + [sq_norm_pinned(means_k[l]) for l in range(1, L)]
-    scores = [None] + [np.maximum(sq_q[l], sq_k[l]) for l in range(1, L)]
+    scores = [None] + [_score(sq_q[l], sq_k[l], score) for l in range(1, L)]
     return scores, sq_q, sq_k
 
 
@@ -220,13 +235,14 @@ def scores_head(means_q, means_k, L: int):
 # (ii-b) hierarchical top-K, tree descent   [LH] §3.1 stage (ii), Fig. 2 (R1, R3, R5)
 # ----------------------------------------------------------------------------
 
-def select_head(scores, p: int, L: int, K: int):
+def select_head(scores, p: int, L: int, K: int, ties: str = "low"):
     """Top-down descent over the pyramid (parents kept, tree pruned: [LH] Fig. 2, step 3).
 
     Candidates at the coarsest level are all its entries. At each level
     l = L-1..1 the first k_l candidates in the order (score desc, index asc)
-    are expanded; the p children of every expanded entry are the candidates
-    (and included entries) one level down.
+    are expanded (ties="high": index desc, the other tie reading R3); the p
+    children of every expanded entry are the candidates (and included
+    entries) one level down.
 
     Returns (sel, included): sel[l] (l >= 1) is the sorted array of expanded
     indices at level l; included[l] the sorted array of level-l entries that
@@ -241,7 +257,8 @@ def select_head(scores, p: int, L: int, K: int):
     for l in range(L - 1, 0, -1):
         k = min(K, len(cand))
         s = scores[l][cand]
-        order = np.lexsort((cand, -s))       # primary: score desc; then index asc (R3)
+        tie_key = cand if ties == "low" else -cand
+        order = np.lexsort((tie_key, -s))    # primary: score desc; then index asc (R3) or desc
         chosen = np.sort(cand[order[:k]])
         sel[l] = chosen
         cand = (chosen[:, None] * p + np.arange(p)[None, :]).reshape(-1)
@@ -253,8 +270,9 @@ def select_head(scores, p: int, L: int, K: int):
 # (ii-c) ordering: topological sort into one causal sequence   [LH] Fig. 1; [LHT] (R6)
 # ----------------------------------------------------------------------------
 
-def order_head(included, p: int, L: int, N: int):
-    """Order the included entries by (last covered token asc, level asc).
+def order_head(included, p: int, L: int, N: int, order: str = "post"):
+    """Order the included entries by (last covered token asc, level asc); with
+    order="pre" (the other reading, R6) by (first covered token asc, level desc).
 
     Returns (lvl, idx): int64 arrays of length S; slot j holds entry
     (lvl[j], idx[j]). With L = 1 every token is its own entry (S = N).
@@ -267,9 +285,15 @@ def order_head(included, p: int, L: int, N: int):
         ix.append(np.asarray(included[l], dtype=np.int64))
     lv = np.concatenate(lv)
     ix = np.concatenate(ix)
-    end = (ix + 1) * (p ** lv) - 1
-    order = np.lexsort((lv, end))            # primary: end asc; then level asc
-    return lv[order], ix[order]
+    if order == "post":
+        end = (ix + 1) * (p ** lv) - 1
+        perm = np.lexsort((lv, end))         # primary: end asc; then level asc
+    elif order == "pre":
+        start = ix * (p ** lv)
+        perm = np.lexsort((-lv, start))      # primary: start asc; then level desc
+    else:
+        raise ValueError(order)
+    return lv[perm], ix[perm]
 
 
 def gather_head(stored, lvl, idx):
@@ -380,13 +404,16 @@ def scatter_head(rows, lvl, idx, p: int, N: int, weighted: bool, mode: str = "fp
     return out
 
 
-def blocksum_head(g: np.ndarray, lvl, idx, p: int):
-    """Adjoint of the weight-1 scatter: row j = sum of g over the tokens entry j covers."""
+def blocksum_head(g: np.ndarray, lvl, idx, p: int, weighted: bool = False):
+    """Adjoint of the forward scatter: row j = sum of g over the tokens entry j
+    covers (weight 1), divided by p^l when the scatter weights are 1/p^l (R7)."""
     out = np.empty((len(lvl), g.shape[1]), dtype=np.float64)
     for j in range(len(lvl)):
         span = p ** int(lvl[j])
         t0 = int(idx[j]) * span
         out[j] = g[t0:t0 + span].sum(axis=0)
+        if weighted:
+            out[j] /= span
     return out
 
 
@@ -399,12 +426,14 @@ def spread_head(g_rows, lvl, idx, p: int, N: int, mode: str = "fp"):
 # whole path, one (batch, head) pair
 # ----------------------------------------------------------------------------
 
-def forward_head(qh, kh, vh, p: int, L: int, K: int, dtype: str, mode: str = "fp"):
+def forward_head(qh, kh, vh, p: int, L: int, K: int, dtype: str, mode: str = "fp", score: str = "max",
+                 ties: str = "low", order: str = "post", weight: str = "one"):
     """Forward pass for one head: tokens [N, D] x3 -> dict of every intermediate.
 
-    Keys: means_*, stored_*, scores, sq_q, sq_k, sel, included, lvl, idx,
-    qs, ks, vs (sub-sequence), os, lse (attention), o ([N, D] output, fp64,
-    not rounded).
+    score, ties, order, weight select the readings R2a, R3, R6, R7 (defaults:
+    the library's). Keys: means_*, stored_*, scores, sq_q, sq_k, sel,
+    included, lvl, idx, qs, ks, vs (sub-sequence), os, lse (attention), o
+    ([N, D] output, fp64, not rounded), weight.
     """
     N, D = qh.shape
     pl = plan(N, p, L, K)
@@ -412,21 +441,21 @@ def forward_head(qh, kh, vh, p: int, L: int, K: int, dtype: str, mode: str = "fp
     mk, sk_ = pool_head(kh, p, L, dtype)
     mv, sv_ = pool_head(vh, p, L, dtype)
     if L > 1:
-        scores, nq, nk = scores_head(mq, mk, L)
-        sel, included = select_head(scores, p, L, K)
+        scores, nq, nk = scores_head(mq, mk, L, score)
+        sel, included = select_head(scores, p, L, K, ties)
     else:
         scores, nq, nk, sel, included = [None], [None], [None], [None], [None]
-    lvl, idx = order_head(included, p, L, N)
+    lvl, idx = order_head(included, p, L, N, order)
     assert len(lvl) == pl.S
     qs = gather_head(sq_, lvl, idx)
     ks = gather_head(sk_, lvl, idx)
     vs = gather_head(sv_, lvl, idx)
     os_, lse = attention_fwd(qs, ks, vs)
-    o = scatter_head(os_, lvl, idx, p, N, weighted=False, mode=mode)
+    o = scatter_head(os_, lvl, idx, p, N, weighted=(weight == "mean"), mode=mode)
     return dict(means_q=mq, means_k=mk, means_v=mv, stored_q=sq_, stored_k=sk_,
                 stored_v=sv_, scores=scores, sq_q=nq, sq_k=nk, sel=sel,
                 included=included, lvl=lvl, idx=idx, qs=qs, ks=ks, vs=vs,
-                os=os_, lse=lse, o=o, plan=pl)
+                os=os_, lse=lse, o=o, plan=pl, weight=weight)
 
 
 def backward_head(fw: dict, doh: np.ndarray, p: int, mode: str = "fp"):
@@ -439,7 +468,7 @@ def backward_head(fw: dict, doh: np.ndarray, p: int, mode: str = "fp"):
     """
     N = doh.shape[0]
     lvl, idx = fw["lvl"], fw["idx"]
-    dos = blocksum_head(doh, lvl, idx, p)
+    dos = blocksum_head(doh, lvl, idx, p, weighted=(fw.get("weight", "one") == "mean"))
     dqs, dks, dvs = attention_bwd(fw["qs"], fw["ks"], fw["vs"], dos)
     dq = spread_head(dqs, lvl, idx, p, N, mode)
     dk = spread_head(dks, lvl, idx, p, N, mode)
@@ -447,7 +476,7 @@ def backward_head(fw: dict, doh: np.ndarray, p: int, mode: str = "fp"):
     return dict(dos=dos, dqs=dqs, dks=dks, dvs=dvs, dq=dq, dk=dk, dv=dv)
 
 
-def forward(Q, K_, V, p: int, L: int, K: int, dtype: str, mode: str = "fp", heads=None):
+def forward(Q, K_, V, p: int, L: int, K: int, dtype: str, mode: str = "fp", heads=None, **readings):
     """Whole-tensor forward. Q, K_, V: [B, N, H, D] fp64. Returns (O [B,N,H,D], per-head dicts).
 
     ``heads`` optionally restricts the work to a list of (b, h) pairs (the
@@ -458,7 +487,7 @@ def forward(Q, K_, V, p: int, L: int, K: int, dtype: str, mode: str = "fp", head
     per = {}
     pairs = heads if heads is not None else [(b, h) for b in range(B) for h in range(H)]
     for b, h in pairs:
-        fw = forward_head(Q[b, :, h, :], K_[b, :, h, :], V[b, :, h, :], p, L, K, dtype, mode)
+        fw = forward_head(Q[b, :, h, :], K_[b, :, h, :], V[b, :, h, :], p, L, K, dtype, mode, **readings)
         O[b, :, h, :] = fw["o"]
         per[(b, h)] = fw
     return O, per

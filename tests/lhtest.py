@@ -35,10 +35,12 @@ def to64(t: torch.Tensor) -> np.ndarray:
 
 
 class Case:
-    def __init__(self, name, B, H, N, D, dtype, p, L, K, recipe="iid", accum="fp", seed=7):
+    def __init__(self, name, B, H, N, D, dtype, p, L, K, recipe="iid", accum="fp", seed=7, **readings):
         self.name, self.B, self.H, self.N, self.D = name, B, H, N, D
         self.dtype, self.p, self.L, self.K = dtype, p, L, K
         self.recipe, self.accum, self.seed = recipe, accum, seed
+        # score / ties / order / weight readings (absent: the library's defaults)
+        self.readings = readings
 
     def workload(self):
         return synth.Workload(self.name, self.B, self.H, self.N, self.D, self.dtype, self.p, self.L,
@@ -46,7 +48,7 @@ class Case:
 
     def cfg(self):
         return lh.make_config(self.B, self.H, self.N, self.D, self.p, self.L, self.K, self.dtype,
-                              self.accum)
+                              self.accum, **self.readings)
 
     def __repr__(self):
         return self.name
@@ -98,7 +100,7 @@ def compare_head(case: Case, res, q, k, v, do, b: int, h: int, check_bwd=True):
     pl = lh.plan(case.cfg())
     ws = res["ws"]
     qh, kh, vh = (to64(x[b, :, h, :]) for x in (q, k, v))
-    fw = orc.forward_head(qh, kh, vh, case.p, case.L, case.K, dt, case.accum)
+    fw = orc.forward_head(qh, kh, vh, case.p, case.L, case.K, dt, case.accum, **case.readings)
     assert fw["plan"].S == pl.S
     # (i) pyramid and squared norms: bit-exact
     for l in range(1, case.L):

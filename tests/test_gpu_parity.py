@@ -30,6 +30,21 @@ SMALL = [
     Case("chunked_topk", 1, 1, 131072, 64, "bf16", 2, 2, 300),                  # 65536 candidates: chunked sort
 ]
 
+# the alternative readings of the open points (score formula, tie-break, entry
+# order, scatter weights), each against the oracle run with the same reading
+READINGS = [
+    Case("score_k", 1, 2, 4096, 128, "bf16", 4, 4, 40, score="k"),
+    Case("score_sum", 1, 2, 4096, 128, "bf16", 4, 4, 40, score="sum"),
+    Case("score_prod", 1, 2, 4096, 128, "bf16", 4, 4, 40, score="prod"),
+    Case("ties_high", 1, 2, 4096, 128, "bf16", 4, 5, 64, recipe="codebook", accum="fixed", ties="high"),
+    Case("ties_high_chunked", 1, 1, 65536, 64, "bf16", 2, 2, 200, recipe="codebook", ties="high"),
+    Case("order_pre", 1, 2, 4096, 128, "bf16", 4, 4, 40, order="pre"),
+    Case("weight_mean", 1, 2, 4096, 128, "bf16", 4, 4, 40, weight="mean"),
+    Case("weight_mean_p3_fixed", 1, 2, 333, 128, "bf16", 3, 3, 5, accum="fixed", weight="mean"),
+    Case("all_alternatives", 2, 3, 2048, 64, "bf16", 4, 3, 37, recipe="token_scale", score="sum",
+         ties="high", order="pre", weight="mean"),
+]
+
 
 def _inputs(case, device=DEV):
     w = case.workload()
@@ -40,6 +55,15 @@ def _inputs(case, device=DEV):
 
 @pytest.mark.parametrize("case", SMALL, ids=repr)
 def test_small_cases_all_heads(case):
+    q, k, v, do = _inputs(case)
+    res = run_gpu(case, q, k, v, do)
+    for b in range(case.B):
+        for h in range(case.H):
+            compare_head(case, res, q, k, v, do, b, h)
+
+
+@pytest.mark.parametrize("case", READINGS, ids=repr)
+def test_alternative_readings_all_heads(case):
     q, k, v, do = _inputs(case)
     res = run_gpu(case, q, k, v, do)
     for b in range(case.B):
