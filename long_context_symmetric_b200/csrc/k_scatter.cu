@@ -529,14 +529,20 @@ __global__ void __launch_bounds__(256, 2) k_blocksum_ring(const T* __restrict__ 
 
   // one included entry: write its row and its delta
   // scale: the entry's weight in the forward scatter (1, or 1/p^l under LH_WEIGHT_MEAN)
-  auto emit = [&](int s, const float (&v0)[8], float scale) {
+  // ov_pre: the entry's os row when already loaded (else it is loaded here)
+  auto emit = [&](int s, const float (&v0)[8], float scale, const float* ov_pre) {
     float v[8];
 #pragma unroll
     for (int d = 0; d < 8; ++d) v[d] = v0[d] * scale;
     float part = 0.f;
     float ov[8];
     if (s >= 0) {
-      load8_f32(os + ((size_t)bh * g.S + s) * g.D + chunk * 8, ov);
+      if (ov_pre) {
+#pragma unroll
+        for (int d = 0; d < 8; ++d) ov[d] = ov_pre[d];
+      } else {
+        load8_f32(os + ((size_t)bh * g.S + s) * g.D + chunk * 8, ov);
+      }
       // delta from the stored (rounded) dos: the values the backward's dP uses
 #pragma unroll
       for (int d = 0; d < 8; ++d)
@@ -571,6 +577,9 @@ __global__ void __launch_bounds__(256, 2) k_blocksum_ring(const T* __restrict__ 
     for (int u0 = 0; u0 < nt; u0 += p, ++i1) {
       const int e1 = e1n;
       if (i1 + 1 < i1_end) e1n = __ldg(slot_h + g.off[1] + (int)(i1 + 1));
+      // the level-1 entry's os row, loaded now so that its latency overlaps the sums
+      float ov1[8];
+      if (e1 >= 0) load8_f32(os + ((size_t)bh * g.S + (e1 >> 1)) * g.D + chunk * 8, ov1);
       typename Vec8<T>::Raw raw[p];
 #pragma unroll
       for (int u = 0; u < p; ++u)
@@ -591,11 +600,11 @@ __global__ void __launch_bounds__(256, 2) k_blocksum_ring(const T* __restrict__ 
 #pragma unroll
           for (int d = 0; d < 8; ++d) sum[d] = __fadd_rn(sum[d], x[d]);
         }
-        if (any_tok) emit(tok_in ? (g.order ? s1 + 1 : s1 - p) + u : -1, x, 1.f);
+        if (any_tok) emit(tok_in ? (g.order ? s1 + 1 : s1 - p) + u : -1, x, 1.f, nullptr);
       }
 #pragma unroll
       for (int d = 0; d < 8; ++d) acc[1][d] = sum[d];
-      if (__any_sync(0xffffffffu, e1 >= 0)) emit(e1 >= 0 ? (e1 >> 1) : -1, sum, wl[1]);
+      if (__any_sync(0xffffffffu, e1 >= 0)) emit(e1 >= 0 ? (e1 >> 1) : -1, sum, wl[1], ov1);
       long long gi = i1;
 #pragma unroll
       for (int l = 2; l <= LV; ++l) {
@@ -610,7 +619,7 @@ __global__ void __launch_bounds__(256, 2) k_blocksum_ring(const T* __restrict__ 
         if (pos != p - 1) break;
         gi /= p;
         const int e = __ldg(slot_h + g.off[l] + (int)gi);
-        if (__any_sync(0xffffffffu, e >= 0)) emit(e >= 0 ? (e >> 1) : -1, acc[l], wl[l]);
+        if (__any_sync(0xffffffffu, e >= 0)) emit(e >= 0 ? (e >> 1) : -1, acc[l], wl[l], nullptr);
       }
     }
     __syncthreads();                    // every thread is done with this stage

@@ -144,6 +144,19 @@ def test_autograd_wrapper_matches_stagewise():
     assert torch.equal(qg.grad, res["dq"]) and torch.equal(kg.grad, res["dk"]) and torch.equal(vg.grad, res["dv"])
 
 
+def test_full_size_alternative_readings_sampled_heads():
+    """The 98K workload (D = 64, 4 levels) with every alternative reading at once,
+    at full size: the first and last heads against the oracle."""
+    w = synth.WORKLOADS["ctx98k"]
+    case = Case("ctx98k_alternatives", w.B, w.H, w.N, w.D, w.dtype, w.p, w.L, w.K, w.recipe, w.mode, w.seed,
+                score="sum", ties="high", order="pre", weight="mean")
+    q, k, v = synth.make_inputs(w, device=DEV)      # the same inputs as the default-reading run
+    do = synth.make_dout(w, device=DEV)
+    res = run_gpu(case, q, k, v, do)
+    for (b, h) in [(0, 0), (w.B - 1, w.H - 1)]:
+        compare_head(case, res, q, k, v, do, b, h)
+
+
 @pytest.mark.parametrize("name", ["ctx98k", "ties131k", "ctx512k"])
 def test_full_size_workloads_sampled_heads(name):
     """Full-size workloads in the launch configuration the bench uses; the oracle
