@@ -26,14 +26,17 @@
 // (an infinite operand times any value, summed in fp32, stays inf or NaN), so
 // the epilogues check their fp32 results and report LH_ERR_DEVICE, detail 101.
 //
-// Pipeline (tensor core order per streamed tile t): dK/dV X(t+1), acc(t),
-// Y(t+1); dQ X(t+1), Y(t+1), acc(t). The compute warps copy X(t) into
+// Pipeline (tensor core order per streamed tile t): dK/dV X(t+1), dV(t),
+// dK(t), Y(t+1); dQ X(t+1), Y(t+1), acc(t). The compute warps copy X(t) into
 // registers and release it at once, so X(t+1) runs while they exponentiate;
-// they read Y(t) and write the fp16 operands of acc(t) into Y's columns, so in
-// the dK/dV kernel (whose TMEM holds two accumulators) Y(t+1) follows acc(t),
-// while the dQ kernel has a second Y buffer and computes Y(t+1) during the
-// compute warps' work on tile t (tcgen05.mma ops issued by one thread execute
-// in order, which orders every reuse of a TMEM column). All score MMAs are
+// they read Y(t) and write the fp16 operands of the accumulating MMAs into
+// Y's columns. In the dK/dV kernel (whose TMEM holds two accumulators) Y(t+1)
+// must follow dK(t) and dV(t); P^T is stored before dS^T is formed and has its
+// own barrier, so dV(t) runs during that work and only dK(t) and Y(t+1) lie
+// between one tile's dS^T and the next. The dQ kernel has a second Y buffer
+// and computes Y(t+1) during the compute warps' work on tile t (tcgen05.mma
+// ops issued by one thread execute in order, which orders every reuse of a
+// TMEM column). All score MMAs are
 // full 128 x 128 tiles: N = 64 halves run at about two thirds of the rate and
 // lose more when the compute warps use TMEM at the same time (measured).
 // Streamed tiles come through a TMA ring whose two operands have their own
@@ -89,7 +92,7 @@ struct BwdLayout {
 // K_j in dq), o = 1 the operand B_t (dO_i in dkdv, V_j in dq).
 struct BwdBars {
   uint64_t fix_full, ring_full[kMaxStages][2], ring_empty[kMaxStages][2];
-  uint64_t x_full, y_full[2], x_free, ds_ready, done, drain;   // y_full[b]: Y buffer b
+  uint64_t x_full, y_full[2], x_free, p_ready, ds_ready, done, drain;   // y_full[b]: Y buffer b
   uint32_t tmem_base;
   Abort abort;
 };
@@ -108,6 +111,7 @@ __device__ __forceinline__ void bwd_setup(BwdBars* bars, int warp) {
     mbar_init(&bars->y_full[0], 1);
     mbar_init(&bars->y_full[1], 1);
     mbar_init(&bars->x_free, kComputeWarps);     // one arrival per compute warp
+    mbar_init(&bars->p_ready, kComputeWarps);    // dkdv: P^T stored
     mbar_init(&bars->ds_ready, kComputeWarps);
     mbar_init(&bars->done, 1);
     mbar_init(&bars->drain, 1);
@@ -181,12 +185,13 @@ __device__ void bwd_produce(uint8_t* sm, BwdBars* bars, const CUtensorMap* f0, c
 // MMA issuer shared by both kernels. For streamed tile t:
 //   X(t) = F0 * A_t^T -> cols 0..127,  Y(t) = F1 * B_t^T -> Y buffer of t
 //   (dkdv: cols 128..255; dq: buffer t & 1 at 128 + 128 (t & 1)),
-//   acc(t), A operand from that Y buffer (fp16 pairs; chunk c = 32 columns of
-//   the tile, its first 16 packed columns hold P^T / dS_hi, the next 16 dS^T /
-//   dS_lo):
-//     dkdv (TWO_ACC): dK += dS^T A_t, then dV += P^T B_t
+//   the accumulating MMAs, A operand from that Y buffer (fp16 pairs; chunk
+//   c = 32 columns of the tile, its first 16 packed columns hold P^T / dS_hi,
+//   the next 16 dS^T / dS_lo):
+//     dkdv (TWO_ACC): dV += P^T B_t once P^T is stored (p_ready), then
+//                     dK += dS^T A_t once dS^T is (ds_ready)
 //     dq:             dQ += dS_hi A_t + dS_lo A_t
-// Issue order: X(0), Y(0), then per t: dkdv X(t+1), acc(t), Y(t+1);
+// Issue order: X(0), Y(0), then per t: dkdv X(t+1), dV(t), dK(t), Y(t+1);
 // dq X(t+1), Y(t+1), acc(t).
 // Run by the whole (converged) MMA warp: every lane takes the same waits and
 // branches, one elected lane issues the MMAs and commits. Shared-memory
@@ -227,22 +232,20 @@ __device__ void bwd_mma(uint8_t* sm, BwdBars* bars, uint32_t tbase, int n, volat
       if (!TWO_ACC) umma_commit(&bars->ring_empty[t % NSTB][1]);   // dq: V_j has no other reader
     }
   };
+  // accumulating MMAs: 16-row slice kk of the streamed tiles (MN-major
+  // descriptor + kk * 2048 bytes) and its packed operand columns in the Y
+  // buffer at acol(kk)
+  auto acol = [](int kk) -> uint32_t { return 32 * (kk >> 1) + 8 * (kk & 1); };
   auto issue_acc = [&](int t) {
-    // 16-row slice kk of the streamed tiles: MN-major descriptor + kk * 2048 bytes;
-    // its packed operand columns in the Y buffer at acol(kk)
-    const uint64_t bA = dAm + (uint64_t)((t % NSTA) * OPB16), bB = dBm + (uint64_t)((t % NSTB) * OPB16);
+    const uint64_t bA = dAm + (uint64_t)((t % NSTA) * OPB16);
     const uint32_t y = tY(t);
-    auto acol = [](int kk) -> uint32_t { return 32 * (kk >> 1) + 8 * (kk & 1); };
     if (!leader) return;
     if (TWO_ACC) {
+      // dK(t); dV(t) went ahead in issue_dv
 #pragma unroll
       for (int kk = 0; kk < kT / 16; ++kk)
         umma_f16_ts(tAcc1, y + acol(kk) + 16, bA + kk * 128, IDACC, (t > 0 || kk > 0) ? 1u : 0u);
       umma_commit(&bars->ring_empty[t % NSTA][0]);
-#pragma unroll
-      for (int kk = 0; kk < kT / 16; ++kk)
-        umma_f16_ts(tAcc0, y + acol(kk), bB + kk * 128, IDACC, (t > 0 || kk > 0) ? 1u : 0u);
-      umma_commit(&bars->ring_empty[t % NSTB][1]);
     } else {
 #pragma unroll
       for (int kk = 0; kk < kT / 16; ++kk) {
@@ -251,6 +254,15 @@ __device__ void bwd_mma(uint8_t* sm, BwdBars* bars, uint32_t tbase, int n, volat
       }
       umma_commit(&bars->ring_empty[t % NSTA][0]);
     }
+  };
+  auto issue_dv = [&](int t) {
+    const uint64_t bB = dBm + (uint64_t)((t % NSTB) * OPB16);
+    const uint32_t y = tY(t);
+    if (!leader) return;
+#pragma unroll
+    for (int kk = 0; kk < kT / 16; ++kk)
+      umma_f16_ts(tAcc0, y + acol(kk), bB + kk * 128, IDACC, (t > 0 || kk > 0) ? 1u : 0u);
+    umma_commit(&bars->ring_empty[t % NSTB][1]);
   };
   auto wait = [&](uint64_t* bar, uint32_t parity, int site) -> bool {
     return __all_sync(0xffffffffu, mbar_wait(bar, parity, ab, err, site));
@@ -276,6 +288,11 @@ __device__ void bwd_mma(uint8_t* sm, BwdBars* bars, uint32_t tbase, int n, volat
         if (!ring_wait(t + 1, 1)) { ok = false; break; }
         issue_y(t + 1);
       }
+    }
+    if (TWO_ACC) {
+      if (!wait(&bars->p_ready, t & 1, 22)) { ok = false; break; }
+      tc_fence_after();
+      issue_dv(t);
     }
     if (!wait(&bars->ds_ready, t & 1, 15)) { ok = false; break; }
     tc_fence_after();
@@ -325,10 +342,16 @@ __device__ __forceinline__ void p_chunk_t(uint32_t (&s)[32], const float* nl2, f
   }
 }
 
-// dS^T = P^T o (dP^T - delta) for 32 columns; P^T and dS^T as fp16 pairs.
-// ndl holds -delta of the 32 query columns.
+// P^T of 32 columns as fp16 pairs.
+__device__ __forceinline__ void pack_h2(const uint32_t (&p)[32], uint32_t (&pk)[16]) {
+#pragma unroll
+  for (int e = 0; e < 32; e += 2) pk[e >> 1] = h2_bits(__float22half2_rn(f2(p[e], p[e + 1])));
+}
+
+// dS^T = P^T o (dP^T - delta) for 32 columns, as fp16 pairs. ndl holds -delta
+// of the 32 query columns.
 __device__ __forceinline__ void ds_chunk_t(const uint32_t (&p)[32], const uint32_t (&dp)[32], const float* ndl,
-                                           uint32_t (&pk)[16], uint32_t (&dk)[16]) {
+                                           uint32_t (&dk)[16]) {
 #pragma unroll
   for (int e = 0; e < 32; e += 4) {
     const float4 b = *reinterpret_cast<const float4*>(ndl + e);
@@ -336,9 +359,7 @@ __device__ __forceinline__ void ds_chunk_t(const uint32_t (&p)[32], const uint32
     for (int u = 0; u < 4; u += 2) {
       const float2 pp = f2(p[e + u], p[e + u + 1]);
       const float2 d = __fadd2_rn(f2(dp[e + u], dp[e + u + 1]), u ? make_float2(b.z, b.w) : make_float2(b.x, b.y));
-      const __half2 ds = __float22half2_rn(__fmul2_rn(pp, d));
-      pk[(e + u) >> 1] = h2_bits(__float22half2_rn(pp));
-      dk[(e + u) >> 1] = h2_bits(ds);
+      dk[(e + u) >> 1] = h2_bits(__float22half2_rn(__fmul2_rn(pp, d)));
     }
   }
 }
@@ -453,19 +474,25 @@ k_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CU
       ok = __all_sync(0xffffffffu, mbar_wait(&bars->y_full[0], t & 1, ab, err, 17));
       if (!ok) continue;
       tc_fence_after();
-      // dP^T: both 32-column chunks, then P^T / dS^T as fp16 into the chunk's
-      // own (already read) columns: P^T at +0..15, dS^T at +16..31
-      uint32_t d0[32], d1[32], pk[16], dk[16];
+      // dP^T: both 32-column chunks, then fp16 pairs into the chunk's own
+      // (already read) columns: P^T at +0..15 first, so that dV(t) runs while
+      // dS^T is formed, then dS^T at +16..31
+      uint32_t d0[32], d1[32], pk[16];
       tmem_ld32(cY, d0);
       tmem_ld32(cY + 32, d1);
       tmem_wait_ld_regs(d0);
       reg_fence32(d1);
-      ds_chunk_t(p0, d0, ndl, pk, dk);
+      pack_h2(p0, pk);
       tmem_st16(cY, pk);
-      tmem_st16(cY + 16, dk);
-      ds_chunk_t(p1, d1, ndl + 32, pk, dk);
+      pack_h2(p1, pk);
       tmem_st16(cY + 32, pk);
-      tmem_st16(cY + 48, dk);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive_warp(&bars->p_ready);
+      ds_chunk_t(p0, d0, ndl, pk);
+      tmem_st16(cY + 16, pk);
+      ds_chunk_t(p1, d1, ndl + 32, pk);
+      tmem_st16(cY + 48, pk);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive_warp(&bars->ds_ready);
