@@ -58,8 +58,8 @@ def workload_desc(w):
 # None when one of them changes.
 DRAM_TRAFFIC = {
     "ctx512k": {
-        "attn_bwd": None,
-        "attn_fwd": 8 * (39.371776e6 + 0.356352e6),
+        "attn_bwd": 8 * (52.885504e6 + 8.821760e6 + 52.882688e6 + 2.786560e6),   # dK/dV + dQ kernels
+        "attn_fwd": 8 * (39.371776e6 + 0.552192e6),
     },
 }
 
