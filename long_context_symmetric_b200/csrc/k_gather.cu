@@ -10,54 +10,73 @@
 // magnitude above 65504 is reported as LH_ERR_DEVICE, detail 102). fp16 keeps
 // 11 significant bits for the attention's P and dS operands where bf16 keeps 8.
 // Reading 16 bytes per thread (8 bf16 -> 8 fp16, or 4 fp32); consecutive
-// threads cover a row, so stores are fully coalesced.
+// threads cover a row, so loads of a row and all stores are coalesced.
+#include <algorithm>
+
 #include "lh_common.cuh"
 
 namespace lh {
 namespace {
 
-template <bool TO_F16>
+// One CTA covers kU * RPB rows of one (b, h) at a time and one of q / k / v
+// (grid.y strides over b * H + h, grid.z = tensor). VPR = 2^LG threads per
+// row, so each thread moves kU independent 16-byte vectors (all loads in
+// flight before the stores) and no per-element index needs a division.
+constexpr int kU = 4;
+
+template <bool TO_F16, int LG>
 __global__ void __launch_bounds__(256) k_gather(const uint4* __restrict__ q, const uint4* __restrict__ k,
                                                 const uint4* __restrict__ v, const uint4* __restrict__ pq,
                                                 const uint4* __restrict__ pk, const uint4* __restrict__ pv,
                                                 const int32_t* __restrict__ map, uint4* __restrict__ qs,
                                                 uint4* __restrict__ ks, uint4* __restrict__ vs, Geom g,
-                                                int vpr /* 16-byte vectors per row */, int* err) {
-  const long long rows = (long long)g.B * g.H * g.S;
-  const long long total = rows * vpr;
-  const int tensor = blockIdx.y;
+                                                int* err) {
+  constexpr int VPR = 1 << LG, RPB = 256 >> LG;
+  const int tensor = blockIdx.z;
   const uint4* x = tensor == 0 ? q : (tensor == 1 ? k : v);
   const uint4* px = tensor == 0 ? pq : (tensor == 1 ? pk : pv);
   uint4* xs = tensor == 0 ? qs : (tensor == 1 ? ks : vs);
+  const int c = threadIdx.x & (VPR - 1);
+  const int s0 = blockIdx.x * (RPB * kU) + (threadIdx.x >> LG);
   bool big = false;
-  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
-       i += (long long)gridDim.x * blockDim.x) {
-    const long long row = i / vpr;
-    const int c = (int)(i - row * vpr);
-    const long long bh = row / g.S;
-    const int e = __ldg(map + row);
-    const int l = map_level(e), idx = map_index(e);
-    const uint4* src;
-    if (l == 0) {
-      const long long b = bh / g.H, h = bh - b * g.H;
-      src = x + ((b * g.N + idx) * g.H + h) * vpr;
-    } else {
-      src = px + (bh * g.E + g.off[l] + idx) * vpr;
-    }
-    const uint4 val = __ldg(src + c);
-    if (TO_F16) {
-      const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&val);
-      uint4 hv;
-      __half2* h2 = reinterpret_cast<__half2*>(&hv);
+  for (int bh = blockIdx.y; bh < g.B * g.H; bh += gridDim.y) {
+    const int b = bh / g.H, h = bh - b * g.H;
+    const int32_t* mrow = map + (size_t)bh * g.S;
+    const uint4* xrow = x + ((size_t)b * g.N * g.H + h) * VPR + c;     // + token * H * VPR
+    const uint4* prow = px + (size_t)bh * g.E * VPR + c;               // + entry * VPR
+    uint4* out = xs + (size_t)bh * g.S * VPR + c;
+    int e[kU];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const float2 f = __bfloat1622float2(b2[u]);
-        big |= !(fabsf(f.x) <= kHalfMax) || !(fabsf(f.y) <= kHalfMax);
-        h2[u] = __float22half2_rn(f);
+    for (int u = 0; u < kU; ++u) {
+      const int s = s0 + u * RPB;
+      e[u] = s < g.S ? __ldg(mrow + s) : -1;
+    }
+    uint4 val[kU];
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      if (e[u] < 0) continue;
+      const int l = map_level(e[u]), idx = map_index(e[u]);
+      const uint4* src = l == 0 ? xrow + (size_t)idx * g.H * VPR : prow + (size_t)(g.off[l] + idx) * VPR;
+      val[u] = __ldg(src);
+    }
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      if (e[u] < 0) continue;
+      uint4* o = out + (size_t)(s0 + u * RPB) * VPR;
+      if (TO_F16) {
+        const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&val[u]);
+        uint4 hv;
+        __half2* h2 = reinterpret_cast<__half2*>(&hv);
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+          const float2 f = __bfloat1622float2(b2[w]);
+          big |= !(fabsf(f.x) <= kHalfMax) || !(fabsf(f.y) <= kHalfMax);
+          h2[w] = __float22half2_rn(f);
+        }
+        *o = hv;
+      } else {
+        *o = val[u];
       }
-      xs[i] = hv;
-    } else {
-      xs[i] = val;
     }
   }
   if (TO_F16 && big) report_error(err, LH_ERR_DEVICE, 102);
@@ -68,20 +87,23 @@ __global__ void __launch_bounds__(256) k_gather(const uint4* __restrict__ q, con
 cudaError_t launch_gather(const Geom& g, lh_dtype dt, const void* q, const void* k, const void* v,
                           const void* pq, const void* pk, const void* pv, const int32_t* map,
                           void* qs, void* ks, void* vs, int* err, cudaStream_t s) {
+  if (g.S == 0 || g.B * g.H == 0) return cudaSuccess;
   const int esz = dt == LH_BF16 ? 2 : 4;
-  const int vpr = g.D * esz / 16;
-  const long long total = (long long)g.B * g.H * g.S * vpr;
-  long long blocks = (total + 255) / 256;
-  if (blocks > 148 * 16) blocks = 148 * 16;
-  dim3 grid((unsigned)blocks, 3);
-  if (dt == LH_BF16)
-    k_gather<true><<<grid, 256, 0, s>>>((const uint4*)q, (const uint4*)k, (const uint4*)v,
-                                        (const uint4*)pq, (const uint4*)pk, (const uint4*)pv, map,
-                                        (uint4*)qs, (uint4*)ks, (uint4*)vs, g, vpr, err);
-  else
-    k_gather<false><<<grid, 256, 0, s>>>((const uint4*)q, (const uint4*)k, (const uint4*)v,
-                                         (const uint4*)pq, (const uint4*)pk, (const uint4*)pv, map,
-                                         (uint4*)qs, (uint4*)ks, (uint4*)vs, g, vpr, err);
+  const int vpr = g.D * esz / 16;                  // 8, 16 or 32 (D = 64 or 128)
+  const int lg = vpr == 8 ? 3 : (vpr == 16 ? 4 : 5);
+  const int rows_per_cta = (256 / vpr) * kU;
+  dim3 grid((unsigned)((g.S + rows_per_cta - 1) / rows_per_cta), (unsigned)std::min(g.B * g.H, 65535), 3);
+  const uint4 *q4 = (const uint4*)q, *k4 = (const uint4*)k, *v4 = (const uint4*)v;
+  const uint4 *pq4 = (const uint4*)pq, *pk4 = (const uint4*)pk, *pv4 = (const uint4*)pv;
+  uint4 *qs4 = (uint4*)qs, *ks4 = (uint4*)ks, *vs4 = (uint4*)vs;
+#define LH_GATHER(F16, LG) \
+  k_gather<F16, LG><<<grid, 256, 0, s>>>(q4, k4, v4, pq4, pk4, pv4, map, qs4, ks4, vs4, g, err)
+  if (dt == LH_BF16) {
+    if (lg == 3) LH_GATHER(true, 3); else LH_GATHER(true, 4);
+  } else {
+    if (lg == 4) LH_GATHER(false, 4); else LH_GATHER(false, 5);
+  }
+#undef LH_GATHER
   count_launch();
   return cudaGetLastError();
 }
