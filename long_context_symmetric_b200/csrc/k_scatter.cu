@@ -589,8 +589,17 @@ __global__ void __launch_bounds__(256, 2) k_blocksum_ring(const T* __restrict__ 
       // tokens are emitted only where some lane of the warp has them included
       const bool any_tok = __any_sync(0xffffffffu, tok_in);
       float sum[8];
+      // the tokens' os rows, loaded TB at a time so that their latencies overlap
+      // (fp32 rows of dout take twice the registers: smaller batches)
+      constexpr int TB = p < 4 ? p : (sizeof(T) == 2 ? 4 : 2);
+      const int tok0 = g.order ? s1 + 1 : s1 - p;
+      float ovt[TB][8];
 #pragma unroll
       for (int u = 0; u < p; ++u) {
+        if (u % TB == 0 && tok_in) {
+#pragma unroll
+          for (int w = 0; w < TB; ++w) load8_f32(os + ((size_t)bh * g.S + tok0 + u + w) * g.D + chunk * 8, ovt[w]);
+        }
         float x[8];
         Vec8<T>::raw_f32(raw[u], x);
         if (u == 0) {
@@ -600,7 +609,7 @@ __global__ void __launch_bounds__(256, 2) k_blocksum_ring(const T* __restrict__ 
 #pragma unroll
           for (int d = 0; d < 8; ++d) sum[d] = __fadd_rn(sum[d], x[d]);
         }
-        if (any_tok) emit(tok_in ? (g.order ? s1 + 1 : s1 - p) + u : -1, x, 1.f, nullptr);
+        if (any_tok) emit(tok_in ? tok0 + u : -1, x, 1.f, ovt[u % TB]);
       }
 #pragma unroll
       for (int d = 0; d < 8; ++d) acc[1][d] = sum[d];
