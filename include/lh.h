@@ -32,7 +32,14 @@
  *   squared norms sq                       [2][B][H][E]   double ([0]: query, [1]: key)
  *   selection sel                          [B][H][L-1][K] int32 (row l-1: level l)
  *   gather map                             [B][H][S]      int32, (level << 28) | index
- *   slot table                             [B][H][E]      int32, 2*slot + expanded, or -1
+ *   slot table                             [B][H][E]      int32, per entry of levels >= 1:
+ *                                                         -1: not a candidate (pruned);
+ *                                                         2*s: in the sub-sequence at slot s;
+ *                                                         2*s + 1: expanded, and under
+ *                                                         LH_INCL_NESTED in the sub-sequence
+ *                                                         at slot s; under LH_INCL_PARTITION
+ *                                                         not in it, s = the first slot of
+ *                                                         its descendants' run
  *   sub-sequence qs, ks, vs, and dos       [B][H][S][D]   attention operand type: fp16 for
  *                                                         bf16 I/O, fp32 for fp32 I/O
  *   attention out os, grads dqs, dks, dvs  [B][H][S][D]   float
@@ -57,7 +64,8 @@ typedef enum {
   LH_ERR_SHAPE = 2,      /* sizes outside the supported set (see lh_plan) */
   LH_ERR_ALIGN = 3,      /* a buffer is not 16-byte aligned */
   LH_ERR_DTYPE = 4,      /* unknown dtype */
-  LH_ERR_MODE = 5,       /* unknown accumulation mode or reading (lh_score, lh_ties, lh_order, lh_weight) */
+  LH_ERR_MODE = 5,       /* unknown accumulation mode or reading (lh_score, lh_ties, lh_order, lh_weight,
+                            lh_inclusion) */
   LH_ERR_WORKSPACE = 6,  /* workspace smaller than plan.ws_bytes */
   LH_ERR_CUDA = 7,       /* a CUDA launch or runtime call failed */
   LH_ERR_TIMEOUT = 8,    /* a bounded device-side wait gave up (reported by lh_get_device_error) */
@@ -105,6 +113,11 @@ typedef enum {
   LH_WEIGHT_ONE = 0,   /* forward scatter adds every covering entry's row with weight 1 */
   LH_WEIGHT_MEAN = 1   /* ... with weight 1/p^l (the block-sum backward takes the same weights) */
 } lh_weight;
+typedef enum {
+  LH_INCL_NESTED = 0,    /* expanded entries stay in the sub-sequence (parents kept: Fig. 2) */
+  LH_INCL_PARTITION = 1  /* expanded entries leave it: the included entries tile the tokens, each
+                            token covered exactly once (the order readings then coincide) */
+} lh_inclusion;
 
 typedef struct {
   int B, H, N, D;   /* batch, heads, tokens, head dim (D in {64, 128}) */
@@ -115,6 +128,7 @@ typedef struct {
   lh_ties ties;     /* tie-break of equal scores (lh_score_topk) */
   lh_order order;   /* entry order of the sub-sequence (lh_score_topk) */
   lh_weight weight; /* weights of the forward scatter and of its adjoint lh_scatter_bwd */
+  lh_inclusion inclusion; /* whether expanded entries stay in the sub-sequence (lh_plan, lh_score_topk) */
 } lh_config;
 
 typedef struct {
@@ -135,10 +149,12 @@ const char* lh_status_string(lh_status s);
 
 /* Sizes of one problem. Pure host function, no CUDA call.
  * Source: [LH] §1 size law S = O(LpK + N/p^(L-1)) under the descent reading:
- * c_{L-1} = n_{L-1}; k_l = min(K, c_l); c_{l-1} = p * k_l.
+ * candidates m_{L-1} = n_{L-1}; k_l = min(K, m_l); m_{l-1} = p * k_l; included
+ * c_l = m_l (LH_INCL_NESTED) or m_l - k_l for l >= 1 (LH_INCL_PARTITION),
+ * c_0 = m_0; S = sum of c_l. ws_bytes = 5 * (sum of m_l) int32 per (b,h).
  * Errors: LH_ERR_NULL, LH_ERR_SHAPE (B,H,N < 1; D not 64/128; p < 2;
  * L outside 1..LH_MAX_LEVELS; K outside 1..LH_MAX_K; N % p^(L-1) != 0;
- * N or S >= 2^28), LH_ERR_DTYPE, LH_ERR_MODE. */
+ * N or the candidate total sum m_l >= 2^28), LH_ERR_DTYPE, LH_ERR_MODE. */
 lh_status lh_plan(const lh_config* cfg, lh_plan_t* out);
 
 /* (i) Pyramid pool + squared norms. [LH] §3.1 stage (i), Fig. 2 steps 1-2.
@@ -154,11 +170,13 @@ lh_status lh_pool(const lh_config* cfg, const void* q, const void* k, const void
 
 /* (ii) Score, top-K descent, ordering. [LH] §3.1 stage (ii), Fig. 2 step 3,
  * Fig. 1 (topological sort into one causal sequence).
- * score(l,i) = max(sq[0], sq[1]). The coarsest level is kept whole; at each
- * level l = L-1..1 the first k_l candidates in the order (score desc, index
- * asc) are expanded (chunked bitonic sort in shared memory) and their p
- * children become the next level's candidates and sub-sequence entries.
- * Entries are ordered by (last covered token, level) ascending.
+ * score(l,i) = max(sq[0], sq[1]). The coarsest level's entries are all
+ * candidates; at each level l = L-1..1 the first k_l candidates in the order
+ * (score desc, index asc) are expanded (radix select, or a chunked bitonic
+ * sort in shared memory) and their p children become the next level's
+ * candidates. The sub-sequence holds every candidate (LH_INCL_NESTED) or
+ * every candidate that was not expanded (LH_INCL_PARTITION), ordered by
+ * (last covered token, level) ascending (LH_ORDER_POST).
  * Outputs: sel (ascending indices, unused tail = -1), map, slot table.
  * ws: device workspace of at least plan.ws_bytes (contents not kept).
  * When L = 1, map is the identity and sel/slot/ws are not touched (may be NULL). */
@@ -264,7 +282,7 @@ lh_status lh_selftest_timeout(long long limit_cycles, int* gave_up, void* stream
  * process exits; nothing is allocated per call.
  * Same inputs, outputs, results and errors as lh_score_topk, plus
  * LH_ERR_WORKSPACE when the problem needs more scratch than the array holds
- * (plan.ws_bytes > 8 MiB, i.e. 5*S*B*H > 2,097,152; checked before any launch).
+ * (plan.ws_bytes > 8 MiB, i.e. 5*B*H*(sum of m_l) > 2,097,152; checked before any launch).
  * The first call on each device looks up the array's device address
  * (cudaGetSymbolAddress), so make that first call before any stream capture.
  * All calls share the one array, and it keeps the previous call's contents

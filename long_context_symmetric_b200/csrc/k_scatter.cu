@@ -111,14 +111,15 @@ __device__ __forceinline__ void chain_sum(const Geom& g, const float* __restrict
   int l = g.L - 1;
   int e = __ldg(slot_h + g.off[l] + (int)(t / g.pl[l]));
   while (true) {
-    const int s = e >> 1;
-    load8_f32(src + ((size_t)bh * g.S + s) * g.D + c8 * 8, x);
-    const double den = WEIGHTED ? (double)g.pl[l] : 1.0;
-    const double inv = g.pow2 ? 1.0 / den : 0.0;     // exact when p is a power of two
-    acc.add(x, WEIGHTED ? (float)(1.0 / den) : 1.f, den, inv);
+    if (slot_in(e, g)) {          // (partition reading: an expanded entry is not in the sub-sequence)
+      load8_f32(src + ((size_t)bh * g.S + (e >> 1)) * g.D + c8 * 8, x);
+      const double den = WEIGHTED ? (double)g.pl[l] : 1.0;
+      const double inv = g.pow2 ? 1.0 / den : 0.0;     // exact when p is a power of two
+      acc.add(x, WEIGHTED ? (float)(1.0 / den) : 1.f, den, inv);
+    }
     if (!(e & 1)) break;          // not expanded: no finer entry covers t
     if (l == 1) {                 // expanded level-1 parent: t itself is in the sub-sequence
-      const int s0 = (g.order ? s + 1 : s - g.p) + (t % g.p);   // tokens before (post) / after (pre) it
+      const int s0 = slot_tokens(e, g) + (t % g.p);
       load8_f32(src + ((size_t)bh * g.S + s0) * g.D + c8 * 8, x);
       acc.add(x, 1.f, 1.0, 1.0);
       break;
@@ -261,14 +262,16 @@ __global__ void __launch_bounds__(256) k_scatter_tree(const float* __restrict__ 
   int rem[LV + 1];                     // tokens left in the current level-l entry
   int idx[LV + 1];                     // index of the current level-l entry
   float x[8];
-  int sl1 = 0, r0 = 0;                 // slot of the current level-1 entry, token offset in it
+  int tok1 = 0, r0 = 0;                // first token slot of the current level-1 entry, offset in it
   {
     const int e = __ldg(slot_h + g.off[LV] + cb);
-    load8_f32(srow + (size_t)(e >> 1) * g.D, x);
     acc[LV].zero();
-    add_level<FIXED, WEIGHTED>(acc[LV], x, g, LV);
+    if (slot_in(e, g)) {
+      load8_f32(srow + (size_t)(e >> 1) * g.D, x);
+      add_level<FIXED, WEIGHTED>(acc[LV], x, g, LV);
+    }
     expd[LV] = e & 1;
-    if (LV == 1) sl1 = e >> 1;
+    if (LV == 1) tok1 = slot_tokens(e, g);
   }
 #pragma unroll
   for (int l = 1; l < LV; ++l) {
@@ -285,11 +288,13 @@ __global__ void __launch_bounds__(256) k_scatter_tree(const float* __restrict__ 
         ++idx[l];
         if (expd[l + 1]) {
           const int e = __ldg(slot_h + g.off[l] + idx[l]);
-          load8_f32(srow + (size_t)(e >> 1) * g.D, x);
           acc[l] = acc[l + 1];
-          add_level<FIXED, WEIGHTED>(acc[l], x, g, l);
+          if (slot_in(e, g)) {
+            load8_f32(srow + (size_t)(e >> 1) * g.D, x);
+            add_level<FIXED, WEIGHTED>(acc[l], x, g, l);
+          }
           expd[l] = e & 1;
-          if (l == 1) sl1 = e >> 1;
+          if (l == 1) tok1 = slot_tokens(e, g);
         } else {
           acc[l] = acc[l + 1];
           expd[l] = false;
@@ -302,8 +307,8 @@ __global__ void __launch_bounds__(256) k_scatter_tree(const float* __restrict__ 
     T* o = out + (size_t)t * tstride;
     if (expd[1]) {                     // the token itself is in the sub-sequence
       // the p tokens of an expanded level-1 entry sit right before it
-      // (post-order) or right after it (pre-order)
-      load8_f32(srow + (size_t)((g.order ? sl1 + 1 : sl1 - g.p) + r0) * g.D, x);
+      // (post-order), right after it (pre-order), or at its run (partition)
+      load8_f32(srow + (size_t)(tok1 + r0) * g.D, x);
       Acc<FIXED> a = acc[1];
       add_level<FIXED, WEIGHTED>(a, x, g, 0);
       Packed<T> q;
@@ -417,8 +422,8 @@ __global__ void __launch_bounds__(256) k_blocksum(const T* __restrict__ dout,
 #pragma unroll
       for (int u = 0; u < 8; ++u)
         if (u < nb && live) Vec8<T>::load_raw(src + (size_t)(g1 * p + c0 + u) * tok_stride, raw[u]);
-      const int s1 = e1 >= 0 ? (e1 >> 1) : -1;
       const bool tok_in = e1 >= 0 && (e1 & 1);               // children (tokens) included
+      const int tok0 = tok_in ? slot_tokens(e1, g) : -1;
       // tokens are emitted only where some lane of the warp has them included
       const bool any_tok = __any_sync(0xffffffffu, tok_in);
 #pragma unroll
@@ -437,13 +442,14 @@ __global__ void __launch_bounds__(256) k_blocksum(const T* __restrict__ dout,
 #pragma unroll
             for (int d = 0; d < 8; ++d) s[d] = __fadd_rn(s[d], x[d]);
           }
-          if (any_tok) emit(tok_in ? (g.order ? s1 + 1 : s1 - p) + c0 + u : -1, x, 1.f);
+          if (any_tok) emit(tok_in ? tok0 + c0 + u : -1, x, 1.f);
         }
       }
     }
 #pragma unroll
     for (int d = 0; d < 8; ++d) acc[1][d] = s[d];
-    if (__any_sync(0xffffffffu, e1 >= 0)) emit(e1 >= 0 ? (e1 >> 1) : -1, s, wl[1]);
+    const bool in1 = slot_in(e1, g);
+    if (__any_sync(0xffffffffu, in1)) emit(in1 ? (e1 >> 1) : -1, s, wl[1]);
     long long gi = i1;
 #pragma unroll
     for (int l = 2; l <= LV; ++l) {
@@ -458,13 +464,15 @@ __global__ void __launch_bounds__(256) k_blocksum(const T* __restrict__ dout,
       if (pos != p - 1) break;
       gi /= p;
       const int e = live ? __ldg(slot_h + g.off[l] + (int)gi) : -1;
-      if (__any_sync(0xffffffffu, e >= 0)) emit(e >= 0 ? (e >> 1) : -1, acc[l], wl[l]);
+      const bool in = slot_in(e, g);
+      if (__any_sync(0xffffffffu, in)) emit(in ? (e >> 1) : -1, acc[l], wl[l]);
     }
   }
 }
 
 // (Token slots: the p tokens of an expanded level-1 entry sit right before its
-// slot in post-order, right after it in pre-order.)
+// slot in post-order, right after it in pre-order, at its run start under the
+// partition reading; slot_tokens.)
 // Same block sums with the token rows streamed through a shared-memory ring
 // filled by 1-D bulk async copies (one CTA per coarsest block and head group;
 // hg * D / 8 threads, a multiple of 32). PP = p, a compile-time 2, 4 or 8 that
@@ -579,12 +587,12 @@ __global__ void __launch_bounds__(256, 2) k_blocksum_ring(const T* __restrict__ 
       if (i1 + 1 < i1_end) e1n = __ldg(slot_h + g.off[1] + (int)(i1 + 1));
       // the level-1 entry's os row, loaded now so that its latency overlaps the sums
       float ov1[8];
-      if (e1 >= 0) load8_f32(os + ((size_t)bh * g.S + (e1 >> 1)) * g.D + chunk * 8, ov1);
+      const bool in1 = slot_in(e1, g);
+      if (in1) load8_f32(os + ((size_t)bh * g.S + (e1 >> 1)) * g.D + chunk * 8, ov1);
       typename Vec8<T>::Raw raw[p];
 #pragma unroll
       for (int u = 0; u < p; ++u)
         raw[u] = *reinterpret_cast<const typename Vec8<T>::Raw*>(buf + (size_t)(u0 + u) * row_bytes);
-      const int s1 = e1 >= 0 ? (e1 >> 1) : -1;
       const bool tok_in = e1 >= 0 && (e1 & 1);               // children (tokens) included
       // tokens are emitted only where some lane of the warp has them included
       const bool any_tok = __any_sync(0xffffffffu, tok_in);
@@ -592,7 +600,7 @@ __global__ void __launch_bounds__(256, 2) k_blocksum_ring(const T* __restrict__ 
       // the tokens' os rows, loaded TB at a time so that their latencies overlap
       // (fp32 rows of dout take twice the registers: smaller batches)
       constexpr int TB = p < 4 ? p : (sizeof(T) == 2 ? 4 : 2);
-      const int tok0 = g.order ? s1 + 1 : s1 - p;
+      const int tok0 = slot_tokens(e1, g);
       float ovt[TB][8];
 #pragma unroll
       for (int u = 0; u < p; ++u) {
@@ -613,7 +621,7 @@ __global__ void __launch_bounds__(256, 2) k_blocksum_ring(const T* __restrict__ 
       }
 #pragma unroll
       for (int d = 0; d < 8; ++d) acc[1][d] = sum[d];
-      if (__any_sync(0xffffffffu, e1 >= 0)) emit(e1 >= 0 ? (e1 >> 1) : -1, sum, wl[1], ov1);
+      if (__any_sync(0xffffffffu, in1)) emit(in1 ? (e1 >> 1) : -1, sum, wl[1], ov1);
       long long gi = i1;
 #pragma unroll
       for (int l = 2; l <= LV; ++l) {
@@ -628,7 +636,8 @@ __global__ void __launch_bounds__(256, 2) k_blocksum_ring(const T* __restrict__ 
         if (pos != p - 1) break;
         gi /= p;
         const int e = __ldg(slot_h + g.off[l] + (int)gi);
-        if (__any_sync(0xffffffffu, e >= 0)) emit(e >= 0 ? (e >> 1) : -1, acc[l], wl[l], nullptr);
+        const bool in = slot_in(e, g);
+        if (__any_sync(0xffffffffu, in)) emit(in ? (e >> 1) : -1, acc[l], wl[l], nullptr);
       }
     }
     __syncthreads();                    // every thread is done with this stage

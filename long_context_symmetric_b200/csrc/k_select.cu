@@ -28,11 +28,16 @@
 // top-down; slot = start + size - 1. This equals sorting the entries by
 // (last covered token, level). Pre-order (the other order reading): the run
 // starts at the entry, slot = start, children runs from start + 1; this equals
-// sorting by (first covered token, coarser level first).
+// sorting by (first covered token, coarser level first). Partition reading
+// (expanded entries leave the sub-sequence): an expanded entry's run is its
+// children's runs alone, the included entries tile the tokens and both orders
+// give the same sequence; the slot table keeps the run start of an expanded
+// entry (2 * start + 1), which locates the tokens of a level-1 entry.
 //
 // Per-level working arrays (candidate index, expanded flag, rank among the
 // expanded, subtree size, run start) live in the caller's workspace
-// (5 * S int32 per (b,h)); the sort keys live in shared memory.
+// (5 int32 per candidate of any level, per (b,h)); the sort keys live in
+// shared memory.
 #include "lh_common.cuh"
 
 namespace lh {
@@ -214,14 +219,14 @@ k_select(const double* __restrict__ sq, int32_t* __restrict__ sel, int32_t* __re
 
   const Geom& g = a.g;
   const int bh = blockIdx.x;
-  const int L = g.L, p = g.p, S = g.S;
+  const int L = g.L, p = g.p, S = g.S, C = g.C;
   const double* sqq = sq + (size_t)bh * g.E;
   const double* sqk = sq + ((size_t)g.B * g.H + bh) * g.E;
-  int32_t* cand = ws + (size_t)bh * 5 * S;
-  int32_t* flag = cand + S;
-  int32_t* rank = flag + S;
-  int32_t* size = rank + S;
-  int32_t* start = size + S;
+  int32_t* cand = ws + (size_t)bh * 5 * C;
+  int32_t* flag = cand + C;
+  int32_t* rank = flag + C;
+  int32_t* size = rank + C;
+  int32_t* start = size + C;
   int32_t* slot_h = slot + (size_t)bh * g.E;
   int32_t* sel_h = sel + (size_t)bh * (L - 1) * g.K;
   int32_t* map_h = map + (size_t)bh * S;
@@ -237,7 +242,7 @@ k_select(const double* __restrict__ sq, int32_t* __restrict__ sel, int32_t* __re
 
   // ---------------- descent
   for (int l = L - 1; l >= 1; --l) {
-    const int c = g.c[l], k = g.k[l];
+    const int c = g.cand[l], k = g.k[l];
     int32_t* cl = cand + a.lvl_base[l];
     int32_t* fl = flag + a.lvl_base[l];
     const double* sq_l = sqq + g.off[l];
@@ -297,7 +302,7 @@ k_select(const double* __restrict__ sq, int32_t* __restrict__ sel, int32_t* __re
   {
     int32_t* f0 = flag + a.lvl_base[0];
     int32_t* s0 = size + a.lvl_base[0];
-    for (int q = threadIdx.x; q < g.c[0]; q += kThreads) { f0[q] = 0; s0[q] = 1; }
+    for (int q = threadIdx.x; q < g.cand[0]; q += kThreads) { f0[q] = 0; s0[q] = 1; }
   }
   __syncthreads();
   for (int l = 1; l <= L - 1; ++l) {
@@ -305,8 +310,8 @@ k_select(const double* __restrict__ sq, int32_t* __restrict__ sel, int32_t* __re
     const int32_t* rl = rank + a.lvl_base[l];
     int32_t* sl = size + a.lvl_base[l];
     const int32_t* sc = size + a.lvl_base[l - 1];
-    for (int q = threadIdx.x; q < g.c[l]; q += kThreads) {
-      int sz = 1;
+    for (int q = threadIdx.x; q < g.cand[l]; q += kThreads) {
+      int sz = (fl[q] && g.incl) ? 0 : 1;   // partition: an expanded entry is not in its run
       if (fl[q]) {
         const int base = rl[q] * p;
         for (int j = 0; j < p; ++j) sz += sc[base + j];
@@ -317,7 +322,7 @@ k_select(const double* __restrict__ sq, int32_t* __restrict__ sel, int32_t* __re
   }
 
   // ---------------- run starts, top-down
-  block_exclusive_scan(size + a.lvl_base[L - 1], start + a.lvl_base[L - 1], g.c[L - 1], warp_tot);
+  block_exclusive_scan(size + a.lvl_base[L - 1], start + a.lvl_base[L - 1], g.cand[L - 1], warp_tot);
   __syncthreads();
   for (int l = L - 1; l >= 1; --l) {
     const int32_t* fl = flag + a.lvl_base[l];
@@ -325,9 +330,10 @@ k_select(const double* __restrict__ sq, int32_t* __restrict__ sel, int32_t* __re
     const int32_t* stl = start + a.lvl_base[l];
     const int32_t* sc = size + a.lvl_base[l - 1];
     int32_t* stc = start + a.lvl_base[l - 1];
-    for (int q = threadIdx.x; q < g.c[l]; q += kThreads) {
+    for (int q = threadIdx.x; q < g.cand[l]; q += kThreads) {
       if (fl[q]) {
-        int s = stl[q] + (g.order ? 1 : 0);   // pre-order: the entry first, then its children's runs
+        // pre-order (nested): the entry first, then its children's runs
+        int s = stl[q] + (g.order && !g.incl ? 1 : 0);
         const int base = rl[q] * p;
         for (int j = 0; j < p; ++j) {
           stc[base + j] = s;
@@ -344,9 +350,13 @@ k_select(const double* __restrict__ sq, int32_t* __restrict__ sel, int32_t* __re
     const int32_t* fl = flag + a.lvl_base[l];
     const int32_t* sl = size + a.lvl_base[l];
     const int32_t* stl = start + a.lvl_base[l];
-    for (int q = threadIdx.x; q < g.c[l]; q += kThreads) {
-      const int sidx = g.order ? stl[q] : stl[q] + sl[q] - 1;
+    for (int q = threadIdx.x; q < g.cand[l]; q += kThreads) {
       const int e = cl[q];
+      if (g.incl && fl[q]) {                // partition: expanded, not in the sub-sequence
+        slot_h[g.off[l] + e] = 2 * stl[q] + 1;
+        continue;
+      }
+      const int sidx = g.order ? stl[q] : stl[q] + sl[q] - 1;
       map_h[sidx] = (l << 28) | e;
       if (l >= 1) slot_h[g.off[l] + e] = 2 * sidx + (fl[q] ? 1 : 0);
     }
@@ -376,7 +386,7 @@ cudaError_t launch_select(const Geom& g, const double* sq, int32_t* sel, int32_t
   int base = 0;
   for (int l = 0; l < LH_MAX_LEVELS; ++l) {
     a.lvl_base[l] = base;
-    if (l < g.L) base += g.c[l];
+    if (l < g.L) base += g.cand[l];
   }
   const size_t smem = (size_t)kChunk * (sizeof(unsigned long long) + sizeof(unsigned));
   cudaError_t e = cudaFuncSetAttribute(k_select, cudaFuncAttributeMaxDynamicSharedMemorySize,

@@ -79,7 +79,8 @@ lh_status make_geom(const lh_config* cfg, Geom* g, lh_plan_t* out) {
   if (cfg->dtype != LH_BF16 && cfg->dtype != LH_FP32) return LH_ERR_DTYPE;
   if (cfg->accum != LH_ACC_FP32 && cfg->accum != LH_ACC_FIXED64) return LH_ERR_MODE;
   if ((unsigned)cfg->score > LH_SCORE_PROD || (unsigned)cfg->ties > LH_TIES_HIGH_FIRST ||
-      (unsigned)cfg->order > LH_ORDER_PRE || (unsigned)cfg->weight > LH_WEIGHT_MEAN)
+      (unsigned)cfg->order > LH_ORDER_PRE || (unsigned)cfg->weight > LH_WEIGHT_MEAN ||
+      (unsigned)cfg->inclusion > LH_INCL_PARTITION)
     return LH_ERR_MODE;
   const int B = cfg->B, H = cfg->H, N = cfg->N, D = cfg->D, p = cfg->p, L = cfg->L, K = cfg->K;
   if (B < 1 || H < 1 || N < 1) return LH_ERR_SHAPE;
@@ -98,17 +99,23 @@ lh_status make_geom(const lh_config* cfg, Geom* g, lh_plan_t* out) {
   G.B = B; G.H = H; G.N = N; G.D = D; G.p = p; G.L = L; G.K = K;
   for (int l = 0; l < LH_MAX_LEVELS; ++l) G.pl[l] = pl[l];
   for (int l = 0; l < L; ++l) G.n[l] = (int)(N / pl[l]);
-  G.c[L - 1] = G.n[L - 1];
+  G.cand[L - 1] = G.n[L - 1];
   long long cand = G.n[L - 1];
   for (int l = L - 1; l >= 1; --l) {
     G.k[l] = (int)(cand < K ? cand : K);
-    G.c[l - 1] = p * G.k[l];
-    cand = G.c[l - 1];
+    G.cand[l - 1] = p * G.k[l];
+    cand = G.cand[l - 1];
   }
-  long long S = 0;
-  for (int l = 0; l < L; ++l) S += G.c[l];
-  if (S >= (1LL << 28)) return LH_ERR_SHAPE;
+  const bool part = cfg->inclusion == LH_INCL_PARTITION;
+  long long S = 0, C = 0;
+  for (int l = 0; l < L; ++l) {
+    G.c[l] = G.cand[l] - (part && l >= 1 ? G.k[l] : 0);
+    S += G.c[l];
+    C += G.cand[l];
+  }
+  if (C >= (1LL << 28)) return LH_ERR_SHAPE;
   G.S = (int)S;
+  G.C = (int)C;
   int E = 0;
   for (int l = 1; l < L; ++l) {
     G.off[l] = E;
@@ -121,6 +128,7 @@ lh_status make_geom(const lh_config* cfg, Geom* g, lh_plan_t* out) {
   G.ties = cfg->ties;
   G.order = cfg->order;
   G.weight = cfg->weight;
+  G.incl = cfg->inclusion;
   *g = G;
   if (out) {
     std::memset(out, 0, sizeof(*out));
@@ -132,7 +140,7 @@ lh_status make_geom(const lh_config* cfg, Geom* g, lh_plan_t* out) {
       out->c[l] = G.c[l];
       out->lvl_off[l] = G.off[l];
     }
-    out->ws_bytes = L > 1 ? (size_t)B * H * 5 * (size_t)G.S * sizeof(int32_t) : 0;
+    out->ws_bytes = L > 1 ? (size_t)B * H * 5 * (size_t)G.C * sizeof(int32_t) : 0;
   }
   return LH_OK;
 }

@@ -15,13 +15,30 @@ struct Geom {
   int B, H, N, D, p, L, K, S, E;
   int n[LH_MAX_LEVELS];
   int k[LH_MAX_LEVELS];
-  int c[LH_MAX_LEVELS];
+  int c[LH_MAX_LEVELS];        // entries of level l in the sub-sequence
+  int cand[LH_MAX_LEVELS];     // candidates at level l (the selection's working arrays)
+  int C;                       // sum of cand
   int off[LH_MAX_LEVELS];      // start of level l (>= 1) in the per-head E axis
   long long pl[LH_MAX_LEVELS]; // p^l
   int pow2;                    // p is a power of two (division by p^l is exact scaling)
   int accum;                   // lh_accum
   int score, ties, order, weight;   // lh_score, lh_ties, lh_order, lh_weight
+  int incl;                         // lh_inclusion
 };
+
+// Slot-table entry e of a level >= 1 entry (written by the selection):
+//   e < 0         not a candidate (pruned): neither in the sub-sequence nor expanded;
+//   e = 2s        in the sub-sequence at slot s, not expanded;
+//   e = 2s + 1    expanded; nested reading: in the sub-sequence at slot s;
+//                 partition reading: not in it, s = first slot of its descendants' run.
+// Every entry a walk from the coarsest level visits is a candidate (e >= 0).
+__host__ __device__ __forceinline__ bool slot_in(int e, const Geom& g) { return e >= 0 && !(g.incl && (e & 1)); }
+// First slot of the p tokens of an expanded level-1 entry: right before its own
+// slot (post-order), right after it (pre-order), or the run start (partition).
+__host__ __device__ __forceinline__ int slot_tokens(int e, const Geom& g) {
+  const int s = e >> 1;
+  return g.incl ? s : (g.order ? s + 1 : s - g.p);
+}
 
 // Element I/O: 8 consecutive components of a dtype row.
 template <typename T> struct Vec8;

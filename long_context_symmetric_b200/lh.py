@@ -37,13 +37,15 @@ class LHError(RuntimeError):
 class Config(ctypes.Structure):
     _fields_ = [("B", c_int), ("H", c_int), ("N", c_int), ("D", c_int), ("p", c_int),
                 ("L", c_int), ("K", c_int), ("dtype", c_int), ("accum", c_int),
-                ("score", c_int), ("ties", c_int), ("order", c_int), ("weight", c_int)]
+                ("score", c_int), ("ties", c_int), ("order", c_int), ("weight", c_int),
+                ("inclusion", c_int)]
 
 
 SCORES = {"max": 0, "k": 1, "sum": 2, "prod": 3}
 TIES = {"low": 0, "high": 1}
 ORDERS = {"post": 0, "pre": 1}
 WEIGHTS = {"one": 0, "mean": 1}
+INCLUSIONS = {"nested": 0, "partition": 1}
 
 
 class Plan(ctypes.Structure):
@@ -133,12 +135,12 @@ def _stream(stream):
 
 
 def make_config(B, H, N, D, p, L, K, dtype="bf16", accum="fp", score="max", ties="low", order="post",
-                weight="one") -> Config:
+                weight="one", inclusion="nested") -> Config:
     """Problem sizes, element type, accumulation mode and the readings of the
     open points (defaults: the library's reading)."""
     return Config(B, H, N, D, p, L, K, {"bf16": LH_BF16, "fp32": LH_FP32}[dtype],
                   {"fp": LH_ACC_FP32, "fixed": LH_ACC_FIXED64}[accum], SCORES[score], TIES[ties],
-                  ORDERS[order], WEIGHTS[weight])
+                  ORDERS[order], WEIGHTS[weight], INCLUSIONS[inclusion])
 
 
 def plan(cfg: Config) -> Plan:

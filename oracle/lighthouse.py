@@ -24,7 +24,10 @@ it is used):
       each level l = L-1..1 the top-k_l candidates are expanded and all p
       children of each expanded entry are included one level down; parents
       stay in the sub-sequence ([LH] Fig. 2: the selector keeps parents and
-      prunes the tree below unselected entries).
+      prunes the tree below unselected entries). The other reading,
+      inclusion="partition": an expanded entry leaves the sub-sequence and is
+      replaced by its children, so the included entries tile the tokens and
+      every token is covered exactly once.
   R2  score of a pyramid entry = max(||mean_Q||^2, ||mean_K||^2) of the fp64
       means (the scorer looks at both the query and the key side: [LH] §1
       and the q/k score labels of Fig. 2);
@@ -80,7 +83,8 @@ class Plan:
 
     n[l]  entries at level l (n_l = N / p^l)            [LH] §3.1 stage (i)
     k[l]  entries expanded at level l (l >= 1)           R5
-    c[l]  entries of level l in the sub-sequence         R1
+    m[l]  candidates at level l                          R1
+    c[l]  entries of level l in the sub-sequence         R1 (m[l], or m[l] - k[l] for l >= 1 under partition)
     S     sub-sequence length = sum_l c[l]               [LH] §1 size law
     """
     N: int
@@ -89,26 +93,28 @@ class Plan:
     K: int
     n: list = field(default_factory=list)
     k: list = field(default_factory=list)
+    m: list = field(default_factory=list)
     c: list = field(default_factory=list)
     S: int = 0
 
 
-def plan(N: int, p: int, L: int, K: int) -> Plan:
+def plan(N: int, p: int, L: int, K: int, inclusion: str = "nested") -> Plan:
     """Sub-sequence sizes under reading R1/R5 ([LH] §1: S = O(LpK + N/p^(L-1)))."""
     if p < 2 or L < 1 or K < 1 or N < 1:
         raise ValueError("need p >= 2, L >= 1, K >= 1, N >= 1")
     if N % (p ** (L - 1)) != 0:
         raise ValueError("N must be a multiple of p^(L-1) (reading R10)")
+    if inclusion not in ("nested", "partition"):
+        raise ValueError(inclusion)
     n = [N // p ** l for l in range(L)]
     k = [0] * L
-    c = [0] * L
-    c[L - 1] = n[L - 1]
-    ncand = n[L - 1]
+    m = [0] * L
+    m[L - 1] = n[L - 1]
     for l in range(L - 1, 0, -1):
-        k[l] = min(K, ncand)
-        c[l - 1] = p * k[l]
-        ncand = c[l - 1]
-    return Plan(N=N, p=p, L=L, K=K, n=n, k=k, c=c, S=sum(c))
+        k[l] = min(K, m[l])
+        m[l - 1] = p * k[l]
+    c = [m[l] - (k[l] if inclusion == "partition" and l >= 1 else 0) for l in range(L)]
+    return Plan(N=N, p=p, L=L, K=K, n=n, k=k, m=m, c=c, S=sum(c))
 
 
 # ----------------------------------------------------------------------------
@@ -235,14 +241,15 @@ def scores_head(means_q, means_k, L: int, score: str = "max"):
 # (ii-b) hierarchical top-K, tree descent   [LH] §3.1 stage (ii), Fig. 2 (R1, R3, R5)
 # ----------------------------------------------------------------------------
 
-def select_head(scores, p: int, L: int, K: int, ties: str = "low"):
+def select_head(scores, p: int, L: int, K: int, ties: str = "low", inclusion: str = "nested"):
     """Top-down descent over the pyramid (parents kept, tree pruned: [LH] Fig. 2, step 3).
 
     Candidates at the coarsest level are all its entries. At each level
     l = L-1..1 the first k_l candidates in the order (score desc, index asc)
     are expanded (ties="high": index desc, the other tie reading R3); the p
-    children of every expanded entry are the candidates (and included
-    entries) one level down.
+    children of every expanded entry are the candidates one level down.
+    Every candidate enters the sub-sequence (R1, nested), or every candidate
+    that was not expanded (inclusion="partition").
 
     Returns (sel, included): sel[l] (l >= 1) is the sorted array of expanded
     indices at level l; included[l] the sorted array of level-l entries that
@@ -261,6 +268,8 @@ def select_head(scores, p: int, L: int, K: int, ties: str = "low"):
         order = np.lexsort((tie_key, -s))    # primary: score desc; then index asc (R3) or desc
         chosen = np.sort(cand[order[:k]])
         sel[l] = chosen
+        if inclusion == "partition":
+            included[l] = np.setdiff1d(included[l], chosen)
         cand = (chosen[:, None] * p + np.arange(p)[None, :]).reshape(-1)
         included[l - 1] = cand.copy()
     return sel, included
@@ -427,22 +436,22 @@ def spread_head(g_rows, lvl, idx, p: int, N: int, mode: str = "fp"):
 # ----------------------------------------------------------------------------
 
 def forward_head(qh, kh, vh, p: int, L: int, K: int, dtype: str, mode: str = "fp", score: str = "max",
-                 ties: str = "low", order: str = "post", weight: str = "one"):
+                 ties: str = "low", order: str = "post", weight: str = "one", inclusion: str = "nested"):
     """Forward pass for one head: tokens [N, D] x3 -> dict of every intermediate.
 
-    score, ties, order, weight select the readings R2a, R3, R6, R7 (defaults:
-    the library's). Keys: means_*, stored_*, scores, sq_q, sq_k, sel,
+    score, ties, order, weight, inclusion select the readings R2a, R3, R6, R7,
+    R1 (defaults: the library's). Keys: means_*, stored_*, scores, sq_q, sq_k, sel,
     included, lvl, idx, qs, ks, vs (sub-sequence), os, lse (attention), o
     ([N, D] output, fp64, not rounded), weight.
     """
     N, D = qh.shape
-    pl = plan(N, p, L, K)
+    pl = plan(N, p, L, K, inclusion)
     mq, sq_ = pool_head(qh, p, L, dtype)
     mk, sk_ = pool_head(kh, p, L, dtype)
     mv, sv_ = pool_head(vh, p, L, dtype)
     if L > 1:
         scores, nq, nk = scores_head(mq, mk, L, score)
-        sel, included = select_head(scores, p, L, K, ties)
+        sel, included = select_head(scores, p, L, K, ties, inclusion)
     else:
         scores, nq, nk, sel, included = [None], [None], [None], [None], [None]
     lvl, idx = order_head(included, p, L, N, order)

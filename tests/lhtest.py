@@ -82,15 +82,24 @@ def run_gpu(case: Case, q, k, v, do=None, stream=None):
 
 
 def expected_slot_table(fw, case: Case, pl) -> np.ndarray:
-    """Slot table implied by the oracle's selection and order."""
+    """Slot table implied by the oracle's selection and order: 2 * slot + expanded
+    for the entries in the sub-sequence; under the partition reading an expanded
+    entry is not in it and holds 2 * (slot of the entry that starts at its first
+    token) + 1 (the entries tile the tokens, so exactly one starts there)."""
     E = pl.E
+    p = case.p
     tab = np.full(max(E, 1), -1, dtype=np.int64)
     slot_of = {(int(l), int(i)): j for j, (l, i) in enumerate(zip(fw["lvl"], fw["idx"]))}
+    part = case.readings.get("inclusion", "nested") == "partition"
+    starts = {int(i) * p ** int(l): j for j, (l, i) in enumerate(zip(fw["lvl"], fw["idx"]))} if part else {}
     for l in range(1, case.L):
         sel = set(int(x) for x in fw["sel"][l]) if fw["sel"][l] is not None else set()
         for i in fw["included"][l]:
             j = slot_of[(l, int(i))]
             tab[pl.lvl_off[l] + int(i)] = 2 * j + (1 if int(i) in sel else 0)
+        if part:
+            for i in sel:
+                tab[pl.lvl_off[l] + i] = 2 * starts[i * p ** l] + 1
     return tab[:E]
 
 

@@ -22,18 +22,19 @@ def test_library_exports_every_declared_symbol():
     assert lh.status_string(0) == "ok"
 
 
+@pytest.mark.parametrize("inclusion", ["nested", "partition"])
 @pytest.mark.parametrize("name", list(synth.WORKLOADS))
-def test_plan_agrees_with_oracle(name):
+def test_plan_agrees_with_oracle(name, inclusion):
     w = synth.WORKLOADS[name]
-    pl = lh.plan(lh.make_config(w.B, w.H, w.N, w.D, w.p, w.L, w.K, w.dtype, w.mode))
-    ref = orc.plan(w.N, w.p, w.L, w.K)
+    pl = lh.plan(lh.make_config(w.B, w.H, w.N, w.D, w.p, w.L, w.K, w.dtype, w.mode, inclusion=inclusion))
+    ref = orc.plan(w.N, w.p, w.L, w.K, inclusion)
     assert pl.S == ref.S
     assert list(pl.n)[:w.L] == ref.n
     assert list(pl.c)[:w.L] == ref.c
     assert list(pl.k)[1:w.L] == ref.k[1:]
     assert pl.E == sum(ref.n[1:])
-    # the descent's workspace: 5 int32 per sub-sequence entry; none without a pyramid
-    assert pl.ws_bytes == (w.B * w.H * 5 * ref.S * 4 if w.L > 1 else 0)
+    # the descent's workspace: 5 int32 per candidate of any level; none without a pyramid
+    assert pl.ws_bytes == (w.B * w.H * 5 * sum(ref.m) * 4 if w.L > 1 else 0)
 
 
 @pytest.mark.parametrize("N,p,L,K", [(64, 2, 1, 5), (48, 3, 2, 1), (243, 3, 5, 2), (4096, 8, 3, 4096),
@@ -61,6 +62,10 @@ def test_plan_rejects_bad_enums():
     cfg = lh.make_config(1, 2, 4096, 64, 4, 3, 16)
     cfg.accum = 3
     assert lh.lib().lh_plan(ctypes.byref(cfg), ctypes.byref(lh.Plan())) == LH_ERR_MODE
+    for field in ("score", "ties", "order", "weight", "inclusion"):
+        cfg = lh.make_config(1, 2, 4096, 64, 4, 3, 16)
+        setattr(cfg, field, 9)
+        assert lh.lib().lh_plan(ctypes.byref(cfg), ctypes.byref(lh.Plan())) == LH_ERR_MODE, field
 
 
 def test_entry_points_validate_before_launch():

@@ -43,6 +43,14 @@ READINGS = [
     Case("weight_mean_p3_fixed", 1, 2, 333, 128, "bf16", 3, 3, 5, accum="fixed", weight="mean"),
     Case("all_alternatives", 2, 3, 2048, 64, "bf16", 4, 3, 37, recipe="token_scale", score="sum",
          ties="high", order="pre", weight="mean"),
+    Case("partition", 1, 2, 4096, 128, "bf16", 4, 4, 40, inclusion="partition"),
+    Case("partition_p3_fixed_mean", 1, 2, 333, 128, "bf16", 3, 3, 5, accum="fixed", weight="mean",
+         inclusion="partition"),
+    Case("partition_chunked", 1, 1, 65536, 64, "bf16", 2, 2, 200, recipe="codebook", inclusion="partition"),
+    Case("partition_full_budget", 1, 2, 2048, 64, "bf16", 2, 3, 1024, inclusion="partition"),
+    Case("partition_fp32", 1, 2, 1024, 64, "fp32", 4, 3, 32, inclusion="partition"),
+    Case("all_alternatives_partition", 2, 3, 2048, 64, "bf16", 4, 3, 37, recipe="token_scale", score="sum",
+         ties="high", order="pre", weight="mean", inclusion="partition"),
 ]
 
 
@@ -142,6 +150,20 @@ def test_autograd_wrapper_matches_stagewise():
     o.backward(do)
     assert torch.equal(o, res["o"])
     assert torch.equal(qg.grad, res["dq"]) and torch.equal(kg.grad, res["dk"]) and torch.equal(vg.grad, res["dv"])
+
+
+def test_full_size_partition_sampled_heads():
+    """The 512K workload under the partition reading (S = 22,528), in the launch
+    configuration the bench uses: the first and last heads against the oracle."""
+    w = synth.WORKLOADS["ctx512k"]
+    case = Case("ctx512k_partition", w.B, w.H, w.N, w.D, w.dtype, w.p, w.L, w.K, w.recipe, w.mode, w.seed,
+                inclusion="partition")
+    q, k, v = synth.make_inputs(w, device=DEV)
+    do = synth.make_dout(w, device=DEV)
+    res = run_gpu(case, q, k, v, do)
+    assert lh.plan(case.cfg()).S == 22528
+    for (b, h) in [(0, 0), (w.B - 1, w.H - 1)]:
+        compare_head(case, res, q, k, v, do, b, h)
 
 
 def test_full_size_alternative_readings_sampled_heads():
