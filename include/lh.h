@@ -99,7 +99,9 @@ typedef enum {
   LH_SCORE_MAX = 0,    /* max(|mean_q|^2, |mean_k|^2) */
   LH_SCORE_K = 1,      /* |mean_k|^2 */
   LH_SCORE_SUM = 2,    /* |mean_q| + |mean_k| (fp64 square roots, then their sum) */
-  LH_SCORE_PROD = 3    /* |mean_q|^2 * |mean_k|^2 (same order as |mean_q| * |mean_k|) */
+  LH_SCORE_PROD = 3,   /* |mean_q|^2 * |mean_k|^2 (same order as |mean_q| * |mean_k|) */
+  LH_SCORE_MAXPOOL = 4 /* bottom-up: a token scores max(|q|^2, |k|^2), an entry the max of its
+                          children's scores (lh_pool then writes tokens' norms max-pooled into sq) */
 } lh_score;
 typedef enum {
   LH_TIES_LOW_FIRST = 0,   /* equal scores: lower index first */
@@ -163,7 +165,9 @@ lh_status lh_plan(const lh_config* cfg, lh_plan_t* out);
  * left-to-right sum of its p children's sums) and rounded to nearest-even
  * into dtype. sq[0] / sq[1] hold the squared l2 norm of the fp64 query / key
  * means in a pinned order (8-component chunks summed left to right, chunk
- * partials combined by a stride-halving tree). Nothing is written when L = 1.
+ * partials combined by a stride-halving tree). Under LH_SCORE_MAXPOOL, sq[0] / sq[1]
+ * hold instead the largest such squared norm among the entry's query / key
+ * token rows. Nothing is written when L = 1.
  * Inputs q, k, v; outputs pyr_q, pyr_k, pyr_v, sq. */
 lh_status lh_pool(const lh_config* cfg, const void* q, const void* k, const void* v,
                   void* pyr_q, void* pyr_k, void* pyr_v, double* sq, void* stream);

@@ -15,6 +15,13 @@
 // combined by a butterfly over the lanes that hold them, which equals the
 // stride-halving tree c[j] += c[j + s] for s = D/16, ..., 1.
 //
+// Max-pool score reading (MP; Fig. 2 step 2 read as "l2 norm of every token,
+// then max-pooled up the levels"): instead of the norms of the means, sq gets,
+// for each entry, the largest pinned-order squared norm among its tokens, for
+// queries and keys separately (a token's norm is formed exactly as a mean's).
+// Taking the max of the two then equals max-pooling the tokens' bidirectional
+// scores level by level, since max commutes.
+//
 // Thread mapping: one thread owns 8 consecutive components of one head; the
 // D/8 lanes of a head are consecutive lanes of one warp. A thread walks the
 // p^(L-1) tokens of one coarsest-level block in order, keeping one running fp64
@@ -56,7 +63,7 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
 // level-1 entry's p token rows are read and widened together, so the widening
 // conversions (a quarter-rate pipe) overlap instead of waiting on the add chain.
 // PP == 0: any p, one token at a time.
-template <typename T, int LV, int PP>
+template <typename T, int LV, int PP, bool MP>
 __global__ void __launch_bounds__(256, 2) k_pool(const T* __restrict__ q, const T* __restrict__ k,
                                                  const T* __restrict__ v, T* __restrict__ pq,
                                                  T* __restrict__ pk, T* __restrict__ pv,
@@ -112,6 +119,15 @@ __global__ void __launch_bounds__(256, 2) k_pool(const T* __restrict__ q, const 
 
   double acc[LV][8];                    // acc[l-1]: running sum of the open entry of level l
   double (&s)[8] = acc[0];
+  double mx[MP ? LV : 1];               // MP: mx[l-1] = largest token norm of the open level-l entry
+  // MP: pinned-order squared norm of one token's row (the same on every lane of the head)
+  auto token_norm = [&](const double (&xr)[8]) -> double {
+    double part = __dmul_rn(xr[0], xr[0]);
+#pragma unroll
+    for (int d = 1; d < 8; ++d) part = __dadd_rn(part, __dmul_rn(xr[d], xr[d]));
+    for (int off = C8 >> 1; off >= 1; off >>= 1) part = __dadd_rn(part, __shfl_xor_sync(wmask, part, off));
+    return part;
+  };
   long long gi1 = (long long)cb * (P / p);   // index of the open level-1 entry
   int c = 0;                            // position of the next token in its level-1 entry
   tc::Abort none{0};
@@ -133,9 +149,11 @@ __global__ void __launch_bounds__(256, 2) k_pool(const T* __restrict__ q, const 
           if (pos == 0) {
 #pragma unroll
             for (int d = 0; d < 8; ++d) acc[l - 1][d] = acc[l - 2][d];
+            if constexpr (MP) mx[l - 1] = mx[l - 2];
           } else {
 #pragma unroll
             for (int d = 0; d < 8; ++d) acc[l - 1][d] = __dadd_rn(acc[l - 1][d], acc[l - 2][d]);
+            if constexpr (MP) mx[l - 1] = fmax(mx[l - 1], mx[l - 2]);
           }
           if (pos != p - 1) break;
           gi /= p;
@@ -153,7 +171,9 @@ __global__ void __launch_bounds__(256, 2) k_pool(const T* __restrict__ q, const 
         }
         const size_t e = (size_t)g.off[l] + gi;
         Vec8<T>::store_f64(dst_head + e * g.D, m);
-        if (tensor < 2) {
+        if (MP) {
+          if (tensor < 2 && chunk == 0) sq_head[e] = mx[l - 1];
+        } else if (tensor < 2) {
           double part = __dmul_rn(m[0], m[0]);
 #pragma unroll
           for (int d = 1; d < 8; ++d) part = __dadd_rn(part, __dmul_rn(m[d], m[d]));
@@ -177,6 +197,12 @@ __global__ void __launch_bounds__(256, 2) k_pool(const T* __restrict__ q, const 
           Vec8<T>::raw_f64(raw[u], xr);
 #pragma unroll
           for (int d = 0; d < 8; ++d) s[d] = u == 0 ? xr[d] : __dadd_rn(s[d], xr[d]);
+          if constexpr (MP) {
+            if (tensor < 2) {
+              const double tn = token_norm(xr);
+              mx[0] = u == 0 ? tn : fmax(mx[0], tn);
+            }
+          }
         }
         complete();
       }
@@ -191,6 +217,12 @@ __global__ void __launch_bounds__(256, 2) k_pool(const T* __restrict__ q, const 
         } else {
 #pragma unroll
           for (int d = 0; d < 8; ++d) s[d] = __dadd_rn(s[d], xr[d]);
+        }
+        if constexpr (MP) {
+          if (tensor < 2) {
+            const double tn = token_norm(xr);
+            mx[0] = c == 0 ? tn : fmax(mx[0], tn);
+          }
         }
         if (++c < p) continue;
         c = 0;
@@ -231,10 +263,12 @@ cudaError_t launch_t(const Geom& g, const void* q, const void* k, const void* v,
   const T* tq = (const T*)q; const T* tk = (const T*)k; const T* tv = (const T*)v;
   T* tpq = (T*)pq; T* tpk = (T*)pk; T* tpv = (T*)pv;
   switch (LV) {
-#define LH_POOL_PP(n, P)                                                                                \
-  e = cudaFuncSetAttribute(k_pool<T, n, P>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);    \
+#define LH_POOL_MP(n, P, M)                                                                             \
+  e = cudaFuncSetAttribute(k_pool<T, n, P, M>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem); \
   if (e != cudaSuccess) return e;                                                                       \
-  k_pool<T, n, P><<<grid, block, smem, s>>>(tq, tk, tv, tpq, tpk, tpv, sq, a, err);
+  k_pool<T, n, P, M><<<grid, block, smem, s>>>(tq, tk, tv, tpq, tpk, tpv, sq, a, err);
+#define LH_POOL_PP(n, P)                                                                                \
+  if (g.score == LH_SCORE_MAXPOOL) { LH_POOL_MP(n, P, true) } else { LH_POOL_MP(n, P, false) }
 #define LH_POOL_CASE(n)                                                                                 \
     case n:                                                                                             \
       if (pp == 8) { LH_POOL_PP(n, 8) } else if (pp == 4) { LH_POOL_PP(n, 4) }                          \
@@ -244,6 +278,7 @@ cudaError_t launch_t(const Geom& g, const void* q, const void* k, const void* v,
     LH_POOL_CASE(5) LH_POOL_CASE(6) LH_POOL_CASE(7)
 #undef LH_POOL_CASE
 #undef LH_POOL_PP
+#undef LH_POOL_MP
     default: return cudaErrorInvalidValue;
   }
   count_launch();

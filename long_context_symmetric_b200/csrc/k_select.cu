@@ -8,7 +8,8 @@
 //
 // Per level l = L-1 .. 1 (all entries of level L-1 are the first candidates):
 //   score = max(|mean_Q|^2, |mean_K|^2) (fp64, from lh_pool); the other
-//   selectable readings: |mean_K|^2, |mean_Q| + |mean_K|, |mean_Q|^2 |mean_K|^2
+//   selectable readings: |mean_K|^2, |mean_Q| + |mean_K|, |mean_Q|^2 |mean_K|^2,
+//   and the max-pool reading (the same max, of lh_pool's max-pooled token norms)
 //   the first k_l candidates in the order (score desc, index asc; or index
 //   desc under the other tie reading) are expanded.
 //   Only the set matters (the sub-sequence order comes from the tree below),
@@ -123,7 +124,7 @@ __device__ __forceinline__ unsigned long long score_bits(const double* sqq, cons
     case 1: s = b; break;                                           // |mean_k|^2
     case 2: s = __dadd_rn(__dsqrt_rn(a), __dsqrt_rn(b)); break;     // |mean_q| + |mean_k|
     case 3: s = __dmul_rn(a, b); break;                             // |mean_q|^2 |mean_k|^2
-    default: s = fmax(a, b);                                        // max of the squared norms
+    default: s = fmax(a, b);   // max of the squared norms (maxpool: of the max-pooled token norms)
   }
   return (unsigned long long)__double_as_longlong(s);
 }

@@ -78,7 +78,7 @@ lh_status make_geom(const lh_config* cfg, Geom* g, lh_plan_t* out) {
   if (!cfg) return LH_ERR_NULL;
   if (cfg->dtype != LH_BF16 && cfg->dtype != LH_FP32) return LH_ERR_DTYPE;
   if (cfg->accum != LH_ACC_FP32 && cfg->accum != LH_ACC_FIXED64) return LH_ERR_MODE;
-  if ((unsigned)cfg->score > LH_SCORE_PROD || (unsigned)cfg->ties > LH_TIES_HIGH_FIRST ||
+  if ((unsigned)cfg->score > LH_SCORE_MAXPOOL || (unsigned)cfg->ties > LH_TIES_HIGH_FIRST ||
       (unsigned)cfg->order > LH_ORDER_PRE || (unsigned)cfg->weight > LH_WEIGHT_MEAN ||
       (unsigned)cfg->inclusion > LH_INCL_PARTITION)
     return LH_ERR_MODE;

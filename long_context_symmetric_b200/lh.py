@@ -41,7 +41,7 @@ class Config(ctypes.Structure):
                 ("inclusion", c_int)]
 
 
-SCORES = {"max": 0, "k": 1, "sum": 2, "prod": 3}
+SCORES = {"max": 0, "k": 1, "sum": 2, "prod": 3, "maxpool": 4}
 TIES = {"low": 0, "high": 1}
 ORDERS = {"post": 0, "pre": 1}
 WEIGHTS = {"one": 0, "mean": 1}

@@ -222,15 +222,36 @@ def _score(a: np.ndarray, b: np.ndarray, score: str) -> np.ndarray:
     raise ValueError(score)
 
 
+def _maxpool(x: np.ndarray, p: int) -> np.ndarray:
+    """Max over each run of p consecutive values (one level up the pyramid)."""
+    return x.reshape(-1, p).max(axis=1)
+
+
 def scores_head(means_q, means_k, L: int, score: str = "max"):
     """Score of every entry of levels 1..L-1 (R2a). Default reading: max of the
     query and key squared norms; the alternatives kept behind this switch:
-    the key norm alone, the sum of the two norms, their product.
+    the key norm alone, the sum of the two norms, their product, and
+    "maxpool" ([LH] Fig. 2 step 2, "l2 norm + max-pool", read bottom-up from
+    level 0): a token scores max(|q|^2, |k|^2) of its own row, and an entry
+    the largest score among its p children.
 
     Level 0 is never ranked (only levels >= 1 are candidates for expansion),
-    so no level-0 score is formed. Returns (scores, sq_q, sq_k): lists indexed
-    by level, None at level 0.
+    so no level-0 score is returned. Returns (scores, sq_q, sq_k): lists
+    indexed by level, None at level 0; under "maxpool" sq_q / sq_k hold the
+    largest token norm under each entry, for queries and keys separately.
     """
+    if score == "maxpool":
+        if L == 1:
+            return [None], [None], [None]
+        p = len(means_q[0]) // len(means_q[1])
+        tq, tk = sq_norm_pinned(means_q[0]), sq_norm_pinned(means_k[0])
+        s = [np.maximum(tq, tk)]
+        sq_q, sq_k = [tq], [tk]
+        for l in range(1, L):
+            s.append(_maxpool(s[l - 1], p))
+            sq_q.append(_maxpool(sq_q[l - 1], p))
+            sq_k.append(_maxpool(sq_k[l - 1], p))
+        return [None] + s[1:], [None] + sq_q[1:], [None] + sq_k[1:]
     sq_q = [None] + [sq_norm_pinned(means_q[l]) for l in range(1, L)]
     sq_k = [None] + [sq_norm_pinned(means_k[l]) for l in range(1, L)]
     scores = [None] + [_score(sq_q[l], sq_k[l], score) for l in range(1, L)]

@@ -51,6 +51,11 @@ READINGS = [
     Case("partition_fp32", 1, 2, 1024, 64, "fp32", 4, 3, 32, inclusion="partition"),
     Case("all_alternatives_partition", 2, 3, 2048, 64, "bf16", 4, 3, 37, recipe="token_scale", score="sum",
          ties="high", order="pre", weight="mean", inclusion="partition"),
+    Case("score_maxpool", 1, 2, 4096, 128, "bf16", 4, 4, 40, score="maxpool"),
+    Case("score_maxpool_p3_fp32", 1, 2, 333, 64, "fp32", 3, 3, 5, score="maxpool"),
+    Case("score_maxpool_chunked_ties", 1, 1, 65536, 64, "bf16", 2, 2, 200, recipe="codebook", score="maxpool"),
+    Case("score_maxpool_partition", 1, 2, 4096, 128, "bf16", 8, 3, 20, recipe="token_scale", score="maxpool",
+         inclusion="partition", weight="mean"),
 ]
 
 

@@ -130,3 +130,39 @@ def test_weighted_scatter_and_blocksum_are_adjoint(weight):
     if w:   # weighted scatter of rows of ones: every token gets one 1/p^l per covering level
         ones = orc.scatter_head(np.ones((len(lvl), D)), lvl, idx, P, N, weighted=True)
         assert np.all(ones >= 1.0 / P ** (L - 1) - 1e-15)
+
+
+@pytest.mark.parametrize("p,l_", [(4, 3), (3, 4), (2, 5)])
+def test_maxpool_score_is_block_maximum_of_token_scores(p, l_):
+    """The recursive max-pool equals, for every entry, the maximum over the
+    tokens it covers of max(|q_t|^2, |k_t|^2) computed directly (a token's
+    squared norm in plain fp64 against the pinned order: the same value within
+    a few ulps, and the same maximiser); the returned per-side maxima
+    reproduce it as their max."""
+    n = p ** (l_ - 1) * 5
+    q, k = _tokens(20, n=n), _tokens(21, n=n)
+    mq, _ = orc.pool_head(q, p, l_, "bf16")
+    mk, _ = orc.pool_head(k, p, l_, "bf16")
+    scores, sq_q, sq_k = orc.scores_head(mq, mk, l_, "maxpool")
+    tok = np.maximum(np.sum(q * q, axis=1), np.sum(k * k, axis=1))
+    for l in range(1, l_):
+        span = p ** l
+        want = tok.reshape(-1, span).max(axis=1)
+        assert np.max(np.abs(scores[l] - want) / want) <= 64 * 2 ** -52
+        assert np.array_equal(scores[l], np.maximum(sq_q[l], sq_k[l]))
+
+
+def test_maxpool_selects_the_outlier_chain():
+    """One token with a much larger norm than all others: under the max-pool
+    score every ancestor of it scores highest at its level and is expanded
+    first, even with a budget of one entry per level; the mean-norm score
+    dilutes it by p^l and need not."""
+    p, l_, n = 4, 4, 4 ** 3 * 4
+    q = _tokens(22, n=n)
+    k = _tokens(23, n=n)
+    t = 137
+    q[t] *= 40.0
+    sel, inc = _select(q, k, "maxpool", p=p, l_=l_, k_=1)
+    for l in range(1, l_):
+        assert list(sel[l]) == [t // p ** l], l
+    assert t in inc[0]
