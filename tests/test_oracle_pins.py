@@ -240,6 +240,16 @@ def test_hand_worked_descent_and_order():
     assert list(fw["sel"][1]) == list(g["sel1"].astype(int))
     assert list(fw["lvl"]) == list(g["map_level"].astype(int))
     assert list(fw["idx"]) == list(g["map_index"].astype(int))
+    for order in ("post", "pre"):
+        fp = orc.forward_head(x, x, v, p, L, K, "bf16", order=order, inclusion="partition")
+        assert list(fp["sel"][2]) == list(g["sel2"].astype(int))
+        assert list(fp["lvl"]) == list(g["part_map_level"].astype(int)), order
+        assert list(fp["idx"]) == list(g["part_map_index"].astype(int)), order
+    fm = orc.forward_head(x, x, v, p, L, K, "bf16", score="maxpool")
+    assert list(fm["sel"][2]) == list(g["mp_sel2"].astype(int))
+    assert list(fm["sel"][1]) == list(g["mp_sel1"].astype(int))
+    assert list(fm["lvl"]) == list(g["mp_map_level"].astype(int))
+    assert list(fm["idx"]) == list(g["mp_map_index"].astype(int))
 
 
 def _check_order_invariants(lvl, idx, p, L, N, pl):
