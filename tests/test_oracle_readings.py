@@ -62,14 +62,16 @@ def test_sum_score_values_against_long_double():
         assert np.max(np.abs(s[l] - ext.astype(np.float64)) / ext.astype(np.float64)) <= 2 ** -52
 
 
+@pytest.mark.parametrize("score", ["max", "maxpool"])
 @pytest.mark.parametrize("ties", ["low", "high"])
-def test_ties_brute_force_on_equal_scores(ties):
-    """All tokens equal: every entry of a level has the same score, so the
-    selection is decided by the tie rule alone; brute force over Python
-    sorting of (score, index) pairs."""
+def test_ties_brute_force_on_equal_scores(ties, score):
+    """All tokens equal: every entry of a level has the same score (under the
+    max-pool reading too), so the selection is decided by the tie rule alone;
+    brute force over Python sorting of (score, index) pairs."""
     x = np.tile(_tokens(8, n=1), (N, 1))
     mq, _ = orc.pool_head(x, P, L, "bf16")
-    scores, _, _ = orc.scores_head(mq, mq, L)
+    scores, _, _ = orc.scores_head(mq, mq, L, score)
+    assert all(np.all(scores[l] == scores[l][0]) for l in range(1, L))
     sel, _ = orc.select_head(scores, P, L, K, ties)
     cand = list(range(len(scores[L - 1])))
     for l in range(L - 1, 0, -1):
