@@ -94,6 +94,19 @@ def stage_work(w, pl):
     }
 
 
+# GEMMs the tensor-core kernels issue per (query tile, key tile) pair of 128 x 128
+# (diagonal tiles included): forward S = Q K^T, then O += P_hi V and O += P_lo V;
+# backward dK/dV kernel S^T, dP^T, dV, dK and dQ kernel S, dP, dQ += dS_hi K,
+# dQ += dS_lo K. The algorithmic counts are 2 (forward) and 5 (backward).
+EXEC_GEMMS = {"attn_fwd": 3, "attn_bwd": 8}
+
+
+def executed_flops(w, pl, stage):
+    """MMA FLOPs the bf16 tensor-core attention kernels execute per launch."""
+    T = (pl.S + 127) // 128
+    return w.B * w.H * (T * (T + 1) // 2) * EXEC_GEMMS[stage] * 2.0 * 128 * 128 * w.D
+
+
 def sdpa_context(q, k, v, do, iters=2):
     """torch's own causal scaled_dot_product_attention, forward + backward, on the
     full token sequence of the same inputs (a library baseline, timed with CUDA
@@ -210,7 +223,9 @@ def run_reference(args, w):
         times.append(dt)
     per_head = sum(times) / len(times)
     value = (w.B * w.N) / (per_head * w.B * w.H)
-    sample = (f"one (b,h) head per step (N={w.N} tokens, whole pyramid, selection, S={lh_plan_S(w)} "
+    import oracle as orc
+    S = orc.plan(w.N, w.p, w.L, w.K).S
+    sample = (f"one (b,h) head per step (N={w.N} tokens, whole pyramid, selection, S={S} "
               f"sub-sequence, attention fwd+bwd, scatter/spread) of {w.B * w.H} heads; "
               f"tokens/s scaled to the whole job")
     line = {
@@ -226,8 +241,73 @@ def run_reference(args, w):
     print(json.dumps(line), flush=True)
 
 
-def lh_plan_S(w):
-    return lh.plan(lh.make_config(w.B, w.H, w.N, w.D, w.p, w.L, w.K, w.dtype, w.mode)).S
+def run_e2e(cfg, w, ws, q, k, v, do, results, stream, dev, world, steps):
+    """End to end through the public calls (lh_forward, lh_backward): every step
+    copies its inputs Q, K, V, dO from pinned host memory to the device and its
+    results O, dQ, dK, dV back into pinned host memory. Inputs of step i+1 go up
+    on one copy stream and results of step i come down on another while the next
+    step computes; each of the two device buffer sets is reused only after its
+    copies are done. `results`: the device-timed run's O, dQ, dK, dV, which the
+    last step's host copies must equal."""
+    hin = [x.cpu().pin_memory() for x in (q, k, v, do)]
+    hout = [torch.empty(q.shape, dtype=q.dtype).pin_memory() for _ in range(4)]
+    din = [[torch.empty_like(q) for _ in range(4)] for _ in range(2)]
+    dout_ = [[torch.empty_like(q) for _ in range(4)] for _ in range(2)]
+    up, down = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_comp = [torch.cuda.Event() for _ in range(2)]
+    ev_out = [torch.cuda.Event() for _ in range(2)]
+    used = [False, False]
+    h2d = sum(x.numel() * x.element_size() for x in hin)
+    d2h = sum(x.numel() * x.element_size() for x in hout)
+
+    def copy_in(i):
+        bi = i & 1
+        if used[bi]:
+            up.wait_event(ev_comp[bi])        # step i-2 is done reading these inputs
+        with torch.cuda.stream(up):
+            for dst, src in zip(din[bi], hin):
+                dst.copy_(src, non_blocking=True)
+        ev_in[bi].record(up)
+
+    def compute(i):
+        bi = i & 1
+        q_, k_, v_, do_ = din[bi]
+        o_, dq_, dk_, dv_ = dout_[bi]
+        stream.wait_event(ev_in[bi])
+        if used[bi]:
+            stream.wait_event(ev_out[bi])     # results of step i-2 are on the host
+        lh.forward(cfg, q_, k_, v_, o_, ws, stream)
+        lh.backward(cfg, do_, dq_, dk_, dv_, ws, stream)
+        ev_comp[bi].record(stream)
+        down.wait_event(ev_comp[bi])
+        with torch.cuda.stream(down):
+            for dst, src in zip(hout, dout_[bi]):
+                dst.copy_(src, non_blocking=True)
+        ev_out[bi].record(down)
+        used[bi] = True
+
+    def run(n):
+        copy_in(0)
+        for i in range(n):
+            if i + 1 < n:
+                copy_in(i + 1)
+            compute(i)
+
+    run(2)
+    torch.cuda.synchronize(dev)
+    lhdist.barrier()
+    a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(up)
+    run(steps)
+    b_.record(down)
+    torch.cuda.synchronize(dev)
+    e2e_ms = lhdist.max_over_ranks(a.elapsed_time(b_) / steps, dev)
+    ok = all(torch.equal(hx.to(dev), dx) for hx, dx in zip(hout, results))
+    return {"value": lhdist.job_throughput(w.B * w.N, world, e2e_ms / 1e3), "unit": "tokens/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "steps": steps,
+            "result": "O, dQ, dK, dV copied to pinned host memory every step",
+            "matches_device_run": ok}
 
 
 def main():
@@ -237,11 +317,13 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="lh", choices=["lh", "reference"])
     ap.add_argument("--workload", default="ctx512k", choices=list(synth.WORKLOADS))
-    ap.add_argument("--e2e-steps", type=int, default=2)
+    ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--sdpa-context", action="store_true",
-                    help="also time torch's scaled_dot_product_attention (causal, fwd+bwd) on the full "
-                         "token sequence of the same inputs, as context for the speed-up over dense attention")
+    ap.add_argument("--no-sdpa-context", action="store_true",
+                    help="skip the timing of torch's scaled_dot_product_attention (causal, fwd+bwd) on the full "
+                         "token sequence of the same inputs (context for the speed-up over dense attention)")
+    ap.add_argument("--no-fixed-mode", action="store_true",
+                    help="skip the timing of the same step in fixed-point accumulation mode")
     ap.add_argument("--heads", type=int, default=None,
                     help="smaller case of the same recipe (fewer heads), e.g. for an ncu capture")
     ap.add_argument("--tokens", type=int, default=None, help="smaller case of the same recipe (fewer tokens)")
@@ -270,122 +352,105 @@ def main():
     o, dq, dk, dv = (torch.empty_like(q) for _ in range(4))
     stream = torch.cuda.current_stream(dev)
     stages = ["pool", "select", "gather", "attn_fwd", "scatter", "scatter_bwd", "attn_bwd", "spread"]
+    fwd_stages = stages[:5]
 
-    def step(ev=None):
+    def step(c, ev=None):
         def mark(i):
             if ev is not None:
                 ev[i].record(stream)
         mark(0)
-        lh.pool(cfg, q, k, v, ws.pyr_q, ws.pyr_k, ws.pyr_v, ws.sq, stream)
+        lh.pool(c, q, k, v, ws.pyr_q, ws.pyr_k, ws.pyr_v, ws.sq, stream)
         mark(1)
-        lh.score_topk(cfg, ws.sq, ws.sel, ws.map, ws.slot, ws.ws, stream=stream)
+        lh.score_topk(c, ws.sq, ws.sel, ws.map, ws.slot, ws.ws, stream=stream)
         mark(2)
-        lh.gather(cfg, q, k, v, ws.pyr_q, ws.pyr_k, ws.pyr_v, ws.map, ws.qs, ws.ks, ws.vs, stream)
+        lh.gather(c, q, k, v, ws.pyr_q, ws.pyr_k, ws.pyr_v, ws.map, ws.qs, ws.ks, ws.vs, stream)
         mark(3)
-        lh.attn_fwd(cfg, ws.qs, ws.ks, ws.vs, ws.os, ws.lse, stream)
+        lh.attn_fwd(c, ws.qs, ws.ks, ws.vs, ws.os, ws.lse, stream)
         mark(4)
-        lh.scatter(cfg, ws.os, ws.slot, o, stream)
+        lh.scatter(c, ws.os, ws.slot, o, stream)
         mark(5)
-        lh.scatter_bwd(cfg, do, ws.os, ws.slot, ws.dos, ws.delta, stream)
+        lh.scatter_bwd(c, do, ws.os, ws.slot, ws.dos, ws.delta, stream)
         mark(6)
-        lh.attn_bwd(cfg, ws.qs, ws.ks, ws.vs, ws.dos, ws.lse, ws.delta, ws.dqs, ws.dks, ws.dvs, stream)
+        lh.attn_bwd(c, ws.qs, ws.ks, ws.vs, ws.dos, ws.lse, ws.delta, ws.dqs, ws.dks, ws.dvs, stream)
         mark(7)
-        lh.spread(cfg, ws.dqs, ws.dks, ws.dvs, ws.slot, dq, dk, dv, stream)
+        lh.spread(c, ws.dqs, ws.dks, ws.dvs, ws.slot, dq, dk, dv, stream)
         mark(8)
 
+    def timed(c, steps, sample_clocks=False):
+        """`steps` steps of config c after a barrier and a synchronize: total and
+        per-stage device ms (CUDA events on the launching stream), launches, clocks."""
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(stages) + 1)] for _ in range(steps)]
+        sampler = ClockSampler(local) if sample_clocks else None
+        lhdist.barrier()
+        torch.cuda.synchronize(dev)
+        if sampler:
+            sampler.start()
+            time.sleep(0.3)
+        launches0 = lh.launch_count()
+        t_start = torch.cuda.Event(enable_timing=True)
+        t_end = torch.cuda.Event(enable_timing=True)
+        t_start.record(stream)
+        for i in range(steps):
+            step(c, evs[i])
+        t_end.record(stream)
+        torch.cuda.synchronize(dev)
+        launches = lh.launch_count() - launches0
+        clocks = sampler.stop() if sampler else None
+        lhdist.barrier()
+        ms_total = lhdist.max_over_ranks(t_start.elapsed_time(t_end), dev)
+        per = {s: sum(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(steps)) / steps
+               for j, s in enumerate(stages)}
+        st, detail = lh.get_device_error(stream)
+        if st != 0:
+            raise RuntimeError(f"device error {st} ({detail}) in a timed region")
+        return ms_total / steps, per, launches, clocks
+
     for _ in range(max(args.warmup, 0)):
-        step()
+        step(cfg)
     torch.cuda.synchronize(dev)
     st, detail = lh.get_device_error(stream)
     if st != 0:
         raise RuntimeError(f"device error {st} ({detail}) during warm-up")
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(stages) + 1)]
-           for _ in range(args.steps)]
-    sampler = ClockSampler(local)
-    lhdist.barrier()
-    torch.cuda.synchronize(dev)
-    sampler.start()
-    time.sleep(0.3)
-    launches0 = lh.launch_count()
-    t_start = torch.cuda.Event(enable_timing=True)
-    t_end = torch.cuda.Event(enable_timing=True)
-    t_start.record(stream)
-    for i in range(args.steps):
-        step(evs[i])
-    t_end.record(stream)
-    torch.cuda.synchronize(dev)
-    launches = lh.launch_count() - launches0
-    clocks = sampler.stop()
-    lhdist.barrier()
-    ms_total = lhdist.max_over_ranks(t_start.elapsed_time(t_end), dev)
-    ms_step = ms_total / args.steps
-    stage_ms = {s: sum(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(args.steps)) / args.steps
-                for j, s in enumerate(stages)}
-    st, detail = lh.get_device_error(stream)
-    if st != 0:
-        raise RuntimeError(f"device error {st} ({detail}) in the timed region")
+    ms_step, stage_ms, launches, clocks = timed(cfg, args.steps, sample_clocks=True)
+    # forward alone: the device time of its five stages inside the same steps
+    fwd_ms = lhdist.max_over_ranks(sum(stage_ms[s] for s in fwd_stages), dev)
 
-    # end-to-end through the public API: pinned host inputs -> device, fwd + bwd, results -> host
+    # The same step in fixed-point accumulation mode (the pages' deterministic
+    # int-atomic scatter-back is their slower variant): only the scatter and the
+    # spread change arithmetic, every other stage is the same kernel.
+    fixed = None
+    if not args.no_fixed_mode and w.mode == "fp":
+        cfg_fx = lh.make_config(w.B, w.H, w.N, w.D, w.p, w.L, w.K, w.dtype, "fixed")
+        for _ in range(2):
+            step(cfg_fx)
+        fx_step, fx_stage, _, _ = timed(cfg_fx, args.steps)
+        fixed = {"ms_per_step": round(fx_step, 4),
+                 "scatter_ms": round(fx_stage["scatter"], 4), "spread_ms": round(fx_stage["spread"], 4),
+                 "int_vs_fp": {"scatter": round(fx_stage["scatter"] / stage_ms["scatter"], 3),
+                               "spread": round(fx_stage["spread"] / stage_ms["spread"], 3),
+                               "scatter_plus_spread": round((fx_stage["scatter"] + fx_stage["spread"]) /
+                                                            (stage_ms["scatter"] + stage_ms["spread"]), 3),
+                               "step": round(fx_step / ms_step, 3)},
+                 "pages": "int-atomic scatter-back 1.2-2x slower than fp-atomic (Lighthouse Attention Technique, "
+                          "throughput paragraph)"}
+        for _ in range(2):
+            step(cfg)                 # leave the default mode's results in place
+        torch.cuda.synchronize(dev)
+
+    # End to end through the public calls (lh_forward, lh_backward): every step
+    # copies its inputs Q, K, V, dO from pinned host memory to the device and its
+    # results O, dQ, dK, dV back into pinned host memory. Inputs of step i+1 go up
+    # on one copy stream and results of step i come down on another while the next
+    # step computes; each of the two device buffer sets is reused only after its
+    # copies are done.
     e2e = None
     if args.e2e_steps > 0:
-        # End to end through the public calls: every step copies its inputs
-        # (Q, K, V, dO) from pinned host memory and reads back the step's loss,
-        # sum(O * dO) as an fp32 scalar; O and the gradients stay on the device,
-        # as in training. The next step's inputs are copied on a second stream
-        # into the other of two device buffer sets while this step computes.
-        hq, hk, hv, hdo = (x.cpu().pin_memory() for x in (q, k, v, do))
-        bufs = [[torch.empty_like(q) for _ in range(4)] for _ in range(2)]
-        o_, dq_, dk_, dv_ = (torch.empty_like(q) for _ in range(4))
-        loss_d = torch.empty((), dtype=torch.float32, device=dev)
-        loss_h = torch.empty((), dtype=torch.float32).pin_memory()
-        cs = torch.cuda.Stream(device=dev)
-        ev_in = [torch.cuda.Event() for _ in range(2)]
-        ev_done = [torch.cuda.Event() for _ in range(2)]
-        h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv, hdo))
-        d2h = loss_h.numel() * loss_h.element_size()
-
-        def copy_in(i):
-            bi = i & 1
-            if i >= 2:
-                cs.wait_event(ev_done[bi])        # step i-2 is done with these buffers
-            with torch.cuda.stream(cs):
-                for dst, src in zip(bufs[bi], (hq, hk, hv, hdo)):
-                    dst.copy_(src, non_blocking=True)
-            ev_in[bi].record(cs)
-
-        def compute(i):
-            bi = i & 1
-            q_, k_, v_, do_ = bufs[bi]
-            stream.wait_event(ev_in[bi])
-            lh.forward(cfg, q_, k_, v_, o_, ws, stream)
-            lh.backward(cfg, do_, dq_, dk_, dv_, ws, stream)
-            with torch.cuda.stream(stream):
-                loss_d.copy_(torch.sum(o_ * do_, dtype=torch.float32))
-                loss_h.copy_(loss_d, non_blocking=True)
-            ev_done[bi].record(stream)
-
-        def run(n):
-            copy_in(0)
-            for i in range(n):
-                if i + 1 < n:
-                    copy_in(i + 1)
-                compute(i)
-
-        run(2)
-        torch.cuda.synchronize(dev)
-        lhdist.barrier()
-        a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(cs)
-        run(args.e2e_steps)
-        b_.record(stream)
-        torch.cuda.synchronize(dev)
-        e2e_ms = lhdist.max_over_ranks(a.elapsed_time(b_) / args.e2e_steps, dev)
-        e2e = {"value": lhdist.job_throughput(w.B * w.N, world, e2e_ms / 1e3), "unit": "tokens/s",
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
-               "result": "loss = sum(O * dO), fp32, read back every step"}
+        e2e = run_e2e(cfg, w, ws, q, k, v, do, (o, dq, dk, dv), stream, dev, world, args.e2e_steps)
+        torch.cuda.empty_cache()
 
     peaks, peak_kind = load_peaks()
+    tc_peak_key = "bf16_tflops"      # a few-second timed region of ~15 ms steps: the burst figure
     work = stage_work(w, pl)
     frac = {}
     for s in stages:
@@ -400,25 +465,30 @@ def main():
         else:
             ach = amount / sec / 1e12
             frac[s] = {"ms": round(stage_ms[s], 4), "achieved": round(ach, 2), "unit": "TFLOP/s",
-                       "frac": round(ach / peaks["bf16_tflops_sustained"], 4), "bound": "tensor"}
+                       "frac": round(ach / peaks[tc_peak_key], 4), "bound": "tensor"}
+            if w.dtype == "bf16":
+                ex = executed_flops(w, pl, s) / sec / 1e12
+                frac[s].update(executed=round(ex, 2), executed_frac=round(ex / peaks[tc_peak_key], 4),
+                               executed_gemms_per_tile_pair=EXEC_GEMMS[s])
     dom = max(frac, key=lambda s: stage_ms[s])
     kind, amount = work[dom]
+    full_size = (w.B, w.H, w.N) == (synth.WORKLOADS[w.name].B, synth.WORKLOADS[w.name].H,
+                                    synth.WORKLOADS[w.name].N)
     roofline = {
         "kernel": dom, "bound": frac[dom]["bound"], "achieved": frac[dom]["achieved"],
-        "peak": peaks["hbm_gbs"] if kind == "bytes" else peaks["bf16_tflops_sustained"],
+        "peak": peaks["hbm_gbs"] if kind == "bytes" else peaks[tc_peak_key],
         "unit": frac[dom]["unit"], "frac": frac[dom]["frac"],
-        "traffic": (DRAM_TRAFFIC.get(w.name, {}).get(dom)
-                    if (w.B, w.H, w.N) == (synth.WORKLOADS[w.name].B, synth.WORKLOADS[w.name].H,
-                                           synth.WORKLOADS[w.name].N) else None),
+        "traffic": DRAM_TRAFFIC.get(w.name, {}).get(dom) if full_size else None,
         "traffic_unit": "bytes per call",
-        "peak_source": f"{peak_kind} ({'hbm_gbs' if kind == 'bytes' else 'bf16_tflops_sustained'})",
+        "peak_source": f"{peak_kind} ({'hbm_gbs' if kind == 'bytes' else tc_peak_key})",
     }
 
     context = None
-    if args.sdpa_context and rank == 0:
+    if not args.no_sdpa_context and rank == 0 and world == 1:
         context = sdpa_context(q, k, v, do)
         if "ms_per_step" in context:
-            context["lighthouse_speedup"] = context["ms_per_step"] / ms_step
+            context["lighthouse_speedup_fwd_bwd"] = round(context["ms_per_step"] / ms_step, 2)
+            context["pages"] = "17.3x fwd+bwd and 21x fwd over standard attention at 512K on one B200 (zubnet)"
 
     cpu_baseline = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -435,9 +505,13 @@ def main():
         "config": {"workload": workload_desc(w), "S": pl.S,
                    "l2": "inputs larger than L2 (Q, K, V, dO: 8.6 GB per step), no flush",
                    "parallelism": f"dp{world} (independent batches per GPU)"},
+        "fwd": {"value": lhdist.job_throughput(w.B * w.N, world, fwd_ms / 1e3), "unit": "tokens/s",
+                "ms": round(fwd_ms, 4), "stages": fwd_stages},
         "roofline": roofline, "stages": frac, "cpu_baseline": cpu_baseline, "e2e": e2e,
         "gpu_launches": launches, "clocks": clocks,
     }
+    if fixed is not None:
+        line["fixed_mode"] = fixed
     if context is not None:
         line["context_sdpa"] = context
     if rank == 0:

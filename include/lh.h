@@ -24,6 +24,11 @@
  *    failed (cudaGetLastError was not cudaSuccess after it).
  *  - Element types: `dtype` buffers hold bf16 or fp32 per lh_config.dtype;
  *    buffers typed float / double / int32_t below are always that type.
+ *  - liblh looks up the device address of its device error word (and, for
+ *    lh_score_topk_noalloc, of its scratch array) once per device and keeps it
+ *    for the life of the process. cudaDeviceReset unloads the library's device
+ *    code and so invalidates those addresses: a process that resets a device
+ *    must not call liblh on that device afterwards.
  *
  * Layouts (row-major, last index fastest):
  *   tokens  Q, K, V, O, dO, dQ, dK, dV     [B][N][H][D]   dtype
@@ -288,7 +293,9 @@ lh_status lh_selftest_timeout(long long limit_cycles, int* gave_up, void* stream
  * LH_ERR_WORKSPACE when the problem needs more scratch than the array holds
  * (plan.ws_bytes > 8 MiB, i.e. 5*B*H*(sum of m_l) > 2,097,152; checked before any launch).
  * The first call on each device looks up the array's device address
- * (cudaGetSymbolAddress), so make that first call before any stream capture.
+ * (cudaGetSymbolAddress), so make that first call before any stream capture;
+ * the address is kept for the life of the process (see the note on
+ * cudaDeviceReset at the top of this file).
  * All calls share the one array, and it keeps the previous call's contents
  * (every scratch word is written before it is read, so nothing needs
  * clearing). Calls that overlap on the GPU, from different streams or host

@@ -146,6 +146,26 @@ def test_repeat_runs_bit_exact():
             assert torch.equal(a, b)
 
 
+def test_ties131k_three_runs_bit_exact():
+    """The tie/determinism workload at full size (B1 H8 N131072 D128, p4 L5 K512,
+    codebook inputs with many exactly tied scores, fixed-point accumulation):
+    three runs of the whole forward and backward give identical bits."""
+    w = synth.WORKLOADS["ties131k"]
+    case = case_of(w)
+    assert case.accum == "fixed"
+    q, k, v = synth.make_inputs(w, device=DEV)
+    do = synth.make_dout(w, device=DEV)
+    outs = []
+    for _ in range(3):
+        r = run_gpu(case, q, k, v, do)
+        ws = r["ws"]
+        outs.append([r[n].clone() for n in ("o", "dq", "dk", "dv")] + [ws.sel.clone(), ws.map.clone()])
+        del r, ws
+    for other in outs[1:]:
+        for a, b in zip(outs[0], other):
+            assert torch.equal(a, b)
+
+
 def test_autograd_wrapper_matches_stagewise():
     case = Case("autograd", 1, 2, 4096, 64, "bf16", 4, 3, 32)
     q, k, v, do = _inputs(case)

@@ -4,6 +4,9 @@ invariances of the selection, a brute-force sort, an independent recursive
 walk of the selection tree, and adjointness of the weighted scatter pair.
 """
 
+import math
+import os
+
 import numpy as np
 import pytest
 
@@ -168,3 +171,35 @@ def test_maxpool_selects_the_outlier_chain():
     for l in range(1, l_):
         assert list(sel[l]) == [t // p ** l], l
     assert t in inc[0]
+
+
+def _read_score_golden():
+    vals = {}
+    with open(os.path.join(os.path.dirname(__file__), "golden", "score_readings.txt")) as f:
+        for line in f:
+            if line.startswith("#") or ":" not in line:
+                continue
+            key, rest = line.split(":", 1)
+            vals[key.strip()] = np.array([float(t) for t in rest.split()])
+    return vals
+
+
+@pytest.mark.parametrize("score", ["max", "k", "sum", "prod"])
+def test_hand_worked_score_readings_with_distinct_queries(score):
+    """Hand-worked scores and selections (tests/golden/score_readings.txt) with
+    Q != K, chosen so that each of the four pooled-entry scores expands a
+    different pair: a slip such as a sum of squared norms, a missing square
+    root or max() in place of the product selects another pair and fails here."""
+    g = _read_score_golden()
+    N, p, L_, K_, D_ = 8, 2, 2, 1, 8
+    q = np.repeat(g["a"][:, None], D_, axis=1)
+    k = np.repeat(g["b"][:, None], D_, axis=1)
+    v = np.repeat(np.arange(N, dtype=np.float64)[:, None], D_, axis=1)
+    fw = orc.forward_head(q, k, v, p, L_, K_, "bf16", score=score)
+    want = g["score_sum_over_sqrt8"] * math.sqrt(8.0) if score == "sum" else g[f"score_{score}"]
+    np.testing.assert_allclose(fw["scores"][1], want, rtol=1e-15, atol=0)
+    assert list(fw["sel"][1]) == [int(g[f"sel_{score}"][0])]
+    assert list(fw["lvl"]) == list(g[f"map_level_{score}"].astype(int))
+    assert list(fw["idx"]) == list(g[f"map_index_{score}"].astype(int))
+    # the four winners are pairwise distinct (the fixture separates the readings)
+    assert len({int(g[f"sel_{s}"][0]) for s in ("max", "k", "sum", "prod")}) == 4
