@@ -14,3 +14,4 @@ description is silent.
 """
 
 from .lighthouse import *  # noqa: F401,F403
+from . import sharded  # noqa: F401,E402

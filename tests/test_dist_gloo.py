@@ -64,3 +64,110 @@ def test_batch_rows_partition(gb, world):
     flat = [i for rr in rows for i in rr]
     assert flat == list(range(gb))
     assert max(len(r) for r in rows) - min(len(r) for r in rows) <= 1
+
+
+# ---------------------------------------------------------------------------
+# sequence-sharded (context-parallel) oracle: distributed top-K descent
+# ---------------------------------------------------------------------------
+
+from oracle import sharded  # noqa: E402
+
+
+class _GlooComm:
+    """all_gather of Python objects over the default torch.distributed group."""
+
+    def __init__(self):
+        import torch.distributed as dist
+        self._dist = dist
+        self.rank, self.world = dist.get_rank(), dist.get_world_size()
+
+    def all_gather(self, obj):
+        out = [None] * self.world
+        self._dist.all_gather_object(out, obj)
+        return out
+
+
+def _cp_inputs(N=512, D=16, seed=3):
+    rng = np.random.default_rng(seed)
+    return [orc.round_to_dtype(rng.standard_normal((N, D)), "bf16") for _ in range(4)]
+
+
+def _cp_worker(rank, world, port, args, out_dir):
+    os.environ.update(RANK=str(rank), WORLD_SIZE=str(world), LOCAL_RANK=str(rank),
+                      MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    assert lhdist.init("gloo", timeout_s=60)
+    q, k, v, do, p, L, K = args
+    comm = _GlooComm()
+    n = q.shape[0] // world
+    sl = slice(rank * n, (rank + 1) * n)
+    fw = sharded.forward_shard(comm, q[sl], k[sl], v[sl], p, L, K, "bf16")
+    bw = sharded.backward_shard(comm, fw, do[sl], p)
+    np.savez(os.path.join(out_dir, f"cp{rank}.npz"), lvl=fw["lvl"], idx=fw["idx"], o=fw["o"],
+             seg=np.array(fw["seg"]), dq=bw["dq"], dk=bw["dk"], dv=bw["dv"],
+             **{f"sel{l}": fw["sel"][l] for l in range(1, L)})
+    lhdist.shutdown()
+
+
+def test_sequence_sharded_oracle_over_gloo_equals_single_process(tmp_path):
+    """Two gloo ranks, each holding half of one head's tokens, run the sharded
+    forward and backward (local pool and scores, per-level all-gather of local
+    top-k candidates, all-gather of the sub-sequence K and V, reduce of the
+    key gradients). The selection, the gather map (the ranks' segments in rank
+    order) and the output equal the single-process oracle bit for bit; the
+    gradients, whose key-side sums are grouped by rank, agree to 1e-12."""
+    world, p, L, K = 2, 4, 3, 6
+    q, k, v, do = _cp_inputs()
+    mp.start_processes(_cp_worker, args=(world, _free_port(), (q, k, v, do, p, L, K), str(tmp_path)),
+                       nprocs=world, join=True, start_method="spawn")
+    parts = [np.load(tmp_path / f"cp{r}.npz") for r in range(world)]
+    ref = orc.forward_head(q, k, v, p, L, K, "bf16")
+    rb = orc.backward_head(ref, do, p)
+    for l in range(1, L):
+        for part in parts:
+            assert np.array_equal(part[f"sel{l}"], ref["sel"][l])
+    assert np.array_equal(np.concatenate([x["lvl"] for x in parts]), ref["lvl"])
+    assert np.array_equal(np.concatenate([x["idx"] for x in parts]), ref["idx"])
+    assert parts[0]["seg"][0] == 0 and parts[1]["seg"][0] == parts[0]["seg"][1]
+    assert np.array_equal(np.concatenate([x["o"] for x in parts]), ref["o"])
+    for name in ("dq", "dk", "dv"):
+        assert np.max(np.abs(np.concatenate([x[name] for x in parts]) - rb[name])) < 1e-12
+
+
+@pytest.mark.parametrize("world", [1, 2, 4, 8])
+@pytest.mark.parametrize("readings", [
+    {}, {"ties": "high"}, {"score": "maxpool"}, {"inclusion": "partition"},
+    {"score": "sum", "order": "pre", "weight": "mean"},
+])
+def test_sequence_sharded_oracle_ranks_in_one_process(world, readings):
+    """The same decomposition with the ranks as threads of one process, for
+    every reading switch and up to 8 ranks (a shard down to one coarsest
+    block), including exactly tied scores (codebook rows)."""
+    p, L, K = 2, 4, 3
+    rng = np.random.default_rng(world)
+    N, D = 128, 8
+    book = orc.round_to_dtype(rng.standard_normal((4, D)), "bf16")
+    q = book[rng.integers(0, 4, N)]                     # many exactly tied scores
+    k = book[rng.integers(0, 4, N)]
+    v, do = (orc.round_to_dtype(rng.standard_normal((N, D)), "bf16") for _ in range(2))
+    n = N // world
+
+    def fn(comm):
+        sl = slice(comm.rank * n, (comm.rank + 1) * n)
+        fw = sharded.forward_shard(comm, q[sl], k[sl], v[sl], p, L, K, "bf16", **readings)
+        return fw, sharded.backward_shard(comm, fw, do[sl], p)
+
+    res = sharded.run_local(world, fn)
+    ref = orc.forward_head(q, k, v, p, L, K, "bf16", **readings)
+    rb = orc.backward_head(ref, do, p)
+    for l in range(1, L):
+        assert all(np.array_equal(f["sel"][l], ref["sel"][l]) for f, _ in res)
+    assert np.array_equal(np.concatenate([f["lvl"] for f, _ in res]), ref["lvl"])
+    assert np.array_equal(np.concatenate([f["idx"] for f, _ in res]), ref["idx"])
+    assert np.array_equal(np.concatenate([f["o"] for f, _ in res]), ref["o"])
+    for name in ("dq", "dk", "dv"):
+        assert np.max(np.abs(np.concatenate([b[name] for _, b in res]) - rb[name])) < 1e-12
+
+
+def test_sequence_sharded_oracle_rejects_unaligned_shards():
+    with pytest.raises(ValueError):
+        sharded.shard_sizes(96, 4, 3, 4)                # 24 tokens per rank, not a multiple of 16
