@@ -241,6 +241,60 @@ def run_reference(args, w):
     print(json.dumps(line), flush=True)
 
 
+def measure_fusion(cfg, w, ws, dev, iters=3):
+    """The path's two ends with the model's projections next to them (x W_q,
+    x W_k, x W_v before the pool; O W_o after the scatter; d_model = H * D,
+    random weights): run one after the other over the whole sequence, and
+    chunk by chunk through L2 (long_context_symmetric_b200.fused). Device ms
+    per call, CUDA events, median of `iters` after one warm-up."""
+    from long_context_symmetric_b200 import fused
+    g = torch.Generator(device=dev).manual_seed(11)
+    B, N, dm = w.B, w.N, w.H * w.D
+    x = torch.randn(B, N, dm, generator=g, device=dev).to(torch.bfloat16)
+    wt = [(torch.randn(dm, dm, generator=g, device=dev) / dm ** 0.5).to(torch.bfloat16) for _ in range(4)]
+    q, k, v, o = (torch.empty(B, N, w.H, w.D, dtype=torch.bfloat16, device=dev) for _ in range(4))
+    y = torch.empty(B, N, dm, dtype=torch.bfloat16, device=dev)
+
+    def qkv_unfused():
+        for b in range(B):
+            for wi, out in zip(wt[:3], (q, k, v)):
+                torch.matmul(x[b], wi, out=out[b].view(N, dm))
+        lh.pool(cfg, q, k, v, ws.pyr_q, ws.pyr_k, ws.pyr_v, ws.sq)
+
+    def qkv_chunked():
+        fused.qkv_project_pool(cfg, ws, x, wt[0], wt[1], wt[2], q, k, v)
+
+    def out_unfused():
+        lh.scatter(cfg, ws.os, ws.slot, o)
+        for b in range(B):
+            torch.matmul(o[b].view(N, dm), wt[3], out=y[b])
+
+    def out_chunked():
+        fused.scatter_project(cfg, ws, wt[3], o, y)
+
+    def timeit(fn):
+        fn()
+        torch.cuda.synchronize(dev)
+        ts = []
+        for _ in range(iters):
+            a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b_.record()
+            torch.cuda.synchronize(dev)
+            ts.append(a.elapsed_time(b_))
+        return round(statistics.median(ts), 4)
+
+    res = {"d_model": dm, "chunk_tokens": fused.chunk_tokens(cfg),
+           "qkv_projection_plus_pool_ms": {"unfused": timeit(qkv_unfused), "chunked_l2": timeit(qkv_chunked)},
+           "scatter_plus_out_projection_ms": {"unfused": timeit(out_unfused), "chunked_l2": timeit(out_chunked)},
+           "projections": "cuBLAS bf16 GEMMs through torch.matmul (the model's, outside the path)"}
+    st, detail = lh.get_device_error()
+    if st != 0:
+        raise RuntimeError(f"device error {st} ({detail}) in the fusion timing")
+    return res
+
+
 def run_e2e(cfg, w, ws, q, k, v, do, results, stream, dev, world, steps):
     """End to end through the public calls (lh_forward, lh_backward): every step
     copies its inputs Q, K, V, dO from pinned host memory to the device and its
@@ -324,6 +378,8 @@ def main():
                          "token sequence of the same inputs (context for the speed-up over dense attention)")
     ap.add_argument("--no-fixed-mode", action="store_true",
                     help="skip the timing of the same step in fixed-point accumulation mode")
+    ap.add_argument("--no-fusion", action="store_true",
+                    help="skip the timing of the projections fused with pool / scatter chunk by chunk")
     ap.add_argument("--heads", type=int, default=None,
                     help="smaller case of the same recipe (fewer heads), e.g. for an ncu capture")
     ap.add_argument("--tokens", type=int, default=None, help="smaller case of the same recipe (fewer tokens)")
@@ -497,6 +553,10 @@ def main():
                         "sample": f"oracle fwd+bwd of head (0,0) of {workload_desc(w)}; {dt:.1f} s; "
                                   f"tokens/s scaled to all {w.B * w.H} heads"}
 
+    fusion = None
+    if not args.no_fusion and rank == 0 and world == 1 and w.dtype == "bf16" and w.L > 1:
+        fusion = measure_fusion(cfg, w, ws, dev)
+
     value = lhdist.job_throughput(w.B * w.N, world, ms_step / 1e3)
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
@@ -514,6 +574,8 @@ def main():
         line["fixed_mode"] = fixed
     if context is not None:
         line["context_sdpa"] = context
+    if fusion is not None:
+        line["fusion"] = fusion
     if rank == 0:
         print(json.dumps(line), flush=True)
     lhdist.shutdown()

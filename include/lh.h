@@ -243,6 +243,23 @@ lh_status lh_attn_bwd(const lh_config* cfg, const void* qs, const void* ks, cons
 lh_status lh_spread(const lh_config* cfg, const float* dqs, const float* dks, const float* dvs,
                     const int32_t* slot, void* dq, void* dk, void* dv, void* stream);
 
+/* Token-range forms of lh_pool and lh_scatter, for fusing the path with the
+ * projections next to it ("Long Context Pre-Training with Lighthouse
+ * Attention", Fig. 1: the Q/K/V projections feed the pyramid pool, the
+ * scatter-back feeds the output projection). A caller that produces Q, K, V
+ * chunk by chunk pools each chunk right after its projection wrote it, while
+ * the chunk is still in L2, and scatters the output chunk by chunk just before
+ * the output projection reads it. Only the tokens [t0, t0 + nt) of every
+ * sequence are read (lh_pool_range) or written (lh_scatter_range), with the
+ * pyramid entries, norms, slot table and sub-sequence rows at their places in
+ * the whole problem's buffers; the results equal lh_pool / lh_scatter's for
+ * those tokens bit for bit. t0 and nt: multiples of p^(L-1), t0 + nt <= N;
+ * L >= 2. Errors as lh_pool / lh_scatter, LH_ERR_SHAPE for a bad range. */
+lh_status lh_pool_range(const lh_config* cfg, int t0, int nt, const void* q, const void* k, const void* v,
+                        void* pyr_q, void* pyr_k, void* pyr_v, double* sq, void* stream);
+lh_status lh_scatter_range(const lh_config* cfg, int t0, int nt, const float* os, const int32_t* slot, void* o,
+                           void* stream);
+
 /* Device buffers of one forward+backward, caller-owned (sizes from lh_plan). */
 typedef struct {
   void *pyr_q, *pyr_k, *pyr_v;   /* [B][H][E][D] dtype */
@@ -264,6 +281,75 @@ lh_status lh_forward(const lh_config* cfg, const void* q, const void* k, const v
 lh_status lh_backward(const lh_config* cfg, const void* dout, void* dq, void* dk, void* dv,
                       const lh_buffers* bufs, void* stream);
 
+/* ---------------------------------------------------------------------------
+ * Sequence-sharded (context-parallel) path. The pages train at 1M-token
+ * context over 32 B200s with context parallelism ("Nous Research's
+ * Lighthouse Attention Trains 1.69x Faster on Million-Token Contexts", key
+ * points; "Lighthouse Attention Technique": past 100K context the model is
+ * scaled with context parallelism). Here rank r of `world` holds tokens
+ * [r n, (r+1) n) of every sequence, n = N / world a multiple of p^(L-1), so
+ * each pyramid entry lies in one shard. `cfg` always describes the WHOLE
+ * sequence (N = world * n); L >= 2. One step, with the collectives the caller
+ * runs between the calls (NCCL over NVLink: the steps are stream-ordered and
+ * never wait on another rank):
+ *   lh_cp_pool                 shard's pyramid and squared norms sq_loc
+ *   all-gather of sq_loc into sq_gathered [world][2][B][H][E_loc]
+ *   lh_cp_assemble_sq          -> sq [2][B][H][E] of the whole sequence
+ *   lh_score_topk              the whole selection, map and slot table (the same
+ *                              on every rank: every rank runs the same descent)
+ *   lh_cp_segment              -> slot_loc [B][H][E_loc] (this rank's entries;
+ *                              values are slots of the whole sub-sequence) and
+ *                              seg [B][H][2] int32 = (first slot, count) of this
+ *                              rank's entries: one contiguous run, since the
+ *                              sub-sequence is sorted by position (Fig. 1)
+ *   lh_cp_gather               rows of qs, ks, vs [B][H][S][D] (S of the whole
+ *                              sequence): this rank's segment, zero elsewhere
+ *   all-reduce (sum) of ks and of vs: every rank then holds all key/value rows
+ *   lh_cp_attn_fwd             the segment's rows of os, lse (queries of the
+ *                              segment over all keys before them)
+ *   lh_cp_scatter              the shard's output tokens
+ * Backward:
+ *   lh_cp_scatter_bwd          the segment's rows of dos, delta (other rows of
+ *                              dos are set to zero)
+ *   lh_cp_attn_bwd             dqs for the segment's rows; dks, dvs for ALL rows:
+ *                              the contribution of this rank's queries
+ *   all-reduce (sum) of dks and of dvs
+ *   lh_cp_spread               the shard's dq, dk, dv
+ * Buffers named like the single-GPU ones have the same layouts, with the
+ * shard's tokens ([B][n][H][D]) and entries (E_loc per (b, h)). The attention
+ * steps need bf16 I/O (tensor-core kernels): LH_ERR_DTYPE otherwise. Errors:
+ * LH_ERR_SHAPE also for world < 1, rank outside [0, world), L < 2, or shards
+ * that are not whole coarsest blocks. */
+typedef struct {
+  int world, rank;
+  int n_loc;                       /* tokens per rank */
+  int E_loc;                       /* entries of levels >= 1 per rank and (b, h) */
+  int lvl_off_loc[LH_MAX_LEVELS];  /* start of level l within E_loc (l >= 1) */
+  lh_plan_t global;                /* plan of the whole sequence (S = rows of qs ... dvs) */
+} lh_cp_plan_t;
+
+lh_status lh_cp_plan(const lh_config* cfg, int world, int rank, lh_cp_plan_t* out);
+lh_status lh_cp_pool(const lh_config* cfg, int world, int rank, const void* q, const void* k, const void* v,
+                     void* pyr_q, void* pyr_k, void* pyr_v, double* sq_loc, void* stream);
+lh_status lh_cp_assemble_sq(const lh_config* cfg, int world, const double* sq_gathered, double* sq,
+                            void* stream);
+lh_status lh_cp_segment(const lh_config* cfg, int world, int rank, const int32_t* map, const int32_t* slot,
+                        int32_t* slot_loc, int32_t* seg, void* stream);
+lh_status lh_cp_gather(const lh_config* cfg, int world, int rank, const void* q, const void* k, const void* v,
+                       const void* pyr_q, const void* pyr_k, const void* pyr_v, const int32_t* map,
+                       const int32_t* seg, void* qs, void* ks, void* vs, void* stream);
+lh_status lh_cp_attn_fwd(const lh_config* cfg, int world, int rank, const int32_t* seg, const void* qs,
+                         const void* ks, const void* vs, float* os, float* lse, void* stream);
+lh_status lh_cp_scatter(const lh_config* cfg, int world, int rank, const float* os, const int32_t* slot_loc,
+                        void* o, void* stream);
+lh_status lh_cp_scatter_bwd(const lh_config* cfg, int world, int rank, const void* dout, const float* os,
+                            const int32_t* slot_loc, const int32_t* seg, void* dos, float* delta, void* stream);
+lh_status lh_cp_attn_bwd(const lh_config* cfg, int world, int rank, const int32_t* seg, const void* qs,
+                         const void* ks, const void* vs, const void* dos, const float* lse, const float* delta,
+                         float* dqs, float* dks, float* dvs, void* stream);
+lh_status lh_cp_spread(const lh_config* cfg, int world, int rank, const float* dqs, const float* dks,
+                       const float* dvs, const int32_t* slot_loc, void* dq, void* dk, void* dv, void* stream);
+
 /* Reads and clears the device error word set by bounded waits and device
  * checks (LH_OK, LH_ERR_TIMEOUT or LH_ERR_DEVICE); *detail receives the
  * kernel-specific code (0 if none). Synchronises `stream`. */
@@ -281,6 +367,16 @@ unsigned long long lh_launch_count(void);
  * when the wait gave up. LH_ERR_NULL / LH_ERR_SHAPE for bad arguments, checked
  * before the launch. */
 lh_status lh_selftest_timeout(long long limit_cycles, int* gave_up, void* stream);
+
+/* Diagnostics (the pages have no counterpart: this checks an arithmetic
+ * building block). The attention kernels compute part of each softmax tile's
+ * exponentials 2^x with a polynomial on the FMA pipe instead of the
+ * special-function unit's ex2.approx (range reduction to [-1/2, 1/2], degree-5
+ * minimax polynomial, exponent added in the bit pattern; inputs below -125 give
+ * 2^-125). This evaluates both on n device floats x: y_fma[i] from the
+ * polynomial, y_sfu[i] from ex2.approx.ftz.f32. Device buffers of n floats.
+ * LH_ERR_NULL / LH_ERR_SHAPE before any launch; LH_ERR_CUDA if the launch fails. */
+lh_status lh_selftest_exp2(const float* x, float* y_fma, float* y_sfu, int n, void* stream);
 
 /* lh_score_topk without a caller workspace (the paper has no counterpart: this
  * is for callers, not the method). Some callers cannot provide or allocate a

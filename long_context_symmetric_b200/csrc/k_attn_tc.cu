@@ -21,7 +21,9 @@
 //             other tile (about 1.5 tiles of MMA time for 1 tile of softmax).
 //   warps 2-5 softmax of tile A, warps 6-9 of tile B; one thread per query row
 //             (= TMEM lane): scores from TMEM, causal mask on the diagonal
-//             tile, online softmax in the exp2 domain with a lazily updated
+//             tile, online softmax in the exp2 domain (a quarter of the
+//             exponentials by a polynomial on the FMA pipe, the rest on the
+//             special-function unit) with a lazily updated
 //             running max (O is rescaled in TMEM only when the max grows by
 //             more than 2^8); P is split into an fp16 head and an fp16
 //             remainder written into the score columns (each 32-column chunk
@@ -51,6 +53,11 @@ constexpr int kBN = 128;       // key rows per tile
 constexpr int kSub = 128 * 64 * 2;   // one 128-row x 64-column 16-bit swizzle tile (16 KB)
 constexpr float kLn2f = 0.6931471805599453f;
 constexpr int kFwdThreads = 320;
+// Column pairs of every 8 whose exponentials run on the FMA pipe (tc::exp2_fma2)
+// instead of the special-function unit: ex2 alone would keep that unit busy
+// 8 cycles per warp instruction while the rest of the softmax needs about
+// 5 issue cycles per pair, so moving a quarter of the pairs balances the two.
+constexpr int kFwdFmaPairs = 3;
 
 // Barriers first, then the swizzled tiles from the next 1024-byte boundary.
 template <int D>
@@ -80,7 +87,7 @@ template <int D>
 __global__ void __launch_bounds__(kFwdThreads, 1)
 k_attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
               const __grid_constant__ CUtensorMap tv, float* __restrict__ os, float* __restrict__ lse,
-              int S, float c2, int* err) {
+              int S, float c2, const int* __restrict__ seg, int* err) {
   using Lay = FwdLayout<D>;
   constexpr int SUB = Lay::SUB;
   constexpr uint32_t IDS = idesc_f16(kBM, kBN, false);    // S = Q K^T, both K-major
@@ -90,13 +97,21 @@ k_attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CU
   uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + Lay::HEAD + 1023) & ~(uintptr_t)1023);
   const uint32_t sbase = smem_u32(sm);
 
-  const int ntiles = (S + kBM - 1) / kBM;
-  const int mp = (int)gridDim.x - 1 - (int)blockIdx.x;
+  // Query rows of this (b, h): rows [q0, q0 + nq) of qs attend to key rows
+  // [0, q0 + nq) of ks / vs (the whole sub-sequence, or one rank's segment of
+  // it in the sequence-sharded path, `seg` = (q0, nq) per (b, h)).
+  const int bh = blockIdx.y;
+  const int q0 = seg ? seg[2 * bh] : 0, nq = seg ? seg[2 * bh + 1] : S;
+  const int ntiles = (nq + kBM - 1) / kBM;
+  const int mp = (ntiles + 1) / 2 - 1 - (int)blockIdx.x;     // heavy (late) pairs first
+  if (mp < 0) return;                                          // whole CTA, before any set-up
   const int itA = 2 * mp, itB = 2 * mp + 1;
   const bool hasB = itB < ntiles;
-  const int nkvA = itA + 1, nkvB = hasB ? itB + 1 : 0;
+  // key tiles up to the one holding the tile's last row, within the keys that exist
+  const int nk_end = (q0 + nq + kBN - 1) / kBN;
+  const int nkvA = min((q0 + itA * kBM + kBM - 1) / kBN + 1, nk_end);
+  const int nkvB = hasB ? min((q0 + itB * kBM + kBM - 1) / kBN + 1, nk_end) : 0;
   const int nkv = hasB ? nkvB : nkvA;
-  const int bh = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
@@ -131,8 +146,8 @@ k_attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CU
       int ik = 0, iv = 0;            // K / V tiles issued
       mbar_expect_tx(&bars->q_full, (hasB ? 2 : 1) * Lay::OPB);
       for (int c = 0; c < SUB; ++c) {
-        tma_load_3d(sm + Lay::Q + c * kSub, &tq, &bars->q_full, 64 * c, itA * kBM, bh);
-        if (hasB) tma_load_3d(sm + Lay::Q + Lay::OPB + c * kSub, &tq, &bars->q_full, 64 * c, itB * kBM, bh);
+        tma_load_3d(sm + Lay::Q + c * kSub, &tq, &bars->q_full, 64 * c, q0 + itA * kBM, bh);
+        if (hasB) tma_load_3d(sm + Lay::Q + Lay::OPB + c * kSub, &tq, &bars->q_full, 64 * c, q0 + itB * kBM, bh);
       }
       for (int j = 0; j < nkv; ++j) {
         const int st = j & 1;
@@ -246,8 +261,8 @@ k_attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CU
       const int r = quarter * 32 + lane;
       const uint32_t la = (uint32_t)(quarter * 32) << 16;
       const uint32_t cS = tbase + la + 256 * t, cO = cS + 128;
-      const int q_row = it * kBM + r;
-      const int nk = it + 1;
+      const int q_row = it * kBM + r;                  // within this head's query rows
+      const int nk = t ? nkvB : nkvA;
       float m_run = 0.f, l_run = 0.f;
       bool ok = true;
       for (int j = 0; j < nk; ++j) {
@@ -261,10 +276,12 @@ k_attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CU
         reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&s[32]));
         reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&s[64]));
         reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&s[96]));
-        // causal mask on the diagonal tile; the running max is taken on the raw
-        // scores (c2 > 0, and rounding is monotone, so max(s) c2 = max(s c2))
-        if (j == it) {
-          const int lim = min(r, S - 1 - j * kBN);   // last valid column of this row
+        // causal mask where the key tile reaches past this row's position; the
+        // running max is taken on the raw scores (c2 > 0, and rounding is
+        // monotone, so max(s) c2 = max(s c2)). Key tile 0 always keeps column 0,
+        // so a row's running max is finite from its first tile on.
+        const int lim = q0 + q_row - j * kBN;            // last valid column of this row
+        if (__any_sync(0xffffffffu, lim < kBN - 1)) {
 #pragma unroll
           for (int c = 0; c < 128; ++c)
             if (c > lim) s[c] = __float_as_uint(-INFINITY);
@@ -313,7 +330,8 @@ k_attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CU
               const int e = 4 * g + u;
               const float2 x = __ffma2_rn(
                   make_float2(__uint_as_float(s[32 * c + 2 * e]), __uint_as_float(s[32 * c + 2 * e + 1])), cc, nm);
-              const float2 pp = make_float2(ex2(x.x), ex2(x.y));
+              // kFwdFmaPairs of every 8 column pairs on the FMA pipe, the rest on ex2
+              const float2 pp = (e & 7) < kFwdFmaPairs ? exp2_fma2(x) : make_float2(ex2(x.x), ex2(x.y));
               acc[u & 1] = __fadd2_rn(acc[u & 1], pp);
               const __half2 h = __float22half2_rn(pp);
               const __half2 l = __float22half2_rn(__ffma2_rn(__half22float2(h), m1, pp));   // p - hi, exact
@@ -336,13 +354,13 @@ k_attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CU
       if (ok && __all_sync(0xffffffffu, mbar_wait(&bars->o_done[t], (nk - 1) & 1, ab, err, 8))) {
         tc_fence_after();
         const float inv = 1.f / l_run;
-        float* dst = os + ((size_t)bh * S + q_row) * D;
+        float* dst = os + ((size_t)bh * S + q0 + q_row) * D;
 #pragma unroll 1
         for (int c = 0; c < D / 32; ++c) {
           uint32_t o[32];
           tmem_ld32(cO + 32 * c, o);
           tmem_wait_ld_regs(o);
-          if (q_row < S) {
+          if (q_row < nq) {
 #pragma unroll
             for (int e = 0; e < 32; e += 4)
               *reinterpret_cast<float4*>(dst + 32 * c + e) =
@@ -350,7 +368,7 @@ k_attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CU
                               __uint_as_float(o[e + 2]) * inv, __uint_as_float(o[e + 3]) * inv);
           }
         }
-        if (q_row < S) lse[(size_t)bh * S + q_row] = (m_run + log2f(l_run)) * kLn2f;
+        if (q_row < nq) lse[(size_t)bh * S + q0 + q_row] = (m_run + log2f(l_run)) * kLn2f;
       }
     }
   }
@@ -393,7 +411,7 @@ bool make_tmap_16(CUtensorMap* m, const void* base, int D, int S, int BH, bool f
 
 template <int D>
 static cudaError_t fwd_tc_t(const Geom& g, const void* qs, const void* ks, const void* vs, float* os,
-                            float* lse, int* err, cudaStream_t s) {
+                            float* lse, const int* seg, int* err, cudaStream_t s) {
   CUtensorMap tq, tk, tv;
   const int BH = g.B * g.H;
   if (!make_tmap_16(&tq, qs, D, g.S, BH, true, kBM) || !make_tmap_16(&tk, ks, D, g.S, BH, true, kBN) ||
@@ -405,15 +423,17 @@ static cudaError_t fwd_tc_t(const Geom& g, const void* qs, const void* ks, const
   const float c2 = (float)(1.4426950408889634 / sqrt((double)D));
   const int ntiles = (g.S + kBM - 1) / kBM;
   dim3 grid((ntiles + 1) / 2, BH);
-  k_attn_fwd_tc<D><<<grid, kFwdThreads, smem, s>>>(tq, tk, tv, os, lse, g.S, c2, err);
+  k_attn_fwd_tc<D><<<grid, kFwdThreads, smem, s>>>(tq, tk, tv, os, lse, g.S, c2, seg, err);
   count_launch();
   return cudaGetLastError();
 }
 
+// seg: nullptr (every row of the sub-sequence is a query) or [B*H][2] device
+// int32 (first query row, number of query rows) per (b, h).
 cudaError_t launch_attn_fwd_tc(const Geom& g, const void* qs, const void* ks, const void* vs,
-                               float* os, float* lse, int* err, cudaStream_t s) {
-  return g.D == 64 ? fwd_tc_t<64>(g, qs, ks, vs, os, lse, err, s)
-                   : fwd_tc_t<128>(g, qs, ks, vs, os, lse, err, s);
+                               float* os, float* lse, const int* seg, int* err, cudaStream_t s) {
+  return g.D == 64 ? fwd_tc_t<64>(g, qs, ks, vs, os, lse, seg, err, s)
+                   : fwd_tc_t<128>(g, qs, ks, vs, os, lse, seg, err, s);
 }
 
 }  // namespace lh

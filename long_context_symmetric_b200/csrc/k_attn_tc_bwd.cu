@@ -138,18 +138,18 @@ __device__ __forceinline__ void bwd_teardown(uint32_t tbase, int warp) {
   }
 }
 
-// Producer: the two fixed tiles once, then `n` streamed tiles of rows
-// (first + t) * 128 of maps ma (operand A_t) and mb (B_t).
+// Producer: the two fixed tiles once (rows frow .. frow + 127), then `n`
+// streamed tiles of rows row0 + t * 128 of maps ma (operand A_t) and mb (B_t).
 template <int D>
 __device__ void bwd_produce(uint8_t* sm, BwdBars* bars, const CUtensorMap* f0, const CUtensorMap* f1,
-                            int frow, const CUtensorMap* ma, const CUtensorMap* mb, int first, int n,
+                            int frow, const CUtensorMap* ma, const CUtensorMap* mb, int row0, int n,
                             int bh, volatile Abort* ab, int* err) {
   using Lay = BwdLayout<D>;
   constexpr int SUB = Lay::SUB, NSTA = Lay::NSTA, NSTB = Lay::NSTB;
   mbar_expect_tx(&bars->fix_full, 2 * Lay::OPB);
   for (int c = 0; c < SUB; ++c) {
-    tma_load_3d(sm + Lay::FIX0 + c * kSub, f0, &bars->fix_full, 64 * c, frow * kT, bh);
-    tma_load_3d(sm + Lay::FIX1 + c * kSub, f1, &bars->fix_full, 64 * c, frow * kT, bh);
+    tma_load_3d(sm + Lay::FIX0 + c * kSub, f0, &bars->fix_full, 64 * c, frow, bh);
+    tma_load_3d(sm + Lay::FIX1 + c * kSub, f1, &bars->fix_full, 64 * c, frow, bh);
   }
   int issued = 0;                        // (tile, operand) loads issued, in order
   for (int t = 0; t < n; ++t) {
@@ -164,7 +164,7 @@ __device__ void bwd_produce(uint8_t* sm, BwdBars* bars, const CUtensorMap* f0, c
       uint8_t* dst = sm + (o ? Lay::RB : Lay::RA) + st * Lay::OPB;
       mbar_expect_tx(full, Lay::OPB);
       for (int c = 0; c < SUB; ++c)
-        tma_load_3d(dst + c * kSub, o ? mb : ma, full, 64 * c, (first + t) * kT, bh);
+        tma_load_3d(dst + c * kSub, o ? mb : ma, full, 64 * c, row0 + t * kT, bh);
       issued = 2 * t + o + 1;
     }
     if (!go) break;
@@ -316,6 +316,13 @@ __device__ __forceinline__ float2 f2(uint32_t a, uint32_t b) {
 }
 __device__ __forceinline__ uint32_t h2_bits(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
 
+// Column pairs of every 8 whose exponentials run on the FMA pipe
+// (tc::exp2_fma2) rather than on the special-function unit, per kernel: the
+// dK/dV compute warps do less other work per pair than the dQ warps (no dS
+// split), so more of their exponentials move.
+constexpr int kDkdvFmaPairs = 3;
+constexpr int kDqFmaPairs = 2;
+
 // 32 columns of this thread's key row (dK/dV kernel): P^T = 2^(S^T c2 - lse2)
 // in place, two columns per packed fp32 instruction. nl2 holds -lse2 of the
 // 32 query columns (the same for every lane: broadcast reads). MASK: columns
@@ -330,7 +337,15 @@ __device__ __forceinline__ void p_chunk_t(uint32_t (&s)[32], const float* nl2, f
 #pragma unroll
     for (int u = 0; u < 4; u += 2) {
       const float2 x = __ffma2_rn(f2(s[e + u], s[e + u + 1]), cc, u ? make_float2(a.z, a.w) : make_float2(a.x, a.y));
-      float p0 = ex2(x.x), p1 = ex2(x.y);
+      float p0, p1;
+      if ((((e + u) >> 1) & 7) < kDkdvFmaPairs) {
+        const float2 pp = exp2_fma2(x);
+        p0 = pp.x;
+        p1 = pp.y;
+      } else {
+        p0 = ex2(x.x);
+        p1 = ex2(x.y);
+      }
       if (MASK) {
         const int col = col0 + e + u;
         if (col < vlo || col > vhi) p0 = 0.f;
@@ -372,7 +387,15 @@ __device__ __forceinline__ void p_chunk(uint32_t (&s)[32], float nl2, float c2, 
 #pragma unroll
   for (int e = 0; e < 32; e += 2) {
     const float2 x = __ffma2_rn(f2(s[e], s[e + 1]), cc, nl);
-    float p0 = ex2(x.x), p1 = ex2(x.y);
+    float p0, p1;
+    if (((e >> 1) & 7) < kDqFmaPairs) {
+      const float2 pp = exp2_fma2(x);
+      p0 = pp.x;
+      p1 = pp.y;
+    } else {
+      p0 = ex2(x.x);
+      p1 = ex2(x.y);
+    }
     if (MASK) {
       if (col0 + e > vhi) p0 = 0.f;
       if (col0 + e + 1 > vhi) p1 = 0.f;
@@ -402,22 +425,36 @@ __global__ void __launch_bounds__(kThreads, 1)
 k_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
               const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tdo,
               const float* __restrict__ lse, const float* __restrict__ delta, float* __restrict__ dks,
-              float* __restrict__ dvs, int S, float c2, float scale, int* err) {
+              float* __restrict__ dvs, int S, float c2, float scale, const int* __restrict__ seg, int* err) {
   using Lay = BwdLayout<D>;
   extern __shared__ __align__(16) uint8_t smem_raw[];
   BwdBars* bars = reinterpret_cast<BwdBars*>(smem_raw);
   uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + Lay::HEAD + 1023) & ~(uintptr_t)1023);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int ntiles = gridDim.x;
-  const int j = blockIdx.x;            // key tile; small j has the most query tiles
+  const int j = blockIdx.x;            // key tile (rows j*128 ..); small j has the most query tiles
   const int bh = blockIdx.y;
-  const int n = ntiles - j;            // query tiles i = j .. ntiles-1
+  // query rows [q0, q0 + nq) of this (b, h) (all S rows, or one rank's segment)
+  const int q0 = seg ? seg[2 * bh] : 0, nq = seg ? seg[2 * bh + 1] : S;
+  const int ntq = (nq + kT - 1) / kT;
+  const int i0 = max(0, j * kT - q0) / kT;   // first query tile with a row at or after key row j*128
+  const int n = ntq - i0;                    // query tiles i = i0 .. ntq-1
+  if (n <= 0) {
+    // no query of this head reaches this key tile: its gradient rows are zero
+    const size_t rows = (size_t)min(kT, S - j * kT);
+    float4* a = reinterpret_cast<float4*>(dks + ((size_t)bh * S + (size_t)j * kT) * D);
+    float4* b = reinterpret_cast<float4*>(dvs + ((size_t)bh * S + (size_t)j * kT) * D);
+    for (size_t x = threadIdx.x; x < rows * D / 4; x += blockDim.x) {
+      a[x] = make_float4(0.f, 0.f, 0.f, 0.f);
+      b[x] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    return;
+  }
   bwd_setup(bars, warp);
   const uint32_t tbase = bars->tmem_base;
   volatile Abort* ab = &bars->abort;
 
   if (warp == 0) {
-    if (lane == 0) bwd_produce<D>(sm, bars, &tk, &tv, j, &tq, &tdo, j, n, bh, ab, err);
+    if (lane == 0) bwd_produce<D>(sm, bars, &tk, &tv, j * kT, &tq, &tdo, q0 + i0 * kT, n, bh, ab, err);
   } else if (warp == 1) {
     bwd_mma<D, true>(sm, bars, tbase, n, ab, err);
   } else {
@@ -435,10 +472,10 @@ k_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CU
     const float* vsrc = (hid < 64 ? lse : delta) + (size_t)bh * S;
     const float vmul = hid < 64 ? -1.4426950408889634f : -1.f;
     auto fetch = [&](int i) -> float {
-      const int q = i * kT + 64 * half + (hid & 63);
-      return q < S ? vsrc[q] : 0.f;
+      const int q = i * kT + 64 * half + (hid & 63);    // within this head's query rows
+      return q < nq ? vsrc[q0 + q] : 0.f;
     };
-    float nxt = fetch(j);
+    float nxt = fetch(i0);
     bool ok = true;
     // this half's 64 query columns
     float* nl2 = vec + 64 * half;
@@ -446,7 +483,7 @@ k_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CU
     // every compute thread runs all n iterations (and their named barriers),
     // also after a wind-down, so no warp can be left waiting at a barrier
     for (int t = 0; t < n; ++t) {
-      const int i = j + t;
+      const int i = i0 + t;
       named_bar_sync(1 + half, kComputeThreads / 2);   // the half is done with tile t-1's vector
       (hid < 64 ? nl2 : ndl)[hid & 63] = nxt * vmul;
       named_bar_sync(1 + half, kComputeThreads / 2);
@@ -462,9 +499,9 @@ k_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CU
       reg_fence32(p1);
       tc_fence_before();
       mbar_arrive_warp(&bars->x_free);
-      const int vlo = i == j ? m : 0;                   // causal: query col >= key row
-      const int vhi = min(kT - 1, S - 1 - i * kT);      // last valid query column
-      if (vlo > 0 || vhi < kT - 1 || i == j) {
+      const int vlo = max(0, key - q0 - i * kT);         // causal: query position >= key position
+      const int vhi = min(kT - 1, nq - 1 - i * kT);      // last valid query column
+      if (vlo > 0 || vhi < kT - 1) {
         p_chunk_t<true>(p0, nl2, c2, 64 * half, vlo, vhi);
         p_chunk_t<true>(p1, nl2 + 32, c2, 64 * half + 32, vlo, vhi);
       } else {
@@ -536,22 +573,25 @@ __global__ void __launch_bounds__(kThreads, 1)
 k_bwd_dq_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tdo,
             const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
             const float* __restrict__ lse, const float* __restrict__ delta, float* __restrict__ dqs,
-            int S, float c2, float scale, int* err) {
+            int S, float c2, float scale, const int* __restrict__ seg, int* err) {
   using Lay = BwdLayout<D>;
   extern __shared__ __align__(16) uint8_t smem_raw[];
   BwdBars* bars = reinterpret_cast<BwdBars*>(smem_raw);
   uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + Lay::HEAD + 1023) & ~(uintptr_t)1023);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int ntiles = gridDim.x;
-  const int i = ntiles - 1 - (int)blockIdx.x;     // query tile; late tiles have the most key tiles
   const int bh = blockIdx.y;
-  const int n = i + 1;                            // key tiles j = 0 .. i
+  const int q0 = seg ? seg[2 * bh] : 0, nq = seg ? seg[2 * bh + 1] : S;
+  const int ntq = (nq + kT - 1) / kT;
+  const int i = ntq - 1 - (int)blockIdx.x;        // query tile; late tiles have the most key tiles
+  if (i < 0) return;                              // whole CTA, before any set-up
+  // key tiles up to the one holding the tile's last row, within the keys that exist
+  const int n = min((q0 + i * kT + kT - 1) / kT + 1, (q0 + nq + kT - 1) / kT);
   bwd_setup(bars, warp);
   const uint32_t tbase = bars->tmem_base;
   volatile Abort* ab = &bars->abort;
 
   if (warp == 0) {
-    if (lane == 0) bwd_produce<D>(sm, bars, &tq, &tdo, i, &tk, &tv, 0, n, bh, ab, err);
+    if (lane == 0) bwd_produce<D>(sm, bars, &tq, &tdo, q0 + i * kT, &tk, &tv, 0, n, bh, ab, err);
   } else if (warp == 1) {
     bwd_mma<D, false>(sm, bars, tbase, n, ab, err);
   } else {
@@ -560,9 +600,9 @@ k_bwd_dq_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
     const int r = quarter * 32 + lane;            // query row within the tile / TMEM lane
     const uint32_t la = (uint32_t)(quarter * 32) << 16;
     const uint32_t cX = tbase + la + 64 * half;
-    const int q = i * kT + r;
-    const float nl2 = q < S ? lse[(size_t)bh * S + q] * -1.4426950408889634f : 0.f;
-    const float ndl = q < S ? -delta[(size_t)bh * S + q] : 0.f;
+    const int q = i * kT + r;                      // within this head's query rows
+    const float nl2 = q < nq ? lse[(size_t)bh * S + q0 + q] * -1.4426950408889634f : 0.f;
+    const float ndl = q < nq ? -delta[(size_t)bh * S + q0 + q] : 0.f;
     bool ok = true;
     for (int jj = 0; jj < n; ++jj) {
       if (!__all_sync(0xffffffffu, mbar_wait(&bars->x_full, jj & 1, ab, err, 19))) { ok = false; break; }
@@ -574,7 +614,7 @@ k_bwd_dq_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
       reg_fence32(p1);
       tc_fence_before();
       mbar_arrive_warp(&bars->x_free);
-      const int klim = min(jj == i ? r : kT - 1, S - 1 - jj * kT);   // last valid key column
+      const int klim = min(q0 + q - jj * kT, kT - 1);   // last valid key column (causal)
       if (klim < kT - 1) {
         p_chunk<true>(p0, nl2, c2, 64 * half, klim);
         p_chunk<true>(p1, nl2, c2, 64 * half + 32, klim);
@@ -603,13 +643,13 @@ k_bwd_dq_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
     }
     if (ok && __all_sync(0xffffffffu, mbar_wait(&bars->done, 0, ab, err, 21))) {
       tc_fence_after();
-      float* dst = dqs + ((size_t)bh * S + q) * D;
+      float* dst = dqs + ((size_t)bh * S + q0 + q) * D;
 #pragma unroll 1
       for (int c = half * (D / 64); c < (half + 1) * (D / 64); ++c) {
         uint32_t a[32];
         tmem_ld32(tbase + la + col_acc(false) + 32 * c, a);
         tmem_wait_ld();
-        if (q < S) {
+        if (q < nq) {
           bool fin = true;
 #pragma unroll
           for (int e = 0; e < 32; ++e) fin &= fabsf(__uint_as_float(a[e])) < INFINITY;
@@ -628,8 +668,8 @@ k_bwd_dq_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
 
 template <int D>
 cudaError_t bwd_tc_t(const Geom& g, const void* qs, const void* ks, const void* vs, const void* dos,
-                     const float* lse, const float* delta, float* dqs, float* dks, float* dvs, int* err,
-                     cudaStream_t s) {
+                     const float* lse, const float* delta, float* dqs, float* dks, float* dvs, const int* seg,
+                     int* err, cudaStream_t s) {
   CUtensorMap tq, tk, tv, tdo;
   const int BH = g.B * g.H;
   if (!make_tmap_16(&tq, qs, D, g.S, BH, true, kT) || !make_tmap_16(&tk, ks, D, g.S, BH, true, kT) ||
@@ -643,22 +683,26 @@ cudaError_t bwd_tc_t(const Geom& g, const void* qs, const void* ks, const void* 
   const float scale = (float)(1.0 / sqrt((double)D));
   const float c2 = (float)(1.4426950408889634 / sqrt((double)D));
   dim3 grid((g.S + kT - 1) / kT, BH);
-  k_bwd_dkdv_tc<D><<<grid, kThreads, smem, s>>>(tk, tv, tq, tdo, lse, delta, dks, dvs, g.S, c2, scale, err);
+  k_bwd_dkdv_tc<D><<<grid, kThreads, smem, s>>>(tk, tv, tq, tdo, lse, delta, dks, dvs, g.S, c2, scale, seg, err);
   count_launch();
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  k_bwd_dq_tc<D><<<grid, kThreads, smem_q, s>>>(tq, tdo, tk, tv, lse, delta, dqs, g.S, c2, scale, err);
+  k_bwd_dq_tc<D><<<grid, kThreads, smem_q, s>>>(tq, tdo, tk, tv, lse, delta, dqs, g.S, c2, scale, seg, err);
   count_launch();
   return cudaGetLastError();
 }
 
 }  // namespace
 
+// seg: nullptr (every row of the sub-sequence is a query) or [B*H][2] device
+// int32 (first query row, number of query rows) per (b, h); then dks / dvs
+// hold every key row's gradient from those queries alone (zero rows where no
+// query reaches), and dqs only the segment's rows.
 cudaError_t launch_attn_bwd_tc(const Geom& g, const void* qs, const void* ks, const void* vs,
                                const void* dos, const float* lse, const float* delta, float* dqs,
-                               float* dks, float* dvs, int* err, cudaStream_t s) {
-  return g.D == 64 ? bwd_tc_t<64>(g, qs, ks, vs, dos, lse, delta, dqs, dks, dvs, err, s)
-                   : bwd_tc_t<128>(g, qs, ks, vs, dos, lse, delta, dqs, dks, dvs, err, s);
+                               float* dks, float* dvs, const int* seg, int* err, cudaStream_t s) {
+  return g.D == 64 ? bwd_tc_t<64>(g, qs, ks, vs, dos, lse, delta, dqs, dks, dvs, seg, err, s)
+                   : bwd_tc_t<128>(g, qs, ks, vs, dos, lse, delta, dqs, dks, dvs, seg, err, s);
 }
 
 }  // namespace lh

@@ -44,6 +44,7 @@ struct PoolArgs {
   int ts;          // tokens per shared-memory stage
   int ns;          // stages in the ring
   int row_bytes;   // bytes of one token row of the head group
+  int cb0;         // first coarsest block (a token range pools blocks cb0 .. cb0 + gridDim.x - 1)
 };
 
 __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
@@ -76,7 +77,7 @@ __global__ void __launch_bounds__(256, 2) k_pool(const T* __restrict__ q, const 
   const int hg0 = blockIdx.y * a.hg;
   const int head = hg0 + threadIdx.x / C8;
   const int chunk = threadIdx.x % C8;
-  const int cb = blockIdx.x;
+  const int cb = a.cb0 + (int)blockIdx.x;
   const T* x = tensor == 0 ? q : (tensor == 1 ? k : v);
   T* pyr = tensor == 0 ? pq : (tensor == 1 ? pk : pv);
   const int p = PP ? PP : g.p;
@@ -236,11 +237,12 @@ __global__ void __launch_bounds__(256, 2) k_pool(const T* __restrict__ q, const 
 
 template <typename T>
 cudaError_t launch_t(const Geom& g, const void* q, const void* k, const void* v, void* pq,
-                     void* pk, void* pv, double* sq, int* err, cudaStream_t s) {
+                     void* pk, void* pv, double* sq, int cb0, int ncb, int* err, cudaStream_t s) {
   const int LV = g.L - 1;
-  if (LV < 1) return cudaSuccess;
+  if (LV < 1 || ncb <= 0) return cudaSuccess;
   PoolArgs a;
   a.g = g;
+  a.cb0 = cb0;
   const int C8 = g.D / 8;
   int hg = g.H;
   while (hg * C8 > 256) {   // largest divisor of H that fits 256 threads
@@ -259,7 +261,7 @@ cudaError_t launch_t(const Geom& g, const void* q, const void* k, const void* v,
   // compile-time p when it divides the stage
   const int pp = (a.ts % g.p == 0 && (g.p == 2 || g.p == 4 || g.p == 8)) ? g.p : 0;
   dim3 block(hg * C8);
-  dim3 grid(g.n[g.L - 1], g.H / hg, 3 * g.B);
+  dim3 grid(ncb, g.H / hg, 3 * g.B);
   const T* tq = (const T*)q; const T* tk = (const T*)k; const T* tv = (const T*)v;
   T* tpq = (T*)pq; T* tpk = (T*)pk; T* tpv = (T*)pv;
   switch (LV) {
@@ -289,8 +291,15 @@ cudaError_t launch_t(const Geom& g, const void* q, const void* k, const void* v,
 
 cudaError_t launch_pool(const Geom& g, lh_dtype dt, const void* q, const void* k, const void* v,
                         void* pq, void* pk, void* pv, double* sq, int* err, cudaStream_t s) {
-  if (dt == LH_BF16) return launch_t<__nv_bfloat16>(g, q, k, v, pq, pk, pv, sq, err, s);
-  return launch_t<float>(g, q, k, v, pq, pk, pv, sq, err, s);
+  return launch_pool_range(g, dt, 0, g.L > 1 ? g.n[g.L - 1] : 0, q, k, v, pq, pk, pv, sq, err, s);
+}
+
+// Coarsest blocks [cb0, cb0 + ncb) of every sequence: the tokens
+// [cb0 p^(L-1), (cb0 + ncb) p^(L-1)) and the pyramid entries above them.
+cudaError_t launch_pool_range(const Geom& g, lh_dtype dt, int cb0, int ncb, const void* q, const void* k,
+                              const void* v, void* pq, void* pk, void* pv, double* sq, int* err, cudaStream_t s) {
+  if (dt == LH_BF16) return launch_t<__nv_bfloat16>(g, q, k, v, pq, pk, pv, sq, cb0, ncb, err, s);
+  return launch_t<float>(g, q, k, v, pq, pk, pv, sq, cb0, ncb, err, s);
 }
 
 }  // namespace lh

@@ -240,14 +240,14 @@ __global__ void __launch_bounds__(256) k_scatter_tree(const float* __restrict__ 
                                                       const int32_t* __restrict__ slot,
                                                       T* __restrict__ d0, T* __restrict__ d1,
                                                       T* __restrict__ d2, Geom g, int hg, int yb,
-                                                      int ntens) {
+                                                      int ntens, int cb0, int cb_end) {
   const int C8 = g.D >> 3;
   const int tensor = blockIdx.z % ntens;
   const int b = blockIdx.z / ntens;
   const int head = blockIdx.y * hg + threadIdx.x / C8;
   const int chunk = threadIdx.x % C8;
-  const int cb = blockIdx.x * yb + threadIdx.y;
-  if (cb >= g.n[LV]) return;           // no collectives below: a thread may leave
+  const int cb = cb0 + (int)blockIdx.x * yb + (int)threadIdx.y;
+  if (cb >= cb_end) return;            // no collectives below: a thread may leave
   const float* src = tensor == 0 ? s0 : (tensor == 1 ? s1 : s2);
   T* dst = tensor == 0 ? d0 : (tensor == 1 ? d1 : d2);
   const long long bh = (long long)b * g.H + head;
@@ -326,23 +326,27 @@ __global__ void __launch_bounds__(256) k_scatter_tree(const float* __restrict__ 
   }
 }
 
+// Coarsest blocks [cb0, cb0 + ncb) (ncb < 0: all of them).
 template <typename T, int FIXED, bool WEIGHTED>
 cudaError_t tree_t(const Geom& g, const float* s0, const float* s1, const float* s2,
-                   const int32_t* slot, T* d0, T* d1, T* d2, int ntens, cudaStream_t s) {
+                   const int32_t* slot, T* d0, T* d1, T* d2, int ntens, cudaStream_t s, int cb0 = 0,
+                   int ncb = -1) {
   const int C8 = g.D / 8;
   int hg = g.H;
   while (hg * C8 > 256) {
     --hg;
     while (g.H % hg) --hg;
   }
-  const int ncoarse = g.n[g.L - 1];
+  const int ncoarse = ncb < 0 ? g.n[g.L - 1] : ncb;
+  if (ncoarse <= 0) return cudaSuccess;
   int yb = 1;
   while (yb * 2 * hg * C8 <= 256 && yb * 2 <= ncoarse) yb *= 2;
   dim3 block(hg * C8, yb);
   dim3 grid((ncoarse + yb - 1) / yb, g.H / hg, g.B * ntens);
+  const int cb_end = cb0 + ncoarse;
   switch (g.L - 1) {
 #define LH_TREE_CASE(n) \
-    case n: k_scatter_tree<T, FIXED, WEIGHTED, n><<<grid, block, 0, s>>>(s0, s1, s2, slot, d0, d1, d2, g, hg, yb, ntens); break;
+    case n: k_scatter_tree<T, FIXED, WEIGHTED, n><<<grid, block, 0, s>>>(s0, s1, s2, slot, d0, d1, d2, g, hg, yb, ntens, cb0, cb_end); break;
     LH_TREE_CASE(1) LH_TREE_CASE(2) LH_TREE_CASE(3) LH_TREE_CASE(4)
     LH_TREE_CASE(5) LH_TREE_CASE(6) LH_TREE_CASE(7)
 #undef LH_TREE_CASE
@@ -680,16 +684,17 @@ int grid_for(long long total) {
 }
 
 template <typename T>
-cudaError_t scatter_t(const Geom& g, const float* os, const int32_t* slot, void* o, cudaStream_t s) {
+cudaError_t scatter_t(const Geom& g, const float* os, const int32_t* slot, void* o, cudaStream_t s,
+                      int cb0 = 0, int ncb = -1) {
   if (g.L > 1) {
     // weights 1 (the default reading) or 1/p^l (LH_WEIGHT_MEAN)
     if (g.weight == LH_WEIGHT_MEAN)
       return g.accum == LH_ACC_FIXED64
-                 ? tree_t<T, 1, true>(g, os, os, os, slot, (T*)o, (T*)o, (T*)o, 1, s)
-                 : tree_t<T, 0, true>(g, os, os, os, slot, (T*)o, (T*)o, (T*)o, 1, s);
+                 ? tree_t<T, 1, true>(g, os, os, os, slot, (T*)o, (T*)o, (T*)o, 1, s, cb0, ncb)
+                 : tree_t<T, 0, true>(g, os, os, os, slot, (T*)o, (T*)o, (T*)o, 1, s, cb0, ncb);
     return g.accum == LH_ACC_FIXED64
-               ? tree_t<T, 1, false>(g, os, os, os, slot, (T*)o, (T*)o, (T*)o, 1, s)
-               : tree_t<T, 0, false>(g, os, os, os, slot, (T*)o, (T*)o, (T*)o, 1, s);
+               ? tree_t<T, 1, false>(g, os, os, os, slot, (T*)o, (T*)o, (T*)o, 1, s, cb0, ncb)
+               : tree_t<T, 0, false>(g, os, os, os, slot, (T*)o, (T*)o, (T*)o, 1, s, cb0, ncb);
   }
   const long long total = (long long)g.B * g.N * g.H * (g.D / 8);
   if (g.accum == LH_ACC_FIXED64)
@@ -794,6 +799,14 @@ cudaError_t launch_scatter(const Geom& g, lh_dtype dt, const float* os, const in
                            void* o, cudaStream_t s) {
   return dt == LH_BF16 ? scatter_t<__nv_bfloat16>(g, os, slot, o, s)
                        : scatter_t<float>(g, os, slot, o, s);
+}
+
+// Tokens of the coarsest blocks [cb0, cb0 + ncb) only (L >= 2).
+cudaError_t launch_scatter_range(const Geom& g, lh_dtype dt, int cb0, int ncb, const float* os,
+                                 const int32_t* slot, void* o, cudaStream_t s) {
+  if (g.L < 2) return cudaErrorInvalidValue;
+  return dt == LH_BF16 ? scatter_t<__nv_bfloat16>(g, os, slot, o, s, cb0, ncb)
+                       : scatter_t<float>(g, os, slot, o, s, cb0, ncb);
 }
 
 cudaError_t launch_spread(const Geom& g, lh_dtype dt, const float* dqs, const float* dks,

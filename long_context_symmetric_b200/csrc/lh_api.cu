@@ -26,7 +26,7 @@ cudaError_t launch_attn_bwd_simt(const Geom& g, lh_dtype dt, const void* qs, con
                                  cudaStream_t s);
 
 cudaError_t launch_attn_fwd_tc(const Geom& g, const void* qs, const void* ks, const void* vs,
-                               float* os, float* lse, int* err, cudaStream_t s);
+                               float* os, float* lse, const int* seg, int* err, cudaStream_t s);
 
 // bf16 I/O runs on the tcgen05 tensor-core kernels (fp16 operands); fp32 on
 // the fp32 SIMT kernels. LH_ATTN_SIMT=1 in the environment routes bf16 I/O
@@ -38,20 +38,21 @@ static bool force_simt() {
 
 cudaError_t launch_attn_fwd(const Geom& g, lh_dtype dt, const void* qs, const void* ks,
                             const void* vs, float* os, float* lse, int* err, cudaStream_t s) {
-  if (dt == LH_BF16 && !force_simt()) return launch_attn_fwd_tc(g, qs, ks, vs, os, lse, err, s);
+  if (dt == LH_BF16 && !force_simt()) return launch_attn_fwd_tc(g, qs, ks, vs, os, lse, nullptr, err, s);
   return launch_attn_fwd_simt(g, dt, qs, ks, vs, os, lse, s);
 }
 
 cudaError_t launch_attn_bwd_tc(const Geom& g, const void* qs, const void* ks, const void* vs,
                                const void* dos, const float* lse, const float* delta, float* dqs,
-                               float* dks, float* dvs, int* err, cudaStream_t s);
+                               float* dks, float* dvs, const int* seg, int* err, cudaStream_t s);
 cudaError_t launch_selftest_wait(long long limit_cycles, int* err, int* gave_up, cudaStream_t s);
+cudaError_t launch_selftest_exp2(const float* x, float* y_fma, float* y_sfu, int n, cudaStream_t s);
 
 cudaError_t launch_attn_bwd(const Geom& g, lh_dtype dt, const void* qs, const void* ks,
                             const void* vs, const void* dos, const float* lse, const float* delta,
                             float* dqs, float* dks, float* dvs, int* err, cudaStream_t s) {
   if (dt == LH_BF16 && !force_simt())
-    return launch_attn_bwd_tc(g, qs, ks, vs, dos, lse, delta, dqs, dks, dvs, err, s);
+    return launch_attn_bwd_tc(g, qs, ks, vs, dos, lse, delta, dqs, dks, dvs, nullptr, err, s);
   return launch_attn_bwd_simt(g, dt, qs, ks, vs, dos, lse, delta, dqs, dks, dvs, s);
 }
 
@@ -142,6 +143,31 @@ lh_status make_geom(const lh_config* cfg, Geom* g, lh_plan_t* out) {
     }
     out->ws_bytes = L > 1 ? (size_t)B * H * 5 * (size_t)G.C * sizeof(int32_t) : 0;
   }
+  return LH_OK;
+}
+
+}  // namespace
+
+// sequence-sharded path (k_cp.cu)
+cudaError_t launch_cp_assemble_sq(const Geom& g, int world, int rank, const double* gath, double* sq,
+                                  cudaStream_t s);
+cudaError_t launch_cp_segment(const Geom& g, int world, int rank, const int32_t* map, const int32_t* slot,
+                              int32_t* slot_loc, int32_t* seg, cudaStream_t s);
+cudaError_t launch_cp_gather(const Geom& g, lh_dtype dt, int world, int rank, const void* q, const void* k,
+                             const void* v, const void* pq, const void* pk, const void* pv, const int32_t* map,
+                             const int32_t* seg, void* qs, void* ks, void* vs, int* err, cudaStream_t s);
+cudaError_t launch_cp_zero_outside(const Geom& g, int elem_bytes, void* x, const int32_t* seg, cudaStream_t s);
+Geom shard_geom(const Geom& g, int world, int rank);
+
+namespace {
+
+// Whole-sequence geometry plus the checks of the sequence-sharded path: L >= 2,
+// 0 <= rank < world, N split evenly into shards of whole coarsest blocks.
+lh_status make_cp_geom_checked(const lh_config* cfg, int world, int rank, Geom* g, lh_plan_t* pl) {
+  lh_status st = make_geom(cfg, g, pl);
+  if (st != LH_OK) return st;
+  if (world < 1 || rank < 0 || rank >= world || g->L < 2) return LH_ERR_SHAPE;
+  if (g->N % world != 0 || (g->N / world) % g->pl[g->L - 1] != 0) return LH_ERR_SHAPE;
   return LH_OK;
 }
 
@@ -320,6 +346,164 @@ lh_status lh_backward(const lh_config* cfg, const void* dout, void* dq, void* dk
   return lh_spread(cfg, b->dqs, b->dks, b->dvs, b->slot, dq, dk, dv, stream);
 }
 
+// ---------------------------------------------------------------- token ranges (fusion with projections)
+
+namespace {
+lh_status check_range(const Geom& g, int t0, int nt) {
+  if (g.L < 2) return LH_ERR_SHAPE;
+  const long long P = g.pl[g.L - 1];
+  if (t0 < 0 || nt < 0 || (long long)t0 + nt > g.N || t0 % P != 0 || nt % P != 0) return LH_ERR_SHAPE;
+  return LH_OK;
+}
+}  // namespace
+
+lh_status lh_pool_range(const lh_config* cfg, int t0, int nt, const void* q, const void* k, const void* v,
+                        void* pyr_q, void* pyr_k, void* pyr_v, double* sq, void* stream) {
+  Geom g;
+  lh_status st = make_geom(cfg, &g, nullptr);
+  if (st != LH_OK) return st;
+  if ((st = check_range(g, t0, nt)) != LH_OK) return st;
+  LH_REQ(q); LH_REQ(k); LH_REQ(v); LH_REQ(pyr_q); LH_REQ(pyr_k); LH_REQ(pyr_v); LH_REQ(sq);
+  const int P = (int)g.pl[g.L - 1];
+  LH_CUDA(launch_pool_range(g, cfg->dtype, t0 / P, nt / P, q, k, v, pyr_q, pyr_k, pyr_v, sq, device_error_ptr(),
+                            (cudaStream_t)stream));
+  return LH_OK;
+}
+
+lh_status lh_scatter_range(const lh_config* cfg, int t0, int nt, const float* os, const int32_t* slot, void* o,
+                           void* stream) {
+  Geom g;
+  lh_status st = make_geom(cfg, &g, nullptr);
+  if (st != LH_OK) return st;
+  if ((st = check_range(g, t0, nt)) != LH_OK) return st;
+  LH_REQ(os); LH_REQ(slot); LH_REQ(o);
+  const int P = (int)g.pl[g.L - 1];
+  LH_CUDA(launch_scatter_range(g, cfg->dtype, t0 / P, nt / P, os, slot, o, (cudaStream_t)stream));
+  return LH_OK;
+}
+
+// ---------------------------------------------------------------- sequence-sharded path
+
+lh_status lh_cp_plan(const lh_config* cfg, int world, int rank, lh_cp_plan_t* out) {
+  if (!out) return LH_ERR_NULL;
+  Geom g;
+  lh_plan_t pl;
+  lh_status st = make_cp_geom_checked(cfg, world, rank, &g, &pl);
+  if (st != LH_OK) return st;
+  const Geom s = shard_geom(g, world, rank);
+  std::memset(out, 0, sizeof(*out));
+  out->world = world;
+  out->rank = rank;
+  out->n_loc = s.N;
+  out->E_loc = s.E;
+  for (int l = 0; l < LH_MAX_LEVELS; ++l) out->lvl_off_loc[l] = l < g.L ? s.off[l] : 0;
+  out->global = pl;
+  return LH_OK;
+}
+
+lh_status lh_cp_pool(const lh_config* cfg, int world, int rank, const void* q, const void* k, const void* v,
+                     void* pyr_q, void* pyr_k, void* pyr_v, double* sq_loc, void* stream) {
+  Geom g;
+  lh_status st = make_cp_geom_checked(cfg, world, rank, &g, nullptr);
+  if (st != LH_OK) return st;
+  LH_REQ(q); LH_REQ(k); LH_REQ(v); LH_REQ(pyr_q); LH_REQ(pyr_k); LH_REQ(pyr_v); LH_REQ(sq_loc);
+  LH_CUDA(launch_pool(shard_geom(g, world, rank), cfg->dtype, q, k, v, pyr_q, pyr_k, pyr_v, sq_loc,
+                      device_error_ptr(), (cudaStream_t)stream));
+  return LH_OK;
+}
+
+lh_status lh_cp_assemble_sq(const lh_config* cfg, int world, const double* sq_gathered, double* sq,
+                            void* stream) {
+  Geom g;
+  lh_status st = make_cp_geom_checked(cfg, world, 0, &g, nullptr);
+  if (st != LH_OK) return st;
+  LH_REQ(sq_gathered); LH_REQ(sq);
+  LH_CUDA(launch_cp_assemble_sq(g, world, 0, sq_gathered, sq, (cudaStream_t)stream));
+  return LH_OK;
+}
+
+lh_status lh_cp_segment(const lh_config* cfg, int world, int rank, const int32_t* map, const int32_t* slot,
+                        int32_t* slot_loc, int32_t* seg, void* stream) {
+  Geom g;
+  lh_status st = make_cp_geom_checked(cfg, world, rank, &g, nullptr);
+  if (st != LH_OK) return st;
+  LH_REQ(map); LH_REQ(slot); LH_REQ(slot_loc); LH_REQ(seg);
+  LH_CUDA(launch_cp_segment(g, world, rank, map, slot, slot_loc, seg, (cudaStream_t)stream));
+  return LH_OK;
+}
+
+lh_status lh_cp_gather(const lh_config* cfg, int world, int rank, const void* q, const void* k, const void* v,
+                       const void* pyr_q, const void* pyr_k, const void* pyr_v, const int32_t* map,
+                       const int32_t* seg, void* qs, void* ks, void* vs, void* stream) {
+  Geom g;
+  lh_status st = make_cp_geom_checked(cfg, world, rank, &g, nullptr);
+  if (st != LH_OK) return st;
+  LH_REQ(q); LH_REQ(k); LH_REQ(v); LH_REQ(pyr_q); LH_REQ(pyr_k); LH_REQ(pyr_v); LH_REQ(map); LH_REQ(seg);
+  LH_REQ(qs); LH_REQ(ks); LH_REQ(vs);
+  LH_CUDA(launch_cp_gather(g, cfg->dtype, world, rank, q, k, v, pyr_q, pyr_k, pyr_v, map, seg, qs, ks, vs,
+                           device_error_ptr(), (cudaStream_t)stream));
+  return LH_OK;
+}
+
+lh_status lh_cp_attn_fwd(const lh_config* cfg, int world, int rank, const int32_t* seg, const void* qs,
+                         const void* ks, const void* vs, float* os, float* lse, void* stream) {
+  Geom g;
+  lh_status st = make_cp_geom_checked(cfg, world, rank, &g, nullptr);
+  if (st != LH_OK) return st;
+  if (cfg->dtype != LH_BF16) return LH_ERR_DTYPE;
+  LH_REQ(seg); LH_REQ(qs); LH_REQ(ks); LH_REQ(vs); LH_REQ(os); LH_REQ(lse);
+  LH_CUDA(launch_attn_fwd_tc(g, qs, ks, vs, os, lse, seg, device_error_ptr(), (cudaStream_t)stream));
+  return LH_OK;
+}
+
+lh_status lh_cp_scatter(const lh_config* cfg, int world, int rank, const float* os, const int32_t* slot_loc,
+                        void* o, void* stream) {
+  Geom g;
+  lh_status st = make_cp_geom_checked(cfg, world, rank, &g, nullptr);
+  if (st != LH_OK) return st;
+  LH_REQ(os); LH_REQ(slot_loc); LH_REQ(o);
+  LH_CUDA(launch_scatter(shard_geom(g, world, rank), cfg->dtype, os, slot_loc, o, (cudaStream_t)stream));
+  return LH_OK;
+}
+
+lh_status lh_cp_scatter_bwd(const lh_config* cfg, int world, int rank, const void* dout, const float* os,
+                            const int32_t* slot_loc, const int32_t* seg, void* dos, float* delta, void* stream) {
+  Geom g;
+  lh_status st = make_cp_geom_checked(cfg, world, rank, &g, nullptr);
+  if (st != LH_OK) return st;
+  if (cfg->dtype != LH_BF16) return LH_ERR_DTYPE;
+  LH_REQ(dout); LH_REQ(os); LH_REQ(slot_loc); LH_REQ(seg); LH_REQ(dos); LH_REQ(delta);
+  LH_CUDA(launch_cp_zero_outside(g, 2, dos, seg, (cudaStream_t)stream));
+  LH_CUDA(launch_scatter_bwd(shard_geom(g, world, rank), cfg->dtype, dout, os, slot_loc, dos, delta,
+                             device_error_ptr(), (cudaStream_t)stream));
+  return LH_OK;
+}
+
+lh_status lh_cp_attn_bwd(const lh_config* cfg, int world, int rank, const int32_t* seg, const void* qs,
+                         const void* ks, const void* vs, const void* dos, const float* lse, const float* delta,
+                         float* dqs, float* dks, float* dvs, void* stream) {
+  Geom g;
+  lh_status st = make_cp_geom_checked(cfg, world, rank, &g, nullptr);
+  if (st != LH_OK) return st;
+  if (cfg->dtype != LH_BF16) return LH_ERR_DTYPE;
+  LH_REQ(seg); LH_REQ(qs); LH_REQ(ks); LH_REQ(vs); LH_REQ(dos); LH_REQ(lse); LH_REQ(delta);
+  LH_REQ(dqs); LH_REQ(dks); LH_REQ(dvs);
+  LH_CUDA(launch_attn_bwd_tc(g, qs, ks, vs, dos, lse, delta, dqs, dks, dvs, seg, device_error_ptr(),
+                             (cudaStream_t)stream));
+  return LH_OK;
+}
+
+lh_status lh_cp_spread(const lh_config* cfg, int world, int rank, const float* dqs, const float* dks,
+                       const float* dvs, const int32_t* slot_loc, void* dq, void* dk, void* dv, void* stream) {
+  Geom g;
+  lh_status st = make_cp_geom_checked(cfg, world, rank, &g, nullptr);
+  if (st != LH_OK) return st;
+  LH_REQ(dqs); LH_REQ(dks); LH_REQ(dvs); LH_REQ(slot_loc); LH_REQ(dq); LH_REQ(dk); LH_REQ(dv);
+  LH_CUDA(launch_spread(shard_geom(g, world, rank), cfg->dtype, dqs, dks, dvs, slot_loc, dq, dk, dv,
+                        (cudaStream_t)stream));
+  return LH_OK;
+}
+
 lh_status lh_selftest_timeout(long long limit_cycles, int* gave_up, void* stream) {
   if (!gave_up) return LH_ERR_NULL;
   if (limit_cycles < 1 || limit_cycles > 2000000000LL) return LH_ERR_SHAPE;
@@ -327,6 +511,13 @@ lh_status lh_selftest_timeout(long long limit_cycles, int* gave_up, void* stream
   if (!err) return LH_ERR_CUDA;
   return lh::launch_selftest_wait(limit_cycles, err, gave_up, (cudaStream_t)stream) == cudaSuccess ? LH_OK
                                                                                                   : LH_ERR_CUDA;
+}
+
+lh_status lh_selftest_exp2(const float* x, float* y_fma, float* y_sfu, int n, void* stream) {
+  if (n < 0) return LH_ERR_SHAPE;
+  if (n == 0) return LH_OK;
+  if (!x || !y_fma || !y_sfu) return LH_ERR_NULL;
+  return lh::launch_selftest_exp2(x, y_fma, y_sfu, n, (cudaStream_t)stream) == cudaSuccess ? LH_OK : LH_ERR_CUDA;
 }
 
 lh_status lh_get_device_error(void* stream, int* detail) {

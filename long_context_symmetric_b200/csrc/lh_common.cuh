@@ -193,6 +193,10 @@ __device__ __forceinline__ int map_index(int e) { return e & 0x0FFFFFFF; }
 namespace lh {
 cudaError_t launch_pool(const Geom& g, lh_dtype dt, const void* q, const void* k, const void* v,
                         void* pq, void* pk, void* pv, double* sq, int* err, cudaStream_t s);
+cudaError_t launch_pool_range(const Geom& g, lh_dtype dt, int cb0, int ncb, const void* q, const void* k,
+                              const void* v, void* pq, void* pk, void* pv, double* sq, int* err, cudaStream_t s);
+cudaError_t launch_scatter_range(const Geom& g, lh_dtype dt, int cb0, int ncb, const float* os,
+                                 const int32_t* slot, void* o, cudaStream_t s);
 cudaError_t launch_select(const Geom& g, const double* sq, int32_t* sel, int32_t* map,
                           int32_t* slot, int32_t* ws, cudaStream_t s);
 cudaError_t launch_gather(const Geom& g, lh_dtype dt, const void* q, const void* k, const void* v,

@@ -272,6 +272,34 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+// 2^x of two values on the FMA and integer pipes, leaving the special-function
+// unit (ex2, 4 lanes per clock per SM sub-partition) to the other elements of a
+// softmax tile. Range reduction x = n + f, n = rint(x), f in [-1/2, 1/2]: adding
+// 1.5 * 2^23 rounds x to an integer in the low mantissa bits of t, so t - 1.5 *
+// 2^23 = n and x - n = f are exact. 2^f: degree-5 polynomial with minimax
+// relative error on [-1/2, 1/2] (Remez exchange; gen_exp2_poly.py beside this
+// file derives the coefficients), 2^-23.7 in exact arithmetic and 2^-22.2
+// evaluated here in fp32 Horner form. 2^n: n added to the exponent field (the
+// low 9 bits of t's bit pattern are n's, so t << 23 is n << 23). Inputs below
+// -125 are clamped to it (2^-125 where 2^x would be smaller or x is -inf), so
+// the result is always a normal fp32 value; inputs must stay below 127.
+__device__ __forceinline__ float2 exp2_fma2(float2 x) {
+  x.x = fmaxf(x.x, -125.f);
+  x.y = fmaxf(x.y, -125.f);
+  const float2 magic = make_float2(12582912.f, 12582912.f);
+  const float2 t = __fadd2_rn(x, magic);
+  const float2 n = __fadd2_rn(t, make_float2(-12582912.f, -12582912.f));
+  const float2 f = __fadd2_rn(x, make_float2(-n.x, -n.y));
+  float2 p = make_float2(0.0013276472454890609f, 0.0013276472454890609f);
+  p = __ffma2_rn(p, f, make_float2(0.009675540961325169f, 0.009675540961325169f));
+  p = __ffma2_rn(p, f, make_float2(0.05550713092088699f, 0.05550713092088699f));
+  p = __ffma2_rn(p, f, make_float2(0.24022120237350464f, 0.24022120237350464f));
+  p = __ffma2_rn(p, f, make_float2(0.6931469440460205f, 0.6931469440460205f));
+  p = __ffma2_rn(p, f, make_float2(1.0000001192092896f, 1.0000001192092896f));
+  return make_float2(__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(t.x) << 23)),
+                     __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(t.y) << 23)));
+}
+
 // three-input max (sm_100 PTX form), NaN-ignoring like fmaxf
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float d;

@@ -53,6 +53,11 @@ class Plan(ctypes.Structure):
                 ("c", c_int * MAX_LEVELS), ("lvl_off", c_int * MAX_LEVELS), ("ws_bytes", c_size_t)]
 
 
+class CPPlan(ctypes.Structure):
+    _fields_ = [("world", c_int), ("rank", c_int), ("n_loc", c_int), ("E_loc", c_int),
+                ("lvl_off_loc", c_int * MAX_LEVELS), ("glob", Plan)]
+
+
 class Buffers(ctypes.Structure):
     _fields_ = [("pyr_q", c_void_p), ("pyr_k", c_void_p), ("pyr_v", c_void_p), ("sq", c_void_p),
                 ("sel", c_void_p), ("map", c_void_p), ("slot", c_void_p), ("qs", c_void_p),
@@ -82,6 +87,19 @@ _SIGS = {
     "lh_launch_count": ([], ctypes.c_ulonglong),
     "lh_selftest_timeout": ([ctypes.c_longlong, c_void_p, c_void_p], c_int),
     "lh_score_topk_noalloc": ([ctypes.POINTER(Config)] + [c_void_p] * 5, c_int),
+    "lh_selftest_exp2": ([c_void_p, c_void_p, c_void_p, c_int, c_void_p], c_int),
+    "lh_pool_range": ([ctypes.POINTER(Config), c_int, c_int] + [c_void_p] * 8, c_int),
+    "lh_scatter_range": ([ctypes.POINTER(Config), c_int, c_int] + [c_void_p] * 4, c_int),
+    "lh_cp_plan": ([ctypes.POINTER(Config), c_int, c_int, ctypes.POINTER(CPPlan)], c_int),
+    "lh_cp_pool": ([ctypes.POINTER(Config), c_int, c_int] + [c_void_p] * 8, c_int),
+    "lh_cp_assemble_sq": ([ctypes.POINTER(Config), c_int] + [c_void_p] * 3, c_int),
+    "lh_cp_segment": ([ctypes.POINTER(Config), c_int, c_int] + [c_void_p] * 5, c_int),
+    "lh_cp_gather": ([ctypes.POINTER(Config), c_int, c_int] + [c_void_p] * 12, c_int),
+    "lh_cp_attn_fwd": ([ctypes.POINTER(Config), c_int, c_int] + [c_void_p] * 7, c_int),
+    "lh_cp_scatter": ([ctypes.POINTER(Config), c_int, c_int] + [c_void_p] * 4, c_int),
+    "lh_cp_scatter_bwd": ([ctypes.POINTER(Config), c_int, c_int] + [c_void_p] * 7, c_int),
+    "lh_cp_attn_bwd": ([ctypes.POINTER(Config), c_int, c_int] + [c_void_p] * 11, c_int),
+    "lh_cp_spread": ([ctypes.POINTER(Config), c_int, c_int] + [c_void_p] * 8, c_int),
 }
 
 
@@ -210,6 +228,78 @@ def selftest_timeout(limit_cycles: int, gave_up: torch.Tensor, stream=None):
     arrives on; after `limit_cycles` SM cycles it gives up and records
     LH_ERR_TIMEOUT (detail 900). `gave_up`: a device int32 tensor, set to 1."""
     _check(lib().lh_selftest_timeout(int(limit_cycles), _p(gave_up), _stream(stream)), "lh_selftest_timeout")
+
+
+def selftest_exp2(x: torch.Tensor, y_fma: torch.Tensor, y_sfu: torch.Tensor, stream=None):
+    """2^x of a device float32 tensor by the attention kernels' FMA-pipe
+    polynomial (y_fma) and by the special-function unit's ex2.approx (y_sfu)."""
+    _check(lib().lh_selftest_exp2(_p(x), _p(y_fma), _p(y_sfu), x.numel(), _stream(stream)), "lh_selftest_exp2")
+
+
+def pool_range(cfg, t0, nt, q, k, v, pyr_q, pyr_k, pyr_v, sq, stream=None):
+    _check(lib().lh_pool_range(ctypes.byref(cfg), t0, nt, _p(q), _p(k), _p(v), _p(pyr_q), _p(pyr_k), _p(pyr_v),
+                               _p(sq), _stream(stream)), "lh_pool_range")
+
+
+def scatter_range(cfg, t0, nt, os_, slot, o, stream=None):
+    _check(lib().lh_scatter_range(ctypes.byref(cfg), t0, nt, _p(os_), _p(slot), _p(o), _stream(stream)),
+           "lh_scatter_range")
+
+
+# ---------------------------------------------------------------------------
+# sequence-sharded (context-parallel) path: the per-rank calls
+# ---------------------------------------------------------------------------
+
+def cp_plan(cfg, world: int, rank: int) -> CPPlan:
+    out = CPPlan()
+    _check(lib().lh_cp_plan(ctypes.byref(cfg), world, rank, ctypes.byref(out)), "lh_cp_plan")
+    return out
+
+
+def cp_pool(cfg, world, rank, q, k, v, pyr_q, pyr_k, pyr_v, sq_loc, stream=None):
+    _check(lib().lh_cp_pool(ctypes.byref(cfg), world, rank, _p(q), _p(k), _p(v), _p(pyr_q), _p(pyr_k),
+                            _p(pyr_v), _p(sq_loc), _stream(stream)), "lh_cp_pool")
+
+
+def cp_assemble_sq(cfg, world, sq_gathered, sq, stream=None):
+    _check(lib().lh_cp_assemble_sq(ctypes.byref(cfg), world, _p(sq_gathered), _p(sq), _stream(stream)),
+           "lh_cp_assemble_sq")
+
+
+def cp_segment(cfg, world, rank, map_, slot, slot_loc, seg, stream=None):
+    _check(lib().lh_cp_segment(ctypes.byref(cfg), world, rank, _p(map_), _p(slot), _p(slot_loc), _p(seg),
+                               _stream(stream)), "lh_cp_segment")
+
+
+def cp_gather(cfg, world, rank, q, k, v, pyr_q, pyr_k, pyr_v, map_, seg, qs, ks, vs, stream=None):
+    _check(lib().lh_cp_gather(ctypes.byref(cfg), world, rank, _p(q), _p(k), _p(v), _p(pyr_q), _p(pyr_k),
+                              _p(pyr_v), _p(map_), _p(seg), _p(qs), _p(ks), _p(vs), _stream(stream)),
+           "lh_cp_gather")
+
+
+def cp_attn_fwd(cfg, world, rank, seg, qs, ks, vs, os_, lse, stream=None):
+    _check(lib().lh_cp_attn_fwd(ctypes.byref(cfg), world, rank, _p(seg), _p(qs), _p(ks), _p(vs), _p(os_),
+                                _p(lse), _stream(stream)), "lh_cp_attn_fwd")
+
+
+def cp_scatter(cfg, world, rank, os_, slot_loc, o, stream=None):
+    _check(lib().lh_cp_scatter(ctypes.byref(cfg), world, rank, _p(os_), _p(slot_loc), _p(o), _stream(stream)),
+           "lh_cp_scatter")
+
+
+def cp_scatter_bwd(cfg, world, rank, dout, os_, slot_loc, seg, dos, delta, stream=None):
+    _check(lib().lh_cp_scatter_bwd(ctypes.byref(cfg), world, rank, _p(dout), _p(os_), _p(slot_loc), _p(seg),
+                                   _p(dos), _p(delta), _stream(stream)), "lh_cp_scatter_bwd")
+
+
+def cp_attn_bwd(cfg, world, rank, seg, qs, ks, vs, dos, lse, delta, dqs, dks, dvs, stream=None):
+    _check(lib().lh_cp_attn_bwd(ctypes.byref(cfg), world, rank, _p(seg), _p(qs), _p(ks), _p(vs), _p(dos),
+                                _p(lse), _p(delta), _p(dqs), _p(dks), _p(dvs), _stream(stream)), "lh_cp_attn_bwd")
+
+
+def cp_spread(cfg, world, rank, dqs, dks, dvs, slot_loc, dq, dk, dv, stream=None):
+    _check(lib().lh_cp_spread(ctypes.byref(cfg), world, rank, _p(dqs), _p(dks), _p(dvs), _p(slot_loc), _p(dq),
+                              _p(dk), _p(dv), _stream(stream)), "lh_cp_spread")
 
 
 # ---------------------------------------------------------------------------

@@ -99,3 +99,25 @@ def test_single_level_needs_no_pyramid_or_workspace():
     before = lh.launch_count()
     assert lib.lh_pool(ctypes.byref(cfg), a, a, a, None, None, None, None, None) == 0
     assert lh.launch_count() == before
+
+
+def test_sharded_entry_points_validate_before_launch():
+    """The sequence-sharded calls refuse bad rank geometry and non-bf16
+    attention before anything is launched (no device needed)."""
+    ptr = 1 << 20                                        # any 16-byte aligned address: nothing is touched
+    f = lh.lib()
+    cfg = lh.make_config(1, 2, 8192, 128, 4, 3, 64)
+    assert f.lh_cp_segment(ctypes.byref(cfg), 3, 0, ptr, ptr, ptr, ptr, None) == LH_ERR_SHAPE   # 8192 / 3
+    assert f.lh_cp_segment(ctypes.byref(cfg), 4, 4, ptr, ptr, ptr, ptr, None) == LH_ERR_SHAPE   # rank 4 of 4
+    assert f.lh_cp_segment(ctypes.byref(cfg), 0, 0, ptr, ptr, ptr, ptr, None) == LH_ERR_SHAPE   # no ranks
+    assert f.lh_cp_segment(ctypes.byref(cfg), 1024, 0, ptr, ptr, ptr, ptr, None) == LH_ERR_SHAPE  # 8 tokens
+    assert f.lh_cp_segment(ctypes.byref(cfg), 2, 0, None, ptr, ptr, ptr, None) == LH_ERR_NULL
+    assert f.lh_cp_segment(ctypes.byref(cfg), 2, 0, ptr + 4, ptr, ptr, ptr, None) == LH_ERR_ALIGN
+    c32 = lh.make_config(1, 2, 8192, 128, 4, 3, 64, "fp32")
+    assert f.lh_cp_attn_fwd(ctypes.byref(c32), 2, 0, *([ptr] * 6), None) == LH_ERR_DTYPE
+    assert f.lh_cp_attn_bwd(ctypes.byref(c32), 2, 0, *([ptr] * 10), None) == LH_ERR_DTYPE
+    c1 = lh.make_config(1, 2, 8192, 128, 4, 1, 64)
+    assert f.lh_cp_plan(ctypes.byref(c1), 2, 0, ctypes.byref(lh.CPPlan())) == LH_ERR_SHAPE    # L = 1
+    pl = lh.cp_plan(cfg, 4, 3)
+    assert (pl.n_loc, pl.E_loc, pl.glob.S) == (2048, 512 + 128, lh.plan(cfg).S)
+    assert list(pl.lvl_off_loc)[1:3] == [0, 512]

@@ -171,3 +171,77 @@ def test_sequence_sharded_oracle_ranks_in_one_process(world, readings):
 def test_sequence_sharded_oracle_rejects_unaligned_shards():
     with pytest.raises(ValueError):
         sharded.shard_sizes(96, 4, 3, 4)                # 24 tokens per rank, not a multiple of 16
+
+
+# ---------------------------------------------------------------------------
+# the sharded driver's collectives (cp.run_distributed) over gloo, on CPU
+# ---------------------------------------------------------------------------
+
+class _RecordingRank:
+    """Stands in for cp.ShardRank on the CPU: each step fills its buffers with
+    rank-tagged values and checks what the collectives delivered, so the
+    driver's order of steps and collectives is exercised without a GPU."""
+
+    def __init__(self, rank, world):
+        self.rank, self.world, self.device = rank, world, torch.device("cpu")
+        self.sq_loc = torch.empty(2, 1, 2, 5, dtype=torch.float64)
+        S = 4 * world
+        self.ks, self.vs = torch.zeros(1, 2, S, 3), torch.zeros(1, 2, S, 3)
+        self.dks, self.dvs = torch.zeros(1, 2, S, 3), torch.zeros(1, 2, S, 3)
+        self.log = []
+
+    def gathered_shape(self):
+        return (self.world,) + tuple(self.sq_loc.shape)
+
+    def pool(self, q, k, v):
+        self.sq_loc.fill_(self.rank + 1)
+        self.log.append("pool")
+
+    def select_gather(self, gathered, q, k, v):
+        for r in range(self.world):                      # every rank's norms, in rank order
+            assert torch.all(gathered[r] == r + 1)
+        rows = slice(4 * self.rank, 4 * self.rank + 4)   # this rank's segment, zero elsewhere
+        self.ks.zero_()
+        self.vs.zero_()
+        self.ks[:, :, rows] = self.rank + 1
+        self.vs[:, :, rows] = -(self.rank + 1)
+        self.log.append("select_gather")
+
+    def attend_scatter(self, o):
+        for r in range(self.world):                      # the all-reduce assembled every segment
+            assert torch.all(self.ks[:, :, 4 * r:4 * r + 4] == r + 1)
+            assert torch.all(self.vs[:, :, 4 * r:4 * r + 4] == -(r + 1))
+        o.fill_(self.rank)
+        self.log.append("attend_scatter")
+
+    def attend_bwd(self, do):
+        self.dks.fill_(self.rank + 1)                    # this rank's queries' part of every key gradient
+        self.dvs.fill_(2 * (self.rank + 1))
+        self.log.append("attend_bwd")
+
+    def spread(self, dq, dk, dv):
+        tot = self.world * (self.world + 1) // 2
+        assert torch.all(self.dks == tot) and torch.all(self.dvs == 2 * tot)
+        self.log.append("spread")
+
+
+def _cp_driver_worker(rank, world, port, out_dir):
+    os.environ.update(RANK=str(rank), WORLD_SIZE=str(world), LOCAL_RANK=str(rank),
+                      MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    assert lhdist.init("gloo", timeout_s=60)
+    from long_context_symmetric_b200 import cp
+    st = _RecordingRank(rank, world)
+    o = torch.empty(3)
+    cp.run_distributed(st, None, None, None, o, do=torch.empty(1), dq=None, dk=None, dv=None)
+    assert torch.all(o == rank)
+    np.save(os.path.join(out_dir, f"log{rank}.npy"), np.array(st.log))
+    lhdist.shutdown()
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_sharded_driver_collectives_over_gloo(tmp_path, world):
+    mp.start_processes(_cp_driver_worker, args=(world, _free_port(), str(tmp_path)), nprocs=world, join=True,
+                       start_method="spawn")
+    for r in range(world):
+        assert list(np.load(tmp_path / f"log{r}.npy")) == ["pool", "select_gather", "attend_scatter",
+                                                            "attend_bwd", "spread"]

@@ -1,0 +1,94 @@
+"""Sequence-sharded (context-parallel) path on one GPU, ranks emulated.
+
+Every rank's steps are the lh_cp_* kernels; the ranks of one job run one
+after another in this process and the collectives are formed from all ranks'
+tensors (cp.run_emulated), so no kernel ever waits on another rank. Checked
+against the single-GPU path on the same whole-sequence inputs, and against
+the fp64 oracle:
+  - selection, gather map and slot table: bit-exact (every rank runs the same
+    descent on the assembled norms);
+  - each rank's segment is the run of slots whose entries lie in its shard;
+  - O and dQ: bit-exact (each query row sees the same key tiles in the same
+    order as on one GPU);
+  - dK, dV: the key gradients are summed over ranks, so they agree with the
+    single-GPU result to fp32 rounding and with the oracle within the stated
+    tolerance.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+from lhtest import ATOL, Case, excess_error, run_gpu, to64
+import oracle as orc
+from long_context_symmetric_b200 import cp, lh, synth
+
+pytestmark = pytest.mark.gpu
+DEV = torch.device("cuda", 0)
+
+CASES = [
+    (Case("cp_w2", 1, 2, 8192, 128, "bf16", 4, 3, 64), 2),
+    (Case("cp_w4", 1, 2, 8192, 128, "bf16", 4, 3, 64), 4),
+    (Case("cp_w4_d64_b2", 2, 3, 8192, 64, "bf16", 4, 4, 40, recipe="token_scale"), 4),
+    (Case("cp_w8_ties", 1, 2, 16384, 128, "bf16", 4, 4, 100, recipe="codebook", accum="fixed"), 8),
+    (Case("cp_w2_pre_partition", 1, 2, 8192, 128, "bf16", 4, 3, 64, order="pre", inclusion="partition",
+          weight="mean"), 2),
+    (Case("cp_w4_p8_l4", 1, 2, 32768, 128, "bf16", 8, 4, 256, recipe="outliers"), 4),
+]
+
+
+def _shard(x, world, r):
+    n = x.shape[1] // world
+    return x[:, r * n:(r + 1) * n].contiguous()
+
+
+@pytest.mark.parametrize("case,world", CASES, ids=[c.name for c, _ in CASES])
+def test_sharded_path_matches_single_gpu_and_oracle(case, world):
+    w = case.workload()
+    q, k, v = (x.to(DEV) for x in synth.make_inputs(w))
+    do = synth.make_dout(w).to(DEV)
+    ref = run_gpu(case, q, k, v, do)                      # the single-GPU path
+    cfg = case.cfg()
+    ranks = [cp.ShardRank(cfg, world, r, DEV) for r in range(world)]
+    sh = lambda x: [_shard(x, world, r) for r in range(world)]
+    qs_, ks_, vs_, dos_ = sh(q), sh(k), sh(v), sh(do)
+    outs = [torch.empty_like(x) for x in qs_]
+    dqs, dks, dvs = ([torch.empty_like(x) for x in qs_] for _ in range(3))
+    cp.run_emulated(ranks, qs_, ks_, vs_, outs, dos_, dqs, dks, dvs)
+    torch.cuda.synchronize()
+    assert lh.get_device_error() == (0, 0)
+    ws = ref["ws"]
+    S = ws.map.shape[-1]
+    starts = np.zeros((case.B, case.H), dtype=np.int64)
+    for r, st in enumerate(ranks):
+        assert torch.equal(st.sel, ws.sel) and torch.equal(st.map, ws.map) and torch.equal(st.slot, ws.slot)
+        seg = st.seg.cpu().numpy()
+        assert np.array_equal(seg[..., 0], starts)          # segments follow each other in rank order
+        m = st.map.cpu().numpy().astype(np.int64)
+        lvl, idx = m >> 28, m & 0x0FFFFFFF
+        first = idx * case.p ** lvl                          # first token each entry covers
+        n = case.N // world
+        for b in range(case.B):
+            for h in range(case.H):
+                mine = (first[b, h] >= r * n) & (first[b, h] < (r + 1) * n)
+                s0, cnt = seg[b, h]
+                assert mine.sum() == cnt and np.all(mine[s0:s0 + cnt])
+        starts += seg[..., 1]
+    assert np.all(starts == S)
+    o = torch.cat(outs, dim=1)
+    dq, dk, dv = (torch.cat(x, dim=1) for x in (dqs, dks, dvs))
+    assert torch.equal(o, ref["o"])
+    assert torch.equal(dq, ref["dq"])
+    for name, got in (("dk", dk), ("dv", dv)):
+        diff = (got.float() - ref[name].float()).abs()
+        ulp = ref[name].float().abs().clamp_min(2 ** -20) * 2 ** -7     # one bf16 ulp (or less)
+        assert bool((diff <= ulp).all()), name
+    # against the fp64 oracle on the first and last heads
+    for (b, h) in [(0, 0), (case.B - 1, case.H - 1)]:
+        qh, kh, vh = (to64(x[b, :, h, :]) for x in (q, k, v))
+        fw = orc.forward_head(qh, kh, vh, case.p, case.L, case.K, case.dtype, case.accum, **case.readings)
+        bw = orc.backward_head(fw, to64(do[b, :, h, :]), case.p, case.accum)
+        assert excess_error(to64(o[b, :, h, :]), fw["o"], case.dtype) <= ATOL[case.dtype]
+        for name, got in (("dq", dq), ("dk", dk), ("dv", dv)):
+            e = excess_error(to64(got[b, :, h, :]), bw[name], case.dtype)
+            assert e <= ATOL[case.dtype], (name, e)

@@ -1,0 +1,68 @@
+"""Fusion with the neighbouring projections, chunk by chunk through L2
+(long_context_symmetric_b200.fused): the pool of each projected chunk and the
+scatter feeding each output-projection chunk equal the whole-sequence
+lh_pool / lh_scatter bit for bit, and the projections equal the same GEMMs
+run on the unfused tensors."""
+
+import pytest
+import torch
+
+from lhtest import Case, compare_head, run_gpu
+from long_context_symmetric_b200 import fused, lh, synth
+
+pytestmark = pytest.mark.gpu
+DEV = torch.device("cuda", 0)
+
+
+@pytest.mark.parametrize("B,H,N,D,p,L,K,chunk", [
+    (1, 4, 16384, 128, 4, 3, 64, 2048),
+    (2, 3, 8192, 64, 8, 3, 16, 1024),
+    (1, 2, 4096, 128, 2, 5, 32, 1 << 12),          # one chunk
+])
+def test_chunked_projection_pool_and_scatter(B, H, N, D, p, L, K, chunk):
+    g = torch.Generator(device=DEV).manual_seed(9)
+    dm = H * D
+    x = torch.randn(B, N, dm, generator=g, device=DEV).to(torch.bfloat16)
+    w = [(torch.randn(dm, dm, generator=g, device=DEV) / dm ** 0.5).to(torch.bfloat16) for _ in range(4)]
+    cfg = lh.make_config(B, H, N, D, p, L, K, "bf16")
+    ws = lh.Workspace(cfg, DEV, backward=False)
+    q, k, v = (torch.empty(B, N, H, D, dtype=torch.bfloat16, device=DEV) for _ in range(3))
+    fused.qkv_project_pool(cfg, ws, x, w[0], w[1], w[2], q, k, v, chunk=chunk)
+    # the unfused reference: the same GEMMs, then the whole-sequence pool
+    qr, kr, vr = (torch.empty_like(q) for _ in range(3))
+    for t0 in range(0, N, chunk):
+        for b in range(B):
+            for wt, out in ((w[0], qr), (w[1], kr), (w[2], vr)):
+                torch.matmul(x[b, t0:t0 + chunk], wt, out=out[b, t0:t0 + chunk].view(chunk, dm))
+    ref = lh.Workspace(cfg, DEV, backward=False)
+    lh.pool(cfg, qr, kr, vr, ref.pyr_q, ref.pyr_k, ref.pyr_v, ref.sq)
+    torch.cuda.synchronize()
+    assert torch.equal(q, qr) and torch.equal(k, kr) and torch.equal(v, vr)
+    for a, b_ in ((ws.pyr_q, ref.pyr_q), (ws.pyr_k, ref.pyr_k), (ws.pyr_v, ref.pyr_v), (ws.sq, ref.sq)):
+        assert torch.equal(a, b_)
+    # rest of the forward, then the chunked scatter + output projection
+    lh.score_topk(cfg, ws.sq, ws.sel, ws.map, ws.slot, ws.ws)
+    lh.gather(cfg, q, k, v, ws.pyr_q, ws.pyr_k, ws.pyr_v, ws.map, ws.qs, ws.ks, ws.vs)
+    lh.attn_fwd(cfg, ws.qs, ws.ks, ws.vs, ws.os, ws.lse)
+    o = torch.empty_like(q)
+    y = torch.empty(B, N, dm, dtype=torch.bfloat16, device=DEV)
+    fused.scatter_project(cfg, ws, w[3], o, y, chunk=chunk)
+    o_ref = torch.empty_like(q)
+    lh.scatter(cfg, ws.os, ws.slot, o_ref)
+    y_ref = torch.empty_like(y)
+    for t0 in range(0, N, chunk):
+        for b in range(B):
+            torch.matmul(o_ref[b, t0:t0 + chunk].view(chunk, dm), w[3], out=y_ref[b, t0:t0 + chunk])
+    torch.cuda.synchronize()
+    assert lh.get_device_error() == (0, 0)
+    assert torch.equal(o, o_ref)
+    assert torch.equal(y, y_ref)
+
+
+def test_ranges_reject_unaligned_tokens():
+    cfg = lh.make_config(1, 2, 4096, 128, 4, 3, 16, "bf16")
+    t = torch.empty(1 << 16, dtype=torch.uint8, device=DEV)
+    with pytest.raises(lh.LHError):
+        lh.pool_range(cfg, 8, 16, t, t, t, t, t, t, t)          # t0 not a multiple of 16
+    with pytest.raises(lh.LHError):
+        lh.scatter_range(cfg, 0, 4112, t, t, t)                # past N
