@@ -261,16 +261,14 @@ def measure_fusion(cfg, w, ws, dev, iters=3):
                 torch.matmul(x[b], wi, out=out[b].view(N, dm))
         lh.pool(cfg, q, k, v, ws.pyr_q, ws.pyr_k, ws.pyr_v, ws.sq)
 
-    def qkv_chunked():
-        fused.qkv_project_pool(cfg, ws, x, wt[0], wt[1], wt[2], q, k, v)
+    qkv_chunked = fused.Graphed(lambda: fused.qkv_project_pool(cfg, ws, x, wt[0], wt[1], wt[2], q, k, v))
 
     def out_unfused():
         lh.scatter(cfg, ws.os, ws.slot, o)
         for b in range(B):
             torch.matmul(o[b].view(N, dm), wt[3], out=y[b])
 
-    def out_chunked():
-        fused.scatter_project(cfg, ws, wt[3], o, y)
+    out_chunked = fused.Graphed(lambda: fused.scatter_project(cfg, ws, wt[3], o, y))
 
     def timeit(fn):
         fn()
@@ -288,7 +286,8 @@ def measure_fusion(cfg, w, ws, dev, iters=3):
     res = {"d_model": dm, "chunk_tokens": fused.chunk_tokens(cfg),
            "qkv_projection_plus_pool_ms": {"unfused": timeit(qkv_unfused), "chunked_l2": timeit(qkv_chunked)},
            "scatter_plus_out_projection_ms": {"unfused": timeit(out_unfused), "chunked_l2": timeit(out_chunked)},
-           "projections": "cuBLAS bf16 GEMMs through torch.matmul (the model's, outside the path)"}
+           "projections": "cuBLAS bf16 GEMMs through torch.matmul (the model's, outside the path)",
+           "chunked_runs_as": "one CUDA graph per chunk loop (captured once, replayed)"}
     st, detail = lh.get_device_error()
     if st != 0:
         raise RuntimeError(f"device error {st} ({detail}) in the fusion timing")

@@ -21,9 +21,7 @@
 //             other tile (about 1.5 tiles of MMA time for 1 tile of softmax).
 //   warps 2-5 softmax of tile A, warps 6-9 of tile B; one thread per query row
 //             (= TMEM lane): scores from TMEM, causal mask on the diagonal
-//             tile, online softmax in the exp2 domain (a quarter of the
-//             exponentials by a polynomial on the FMA pipe, the rest on the
-//             special-function unit) with a lazily updated
+//             tile, online softmax in the exp2 domain with a lazily updated
 //             running max (O is rescaled in TMEM only when the max grows by
 //             more than 2^8); P is split into an fp16 head and an fp16
 //             remainder written into the score columns (each 32-column chunk
@@ -53,11 +51,6 @@ constexpr int kBN = 128;       // key rows per tile
 constexpr int kSub = 128 * 64 * 2;   // one 128-row x 64-column 16-bit swizzle tile (16 KB)
 constexpr float kLn2f = 0.6931471805599453f;
 constexpr int kFwdThreads = 320;
-// Column pairs of every 8 whose exponentials run on the FMA pipe (tc::exp2_fma2)
-// instead of the special-function unit: ex2 alone would keep that unit busy
-// 8 cycles per warp instruction while the rest of the softmax needs about
-// 5 issue cycles per pair, so moving a quarter of the pairs balances the two.
-constexpr int kFwdFmaPairs = 3;
 
 // Barriers first, then the swizzled tiles from the next 1024-byte boundary.
 template <int D>
@@ -83,7 +76,9 @@ struct FwdBars {
 };
 static_assert(sizeof(FwdBars) <= 256, "barrier block");
 
-template <int D>
+// SEG: the queries are one per-(b, h) segment of the rows (seg); without it,
+// every row is a query (q0 = 0, nq = S at compile time).
+template <int D, bool SEG>
 __global__ void __launch_bounds__(kFwdThreads, 1)
 k_attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
               const __grid_constant__ CUtensorMap tv, float* __restrict__ os, float* __restrict__ lse,
@@ -101,7 +96,7 @@ k_attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CU
   // [0, q0 + nq) of ks / vs (the whole sub-sequence, or one rank's segment of
   // it in the sequence-sharded path, `seg` = (q0, nq) per (b, h)).
   const int bh = blockIdx.y;
-  const int q0 = seg ? seg[2 * bh] : 0, nq = seg ? seg[2 * bh + 1] : S;
+  const int q0 = SEG ? seg[2 * bh] : 0, nq = SEG ? seg[2 * bh + 1] : S;
   const int ntiles = (nq + kBM - 1) / kBM;
   const int mp = (ntiles + 1) / 2 - 1 - (int)blockIdx.x;     // heavy (late) pairs first
   if (mp < 0) return;                                          // whole CTA, before any set-up
@@ -330,8 +325,7 @@ k_attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CU
               const int e = 4 * g + u;
               const float2 x = __ffma2_rn(
                   make_float2(__uint_as_float(s[32 * c + 2 * e]), __uint_as_float(s[32 * c + 2 * e + 1])), cc, nm);
-              // kFwdFmaPairs of every 8 column pairs on the FMA pipe, the rest on ex2
-              const float2 pp = (e & 7) < kFwdFmaPairs ? exp2_fma2(x) : make_float2(ex2(x.x), ex2(x.y));
+              const float2 pp = make_float2(ex2(x.x), ex2(x.y));
               acc[u & 1] = __fadd2_rn(acc[u & 1], pp);
               const __half2 h = __float22half2_rn(pp);
               const __half2 l = __float22half2_rn(__ffma2_rn(__half22float2(h), m1, pp));   // p - hi, exact
@@ -418,12 +412,13 @@ static cudaError_t fwd_tc_t(const Geom& g, const void* qs, const void* ks, const
       !make_tmap_16(&tv, vs, D, g.S, BH, true, kBN))
     return cudaErrorInvalidValue;
   const int smem = FwdLayout<D>::BYTES;
-  cudaError_t e = cudaFuncSetAttribute(k_attn_fwd_tc<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  auto kern = seg ? k_attn_fwd_tc<D, true> : k_attn_fwd_tc<D, false>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   const float c2 = (float)(1.4426950408889634 / sqrt((double)D));
   const int ntiles = (g.S + kBM - 1) / kBM;
   dim3 grid((ntiles + 1) / 2, BH);
-  k_attn_fwd_tc<D><<<grid, kFwdThreads, smem, s>>>(tq, tk, tv, os, lse, g.S, c2, seg, err);
+  kern<<<grid, kFwdThreads, smem, s>>>(tq, tk, tv, os, lse, g.S, c2, seg, err);
   count_launch();
   return cudaGetLastError();
 }

@@ -316,13 +316,6 @@ __device__ __forceinline__ float2 f2(uint32_t a, uint32_t b) {
 }
 __device__ __forceinline__ uint32_t h2_bits(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
 
-// Column pairs of every 8 whose exponentials run on the FMA pipe
-// (tc::exp2_fma2) rather than on the special-function unit, per kernel: the
-// dK/dV compute warps do less other work per pair than the dQ warps (no dS
-// split), so more of their exponentials move.
-constexpr int kDkdvFmaPairs = 3;
-constexpr int kDqFmaPairs = 2;
-
 // 32 columns of this thread's key row (dK/dV kernel): P^T = 2^(S^T c2 - lse2)
 // in place, two columns per packed fp32 instruction. nl2 holds -lse2 of the
 // 32 query columns (the same for every lane: broadcast reads). MASK: columns
@@ -337,15 +330,7 @@ __device__ __forceinline__ void p_chunk_t(uint32_t (&s)[32], const float* nl2, f
 #pragma unroll
     for (int u = 0; u < 4; u += 2) {
       const float2 x = __ffma2_rn(f2(s[e + u], s[e + u + 1]), cc, u ? make_float2(a.z, a.w) : make_float2(a.x, a.y));
-      float p0, p1;
-      if ((((e + u) >> 1) & 7) < kDkdvFmaPairs) {
-        const float2 pp = exp2_fma2(x);
-        p0 = pp.x;
-        p1 = pp.y;
-      } else {
-        p0 = ex2(x.x);
-        p1 = ex2(x.y);
-      }
+      float p0 = ex2(x.x), p1 = ex2(x.y);
       if (MASK) {
         const int col = col0 + e + u;
         if (col < vlo || col > vhi) p0 = 0.f;
@@ -387,15 +372,7 @@ __device__ __forceinline__ void p_chunk(uint32_t (&s)[32], float nl2, float c2, 
 #pragma unroll
   for (int e = 0; e < 32; e += 2) {
     const float2 x = __ffma2_rn(f2(s[e], s[e + 1]), cc, nl);
-    float p0, p1;
-    if (((e >> 1) & 7) < kDqFmaPairs) {
-      const float2 pp = exp2_fma2(x);
-      p0 = pp.x;
-      p1 = pp.y;
-    } else {
-      p0 = ex2(x.x);
-      p1 = ex2(x.y);
-    }
+    float p0 = ex2(x.x), p1 = ex2(x.y);
     if (MASK) {
       if (col0 + e > vhi) p0 = 0.f;
       if (col0 + e + 1 > vhi) p1 = 0.f;
@@ -420,7 +397,9 @@ __device__ __forceinline__ void ds_chunk(const uint32_t (&p)[32], const uint32_t
 }
 
 // ---------------------------------------------------------------- dK, dV
-template <int D>
+// SEG: the queries are one per-(b, h) segment of the rows (seg); without it,
+// every row is a query (q0 = 0, nq = S at compile time).
+template <int D, bool SEG>
 __global__ void __launch_bounds__(kThreads, 1)
 k_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
               const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tdo,
@@ -434,7 +413,7 @@ k_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CU
   const int j = blockIdx.x;            // key tile (rows j*128 ..); small j has the most query tiles
   const int bh = blockIdx.y;
   // query rows [q0, q0 + nq) of this (b, h) (all S rows, or one rank's segment)
-  const int q0 = seg ? seg[2 * bh] : 0, nq = seg ? seg[2 * bh + 1] : S;
+  const int q0 = SEG ? seg[2 * bh] : 0, nq = SEG ? seg[2 * bh + 1] : S;
   const int ntq = (nq + kT - 1) / kT;
   const int i0 = max(0, j * kT - q0) / kT;   // first query tile with a row at or after key row j*128
   const int n = ntq - i0;                    // query tiles i = i0 .. ntq-1
@@ -568,7 +547,7 @@ k_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CU
 }
 
 // ---------------------------------------------------------------- dQ
-template <int D>
+template <int D, bool SEG>
 __global__ void __launch_bounds__(kThreads, 1)
 k_bwd_dq_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tdo,
             const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
@@ -580,7 +559,7 @@ k_bwd_dq_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
   uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + Lay::HEAD + 1023) & ~(uintptr_t)1023);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int bh = blockIdx.y;
-  const int q0 = seg ? seg[2 * bh] : 0, nq = seg ? seg[2 * bh + 1] : S;
+  const int q0 = SEG ? seg[2 * bh] : 0, nq = SEG ? seg[2 * bh + 1] : S;
   const int ntq = (nq + kT - 1) / kT;
   const int i = ntq - 1 - (int)blockIdx.x;        // query tile; late tiles have the most key tiles
   if (i < 0) return;                              // whole CTA, before any set-up
@@ -676,18 +655,20 @@ cudaError_t bwd_tc_t(const Geom& g, const void* qs, const void* ks, const void* 
       !make_tmap_16(&tv, vs, D, g.S, BH, true, kT) || !make_tmap_16(&tdo, dos, D, g.S, BH, true, kT))
     return cudaErrorInvalidValue;
   const int smem = BwdLayout<D>::BYTES, smem_q = smem;
-  cudaError_t e = cudaFuncSetAttribute(k_bwd_dkdv_tc<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  auto dkdv = seg ? k_bwd_dkdv_tc<D, true> : k_bwd_dkdv_tc<D, false>;
+  auto dq = seg ? k_bwd_dq_tc<D, true> : k_bwd_dq_tc<D, false>;
+  cudaError_t e = cudaFuncSetAttribute(dkdv, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(k_bwd_dq_tc<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_q);
+  e = cudaFuncSetAttribute(dq, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_q);
   if (e != cudaSuccess) return e;
   const float scale = (float)(1.0 / sqrt((double)D));
   const float c2 = (float)(1.4426950408889634 / sqrt((double)D));
   dim3 grid((g.S + kT - 1) / kT, BH);
-  k_bwd_dkdv_tc<D><<<grid, kThreads, smem, s>>>(tk, tv, tq, tdo, lse, delta, dks, dvs, g.S, c2, scale, seg, err);
+  dkdv<<<grid, kThreads, smem, s>>>(tk, tv, tq, tdo, lse, delta, dks, dvs, g.S, c2, scale, seg, err);
   count_launch();
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  k_bwd_dq_tc<D><<<grid, kThreads, smem_q, s>>>(tq, tdo, tk, tv, lse, delta, dqs, g.S, c2, scale, seg, err);
+  dq<<<grid, kThreads, smem_q, s>>>(tq, tdo, tk, tv, lse, delta, dqs, g.S, c2, scale, seg, err);
   count_launch();
   return cudaGetLastError();
 }

@@ -272,9 +272,13 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
-// 2^x of two values on the FMA and integer pipes, leaving the special-function
-// unit (ex2, 4 lanes per clock per SM sub-partition) to the other elements of a
-// softmax tile. Range reduction x = n + f, n = rint(x), f in [-1/2, 1/2]: adding
+// 2^x of two values on the FMA and integer pipes instead of the
+// special-function unit (ex2, 4 lanes per clock per SM sub-partition). Measured
+// in the attention kernels with a quarter to three eighths of each softmax
+// tile's exponentials moved here, it made the forward 5-20 % slower and left the
+// backward unchanged at 512K context (the kernels are not limited by the
+// special-function unit), so the kernels keep ex2; lh_selftest_exp2 evaluates
+// it. Range reduction x = n + f, n = rint(x), f in [-1/2, 1/2]: adding
 // 1.5 * 2^23 rounds x to an integer in the low mantissa bits of t, so t - 1.5 *
 // 2^23 = n and x - n = f are exact. 2^f: degree-5 polynomial with minimax
 // relative error on [-1/2, 1/2] (Remez exchange; gen_exp2_poly.py beside this

@@ -18,7 +18,10 @@ into chunks of whole coarsest blocks small enough to stay in the 126 MB L2:
 
 The projections are plain library GEMMs (they are the model's, not the path's);
 every step of the path stays a liblh kernel. The pool and scatter results
-are bit-identical to lh_pool and lh_scatter over the whole sequence.
+are bit-identical to lh_pool and lh_scatter over the whole sequence. A 512K
+sequence is 128 chunks of several launches each, too many for the host to
+issue at GPU speed, so ``Graphed`` captures a chunk loop once as a CUDA graph
+and replays it.
 """
 
 from __future__ import annotations
@@ -27,7 +30,7 @@ import torch
 
 from . import lh
 
-__all__ = ["chunk_tokens", "qkv_project_pool", "scatter_project"]
+__all__ = ["chunk_tokens", "qkv_project_pool", "scatter_project", "Graphed"]
 
 
 def chunk_tokens(cfg, target: int = 4096) -> int:
@@ -85,3 +88,26 @@ def scatter_project(cfg, ws, w_o, o, y, chunk=None, side=None):
         d.record(main)
         done.append(d)
     main.wait_stream(side)
+
+
+class Graphed:
+    """A stream-ordered function (such as a chunk loop above) captured once as a
+    CUDA graph and replayed by calling the object: the host issues one graph
+    launch instead of several hundred kernel launches. The function runs once
+    un-captured first (library handles, device-symbol lookups and kernel
+    attributes are set up outside the capture). It must read and write the same
+    tensors on every call."""
+
+    def __init__(self, fn):
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            fn()
+        torch.cuda.current_stream().wait_stream(side)
+        torch.cuda.synchronize()
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph):
+            fn()
+
+    def __call__(self):
+        self.graph.replay()

@@ -1,13 +1,14 @@
 """The FMA-pipe 2^x of the attention softmax against fp64 and against ex2.approx.
 
-The tensor-core attention kernels take part of every softmax tile's
-exponentials off the special-function unit: range reduction to [-1/2, 1/2], a
-degree-5 polynomial with minimax relative error there (Remez exchange), and
-the exponent added in the bit pattern. Its maximum relative error must stay
-within that of the ex2.approx.ftz.f32 it stands in for (the PTX ISA states
-about 2^-22 for ex2.approx.f32); it is checked here against 2^x in fp64 over
-the whole range the kernels use, with the special-function result measured
-beside it.
+A 2^x for the FMA pipe (range reduction to [-1/2, 1/2], a degree-5 polynomial
+with minimax relative error there found by the Remez exchange, and the
+exponent added in the bit pattern), built to take part of each softmax
+tile's exponentials off the special-function unit. Its maximum relative error
+must stay within that of the ex2.approx.ftz.f32 it would stand in for (the PTX
+ISA states about 2^-22 for ex2.approx.f32); it is checked here against 2^x in
+fp64 over the range the softmax uses, with the special-function result
+measured beside it. (Measured inside the attention kernels it did not pay off;
+they keep ex2.)
 """
 
 import numpy as np
@@ -49,4 +50,4 @@ def test_exp2_polynomial_clamps_below_range():
     lh.selftest_exp2(x, y_fma, y_sfu)
     torch.cuda.synchronize()
     got = y_fma.cpu().numpy().astype(np.float64)
-    assert np.all(got == 2.0 ** -125)
+    assert np.all(np.abs(got / 2.0 ** -125 - 1) <= 2.0 ** -22)      # 2^-125 to the polynomial's accuracy

@@ -80,8 +80,12 @@ def test_sharded_path_matches_single_gpu_and_oracle(case, world):
     assert torch.equal(o, ref["o"])
     assert torch.equal(dq, ref["dq"])
     for name, got in (("dk", dk), ("dv", dv)):
-        diff = (got.float() - ref[name].float()).abs()
-        ulp = ref[name].float().abs().clamp_min(2 ** -20) * 2 ** -7     # one bf16 ulp (or less)
+        # the key gradients' fp32 sums are grouped by rank: one bf16 ulp apart,
+        # or more where the ranks' parts cancel, by at most fp32 rounding of the parts
+        r32 = ref[name].float()
+        diff = (got.float() - r32).abs()
+        ulp = r32.abs() * 2 ** -7 + 2 ** -16 * r32.abs().max()
+        print(name, "max |sharded - single GPU|", float(diff.max()), "of max", float(r32.abs().max()))
         assert bool((diff <= ulp).all()), name
     # against the fp64 oracle on the first and last heads
     for (b, h) in [(0, 0), (case.B - 1, case.H - 1)]:

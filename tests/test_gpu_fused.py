@@ -59,6 +59,40 @@ def test_chunked_projection_pool_and_scatter(B, H, N, D, p, L, K, chunk):
     assert torch.equal(y, y_ref)
 
 
+def test_graphed_chunk_loop_replays_the_same_results():
+    """The chunk loops captured as CUDA graphs (fused.Graphed) give the same
+    pyramid, norms and output as the un-captured loops."""
+    B, H, N, D, p, L, K, chunk = 1, 2, 8192, 128, 4, 3, 32, 1024
+    g = torch.Generator(device=DEV).manual_seed(3)
+    dm = H * D
+    x = torch.randn(B, N, dm, generator=g, device=DEV).to(torch.bfloat16)
+    w = [(torch.randn(dm, dm, generator=g, device=DEV) / dm ** 0.5).to(torch.bfloat16) for _ in range(4)]
+    cfg = lh.make_config(B, H, N, D, p, L, K, "bf16")
+    ws, ref = lh.Workspace(cfg, DEV, backward=False), lh.Workspace(cfg, DEV, backward=False)
+    q, k, v, o = (torch.empty(B, N, H, D, dtype=torch.bfloat16, device=DEV) for _ in range(4))
+    y = torch.empty(B, N, dm, dtype=torch.bfloat16, device=DEV)
+    fused.qkv_project_pool(cfg, ref, x, w[0], w[1], w[2], q, k, v, chunk=chunk)
+    lh.score_topk(cfg, ref.sq, ref.sel, ref.map, ref.slot, ref.ws)
+    lh.gather(cfg, q, k, v, ref.pyr_q, ref.pyr_k, ref.pyr_v, ref.map, ref.qs, ref.ks, ref.vs)
+    lh.attn_fwd(cfg, ref.qs, ref.ks, ref.vs, ref.os, ref.lse)
+    fused.scatter_project(cfg, ref, w[3], o, y, chunk=chunk)
+    torch.cuda.synchronize()
+    y_ref = y.clone()
+    gq = fused.Graphed(lambda: fused.qkv_project_pool(cfg, ws, x, w[0], w[1], w[2], q, k, v, chunk=chunk))
+    ws.os.copy_(ref.os)
+    ws.slot.copy_(ref.slot)
+    go = fused.Graphed(lambda: fused.scatter_project(cfg, ws, w[3], o, y, chunk=chunk))
+    for _ in range(2):
+        ws.sq.zero_()
+        y.zero_()
+        gq()
+        go()
+        torch.cuda.synchronize()
+        assert torch.equal(ws.sq, ref.sq) and torch.equal(ws.pyr_k, ref.pyr_k)
+        assert torch.equal(y, y_ref)
+    assert lh.get_device_error() == (0, 0)
+
+
 def test_ranges_reject_unaligned_tokens():
     cfg = lh.make_config(1, 2, 4096, 128, 4, 3, 16, "bf16")
     t = torch.empty(1 << 16, dtype=torch.uint8, device=DEV)
