@@ -58,8 +58,8 @@ def workload_desc(w):
 # None when one of them changes.
 DRAM_TRAFFIC = {
     "ctx512k": {
-        "attn_bwd": 8 * (52.885504e6 + 8.821760e6 + 52.882688e6 + 2.786560e6),   # dK/dV + dQ kernels
-        "attn_fwd": 8 * (39.371776e6 + 0.552192e6),
+        "attn_bwd": 8 * (52.938240e6 + 9.091328e6 + 52.884992e6 + 3.098624e6),   # dK/dV + dQ kernels
+        "attn_fwd": 8 * (39.404288e6 + 0.345600e6),
     },
 }
 
@@ -259,7 +259,7 @@ def measure_fusion(cfg, w, ws, dev, iters=3):
         for b in range(B):
             for wi, out in zip(wt[:3], (q, k, v)):
                 torch.matmul(x[b], wi, out=out[b].view(N, dm))
-        lh.pool(cfg, q, k, v, ws.pyr_q, ws.pyr_k, ws.pyr_v, ws.sq)
+        lh.pool(cfg, q, k, v, ws.pyr_q, ws.pyr_k, ws.pyr_v, ws.sq, ws.scale)
 
     qkv_chunked = fused.Graphed(lambda: fused.qkv_project_pool(cfg, ws, x, wt[0], wt[1], wt[2], q, k, v))
 
@@ -414,19 +414,19 @@ def main():
             if ev is not None:
                 ev[i].record(stream)
         mark(0)
-        lh.pool(c, q, k, v, ws.pyr_q, ws.pyr_k, ws.pyr_v, ws.sq, stream)
+        lh.pool(c, q, k, v, ws.pyr_q, ws.pyr_k, ws.pyr_v, ws.sq, ws.scale, stream)
         mark(1)
         lh.score_topk(c, ws.sq, ws.sel, ws.map, ws.slot, ws.ws, stream=stream)
         mark(2)
-        lh.gather(c, q, k, v, ws.pyr_q, ws.pyr_k, ws.pyr_v, ws.map, ws.qs, ws.ks, ws.vs, stream)
+        lh.gather(c, q, k, v, ws.pyr_q, ws.pyr_k, ws.pyr_v, ws.map, ws.scale, ws.qs, ws.ks, ws.vs, stream)
         mark(3)
-        lh.attn_fwd(c, ws.qs, ws.ks, ws.vs, ws.os, ws.lse, stream)
+        lh.attn_fwd(c, ws.qs, ws.ks, ws.vs, ws.scale, ws.os, ws.lse, stream)
         mark(4)
         lh.scatter(c, ws.os, ws.slot, o, stream)
         mark(5)
-        lh.scatter_bwd(c, do, ws.os, ws.slot, ws.dos, ws.delta, stream)
+        lh.scatter_bwd(c, do, ws.os, ws.slot, ws.dos, ws.delta, ws.scale, stream)
         mark(6)
-        lh.attn_bwd(c, ws.qs, ws.ks, ws.vs, ws.dos, ws.lse, ws.delta, ws.dqs, ws.dks, ws.dvs, stream)
+        lh.attn_bwd(c, ws.qs, ws.ks, ws.vs, ws.dos, ws.lse, ws.delta, ws.scale, ws.dqs, ws.dks, ws.dvs, stream)
         mark(7)
         lh.spread(c, ws.dqs, ws.dks, ws.dvs, ws.slot, dq, dk, dv, stream)
         mark(8)

@@ -46,7 +46,25 @@
  *                                                         not in it, s = the first slot of
  *                                                         its descendants' run
  *   sub-sequence qs, ks, vs, and dos       [B][H][S][D]   attention operand type: fp16 for
- *                                                         bf16 I/O, fp32 for fp32 I/O
+ *                                                         bf16 I/O (x * 2^-e, e the head's
+ *                                                         exponent from `scale`), fp32 for
+ *                                                         fp32 I/O
+ *   operand scale                          [4][B][H]      uint32: the largest magnitude (fp32
+ *                                                         bit pattern) of the head's queries,
+ *                                                         keys, values (lh_pool) and dO block
+ *                                                         sums (lh_scatter_bwd). The fp16
+ *                                                         operands of bf16 I/O are x * 2^-e,
+ *                                                         e = 0 while that magnitude is in
+ *                                                         [4, 256), else the exponent that
+ *                                                         brings it into [4, 8): a power of
+ *                                                         two moves no significant bit, so
+ *                                                         every bf16 value within 2^19 of its
+ *                                                         head's largest enters exactly (bf16's
+ *                                                         range beyond fp16's 65504 and below
+ *                                                         its 2^-14 included), and the kernels
+ *                                                         take the powers of two out of their
+ *                                                         results. Magnitudes are handled from
+ *                                                         2^-60 to 2^60.
  *   attention out os, grads dqs, dks, dvs  [B][H][S][D]   float
  *   lse, delta                             [B][H][S]      float
  */
@@ -165,6 +183,8 @@ const char* lh_status_string(lh_status s);
 lh_status lh_plan(const lh_config* cfg, lh_plan_t* out);
 
 /* (i) Pyramid pool + squared norms. [LH] §3.1 stage (i), Fig. 2 steps 1-2.
+ * Also writes rows 0-2 (queries, keys, values) of `scale`: each head's largest
+ * token magnitude (pooled means are no larger); for L = 1 only this is done.
  * For levels l = 1..L-1: entry i of pyr_x holds mean of tokens
  * [i p^l, (i+1) p^l), formed in fp64 level by level (each level's sum is the
  * left-to-right sum of its p children's sums) and rounded to nearest-even
@@ -173,9 +193,9 @@ lh_status lh_plan(const lh_config* cfg, lh_plan_t* out);
  * partials combined by a stride-halving tree). Under LH_SCORE_MAXPOOL, sq[0] / sq[1]
  * hold instead the largest such squared norm among the entry's query / key
  * token rows. Nothing is written when L = 1.
- * Inputs q, k, v; outputs pyr_q, pyr_k, pyr_v, sq. */
+ * Inputs q, k, v; outputs pyr_q, pyr_k, pyr_v, sq (may be NULL when L = 1), scale. */
 lh_status lh_pool(const lh_config* cfg, const void* q, const void* k, const void* v,
-                  void* pyr_q, void* pyr_k, void* pyr_v, double* sq, void* stream);
+                  void* pyr_q, void* pyr_k, void* pyr_v, double* sq, uint32_t* scale, void* stream);
 
 /* (ii) Score, top-K descent, ordering. [LH] §3.1 stage (ii), Fig. 2 step 3,
  * Fig. 1 (topological sort into one causal sequence).
@@ -194,22 +214,24 @@ lh_status lh_score_topk(const lh_config* cfg, const double* sq, int32_t* sel, in
 
 /* Dense gather: sub-sequence row j of xs = entry map[j] of x (level 0: the
  * token row of q/k/v; level >= 1: the pyramid row), in the attention operand
- * type: an exact copy for fp32 I/O; for bf16 I/O the value in fp16, rounded to
- * nearest-even, which is exact for every bf16 magnitude in [2^-14, 65504] (a
- * magnitude above 65504 is reported by lh_get_device_error: LH_ERR_DEVICE,
- * detail 102). fp16 gives the attention's P and dS operands 11 significant
- * bits instead of bf16's 8. [LH] Fig. 1 (dense gather); "Lighthouse Attention
- * Technique" (sort, then gather). */
+ * type: an exact copy for fp32 I/O; for bf16 I/O x * 2^-e in fp16 (e from the
+ * head's row of `scale`, written by lh_pool), exact for every bf16 value within
+ * 2^19 of the head's largest (a non-finite value is reported by
+ * lh_get_device_error: LH_ERR_DEVICE, detail 102). fp16 gives the attention's P
+ * and dS operands 11 significant bits instead of bf16's 8. [LH] Fig. 1 (dense
+ * gather); "Lighthouse Attention Technique" (sort, then gather). */
 lh_status lh_gather(const lh_config* cfg, const void* q, const void* k, const void* v,
                     const void* pyr_q, const void* pyr_k, const void* pyr_v, const int32_t* map,
-                    void* qs, void* ks, void* vs, void* stream);
+                    const uint32_t* scale, void* qs, void* ks, void* vs, void* stream);
 
 /* (iii) Causal attention on the sub-sequence, [LH] Eq. (1), scale 1/sqrt(D):
  * os = softmax(qs ks^T / sqrt(D) + causal mask) vs, lse = natural log of each
  * row's softmax denominator. bf16 I/O: tcgen05 tensor cores on the fp16
- * sub-sequence, P as fp16, fp32 accumulate; fp32 I/O: fp32 SIMT. */
+ * sub-sequence, P as fp16, fp32 accumulate; the operands' powers of two (from
+ * `scale`) are taken out of the softmax scale and of os. fp32 I/O: fp32 SIMT
+ * (`scale` unused). */
 lh_status lh_attn_fwd(const lh_config* cfg, const void* qs, const void* ks, const void* vs,
-                      float* os, float* lse, void* stream);
+                      const uint32_t* scale, float* os, float* lse, void* stream);
 
 /* (iv) Scatter back, [LH] §3.1 stage (iv): token t of o receives, for every
  * sub-sequence entry covering t, that entry's row of os (weight 1), summed
@@ -221,20 +243,24 @@ lh_status lh_scatter(const lh_config* cfg, const float* os, const int32_t* slot,
  * sum of dout over the tokens entry j covers (fp32, level by level), stored
  * as the backward operand type (fp16 for bf16 I/O: the block sums of pooled
  * entries need more significand than bf16 has; fp32 for fp32 I/O);
- * delta[j] = sum_d (fp32 block sum)[d] * os[j][d]. A block sum beyond the fp16
- * range is reported by lh_get_device_error (LH_ERR_DEVICE, detail 100). */
+ * delta[j] = sum_d (stored block sum)[d] * os[j][d]. For bf16 I/O the stored
+ * sums are sum * 2^-e with the head's exponent from its largest block sum,
+ * recorded in row 3 of `scale` (a first pass records it; a second redoes the
+ * heads that need e != 0). A non-finite block sum is reported by
+ * lh_get_device_error (LH_ERR_DEVICE, detail 100). */
 lh_status lh_scatter_bwd(const lh_config* cfg, const void* dout, const float* os,
-                         const int32_t* slot, void* dos, float* delta, void* stream);
+                         const int32_t* slot, void* dos, float* delta, uint32_t* scale, void* stream);
 
 /* Backward of (iii): gradients of Eq. (1) with P recomputed from lse:
  * dvs = P^T dos, dP = dos vs^T, dS = P o (dP - delta), dqs = dS ks / sqrt(D),
  * dks = dS^T qs / sqrt(D). Deterministic (no atomics). bf16 I/O: tcgen05
  * kernels on the fp16 sub-sequence and fp16 dos, fp32 accumulate (dS feeding
- * dqs is split into an fp16 head and remainder); fp32 I/O: SIMT kernels. A dS
- * beyond the fp16 range is reported by lh_get_device_error (LH_ERR_DEVICE,
- * detail 101). */
+ * dqs is split into an fp16 head and remainder), the operands' powers of two
+ * (from `scale`) taken out of P, delta and the three results; fp32 I/O: SIMT
+ * kernels. A non-finite dQ or dK (a dS beyond the fp16 range, or non-finite
+ * data) is reported by lh_get_device_error (LH_ERR_DEVICE, detail 101). */
 lh_status lh_attn_bwd(const lh_config* cfg, const void* qs, const void* ks, const void* vs,
-                      const void* dos, const float* lse, const float* delta,
+                      const void* dos, const float* lse, const float* delta, const uint32_t* scale,
                       float* dqs, float* dks, float* dvs, void* stream);
 
 /* Backward of gather + mean-pool ([LH] Fig. 1 gradient path): token t of dx
@@ -254,9 +280,11 @@ lh_status lh_spread(const lh_config* cfg, const float* dqs, const float* dks, co
  * pyramid entries, norms, slot table and sub-sequence rows at their places in
  * the whole problem's buffers; the results equal lh_pool / lh_scatter's for
  * those tokens bit for bit. t0 and nt: multiples of p^(L-1), t0 + nt <= N;
- * L >= 2. Errors as lh_pool / lh_scatter, LH_ERR_SHAPE for a bad range. */
+ * L >= 2. lh_pool_range accumulates the magnitude rows of `scale` over its
+ * calls; the call with t0 == 0 resets them first, so cover a sequence in order
+ * from its start. Errors as lh_pool / lh_scatter, LH_ERR_SHAPE for a bad range. */
 lh_status lh_pool_range(const lh_config* cfg, int t0, int nt, const void* q, const void* k, const void* v,
-                        void* pyr_q, void* pyr_k, void* pyr_v, double* sq, void* stream);
+                        void* pyr_q, void* pyr_k, void* pyr_v, double* sq, uint32_t* scale, void* stream);
 lh_status lh_scatter_range(const lh_config* cfg, int t0, int nt, const float* os, const int32_t* slot, void* o,
                            void* stream);
 
@@ -270,6 +298,7 @@ typedef struct {
   void* ws; size_t ws_bytes;     /* plan.ws_bytes */
   void* dos; float* delta;       /* [B][H][S][D] fp16 (bf16 I/O) or fp32, [B][H][S] */
   float *dqs, *dks, *dvs;        /* [B][H][S][D] */
+  uint32_t* scale;               /* [4][B][H] operand magnitudes (see the layouts above) */
 } lh_buffers;
 
 /* Whole forward: lh_pool, lh_score_topk, lh_gather, lh_attn_fwd, lh_scatter. */
@@ -292,8 +321,10 @@ lh_status lh_backward(const lh_config* cfg, const void* dout, void* dq, void* dk
  * sequence (N = world * n); L >= 2. One step, with the collectives the caller
  * runs between the calls (NCCL over NVLink: the steps are stream-ordered and
  * never wait on another rank):
- *   lh_cp_pool                 shard's pyramid and squared norms sq_loc
- *   all-gather of sq_loc into sq_gathered [world][2][B][H][E_loc]
+ *   lh_cp_pool                 shard's pyramid, squared norms sq_loc and magnitude
+ *                              rows 0-2 of scale
+ *   all-gather of sq_loc into sq_gathered [world][2][B][H][E_loc]; all-reduce
+ *   (max) of rows 0-2 of scale (uint32: the bit patterns order like the values)
  *   lh_cp_assemble_sq          -> sq [2][B][H][E] of the whole sequence
  *   lh_score_topk              the whole selection, map and slot table (the same
  *                              on every rank: every rank runs the same descent)
@@ -310,7 +341,8 @@ lh_status lh_backward(const lh_config* cfg, const void* dout, void* dq, void* dk
  *   lh_cp_scatter              the shard's output tokens
  * Backward:
  *   lh_cp_scatter_bwd          the segment's rows of dos, delta (other rows of
- *                              dos are set to zero)
+ *                              dos are set to zero) and row 3 of scale (this
+ *                              rank's own: dO's exponent may differ per rank)
  *   lh_cp_attn_bwd             dqs for the segment's rows; dks, dvs for ALL rows:
  *                              the contribution of this rank's queries
  *   all-reduce (sum) of dks and of dvs
@@ -330,23 +362,25 @@ typedef struct {
 
 lh_status lh_cp_plan(const lh_config* cfg, int world, int rank, lh_cp_plan_t* out);
 lh_status lh_cp_pool(const lh_config* cfg, int world, int rank, const void* q, const void* k, const void* v,
-                     void* pyr_q, void* pyr_k, void* pyr_v, double* sq_loc, void* stream);
+                     void* pyr_q, void* pyr_k, void* pyr_v, double* sq_loc, uint32_t* scale, void* stream);
 lh_status lh_cp_assemble_sq(const lh_config* cfg, int world, const double* sq_gathered, double* sq,
                             void* stream);
 lh_status lh_cp_segment(const lh_config* cfg, int world, int rank, const int32_t* map, const int32_t* slot,
                         int32_t* slot_loc, int32_t* seg, void* stream);
 lh_status lh_cp_gather(const lh_config* cfg, int world, int rank, const void* q, const void* k, const void* v,
                        const void* pyr_q, const void* pyr_k, const void* pyr_v, const int32_t* map,
-                       const int32_t* seg, void* qs, void* ks, void* vs, void* stream);
+                       const int32_t* seg, const uint32_t* scale, void* qs, void* ks, void* vs, void* stream);
 lh_status lh_cp_attn_fwd(const lh_config* cfg, int world, int rank, const int32_t* seg, const void* qs,
-                         const void* ks, const void* vs, float* os, float* lse, void* stream);
+                         const void* ks, const void* vs, const uint32_t* scale, float* os, float* lse,
+                         void* stream);
 lh_status lh_cp_scatter(const lh_config* cfg, int world, int rank, const float* os, const int32_t* slot_loc,
                         void* o, void* stream);
 lh_status lh_cp_scatter_bwd(const lh_config* cfg, int world, int rank, const void* dout, const float* os,
-                            const int32_t* slot_loc, const int32_t* seg, void* dos, float* delta, void* stream);
+                            const int32_t* slot_loc, const int32_t* seg, void* dos, float* delta, uint32_t* scale,
+                            void* stream);
 lh_status lh_cp_attn_bwd(const lh_config* cfg, int world, int rank, const int32_t* seg, const void* qs,
                          const void* ks, const void* vs, const void* dos, const float* lse, const float* delta,
-                         float* dqs, float* dks, float* dvs, void* stream);
+                         const uint32_t* scale, float* dqs, float* dks, float* dvs, void* stream);
 lh_status lh_cp_spread(const lh_config* cfg, int world, int rank, const float* dqs, const float* dks,
                        const float* dvs, const int32_t* slot_loc, void* dq, void* dk, void* dv, void* stream);
 

@@ -61,6 +61,8 @@ class ShardRank:
         self.slot = z(B, H, E, dtype=i32)
         self.slot_loc = z(B, H, El, dtype=i32)
         self.seg = z(B, H, 2, dtype=i32)
+        # per-head operand magnitudes [4][B][H]: rows 0-2 max-reduced over the ranks
+        self.scale = torch.zeros(4, B, H, dtype=i32, device=device)
         self.ws = z(max(pl.ws_bytes, 16), dtype=torch.uint8)
         self.qs, self.ks, self.vs = (z(B, H, S, D, dtype=f16) for _ in range(3))
         self.os = z(B, H, S, D, dtype=f32)
@@ -75,27 +77,27 @@ class ShardRank:
     # ---- forward
     def pool(self, q, k, v, stream=None):
         lh.cp_pool(self.cfg, self.world, self.rank, q, k, v, self.pyr_q, self.pyr_k, self.pyr_v, self.sq_loc,
-                   stream)
+                   self.scale, stream)
 
     def select_gather(self, sq_gathered, q, k, v, stream=None):
         c, W, r = self.cfg, self.world, self.rank
         lh.cp_assemble_sq(c, W, sq_gathered, self.sq, stream)
         lh.score_topk(c, self.sq, self.sel, self.map, self.slot, self.ws, stream=stream)
         lh.cp_segment(c, W, r, self.map, self.slot, self.slot_loc, self.seg, stream)
-        lh.cp_gather(c, W, r, q, k, v, self.pyr_q, self.pyr_k, self.pyr_v, self.map, self.seg, self.qs, self.ks,
-                     self.vs, stream)
+        lh.cp_gather(c, W, r, q, k, v, self.pyr_q, self.pyr_k, self.pyr_v, self.map, self.seg, self.scale, self.qs,
+                     self.ks, self.vs, stream)
 
     def attend_scatter(self, o, stream=None):
         c, W, r = self.cfg, self.world, self.rank
-        lh.cp_attn_fwd(c, W, r, self.seg, self.qs, self.ks, self.vs, self.os, self.lse, stream)
+        lh.cp_attn_fwd(c, W, r, self.seg, self.qs, self.ks, self.vs, self.scale, self.os, self.lse, stream)
         lh.cp_scatter(c, W, r, self.os, self.slot_loc, o, stream)
 
     # ---- backward
     def attend_bwd(self, do, stream=None):
         c, W, r = self.cfg, self.world, self.rank
-        lh.cp_scatter_bwd(c, W, r, do, self.os, self.slot_loc, self.seg, self.dos, self.delta, stream)
-        lh.cp_attn_bwd(c, W, r, self.seg, self.qs, self.ks, self.vs, self.dos, self.lse, self.delta, self.dqs,
-                       self.dks, self.dvs, stream)
+        lh.cp_scatter_bwd(c, W, r, do, self.os, self.slot_loc, self.seg, self.dos, self.delta, self.scale, stream)
+        lh.cp_attn_bwd(c, W, r, self.seg, self.qs, self.ks, self.vs, self.dos, self.lse, self.delta, self.scale,
+                       self.dqs, self.dks, self.dvs, stream)
 
     def spread(self, dq, dk, dv, stream=None):
         lh.cp_spread(self.cfg, self.world, self.rank, self.dqs, self.dks, self.dvs, self.slot_loc, dq, dk, dv,
@@ -112,6 +114,9 @@ def run_distributed(rank_obj, q, k, v, o, do=None, dq=None, dk=None, dv=None, gr
     shape = st.gathered_shape()
     flat = torch.empty(shape[0] * st.sq_loc.numel(), dtype=st.sq_loc.dtype, device=st.device)
     dist.all_gather_into_tensor(flat, st.sq_loc.reshape(-1), group=group)    # rank-major concatenation
+    # the operands' largest magnitudes over all shards (fp32 bit patterns of
+    # non-negative values order like the values)
+    dist.all_reduce(st.scale[:3], op=dist.ReduceOp.MAX, group=group)
     st.select_gather(flat.view(shape), q, k, v)
     dist.all_reduce(st.ks, group=group)
     dist.all_reduce(st.vs, group=group)
@@ -132,6 +137,9 @@ def run_emulated(ranks, qs, ks, vs, os_, dos=None, dqs=None, dks=None, dvs=None)
     for st, q, k, v in zip(ranks, qs, ks, vs):
         st.pool(q, k, v)
     gathered = torch.stack([st.sq_loc for st in ranks])
+    amax = torch.stack([st.scale[:3] for st in ranks]).amax(dim=0)          # all-reduce (max)
+    for st in ranks:
+        st.scale[:3].copy_(amax)
     for st, q, k, v in zip(ranks, qs, ks, vs):
         st.select_gather(gathered, q, k, v)
 

@@ -82,7 +82,7 @@ template <int D, bool SEG>
 __global__ void __launch_bounds__(kFwdThreads, 1)
 k_attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
               const __grid_constant__ CUtensorMap tv, float* __restrict__ os, float* __restrict__ lse,
-              int S, float c2, const int* __restrict__ seg, int* err) {
+              int S, float c2, const int* __restrict__ seg, const uint32_t* __restrict__ scale, int* err) {
   using Lay = FwdLayout<D>;
   constexpr int SUB = Lay::SUB;
   constexpr uint32_t IDS = idesc_f16(kBM, kBN, false);    // S = Q K^T, both K-major
@@ -108,6 +108,12 @@ k_attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CU
   const int nkvB = hasB ? min((q0 + itB * kBM + kBM - 1) / kBN + 1, nk_end) : 0;
   const int nkv = hasB ? nkvB : nkvA;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // the operands are q * 2^-eq, k * 2^-ek, v * 2^-ev (lh_gather): scores carry
+  // 2^-(eq+ek), taken out in the softmax scale, and O carries 2^-ev
+  const int BH = (int)gridDim.y;
+  const int eq = scale_exp(scale[kScaleQ * BH + bh]), ek = scale_exp(scale[kScaleK * BH + bh]);
+  const int ev = scale_exp(scale[kScaleV * BH + bh]);
+  c2 *= pow2f(eq + ek);
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->q_full, 1);
@@ -347,7 +353,7 @@ k_attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CU
       // only one left: its parity identifies it
       if (ok && __all_sync(0xffffffffu, mbar_wait(&bars->o_done[t], (nk - 1) & 1, ab, err, 8))) {
         tc_fence_after();
-        const float inv = 1.f / l_run;
+        const float inv = pow2f(ev) / l_run;
         float* dst = os + ((size_t)bh * S + q0 + q_row) * D;
 #pragma unroll 1
         for (int c = 0; c < D / 32; ++c) {
@@ -405,7 +411,7 @@ bool make_tmap_16(CUtensorMap* m, const void* base, int D, int S, int BH, bool f
 
 template <int D>
 static cudaError_t fwd_tc_t(const Geom& g, const void* qs, const void* ks, const void* vs, float* os,
-                            float* lse, const int* seg, int* err, cudaStream_t s) {
+                            float* lse, const int* seg, const uint32_t* scale, int* err, cudaStream_t s) {
   CUtensorMap tq, tk, tv;
   const int BH = g.B * g.H;
   if (!make_tmap_16(&tq, qs, D, g.S, BH, true, kBM) || !make_tmap_16(&tk, ks, D, g.S, BH, true, kBN) ||
@@ -418,17 +424,19 @@ static cudaError_t fwd_tc_t(const Geom& g, const void* qs, const void* ks, const
   const float c2 = (float)(1.4426950408889634 / sqrt((double)D));
   const int ntiles = (g.S + kBM - 1) / kBM;
   dim3 grid((ntiles + 1) / 2, BH);
-  kern<<<grid, kFwdThreads, smem, s>>>(tq, tk, tv, os, lse, g.S, c2, seg, err);
+  kern<<<grid, kFwdThreads, smem, s>>>(tq, tk, tv, os, lse, g.S, c2, seg, scale, err);
   count_launch();
   return cudaGetLastError();
 }
 
 // seg: nullptr (every row of the sub-sequence is a query) or [B*H][2] device
 // int32 (first query row, number of query rows) per (b, h).
+// scale: [kScaleRows][B*H] largest magnitudes (the operands' power-of-two exponents).
 cudaError_t launch_attn_fwd_tc(const Geom& g, const void* qs, const void* ks, const void* vs,
-                               float* os, float* lse, const int* seg, int* err, cudaStream_t s) {
-  return g.D == 64 ? fwd_tc_t<64>(g, qs, ks, vs, os, lse, seg, err, s)
-                   : fwd_tc_t<128>(g, qs, ks, vs, os, lse, seg, err, s);
+                               float* os, float* lse, const int* seg, const uint32_t* scale, int* err,
+                               cudaStream_t s) {
+  return g.D == 64 ? fwd_tc_t<64>(g, qs, ks, vs, os, lse, seg, scale, err, s)
+                   : fwd_tc_t<128>(g, qs, ks, vs, os, lse, seg, scale, err, s);
 }
 
 }  // namespace lh

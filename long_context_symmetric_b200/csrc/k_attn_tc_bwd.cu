@@ -404,7 +404,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 k_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
               const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tdo,
               const float* __restrict__ lse, const float* __restrict__ delta, float* __restrict__ dks,
-              float* __restrict__ dvs, int S, float c2, float scale, const int* __restrict__ seg, int* err) {
+              float* __restrict__ dvs, int S, float c2, float scale, const int* __restrict__ seg,
+              const uint32_t* __restrict__ amax, int* err) {
   using Lay = BwdLayout<D>;
   extern __shared__ __align__(16) uint8_t smem_raw[];
   BwdBars* bars = reinterpret_cast<BwdBars*>(smem_raw);
@@ -417,6 +418,13 @@ k_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CU
   const int ntq = (nq + kT - 1) / kT;
   const int i0 = max(0, j * kT - q0) / kT;   // first query tile with a row at or after key row j*128
   const int n = ntq - i0;                    // query tiles i = i0 .. ntq-1
+  // operands q * 2^-eq, k * 2^-ek, v * 2^-ev (lh_gather) and dO * 2^-edo
+  // (lh_scatter_bwd): scores carry 2^-(eq+ek), dP and delta 2^-(edo+ev),
+  // dV 2^-edo, dK 2^-(edo+ev+eq); each is taken out where it is used
+  const int BH = (int)gridDim.y;
+  const int eq = scale_exp(amax[kScaleQ * BH + bh]), ek = scale_exp(amax[kScaleK * BH + bh]);
+  const int ev = scale_exp(amax[kScaleV * BH + bh]), edo = scale_exp(amax[kScaleDO * BH + bh]);
+  c2 *= pow2f(eq + ek);
   if (n <= 0) {
     // no query of this head reaches this key tile: its gradient rows are zero
     const size_t rows = (size_t)min(kT, S - j * kT);
@@ -449,7 +457,7 @@ k_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CU
     // half: column 64*half + (hid & 63)), fetched one tile ahead
     const int hid = ctid & 127;
     const float* vsrc = (hid < 64 ? lse : delta) + (size_t)bh * S;
-    const float vmul = hid < 64 ? -1.4426950408889634f : -1.f;
+    const float vmul = hid < 64 ? -1.4426950408889634f : -pow2f(-(edo + ev));
     auto fetch = [&](int i) -> float {
       const int q = i * kT + 64 * half + (hid & 63);    // within this head's query rows
       return q < nq ? vsrc[q0 + q] : 0.f;
@@ -515,6 +523,7 @@ k_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CU
     }
     if (ok && __all_sync(0xffffffffu, mbar_wait(&bars->done, 0, ab, err, 18))) {
       tc_fence_after();
+      const float mv = pow2f(edo), mk = scale * pow2f(edo + ev + eq);
       float* ddv = dvs + ((size_t)bh * S + key) * D;
       float* ddk = dks + ((size_t)bh * S + key) * D;
 #pragma unroll 1
@@ -533,11 +542,11 @@ k_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CU
 #pragma unroll
           for (int e = 0; e < 32; e += 4) {
             *reinterpret_cast<float4*>(ddv + 32 * c + e) =
-                make_float4(__uint_as_float(a[e]), __uint_as_float(a[e + 1]), __uint_as_float(a[e + 2]),
-                            __uint_as_float(a[e + 3]));
+                make_float4(__uint_as_float(a[e]) * mv, __uint_as_float(a[e + 1]) * mv,
+                            __uint_as_float(a[e + 2]) * mv, __uint_as_float(a[e + 3]) * mv);
             *reinterpret_cast<float4*>(ddk + 32 * c + e) =
-                make_float4(__uint_as_float(b[e]) * scale, __uint_as_float(b[e + 1]) * scale,
-                            __uint_as_float(b[e + 2]) * scale, __uint_as_float(b[e + 3]) * scale);
+                make_float4(__uint_as_float(b[e]) * mk, __uint_as_float(b[e + 1]) * mk,
+                            __uint_as_float(b[e + 2]) * mk, __uint_as_float(b[e + 3]) * mk);
           }
         }
       }
@@ -552,7 +561,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 k_bwd_dq_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tdo,
             const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
             const float* __restrict__ lse, const float* __restrict__ delta, float* __restrict__ dqs,
-            int S, float c2, float scale, const int* __restrict__ seg, int* err) {
+            int S, float c2, float scale, const int* __restrict__ seg, const uint32_t* __restrict__ amax,
+            int* err) {
   using Lay = BwdLayout<D>;
   extern __shared__ __align__(16) uint8_t smem_raw[];
   BwdBars* bars = reinterpret_cast<BwdBars*>(smem_raw);
@@ -565,6 +575,11 @@ k_bwd_dq_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
   if (i < 0) return;                              // whole CTA, before any set-up
   // key tiles up to the one holding the tile's last row, within the keys that exist
   const int n = min((q0 + i * kT + kT - 1) / kT + 1, (q0 + nq + kT - 1) / kT);
+  // operand exponents as in the dK/dV kernel: dQ carries 2^-(edo+ev+ek)
+  const int BH = (int)gridDim.y;
+  const int eq = scale_exp(amax[kScaleQ * BH + bh]), ek = scale_exp(amax[kScaleK * BH + bh]);
+  const int ev = scale_exp(amax[kScaleV * BH + bh]), edo = scale_exp(amax[kScaleDO * BH + bh]);
+  c2 *= pow2f(eq + ek);
   bwd_setup(bars, warp);
   const uint32_t tbase = bars->tmem_base;
   volatile Abort* ab = &bars->abort;
@@ -581,7 +596,7 @@ k_bwd_dq_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
     const uint32_t cX = tbase + la + 64 * half;
     const int q = i * kT + r;                      // within this head's query rows
     const float nl2 = q < nq ? lse[(size_t)bh * S + q0 + q] * -1.4426950408889634f : 0.f;
-    const float ndl = q < nq ? -delta[(size_t)bh * S + q0 + q] : 0.f;
+    const float ndl = q < nq ? -delta[(size_t)bh * S + q0 + q] * pow2f(-(edo + ev)) : 0.f;
     bool ok = true;
     for (int jj = 0; jj < n; ++jj) {
       if (!__all_sync(0xffffffffu, mbar_wait(&bars->x_full, jj & 1, ab, err, 19))) { ok = false; break; }
@@ -623,6 +638,7 @@ k_bwd_dq_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
     if (ok && __all_sync(0xffffffffu, mbar_wait(&bars->done, 0, ab, err, 21))) {
       tc_fence_after();
       float* dst = dqs + ((size_t)bh * S + q0 + q) * D;
+      const float mq = scale * pow2f(edo + ev + ek);
 #pragma unroll 1
       for (int c = half * (D / 64); c < (half + 1) * (D / 64); ++c) {
         uint32_t a[32];
@@ -636,8 +652,8 @@ k_bwd_dq_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
 #pragma unroll
           for (int e = 0; e < 32; e += 4)
             *reinterpret_cast<float4*>(dst + 32 * c + e) =
-                make_float4(__uint_as_float(a[e]) * scale, __uint_as_float(a[e + 1]) * scale,
-                            __uint_as_float(a[e + 2]) * scale, __uint_as_float(a[e + 3]) * scale);
+                make_float4(__uint_as_float(a[e]) * mq, __uint_as_float(a[e + 1]) * mq,
+                            __uint_as_float(a[e + 2]) * mq, __uint_as_float(a[e + 3]) * mq);
         }
       }
     }
@@ -648,7 +664,7 @@ k_bwd_dq_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
 template <int D>
 cudaError_t bwd_tc_t(const Geom& g, const void* qs, const void* ks, const void* vs, const void* dos,
                      const float* lse, const float* delta, float* dqs, float* dks, float* dvs, const int* seg,
-                     int* err, cudaStream_t s) {
+                     const uint32_t* amax, int* err, cudaStream_t s) {
   CUtensorMap tq, tk, tv, tdo;
   const int BH = g.B * g.H;
   if (!make_tmap_16(&tq, qs, D, g.S, BH, true, kT) || !make_tmap_16(&tk, ks, D, g.S, BH, true, kT) ||
@@ -664,11 +680,11 @@ cudaError_t bwd_tc_t(const Geom& g, const void* qs, const void* ks, const void* 
   const float scale = (float)(1.0 / sqrt((double)D));
   const float c2 = (float)(1.4426950408889634 / sqrt((double)D));
   dim3 grid((g.S + kT - 1) / kT, BH);
-  dkdv<<<grid, kThreads, smem, s>>>(tk, tv, tq, tdo, lse, delta, dks, dvs, g.S, c2, scale, seg, err);
+  dkdv<<<grid, kThreads, smem, s>>>(tk, tv, tq, tdo, lse, delta, dks, dvs, g.S, c2, scale, seg, amax, err);
   count_launch();
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  dq<<<grid, kThreads, smem_q, s>>>(tq, tdo, tk, tv, lse, delta, dqs, g.S, c2, scale, seg, err);
+  dq<<<grid, kThreads, smem_q, s>>>(tq, tdo, tk, tv, lse, delta, dqs, g.S, c2, scale, seg, amax, err);
   count_launch();
   return cudaGetLastError();
 }
@@ -681,9 +697,10 @@ cudaError_t bwd_tc_t(const Geom& g, const void* qs, const void* ks, const void* 
 // query reaches), and dqs only the segment's rows.
 cudaError_t launch_attn_bwd_tc(const Geom& g, const void* qs, const void* ks, const void* vs,
                                const void* dos, const float* lse, const float* delta, float* dqs,
-                               float* dks, float* dvs, const int* seg, int* err, cudaStream_t s) {
-  return g.D == 64 ? bwd_tc_t<64>(g, qs, ks, vs, dos, lse, delta, dqs, dks, dvs, seg, err, s)
-                   : bwd_tc_t<128>(g, qs, ks, vs, dos, lse, delta, dqs, dks, dvs, seg, err, s);
+                               float* dks, float* dvs, const int* seg, const uint32_t* amax, int* err,
+                               cudaStream_t s) {
+  return g.D == 64 ? bwd_tc_t<64>(g, qs, ks, vs, dos, lse, delta, dqs, dks, dvs, seg, amax, err, s)
+                   : bwd_tc_t<128>(g, qs, ks, vs, dos, lse, delta, dqs, dks, dvs, seg, amax, err, s);
 }
 
 }  // namespace lh

@@ -108,7 +108,8 @@ __global__ void __launch_bounds__(256) k_cp_gather(const uint4* __restrict__ q, 
                                                    const uint4* __restrict__ v, const uint4* __restrict__ pq,
                                                    const uint4* __restrict__ pk, const uint4* __restrict__ pv,
                                                    const int32_t* __restrict__ map, const int32_t* __restrict__ seg,
-                                                   uint4* __restrict__ qs, uint4* __restrict__ ks,
+                                                   const uint32_t* __restrict__ scale, uint4* __restrict__ qs,
+                                                   uint4* __restrict__ ks,
                                                    uint4* __restrict__ vs, Geom g, CpGeom c, int vin, int vout,
                                                    int* err) {
   const int tensor = blockIdx.z;
@@ -118,6 +119,7 @@ __global__ void __launch_bounds__(256) k_cp_gather(const uint4* __restrict__ q, 
   const int bh = blockIdx.y;
   const int b = bh / g.H, h = bh - b * g.H;
   const int s0 = seg[2 * bh], len = seg[2 * bh + 1];
+  const float mul = TO_F16 ? pow2f(-scale_exp(scale[(size_t)tensor * g.B * g.H + bh])) : 1.f;
   bool big = false;
   const long long total = (long long)g.S * vout;
   for (long long t = blockIdx.x * (long long)blockDim.x + threadIdx.x; t < total;
@@ -136,7 +138,9 @@ __global__ void __launch_bounds__(256) k_cp_gather(const uint4* __restrict__ q, 
         __half2* h2 = reinterpret_cast<__half2*>(&out);
 #pragma unroll
         for (int w = 0; w < 4; ++w) {
-          const float2 f = __bfloat1622float2(b2[w]);
+          float2 f = __bfloat1622float2(b2[w]);
+          f.x *= mul;                 // the head's power-of-two exponent (exact)
+          f.y *= mul;
           big |= !(fabsf(f.x) <= kHalfMax) || !(fabsf(f.y) <= kHalfMax);
           h2[w] = __float22half2_rn(f);
         }
@@ -211,7 +215,8 @@ cudaError_t launch_cp_segment(const Geom& g, int world, int rank, const int32_t*
 
 cudaError_t launch_cp_gather(const Geom& g, lh_dtype dt, int world, int rank, const void* q, const void* k,
                              const void* v, const void* pq, const void* pk, const void* pv, const int32_t* map,
-                             const int32_t* seg, void* qs, void* ks, void* vs, int* err, cudaStream_t s) {
+                             const int32_t* seg, const uint32_t* scale, void* qs, void* ks, void* vs, int* err,
+                             cudaStream_t s) {
   const CpGeom c = make_cp_geom(g, world, rank);
   const int esz = dt == LH_BF16 ? 2 : 4;
   const int vin = g.D * esz / 16;                  // 16-byte vectors per input row
@@ -220,12 +225,12 @@ cudaError_t launch_cp_gather(const Geom& g, lh_dtype dt, int world, int rank, co
   dim3 grid((unsigned)((per + 255) / 256 < 4096 ? (per + 255) / 256 : 4096), (unsigned)(g.B * g.H), 3);
   if (dt == LH_BF16)
     k_cp_gather<true><<<grid, 256, 0, s>>>((const uint4*)q, (const uint4*)k, (const uint4*)v, (const uint4*)pq,
-                                           (const uint4*)pk, (const uint4*)pv, map, seg, (uint4*)qs, (uint4*)ks,
-                                           (uint4*)vs, g, c, vin, vout, err);
+                                           (const uint4*)pk, (const uint4*)pv, map, seg, scale, (uint4*)qs,
+                                           (uint4*)ks, (uint4*)vs, g, c, vin, vout, err);
   else
     k_cp_gather<false><<<grid, 256, 0, s>>>((const uint4*)q, (const uint4*)k, (const uint4*)v, (const uint4*)pq,
-                                            (const uint4*)pk, (const uint4*)pv, map, seg, (uint4*)qs, (uint4*)ks,
-                                            (uint4*)vs, g, c, vin, vout, err);
+                                            (const uint4*)pk, (const uint4*)pv, map, seg, scale, (uint4*)qs,
+                                            (uint4*)ks, (uint4*)vs, g, c, vin, vout, err);
   count_launch();
   return cudaGetLastError();
 }

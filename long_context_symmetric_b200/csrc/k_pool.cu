@@ -68,7 +68,8 @@ template <typename T, int LV, int PP, bool MP>
 __global__ void __launch_bounds__(256, 2) k_pool(const T* __restrict__ q, const T* __restrict__ k,
                                                  const T* __restrict__ v, T* __restrict__ pq,
                                                  T* __restrict__ pk, T* __restrict__ pv,
-                                                 double* __restrict__ sq, PoolArgs a, int* err) {
+                                                 double* __restrict__ sq, uint32_t* __restrict__ scale,
+                                                 PoolArgs a, int* err) {
   extern __shared__ __align__(128) uint8_t smem[];
   const Geom& g = a.g;
   const int C8 = g.D >> 3;
@@ -129,6 +130,7 @@ __global__ void __launch_bounds__(256, 2) k_pool(const T* __restrict__ q, const 
     for (int off = C8 >> 1; off >= 1; off >>= 1) part = __dadd_rn(part, __shfl_xor_sync(wmask, part, off));
     return part;
   };
+  uint32_t amax = 0;                    // bf16 I/O: largest |x| of this thread's components (fp32 bits)
   long long gi1 = (long long)cb * (P / p);   // index of the open level-1 entry
   int c = 0;                            // position of the next token in its level-1 entry
   tc::Abort none{0};
@@ -194,6 +196,7 @@ __global__ void __launch_bounds__(256, 2) k_pool(const T* __restrict__ q, const 
           raw[u] = *reinterpret_cast<const typename Vec8<T>::Raw*>(buf + (size_t)(u0 + u) * row_bytes);
 #pragma unroll
         for (int u = 0; u < PP; ++u) {
+          if constexpr (sizeof(T) == 2) amax = max(amax, absmax8_bf16(raw[u].a));
           double xr[8];
           Vec8<T>::raw_f64(raw[u], xr);
 #pragma unroll
@@ -210,6 +213,7 @@ __global__ void __launch_bounds__(256, 2) k_pool(const T* __restrict__ q, const 
     } else {
       for (int u = 0; u < nt; ++u) {
         typename Vec8<T>::Raw raw = *reinterpret_cast<const typename Vec8<T>::Raw*>(buf + (size_t)u * row_bytes);
+        if constexpr (sizeof(T) == 2) amax = max(amax, absmax8_bf16(raw.a));
         double xr[8];
         Vec8<T>::raw_f64(raw, xr);
         if (c == 0) {
@@ -233,13 +237,58 @@ __global__ void __launch_bounds__(256, 2) k_pool(const T* __restrict__ q, const 
     __syncthreads();                    // every thread is done with this stage
     if (threadIdx.x == 0 && kk + a.ns < nstages) issue(kk + a.ns);
   }
+  if constexpr (sizeof(T) == 2) {
+    // the head's largest magnitude (tokens; pooled means are no larger)
+    for (int off = C8 >> 1; off >= 1; off >>= 1) amax = max(amax, __shfl_xor_sync(wmask, amax, off));
+    if (chunk == 0 && amax) atomicMax(scale + (size_t)tensor * g.B * g.H + (size_t)b * g.H + head, amax);
+  }
+}
+
+// rows [r0, r0 + nr) of the scale buffer ([kScaleRows][B*H]) set to zero
+__global__ void k_scale_zero(uint32_t* __restrict__ scale, int r0, int nr, int bh) {
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < nr * bh; i += gridDim.x * blockDim.x)
+    scale[(size_t)r0 * bh + i] = 0u;
+}
+
+// L = 1 (no pyramid): the largest |x| of each (b, h) of q, k, v over all tokens.
+// grid (token blocks, B*H, 3); each thread walks tokens t = threadIdx.x + ...,
+// reading the head's D components of a token (contiguous), then one atomic
+// per warp.
+__global__ void __launch_bounds__(256) k_absmax_tokens(const uint4* __restrict__ q, const uint4* __restrict__ k,
+                                                       const uint4* __restrict__ v, uint32_t* __restrict__ scale,
+                                                       Geom g) {
+  const int tensor = blockIdx.z;
+  const uint4* x = tensor == 0 ? q : (tensor == 1 ? k : v);
+  const int bh = blockIdx.y, b = bh / g.H, h = bh - b * g.H;
+  const int vpr = g.D / 8;                      // 16-byte vectors of one head row
+  uint32_t m = 0;
+  for (int t = blockIdx.x * blockDim.x + threadIdx.x; t < g.N; t += gridDim.x * blockDim.x) {
+    const uint4* row = x + (((size_t)b * g.N + t) * g.H + h) * vpr;
+    for (int c = 0; c < vpr; ++c) m = max(m, absmax8_bf16(__ldg(row + c)));
+  }
+  m = __reduce_max_sync(0xffffffffu, m);
+  if ((threadIdx.x & 31) == 0 && m) atomicMax(scale + (size_t)tensor * g.B * g.H + bh, m);
 }
 
 template <typename T>
 cudaError_t launch_t(const Geom& g, const void* q, const void* k, const void* v, void* pq,
-                     void* pk, void* pv, double* sq, int cb0, int ncb, int* err, cudaStream_t s) {
+                     void* pk, void* pv, double* sq, uint32_t* scale, int cb0, int ncb, int* err,
+                     cudaStream_t s) {
   const int LV = g.L - 1;
-  if (LV < 1 || ncb <= 0) return cudaSuccess;
+  if (cb0 == 0 && scale) {
+    // the maxima accumulate over the calls that start from the sequence's first block
+    k_scale_zero<<<1, 256, 0, s>>>(scale, kScaleQ, 3, g.B * g.H);
+    count_launch();
+  }
+  if (LV < 1) {
+    if (sizeof(T) == 2 && scale) {
+      dim3 grid((unsigned)((g.N + 255) / 256 < 64 ? (g.N + 255) / 256 : 64), (unsigned)(g.B * g.H), 3);
+      k_absmax_tokens<<<grid, 256, 0, s>>>((const uint4*)q, (const uint4*)k, (const uint4*)v, scale, g);
+      count_launch();
+    }
+    return cudaGetLastError();
+  }
+  if (ncb <= 0) return cudaGetLastError();
   PoolArgs a;
   a.g = g;
   a.cb0 = cb0;
@@ -249,11 +298,12 @@ cudaError_t launch_t(const Geom& g, const void* q, const void* k, const void* v,
     --hg;
     while (g.H % hg) --hg;
   }
+  const int stage_bytes = 32768;
   a.hg = hg;
   a.row_bytes = hg * g.D * (int)sizeof(T);
   const long long P = g.pl[LV];
   int ts = 1;
-  while (ts * 2 * a.row_bytes <= 32768 && ts * 2 <= P) ts *= 2;
+  while (ts * 2 * a.row_bytes <= stage_bytes && ts * 2 <= P) ts *= 2;
   a.ts = ts;
   a.ns = 3;
   const size_t smem = (size_t)a.ns * a.ts * a.row_bytes + a.ns * sizeof(uint64_t);
@@ -268,7 +318,7 @@ cudaError_t launch_t(const Geom& g, const void* q, const void* k, const void* v,
 #define LH_POOL_MP(n, P, M)                                                                             \
   e = cudaFuncSetAttribute(k_pool<T, n, P, M>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem); \
   if (e != cudaSuccess) return e;                                                                       \
-  k_pool<T, n, P, M><<<grid, block, smem, s>>>(tq, tk, tv, tpq, tpk, tpv, sq, a, err);
+  k_pool<T, n, P, M><<<grid, block, smem, s>>>(tq, tk, tv, tpq, tpk, tpv, sq, scale, a, err);
 #define LH_POOL_PP(n, P)                                                                                \
   if (g.score == LH_SCORE_MAXPOOL) { LH_POOL_MP(n, P, true) } else { LH_POOL_MP(n, P, false) }
 #define LH_POOL_CASE(n)                                                                                 \
@@ -289,17 +339,25 @@ cudaError_t launch_t(const Geom& g, const void* q, const void* k, const void* v,
 
 }  // namespace
 
+cudaError_t launch_scale_zero(uint32_t* scale, int r0, int nr, int bh, cudaStream_t s) {
+  k_scale_zero<<<1, 256, 0, s>>>(scale, r0, nr, bh);
+  count_launch();
+  return cudaGetLastError();
+}
+
 cudaError_t launch_pool(const Geom& g, lh_dtype dt, const void* q, const void* k, const void* v,
-                        void* pq, void* pk, void* pv, double* sq, int* err, cudaStream_t s) {
-  return launch_pool_range(g, dt, 0, g.L > 1 ? g.n[g.L - 1] : 0, q, k, v, pq, pk, pv, sq, err, s);
+                        void* pq, void* pk, void* pv, double* sq, uint32_t* scale, int* err, cudaStream_t s) {
+  return launch_pool_range(g, dt, 0, g.L > 1 ? g.n[g.L - 1] : 0, q, k, v, pq, pk, pv, sq, scale, err, s);
 }
 
 // Coarsest blocks [cb0, cb0 + ncb) of every sequence: the tokens
 // [cb0 p^(L-1), (cb0 + ncb) p^(L-1)) and the pyramid entries above them.
+// scale: [kScaleRows][B][H] (rows q, k, v written; zeroed first when cb0 == 0).
 cudaError_t launch_pool_range(const Geom& g, lh_dtype dt, int cb0, int ncb, const void* q, const void* k,
-                              const void* v, void* pq, void* pk, void* pv, double* sq, int* err, cudaStream_t s) {
-  if (dt == LH_BF16) return launch_t<__nv_bfloat16>(g, q, k, v, pq, pk, pv, sq, cb0, ncb, err, s);
-  return launch_t<float>(g, q, k, v, pq, pk, pv, sq, cb0, ncb, err, s);
+                              const void* v, void* pq, void* pk, void* pv, double* sq, uint32_t* scale, int* err,
+                              cudaStream_t s) {
+  if (dt == LH_BF16) return launch_t<__nv_bfloat16>(g, q, k, v, pq, pk, pv, sq, scale, cb0, ncb, err, s);
+  return launch_t<float>(g, q, k, v, pq, pk, pv, sq, scale, cb0, ncb, err, s);
 }
 
 }  // namespace lh

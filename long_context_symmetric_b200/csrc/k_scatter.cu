@@ -129,25 +129,29 @@ __device__ __forceinline__ void chain_sum(const Geom& g, const float* __restrict
   }
 }
 
-// o[b][t][h][:] = sum of os rows covering t. One thread per 8 output components.
-template <typename T, int FIXED>
+// o[b][t][h][:] = sum of os rows covering t (weights 1, or 1/p^l when
+// WEIGHTED), for the tokens t0 .. t0 + nt - 1 of every sequence. One thread per
+// 8 output components, each walking its token's chain of covering entries: the
+// same sums in the same order as k_scatter_tree, with parallelism over tokens
+// (the form a short token range needs).
+template <typename T, int FIXED, bool WEIGHTED>
 __global__ void __launch_bounds__(256) k_scatter(const float* __restrict__ os,
                                                  const int32_t* __restrict__ slot,
-                                                 T* __restrict__ o, Geom g) {
+                                                 T* __restrict__ o, Geom g, int t0, int nt) {
   const int C8 = g.D >> 3;
-  const long long total = (long long)g.B * g.N * g.H * C8;
+  const long long total = (long long)g.B * nt * g.H * C8;
   for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
        i += (long long)gridDim.x * blockDim.x) {
     const int c8 = (int)(i % C8);
-    const long long r = i / C8;                 // (b, t, h) row
+    const long long r = i / C8;                 // (b, t - t0, h) within the range
     const int h = (int)(r % g.H);
     const long long bt = r / g.H;
-    const int t = (int)(bt % g.N);
-    const long long b = bt / g.N;
+    const int t = t0 + (int)(bt % nt);
+    const long long b = bt / nt;
     const long long bh = b * g.H + h;
     Acc<FIXED> acc;
-    chain_sum<FIXED, false>(g, os, slot + bh * g.E, bh, t, c8, acc);
-    store_acc<T, FIXED>(o + r * g.D + c8 * 8, acc);
+    chain_sum<FIXED, WEIGHTED>(g, os, slot + bh * g.E, bh, t, c8, acc);
+    store_acc<T, FIXED>(o + (((size_t)b * g.N + t) * g.H + h) * g.D + c8 * 8, acc);
   }
 }
 
@@ -358,18 +362,23 @@ cudaError_t tree_t(const Geom& g, const float* s0, const float* s1, const float*
 
 // Backward of the scatter: dos[j] = sum of dout over the tokens entry j covers,
 // delta[j] = <dos[j], os[j]> with dos as stored. dos is stored as the backward's operand
-// type TO (fp16 for bf16 I/O: block sums of up to p^(L-1) tokens need more
-// significand than bf16 has; a sum beyond the fp16 range is reported as
-// LH_ERR_DEVICE, detail 100). A thread owns 8 components of one head and
+// type TO: for bf16 I/O fp16 (block sums of up to p^(L-1) tokens need more
+// significand than bf16 has) of the sum times 2^-e, e the head's power-of-two
+// exponent (scale_exp of its largest block-sum magnitude). A first pass
+// (REDO = false) stores with e = 0 and records each head's largest magnitude in
+// the scale buffer; a second launch (REDO = true) redoes, with their exponent,
+// only the heads whose largest magnitude lies outside [4, 256) (its CTAs of
+// other heads leave at once). A non-finite block sum is reported as
+// LH_ERR_DEVICE, detail 100. A thread owns 8 components of one head and
 // walks the tokens of one coarsest block in order; level sums are fp32 and
 // formed level by level (each the left-to-right sum of its p children), so
-// every token row of dout is read exactly once.
-template <typename T, typename TO, int LV>
+// every token row of dout is read exactly once per pass.
+template <typename T, typename TO, int LV, bool REDO>
 __global__ void __launch_bounds__(256) k_blocksum(const T* __restrict__ dout,
                                                   const float* __restrict__ os,
                                                   const int32_t* __restrict__ slot,
                                                   TO* __restrict__ dos, float* __restrict__ delta,
-                                                  Geom g, int hg, int yb, int* err) {
+                                                  uint32_t* __restrict__ amax, Geom g, int hg, int yb, int* err) {
   const int C8 = g.D >> 3;
   const int b = blockIdx.z;
   const int head = blockIdx.y * hg + threadIdx.x / C8;
@@ -377,6 +386,11 @@ __global__ void __launch_bounds__(256) k_blocksum(const T* __restrict__ dout,
   const int cb = blockIdx.x * yb + threadIdx.y;
   const int ncoarse = g.n[g.L - 1];
   const bool live = head < g.H && cb < ncoarse;
+  const int ex = (REDO && sizeof(TO) == 2 && head < g.H)
+                     ? scale_exp(amax[(size_t)kScaleDO * g.B * g.H + (size_t)b * g.H + head]) : 0;
+  if (REDO && __syncthreads_and(ex == 0)) return;       // nothing of this CTA to redo
+  const float mul = pow2f(-ex), unmul = pow2f(ex);
+  uint32_t vmax = 0;                                     // largest |block sum| (fp32 bits), first pass
   const int p = g.p;
   const long long P = g.pl[LV];
   const size_t tok_stride = (size_t)g.H * g.D;
@@ -390,8 +404,16 @@ __global__ void __launch_bounds__(256) k_blocksum(const T* __restrict__ dout,
     float v[8];
 #pragma unroll
     for (int d = 0; d < 8; ++d) v[d] = v0[d] * scale;
+    float mx = 0.f;
+#pragma unroll
+    for (int d = 0; d < 8; ++d) mx = fmaxf(mx, fabsf(v[d]));
+    if (sizeof(TO) == 2) {
+#pragma unroll
+      for (int d = 0; d < 8; ++d) v[d] *= mul;         // a power of two: exact
+    }
     float part = 0.f;
     float ov[8];
+    if (s >= 0 && !LH_BOUNDS(s < g.S, err, 303)) s = -1;
     if (live && s >= 0) {
       load8_f32(os + ((size_t)bh * g.S + s) * g.D + chunk * 8, ov);
       // delta from the stored (rounded) dos: the values the backward's dP uses
@@ -402,11 +424,11 @@ __global__ void __launch_bounds__(256) k_blocksum(const T* __restrict__ dout,
     for (int off = C8 >> 1; off >= 1; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
     if (live && s >= 0) {
       Vec8<TO>::store_f32(dos + ((size_t)bh * g.S + s) * g.D + chunk * 8, v);
-      if (chunk == 0) delta[(size_t)bh * g.S + s] = part;
-      float mx = 0.f;
-#pragma unroll
-      for (int d = 0; d < 8; ++d) mx = fmaxf(mx, fabsf(v[d]));
-      if (sizeof(TO) == 2 && !(mx <= kHalfMax)) report_error(err, LH_ERR_DEVICE, 100);
+      if (chunk == 0) delta[(size_t)bh * g.S + s] = part * unmul;
+      if (sizeof(TO) == 2) {
+        if (!(mx < INFINITY)) report_error(err, LH_ERR_DEVICE, 100);
+        if (!REDO) vmax = max(vmax, __float_as_uint(mx));
+      }
     }
   };
 
@@ -472,6 +494,10 @@ __global__ void __launch_bounds__(256) k_blocksum(const T* __restrict__ dout,
       if (__any_sync(0xffffffffu, in)) emit(in ? (e >> 1) : -1, acc[l], wl[l]);
     }
   }
+  if (!REDO && sizeof(TO) == 2) {
+    for (int off = C8 >> 1; off >= 1; off >>= 1) vmax = max(vmax, __shfl_xor_sync(0xffffffffu, vmax, off));
+    if (live && chunk == 0 && vmax) atomicMax(amax + (size_t)kScaleDO * g.B * g.H + bh, vmax);
+  }
 }
 
 // (Token slots: the p tokens of an expanded level-1 entry sit right before its
@@ -495,12 +521,13 @@ __device__ __forceinline__ void bs_bulk_load(void* dst, const void* src, uint32_
                : "memory");
 }
 
-template <typename T, typename TO, int LV, int PP>
+template <typename T, typename TO, int LV, int PP, bool REDO>
 __global__ void __launch_bounds__(256, 2) k_blocksum_ring(const T* __restrict__ dout,
                                                           const float* __restrict__ os,
                                                           const int32_t* __restrict__ slot,
                                                           TO* __restrict__ dos, float* __restrict__ delta,
-                                                          Geom g, RingArgs a, int* err) {
+                                                          uint32_t* __restrict__ amax, Geom g, RingArgs a,
+                                                          int* err) {
   extern __shared__ __align__(128) uint8_t smem[];
   const int C8 = g.D >> 3;
   const int b = blockIdx.z;
@@ -514,6 +541,11 @@ __global__ void __launch_bounds__(256, 2) k_blocksum_ring(const T* __restrict__ 
   const long long bh = (long long)b * g.H + head;
   const T* src0 = dout + ((size_t)b * g.N + (size_t)cb * P) * tok_stride + (size_t)hg0 * g.D;
   const int32_t* slot_h = slot + bh * g.E;
+  // the head's power-of-two exponent (second pass only; see k_blocksum)
+  const int ex = (REDO && sizeof(TO) == 2) ? scale_exp(amax[(size_t)kScaleDO * g.B * g.H + bh]) : 0;
+  if (REDO && __syncthreads_and(ex == 0)) return;       // nothing of this CTA to redo
+  const float mul = pow2f(-ex), unmul = pow2f(ex);
+  uint32_t vmax = 0;
   const int row_bytes = a.row_bytes;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + (size_t)a.ns * a.ts * row_bytes);
   const int nstages = (int)((P + a.ts - 1) / a.ts);
@@ -546,8 +578,16 @@ __global__ void __launch_bounds__(256, 2) k_blocksum_ring(const T* __restrict__ 
     float v[8];
 #pragma unroll
     for (int d = 0; d < 8; ++d) v[d] = v0[d] * scale;
+    float mx = 0.f;
+#pragma unroll
+    for (int d = 0; d < 8; ++d) mx = fmaxf(mx, fabsf(v[d]));
+    if (sizeof(TO) == 2) {
+#pragma unroll
+      for (int d = 0; d < 8; ++d) v[d] *= mul;         // a power of two: exact
+    }
     float part = 0.f;
     float ov[8];
+    if (s >= 0 && !LH_BOUNDS(s < g.S, err, 303)) s = -1;
     if (s >= 0) {
       if (ov_pre) {
 #pragma unroll
@@ -563,11 +603,11 @@ __global__ void __launch_bounds__(256, 2) k_blocksum_ring(const T* __restrict__ 
     for (int off = C8 >> 1; off >= 1; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
     if (s >= 0) {
       Vec8<TO>::store_f32(dos + ((size_t)bh * g.S + s) * g.D + chunk * 8, v);
-      if (chunk == 0) delta[(size_t)bh * g.S + s] = part;
-      float mx = 0.f;
-#pragma unroll
-      for (int d = 0; d < 8; ++d) mx = fmaxf(mx, fabsf(v[d]));
-      if (sizeof(TO) == 2 && !(mx <= kHalfMax)) report_error(err, LH_ERR_DEVICE, 100);
+      if (chunk == 0) delta[(size_t)bh * g.S + s] = part * unmul;
+      if (sizeof(TO) == 2) {
+        if (!(mx < INFINITY)) report_error(err, LH_ERR_DEVICE, 100);
+        if (!REDO) vmax = max(vmax, __float_as_uint(mx));
+      }
     }
   };
 
@@ -591,13 +631,14 @@ __global__ void __launch_bounds__(256, 2) k_blocksum_ring(const T* __restrict__ 
       if (i1 + 1 < i1_end) e1n = __ldg(slot_h + g.off[1] + (int)(i1 + 1));
       // the level-1 entry's os row, loaded now so that its latency overlaps the sums
       float ov1[8];
-      const bool in1 = slot_in(e1, g);
+      const bool in1 = slot_in(e1, g) && LH_BOUNDS((e1 >> 1) < g.S, err, 303);
       if (in1) load8_f32(os + ((size_t)bh * g.S + (e1 >> 1)) * g.D + chunk * 8, ov1);
       typename Vec8<T>::Raw raw[p];
 #pragma unroll
       for (int u = 0; u < p; ++u)
         raw[u] = *reinterpret_cast<const typename Vec8<T>::Raw*>(buf + (size_t)(u0 + u) * row_bytes);
-      const bool tok_in = e1 >= 0 && (e1 & 1);               // children (tokens) included
+      const bool tok_in = e1 >= 0 && (e1 & 1) &&              // children (tokens) included
+                          LH_BOUNDS(slot_tokens(e1, g) >= 0 && slot_tokens(e1, g) + p <= g.S, err, 303);
       // tokens are emitted only where some lane of the warp has them included
       const bool any_tok = __any_sync(0xffffffffu, tok_in);
       float sum[8];
@@ -647,31 +688,63 @@ __global__ void __launch_bounds__(256, 2) k_blocksum_ring(const T* __restrict__ 
     __syncthreads();                    // every thread is done with this stage
     if (threadIdx.x == 0 && kk + a.ns < nstages) issue(kk + a.ns);
   }
+  if (!REDO && sizeof(TO) == 2) {
+    for (int off = C8 >> 1; off >= 1; off >>= 1) vmax = max(vmax, __shfl_xor_sync(0xffffffffu, vmax, off));
+    if (chunk == 0 && vmax) atomicMax(amax + (size_t)kScaleDO * g.B * g.H + bh, vmax);
+  }
 }
 
-// L == 1: dos = dout transposed to [B][H][N][D]; delta = <dout, os>.
-template <typename T, typename TO>
+// L == 1: dos = dout transposed to [B][H][N][D] (times the head's 2^-e, two
+// passes as k_blocksum); delta = <dout, os>.
+template <typename T, typename TO, bool REDO>
 __global__ void __launch_bounds__(256) k_blocksum_l1(const T* __restrict__ dout,
                                                      const float* __restrict__ os,
                                                      TO* __restrict__ dos, float* __restrict__ delta,
-                                                     Geom g) {
+                                                     uint32_t* __restrict__ amax, Geom g) {
   const int C8 = g.D >> 3;
   const long long total = (long long)g.B * g.H * g.N * C8;
-  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
-       i += (long long)gridDim.x * blockDim.x) {
-    const int c8 = (int)(i % C8);
-    const long long r = i / C8;          // (b, h, t) row of dos
+  const size_t row_do = (size_t)kScaleDO * g.B * g.H;
+  const long long stride = (long long)gridDim.x * blockDim.x;
+  // every lane of a warp takes every iteration (the shuffles below need them
+  // all); lanes past the end or with nothing to redo only skip the memory work
+  for (long long base = (long long)blockIdx.x * blockDim.x; base < total; base += stride) {
+    const long long i = base + threadIdx.x;
+    const bool in = i < total;
+    const long long ii = in ? i : total - 1;
+    const int c8 = (int)(ii % C8);
+    const long long r = ii / C8;         // (b, h, t) row of dos
     const int t = (int)(r % g.N);
     const long long bh = r / g.N;
     const int h = (int)(bh % g.H);
     const long long b = bh / g.H;
+    const int ex = (REDO && sizeof(TO) == 2) ? scale_exp(amax[row_do + bh]) : 0;
+    const bool work = in && !(REDO && ex == 0);
     float x[8], ov[8];
-    Vec8<T>::load_f32(dout + ((b * g.N + t) * g.H + h) * g.D + c8 * 8, x);
-    load8_f32(os + r * g.D + c8 * 8, ov);
+    if (work) {
+      Vec8<T>::load_f32(dout + ((b * g.N + t) * g.H + h) * g.D + c8 * 8, x);
+      load8_f32(os + r * g.D + c8 * 8, ov);
+    } else {
+#pragma unroll
+      for (int d = 0; d < 8; ++d) x[d] = ov[d] = 0.f;
+    }
     float part = 0.f;
 #pragma unroll
     for (int d = 0; d < 8; ++d) part = fmaf(x[d], ov[d], part);
     for (int off = C8 >> 1; off >= 1; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
+    if (sizeof(TO) == 2 && !REDO) {
+      // the row's largest magnitude (its C8 lanes), one atomic per row
+      float mx = 0.f;
+#pragma unroll
+      for (int d = 0; d < 8; ++d) mx = fmaxf(mx, fabsf(x[d]));
+      for (int off = C8 >> 1; off >= 1; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+      if (work && c8 == 0 && mx > 0.f) atomicMax(amax + row_do + bh, __float_as_uint(mx));
+    }
+    if (!work) continue;
+    if (sizeof(TO) == 2) {
+      const float mul = pow2f(-ex);
+#pragma unroll
+      for (int d = 0; d < 8; ++d) x[d] *= mul;
+    }
     Vec8<TO>::store_f32(dos + r * g.D + c8 * 8, x);
     if (c8 == 0) delta[r] = part;
   }
@@ -698,9 +771,28 @@ cudaError_t scatter_t(const Geom& g, const float* os, const int32_t* slot, void*
   }
   const long long total = (long long)g.B * g.N * g.H * (g.D / 8);
   if (g.accum == LH_ACC_FIXED64)
-    k_scatter<T, 1><<<grid_for(total), 256, 0, s>>>(os, slot, (T*)o, g);
+    k_scatter<T, 1, false><<<grid_for(total), 256, 0, s>>>(os, slot, (T*)o, g, 0, g.N);
   else
-    k_scatter<T, 0><<<grid_for(total), 256, 0, s>>>(os, slot, (T*)o, g);
+    k_scatter<T, 0, false><<<grid_for(total), 256, 0, s>>>(os, slot, (T*)o, g, 0, g.N);
+  count_launch();
+  return cudaGetLastError();
+}
+
+// A token range: the per-token chain walk (many threads even for a few
+// coarsest blocks), bit-identical to the tree walk of the whole sequence.
+template <typename T>
+cudaError_t scatter_tokens_t(const Geom& g, const float* os, const int32_t* slot, void* o, int t0, int nt,
+                             cudaStream_t s) {
+  const long long total = (long long)g.B * nt * g.H * (g.D / 8);
+  if (total <= 0) return cudaSuccess;
+  const bool w = g.weight == LH_WEIGHT_MEAN;
+  if (g.accum == LH_ACC_FIXED64) {
+    if (w) k_scatter<T, 1, true><<<grid_for(total), 256, 0, s>>>(os, slot, (T*)o, g, t0, nt);
+    else k_scatter<T, 1, false><<<grid_for(total), 256, 0, s>>>(os, slot, (T*)o, g, t0, nt);
+  } else {
+    if (w) k_scatter<T, 0, true><<<grid_for(total), 256, 0, s>>>(os, slot, (T*)o, g, t0, nt);
+    else k_scatter<T, 0, false><<<grid_for(total), 256, 0, s>>>(os, slot, (T*)o, g, t0, nt);
+  }
   count_launch();
   return cudaGetLastError();
 }
@@ -722,13 +814,13 @@ cudaError_t spread_t(const Geom& g, const float* dqs, const float* dks, const fl
   return cudaGetLastError();
 }
 
-template <typename T>
-cudaError_t blocksum_t(const Geom& g, const void* dout, const float* os, const int32_t* slot,
-                       void* dos, float* delta, int* err, cudaStream_t s) {
+template <typename T, bool REDO>
+cudaError_t blocksum_pass(const Geom& g, const void* dout, const float* os, const int32_t* slot,
+                          void* dos, float* delta, uint32_t* amax, int* err, cudaStream_t s) {
   using TO = typename BwdOperand<T>::type;
   if (g.L == 1) {
     const long long total = (long long)g.B * g.H * g.N * (g.D / 8);
-    k_blocksum_l1<T, TO><<<grid_for(total), 256, 0, s>>>((const T*)dout, os, (TO*)dos, delta, g);
+    k_blocksum_l1<T, TO, REDO><<<grid_for(total), 256, 0, s>>>((const T*)dout, os, (TO*)dos, delta, amax, g);
     count_launch();
     return cudaGetLastError();
   }
@@ -756,10 +848,10 @@ cudaError_t blocksum_t(const Geom& g, const void* dout, const float* os, const i
       TO* o = (TO*)dos;
       cudaError_t e = cudaSuccess;
 #define LH_BSR(n, P)                                                                                     \
-  e = cudaFuncSetAttribute(k_blocksum_ring<T, TO, n, P>, cudaFuncAttributeMaxDynamicSharedMemorySize,    \
+  e = cudaFuncSetAttribute(k_blocksum_ring<T, TO, n, P, REDO>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
                            (int)smem);                                                                   \
   if (e != cudaSuccess) return e;                                                                        \
-  k_blocksum_ring<T, TO, n, P><<<rgrid, hg * C8, smem, s>>>(d, os, slot, o, delta, g, a, err);
+  k_blocksum_ring<T, TO, n, P, REDO><<<rgrid, hg * C8, smem, s>>>(d, os, slot, o, delta, amax, g, a, err);
 #define LH_BSR_CASE(n)                                                                                   \
     case n:                                                                                              \
       if (g.p == 8) { LH_BSR(n, 8) } else if (g.p == 4) { LH_BSR(n, 4) } else { LH_BSR(n, 2) }          \
@@ -783,7 +875,7 @@ cudaError_t blocksum_t(const Geom& g, const void* dout, const float* os, const i
   TO* o = (TO*)dos;
   switch (g.L - 1) {
 #define LH_BS_CASE(n) \
-    case n: k_blocksum<T, TO, n><<<grid, block, 0, s>>>(d, os, slot, o, delta, g, hg, yb, err); break;
+    case n: k_blocksum<T, TO, n, REDO><<<grid, block, 0, s>>>(d, os, slot, o, delta, amax, g, hg, yb, err); break;
     LH_BS_CASE(1) LH_BS_CASE(2) LH_BS_CASE(3) LH_BS_CASE(4)
     LH_BS_CASE(5) LH_BS_CASE(6) LH_BS_CASE(7)
 #undef LH_BS_CASE
@@ -791,6 +883,23 @@ cudaError_t blocksum_t(const Geom& g, const void* dout, const float* os, const i
   }
   count_launch();
   return cudaGetLastError();
+}
+
+// bf16 I/O: the dO row of the scale buffer is zeroed, the first pass stores the
+// block sums unscaled and records each head's largest magnitude, the second
+// redoes the heads whose magnitude needs a power-of-two exponent. fp32 I/O:
+// one pass, no scaling.
+template <typename T>
+cudaError_t blocksum_t(const Geom& g, const void* dout, const float* os, const int32_t* slot,
+                       void* dos, float* delta, uint32_t* amax, int* err, cudaStream_t s) {
+  constexpr bool F16 = sizeof(typename BwdOperand<T>::type) == 2;
+  if (F16) {
+    cudaError_t e = launch_scale_zero(amax, kScaleDO, 1, g.B * g.H, s);
+    if (e != cudaSuccess) return e;
+  }
+  cudaError_t e = blocksum_pass<T, false>(g, dout, os, slot, dos, delta, amax, err, s);
+  if (e != cudaSuccess || !F16) return e;
+  return blocksum_pass<T, true>(g, dout, os, slot, dos, delta, amax, err, s);
 }
 
 }  // namespace
@@ -801,10 +910,17 @@ cudaError_t launch_scatter(const Geom& g, lh_dtype dt, const float* os, const in
                        : scatter_t<float>(g, os, slot, o, s);
 }
 
-// Tokens of the coarsest blocks [cb0, cb0 + ncb) only (L >= 2).
+// Tokens of the coarsest blocks [cb0, cb0 + ncb) only (L >= 2). Ranges of
+// fewer blocks than the GPU has SMs run the per-token walk; longer ones the
+// tree walk of the whole sequence restricted to their blocks.
 cudaError_t launch_scatter_range(const Geom& g, lh_dtype dt, int cb0, int ncb, const float* os,
                                  const int32_t* slot, void* o, cudaStream_t s) {
   if (g.L < 2) return cudaErrorInvalidValue;
+  if (ncb * (long long)g.B < 148) {
+    const int P = (int)g.pl[g.L - 1];
+    return dt == LH_BF16 ? scatter_tokens_t<__nv_bfloat16>(g, os, slot, o, cb0 * P, ncb * P, s)
+                         : scatter_tokens_t<float>(g, os, slot, o, cb0 * P, ncb * P, s);
+  }
   return dt == LH_BF16 ? scatter_t<__nv_bfloat16>(g, os, slot, o, s, cb0, ncb)
                        : scatter_t<float>(g, os, slot, o, s, cb0, ncb);
 }
@@ -817,9 +933,10 @@ cudaError_t launch_spread(const Geom& g, lh_dtype dt, const float* dqs, const fl
 }
 
 cudaError_t launch_scatter_bwd(const Geom& g, lh_dtype dt, const void* dout, const float* os,
-                               const int32_t* slot, void* dos, float* delta, int* err, cudaStream_t s) {
-  return dt == LH_BF16 ? blocksum_t<__nv_bfloat16>(g, dout, os, slot, dos, delta, err, s)
-                       : blocksum_t<float>(g, dout, os, slot, dos, delta, err, s);
+                               const int32_t* slot, void* dos, float* delta, uint32_t* scale, int* err,
+                               cudaStream_t s) {
+  return dt == LH_BF16 ? blocksum_t<__nv_bfloat16>(g, dout, os, slot, dos, delta, scale, err, s)
+                       : blocksum_t<float>(g, dout, os, slot, dos, delta, scale, err, s);
 }
 
 }  // namespace lh

@@ -9,7 +9,25 @@
 
 #include "lh_common.cuh"
 
+#ifndef LH_NO_NVTX
+#include <nvtx3/nvToolsExt.h>
+#endif
+
 namespace lh {
+
+// NVTX range over one entry point (named like the entry point), so a profiler
+// timeline shows each step of the path with the kernels it launched. The
+// header-only NVTX costs a branch when no tool is attached; building with
+// -DLH_NO_NVTX removes it.
+struct NvtxRange {
+#ifndef LH_NO_NVTX
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+#else
+  explicit NvtxRange(const char*) {}
+#endif
+};
+#define LH_RANGE(name) ::lh::NvtxRange lh_nvtx_range_(name)
 
 // Device error word: [0] = lh_status, [1] = kernel-specific detail. Kernels with
 // bounded waits write it (first writer wins) instead of trapping.
@@ -26,7 +44,8 @@ cudaError_t launch_attn_bwd_simt(const Geom& g, lh_dtype dt, const void* qs, con
                                  cudaStream_t s);
 
 cudaError_t launch_attn_fwd_tc(const Geom& g, const void* qs, const void* ks, const void* vs,
-                               float* os, float* lse, const int* seg, int* err, cudaStream_t s);
+                               float* os, float* lse, const int* seg, const uint32_t* scale, int* err,
+                               cudaStream_t s);
 
 // bf16 I/O runs on the tcgen05 tensor-core kernels (fp16 operands); fp32 on
 // the fp32 SIMT kernels. LH_ATTN_SIMT=1 in the environment routes bf16 I/O
@@ -37,22 +56,24 @@ static bool force_simt() {
 }
 
 cudaError_t launch_attn_fwd(const Geom& g, lh_dtype dt, const void* qs, const void* ks,
-                            const void* vs, float* os, float* lse, int* err, cudaStream_t s) {
-  if (dt == LH_BF16 && !force_simt()) return launch_attn_fwd_tc(g, qs, ks, vs, os, lse, nullptr, err, s);
+                            const void* vs, float* os, float* lse, const uint32_t* scale, int* err,
+                            cudaStream_t s) {
+  if (dt == LH_BF16 && !force_simt()) return launch_attn_fwd_tc(g, qs, ks, vs, os, lse, nullptr, scale, err, s);
   return launch_attn_fwd_simt(g, dt, qs, ks, vs, os, lse, s);
 }
 
 cudaError_t launch_attn_bwd_tc(const Geom& g, const void* qs, const void* ks, const void* vs,
                                const void* dos, const float* lse, const float* delta, float* dqs,
-                               float* dks, float* dvs, const int* seg, int* err, cudaStream_t s);
+                               float* dks, float* dvs, const int* seg, const uint32_t* amax, int* err,
+                               cudaStream_t s);
 cudaError_t launch_selftest_wait(long long limit_cycles, int* err, int* gave_up, cudaStream_t s);
 cudaError_t launch_selftest_exp2(const float* x, float* y_fma, float* y_sfu, int n, cudaStream_t s);
 
 cudaError_t launch_attn_bwd(const Geom& g, lh_dtype dt, const void* qs, const void* ks,
                             const void* vs, const void* dos, const float* lse, const float* delta,
-                            float* dqs, float* dks, float* dvs, int* err, cudaStream_t s) {
+                            const uint32_t* scale, float* dqs, float* dks, float* dvs, int* err, cudaStream_t s) {
   if (dt == LH_BF16 && !force_simt())
-    return launch_attn_bwd_tc(g, qs, ks, vs, dos, lse, delta, dqs, dks, dvs, nullptr, err, s);
+    return launch_attn_bwd_tc(g, qs, ks, vs, dos, lse, delta, dqs, dks, dvs, nullptr, scale, err, s);
   return launch_attn_bwd_simt(g, dt, qs, ks, vs, dos, lse, delta, dqs, dks, dvs, s);
 }
 
@@ -155,7 +176,8 @@ cudaError_t launch_cp_segment(const Geom& g, int world, int rank, const int32_t*
                               int32_t* slot_loc, int32_t* seg, cudaStream_t s);
 cudaError_t launch_cp_gather(const Geom& g, lh_dtype dt, int world, int rank, const void* q, const void* k,
                              const void* v, const void* pq, const void* pk, const void* pv, const int32_t* map,
-                             const int32_t* seg, void* qs, void* ks, void* vs, int* err, cudaStream_t s);
+                             const int32_t* seg, const uint32_t* scale, void* qs, void* ks, void* vs, int* err,
+                             cudaStream_t s);
 cudaError_t launch_cp_zero_outside(const Geom& g, int elem_bytes, void* x, const int32_t* seg, cudaStream_t s);
 Geom shard_geom(const Geom& g, int world, int rank);
 
@@ -206,20 +228,21 @@ lh_status lh_plan(const lh_config* cfg, lh_plan_t* out) {
 }
 
 lh_status lh_pool(const lh_config* cfg, const void* q, const void* k, const void* v, void* pyr_q,
-                  void* pyr_k, void* pyr_v, double* sq, void* stream) {
+                  void* pyr_k, void* pyr_v, double* sq, uint32_t* scale, void* stream) {
+  LH_RANGE("lh_pool");
   Geom g;
   lh_status st = make_geom(cfg, &g, nullptr);
   if (st != LH_OK) return st;
-  LH_REQ(q); LH_REQ(k); LH_REQ(v);
-  if (g.L == 1) return LH_OK;
-  LH_REQ(pyr_q); LH_REQ(pyr_k); LH_REQ(pyr_v); LH_REQ(sq);
-  LH_CUDA(launch_pool(g, cfg->dtype, q, k, v, pyr_q, pyr_k, pyr_v, sq, device_error_ptr(),
+  LH_REQ(q); LH_REQ(k); LH_REQ(v); LH_REQ(scale);
+  if (g.L > 1) { LH_REQ(pyr_q); LH_REQ(pyr_k); LH_REQ(pyr_v); LH_REQ(sq); }
+  LH_CUDA(launch_pool(g, cfg->dtype, q, k, v, pyr_q, pyr_k, pyr_v, sq, scale, device_error_ptr(),
                       (cudaStream_t)stream));
   return LH_OK;
 }
 
 lh_status lh_score_topk(const lh_config* cfg, const double* sq, int32_t* sel, int32_t* map,
                         int32_t* slot, void* ws, size_t ws_bytes, void* stream) {
+  LH_RANGE("lh_score_topk");
   Geom g;
   lh_plan_t pl;
   lh_status st = make_geom(cfg, &g, &pl);
@@ -235,30 +258,33 @@ lh_status lh_score_topk(const lh_config* cfg, const double* sq, int32_t* sel, in
 
 lh_status lh_gather(const lh_config* cfg, const void* q, const void* k, const void* v,
                     const void* pyr_q, const void* pyr_k, const void* pyr_v, const int32_t* map,
-                    void* qs, void* ks, void* vs, void* stream) {
+                    const uint32_t* scale, void* qs, void* ks, void* vs, void* stream) {
+  LH_RANGE("lh_gather");
   Geom g;
   lh_status st = make_geom(cfg, &g, nullptr);
   if (st != LH_OK) return st;
-  LH_REQ(q); LH_REQ(k); LH_REQ(v); LH_REQ(map); LH_REQ(qs); LH_REQ(ks); LH_REQ(vs);
+  LH_REQ(q); LH_REQ(k); LH_REQ(v); LH_REQ(map); LH_REQ(scale); LH_REQ(qs); LH_REQ(ks); LH_REQ(vs);
   if (g.L > 1) { LH_REQ(pyr_q); LH_REQ(pyr_k); LH_REQ(pyr_v); }
-  LH_CUDA(launch_gather(g, cfg->dtype, q, k, v, pyr_q, pyr_k, pyr_v, map, qs, ks, vs,
+  LH_CUDA(launch_gather(g, cfg->dtype, q, k, v, pyr_q, pyr_k, pyr_v, map, scale, qs, ks, vs,
                         device_error_ptr(), (cudaStream_t)stream));
   return LH_OK;
 }
 
 lh_status lh_attn_fwd(const lh_config* cfg, const void* qs, const void* ks, const void* vs,
-                      float* os, float* lse, void* stream) {
+                      const uint32_t* scale, float* os, float* lse, void* stream) {
+  LH_RANGE("lh_attn_fwd");
   Geom g;
   lh_status st = make_geom(cfg, &g, nullptr);
   if (st != LH_OK) return st;
-  LH_REQ(qs); LH_REQ(ks); LH_REQ(vs); LH_REQ(os); LH_REQ(lse);
-  LH_CUDA(launch_attn_fwd(g, cfg->dtype, qs, ks, vs, os, lse, device_error_ptr(),
+  LH_REQ(qs); LH_REQ(ks); LH_REQ(vs); LH_REQ(scale); LH_REQ(os); LH_REQ(lse);
+  LH_CUDA(launch_attn_fwd(g, cfg->dtype, qs, ks, vs, os, lse, scale, device_error_ptr(),
                           (cudaStream_t)stream));
   return LH_OK;
 }
 
 lh_status lh_scatter(const lh_config* cfg, const float* os, const int32_t* slot, void* o,
                      void* stream) {
+  LH_RANGE("lh_scatter");
   Geom g;
   lh_status st = make_geom(cfg, &g, nullptr);
   if (st != LH_OK) return st;
@@ -269,32 +295,35 @@ lh_status lh_scatter(const lh_config* cfg, const float* os, const int32_t* slot,
 }
 
 lh_status lh_scatter_bwd(const lh_config* cfg, const void* dout, const float* os,
-                         const int32_t* slot, void* dos, float* delta, void* stream) {
+                         const int32_t* slot, void* dos, float* delta, uint32_t* scale, void* stream) {
+  LH_RANGE("lh_scatter_bwd");
   Geom g;
   lh_status st = make_geom(cfg, &g, nullptr);
   if (st != LH_OK) return st;
-  LH_REQ(dout); LH_REQ(os); LH_REQ(dos); LH_REQ(delta);
+  LH_REQ(dout); LH_REQ(os); LH_REQ(dos); LH_REQ(delta); LH_REQ(scale);
   if (g.L > 1) LH_REQ(slot);
-  LH_CUDA(launch_scatter_bwd(g, cfg->dtype, dout, os, slot, dos, delta, device_error_ptr(),
+  LH_CUDA(launch_scatter_bwd(g, cfg->dtype, dout, os, slot, dos, delta, scale, device_error_ptr(),
                              (cudaStream_t)stream));
   return LH_OK;
 }
 
 lh_status lh_attn_bwd(const lh_config* cfg, const void* qs, const void* ks, const void* vs,
-                      const void* dos, const float* lse, const float* delta, float* dqs,
-                      float* dks, float* dvs, void* stream) {
+                      const void* dos, const float* lse, const float* delta, const uint32_t* scale,
+                      float* dqs, float* dks, float* dvs, void* stream) {
+  LH_RANGE("lh_attn_bwd");
   Geom g;
   lh_status st = make_geom(cfg, &g, nullptr);
   if (st != LH_OK) return st;
-  LH_REQ(qs); LH_REQ(ks); LH_REQ(vs); LH_REQ(dos); LH_REQ(lse); LH_REQ(delta);
+  LH_REQ(qs); LH_REQ(ks); LH_REQ(vs); LH_REQ(dos); LH_REQ(lse); LH_REQ(delta); LH_REQ(scale);
   LH_REQ(dqs); LH_REQ(dks); LH_REQ(dvs);
-  LH_CUDA(launch_attn_bwd(g, cfg->dtype, qs, ks, vs, dos, lse, delta, dqs, dks, dvs,
+  LH_CUDA(launch_attn_bwd(g, cfg->dtype, qs, ks, vs, dos, lse, delta, scale, dqs, dks, dvs,
                           device_error_ptr(), (cudaStream_t)stream));
   return LH_OK;
 }
 
 lh_status lh_spread(const lh_config* cfg, const float* dqs, const float* dks, const float* dvs,
                     const int32_t* slot, void* dq, void* dk, void* dv, void* stream) {
+  LH_RANGE("lh_spread");
   Geom g;
   lh_status st = make_geom(cfg, &g, nullptr);
   if (st != LH_OK) return st;
@@ -306,6 +335,7 @@ lh_status lh_spread(const lh_config* cfg, const float* dqs, const float* dks, co
 
 lh_status lh_forward(const lh_config* cfg, const void* q, const void* k, const void* v, void* o,
                      const lh_buffers* b, void* stream) {
+  LH_RANGE("lh_forward");
   if (!b) return LH_ERR_NULL;
   Geom g;
   lh_plan_t pl;
@@ -313,34 +343,35 @@ lh_status lh_forward(const lh_config* cfg, const void* q, const void* k, const v
   if (st != LH_OK) return st;
   // validate everything up front so that nothing is launched on error
   LH_REQ(q); LH_REQ(k); LH_REQ(v); LH_REQ(o); LH_REQ(b->map); LH_REQ(b->qs); LH_REQ(b->ks);
-  LH_REQ(b->vs); LH_REQ(b->os); LH_REQ(b->lse);
+  LH_REQ(b->vs); LH_REQ(b->os); LH_REQ(b->lse); LH_REQ(b->scale);
   if (g.L > 1) {
     LH_REQ(b->pyr_q); LH_REQ(b->pyr_k); LH_REQ(b->pyr_v); LH_REQ(b->sq); LH_REQ(b->sel);
     LH_REQ(b->slot); LH_REQ(b->ws);
     if (b->ws_bytes < pl.ws_bytes) return LH_ERR_WORKSPACE;
   }
-  if ((st = lh_pool(cfg, q, k, v, b->pyr_q, b->pyr_k, b->pyr_v, b->sq, stream)) != LH_OK) return st;
+  if ((st = lh_pool(cfg, q, k, v, b->pyr_q, b->pyr_k, b->pyr_v, b->sq, b->scale, stream)) != LH_OK) return st;
   if ((st = lh_score_topk(cfg, b->sq, b->sel, b->map, b->slot, b->ws, b->ws_bytes, stream)) != LH_OK)
     return st;
-  if ((st = lh_gather(cfg, q, k, v, b->pyr_q, b->pyr_k, b->pyr_v, b->map, b->qs, b->ks, b->vs,
+  if ((st = lh_gather(cfg, q, k, v, b->pyr_q, b->pyr_k, b->pyr_v, b->map, b->scale, b->qs, b->ks, b->vs,
                       stream)) != LH_OK)
     return st;
-  if ((st = lh_attn_fwd(cfg, b->qs, b->ks, b->vs, b->os, b->lse, stream)) != LH_OK) return st;
+  if ((st = lh_attn_fwd(cfg, b->qs, b->ks, b->vs, b->scale, b->os, b->lse, stream)) != LH_OK) return st;
   return lh_scatter(cfg, b->os, b->slot, o, stream);
 }
 
 lh_status lh_backward(const lh_config* cfg, const void* dout, void* dq, void* dk, void* dv,
                       const lh_buffers* b, void* stream) {
+  LH_RANGE("lh_backward");
   if (!b) return LH_ERR_NULL;
   Geom g;
   lh_status st = make_geom(cfg, &g, nullptr);
   if (st != LH_OK) return st;
   LH_REQ(dout); LH_REQ(dq); LH_REQ(dk); LH_REQ(dv); LH_REQ(b->os); LH_REQ(b->dos);
   LH_REQ(b->delta); LH_REQ(b->qs); LH_REQ(b->ks); LH_REQ(b->vs); LH_REQ(b->lse);
-  LH_REQ(b->dqs); LH_REQ(b->dks); LH_REQ(b->dvs);
+  LH_REQ(b->dqs); LH_REQ(b->dks); LH_REQ(b->dvs); LH_REQ(b->scale);
   if (g.L > 1) LH_REQ(b->slot);
-  if ((st = lh_scatter_bwd(cfg, dout, b->os, b->slot, b->dos, b->delta, stream)) != LH_OK) return st;
-  if ((st = lh_attn_bwd(cfg, b->qs, b->ks, b->vs, b->dos, b->lse, b->delta, b->dqs, b->dks, b->dvs,
+  if ((st = lh_scatter_bwd(cfg, dout, b->os, b->slot, b->dos, b->delta, b->scale, stream)) != LH_OK) return st;
+  if ((st = lh_attn_bwd(cfg, b->qs, b->ks, b->vs, b->dos, b->lse, b->delta, b->scale, b->dqs, b->dks, b->dvs,
                         stream)) != LH_OK)
     return st;
   return lh_spread(cfg, b->dqs, b->dks, b->dvs, b->slot, dq, dk, dv, stream);
@@ -358,20 +389,22 @@ lh_status check_range(const Geom& g, int t0, int nt) {
 }  // namespace
 
 lh_status lh_pool_range(const lh_config* cfg, int t0, int nt, const void* q, const void* k, const void* v,
-                        void* pyr_q, void* pyr_k, void* pyr_v, double* sq, void* stream) {
+                        void* pyr_q, void* pyr_k, void* pyr_v, double* sq, uint32_t* scale, void* stream) {
+  LH_RANGE("lh_pool_range");
   Geom g;
   lh_status st = make_geom(cfg, &g, nullptr);
   if (st != LH_OK) return st;
   if ((st = check_range(g, t0, nt)) != LH_OK) return st;
-  LH_REQ(q); LH_REQ(k); LH_REQ(v); LH_REQ(pyr_q); LH_REQ(pyr_k); LH_REQ(pyr_v); LH_REQ(sq);
+  LH_REQ(q); LH_REQ(k); LH_REQ(v); LH_REQ(pyr_q); LH_REQ(pyr_k); LH_REQ(pyr_v); LH_REQ(sq); LH_REQ(scale);
   const int P = (int)g.pl[g.L - 1];
-  LH_CUDA(launch_pool_range(g, cfg->dtype, t0 / P, nt / P, q, k, v, pyr_q, pyr_k, pyr_v, sq, device_error_ptr(),
-                            (cudaStream_t)stream));
+  LH_CUDA(launch_pool_range(g, cfg->dtype, t0 / P, nt / P, q, k, v, pyr_q, pyr_k, pyr_v, sq, scale,
+                            device_error_ptr(), (cudaStream_t)stream));
   return LH_OK;
 }
 
 lh_status lh_scatter_range(const lh_config* cfg, int t0, int nt, const float* os, const int32_t* slot, void* o,
                            void* stream) {
+  LH_RANGE("lh_scatter_range");
   Geom g;
   lh_status st = make_geom(cfg, &g, nullptr);
   if (st != LH_OK) return st;
@@ -402,18 +435,20 @@ lh_status lh_cp_plan(const lh_config* cfg, int world, int rank, lh_cp_plan_t* ou
 }
 
 lh_status lh_cp_pool(const lh_config* cfg, int world, int rank, const void* q, const void* k, const void* v,
-                     void* pyr_q, void* pyr_k, void* pyr_v, double* sq_loc, void* stream) {
+                     void* pyr_q, void* pyr_k, void* pyr_v, double* sq_loc, uint32_t* scale, void* stream) {
+  LH_RANGE("lh_cp_pool");
   Geom g;
   lh_status st = make_cp_geom_checked(cfg, world, rank, &g, nullptr);
   if (st != LH_OK) return st;
-  LH_REQ(q); LH_REQ(k); LH_REQ(v); LH_REQ(pyr_q); LH_REQ(pyr_k); LH_REQ(pyr_v); LH_REQ(sq_loc);
-  LH_CUDA(launch_pool(shard_geom(g, world, rank), cfg->dtype, q, k, v, pyr_q, pyr_k, pyr_v, sq_loc,
+  LH_REQ(q); LH_REQ(k); LH_REQ(v); LH_REQ(pyr_q); LH_REQ(pyr_k); LH_REQ(pyr_v); LH_REQ(sq_loc); LH_REQ(scale);
+  LH_CUDA(launch_pool(shard_geom(g, world, rank), cfg->dtype, q, k, v, pyr_q, pyr_k, pyr_v, sq_loc, scale,
                       device_error_ptr(), (cudaStream_t)stream));
   return LH_OK;
 }
 
 lh_status lh_cp_assemble_sq(const lh_config* cfg, int world, const double* sq_gathered, double* sq,
                             void* stream) {
+  LH_RANGE("lh_cp_assemble_sq");
   Geom g;
   lh_status st = make_cp_geom_checked(cfg, world, 0, &g, nullptr);
   if (st != LH_OK) return st;
@@ -424,6 +459,7 @@ lh_status lh_cp_assemble_sq(const lh_config* cfg, int world, const double* sq_ga
 
 lh_status lh_cp_segment(const lh_config* cfg, int world, int rank, const int32_t* map, const int32_t* slot,
                         int32_t* slot_loc, int32_t* seg, void* stream) {
+  LH_RANGE("lh_cp_segment");
   Geom g;
   lh_status st = make_cp_geom_checked(cfg, world, rank, &g, nullptr);
   if (st != LH_OK) return st;
@@ -434,30 +470,34 @@ lh_status lh_cp_segment(const lh_config* cfg, int world, int rank, const int32_t
 
 lh_status lh_cp_gather(const lh_config* cfg, int world, int rank, const void* q, const void* k, const void* v,
                        const void* pyr_q, const void* pyr_k, const void* pyr_v, const int32_t* map,
-                       const int32_t* seg, void* qs, void* ks, void* vs, void* stream) {
+                       const int32_t* seg, const uint32_t* scale, void* qs, void* ks, void* vs, void* stream) {
+  LH_RANGE("lh_cp_gather");
   Geom g;
   lh_status st = make_cp_geom_checked(cfg, world, rank, &g, nullptr);
   if (st != LH_OK) return st;
   LH_REQ(q); LH_REQ(k); LH_REQ(v); LH_REQ(pyr_q); LH_REQ(pyr_k); LH_REQ(pyr_v); LH_REQ(map); LH_REQ(seg);
-  LH_REQ(qs); LH_REQ(ks); LH_REQ(vs);
-  LH_CUDA(launch_cp_gather(g, cfg->dtype, world, rank, q, k, v, pyr_q, pyr_k, pyr_v, map, seg, qs, ks, vs,
+  LH_REQ(scale); LH_REQ(qs); LH_REQ(ks); LH_REQ(vs);
+  LH_CUDA(launch_cp_gather(g, cfg->dtype, world, rank, q, k, v, pyr_q, pyr_k, pyr_v, map, seg, scale, qs, ks, vs,
                            device_error_ptr(), (cudaStream_t)stream));
   return LH_OK;
 }
 
 lh_status lh_cp_attn_fwd(const lh_config* cfg, int world, int rank, const int32_t* seg, const void* qs,
-                         const void* ks, const void* vs, float* os, float* lse, void* stream) {
+                         const void* ks, const void* vs, const uint32_t* scale, float* os, float* lse,
+                         void* stream) {
+  LH_RANGE("lh_cp_attn_fwd");
   Geom g;
   lh_status st = make_cp_geom_checked(cfg, world, rank, &g, nullptr);
   if (st != LH_OK) return st;
   if (cfg->dtype != LH_BF16) return LH_ERR_DTYPE;
-  LH_REQ(seg); LH_REQ(qs); LH_REQ(ks); LH_REQ(vs); LH_REQ(os); LH_REQ(lse);
-  LH_CUDA(launch_attn_fwd_tc(g, qs, ks, vs, os, lse, seg, device_error_ptr(), (cudaStream_t)stream));
+  LH_REQ(seg); LH_REQ(qs); LH_REQ(ks); LH_REQ(vs); LH_REQ(scale); LH_REQ(os); LH_REQ(lse);
+  LH_CUDA(launch_attn_fwd_tc(g, qs, ks, vs, os, lse, seg, scale, device_error_ptr(), (cudaStream_t)stream));
   return LH_OK;
 }
 
 lh_status lh_cp_scatter(const lh_config* cfg, int world, int rank, const float* os, const int32_t* slot_loc,
                         void* o, void* stream) {
+  LH_RANGE("lh_cp_scatter");
   Geom g;
   lh_status st = make_cp_geom_checked(cfg, world, rank, &g, nullptr);
   if (st != LH_OK) return st;
@@ -467,34 +507,38 @@ lh_status lh_cp_scatter(const lh_config* cfg, int world, int rank, const float* 
 }
 
 lh_status lh_cp_scatter_bwd(const lh_config* cfg, int world, int rank, const void* dout, const float* os,
-                            const int32_t* slot_loc, const int32_t* seg, void* dos, float* delta, void* stream) {
+                            const int32_t* slot_loc, const int32_t* seg, void* dos, float* delta, uint32_t* scale,
+                            void* stream) {
+  LH_RANGE("lh_cp_scatter_bwd");
   Geom g;
   lh_status st = make_cp_geom_checked(cfg, world, rank, &g, nullptr);
   if (st != LH_OK) return st;
   if (cfg->dtype != LH_BF16) return LH_ERR_DTYPE;
-  LH_REQ(dout); LH_REQ(os); LH_REQ(slot_loc); LH_REQ(seg); LH_REQ(dos); LH_REQ(delta);
+  LH_REQ(dout); LH_REQ(os); LH_REQ(slot_loc); LH_REQ(seg); LH_REQ(dos); LH_REQ(delta); LH_REQ(scale);
   LH_CUDA(launch_cp_zero_outside(g, 2, dos, seg, (cudaStream_t)stream));
-  LH_CUDA(launch_scatter_bwd(shard_geom(g, world, rank), cfg->dtype, dout, os, slot_loc, dos, delta,
+  LH_CUDA(launch_scatter_bwd(shard_geom(g, world, rank), cfg->dtype, dout, os, slot_loc, dos, delta, scale,
                              device_error_ptr(), (cudaStream_t)stream));
   return LH_OK;
 }
 
 lh_status lh_cp_attn_bwd(const lh_config* cfg, int world, int rank, const int32_t* seg, const void* qs,
                          const void* ks, const void* vs, const void* dos, const float* lse, const float* delta,
-                         float* dqs, float* dks, float* dvs, void* stream) {
+                         const uint32_t* scale, float* dqs, float* dks, float* dvs, void* stream) {
+  LH_RANGE("lh_cp_attn_bwd");
   Geom g;
   lh_status st = make_cp_geom_checked(cfg, world, rank, &g, nullptr);
   if (st != LH_OK) return st;
   if (cfg->dtype != LH_BF16) return LH_ERR_DTYPE;
-  LH_REQ(seg); LH_REQ(qs); LH_REQ(ks); LH_REQ(vs); LH_REQ(dos); LH_REQ(lse); LH_REQ(delta);
+  LH_REQ(seg); LH_REQ(qs); LH_REQ(ks); LH_REQ(vs); LH_REQ(dos); LH_REQ(lse); LH_REQ(delta); LH_REQ(scale);
   LH_REQ(dqs); LH_REQ(dks); LH_REQ(dvs);
-  LH_CUDA(launch_attn_bwd_tc(g, qs, ks, vs, dos, lse, delta, dqs, dks, dvs, seg, device_error_ptr(),
+  LH_CUDA(launch_attn_bwd_tc(g, qs, ks, vs, dos, lse, delta, dqs, dks, dvs, seg, scale, device_error_ptr(),
                              (cudaStream_t)stream));
   return LH_OK;
 }
 
 lh_status lh_cp_spread(const lh_config* cfg, int world, int rank, const float* dqs, const float* dks,
                        const float* dvs, const int32_t* slot_loc, void* dq, void* dk, void* dv, void* stream) {
+  LH_RANGE("lh_cp_spread");
   Geom g;
   lh_status st = make_cp_geom_checked(cfg, world, rank, &g, nullptr);
   if (st != LH_OK) return st;

@@ -6,6 +6,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <cstring>
+
 #include "lh.h"
 
 namespace lh {
@@ -172,9 +174,61 @@ template <> struct BwdOperand<__nv_bfloat16> { using type = __half; };
 // Largest finite fp16 value; block sums beyond it are reported, not stored as inf.
 constexpr float kHalfMax = 65504.f;
 
+// Power-of-two scaling of the fp16 attention operands (bf16 I/O). The scale
+// buffer holds, per (b, h), the largest magnitude (fp32 bit pattern; the
+// pattern of a non-negative float orders like the value) of the sub-sequence
+// queries, keys, values and of the block sums of dO: [4][B][H] uint32. An
+// operand x enters fp16 as x * 2^-e, e = scale_exp(largest magnitude): 0 while
+// that magnitude is in [4, 256), otherwise the exponent that puts it in [4, 8).
+// A power of two moves no significant bit, so every bf16 value within 2^19 of
+// its head's largest stays exact in fp16 (the wider range of bf16, beyond
+// fp16's 65504 and below its 2^-14, included), and the products and sums formed
+// from the scaled operands are those of the unscaled ones times powers of two
+// that the kernels take out again. With every operand below 256 in magnitude a
+// dS of 128-term dot products stays inside fp16 for any data of that range.
+enum { kScaleQ = 0, kScaleK = 1, kScaleV = 2, kScaleDO = 3, kScaleRows = 4 };
+constexpr int kScaleMaxExp = 60;      // |e| beyond this is clamped (magnitudes outside 2^-60 .. 2^60)
+
+__host__ __device__ __forceinline__ int scale_exp(uint32_t amax_bits) {
+  const int E = (int)((amax_bits >> 23) & 0xFFu);
+  if (E == 0 || E == 255) return 0;   // zero / fp32-subnormal, or inf / NaN (reported where it is used)
+  const int ex = E - 127;             // floor(log2(largest magnitude))
+  if (ex >= 2 && ex < 8) return 0;
+  const int e = ex - 2;
+  return e < -kScaleMaxExp ? -kScaleMaxExp : (e > kScaleMaxExp ? kScaleMaxExp : e);
+}
+// 2^e as fp32 for |e| <= 126 (exact).
+__host__ __device__ __forceinline__ float pow2f(int e) {
+  const uint32_t b = (uint32_t)(127 + e) << 23;
+  float f;
+  memcpy(&f, &b, sizeof(f));
+  return f;
+}
+// |x| of eight bf16 (a 16-byte vector) as the fp32 bit pattern of the largest.
+__device__ __forceinline__ uint32_t absmax8_bf16(const uint4& r) {
+  uint32_t m = __vmaxu2(__vmaxu2(r.x & 0x7FFF7FFFu, r.y & 0x7FFF7FFFu), __vmaxu2(r.z & 0x7FFF7FFFu, r.w & 0x7FFF7FFFu));
+  return max(m & 0xFFFFu, m >> 16) << 16;
+}
+
 __device__ __forceinline__ void report_error(int* err, int code, int detail) {
   if (err && atomicCAS(err, 0, code) == 0) atomicExch(err + 1, detail);
 }
+
+// Debug build (-DLH_DEBUG_BOUNDS, liblh_debug.so): the indices the memory
+// kernels read from the gather map and the slot table are checked against the
+// buffers they address before use; a bad one is reported as LH_ERR_DEVICE with
+// the site's detail (301 gather map entry, 302 scatter / spread slot, 303
+// block-sum slot) and its access is skipped. The release build compiles the
+// checks away.
+#ifdef LH_DEBUG_BOUNDS
+__device__ __forceinline__ bool lh_bounds_ok(bool ok, int* err, int detail) {
+  if (!ok) report_error(err, LH_ERR_DEVICE, detail);
+  return ok;
+}
+#define LH_BOUNDS(cond, err, detail) ::lh::lh_bounds_ok((cond), (err), (detail))
+#else
+#define LH_BOUNDS(cond, err, detail) true
+#endif
 
 __device__ __forceinline__ void load8_f32(const float* p, float (&x)[8]) {
   float4 a = __ldg(reinterpret_cast<const float4*>(p));
@@ -192,27 +246,31 @@ __device__ __forceinline__ int map_index(int e) { return e & 0x0FFFFFFF; }
 // Host-side launchers (defined next to each kernel, called by lh_api.cu).
 namespace lh {
 cudaError_t launch_pool(const Geom& g, lh_dtype dt, const void* q, const void* k, const void* v,
-                        void* pq, void* pk, void* pv, double* sq, int* err, cudaStream_t s);
+                        void* pq, void* pk, void* pv, double* sq, uint32_t* scale, int* err, cudaStream_t s);
+cudaError_t launch_scale_zero(uint32_t* scale, int r0, int nr, int bh, cudaStream_t s);
 cudaError_t launch_pool_range(const Geom& g, lh_dtype dt, int cb0, int ncb, const void* q, const void* k,
-                              const void* v, void* pq, void* pk, void* pv, double* sq, int* err, cudaStream_t s);
+                              const void* v, void* pq, void* pk, void* pv, double* sq, uint32_t* scale, int* err,
+                              cudaStream_t s);
 cudaError_t launch_scatter_range(const Geom& g, lh_dtype dt, int cb0, int ncb, const float* os,
                                  const int32_t* slot, void* o, cudaStream_t s);
 cudaError_t launch_select(const Geom& g, const double* sq, int32_t* sel, int32_t* map,
                           int32_t* slot, int32_t* ws, cudaStream_t s);
 cudaError_t launch_gather(const Geom& g, lh_dtype dt, const void* q, const void* k, const void* v,
                           const void* pq, const void* pk, const void* pv, const int32_t* map,
-                          void* qs, void* ks, void* vs, int* err, cudaStream_t s);
+                          const uint32_t* scale, void* qs, void* ks, void* vs, int* err, cudaStream_t s);
 cudaError_t launch_scatter(const Geom& g, lh_dtype dt, const float* os, const int32_t* slot,
                            void* o, cudaStream_t s);
 cudaError_t launch_scatter_bwd(const Geom& g, lh_dtype dt, const void* dout, const float* os,
-                               const int32_t* slot, void* dos, float* delta, int* err, cudaStream_t s);
+                               const int32_t* slot, void* dos, float* delta, uint32_t* scale, int* err,
+                               cudaStream_t s);
 cudaError_t launch_spread(const Geom& g, lh_dtype dt, const float* dqs, const float* dks,
                           const float* dvs, const int32_t* slot, void* dq, void* dk, void* dv,
                           cudaStream_t s);
 cudaError_t launch_attn_fwd(const Geom& g, lh_dtype dt, const void* qs, const void* ks,
-                            const void* vs, float* os, float* lse, int* err, cudaStream_t s);
+                            const void* vs, float* os, float* lse, const uint32_t* scale, int* err,
+                            cudaStream_t s);
 cudaError_t launch_attn_bwd(const Geom& g, lh_dtype dt, const void* qs, const void* ks,
                             const void* vs, const void* dos, const float* lse, const float* delta,
-                            float* dqs, float* dks, float* dvs, int* err, cudaStream_t s);
+                            const uint32_t* scale, float* dqs, float* dks, float* dvs, int* err, cudaStream_t s);
 void count_launch(int n = 1);
 }  // namespace lh

@@ -60,7 +60,7 @@ def qkv_project_pool(cfg, ws, x, w_q, w_k, w_v, q, k, v, chunk=None, side=None):
         ev = torch.cuda.Event()
         ev.record(main)
         side.wait_event(ev)
-        lh.pool_range(cfg, t0, c, q, k, v, ws.pyr_q, ws.pyr_k, ws.pyr_v, ws.sq, stream=side)
+        lh.pool_range(cfg, t0, c, q, k, v, ws.pyr_q, ws.pyr_k, ws.pyr_v, ws.sq, ws.scale, stream=side)
     main.wait_stream(side)
 
 

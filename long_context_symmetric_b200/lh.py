@@ -63,7 +63,7 @@ class Buffers(ctypes.Structure):
                 ("sel", c_void_p), ("map", c_void_p), ("slot", c_void_p), ("qs", c_void_p),
                 ("ks", c_void_p), ("vs", c_void_p), ("os", c_void_p), ("lse", c_void_p),
                 ("ws", c_void_p), ("ws_bytes", c_size_t), ("dos", c_void_p), ("delta", c_void_p),
-                ("dqs", c_void_p), ("dks", c_void_p), ("dvs", c_void_p)]
+                ("dqs", c_void_p), ("dks", c_void_p), ("dvs", c_void_p), ("scale", c_void_p)]
 
 
 _lib = None
@@ -72,14 +72,14 @@ _SIGS = {
     "lh_version": ([], c_int),
     "lh_status_string": ([c_int], ctypes.c_char_p),
     "lh_plan": ([ctypes.POINTER(Config), ctypes.POINTER(Plan)], c_int),
-    "lh_pool": ([ctypes.POINTER(Config)] + [c_void_p] * 8, c_int),
+    "lh_pool": ([ctypes.POINTER(Config)] + [c_void_p] * 9, c_int),
     "lh_score_topk": ([ctypes.POINTER(Config), c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                        c_size_t, c_void_p], c_int),
-    "lh_gather": ([ctypes.POINTER(Config)] + [c_void_p] * 11, c_int),
-    "lh_attn_fwd": ([ctypes.POINTER(Config)] + [c_void_p] * 6, c_int),
+    "lh_gather": ([ctypes.POINTER(Config)] + [c_void_p] * 12, c_int),
+    "lh_attn_fwd": ([ctypes.POINTER(Config)] + [c_void_p] * 7, c_int),
     "lh_scatter": ([ctypes.POINTER(Config)] + [c_void_p] * 4, c_int),
-    "lh_scatter_bwd": ([ctypes.POINTER(Config)] + [c_void_p] * 6, c_int),
-    "lh_attn_bwd": ([ctypes.POINTER(Config)] + [c_void_p] * 10, c_int),
+    "lh_scatter_bwd": ([ctypes.POINTER(Config)] + [c_void_p] * 7, c_int),
+    "lh_attn_bwd": ([ctypes.POINTER(Config)] + [c_void_p] * 11, c_int),
     "lh_spread": ([ctypes.POINTER(Config)] + [c_void_p] * 8, c_int),
     "lh_forward": ([ctypes.POINTER(Config)] + [c_void_p] * 4 + [ctypes.POINTER(Buffers), c_void_p], c_int),
     "lh_backward": ([ctypes.POINTER(Config)] + [c_void_p] * 4 + [ctypes.POINTER(Buffers), c_void_p], c_int),
@@ -88,17 +88,17 @@ _SIGS = {
     "lh_selftest_timeout": ([ctypes.c_longlong, c_void_p, c_void_p], c_int),
     "lh_score_topk_noalloc": ([ctypes.POINTER(Config)] + [c_void_p] * 5, c_int),
     "lh_selftest_exp2": ([c_void_p, c_void_p, c_void_p, c_int, c_void_p], c_int),
-    "lh_pool_range": ([ctypes.POINTER(Config), c_int, c_int] + [c_void_p] * 8, c_int),
+    "lh_pool_range": ([ctypes.POINTER(Config), c_int, c_int] + [c_void_p] * 9, c_int),
     "lh_scatter_range": ([ctypes.POINTER(Config), c_int, c_int] + [c_void_p] * 4, c_int),
     "lh_cp_plan": ([ctypes.POINTER(Config), c_int, c_int, ctypes.POINTER(CPPlan)], c_int),
-    "lh_cp_pool": ([ctypes.POINTER(Config), c_int, c_int] + [c_void_p] * 8, c_int),
+    "lh_cp_pool": ([ctypes.POINTER(Config), c_int, c_int] + [c_void_p] * 9, c_int),
     "lh_cp_assemble_sq": ([ctypes.POINTER(Config), c_int] + [c_void_p] * 3, c_int),
     "lh_cp_segment": ([ctypes.POINTER(Config), c_int, c_int] + [c_void_p] * 5, c_int),
-    "lh_cp_gather": ([ctypes.POINTER(Config), c_int, c_int] + [c_void_p] * 12, c_int),
-    "lh_cp_attn_fwd": ([ctypes.POINTER(Config), c_int, c_int] + [c_void_p] * 7, c_int),
+    "lh_cp_gather": ([ctypes.POINTER(Config), c_int, c_int] + [c_void_p] * 13, c_int),
+    "lh_cp_attn_fwd": ([ctypes.POINTER(Config), c_int, c_int] + [c_void_p] * 8, c_int),
     "lh_cp_scatter": ([ctypes.POINTER(Config), c_int, c_int] + [c_void_p] * 4, c_int),
-    "lh_cp_scatter_bwd": ([ctypes.POINTER(Config), c_int, c_int] + [c_void_p] * 7, c_int),
-    "lh_cp_attn_bwd": ([ctypes.POINTER(Config), c_int, c_int] + [c_void_p] * 11, c_int),
+    "lh_cp_scatter_bwd": ([ctypes.POINTER(Config), c_int, c_int] + [c_void_p] * 8, c_int),
+    "lh_cp_attn_bwd": ([ctypes.POINTER(Config), c_int, c_int] + [c_void_p] * 12, c_int),
     "lh_cp_spread": ([ctypes.POINTER(Config), c_int, c_int] + [c_void_p] * 8, c_int),
 }
 
@@ -167,9 +167,9 @@ def plan(cfg: Config) -> Plan:
     return out
 
 
-def pool(cfg, q, k, v, pyr_q, pyr_k, pyr_v, sq, stream=None):
+def pool(cfg, q, k, v, pyr_q, pyr_k, pyr_v, sq, scale, stream=None):
     _check(lib().lh_pool(ctypes.byref(cfg), _p(q), _p(k), _p(v), _p(pyr_q), _p(pyr_k), _p(pyr_v),
-                         _p(sq), _stream(stream)), "lh_pool")
+                         _p(sq), _p(scale), _stream(stream)), "lh_pool")
 
 
 def score_topk(cfg, sq, sel, map_, slot, ws, ws_bytes=None, stream=None):
@@ -184,13 +184,13 @@ def score_topk_noalloc(cfg, sq, sel, map_, slot, stream=None):
                                        _stream(stream)), "lh_score_topk_noalloc")
 
 
-def gather(cfg, q, k, v, pyr_q, pyr_k, pyr_v, map_, qs, ks, vs, stream=None):
+def gather(cfg, q, k, v, pyr_q, pyr_k, pyr_v, map_, scale, qs, ks, vs, stream=None):
     _check(lib().lh_gather(ctypes.byref(cfg), _p(q), _p(k), _p(v), _p(pyr_q), _p(pyr_k), _p(pyr_v),
-                           _p(map_), _p(qs), _p(ks), _p(vs), _stream(stream)), "lh_gather")
+                           _p(map_), _p(scale), _p(qs), _p(ks), _p(vs), _stream(stream)), "lh_gather")
 
 
-def attn_fwd(cfg, qs, ks, vs, os_, lse, stream=None):
-    _check(lib().lh_attn_fwd(ctypes.byref(cfg), _p(qs), _p(ks), _p(vs), _p(os_), _p(lse),
+def attn_fwd(cfg, qs, ks, vs, scale, os_, lse, stream=None):
+    _check(lib().lh_attn_fwd(ctypes.byref(cfg), _p(qs), _p(ks), _p(vs), _p(scale), _p(os_), _p(lse),
                              _stream(stream)), "lh_attn_fwd")
 
 
@@ -198,14 +198,14 @@ def scatter(cfg, os_, slot, o, stream=None):
     _check(lib().lh_scatter(ctypes.byref(cfg), _p(os_), _p(slot), _p(o), _stream(stream)), "lh_scatter")
 
 
-def scatter_bwd(cfg, dout, os_, slot, dos, delta, stream=None):
-    _check(lib().lh_scatter_bwd(ctypes.byref(cfg), _p(dout), _p(os_), _p(slot), _p(dos), _p(delta),
+def scatter_bwd(cfg, dout, os_, slot, dos, delta, scale, stream=None):
+    _check(lib().lh_scatter_bwd(ctypes.byref(cfg), _p(dout), _p(os_), _p(slot), _p(dos), _p(delta), _p(scale),
                                 _stream(stream)), "lh_scatter_bwd")
 
 
-def attn_bwd(cfg, qs, ks, vs, dos, lse, delta, dqs, dks, dvs, stream=None):
+def attn_bwd(cfg, qs, ks, vs, dos, lse, delta, scale, dqs, dks, dvs, stream=None):
     _check(lib().lh_attn_bwd(ctypes.byref(cfg), _p(qs), _p(ks), _p(vs), _p(dos), _p(lse), _p(delta),
-                             _p(dqs), _p(dks), _p(dvs), _stream(stream)), "lh_attn_bwd")
+                             _p(scale), _p(dqs), _p(dks), _p(dvs), _stream(stream)), "lh_attn_bwd")
 
 
 def spread(cfg, dqs, dks, dvs, slot, dq, dk, dv, stream=None):
@@ -236,9 +236,9 @@ def selftest_exp2(x: torch.Tensor, y_fma: torch.Tensor, y_sfu: torch.Tensor, str
     _check(lib().lh_selftest_exp2(_p(x), _p(y_fma), _p(y_sfu), x.numel(), _stream(stream)), "lh_selftest_exp2")
 
 
-def pool_range(cfg, t0, nt, q, k, v, pyr_q, pyr_k, pyr_v, sq, stream=None):
+def pool_range(cfg, t0, nt, q, k, v, pyr_q, pyr_k, pyr_v, sq, scale, stream=None):
     _check(lib().lh_pool_range(ctypes.byref(cfg), t0, nt, _p(q), _p(k), _p(v), _p(pyr_q), _p(pyr_k), _p(pyr_v),
-                               _p(sq), _stream(stream)), "lh_pool_range")
+                               _p(sq), _p(scale), _stream(stream)), "lh_pool_range")
 
 
 def scatter_range(cfg, t0, nt, os_, slot, o, stream=None):
@@ -256,9 +256,9 @@ def cp_plan(cfg, world: int, rank: int) -> CPPlan:
     return out
 
 
-def cp_pool(cfg, world, rank, q, k, v, pyr_q, pyr_k, pyr_v, sq_loc, stream=None):
+def cp_pool(cfg, world, rank, q, k, v, pyr_q, pyr_k, pyr_v, sq_loc, scale, stream=None):
     _check(lib().lh_cp_pool(ctypes.byref(cfg), world, rank, _p(q), _p(k), _p(v), _p(pyr_q), _p(pyr_k),
-                            _p(pyr_v), _p(sq_loc), _stream(stream)), "lh_cp_pool")
+                            _p(pyr_v), _p(sq_loc), _p(scale), _stream(stream)), "lh_cp_pool")
 
 
 def cp_assemble_sq(cfg, world, sq_gathered, sq, stream=None):
@@ -271,15 +271,15 @@ def cp_segment(cfg, world, rank, map_, slot, slot_loc, seg, stream=None):
                                _stream(stream)), "lh_cp_segment")
 
 
-def cp_gather(cfg, world, rank, q, k, v, pyr_q, pyr_k, pyr_v, map_, seg, qs, ks, vs, stream=None):
+def cp_gather(cfg, world, rank, q, k, v, pyr_q, pyr_k, pyr_v, map_, seg, scale, qs, ks, vs, stream=None):
     _check(lib().lh_cp_gather(ctypes.byref(cfg), world, rank, _p(q), _p(k), _p(v), _p(pyr_q), _p(pyr_k),
-                              _p(pyr_v), _p(map_), _p(seg), _p(qs), _p(ks), _p(vs), _stream(stream)),
+                              _p(pyr_v), _p(map_), _p(seg), _p(scale), _p(qs), _p(ks), _p(vs), _stream(stream)),
            "lh_cp_gather")
 
 
-def cp_attn_fwd(cfg, world, rank, seg, qs, ks, vs, os_, lse, stream=None):
-    _check(lib().lh_cp_attn_fwd(ctypes.byref(cfg), world, rank, _p(seg), _p(qs), _p(ks), _p(vs), _p(os_),
-                                _p(lse), _stream(stream)), "lh_cp_attn_fwd")
+def cp_attn_fwd(cfg, world, rank, seg, qs, ks, vs, scale, os_, lse, stream=None):
+    _check(lib().lh_cp_attn_fwd(ctypes.byref(cfg), world, rank, _p(seg), _p(qs), _p(ks), _p(vs), _p(scale),
+                                _p(os_), _p(lse), _stream(stream)), "lh_cp_attn_fwd")
 
 
 def cp_scatter(cfg, world, rank, os_, slot_loc, o, stream=None):
@@ -287,14 +287,15 @@ def cp_scatter(cfg, world, rank, os_, slot_loc, o, stream=None):
            "lh_cp_scatter")
 
 
-def cp_scatter_bwd(cfg, world, rank, dout, os_, slot_loc, seg, dos, delta, stream=None):
+def cp_scatter_bwd(cfg, world, rank, dout, os_, slot_loc, seg, dos, delta, scale, stream=None):
     _check(lib().lh_cp_scatter_bwd(ctypes.byref(cfg), world, rank, _p(dout), _p(os_), _p(slot_loc), _p(seg),
-                                   _p(dos), _p(delta), _stream(stream)), "lh_cp_scatter_bwd")
+                                   _p(dos), _p(delta), _p(scale), _stream(stream)), "lh_cp_scatter_bwd")
 
 
-def cp_attn_bwd(cfg, world, rank, seg, qs, ks, vs, dos, lse, delta, dqs, dks, dvs, stream=None):
+def cp_attn_bwd(cfg, world, rank, seg, qs, ks, vs, dos, lse, delta, scale, dqs, dks, dvs, stream=None):
     _check(lib().lh_cp_attn_bwd(ctypes.byref(cfg), world, rank, _p(seg), _p(qs), _p(ks), _p(vs), _p(dos),
-                                _p(lse), _p(delta), _p(dqs), _p(dks), _p(dvs), _stream(stream)), "lh_cp_attn_bwd")
+                                _p(lse), _p(delta), _p(scale), _p(dqs), _p(dks), _p(dvs), _stream(stream)),
+           "lh_cp_attn_bwd")
 
 
 def cp_spread(cfg, world, rank, dqs, dks, dvs, slot_loc, dq, dk, dv, stream=None):
@@ -330,6 +331,8 @@ class Workspace:
         self.os = z(B, H, S, D, dtype=f32)
         self.lse = z(B, H, S, dtype=f32)
         self.ws = z(max(pl.ws_bytes, 16), dtype=torch.uint8)
+        # per-head operand magnitudes [4][B][H] (uint32 bit patterns, held as int32)
+        self.scale = torch.zeros(4, B, H, dtype=torch.int32, device=device)
         if backward:
             self.dos = z(B, H, S, D, dtype=bop)
             self.delta = z(B, H, S, dtype=f32)
@@ -340,7 +343,7 @@ class Workspace:
             _p(self.pyr_q), _p(self.pyr_k), _p(self.pyr_v), _p(self.sq), _p(self.sel), _p(self.map),
             _p(self.slot), _p(self.qs), _p(self.ks), _p(self.vs), _p(self.os), _p(self.lse),
             _p(self.ws), self.ws.numel(), _p(self.dos), _p(self.delta), _p(self.dqs), _p(self.dks),
-            _p(self.dvs))
+            _p(self.dvs), _p(self.scale))
 
 
 def forward(cfg, q, k, v, o, ws: Workspace, stream=None):

@@ -45,6 +45,28 @@ def to64(t: torch.Tensor) -> np.ndarray:
     return t.detach().to("cpu", torch.float64).numpy()
 
 
+def scale_exp(amax_bits: int) -> int:
+    """The power-of-two exponent e the library applies to a head's fp16
+    operands (x * 2^-e), from the head's largest magnitude (fp32 bit pattern):
+    0 while that magnitude is in [4, 256), else the exponent that brings it
+    into [4, 8) (clamped to +-60)."""
+    E = (int(amax_bits) >> 23) & 0xFF
+    if E in (0, 255):
+        return 0
+    ex = E - 127
+    if 2 <= ex < 8:
+        return 0
+    return max(-60, min(60, ex - 2))
+
+
+def f32_bits(x: float) -> int:
+    return int(np.array([x], dtype=np.float32).view(np.uint32)[0])
+
+
+def struct_f32(bits: int) -> float:
+    return float(np.array([bits & 0xFFFFFFFF], dtype=np.uint32).view(np.float32)[0])
+
+
 class Case:
     def __init__(self, name, B, H, N, D, dtype, p, L, K, recipe="iid", accum="fp", seed=7, **readings):
         self.name, self.B, self.H, self.N, self.D = name, B, H, N, D
@@ -74,16 +96,16 @@ def run_gpu(case: Case, q, k, v, do=None, stream=None):
     cfg = case.cfg()
     ws = lh.Workspace(cfg, q.device, backward=do is not None)
     o = torch.empty_like(q)
-    lh.pool(cfg, q, k, v, ws.pyr_q, ws.pyr_k, ws.pyr_v, ws.sq, stream)
+    lh.pool(cfg, q, k, v, ws.pyr_q, ws.pyr_k, ws.pyr_v, ws.sq, ws.scale, stream)
     lh.score_topk(cfg, ws.sq, ws.sel, ws.map, ws.slot, ws.ws, stream=stream)
-    lh.gather(cfg, q, k, v, ws.pyr_q, ws.pyr_k, ws.pyr_v, ws.map, ws.qs, ws.ks, ws.vs, stream)
-    lh.attn_fwd(cfg, ws.qs, ws.ks, ws.vs, ws.os, ws.lse, stream)
+    lh.gather(cfg, q, k, v, ws.pyr_q, ws.pyr_k, ws.pyr_v, ws.map, ws.scale, ws.qs, ws.ks, ws.vs, stream)
+    lh.attn_fwd(cfg, ws.qs, ws.ks, ws.vs, ws.scale, ws.os, ws.lse, stream)
     lh.scatter(cfg, ws.os, ws.slot, o, stream)
     out = dict(ws=ws, o=o)
     if do is not None:
         dq, dk, dv = (torch.empty_like(q) for _ in range(3))
-        lh.scatter_bwd(cfg, do, ws.os, ws.slot, ws.dos, ws.delta, stream)
-        lh.attn_bwd(cfg, ws.qs, ws.ks, ws.vs, ws.dos, ws.lse, ws.delta, ws.dqs, ws.dks, ws.dvs, stream)
+        lh.scatter_bwd(cfg, do, ws.os, ws.slot, ws.dos, ws.delta, ws.scale, stream)
+        lh.attn_bwd(cfg, ws.qs, ws.ks, ws.vs, ws.dos, ws.lse, ws.delta, ws.scale, ws.dqs, ws.dks, ws.dvs, stream)
         lh.spread(cfg, ws.dqs, ws.dks, ws.dvs, ws.slot, dq, dk, dv, stream)
         out.update(dq=dq, dk=dk, dv=dv)
     torch.cuda.synchronize()
@@ -142,9 +164,16 @@ def compare_head(case: Case, res, q, k, v, do, b: int, h: int, check_bwd=True):
     if case.L > 1:
         assert np.array_equal(ws.slot[b, h].cpu().numpy().astype(np.int64),
                               expected_slot_table(fw, case, pl)), "slot table"
-    # gather: bit-exact (bf16 I/O: the stored entries in fp16, nearest-even)
-    for name, gpu_t, ref in (("qs", ws.qs, fw["qs"]), ("ks", ws.ks, fw["ks"]), ("vs", ws.vs, fw["vs"])):
-        want = ref.astype(np.float16).astype(np.float64) if dt == "bf16" else ref
+    # the head's largest magnitudes (bf16 I/O): exactly the largest |x| of its tokens
+    ex = [0, 0, 0, 0]
+    if dt == "bf16":
+        for t, x in enumerate((qh, kh, vh)):
+            bits = int(ws.scale[t, b, h].item()) & 0xFFFFFFFF
+            assert bits == f32_bits(np.max(np.abs(x))), f"scale row {t}"
+            ex[t] = scale_exp(bits)
+    # gather: bit-exact (bf16 I/O: the stored entries times 2^-e in fp16, nearest-even)
+    for t, (name, gpu_t, ref) in enumerate((("qs", ws.qs, fw["qs"]), ("ks", ws.ks, fw["ks"]), ("vs", ws.vs, fw["vs"]))):
+        want = (ref * 2.0 ** -ex[t]).astype(np.float16).astype(np.float64) if dt == "bf16" else ref
         assert np.array_equal(to64(gpu_t[b, h]), want), name
     # (iii) attention
     atol = ATOL[dt]
@@ -164,7 +193,11 @@ def compare_head(case: Case, res, q, k, v, do, b: int, h: int, check_bwd=True):
     # dos: the fp16 block sums (an intermediate); its bound scales with the
     # largest block sum, since a block sum of p^l token gradients is stored with
     # fp16's relative precision
-    err_dos = excess_error(to64(ws.dos[b, h]), bw["dos"], dt)
+    edo = scale_exp(int(ws.scale[3, b, h].item()) & 0xFFFFFFFF) if dt == "bf16" else 0
+    if dt == "bf16":
+        assert (int(ws.scale[3, b, h].item()) & 0xFFFFFFFF) == f32_bits(np.max(np.abs(bw["dos"]))) or \
+            abs(struct_f32(int(ws.scale[3, b, h].item())) / np.max(np.abs(bw["dos"])) - 1) < 1e-5, "scale row 3"
+    err_dos = excess_error(to64(ws.dos[b, h]) * 2.0 ** edo, bw["dos"], dt)
     assert err_dos <= atol * max(1.0, float(np.max(np.abs(bw["dos"])))) , f"dos err {err_dos}"
     for name in ("dq", "dk", "dv"):
         rep[name] = error_report(to64(res[name][b, :, h, :]), bw[name], dt, atol)

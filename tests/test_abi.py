@@ -75,29 +75,36 @@ def test_entry_points_validate_before_launch():
     r = ctypes.byref(cfg)
     a = 1 << 20        # a fake, aligned address: never dereferenced on these paths
     m = a + 8          # misaligned
-    assert lib.lh_pool(r, None, a, a, a, a, a, a, None) == LH_ERR_NULL
-    assert lib.lh_pool(r, m, a, a, a, a, a, a, None) == LH_ERR_ALIGN
+    assert lib.lh_pool(r, None, a, a, a, a, a, a, a, None) == LH_ERR_NULL
+    assert lib.lh_pool(r, m, a, a, a, a, a, a, a, None) == LH_ERR_ALIGN
+    assert lib.lh_pool(r, a, a, a, a, a, a, a, None, None) == LH_ERR_NULL         # no scale buffer
     assert lib.lh_score_topk(r, a, a, a, a, a, 16, None) == LH_ERR_WORKSPACE
-    assert lib.lh_gather(r, a, a, a, a, a, a, None, a, a, a, None) == LH_ERR_NULL
-    assert lib.lh_attn_fwd(r, a, a, a, m, a, None) == LH_ERR_ALIGN
+    assert lib.lh_gather(r, a, a, a, a, a, a, None, a, a, a, a, None) == LH_ERR_NULL
+    assert lib.lh_gather(r, a, a, a, a, a, a, a, None, a, a, a, None) == LH_ERR_NULL  # no scale buffer
+    assert lib.lh_attn_fwd(r, a, a, a, a, m, a, None) == LH_ERR_ALIGN
+    assert lib.lh_attn_fwd(r, a, a, a, None, a, a, None) == LH_ERR_NULL
     assert lib.lh_scatter(r, a, None, a, None) == LH_ERR_NULL
-    assert lib.lh_scatter_bwd(r, a, a, a, a, None, None) == LH_ERR_NULL
-    assert lib.lh_attn_bwd(r, a, a, a, a, a, a, a, a, None, None) == LH_ERR_NULL
+    assert lib.lh_scatter_bwd(r, a, a, a, a, None, a, None) == LH_ERR_NULL
+    assert lib.lh_scatter_bwd(r, a, a, a, a, a, None, None) == LH_ERR_NULL
+    assert lib.lh_attn_bwd(r, a, a, a, a, a, a, a, a, a, None, None) == LH_ERR_NULL
+    assert lib.lh_attn_bwd(r, a, a, a, a, a, a, None, a, a, a, None) == LH_ERR_NULL
     assert lib.lh_spread(r, a, a, a, a, a, a, m, None) == LH_ERR_ALIGN
     assert lib.lh_forward(r, a, a, a, a, None, None) == LH_ERR_NULL
     bufs = lh.Buffers()
     assert lib.lh_forward(r, a, a, a, a, ctypes.byref(bufs), None) == LH_ERR_NULL
     bad = lh.make_config(1, 2, 4096, 96, 4, 3, 16)
-    assert lib.lh_pool(ctypes.byref(bad), a, a, a, a, a, a, a, None) == LH_ERR_SHAPE
+    assert lib.lh_pool(ctypes.byref(bad), a, a, a, a, a, a, a, a, None) == LH_ERR_SHAPE
 
 
 def test_single_level_needs_no_pyramid_or_workspace():
-    """With L = 1 the pool is a no-op and needs no pyramid buffers (no launch either)."""
+    """With L = 1 the pool needs no pyramid or norm buffers (it only records the
+    operands' magnitudes into the scale buffer): validation passes them as
+    NULL and stops only at the missing scale buffer, before any launch."""
     lib = lh.lib()
     cfg = lh.make_config(1, 2, 4096, 64, 4, 1, 16)
     a = 1 << 20
     before = lh.launch_count()
-    assert lib.lh_pool(ctypes.byref(cfg), a, a, a, None, None, None, None, None) == 0
+    assert lib.lh_pool(ctypes.byref(cfg), a, a, a, None, None, None, None, None, None) == LH_ERR_NULL
     assert lh.launch_count() == before
 
 
@@ -114,8 +121,8 @@ def test_sharded_entry_points_validate_before_launch():
     assert f.lh_cp_segment(ctypes.byref(cfg), 2, 0, None, ptr, ptr, ptr, None) == LH_ERR_NULL
     assert f.lh_cp_segment(ctypes.byref(cfg), 2, 0, ptr + 4, ptr, ptr, ptr, None) == LH_ERR_ALIGN
     c32 = lh.make_config(1, 2, 8192, 128, 4, 3, 64, "fp32")
-    assert f.lh_cp_attn_fwd(ctypes.byref(c32), 2, 0, *([ptr] * 6), None) == LH_ERR_DTYPE
-    assert f.lh_cp_attn_bwd(ctypes.byref(c32), 2, 0, *([ptr] * 10), None) == LH_ERR_DTYPE
+    assert f.lh_cp_attn_fwd(ctypes.byref(c32), 2, 0, *([ptr] * 7), None) == LH_ERR_DTYPE
+    assert f.lh_cp_attn_bwd(ctypes.byref(c32), 2, 0, *([ptr] * 11), None) == LH_ERR_DTYPE
     c1 = lh.make_config(1, 2, 8192, 128, 4, 1, 64)
     assert f.lh_cp_plan(ctypes.byref(c1), 2, 0, ctypes.byref(lh.CPPlan())) == LH_ERR_SHAPE    # L = 1
     pl = lh.cp_plan(cfg, 4, 3)

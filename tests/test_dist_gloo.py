@@ -185,6 +185,7 @@ class _RecordingRank:
     def __init__(self, rank, world):
         self.rank, self.world, self.device = rank, world, torch.device("cpu")
         self.sq_loc = torch.empty(2, 1, 2, 5, dtype=torch.float64)
+        self.scale = torch.zeros(4, 1, 2, dtype=torch.int32)
         S = 4 * world
         self.ks, self.vs = torch.zeros(1, 2, S, 3), torch.zeros(1, 2, S, 3)
         self.dks, self.dvs = torch.zeros(1, 2, S, 3), torch.zeros(1, 2, S, 3)
@@ -195,11 +196,16 @@ class _RecordingRank:
 
     def pool(self, q, k, v):
         self.sq_loc.fill_(self.rank + 1)
+        self.scale[:3] = torch.tensor([10, 20, 30]).view(3, 1, 1) * (self.rank + 1) % 7   # per-rank maxima
+        self.scale[3] = -1
         self.log.append("pool")
 
     def select_gather(self, gathered, q, k, v):
         for r in range(self.world):                      # every rank's norms, in rank order
             assert torch.all(gathered[r] == r + 1)
+        want = torch.stack([torch.tensor([10, 20, 30])[i] * torch.arange(1, self.world + 1) % 7 for i in range(3)])
+        assert torch.equal(self.scale[:3, 0, 0], want.max(dim=1).values.int())   # max over the ranks
+        assert torch.all(self.scale[3] == -1)            # the dO row stays the rank's own
         rows = slice(4 * self.rank, 4 * self.rank + 4)   # this rank's segment, zero elsewhere
         self.ks.zero_()
         self.vs.zero_()

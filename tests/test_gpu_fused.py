@@ -35,15 +35,15 @@ def test_chunked_projection_pool_and_scatter(B, H, N, D, p, L, K, chunk):
             for wt, out in ((w[0], qr), (w[1], kr), (w[2], vr)):
                 torch.matmul(x[b, t0:t0 + chunk], wt, out=out[b, t0:t0 + chunk].view(chunk, dm))
     ref = lh.Workspace(cfg, DEV, backward=False)
-    lh.pool(cfg, qr, kr, vr, ref.pyr_q, ref.pyr_k, ref.pyr_v, ref.sq)
+    lh.pool(cfg, qr, kr, vr, ref.pyr_q, ref.pyr_k, ref.pyr_v, ref.sq, ref.scale)
     torch.cuda.synchronize()
     assert torch.equal(q, qr) and torch.equal(k, kr) and torch.equal(v, vr)
     for a, b_ in ((ws.pyr_q, ref.pyr_q), (ws.pyr_k, ref.pyr_k), (ws.pyr_v, ref.pyr_v), (ws.sq, ref.sq)):
         assert torch.equal(a, b_)
     # rest of the forward, then the chunked scatter + output projection
     lh.score_topk(cfg, ws.sq, ws.sel, ws.map, ws.slot, ws.ws)
-    lh.gather(cfg, q, k, v, ws.pyr_q, ws.pyr_k, ws.pyr_v, ws.map, ws.qs, ws.ks, ws.vs)
-    lh.attn_fwd(cfg, ws.qs, ws.ks, ws.vs, ws.os, ws.lse)
+    lh.gather(cfg, q, k, v, ws.pyr_q, ws.pyr_k, ws.pyr_v, ws.map, ws.scale, ws.qs, ws.ks, ws.vs)
+    lh.attn_fwd(cfg, ws.qs, ws.ks, ws.vs, ws.scale, ws.os, ws.lse)
     o = torch.empty_like(q)
     y = torch.empty(B, N, dm, dtype=torch.bfloat16, device=DEV)
     fused.scatter_project(cfg, ws, w[3], o, y, chunk=chunk)
@@ -73,8 +73,8 @@ def test_graphed_chunk_loop_replays_the_same_results():
     y = torch.empty(B, N, dm, dtype=torch.bfloat16, device=DEV)
     fused.qkv_project_pool(cfg, ref, x, w[0], w[1], w[2], q, k, v, chunk=chunk)
     lh.score_topk(cfg, ref.sq, ref.sel, ref.map, ref.slot, ref.ws)
-    lh.gather(cfg, q, k, v, ref.pyr_q, ref.pyr_k, ref.pyr_v, ref.map, ref.qs, ref.ks, ref.vs)
-    lh.attn_fwd(cfg, ref.qs, ref.ks, ref.vs, ref.os, ref.lse)
+    lh.gather(cfg, q, k, v, ref.pyr_q, ref.pyr_k, ref.pyr_v, ref.map, ref.scale, ref.qs, ref.ks, ref.vs)
+    lh.attn_fwd(cfg, ref.qs, ref.ks, ref.vs, ref.scale, ref.os, ref.lse)
     fused.scatter_project(cfg, ref, w[3], o, y, chunk=chunk)
     torch.cuda.synchronize()
     y_ref = y.clone()
@@ -97,6 +97,6 @@ def test_ranges_reject_unaligned_tokens():
     cfg = lh.make_config(1, 2, 4096, 128, 4, 3, 16, "bf16")
     t = torch.empty(1 << 16, dtype=torch.uint8, device=DEV)
     with pytest.raises(lh.LHError):
-        lh.pool_range(cfg, 8, 16, t, t, t, t, t, t, t)          # t0 not a multiple of 16
+        lh.pool_range(cfg, 8, 16, t, t, t, t, t, t, t, t)          # t0 not a multiple of 16
     with pytest.raises(lh.LHError):
         lh.scatter_range(cfg, 0, 4112, t, t, t)                # past N

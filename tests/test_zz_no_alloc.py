@@ -39,7 +39,7 @@ def test_noalloc_matches_workspace_version(name, N, H, p, L, K):
     q, k, v = (x.cuda() for x in synth.make_inputs(w))
     cfg = lh.make_config(1, H, N, 128, p, L, K, "bf16")
     ws = lh.Workspace(cfg, q.device, backward=False)
-    lh.pool(cfg, q, k, v, ws.pyr_q, ws.pyr_k, ws.pyr_v, ws.sq)
+    lh.pool(cfg, q, k, v, ws.pyr_q, ws.pyr_k, ws.pyr_v, ws.sq, ws.scale)
     lh.score_topk(cfg, ws.sq, ws.sel, ws.map, ws.slot, ws.ws)
     torch.cuda.synchronize()
     for call in range(2):
