@@ -96,3 +96,38 @@ def test_sharded_path_matches_single_gpu_and_oracle(case, world):
         for name, got in (("dq", dq), ("dk", dk), ("dv", dv)):
             e = excess_error(to64(got[b, :, h, :]), bw[name], case.dtype)
             assert e <= ATOL[case.dtype], (name, e)
+
+
+def test_sharded_path_full_size_512k_four_ranks():
+    """The 512K workload (B1 H16 N524288 D128, p8 L4 K1024) split over 4
+    emulated ranks of 131,072 tokens: selection and map equal the single-GPU
+    path's, O and dQ bit for bit, dK and dV to the ranks' regrouped fp32 sums
+    (the single-GPU path itself is held to the oracle at this size by
+    test_gpu_parity.py)."""
+    w = synth.WORKLOADS["ctx512k"]
+    case = Case("cp_ctx512k_w4", w.B, w.H, w.N, w.D, w.dtype, w.p, w.L, w.K, w.recipe, w.mode, w.seed)
+    world = 4
+    q, k, v = synth.make_inputs(w, device=DEV)
+    do = synth.make_dout(w, device=DEV)
+    ref = run_gpu(case, q, k, v, do)
+    cfg = case.cfg()
+    ranks = [cp.ShardRank(cfg, world, r, DEV) for r in range(world)]
+    sh = lambda x: [_shard(x, world, r) for r in range(world)]
+    qs_, ks_, vs_, dos_ = sh(q), sh(k), sh(v), sh(do)
+    outs = [torch.empty_like(x) for x in qs_]
+    dqs, dks, dvs = ([torch.empty_like(x) for x in qs_] for _ in range(3))
+    cp.run_emulated(ranks, qs_, ks_, vs_, outs, dos_, dqs, dks, dvs)
+    torch.cuda.synchronize()
+    assert lh.get_device_error() == (0, 0)
+    ws = ref["ws"]
+    for st in ranks:
+        assert torch.equal(st.map, ws.map) and torch.equal(st.slot, ws.slot)
+    o = torch.cat(outs, dim=1)
+    assert torch.equal(o, ref["o"])
+    assert torch.equal(torch.cat(dqs, dim=1), ref["dq"])
+    for name, parts in (("dk", dks), ("dv", dvs)):
+        got, r32 = torch.cat(parts, dim=1).float(), ref[name].float()
+        diff = (got - r32).abs()
+        assert bool((diff <= r32.abs() * 2 ** -7 + 2 ** -16 * r32.abs().max()).all()), name
+        print(name, "max |sharded - single GPU|", float(diff.max()), "of max", float(r32.abs().max()))
+    del ranks, outs, dqs, dks, dvs
