@@ -204,9 +204,21 @@ __host__ __device__ __forceinline__ float pow2f(int e) {
   memcpy(&f, &b, sizeof(f));
   return f;
 }
+// Lane-wise max / min of two pairs of unsigned 16-bit values, one instruction
+// each (PTX max.u16x2 / min.u16x2, sm_90 and later).
+__device__ __forceinline__ uint32_t max_u16x2(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("max.u16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+__device__ __forceinline__ uint32_t min_u16x2(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("min.u16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
 // |x| of eight bf16 (a 16-byte vector) as the fp32 bit pattern of the largest.
 __device__ __forceinline__ uint32_t absmax8_bf16(const uint4& r) {
-  uint32_t m = __vmaxu2(__vmaxu2(r.x & 0x7FFF7FFFu, r.y & 0x7FFF7FFFu), __vmaxu2(r.z & 0x7FFF7FFFu, r.w & 0x7FFF7FFFu));
+  uint32_t m = max_u16x2(max_u16x2(r.x & 0x7FFF7FFFu, r.y & 0x7FFF7FFFu), max_u16x2(r.z & 0x7FFF7FFFu, r.w & 0x7FFF7FFFu));
   return max(m & 0xFFFFu, m >> 16) << 16;
 }
 
