@@ -548,10 +548,17 @@ __global__ void __launch_bounds__(256, 2) k_blocksum_ring(const T* __restrict__ 
   uint32_t vmax = 0;
   const int row_bytes = a.row_bytes;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + (size_t)a.ns * a.ts * row_bytes);
+  int* done = reinterpret_cast<int*>(full + a.ns);   // warps done with each stage
+  __shared__ tc::Abort ab;
   const int nstages = (int)((P + a.ts - 1) / a.ts);
   const bool contiguous = (a.hg == g.H);
+  const int nwarps = (blockDim.x + 31) >> 5;
   if (threadIdx.x == 0) {
-    for (int s2 = 0; s2 < a.ns; ++s2) tc::mbar_init(&full[s2], 1);
+    ab.flag = 0;
+    for (int s2 = 0; s2 < a.ns; ++s2) {
+      tc::mbar_init(&full[s2], 1);
+      done[s2] = 0;
+    }
     tc::fence_mbar_init();
   }
   __syncthreads();
@@ -618,11 +625,10 @@ __global__ void __launch_bounds__(256, 2) k_blocksum_ring(const T* __restrict__ 
   const long long i1_end = (long long)(cb + 1) * (P / p);
   long long i1 = (long long)cb * (P / p);          // level-1 index of the next group
   int e1n = __ldg(slot_h + g.off[1] + (int)i1);    // its slot entry, fetched one group ahead
-  tc::Abort none{0};
   for (int kk = 0; kk < nstages; ++kk) {
     const int si = kk % a.ns;
-    const bool ok = tc::mbar_wait(&full[si], (kk / a.ns) & 1, &none, err, 201);
-    if (__syncthreads_or(!ok)) break;   // copies never landed: reported, all threads leave
+    const bool ok = tc::mbar_wait(&full[si], (kk / a.ns) & 1, &ab, err, 201);
+    if (!__all_sync(0xffffffffu, ok)) break;   // copies never landed: reported, the warp leaves
     const long long t0 = (long long)kk * a.ts;
     const int nt = (int)min((long long)a.ts, P - t0);
     const uint8_t* buf = smem + (size_t)si * a.ts * row_bytes + (size_t)threadIdx.x * 8 * sizeof(T);
@@ -685,8 +691,17 @@ __global__ void __launch_bounds__(256, 2) k_blocksum_ring(const T* __restrict__ 
         if (__any_sync(0xffffffffu, in)) emit(in ? (e >> 1) : -1, acc[l], wl[l], nullptr);
       }
     }
-    __syncthreads();                    // every thread is done with this stage
-    if (threadIdx.x == 0 && kk + a.ns < nstages) issue(kk + a.ns);
+    // the last warp to finish with this stage refills it (no CTA-wide barrier:
+    // a warp moves on to the next stage as soon as it has landed)
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) {
+      __threadfence_block();
+      if (atomicAdd(&done[si], 1) == nwarps - 1) {
+        atomicExch(&done[si], 0);
+        __threadfence_block();
+        if (kk + a.ns < nstages) issue(kk + a.ns);
+      }
+    }
   }
   if (!REDO && sizeof(TO) == 2) {
     for (int off = C8 >> 1; off >= 1; off >>= 1) vmax = max(vmax, __shfl_xor_sync(0xffffffffu, vmax, off));
@@ -842,7 +857,7 @@ cudaError_t blocksum_pass(const Geom& g, const void* dout, const float* os, cons
     a.ts = ts;
     a.ns = 3;
     if (ts % g.p == 0) {
-      const size_t smem = (size_t)a.ns * a.ts * a.row_bytes + a.ns * sizeof(uint64_t);
+      const size_t smem = (size_t)a.ns * a.ts * a.row_bytes + a.ns * (sizeof(uint64_t) + sizeof(int));
       dim3 rgrid(ncoarse, g.H / hg, g.B);
       const T* d = (const T*)dout;
       TO* o = (TO*)dos;
