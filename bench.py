@@ -562,7 +562,8 @@ def main():
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
         "config": {"workload": workload_desc(w), "S": pl.S,
-                   "l2": "inputs larger than L2 (Q, K, V, dO: 8.6 GB per step), no flush",
+                   "l2": "inputs larger than L2 (Q, K, V, dO: %.1f GB per step), no flush"
+                         % (4 * w.B * w.N * w.H * w.D * (2 if w.dtype == "bf16" else 4) / 1e9),
                    "parallelism": f"dp{world} (independent batches per GPU)"},
         "fwd": {"value": lhdist.job_throughput(w.B * w.N, world, fwd_ms / 1e3), "unit": "tokens/s",
                 "ms": round(fwd_ms, 4), "stages": fwd_stages},
