@@ -244,22 +244,26 @@ __global__ void __launch_bounds__(256) k_scatter_tree(const float* __restrict__ 
                                                       const int32_t* __restrict__ slot,
                                                       T* __restrict__ d0, T* __restrict__ d1,
                                                       T* __restrict__ d2, Geom g, int hg, int yb,
-                                                      int ntens, int cb0, int cb_end) {
+                                                      int ntens, int cb0, int cb_end, int nseg) {
   const int C8 = g.D >> 3;
   const int tensor = blockIdx.z % ntens;
   const int b = blockIdx.z / ntens;
   const int head = blockIdx.y * hg + threadIdx.x / C8;
   const int chunk = threadIdx.x % C8;
-  const int cb = cb0 + (int)blockIdx.x * yb + (int)threadIdx.y;
-  if (cb >= cb_end) return;            // no collectives below: a thread may leave
+  // segment sg of coarsest block cb (nseg equal token segments per block)
+  const int cs = cb0 * nseg + (int)blockIdx.x * yb + (int)threadIdx.y;
+  if (cs >= cb_end * nseg) return;     // no collectives below: a thread may leave
+  const int cb = cs / nseg, sg = cs - cb * nseg;
   const float* src = tensor == 0 ? s0 : (tensor == 1 ? s1 : s2);
   T* dst = tensor == 0 ? d0 : (tensor == 1 ? d1 : d2);
   const long long bh = (long long)b * g.H + head;
   const int32_t* slot_h = slot + bh * g.E;
   const float* srow = src + (size_t)bh * g.S * g.D + chunk * 8;
   const long long P = g.pl[LV];
+  const long long seglen = P / nseg;
+  const long long t_begin = (long long)sg * seglen;    // first token of the segment within the block
   const size_t tstride = (size_t)g.H * g.D;
-  T* out = dst + ((size_t)b * g.N + (size_t)cb * P) * tstride + (size_t)head * g.D + chunk * 8;
+  T* out = dst + ((size_t)b * g.N + (size_t)cb * P + (size_t)t_begin) * tstride + (size_t)head * g.D + chunk * 8;
 
   Acc<FIXED> acc[LV + 1];              // acc[l]: contributions of levels >= l (l >= 1)
   bool expd[LV + 1];                   // entry of level l expanded (its children included)
@@ -277,14 +281,31 @@ __global__ void __launch_bounds__(256) k_scatter_tree(const float* __restrict__ 
     expd[LV] = e & 1;
     if (LV == 1) tok1 = slot_tokens(e, g);
   }
+  // the entries of levels LV-1 .. 1 that cover the segment's first token, as
+  // the walk below meets an entry start (a segment starts on a level-1
+  // boundary: seglen is a multiple of p)
 #pragma unroll
-  for (int l = 1; l < LV; ++l) {
-    rem[l] = 0;
-    idx[l] = (int)((long long)cb * (P / g.pl[l])) - 1;
+  for (int l = LV - 1; l >= 1; --l) {
+    const long long pos = t_begin % g.pl[l];
+    rem[l] = (int)(g.pl[l] - pos);
+    idx[l] = (int)(((long long)cb * P + t_begin) / g.pl[l]);
+    if (expd[l + 1]) {
+      const int e = __ldg(slot_h + g.off[l] + idx[l]);
+      acc[l] = acc[l + 1];
+      if (slot_in(e, g)) {
+        load8_f32(srow + (size_t)(e >> 1) * g.D, x);
+        add_level<FIXED, WEIGHTED>(acc[l], x, g, l);
+      }
+      expd[l] = e & 1;
+      if (l == 1) tok1 = slot_tokens(e, g);
+    } else {
+      acc[l] = acc[l + 1];
+      expd[l] = false;
+    }
   }
   Packed<T> pk;
   bool pk_ok = false;
-  for (long long t = 0; t < P; ++t) {
+  for (long long t = 0; t < seglen; ++t) {
 #pragma unroll
     for (int l = LV - 1; l >= 1; --l) {
       if (rem[l] == 0) {               // a level-l entry starts here (finer ones too)
@@ -343,14 +364,27 @@ cudaError_t tree_t(const Geom& g, const float* s0, const float* s1, const float*
   }
   const int ncoarse = ncb < 0 ? g.n[g.L - 1] : ncb;
   if (ncoarse <= 0) return cudaSuccess;
+  // split a block's token walk into nseg segments (each a multiple of 64 tokens)
+  // while there are fewer than 32 CTAs per SM: shorter walks, a smaller tail
+  // (512K, fp32 accumulation: scatter 0.47 -> 0.42 ms, spread 1.29 -> 1.27 ms)
+  int dev = 0, nsm = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+  const long long P = g.pl[g.L - 1];
+  int nseg = 1;
+  if (g.L > 2 && !FIXED)   // (the fixed-point walks, at 2 CTAs per SM, measured slower split)
+    while (P / (2 * nseg) >= 64 && (P / (2 * nseg)) % g.p == 0 &&
+           (long long)ncoarse * nseg * (g.H / hg) * g.B * ntens < 32LL * nsm)
+      nseg *= 2;
+  const int nunits = ncoarse * nseg;
   int yb = 1;
-  while (yb * 2 * hg * C8 <= 256 && yb * 2 <= ncoarse) yb *= 2;
+  while (yb * 2 * hg * C8 <= 256 && yb * 2 <= nunits) yb *= 2;
   dim3 block(hg * C8, yb);
-  dim3 grid((ncoarse + yb - 1) / yb, g.H / hg, g.B * ntens);
+  dim3 grid((nunits + yb - 1) / yb, g.H / hg, g.B * ntens);
   const int cb_end = cb0 + ncoarse;
   switch (g.L - 1) {
 #define LH_TREE_CASE(n) \
-    case n: k_scatter_tree<T, FIXED, WEIGHTED, n><<<grid, block, 0, s>>>(s0, s1, s2, slot, d0, d1, d2, g, hg, yb, ntens, cb0, cb_end); break;
+    case n: k_scatter_tree<T, FIXED, WEIGHTED, n><<<grid, block, 0, s>>>(s0, s1, s2, slot, d0, d1, d2, g, hg, yb, ntens, cb0, cb_end, nseg); break;
     LH_TREE_CASE(1) LH_TREE_CASE(2) LH_TREE_CASE(3) LH_TREE_CASE(4)
     LH_TREE_CASE(5) LH_TREE_CASE(6) LH_TREE_CASE(7)
 #undef LH_TREE_CASE
