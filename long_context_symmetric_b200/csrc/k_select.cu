@@ -132,7 +132,7 @@ __device__ __forceinline__ unsigned long long score_bits(const double* sqq, cons
 // Flags fl[q] = 1 for the k (< c <= kChunk) candidates q first in the order
 // (score desc, q asc; q desc if high_first), 0 for the rest. Key of q: hi =
 // score bits, lo = c-1-q (q if high_first), compared as (hi, lo) descending;
-// keys are unique. hist: 257 ints of shared memory, bc: 2 ints. All threads
+// keys are unique. hist: 257 ints of shared memory, bc: 3 ints. All threads
 // must call it.
 __device__ void radix_select_flags(const double* sq_l, const double* sk_l, const int32_t* cl, int c, int k,
                                    int score_mode, bool high_first, int32_t* fl, int* hist, int* bc) {
@@ -190,7 +190,11 @@ __device__ void radix_select_flags(const double* sq_l, const double* sk_l, const
       if (above < kk && kk <= incl) {
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
-          if (above < kk && kk <= above + loc[u]) { bc[0] = 255 - 8 * lane - u; bc[1] = kk - above; }
+          if (above < kk && kk <= above + loc[u]) {
+            bc[0] = 255 - 8 * lane - u;
+            bc[1] = kk - above;
+            bc[2] = loc[u];
+          }
           above += loc[u];
         }
       }
@@ -198,9 +202,14 @@ __device__ void radix_select_flags(const double* sq_l, const double* sk_l, const
     __syncthreads();
     const int b = bc[0];
     kk = bc[1];
+    // the threshold is the bin's last key and the bin is taken whole: every key
+    // with this prefix is expanded, so the digits below can stay zero (with
+    // continuous scores this ends the select after two or three passes)
+    const bool whole = bc[2] == kk;
     if (pass < 8) thi |= (unsigned long long)b << (56 - 8 * pass);
     else tlo |= (unsigned)b << (8 * (9 - pass));
     __syncthreads();               // bc is rewritten by the next pass
+    if (whole) break;
   }
 #pragma unroll
   for (int j = 0; j < KPT; ++j) {
@@ -216,7 +225,7 @@ k_select(const double* __restrict__ sq, int32_t* __restrict__ sel, int32_t* __re
   unsigned long long* sk = reinterpret_cast<unsigned long long*>(smem_raw);
   unsigned* sp = reinterpret_cast<unsigned*>(sk + kChunk);
   __shared__ int warp_tot[33];
-  __shared__ int hist[257], bcast[2];
+  __shared__ int hist[257], bcast[3];
 
   const Geom& g = a.g;
   const int bh = blockIdx.x;
