@@ -22,11 +22,18 @@
 // Taking the max of the two then equals max-pooling the tokens' bidirectional
 // scores level by level, since max commutes.
 //
-// Thread mapping: one thread owns 8 consecutive components of one head; the
-// D/8 lanes of a head are consecutive lanes of one warp. A thread walks the
-// p^(L-1) tokens of one coarsest-level block in order, keeping one running fp64
-// sum per level (carry chain), and emits each entry when its last child is in.
-// Rows arrive through a shared-memory ring filled by bulk async copies.
+// Two kernel forms with the same arithmetic (bit-identical results):
+//  - ring form (k_pool): one thread owns 8 consecutive components of one head;
+//    the D/8 lanes of a head are consecutive lanes of one warp. A thread walks
+//    the p^(L-1) tokens of one coarsest-level block in order, keeping one
+//    running fp64 sum per level (carry chain), and emits each entry when its
+//    last child is in. Rows arrive through a shared-memory ring filled by bulk
+//    async copies; the last warp done with a stage refills it.
+//  - block-parallel form (k_pool_par, bf16): one CTA per (block, head,
+//    tensor), a thread per level-1 entry and 8 components, higher levels from
+//    shared-memory sums; for short token ranges and few heads.
+// For bf16 and p in {2, 4, 8}, a level-1 entry's p values are summed in fp32
+// where that chain is provably exact (sum_rows_bf16), else in fp64.
 // HBM traffic: every token row is read once; pyramid rows and norms written once.
 #include <algorithm>
 
