@@ -98,11 +98,13 @@ def _check_against_oracle(cfg, ws, q, k, v, p, L):
 # H = 2: the block-parallel kernel (coarsest blocks of 512, 64, 64, 16, 16 and
 # 8 tokens) and, where its level sums do not fit in shared memory (blocks of
 # 4096 tokens), the shared-memory ring kernel; H = 16 with enough blocks: the
-# ring kernel on whole CTAs
-@pytest.mark.parametrize("p,L,N,H", [(8, 4, 4096, 2), (4, 4, 2048, 2), (2, 7, 1024, 2), (4, 3, 2048, 2),
-                                     (2, 5, 1024, 2), (8, 2, 1024, 2), (8, 5, 8192, 2), (4, 4, 16384, 16)])
-def test_pool_exact_at_exponent_bounds(p, L, N, H):
-    B, D = 1, 128
+# ring kernel (8 warps per CTA at D = 128, 4 at D = 64)
+@pytest.mark.parametrize("p,L,N,H,D", [(8, 4, 4096, 2, 128), (4, 4, 2048, 2, 128), (2, 7, 1024, 2, 128),
+                                       (4, 3, 2048, 2, 128), (2, 5, 1024, 2, 128), (8, 2, 1024, 2, 128),
+                                       (8, 5, 8192, 2, 128), (4, 4, 16384, 16, 128), (8, 4, 4096, 2, 64),
+                                       (4, 4, 16384, 16, 64)])
+def test_pool_exact_at_exponent_bounds(p, L, N, H, D):
+    B = 1
     q, k, v = _inputs(B, H, N, D, p, seed=100 + p + L)
     cfg = lh.make_config(B, H, N, D, p, L, 16, "bf16")
     ws = lh.Workspace(cfg, DEV, backward=False)
