@@ -74,7 +74,7 @@ def _inputs(B, H, N, D, p, seed):
     return out
 
 
-def _check_against_oracle(cfg, ws, q, k, v, p, L):
+def _check_against_oracle(cfg, ws, q, k, v, p, L, dtype="bf16", score="max"):
     pl = lh.plan(cfg)
     B, H = q.shape[0], q.shape[2]
     for b in range(B):
@@ -82,17 +82,18 @@ def _check_against_oracle(cfg, ws, q, k, v, p, L):
             means = {}
             for name, x, pyr in (("q", q, ws.pyr_q), ("k", k, ws.pyr_k), ("v", v, ws.pyr_v)):
                 xm = x[b, :, h, :].float().double().numpy()
-                m, stored = orc.pool_head(xm, p, L, "bf16")
+                m, stored = orc.pool_head(xm, p, L, dtype)
                 means[name] = m
                 for l in range(1, L):
                     o0, n = pl.lvl_off[l], pl.n[l]
                     got = pyr[b, h, o0:o0 + n].float().double().cpu().numpy()
                     assert np.array_equal(got, stored[l]), (name, b, h, l)
-            for row, name in ((0, "q"), (1, "k")):
+            _, sq_q, sq_k = orc.scores_head(means["q"], means["k"], L, score)
+            for row, ref in ((0, sq_q), (1, sq_k)):
                 for l in range(1, L):
                     o0, n = pl.lvl_off[l], pl.n[l]
                     got = ws.sq[row, b, h, o0:o0 + n].cpu().numpy()
-                    assert np.array_equal(got, orc.sq_norm_pinned(means[name][l])), ("sq", name, b, h, l)
+                    assert np.array_equal(got, ref[l]), ("sq", row, b, h, l)
 
 
 # H = 2: the block-parallel kernel (coarsest blocks of 512, 64, 64, 16, 16 and
@@ -128,3 +129,21 @@ def test_pool_exact_at_exponent_bounds(p, L, N, H, D):
                   (ws.scale[:3], ws2.scale[:3])):
         assert torch.equal(a.view(torch.int16) if a.dtype == torch.bfloat16 else a,
                            b_.view(torch.int16) if b_.dtype == torch.bfloat16 else b_)
+
+
+@pytest.mark.parametrize("p,L,N,H,dtype,score", [(8, 4, 4096, 2, "bf16", "maxpool"), (4, 4, 16384, 16, "bf16", "maxpool"),
+                                                 (8, 4, 4096, 2, "fp32", "max"), (4, 4, 16384, 16, "fp32", "max")])
+def test_pool_exponent_bounds_other_paths(p, L, N, H, dtype, score):
+    """The same inputs through the paths that keep the fp64 chain throughout:
+    the max-pool score reading (token norms pooled by max) and fp32 I/O."""
+    B, D = 1, 128
+    q, k, v = _inputs(B, H, N, D, p, seed=200 + p + L)
+    if dtype == "fp32":
+        q, k, v = (x.float() for x in (q, k, v))
+    cfg = lh.make_config(B, H, N, D, p, L, 16, dtype, score=score)
+    ws = lh.Workspace(cfg, DEV, backward=False)
+    qd, kd, vd = (x.to(DEV) for x in (q, k, v))
+    lh.pool(cfg, qd, kd, vd, ws.pyr_q, ws.pyr_k, ws.pyr_v, ws.sq, ws.scale)
+    torch.cuda.synchronize()
+    assert lh.get_device_error() == (0, 0)
+    _check_against_oracle(cfg, ws, q, k, v, p, L, dtype, score)
