@@ -10,11 +10,12 @@ of these steps streams its tensors through HBM: the projections write Q, K, V
 into chunks of whole coarsest blocks small enough to stay in the 126 MB L2:
 
   qkv_project_pool   chunk i: Q, K, V = X W_q, X W_k, X W_v (cuBLAS through
-                     torch.matmul), then lh_pool_range on a second stream while
-                     the projections of chunk i+1 run, reading chunk i from L2;
+                     torch.matmul, the three at once on three streams), then
+                     lh_pool_range on another stream while the projections of
+                     chunk i+1 run, reading chunk i from L2;
   scatter_project    chunk i: lh_scatter_range on a second stream, then
-                     Y = O W_o on the main stream, reading chunk i of O from L2
-                     while chunk i+1 is being scattered.
+                     Y = O W_o (on two streams in turn), reading chunk i of O
+                     from L2 while chunk i+1 is being scattered.
 
 The projections are plain library GEMMs (they are the model's, not the path's);
 every step of the path stays a liblh kernel. The pool and scatter results
@@ -33,7 +34,7 @@ from . import lh
 __all__ = ["chunk_tokens", "qkv_project_pool", "scatter_project", "Graphed"]
 
 
-def chunk_tokens(cfg, target: int = 4096) -> int:
+def chunk_tokens(cfg, target: int = 8192) -> int:
     """Chunk length: a multiple of p^(L-1) close to `target` tokens (at least one block)."""
     P = cfg.p ** (cfg.L - 1)
     c = max(P, (target // P) * P)
@@ -42,38 +43,51 @@ def chunk_tokens(cfg, target: int = 4096) -> int:
     return c
 
 
-def qkv_project_pool(cfg, ws, x, w_q, w_k, w_v, q, k, v, chunk=None, side=None):
+def _streams(n, given):
+    return list(given) if given is not None else [torch.cuda.Stream() for _ in range(n)]
+
+
+def qkv_project_pool(cfg, ws, x, w_q, w_k, w_v, q, k, v, chunk=None, side=None, gemm_streams=None):
     """q, k, v [B, N, H, D] = x [B, N, d_model] @ w_* [d_model, H*D], and the
     pyramid / norms of ws (lh.Workspace) by lh_pool_range, chunk by chunk.
-    Runs on the current stream; the pool runs on `side` (a second stream)."""
+    A chunk's three projections run at once (the current stream and two of
+    `gemm_streams`), so that together they fill the GPU; the pool of chunk i
+    runs on `side` once all three have written it."""
     B, N = cfg.B, cfg.N
     HD = cfg.H * cfg.D
     c = chunk or chunk_tokens(cfg)
     main = torch.cuda.current_stream()
     side = side or torch.cuda.Stream()
-    side.wait_stream(main)
+    gs = [main] + _streams(2, gemm_streams)
+    for st in gs[1:] + [side]:
+        st.wait_stream(main)
     for t0 in range(0, N, c):
-        for b in range(B):
-            xs = x[b, t0:t0 + c]
-            for w, out in ((w_q, q), (w_k, k), (w_v, v)):
-                torch.matmul(xs, w, out=out[b, t0:t0 + c].view(c, HD))
-        ev = torch.cuda.Event()
-        ev.record(main)
-        side.wait_event(ev)
+        for (w, out), st in zip(((w_q, q), (w_k, k), (w_v, v)), gs):
+            with torch.cuda.stream(st):
+                for b in range(B):
+                    torch.matmul(x[b, t0:t0 + c], w, out=out[b, t0:t0 + c].view(c, HD))
+            ev = torch.cuda.Event()
+            ev.record(st)
+            side.wait_event(ev)
         lh.pool_range(cfg, t0, c, q, k, v, ws.pyr_q, ws.pyr_k, ws.pyr_v, ws.sq, ws.scale, stream=side)
-    main.wait_stream(side)
+    for st in gs[1:] + [side]:
+        main.wait_stream(st)
 
 
-def scatter_project(cfg, ws, w_o, o, y, chunk=None, side=None):
+def scatter_project(cfg, ws, w_o, o, y, chunk=None, side=None, gemm_streams=None):
     """o [B, N, H, D] = scatter of ws.os by lh_scatter_range, and
     y [B, N, d_out] = o @ w_o [H*D, d_out], chunk by chunk: chunk i's GEMM reads
-    the rows the scatter of chunk i has just written."""
+    the rows the scatter of chunk i has just written. Consecutive chunks' GEMMs
+    alternate between the current stream and one of `gemm_streams`, so that one
+    chunk's GEMM fills the tail of the previous one."""
     B, N = cfg.B, cfg.N
     HD = cfg.H * cfg.D
     c = chunk or chunk_tokens(cfg)
     main = torch.cuda.current_stream()
     side = side or torch.cuda.Stream()
-    side.wait_stream(main)
+    gs = [main] + _streams(1, gemm_streams)
+    for st in gs[1:] + [side]:
+        st.wait_stream(main)
     done = []
     for i, t0 in enumerate(range(0, N, c)):
         if i >= 2:
@@ -81,13 +95,16 @@ def scatter_project(cfg, ws, w_o, o, y, chunk=None, side=None):
         lh.scatter_range(cfg, t0, c, ws.os, ws.slot, o, stream=side)
         ev = torch.cuda.Event()
         ev.record(side)
-        main.wait_event(ev)
-        for b in range(B):
-            torch.matmul(o[b, t0:t0 + c].view(c, HD), w_o, out=y[b, t0:t0 + c])
+        st = gs[i % 2]
+        st.wait_event(ev)
+        with torch.cuda.stream(st):
+            for b in range(B):
+                torch.matmul(o[b, t0:t0 + c].view(c, HD), w_o, out=y[b, t0:t0 + c])
         d = torch.cuda.Event()
-        d.record(main)
+        d.record(st)
         done.append(d)
-    main.wait_stream(side)
+    for st in gs[1:] + [side]:
+        main.wait_stream(st)
 
 
 class Graphed:
