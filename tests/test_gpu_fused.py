@@ -18,6 +18,7 @@ DEV = torch.device("cuda", 0)
     (1, 4, 16384, 128, 4, 3, 64, 2048),
     (2, 3, 8192, 64, 8, 3, 16, 1024),
     (1, 2, 4096, 128, 2, 5, 32, 1 << 12),          # one chunk
+    (1, 2, 8192, 128, 8, 4, 64, 2048),             # 4 coarsest blocks a chunk: the per-token scatter walk
 ])
 def test_chunked_projection_pool_and_scatter(B, H, N, D, p, L, K, chunk):
     g = torch.Generator(device=DEV).manual_seed(9)
